@@ -1,0 +1,183 @@
+"""fp64 CPU oracle of the QSA hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library
+and its binding) never imports it and never falls back to it.
+
+The arithmetic lives in ``qsa_oracle.c`` (plain fp64 C); this module only
+marshals numpy arrays.  bf16 tensors are passed as their raw uint16 bit
+patterns.  Sources: the pages "Qwen4 architecture: QSA, GR, PLE" (section
+"1. QSA: not looking at every token equally") and "Qwen4 in llama.cpp:
+Dissecting PR #27742" (section "QSA Is an Address-Selection Problem, Not a
+New Attention Equation").
+
+Parity status of each function is stated in its docstring; every function
+here is pinned by ``tests/test_oracle_pins.py``.
+"""
+import ctypes
+import math
+import os
+
+import numpy as np
+
+from . import build as _build
+
+BLOCK = 64  # key block size fixed by the build's parameterization
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        Dd = ctypes.c_double
+        lib.qsa_oracle_threads.restype = I
+        lib.qsa_oracle_compress_keys.argtypes = [P, I, I, I, I, I, I, I, P]
+        lib.qsa_oracle_compress_keys.restype = None
+        lib.qsa_oracle_pool_queries.argtypes = [P, I, I, I, I, I, I, P]
+        lib.qsa_oracle_pool_queries.restype = None
+        lib.qsa_oracle_select.argtypes = [P, P, I, I, I, I, I, I, I, I, I, I, Dd,
+                                          P, I, P, P, P, P]
+        lib.qsa_oracle_select.restype = I
+        lib.qsa_oracle_attend.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, I,
+                                          Dd, P, I, P, P]
+        lib.qsa_oracle_attend.restype = I
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else ctypes.c_void_p(a.ctypes.data)
+
+
+def _bits(x):
+    """bf16 data as a C-contiguous uint16 array (accepts torch bf16 or uint16)."""
+    if hasattr(x, "dtype") and str(x.dtype) == "torch.bfloat16":
+        import torch
+        x = x.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint16:
+        raise TypeError("bf16 inputs must be torch.bfloat16 or raw uint16 bits")
+    return x
+
+
+def threads() -> int:
+    """Threads the oracle's parallel loops use."""
+    return int(_load().qsa_oracle_threads())
+
+
+def compress_keys(K, blk_begin=0, blk_end=None, blk=BLOCK):
+    """Mean-pooled key summaries, fp64.
+
+    K: bf16 [B, H, T, d].  Returns Kc [B, H, T//blk, d]; only blocks in
+    [blk_begin, blk_end) are written (others are zero).
+    """
+    K = _bits(K)
+    B, H, T, d = K.shape
+    NB = T // blk
+    if blk_end is None:
+        blk_end = NB
+    assert 0 <= blk_begin <= blk_end <= NB
+    Kc = np.zeros((B, H, NB, d), dtype=np.float64)
+    _load().qsa_oracle_compress_keys(_ptr(K), B, H, T, d, blk, blk_begin, blk_end, _ptr(Kc))
+    return Kc
+
+
+def pool_queries(Q, Hkv, qblk=BLOCK):
+    """Pooled query of each selection row, fp64.  Q: bf16 [B, Tq, Hq, d].
+    Returns Qbar [B, Hkv, ceil(Tq/qblk), d]."""
+    Q = _bits(Q)
+    B, Tq, Hq, d = Q.shape
+    assert Hq % Hkv == 0
+    NR = -(-Tq // qblk)
+    Qbar = np.zeros((B, Hkv, NR, d), dtype=np.float64)
+    _load().qsa_oracle_pool_queries(_ptr(Q), B, Tq, Hq, Hkv, d, qblk, _ptr(Qbar))
+    return Qbar
+
+
+def select(Qbar, Kc, Tq, q_pos0, qblk, topk, sm_scale, rows=None, blk=BLOCK,
+           want_scores=False):
+    """Score + top-k select.  Returns dict with ``idx`` ([nrows, topk] int32,
+    or [B, Hkv, NR, topk] when rows is None), ``gap``, ``m`` and optionally
+    ``scores`` ([nrows, NB], NaN for non-candidates)."""
+    Qbar = np.ascontiguousarray(Qbar, dtype=np.float64)
+    Kc = np.ascontiguousarray(Kc, dtype=np.float64)
+    B, Hkv, NR, d = Qbar.shape
+    NB = Kc.shape[2]
+    assert Kc.shape[:2] == (B, Hkv) and Kc.shape[3] == d
+    rows_arr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    nrows = B * Hkv * NR if rows is None else len(rows_arr)
+    idx = np.empty((nrows, topk), dtype=np.int32)
+    gap = np.empty(nrows, dtype=np.float64)
+    m = np.empty(nrows, dtype=np.int32)
+    scores = np.empty((nrows, NB), dtype=np.float64) if want_scores else None
+    rc = _load().qsa_oracle_select(_ptr(Qbar), _ptr(Kc), B, Hkv, NR, NB, d, Tq, q_pos0,
+                                   qblk, blk, topk, float(sm_scale), _ptr(rows_arr), nrows,
+                                   _ptr(idx), _ptr(gap), _ptr(m), _ptr(scores))
+    if rc != 0:
+        raise ValueError("oracle select: topk must be >= 2")
+    if rows is None:
+        idx = idx.reshape(B, Hkv, NR, topk)
+        gap = gap.reshape(B, Hkv, NR)
+        m = m.reshape(B, Hkv, NR)
+    out = {"idx": idx, "gap": gap, "m": m}
+    if want_scores:
+        out["scores"] = scores
+    return out
+
+
+def attend(Q, K, V, idx, q_pos0, qblk, sm_scale, tokens=None, blk=BLOCK, want_lse=False):
+    """Exact softmax attention over the selected blocks, fp64.
+
+    Q: bf16 [B, Tq, Hq, d]; K, V: bf16 [B, Hkv, T_kv, d];
+    idx: int32 [B, Hkv, NR, topk].  Returns O [ntok, Hq, d] for the listed
+    flat tokens (b*Tq + t), or [B, Tq, Hq, d] when tokens is None.
+    """
+    Q, K, V = _bits(Q), _bits(K), _bits(V)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    B, Tq, Hq, d = Q.shape
+    _, Hkv, T_kv, _ = K.shape
+    NR = -(-Tq // qblk)
+    assert idx.shape[:3] == (B, Hkv, NR), (idx.shape, (B, Hkv, NR))
+    topk = idx.shape[3]
+    tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int32)
+    ntok = B * Tq if tokens is None else len(tok)
+    O = np.empty((ntok, Hq, d), dtype=np.float64)
+    lse = np.empty((ntok, Hq), dtype=np.float64) if want_lse else None
+    rc = _load().qsa_oracle_attend(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), B, Tq, Hq, Hkv,
+                                   T_kv, d, q_pos0, qblk, blk, topk, float(sm_scale),
+                                   _ptr(tok), ntok, _ptr(O), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle attend: a selected block lies outside the cache "
+                         "or after its query token")
+    if tokens is None:
+        O = O.reshape(B, Tq, Hq, d)
+        if want_lse:
+            lse = lse.reshape(B, Tq, Hq)
+    return (O, lse) if want_lse else O
+
+
+def qsa_forward(Q, K, V, Hkv, topk, q_pos0=0, qblk=BLOCK, sm_scale=None, blk=BLOCK,
+                tokens=None):
+    """The whole path: compress -> pool -> score/select -> attend.
+
+    Keys of the cache (and of the new tokens) sit in K/V [B, Hkv, T_kv, d];
+    the Tq query tokens sit at positions q_pos0 .. q_pos0+Tq-1.
+    Returns (sel dict, O).
+    """
+    Qb = _bits(Q)
+    d = Qb.shape[3]
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    Tq = Qb.shape[1]
+    T_kv = _bits(K).shape[2] if not hasattr(K, "shape") else K.shape[2]
+    n_complete = (q_pos0 + Tq) // blk
+    Kc = compress_keys(K, 0, min(n_complete, T_kv // blk), blk=blk)
+    Qbar = pool_queries(Q, Hkv, qblk)
+    sel = select(Qbar, Kc, Tq, q_pos0, qblk, topk, sm_scale, blk=blk)
+    O = attend(Q, K, V, sel["idx"], q_pos0, qblk, sm_scale, tokens=tokens, blk=blk)
+    return sel, O

@@ -1,0 +1,296 @@
+/*
+ * QSA reference oracle: plain, slow, fp64 CPU implementation of the Qwen
+ * Sparse Attention hot path (compress -> score -> top-k select -> attend).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or helper with the CUDA path and must never serve as a
+ * fallback for it.
+ *
+ * Sources (web pages on the method):
+ *  - "Qwen4 architecture: QSA, GR, PLE" (codebridge-ai.com), section
+ *    "1. QSA: not looking at every token equally": keys are compressed into
+ *    small blocks, the blocks are scored, the most relevant contiguous token
+ *    blocks are selected, and attention runs closely over those regions only.
+ *  - "Qwen4 in llama.cpp: Dissecting PR #27742" (ramgpt.org), section
+ *    "QSA Is an Address-Selection Problem, Not a New Attention Equation":
+ *    compressed-block representation -> indexer scoring -> top-k selection ->
+ *    visible cache cells -> ordinary softmax attention over those cells.
+ *
+ * The pages give no formulas for the compression, the score or the
+ * aggregation; this file uses the fixed parameterization of the build:
+ * mean-pooled keys per block, scores = <mean pooled query, key summary>
+ * scaled by sm_scale, selection shared by one query block and all query
+ * heads of a KV group, block 0 (sink) and the causal diagonal block always
+ * kept, ties broken by the lower block index.
+ *
+ * Every floating-point quantity is fp64.  bf16 inputs are widened exactly.
+ * OpenMP only splits independent rows/tokens; no step is reordered.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Exact widening of a bf16 bit pattern: bf16 is the top half of an fp32. */
+static double bf16_to_f64(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+int qsa_oracle_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * Step 1 -- compress keys ("compress into small blocks", page
+ * "Qwen4 architecture: QSA, GR, PLE", section 1; "compressed-block
+ * representation", page "Qwen4 in llama.cpp", section "QSA Is an
+ * Address-Selection Problem").
+ *
+ * K  : [B][H][T][d] bf16 bits.  Kc : [B][H][T/blk][d] fp64.
+ * For every complete block j in [jb, je):
+ *     Kc[b][h][j][c] = (1/blk) * sum_{r=0}^{blk-1} K[b][h][j*blk + r][c]
+ */
+void qsa_oracle_compress_keys(const uint16_t *K, int B, int H, int T, int d,
+                              int blk, int jb, int je, double *Kc)
+{
+    const int64_t NB = T / blk;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int bh = 0; bh < B * H; bh++) {
+        for (int j = jb; j < je; j++) {
+            const uint16_t *base = K + ((int64_t)bh * T + (int64_t)j * blk) * d;
+            double *out = Kc + ((int64_t)bh * NB + j) * d;
+            for (int c = 0; c < d; c++) {
+                double s = 0.0;
+                for (int r = 0; r < blk; r++)
+                    s += bf16_to_f64(base[(int64_t)r * d + c]);
+                out[c] = s / (double)blk;
+            }
+        }
+    }
+}
+
+/*
+ * Step 2 -- pooled query of a selection row.  One selection row is one
+ * query block (qblk consecutive query tokens; 1 in decode) of one KV group;
+ * the selection is shared by all query heads of the group.  The row's query
+ * is the mean over the group's G heads and the block's valid tokens, so its
+ * score equals the mean of the per-(head, token) block scores.
+ *
+ * Q : [B][Tq][Hq][d] bf16 bits.  Qbar : [B][Hkv][NR][d] fp64, NR = ceil(Tq/qblk).
+ * Query head h belongs to group h / (Hq/Hkv).
+ */
+void qsa_oracle_pool_queries(const uint16_t *Q, int B, int Tq, int Hq, int Hkv,
+                             int d, int qblk, double *Qbar)
+{
+    const int G = Hq / Hkv;
+    const int NR = (Tq + qblk - 1) / qblk;
+#pragma omp parallel for collapse(3) schedule(static)
+    for (int b = 0; b < B; b++) {
+        for (int g = 0; g < Hkv; g++) {
+            for (int i = 0; i < NR; i++) {
+                const int t0 = i * qblk;
+                const int t1 = (t0 + qblk < Tq) ? t0 + qblk : Tq;
+                const double n = (double)(t1 - t0) * (double)G;
+                double *out = Qbar + (((int64_t)b * Hkv + g) * NR + i) * d;
+                for (int c = 0; c < d; c++) {
+                    double s = 0.0;
+                    for (int t = t0; t < t1; t++)
+                        for (int h = g * G; h < (g + 1) * G; h++)
+                            s += bf16_to_f64(Q[(((int64_t)b * Tq + t) * Hq + h) * d + c]);
+                    out[c] = s / n;
+                }
+            }
+        }
+    }
+}
+
+typedef struct {
+    double s;
+    int j;
+} scored_block;
+
+/* Total order of the top-k: higher score first, then the lower block index. */
+static int by_score_then_index(const void *pa, const void *pb)
+{
+    const scored_block *a = (const scored_block *)pa;
+    const scored_block *b = (const scored_block *)pb;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+    return (a->j < b->j) ? -1 : (a->j > b->j);
+}
+
+/* The causal diagonal block of selection row i: the block holding the row's
+ * last query position. */
+static int diagonal_block(int i, int Tq, int q_pos0, int qblk, int blk)
+{
+    int t_last = (i + 1) * qblk - 1;
+    if (t_last > Tq - 1) t_last = Tq - 1;
+    return (q_pos0 + t_last) / blk;
+}
+
+/*
+ * Steps 3 and 4 -- score the compressed key blocks against the row's pooled
+ * query ("indexer scoring") and keep the top-k blocks ("top-k selection"),
+ * page "Qwen4 in llama.cpp", section "QSA Is an Address-Selection Problem".
+ *
+ * For selection row (b, g, i) with diagonal block D:
+ *   candidates C = {1, ..., D-1}  (complete blocks strictly before D; the
+ *                                  diagonal's summary would see the future)
+ *   s_j = sm_scale * <Qbar[b][g][i], Kc[b][g][j]>
+ *   F   = {0} plus {D} if D > 0   (sink and diagonal, always kept; they
+ *                                  count toward topk)
+ *   m   = min(topk - |F|, |C|) candidates taken in the order
+ *         (s descending, j ascending)
+ *   out = F plus the chosen, ascending, padded with -1 to topk entries.
+ *
+ * rows    : list of flat row ids ((b*Hkv + g)*NR + i), or NULL for all rows
+ * idx     : [nrows][topk] int32
+ * gap     : [nrows] s_(m) - s_(m+1) among the candidates, +inf when the set
+ *           does not depend on the scores (m == 0 or m == |C|)
+ * m_out   : [nrows] number of chosen candidates
+ * scores  : optional [nrows][NB] -- s_j for candidates, NaN elsewhere
+ * Qbar    : [B][Hkv][NR][d]; Kc : [B][Hkv][NB][d]
+ * Returns 0, or -1 if topk < 2.
+ */
+int qsa_oracle_select(const double *Qbar, const double *Kc, int B, int Hkv, int NR,
+                      int NB, int d, int Tq, int q_pos0, int qblk, int blk, int topk,
+                      double sm_scale, const int32_t *rows, int nrows, int32_t *idx,
+                      double *gap, int32_t *m_out, double *scores)
+{
+    if (topk < 2) return -1;
+    const int total = B * Hkv * NR;
+    if (!rows) nrows = total;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < nrows; r++) {
+        const int row = rows ? rows[r] : r;
+        const int i = row % NR;
+        const int bg = row / NR;
+        const int D = diagonal_block(i, Tq, q_pos0, qblk, blk);
+        const int ncand = D > 1 ? D - 1 : 0;
+        const double *q = Qbar + (int64_t)row * d;
+        scored_block *cand = (scored_block *)malloc(sizeof(scored_block) * (ncand > 0 ? ncand : 1));
+        for (int j = 1; j < D; j++) {
+            const double *kc = Kc + ((int64_t)bg * NB + j) * d;
+            double dot = 0.0;
+            for (int c = 0; c < d; c++) dot += q[c] * kc[c];
+            cand[j - 1].s = sm_scale * dot;
+            cand[j - 1].j = j;
+        }
+        if (scores) {
+            double *srow = scores + (int64_t)r * NB;
+            for (int j = 0; j < NB; j++) srow[j] = NAN;
+            for (int n = 0; n < ncand; n++) srow[cand[n].j] = cand[n].s;
+        }
+        qsort(cand, (size_t)ncand, sizeof(scored_block), by_score_then_index);
+        const int nforced = D > 0 ? 2 : 1;
+        int m = topk - nforced;
+        if (m > ncand) m = ncand;
+        gap[r] = (m == 0 || m == ncand) ? INFINITY : cand[m - 1].s - cand[m].s;
+        m_out[r] = m;
+
+        /* ascending output: 0, chosen blocks in increasing index, D */
+        int32_t *out = idx + (int64_t)r * topk;
+        int n = 0;
+        out[n++] = 0;
+        for (int j = 1; j < D; j++) {
+            int chosen = 0;
+            for (int c = 0; c < m; c++)
+                if (cand[c].j == j) { chosen = 1; break; }
+            if (chosen) out[n++] = j;
+        }
+        if (D > 0) out[n++] = D;
+        while (n < topk) out[n++] = -1;
+        free(cand);
+    }
+    return 0;
+}
+
+/*
+ * Step 5 -- exact softmax attention over the selected blocks only ("attend
+ * closely to the selected regions", page "Qwen4 architecture: QSA, GR,
+ * PLE", section 1; "attention over those cells", page "Qwen4 in llama.cpp",
+ * section "QSA Is an Address-Selection Problem").
+ *
+ * Query token t of batch b sits at absolute position p = q_pos0 + t and
+ * uses the selection of its row i = t / qblk in its head's group.  Visible
+ * keys: u in the selected blocks with u <= p.
+ *   z_u = sm_scale * <q, k_u>,  O = sum_u exp(z_u - max z) v_u / sum_u exp(z_u - max z)
+ *   lse = max z + log(sum_u exp(z_u - max z))
+ *
+ * Q : [B][Tq][Hq][d]; K, V : [B][Hkv][T_kv][d] (bf16 bits)
+ * idx : [B][Hkv][NR][topk] int32, -1 = unused slot
+ * tokens : list of flat tokens (b*Tq + t), or NULL for all
+ * O : [ntok][Hq][d] fp64; lse : optional [ntok][Hq]
+ * Returns 0, or -1 if an index lies outside the cache or after the token.
+ */
+int qsa_oracle_attend(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                      const int32_t *idx, int B, int Tq, int Hq, int Hkv, int T_kv,
+                      int d, int q_pos0, int qblk, int blk, int topk, double sm_scale,
+                      const int32_t *tokens, int ntok, double *O, double *lse)
+{
+    const int G = Hq / Hkv;
+    const int NR = (Tq + qblk - 1) / qblk;
+    if (!tokens) ntok = B * Tq;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int n = 0; n < ntok; n++) {
+        const int flat = tokens ? tokens[n] : n;
+        const int b = flat / Tq, t = flat % Tq;
+        const int64_t p = (int64_t)q_pos0 + t;
+        const int i = t / qblk;
+        double *z = (double *)malloc(sizeof(double) * (size_t)topk * blk);
+        int64_t *u_of = (int64_t *)malloc(sizeof(int64_t) * (size_t)topk * blk);
+        for (int h = 0; h < Hq; h++) {
+            const int g = h / G;
+            const int32_t *sel = idx + (((int64_t)b * Hkv + g) * NR + i) * topk;
+            const uint16_t *q = Q + (((int64_t)b * Tq + t) * Hq + h) * d;
+            const uint16_t *Kbg = K + ((int64_t)b * Hkv + g) * (int64_t)T_kv * d;
+            const uint16_t *Vbg = V + ((int64_t)b * Hkv + g) * (int64_t)T_kv * d;
+            int nvis = 0;
+            for (int s = 0; s < topk; s++) {
+                const int j = sel[s];
+                if (j < 0) continue;
+                if ((int64_t)j * blk > p || p >= T_kv) { bad = 1; continue; }
+                for (int r = 0; r < blk; r++) {
+                    const int64_t u = (int64_t)j * blk + r;
+                    if (u > p) break;
+                    double dot = 0.0;
+                    for (int c = 0; c < d; c++)
+                        dot += bf16_to_f64(q[c]) * bf16_to_f64(Kbg[u * d + c]);
+                    z[nvis] = sm_scale * dot;
+                    u_of[nvis] = u;
+                    nvis++;
+                }
+            }
+            double *o = O + ((int64_t)n * Hq + h) * d;
+            double zmax = -INFINITY;
+            for (int e = 0; e < nvis; e++)
+                if (z[e] > zmax) zmax = z[e];
+            double l = 0.0;
+            for (int c = 0; c < d; c++) o[c] = 0.0;
+            for (int e = 0; e < nvis; e++) {
+                const double w = exp(z[e] - zmax);
+                l += w;
+                for (int c = 0; c < d; c++) o[c] += w * bf16_to_f64(Vbg[u_of[e] * d + c]);
+            }
+            for (int c = 0; c < d; c++) o[c] = nvis ? o[c] / l : 0.0;
+            if (lse) lse[(int64_t)n * Hq + h] = nvis ? zmax + log(l) : -INFINITY;
+        }
+        free(z);
+        free(u_of);
+    }
+    return bad ? -1 : 0;
+}

@@ -1,0 +1,327 @@
+"""Pins of the fp64 oracle to facts other than itself: closed forms,
+invariants, brute force on tiny inputs, and library routines (torch SDPA in
+fp64) in the regimes where QSA reduces to plain attention.
+
+The regime pins follow the page "Qwen4 in llama.cpp: Dissecting PR #27742",
+section "QSA Is an Address-Selection Problem, Not a New Attention Equation"
+(below the budget nothing can be dropped, so sparse equals dense; above it,
+compare set overlap), section "The PR's Numerical Evidence Is Layered
+Correctly" (a CPU semantic oracle; QSA equals dense below the sparse
+threshold), and section "Quantized KV Exposed a Backend Storage Invariant"
+(Q' = HQ, K' = HK with H orthonormal preserves Q^T K).
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+
+BLK = 64
+
+
+def bf16(x):
+    return torch.as_tensor(x, dtype=torch.float32).to(torch.bfloat16)
+
+
+def f64(x_bf16):
+    return x_bf16.to(torch.float64).numpy()
+
+
+def rand_grid(shape, gen, lo=-4.0, hi=4.0, step=0.125):
+    """Random values on a coarse grid: exactly representable in bf16, and
+    closed under the affine maps the invariance pins apply."""
+    n = int(round((hi - lo) / step))
+    ints = torch.randint(0, n + 1, shape, generator=gen)
+    return bf16(lo + step * ints.to(torch.float32))
+
+
+# ----------------------------------------------------------------- compress
+def test_compress_closed_form_ramp():
+    B, H, T, d = 2, 2, 256, 16
+    t = torch.arange(T).view(1, 1, T, 1) % BLK
+    c = torch.arange(d).view(1, 1, 1, d)
+    h = torch.arange(H).view(1, H, 1, 1)
+    K = bf16((t + c + 3 * h).expand(B, H, T, d).clone())
+    Kc = oracle.compress_keys(K)
+    # mean of r = 0..63 is 31.5
+    expect = 31.5 + np.arange(d)[None, None, None, :] + 3 * np.arange(H)[None, :, None, None]
+    assert np.array_equal(Kc, np.broadcast_to(expect, Kc.shape))
+
+
+def test_compress_shift_and_block_range():
+    g = torch.Generator().manual_seed(1)
+    K = rand_grid((1, 2, 512, 32), g)
+    Kc = oracle.compress_keys(K, 2, 6)
+    Kc_shift = oracle.compress_keys(bf16(K.float() + 1.0), 2, 6)
+    assert np.allclose(Kc_shift[:, :, 2:6], Kc[:, :, 2:6] + 1.0, atol=0, rtol=1e-15)
+    assert np.all(Kc[:, :, :2] == 0) and np.all(Kc[:, :, 6:] == 0)
+    # a constant block compresses to that constant
+    Kconst = bf16(torch.full((1, 1, 128, 8), 0.375))
+    assert np.all(oracle.compress_keys(Kconst) == 0.375)
+
+
+def test_compress_page_candidate_count():
+    """Page "Qwen4 in llama.cpp", section "Why Short-Context Tests Can Lie":
+    262144 positions at compression ratio 4 give 65536 compressed blocks."""
+    import json, os
+    facts = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "page_facts.json")))
+    f = facts["candidate_count"]
+    K = bf16(torch.ones((1, 1, f["n_kv"], 1)))
+    Kc = oracle.compress_keys(K, blk=f["ratio"])
+    assert Kc.shape[2] == f["blocks"]
+
+
+# --------------------------------------------------------------------- pool
+def test_pool_closed_form_with_tail():
+    B, Tq, Hq, Hkv, d = 1, 100, 8, 2, 4      # rows: 64 tokens, then a 36-token tail
+    t = torch.arange(Tq).view(1, Tq, 1, 1).float()
+    h = torch.arange(Hq).view(1, 1, Hq, 1).float()
+    c = torch.arange(d).view(1, 1, 1, d).float()
+    Q = bf16((t + 10 * h + c).expand(B, Tq, Hq, d).clone())
+    Qbar = oracle.pool_queries(Q, Hkv, 64)
+    G = Hq // Hkv
+    for g in range(Hkv):
+        hmean = 10 * (g * G + (G - 1) / 2)
+        assert np.allclose(Qbar[0, g, 0], 31.5 + hmean + np.arange(d), rtol=0, atol=1e-12)
+        assert np.allclose(Qbar[0, g, 1], (64 + 99) / 2 + hmean + np.arange(d), rtol=0, atol=1e-12)
+
+
+def test_pool_identity_and_head_permutation():
+    g = torch.Generator().manual_seed(2)
+    Q = rand_grid((2, 5, 2, 8), g)
+    # one head per group, one token per row: pooling is the identity
+    Qbar = oracle.pool_queries(Q, 2, 1)
+    assert np.array_equal(Qbar.transpose(0, 2, 1, 3), f64(Q))
+    Q8 = rand_grid((1, 128, 8, 16), g)
+    perm = torch.tensor([2, 0, 3, 1, 7, 5, 4, 6])      # within each group of 4
+    a = oracle.pool_queries(Q8, 2, 64)
+    b = oracle.pool_queries(Q8[:, :, perm], 2, 64)
+    assert np.allclose(a, b, rtol=0, atol=1e-14)
+
+
+# -------------------------------------------------------------------- score
+def _rand_case(seed, Tq=256, T_kv=None, Hq=8, Hkv=2, d=32, topk=4, q_pos0=None, qblk=64):
+    w = synthetic.custom(Tq=Tq, T_kv=T_kv, Hq=Hq, Hkv=Hkv, d=d, topk=topk,
+                         q_pos0=q_pos0, qblk=qblk, seed=seed)
+    return w, synthetic.generate(w)
+
+
+def test_score_equals_mean_of_per_token_logits():
+    """Pooled-query score == mean over (head, token) of each token's logit
+    against the block summary (computed here without any pooling)."""
+    w, x = _rand_case(3, Tq=192, T_kv=448, q_pos0=256)
+    Kc = oracle.compress_keys(x["K"])
+    Qbar = oracle.pool_queries(x["Q"], w.Hkv, 64)
+    out = oracle.select(Qbar, Kc, w.Tq, w.q_pos0, 64, w.topk, w.sm_scale, want_scores=True)
+    S = out["scores"].reshape(w.B, w.Hkv, w.n_rows, -1)
+    q = f64(x["Q"])
+    G = w.Hq // w.Hkv
+    Kbf = f64(x["K"])
+    for g in range(w.Hkv):
+        for i in range(w.n_rows):
+            D = (w.q_pos0 + min((i + 1) * 64, w.Tq) - 1) // 64
+            toks = q[0, i * 64:(i + 1) * 64, g * G:(g + 1) * G, :].reshape(-1, w.d)
+            for j in range(1, D):
+                kc = Kbf[0, g, j * 64:(j + 1) * 64].sum(axis=0) / 64.0
+                logits = toks @ kc * w.sm_scale
+                assert abs(S[0, g, i, j] - logits.mean()) < 1e-12
+            assert np.all(np.isnan(S[0, g, i, D:])) and np.isnan(S[0, g, i, 0])
+
+
+def test_score_rotation_and_shift_invariance():
+    """Q' = HQ, K' = HK with H orthonormal preserves every score; adding one
+    vector c to every key shifts a row's scores by a constant, so neither
+    changes the selection."""
+    w, x = _rand_case(4, Tq=256, T_kv=1024, q_pos0=768, d=32, topk=6)
+    Kc = oracle.compress_keys(x["K"])
+    Qbar = oracle.pool_queries(x["Q"], w.Hkv, 64)
+    base = oracle.select(Qbar, Kc, w.Tq, w.q_pos0, 64, w.topk, w.sm_scale, want_scores=True)
+    H, _ = np.linalg.qr(np.random.default_rng(0).standard_normal((w.d, w.d)))
+    rot = oracle.select(Qbar @ H.T, Kc @ H.T, w.Tq, w.q_pos0, 64, w.topk, w.sm_scale,
+                        want_scores=True)
+    m = ~np.isnan(base["scores"])
+    assert np.allclose(rot["scores"][m], base["scores"][m], rtol=0, atol=1e-12)
+    ok = base["gap"].reshape(-1) > 1e-9
+    assert np.array_equal(rot["idx"].reshape(-1, w.topk)[ok], base["idx"].reshape(-1, w.topk)[ok])
+    c = np.random.default_rng(1).standard_normal(w.d)
+    sh = oracle.select(Qbar, Kc + c, w.Tq, w.q_pos0, 64, w.topk, w.sm_scale, want_scores=True)
+    delta = (sh["scores"] - base["scores"]).reshape(w.B, w.Hkv, w.n_rows, -1)
+    for g in range(w.Hkv):
+        for i in range(w.n_rows):
+            row = delta[0, g, i][~np.isnan(delta[0, g, i])]
+            assert np.allclose(row, w.sm_scale * Qbar[0, g, i] @ c, rtol=0, atol=1e-12)
+    assert np.array_equal(sh["idx"].reshape(-1, w.topk)[ok], base["idx"].reshape(-1, w.topk)[ok])
+
+
+# ------------------------------------------------------------------- select
+def _check_selection(idx_row, scores_row, D, topk):
+    """Brute-force validity of one selection row under (score desc, index asc)."""
+    sel = [j for j in idx_row if j >= 0]
+    assert sel == sorted(set(sel)), "ascending and duplicate-free"
+    assert all(0 <= j <= D for j in sel)
+    assert 0 in sel and (D == 0 or D in sel), "sink and diagonal always kept"
+    assert len(idx_row) == topk
+    cand = list(range(1, D))
+    chosen = [j for j in sel if 1 <= j < D]
+    m = min(topk - (2 if D > 0 else 1), len(cand))
+    assert len(chosen) == m
+    key = lambda j: (scores_row[j], -j)
+    unchosen = [j for j in cand if j not in chosen]
+    if chosen and unchosen:
+        assert min(key(j) for j in chosen) > max(key(j) for j in unchosen)
+    return chosen
+
+
+def test_select_brute_force_with_ties():
+    rng = np.random.default_rng(5)
+    for trial in range(30):
+        d = 4
+        NB = 24
+        Kc = rng.integers(-2, 3, size=(1, 1, NB, d)).astype(np.float64)   # many ties
+        Qbar = rng.integers(-2, 3, size=(1, 1, 1, d)).astype(np.float64)
+        topk = int(rng.integers(2, 10))
+        D = int(rng.integers(0, NB))
+        q_pos0 = D * 64 + int(rng.integers(0, 64))
+        out = oracle.select(Qbar, Kc, 1, q_pos0, 1, topk, 1.0, want_scores=True)
+        s = out["scores"][0]
+        chosen = _check_selection(list(out["idx"][0, 0, 0]), s, D, topk)
+        # brute force over all subsets of the right size
+        cand = list(range(1, D))
+        m = len(chosen)
+        if m == 0 or m == len(cand):
+            assert out["gap"][0, 0, 0] == math.inf
+            continue
+        srt = sorted((s[j] for j in cand), reverse=True)
+        assert out["gap"][0, 0, 0] == pytest.approx(srt[m - 1] - srt[m], abs=1e-15)
+        if len(cand) <= 14:
+            best = None
+            for sub in itertools.combinations(cand, m):
+                k = sorted(((s[j], -j) for j in sub), reverse=True)
+                if best is None or k > best[0]:
+                    best = (k, sub)
+            assert sorted(best[1]) == chosen
+
+
+def test_select_special_cases():
+    d = 8
+    Kc = np.zeros((1, 1, 40, d))
+    Qbar = np.zeros((1, 1, 1, d))
+    run = lambda q_pos0, topk: oracle.select(Qbar, Kc, 1, q_pos0, 1, topk, 1.0)["idx"][0, 0, 0]
+    assert list(run(10, 4)) == [0, -1, -1, -1]                  # D = 0
+    assert list(run(64, 4)) == [0, 1, -1, -1]                   # D = 1: no candidates
+    assert list(run(64 * 5 + 3, 8)) == [0, 1, 2, 3, 4, 5, -1, -1]  # k >= D+1 keeps all
+    # all scores tie: the lowest indices win
+    assert list(run(64 * 30, 5)) == [0, 1, 2, 3, 30]
+    with pytest.raises(ValueError):
+        oracle.select(Qbar, Kc, 1, 100, 1, 1, 1.0)
+
+
+def test_select_planted_tiny_config_statistic():
+    w = synthetic.CONFIGS["tiny_prefill_1k"]
+    x = synthetic.generate(w)
+    sel, _ = oracle.qsa_forward(x["Q"], x["K"], x["V"], w.Hkv, w.topk, tokens=[0])
+    hit = sum(1 for (b, g, j, i) in x["planted"] if j in sel["idx"][b, g, i])
+    assert hit >= 0.8 * len(x["planted"])
+
+
+# ------------------------------------------------------------------ attend
+def _sdpa_f64(Q, K, V, mask, scale):
+    """torch SDPA in fp64 on [B, Tq, Hq, d] / [B, Hkv, T, d] with GQA expansion."""
+    B, Tq, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    q = Q.to(torch.float64).permute(0, 2, 1, 3)
+    k = K.to(torch.float64).repeat_interleave(G, dim=1)
+    v = V.to(torch.float64).repeat_interleave(G, dim=1)
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=scale)
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+def test_attend_dense_equivalence_below_budget():
+    """k >= number of causal blocks: nothing can be dropped, QSA equals dense
+    causal attention (page: bit identical below the sparse budget).  Against
+    torch SDPA in fp64, and bit-identical to itself with a larger k."""
+    w, x = _rand_case(6, Tq=300, T_kv=300, Hq=8, Hkv=2, d=32, topk=5)
+    sel, O = oracle.qsa_forward(x["Q"], x["K"], x["V"], w.Hkv, 5, q_pos0=0)
+    causal = torch.ones(300, 300, dtype=torch.bool).tril()
+    ref = _sdpa_f64(x["Q"], x["K"], x["V"], causal, w.sm_scale)
+    assert np.abs(O - ref).max() < 1e-12
+    _, O9 = oracle.qsa_forward(x["Q"], x["K"], x["V"], w.Hkv, 9, q_pos0=0)
+    assert np.array_equal(O, O9)
+
+
+def test_attend_masked_brute_force_and_decode():
+    """Any selection: equals SDPA with the dense T x T mask built from the
+    selected blocks (prefill with a cache offset, and per-token decode)."""
+    for (Tq, T_kv, q_pos0, qblk, topk, seed) in [(192, 704, 512, 64, 4, 8),
+                                                 (3, 900, 897, 1, 5, 9)]:
+        w, x = _rand_case(seed, Tq=Tq, T_kv=T_kv, q_pos0=q_pos0, qblk=qblk, topk=topk)
+        sel, O = oracle.qsa_forward(x["Q"], x["K"], x["V"], w.Hkv, topk, q_pos0=q_pos0,
+                                    qblk=qblk)
+        G = w.Hq // w.Hkv
+        mask = torch.zeros(w.B, w.Hq, Tq, T_kv, dtype=torch.bool)
+        for b in range(w.B):
+            for h in range(w.Hq):
+                for t in range(Tq):
+                    p = q_pos0 + t
+                    for j in sel["idx"][b, h // G, t // qblk]:
+                        if j >= 0:
+                            mask[b, h, t, j * 64:min((j + 1) * 64, p + 1)] = True
+        ref = _sdpa_f64(x["Q"], x["K"], x["V"], mask, w.sm_scale)
+        assert np.abs(O - ref).max() < 1e-12
+        if qblk == 1:
+            # decode with every block kept == last rows of dense causal attention
+            _, Ofull = oracle.qsa_forward(x["Q"], x["K"], x["V"], w.Hkv, T_kv // 64 + 1,
+                                          q_pos0=q_pos0, qblk=1)
+            causal = torch.zeros(Tq, T_kv, dtype=torch.bool)
+            for t in range(Tq):
+                causal[t, :q_pos0 + t + 1] = True
+            ref = _sdpa_f64(x["Q"], x["K"], x["V"], causal, w.sm_scale)
+            assert np.abs(Ofull - ref).max() < 1e-12
+
+
+def test_attend_affine_uniform_and_permutation():
+    g = torch.Generator().manual_seed(10)
+    B, Tq, Hq, Hkv, d, T_kv, topk = 1, 128, 8, 2, 16, 512, 3
+    Q = rand_grid((B, Tq, Hq, d), g)
+    K = rand_grid((B, Hkv, T_kv, d), g)
+    V = rand_grid((B, Hkv, T_kv, d), g)
+    idx = np.full((B, Hkv, 2, topk), -1, dtype=np.int32)
+    idx[0, :, 0] = [0, 3, 6]
+    idx[0, :, 1] = [0, 2, 7]
+    q_pos0 = 384
+    O = oracle.attend(Q, K, V, idx, q_pos0, 64, 0.25)
+    O2 = oracle.attend(Q, K, bf16(2.0 * V.float() + 1.0), idx, q_pos0, 64, 0.25)
+    assert np.allclose(O2, 2.0 * O + 1.0, rtol=0, atol=1e-12)
+    # zero queries: uniform weights -> mean of the visible values; lse = log(n)
+    Z = bf16(torch.zeros_like(Q.float()))
+    Oz, lse = oracle.attend(Z, K, V, idx, q_pos0, 64, 0.25, want_lse=True)
+    Vf = f64(V)
+    for t in [0, 5, 63, 64, 100, 127]:
+        p = q_pos0 + t
+        blocks = idx[0, 0, t // 64]
+        rows = [u for j in blocks for u in range(j * 64, (j + 1) * 64) if u <= p]
+        assert np.allclose(Oz[0, t, 0], Vf[0, 0, rows].mean(axis=0), rtol=0, atol=1e-12)
+        assert lse[0, t, 0] == pytest.approx(math.log(len(rows)), abs=1e-12)
+    # permuting heads within a group permutes the output the same way
+    perm = torch.tensor([1, 3, 0, 2, 6, 4, 7, 5])
+    Op = oracle.attend(Q[:, :, perm], K, V, idx, q_pos0, 64, 0.25)
+    assert np.array_equal(Op, O[:, :, perm.numpy()])
+    # an index after the token's position is an error
+    bad = idx.copy()
+    bad[0, 0, 0, 2] = 7
+    with pytest.raises(ValueError):
+        oracle.attend(Q, K, V, bad, q_pos0, 64, 0.25)
+
+
+def test_jaccard_definition():
+    """J(A,B) = |A n B| / |A u B| (page "Qwen4 in llama.cpp", section "QSA Is
+    an Address-Selection Problem")."""
+    from tests.helpers import jaccard
+    assert jaccard([0, 1, 2, 5], [0, 2, 5, 7]) == pytest.approx(3 / 5)
+    assert jaccard([0, 3], [0, 3]) == 1.0
+    assert jaccard([0, -1, 4], [0, 4, -1]) == 1.0
