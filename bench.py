@@ -1,0 +1,448 @@
+"""QSA hot-path benchmark (one JSON line on rank 0).
+
+Headline: QSA prefill tokens/s at a 128K context (batch 1, T=131072, 16 q
+heads / 2 KV heads, d=128, 64-token blocks, top-32), one step = compress
+the new key blocks -> pool/score/select -> sparse attention, with inputs
+resident in HBM.  Also reported: decode microseconds per token at 128K
+(32 sequences x 131072-token caches, top-64 per token; one step =
+per-token selection + split-K attention; the cache summaries are the
+persistent state and are built before timing).
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier
+and a device synchronise on both sides; each step is bracketed by CUDA
+events on the launching stream and an L2 flush (a 256 MiB write) runs
+between steps outside the events.  Multi-GPU: one process per GPU, each
+rank runs its own sequence (weak scaling, no data-path collective); the
+time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the path's reference
+implementation here) on a bounded sample of the same workload.
+"""
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+PREFILL = "prefill_128k"
+DECODE = "decode_128k"
+METRIC = "QSA prefill tokens/s and decode us/token at 128K ctx; % of TC / HBM roofline"
+UNIT = "tokens/s"
+
+
+# ------------------------------------------------------------ utilities
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def prefill_flops(w):
+    """Algorithmic FLOPs of the sparse attention: 4*d*Hq per unmasked
+    (query, key) pair inside the selected blocks (masked half of the
+    diagonal block excluded)."""
+    pairs = 0
+    for i in range(w.n_rows):
+        t0, t1 = i * 64, min((i + 1) * 64, w.Tq)
+        D = (w.q_pos0 + t1 - 1) // 64
+        nsel = min(w.topk, D + 1)
+        full = nsel - 1                      # fully visible non-diagonal blocks
+        for t in range(t0, t1):
+            p = w.q_pos0 + t
+            pairs += 64 * full + (p - 64 * D + 1)
+    return 4.0 * w.d * w.Hq * pairs * w.B
+
+
+def decode_bytes(w):
+    """Selected K+V bytes per decode step (all sequences)."""
+    D = (w.q_pos0) // 64
+    nsel = min(w.topk, D + 1)
+    keys = 64 * (nsel - 1) + (w.q_pos0 - 64 * D + 1)
+    return 2 * 2 * w.d * w.Hkv * keys * w.B
+
+
+# ------------------------------------------------------------- our arm
+def run_qsa(args, ws, rank, local):
+    import block_sparse_long_compress_b200 as qsa
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    wp = synthetic.CONFIGS[args.workload]
+    if ws > 1:
+        wp = synthetic.Workload(**{**wp.__dict__, "seed": wp.seed + 1000 * rank})
+    x = synthetic.generate(wp, dev)
+    Q, K, V = x["Q"], x["K"], x["V"]
+    run = qsa.QSAPrefill(wp.B, wp.Tq, wp.Hq, wp.Hkv, wp.d, wp.T_kv, wp.topk, wp.q_pos0, device=dev)
+    run.precompress_cache(K)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        if ev is None:
+            return run(Q, K, V)
+        ev[0].record(stream)
+        qsa.compress_keys(K, run.Kc, run.blk_begin, run.blk_end)
+        ev[1].record(stream)
+        qsa.score_select(Q, run.Kc, run.idx, run.topk, run.q_pos0, 64, run.sm_scale, run.ws)
+        ev[2].record(stream)
+        qsa.sparse_attn_prefill(Q, K, V, run.idx, run.O, run.q_pos0, run.sm_scale, run.lse)
+        ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, det = qsa.device_status()
+    if st != "QSA_OK":
+        raise RuntimeError(f"device status {st} ({det})")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    n0 = qsa.launch_count()
+    with ClockSampler(local) as clk:
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)
+            step(evs[k])
+        torch.cuda.synchronize()
+    n_launch = qsa.launch_count() - n0
+    if ws > 1:
+        torch.distributed.barrier()
+    st, det = qsa.device_status()
+    if st != "QSA_OK":
+        raise RuntimeError(f"device status {st} ({det})")
+    t_comp = np.array([e[0].elapsed_time(e[1]) for e in evs])
+    t_sel = np.array([e[1].elapsed_time(e[2]) for e in evs])
+    t_att = np.array([e[2].elapsed_time(e[3]) for e in evs])
+    t_step = np.array([e[0].elapsed_time(e[3]) for e in evs])
+    ms = float(t_step.sum() / args.steps)
+    ms_all = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if ws > 1:
+        torch.distributed.all_reduce(ms_all, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(ms_all.item())
+    tokens = wp.B * wp.Tq
+    value = tokens * ws / (ms_max * 1e-3)
+
+    flops = prefill_flops(wp)
+    att_s = float(t_att.mean()) * 1e-3
+    achieved = flops / att_s / 1e12
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wp.name, "batch": wp.B, "seq_len": wp.Tq, "q_heads": wp.Hq,
+                   "kv_heads": wp.Hkv, "head_dim": wp.d, "block": 64, "topk": wp.topk,
+                   "parallelism": f"dp{ws} (independent sequences)",
+                   "l2": "flushed between steps (256 MiB write); inputs also exceed L2"},
+        "breakdown_ms": {"compress": float(t_comp.mean()), "score_select": float(t_sel.mean()),
+                         "attention": float(t_att.mean())},
+        "roofline": {"bound": "tensor", "kernel": "sparse_attn_prefill_kernel",
+                     "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"],
+                     "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
+                                           if peaks.get("bf16_tflops_sustained") else None),
+                     "peak_source": peaks["source"] + " bf16 burst", "flops_per_launch": flops,
+                     "traffic": None},
+        "gpu_launches": int(n_launch),
+        "clocks": clk.summary(),
+    }
+
+    # ---- decode at 128K (same process, after the prefill tensors are freed)
+    if not args.no_decode:
+        del Q, K, V, run, x
+        torch.cuda.empty_cache()
+        result["decode"] = bench_decode(args, qsa, dev, peaks, ws, rank, flush)
+
+    # ---- e2e through the public API with host buffers
+    if not args.no_e2e:
+        result["e2e"] = bench_e2e(args, qsa, dev, wp, ws)
+    return result
+
+
+def bench_decode(args, qsa, dev, peaks, ws, rank, flush):
+    wd = synthetic.CONFIGS[args.decode_workload]
+    if ws > 1:
+        wd = synthetic.Workload(**{**wd.__dict__, "seed": wd.seed + 1000 * rank})
+    x = synthetic.generate(wd, dev)
+    q = x["Q"].view(wd.B, wd.Hq, wd.d)
+    K, V = x["K"], x["V"]
+    L = wd.q_pos0 + 1
+    dec = qsa.QSADecode(wd.B, wd.Hq, wd.Hkv, wd.d, wd.T_kv, wd.topk, device=dev)
+    dec.compress(K, 0, L // 64)           # persistent summaries (untimed)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        dec(q, K, V, L)
+    torch.cuda.synchronize()
+    steps = max(args.steps, 20)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    sel_ws = dec._sel_ws[L]
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for k in range(steps):
+        flush.fill_(k & 0xFF)
+        evs[k][0].record(stream)
+        qsa.score_select(q.view(wd.B, 1, wd.Hq, wd.d), dec.Kc, dec.idx, wd.topk, L - 1, 1,
+                         dec.sm_scale, sel_ws)
+        evs[k][1].record(stream)
+        qsa.decode(q, K, V, dec.idx, dec.o, L, dec.sm_scale, dec.ws_dec)
+        evs[k][2].record(stream)
+    torch.cuda.synchronize()
+    st, det = qsa.device_status()
+    if st != "QSA_OK":
+        raise RuntimeError(f"decode device status {st} ({det})")
+    t_sel = np.array([e[0].elapsed_time(e[1]) for e in evs])
+    t_att = np.array([e[1].elapsed_time(e[2]) for e in evs])
+    t_step = t_sel + t_att
+    us_step = float(t_step.mean()) * 1e3
+    by = decode_bytes(wd)
+    att_gbs = by / (float(t_att.mean()) * 1e-3) / 1e9
+    sel_bytes = wd.B * wd.Hkv * ((L - 1) // 64) * wd.d * 4   # fp32 summaries read by scoring
+    return {"workload": wd.name, "batch": wd.B, "context": L, "topk": wd.topk,
+            "us_per_step": us_step, "us_per_token": us_step / wd.B,
+            "breakdown_us": {"score_select": float(t_sel.mean()) * 1e3,
+                             "attention": float(t_att.mean()) * 1e3},
+            "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": att_gbs,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": att_gbs / peaks["hbm_gbs"], "bytes_per_launch": by,
+                         "traffic": None},
+            "select_gbs": sel_bytes / (float(t_sel.mean()) * 1e-3) / 1e9}
+
+
+def bench_e2e(args, qsa, dev, wp, ws):
+    """Same metric through the public API, host buffers in and out: every
+    step copies Q, K, V from pinned host memory and reads O back."""
+    g = synthetic.generate(wp, dev)
+    x = {k: g[k].cpu() for k in ("Q", "K", "V")}
+    del g
+    hQ, hK, hV = (x[k].pin_memory() for k in ("Q", "K", "V"))
+    hO = torch.empty((wp.B, wp.Tq, wp.Hq, wp.d), dtype=torch.bfloat16).pin_memory()
+    dQ, dK, dV = (torch.empty_like(t, device=dev) for t in (hQ, hK, hV))
+    run = qsa.QSAPrefill(wp.B, wp.Tq, wp.Hq, wp.Hkv, wp.d, wp.T_kv, wp.topk, wp.q_pos0, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        dQ.copy_(hQ, non_blocking=True)
+        dK.copy_(hK, non_blocking=True)
+        dV.copy_(hV, non_blocking=True)
+        if run.blk_begin > 0:
+            run.precompress_cache(dK)
+        O = run(dQ, dK, dV)
+        hO.copy_(O, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if ws > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms = float(t.item())
+    h2d = sum(a.numel() * a.element_size() for a in (hQ, hK, hV))
+    d2h = hO.numel() * hO.element_size()
+    return {"value": wp.B * wp.Tq * ws / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+# ----------------------------------------------------- CPU oracle timing
+def oracle_sample(wp, x_cpu, budget_s):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the
+    workload: all summaries up to the sampled rows, the pooled queries, the
+    selection of the sampled query blocks and the attention of all their
+    tokens.  Returns (tokens/s, description, threads)."""
+    import oracle
+
+    nthreads = oracle.threads()
+    # rows taken from the end of the sequence (full top-k), one per group
+    # pair, as many as fit the budget after a one-row probe
+    def run(rows):
+        t0 = time.perf_counter()
+        n_complete = (wp.q_pos0 + wp.Tq) // 64
+        Kc = oracle.compress_keys(x_cpu["K"], 0, n_complete)
+        Qbar = oracle.pool_queries(x_cpu["Q"], wp.Hkv, wp.qblk)
+        flat = [(b * wp.Hkv + g) * wp.n_rows + i
+                for b in range(wp.B) for g in range(wp.Hkv) for i in rows]
+        sel = oracle.select(Qbar, Kc, wp.Tq, wp.q_pos0, wp.qblk, wp.topk, wp.sm_scale, rows=flat)
+        idx = np.full((wp.B * wp.Hkv * wp.n_rows, wp.topk), -1, dtype=np.int32)
+        idx[flat] = sel["idx"]
+        idx = idx.reshape(wp.B, wp.Hkv, wp.n_rows, wp.topk)
+        toks = [b * wp.Tq + t for b in range(wp.B) for i in rows
+                for t in range(i * wp.qblk, min((i + 1) * wp.qblk, wp.Tq))]
+        oracle.attend(x_cpu["Q"], x_cpu["K"], x_cpu["V"], idx, wp.q_pos0, wp.qblk,
+                      wp.sm_scale, tokens=toks)
+        return time.perf_counter() - t0, len(toks)
+
+    t1, n1 = run([wp.n_rows - 1])
+    nrows = max(1, min(wp.n_rows, int(budget_s / max(t1, 1e-3))))
+    rows = list(range(wp.n_rows - nrows, wp.n_rows))
+    t, n = run(rows)
+    desc = (f"{len(rows)} query blocks x {wp.B} seq ({n} query tokens, all {wp.Hq} heads) of "
+            f"{wp.name}: whole-cache compress + pooling of all rows + selection and attention of the "
+            f"sampled rows, fp64")
+    return n / t, desc, nthreads
+
+
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return None
+    wp = synthetic.CONFIGS[args.workload]
+    x = synthetic.generate(wp, "cuda" if torch.cuda.is_available() else "cpu")
+    x_cpu = {k: x[k].cpu() for k in ("Q", "K", "V")}
+    del x
+    per_step = []
+    desc = threads = None
+    budget = max(2.0, args.ref_budget / max(1, args.steps + args.warmup))
+    for k in range(args.warmup + args.steps):
+        v, desc, threads = oracle_sample(wp, x_cpu, budget)
+        if k >= args.warmup:
+            per_step.append(v)
+    value = float(np.mean(per_step))
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": wp.name, "batch": wp.B, "seq_len": wp.Tq, "q_heads": wp.Hq,
+                       "kv_heads": wp.Hkv, "head_dim": wp.d, "block": 64, "topk": wp.topk},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="qsa", choices=["qsa", "reference"])
+    ap.add_argument("--workload", default=PREFILL, choices=sorted(synthetic.CONFIGS))
+    ap.add_argument("--decode-workload", default=DECODE, choices=sorted(synthetic.CONFIGS))
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
+    ap.add_argument("--ref-budget", type=float, default=60.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import datetime
+        backend = "nccl" if args.impl == "qsa" else "gloo"
+        if args.impl == "reference" and rank != 0:
+            return
+        if args.impl == "qsa":
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    if args.impl == "reference":
+        res = run_reference(args, ws, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    res = run_qsa(args, ws, rank, local)
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        wp = synthetic.CONFIGS[args.workload]
+        g = synthetic.generate(wp, torch.device("cuda", local))
+        x_cpu = {k: g[k].cpu() for k in ("Q", "K", "V")}
+        del g
+        v, desc, threads = oracle_sample(wp, x_cpu, args.cpu_budget)
+        res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+                               "sample": desc}
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,269 @@
+"""B200-native Qwen Sparse Attention (QSA) hot path.
+
+Thin ctypes binding over ``libqsa.so`` (C ABI in ``include/qsa.h``).  Every
+step of the path runs in the library's sm_100a kernels; this module only
+checks tensor metadata and passes pointers, sizes and the current CUDA
+stream.  PyTorch supplies device memory and streams.  There is no CPU or
+PyTorch fallback: if the library is missing, importing this package raises.
+
+Steps (pages "Qwen4 architecture: QSA, GR, PLE", section "1. QSA: not
+looking at every token equally"; "Qwen4 in llama.cpp: Dissecting PR
+#27742", section "QSA Is an Address-Selection Problem, Not a New Attention
+Equation"):
+    compress_keys        mean-pooled 64-token key summaries (fp32)
+    score_select         pooled-query fp32 block scores -> top-k block ids
+    sparse_attn_prefill  tcgen05/TMEM attention over the selected blocks
+    decode               split-K single-token attention over the selected blocks
+"""
+import ctypes
+import os
+import re
+
+import torch
+
+BLOCK = 64
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqsa.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "qsa.h")
+
+STATUS = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_UNSUPPORTED", 3: "QSA_ERR_CUDA",
+          4: "QSA_ERR_TIMEOUT", 5: "QSA_ERR_BOUNDS", 6: "QSA_ERR_WORKSPACE"}
+
+
+class QSAError(RuntimeError):
+    def __init__(self, code, what):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)}")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing; build it with "
+            "`python block_sparse_long_compress_b200/build.py` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, S, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    sig = {
+        "qsa_compress_keys": (I, [P, P, I, I, I, I, I, I, P]),
+        "qsa_score_select_workspace": (S, [I, I, I, I, I, I, I, I]),
+        "qsa_score_select": (I, [P, P, P, I, I, I, I, I, I, I, I, I, F, P, S, P]),
+        "qsa_sparse_attn_prefill": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P]),
+        "qsa_decode_workspace": (S, [I, I, I, I, I]),
+        "qsa_decode": (I, [P, P, P, P, P, I, I, I, I, I, I, I, F, P, S, P]),
+        "qsa_get_device_status": (I, [P, ctypes.POINTER(I)]),
+        "qsa_selftest_wait_timeout": (I, [ctypes.c_uint64, P]),
+        "qsa_status_string": (ctypes.c_char_p, [I]),
+        "qsa_last_error": (ctypes.c_char_p, []),
+        "qsa_launch_count": (ctypes.c_ulonglong, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    """The loaded ctypes library handle."""
+    return _lib
+
+
+def declared_symbols():
+    """Entry points declared in include/qsa.h."""
+    text = open(HEADER_PATH).read()
+    return re.findall(r"QSA_API\s+[\w\s\*]+?\b(qsa_\w+)\s*\(", text)
+
+
+def _check(rc, what):
+    if rc != 0:
+        msg = _lib.qsa_last_error().decode()
+        raise QSAError(rc, f"{what} ({msg})" if msg else what)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t, dtype, name):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+# ------------------------------------------------------------------ steps
+def compress_keys(K, Kc, blk_begin=0, blk_end=None, stream=None):
+    """Kc[b,h,j,:] = mean of K[b,h,64j:64j+64,:] for j in [blk_begin, blk_end).
+    K: bf16 [B, Hkv, T_kv_max, d]; Kc: fp32 [B, Hkv, T_kv_max//64, d]."""
+    B, Hkv, T, d = K.shape
+    if blk_end is None:
+        blk_end = T // BLOCK
+    if tuple(Kc.shape) != (B, Hkv, T // BLOCK, d):
+        raise ValueError("Kc shape must be [B, Hkv, T_kv_max//64, d]")
+    _check(_lib.qsa_compress_keys(_ptr(K, torch.bfloat16, "K"), _ptr(Kc, torch.float32, "Kc"),
+                                  B, Hkv, T, d, blk_begin, blk_end, _stream(stream)),
+           "qsa_compress_keys")
+    return Kc
+
+
+def score_select_workspace(B, Hq, Hkv, Tq, q_pos0, qblk, d, topk):
+    return int(_lib.qsa_score_select_workspace(B, Hq, Hkv, Tq, q_pos0, qblk, d, topk))
+
+
+def score_select(Q, Kc, idx, topk, q_pos0, qblk=BLOCK, sm_scale=None, workspace=None,
+                 stream=None):
+    """Top-k block selection per (query block or token, KV group).
+    Q: bf16 [B, Tq, Hq, d]; Kc: fp32 [B, Hkv, T_kv_max//64, d];
+    idx: int32 [B, Hkv, ceil(Tq/qblk), topk] (written)."""
+    B, Tq, Hq, d = Q.shape
+    _, Hkv, nblk, _ = Kc.shape
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    need = score_select_workspace(B, Hq, Hkv, Tq, q_pos0, qblk, d, topk)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    _check(_lib.qsa_score_select(_ptr(Q, torch.bfloat16, "Q"), _ptr(Kc, torch.float32, "Kc"),
+                                 _ptr(idx, torch.int32, "idx"), B, Hq, Hkv, Tq, q_pos0, qblk,
+                                 nblk * BLOCK, d, topk, float(sm_scale),
+                                 _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                                 _stream(stream)),
+           "qsa_score_select")
+    return idx
+
+
+def sparse_attn_prefill(Q, K, V, idx, O, q_pos0=0, sm_scale=None, lse=None, stream=None):
+    """O = softmax attention of Q over the blocks in idx (keys <= position).
+    Q, O: bf16 [B, Tq, Hq, d]; K, V: bf16 [B, Hkv, T_kv_max, d];
+    idx: int32 [B, Hkv, ceil(Tq/64), topk]; lse: optional fp32 [B, Tq, Hq]."""
+    B, Tq, Hq, d = Q.shape
+    _, Hkv, T, _ = K.shape
+    topk = idx.shape[-1]
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    _check(_lib.qsa_sparse_attn_prefill(
+        _ptr(Q, torch.bfloat16, "Q"), _ptr(K, torch.bfloat16, "K"), _ptr(V, torch.bfloat16, "V"),
+        _ptr(idx, torch.int32, "idx"), _ptr(O, torch.bfloat16, "O"),
+        _ptr(lse, torch.float32, "lse"), B, Hq, Hkv, Tq, q_pos0, T, d, topk, float(sm_scale),
+        _stream(stream)), "qsa_sparse_attn_prefill")
+    return O
+
+
+def decode_workspace(B, Hq, Hkv, d, topk):
+    return int(_lib.qsa_decode_workspace(B, Hq, Hkv, d, topk))
+
+
+def decode(q, K, V, idx, o, L, sm_scale=None, workspace=None, stream=None):
+    """Single-token attention per sequence over its selected blocks.
+    q, o: bf16 [B, Hq, d] (or [B, 1, Hq, d]); K, V: bf16 [B, Hkv, T_kv_max, d];
+    idx: int32 [B, Hkv, 1, topk]; L: cache length (query at position L-1)."""
+    B, Hkv, T, d = K.shape
+    Hq = q.shape[-2]
+    topk = idx.shape[-1]
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    need = decode_workspace(B, Hq, Hkv, d, topk)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check(_lib.qsa_decode(
+        _ptr(q, torch.bfloat16, "q"), _ptr(K, torch.bfloat16, "K"), _ptr(V, torch.bfloat16, "V"),
+        _ptr(idx, torch.int32, "idx"), _ptr(o, torch.bfloat16, "o"), B, Hq, Hkv, L, T, d, topk,
+        float(sm_scale), _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+        _stream(stream)), "qsa_decode")
+    return o
+
+
+def device_status(stream=None):
+    """Synchronise the stream; return (and clear) the kernels' status word."""
+    det = ctypes.c_int(0)
+    rc = _lib.qsa_get_device_status(_stream(stream), ctypes.byref(det))
+    return STATUS.get(rc, rc), det.value
+
+
+def selftest_wait_timeout(timeout_ns, stream=None):
+    _check(_lib.qsa_selftest_wait_timeout(int(timeout_ns), _stream(stream)),
+           "qsa_selftest_wait_timeout")
+
+
+def launch_count():
+    """Kernels launched by the library so far in this process."""
+    return int(_lib.qsa_launch_count())
+
+
+# --------------------------------------------------------------- pipeline
+class QSAPrefill:
+    """The whole prefill path for one shape: compress the new complete
+    blocks, select, attend.  Owns its workspace, summaries and outputs
+    (allocated once with torch)."""
+
+    def __init__(self, B, Tq, Hq, Hkv, d, T_kv_max, topk, q_pos0=0, device="cuda",
+                 with_lse=False):
+        self.B, self.Tq, self.Hq, self.Hkv, self.d = B, Tq, Hq, Hkv, d
+        self.T_kv_max, self.topk, self.q_pos0 = T_kv_max, topk, q_pos0
+        self.sm_scale = d ** -0.5
+        NR = -(-Tq // BLOCK)
+        dev = torch.device(device)
+        self.Kc = torch.zeros((B, Hkv, T_kv_max // BLOCK, d), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((B, Hkv, NR, topk), dtype=torch.int32, device=dev)
+        self.O = torch.empty((B, Tq, Hq, d), dtype=torch.bfloat16, device=dev)
+        self.lse = (torch.empty((B, Tq, Hq), dtype=torch.float32, device=dev)
+                    if with_lse else None)
+        self.ws = torch.empty(max(1, score_select_workspace(B, Hq, Hkv, Tq, q_pos0, BLOCK, d, topk)),
+                              dtype=torch.uint8, device=dev)
+        # blocks whose summaries this step must (re)compute: the complete
+        # blocks that the new tokens finish
+        self.blk_begin = q_pos0 // BLOCK
+        self.blk_end = (q_pos0 + Tq) // BLOCK
+
+    def precompress_cache(self, K, stream=None):
+        """Summaries of the cache blocks before the new tokens (persistent state)."""
+        if self.blk_begin > 0:
+            compress_keys(K, self.Kc, 0, self.blk_begin, stream)
+
+    def __call__(self, Q, K, V, stream=None):
+        compress_keys(K, self.Kc, self.blk_begin, self.blk_end, stream)
+        score_select(Q, self.Kc, self.idx, self.topk, self.q_pos0, BLOCK, self.sm_scale,
+                     self.ws, stream)
+        sparse_attn_prefill(Q, K, V, self.idx, self.O, self.q_pos0, self.sm_scale, self.lse,
+                            stream)
+        return self.O
+
+
+class QSADecode:
+    """The whole decode path for a batch of single-token queries: select
+    (per token) then split-K attention.  Summaries of complete blocks are
+    persistent state; compress_block() adds one as it completes."""
+
+    def __init__(self, B, Hq, Hkv, d, T_kv_max, topk, device="cuda"):
+        self.B, self.Hq, self.Hkv, self.d = B, Hq, Hkv, d
+        self.T_kv_max, self.topk = T_kv_max, topk
+        self.sm_scale = d ** -0.5
+        dev = torch.device(device)
+        self.Kc = torch.zeros((B, Hkv, T_kv_max // BLOCK, d), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((B, Hkv, 1, topk), dtype=torch.int32, device=dev)
+        self.o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
+        self.ws_dec = torch.empty(decode_workspace(B, Hq, Hkv, d, topk), dtype=torch.uint8,
+                                  device=dev)
+        self._sel_ws = {}
+
+    def compress(self, K, blk_begin, blk_end, stream=None):
+        compress_keys(K, self.Kc, blk_begin, blk_end, stream)
+
+    def __call__(self, q, K, V, L, stream=None):
+        q4 = q.view(self.B, 1, self.Hq, self.d)
+        key = L
+        if key not in self._sel_ws:
+            n = score_select_workspace(self.B, self.Hq, self.Hkv, 1, L - 1, 1, self.d, self.topk)
+            self._sel_ws[key] = torch.empty(max(1, n), dtype=torch.uint8, device=q.device)
+        score_select(q4, self.Kc, self.idx, self.topk, L - 1, 1, self.sm_scale,
+                     self._sel_ws[key], stream)
+        decode(q, K, V, self.idx, self.o, L, self.sm_scale, self.ws_dec, stream)
+        return self.o

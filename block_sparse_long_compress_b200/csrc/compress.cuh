@@ -1,0 +1,63 @@
+// Step 1 -- key compression: the fp32 mean of the 64 keys of a block
+// (pages "Qwen4 architecture: QSA, GR, PLE", section 1, "compress into
+// small blocks"; "Qwen4 in llama.cpp: Dissecting PR #27742", section "QSA Is
+// an Address-Selection Problem, Not a New Attention Equation",
+// "compressed-block representation").
+//
+// HBM-bound: per block it reads 64*d bf16 and writes d fp32.  One CTA of
+// 128 threads per (b, h, block); thread t owns the 16-byte column chunk
+// t % (d/8) and the rows r = t / (d/8) + k*R (R = 128 / (d/8) row lanes),
+// issuing all its loads before the first add.  The reduction order is fixed
+// (each thread adds its rows in increasing r, then row lanes are added in
+// increasing lane order), so results are bit-reproducible.
+#pragma once
+#include "device.cuh"
+
+namespace qsa {
+
+template <int D>
+__global__ void __launch_bounds__(128) compress_keys_kernel(const __nv_bfloat16 *__restrict__ K,
+                                                            float *__restrict__ Kc, int T_kv_max,
+                                                            int nblk_max, int blk_begin,
+                                                            int nblk)
+{
+    constexpr int CHUNKS = D / 8;            // 16-byte chunks per key row
+    constexpr int LANES = 128 / CHUNKS;      // row lanes
+    constexpr int ROWS = 64 / LANES;         // rows per thread
+    __shared__ float part[LANES][D];
+
+    const int j = blk_begin + (int)(blockIdx.x % (unsigned)nblk);
+    const long bh = blockIdx.x / (unsigned)nblk;
+    const int t = threadIdx.x;
+    const int c = t % CHUNKS, lane = t / CHUNKS;
+
+    const uint4 *src = reinterpret_cast<const uint4 *>(K + ((bh * T_kv_max) + (long)j * 64) * D);
+    uint4 v[ROWS];
+#pragma unroll
+    for (int k = 0; k < ROWS; k++) v[k] = __ldg(src + (long)(lane + k * LANES) * CHUNKS + c);
+
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; e++) acc[e] = 0.f;
+#pragma unroll
+    for (int k = 0; k < ROWS; k++) {
+        const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&v[k]);
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            float2 f = __bfloat1622float2(p[e]);
+            acc[2 * e] += f.x;
+            acc[2 * e + 1] += f.y;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; e++) part[lane][c * 8 + e] = acc[e];
+    __syncthreads();
+    if (t < D) {
+        float s = 0.f;
+#pragma unroll
+        for (int l = 0; l < LANES; l++) s += part[l][t];
+        Kc[(bh * nblk_max + j) * D + t] = s * (1.0f / 64.0f);
+    }
+}
+
+}  // namespace qsa

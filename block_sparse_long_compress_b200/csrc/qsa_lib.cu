@@ -1,0 +1,416 @@
+// libqsa.so -- host side of the C ABI declared in include/qsa.h.
+// One translation unit holds every kernel (so the device status word is a
+// single symbol) and the launch code: argument checks, TMA descriptor
+// encoding, grid sizing and launches on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "../../include/qsa.h"
+#include "compress.cuh"
+#include "decode.cuh"
+#include "device.cuh"
+#include "prefill.cuh"
+#include "select.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+std::atomic<unsigned long long> g_launches{0};
+
+qsa_status fail(qsa_status s, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+qsa_status check_launch(const char *what)
+{
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return QSA_OK;
+}
+
+// Called after each kernel launch of the library.
+qsa_status launched(const char *what)
+{
+    qsa_status s = check_launch(what);
+    if (s == QSA_OK) g_launches.fetch_add(1, std::memory_order_relaxed);
+    return s;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 view [rows][cols] (cols contiguous) with 64 x 64 boxes, 128-byte swizzle.
+qsa_status make_map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(QSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(QSA_ERR_CUDA, "cuTensorMapEncodeTiled(2d) failed: %d", (int)r);
+    return QSA_OK;
+}
+
+// 3-D bf16 view of Q: [tokens][heads][d] with boxes (64 cols, G heads, TOK tokens).
+qsa_status make_map_q(CUtensorMap *m, const void *base, uint64_t tokens, uint64_t heads, uint64_t d,
+                      uint32_t box_heads, uint32_t box_tokens)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(QSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[3] = {d, heads, tokens};
+    cuuint64_t strides[2] = {d * 2, heads * d * 2};
+    cuuint32_t box[3] = {64, box_heads, box_tokens};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(QSA_ERR_CUDA, "cuTensorMapEncodeTiled(3d) failed: %d", (int)r);
+    return QSA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool supported_d(int d) { return d == 64 || d == 128; }
+
+// ------------------------------------------------------- select geometry
+struct SelectPlan {
+    int NR, CH, maxchunks;
+    size_t qbar_bytes, part_bytes;
+};
+
+SelectPlan plan_select(int B, int Hkv, int Tq, int q_pos0, int qblk, int d)
+{
+    SelectPlan p;
+    p.NR = (Tq + qblk - 1) / qblk;
+    const int Dmax = (q_pos0 + Tq - 1) / 64;
+    const int ncand = Dmax > 1 ? Dmax - 1 : 0;
+    const long rows = (long)B * Hkv * p.NR;
+    int CH = 2048;
+    // enough CTAs to cover the SMs a few times over
+    while (CH > 512 && rows * ((ncand + CH - 1) / CH) < 4 * 148) CH /= 2;
+    p.CH = CH;
+    p.maxchunks = ncand > 0 ? (ncand + CH - 1) / CH : 1;
+    p.qbar_bytes = align256((size_t)rows * d * sizeof(float));
+    p.part_bytes = p.maxchunks > 1 ? align256((size_t)rows * p.maxchunks * qsa::kMaxChosen * 8) : 0;
+    return p;
+}
+
+// ------------------------------------------------------- decode geometry
+constexpr int kDecodeWarps = 2;
+
+struct DecodePlan {
+    int nsplit;
+    size_t m_off, l_off, o_off, t_off, total;
+};
+
+DecodePlan plan_decode(int B, int Hkv, int d, int topk)
+{
+    DecodePlan p;
+    p.nsplit = (topk + kDecodeWarps - 1) / kDecodeWarps;
+    const size_t rows = (size_t)B * Hkv * p.nsplit * 8;
+    p.m_off = 0;
+    p.l_off = align256(rows * 4);
+    p.o_off = p.l_off + align256(rows * 4);
+    p.t_off = p.o_off + align256(rows * d * 4);
+    p.total = p.t_off + align256((size_t)B * Hkv * 4);
+    return p;
+}
+
+template <typename K>
+qsa_status set_smem(K kernel, int bytes)
+{
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return check_launch("cudaFuncSetAttribute");
+    return QSA_OK;
+}
+
+// ------------------------------------------------------------ launchers
+template <int D, int G>
+qsa_status launch_prefill(const void *Q, const void *K, const void *V, const int32_t *idx, void *O,
+                          float *lse, int B, int Hq, int Hkv, int Tq, int q_pos0, int T_kv_max,
+                          int topk, float sm_scale, cudaStream_t s)
+{
+    using C = qsa::PrefillCfg<D, G>;
+    CUtensorMap mq, mk, mv;
+    qsa_status st;
+    if ((st = make_map_q(&mq, Q, (uint64_t)B * Tq, Hq, D, G, C::TOK)) != QSA_OK) return st;
+    if ((st = make_map_2d(&mk, K, (uint64_t)B * Hkv * T_kv_max, D)) != QSA_OK) return st;
+    if ((st = make_map_2d(&mv, V, (uint64_t)B * Hkv * T_kv_max, D)) != QSA_OK) return st;
+    auto kern = qsa::sparse_attn_prefill_kernel<D, G>;
+    if ((st = set_smem(kern, C::SMEM_REQUEST)) != QSA_OK) return st;
+    const int NR = (Tq + 63) / 64;
+    dim3 grid(NR * C::TILES, B * Hkv);
+    kern<<<grid, C::THREADS, C::SMEM_REQUEST, s>>>(mq, mk, mv, idx, (__nv_bfloat16 *)O, lse, Tq, Hq, Hkv,
+                                                   q_pos0, T_kv_max, topk,
+                                                   sm_scale * 1.4426950408889634f);
+    return launched("sparse_attn_prefill_kernel");
+}
+
+template <int D, int G>
+qsa_status launch_decode(const void *q, const void *K, const void *V, const int32_t *idx, void *o,
+                         int B, int Hq, int Hkv, int L, int T_kv_max, int topk, float sm_scale,
+                         void *ws, cudaStream_t s)
+{
+    using C = qsa::DecodeCfg<D>;
+    CUtensorMap mk, mv;
+    qsa_status st;
+    if ((st = make_map_2d(&mk, K, (uint64_t)B * Hkv * T_kv_max, D)) != QSA_OK) return st;
+    if ((st = make_map_2d(&mv, V, (uint64_t)B * Hkv * T_kv_max, D)) != QSA_OK) return st;
+    const DecodePlan p = plan_decode(B, Hkv, D, topk);
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    qsa::DecodePartial part{reinterpret_cast<float *>(w + p.m_off), reinterpret_cast<float *>(w + p.l_off),
+                            reinterpret_cast<float *>(w + p.o_off), reinterpret_cast<int *>(w + p.t_off)};
+    if (cudaMemsetAsync(part.ticket, 0, (size_t)B * Hkv * 4, s) != cudaSuccess) return check_launch("memset");
+    auto kern = qsa::decode_kernel<D, G, kDecodeWarps>;
+    const int smem = kDecodeWarps * C::WARP_BYTES + 1024;
+    if ((st = set_smem(kern, smem)) != QSA_OK) return st;
+    dim3 grid(p.nsplit, B * Hkv);
+    kern<<<grid, kDecodeWarps * 32, smem, s>>>(mk, mv, (const __nv_bfloat16 *)q, idx, (__nv_bfloat16 *)o, part,
+                                              Hq, Hkv, L, T_kv_max, topk, sm_scale * 1.4426950408889634f);
+    return launched("decode_kernel");
+}
+
+__global__ void selftest_wait_kernel(uint64_t limit_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        qsa::mbar_init(&bar, 1);   // nothing ever arrives
+        qsa::fence_barrier_init();
+    }
+    __syncthreads();
+    qsa::mbar_wait(&bar, 0, &abort_flag, 99, limit_ns);
+}
+
+}  // namespace
+
+// ===================================================================== C ABI
+extern "C" {
+
+qsa_status qsa_compress_keys(const void *K, float *Kc, int B, int Hkv, int T_kv_max, int d, int blk_begin,
+                             int blk_end, qsa_stream_t stream)
+{
+    if (!K || !Kc) return fail(QSA_ERR_INVALID_ARG, "qsa_compress_keys: null pointer");
+    if (B <= 0 || Hkv <= 0 || T_kv_max <= 0 || T_kv_max % 64)
+        return fail(QSA_ERR_INVALID_ARG, "qsa_compress_keys: bad shape");
+    const int nblk_max = T_kv_max / 64;
+    if (blk_begin < 0 || blk_end < blk_begin || blk_end > nblk_max)
+        return fail(QSA_ERR_INVALID_ARG, "qsa_compress_keys: block range [%d,%d) outside [0,%d]", blk_begin,
+                    blk_end, nblk_max);
+    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "qsa_compress_keys: d=%d", d);
+    if (!aligned16(K) || !aligned16(Kc)) return fail(QSA_ERR_INVALID_ARG, "qsa_compress_keys: misaligned");
+    const int nblk = blk_end - blk_begin;
+    if (nblk == 0) return QSA_OK;
+    const long grid = (long)B * Hkv * nblk;
+    if (grid >= (1L << 31)) return fail(QSA_ERR_UNSUPPORTED, "qsa_compress_keys: too many blocks");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 128)
+        qsa::compress_keys_kernel<128><<<(unsigned)grid, 128, 0, s>>>((const __nv_bfloat16 *)K, Kc, T_kv_max,
+                                                                      nblk_max, blk_begin, nblk);
+    else
+        qsa::compress_keys_kernel<64><<<(unsigned)grid, 128, 0, s>>>((const __nv_bfloat16 *)K, Kc, T_kv_max,
+                                                                     nblk_max, blk_begin, nblk);
+    return launched("compress_keys_kernel");
+}
+
+size_t qsa_score_select_workspace(int B, int Hq, int Hkv, int Tq, int q_pos0, int qblk, int d, int topk)
+{
+    (void)Hq;
+    (void)topk;
+    if (B <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || (qblk != 1 && qblk != 64) || !supported_d(d)) return 0;
+    const SelectPlan p = plan_select(B, Hkv, Tq, q_pos0, qblk, d);
+    return p.qbar_bytes + p.part_bytes;
+}
+
+qsa_status qsa_score_select(const void *Q, const float *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
+                            int q_pos0, int qblk, int T_kv_max, int d, int topk, float sm_scale,
+                            void *workspace, size_t workspace_bytes, qsa_stream_t stream)
+{
+    if (!Q || !Kc || !idx) return fail(QSA_ERR_INVALID_ARG, "qsa_score_select: null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || T_kv_max <= 0 || T_kv_max % 64 ||
+        Hq % Hkv)
+        return fail(QSA_ERR_INVALID_ARG, "qsa_score_select: bad shape");
+    if (qblk != 1 && qblk != 64) return fail(QSA_ERR_UNSUPPORTED, "qsa_score_select: qblk=%d", qblk);
+    if (qblk == 64 && q_pos0 % 64)
+        return fail(QSA_ERR_INVALID_ARG, "qsa_score_select: q_pos0 must be a multiple of 64 when qblk=64");
+    if ((long)q_pos0 + Tq > T_kv_max) return fail(QSA_ERR_INVALID_ARG, "qsa_score_select: queries past the cache");
+    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "qsa_score_select: d=%d", d);
+    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "qsa_score_select: topk=%d", topk);
+    if ((long)Hq * d / 8 > 1024) return fail(QSA_ERR_UNSUPPORTED, "qsa_score_select: Hq*d too large");
+    if (!aligned16(Q) || !aligned16(Kc) || !aligned16(idx))
+        return fail(QSA_ERR_INVALID_ARG, "qsa_score_select: misaligned pointer");
+    const SelectPlan p = plan_select(B, Hkv, Tq, q_pos0, qblk, d);
+    if (p.maxchunks * qsa::kMaxChosen * 8 > 200 * 1024)
+        return fail(QSA_ERR_UNSUPPORTED, "qsa_score_select: context too long");
+    if (!workspace || workspace_bytes < p.qbar_bytes + p.part_bytes || !aligned16(workspace))
+        return fail(QSA_ERR_WORKSPACE, "qsa_score_select: workspace needs %zu bytes",
+                    p.qbar_bytes + p.part_bytes);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float *Qbar = static_cast<float *>(workspace);
+    uint64_t *part = reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(workspace) + p.qbar_bytes);
+    const int nblk_max = T_kv_max / 64;
+    const int pool_threads = ((Hq * d / 8) + 31) / 32 * 32;
+    const int pool_smem = Hq * d * 4;
+    dim3 pgrid(p.NR, B), sgrid(p.maxchunks, p.NR, B * Hkv), mgrid(p.NR, B * Hkv);
+    const int ssmem = p.CH * 8;
+    qsa_status st;
+    if (d == 128) {
+        if ((st = set_smem(qsa::pool_queries_kernel<128>, pool_smem)) != QSA_OK) return st;
+        qsa::pool_queries_kernel<128><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq,
+                                                                             Hq, Hkv, qblk);
+        if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
+        if ((st = set_smem(qsa::score_select_kernel<128>, ssmem)) != QSA_OK) return st;
+        qsa::score_select_kernel<128><<<sgrid, qsa::kSelThreads, ssmem, s>>>(
+            Qbar, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk, sm_scale, p.CH, p.maxchunks);
+    } else {
+        if ((st = set_smem(qsa::pool_queries_kernel<64>, pool_smem)) != QSA_OK) return st;
+        qsa::pool_queries_kernel<64><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq,
+                                                                            Hq, Hkv, qblk);
+        if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
+        if ((st = set_smem(qsa::score_select_kernel<64>, ssmem)) != QSA_OK) return st;
+        qsa::score_select_kernel<64><<<sgrid, qsa::kSelThreads, ssmem, s>>>(
+            Qbar, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk, sm_scale, p.CH, p.maxchunks);
+    }
+    if ((st = launched("score_select_kernel")) != QSA_OK) return st;
+    if (p.maxchunks > 1) {
+        const int msmem = p.maxchunks * qsa::kMaxChosen * 8;
+        if ((st = set_smem(qsa::merge_select_kernel, msmem)) != QSA_OK) return st;
+        qsa::merge_select_kernel<<<mgrid, qsa::kSelThreads, msmem, s>>>(part, idx, Tq, q_pos0, qblk, topk, p.CH,
+                                                                       p.maxchunks);
+        if ((st = launched("merge_select_kernel")) != QSA_OK) return st;
+    }
+    return QSA_OK;
+}
+
+qsa_status qsa_sparse_attn_prefill(const void *Q, const void *K, const void *V, const int32_t *idx, void *O,
+                                   float *lse, int B, int Hq, int Hkv, int Tq, int q_pos0, int T_kv_max, int d,
+                                   int topk, float sm_scale, qsa_stream_t stream)
+{
+    if (!Q || !K || !V || !idx || !O) return fail(QSA_ERR_INVALID_ARG, "qsa_sparse_attn_prefill: null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || T_kv_max <= 0 || T_kv_max % 64 || Hq % Hkv)
+        return fail(QSA_ERR_INVALID_ARG, "qsa_sparse_attn_prefill: bad shape");
+    if (q_pos0 % 64) return fail(QSA_ERR_INVALID_ARG, "qsa_sparse_attn_prefill: q_pos0 must be a multiple of 64");
+    if ((long)q_pos0 + Tq > T_kv_max)
+        return fail(QSA_ERR_INVALID_ARG, "qsa_sparse_attn_prefill: queries past the cache");
+    if ((long)B * Hkv * T_kv_max >= (1L << 31) || (long)B * Tq >= (1L << 31))
+        return fail(QSA_ERR_UNSUPPORTED, "qsa_sparse_attn_prefill: tensor too large");
+    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "qsa_sparse_attn_prefill: d=%d", d);
+    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "qsa_sparse_attn_prefill: topk=%d", topk);
+    const int G = Hq / Hkv;
+    if (G != 4 && G != 8) return fail(QSA_ERR_UNSUPPORTED, "qsa_sparse_attn_prefill: Hq/Hkv=%d", G);
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(idx) || !aligned16(O))
+        return fail(QSA_ERR_INVALID_ARG, "qsa_sparse_attn_prefill: misaligned pointer");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 128 && G == 8) return launch_prefill<128, 8>(Q, K, V, idx, O, lse, B, Hq, Hkv, Tq, q_pos0, T_kv_max, topk, sm_scale, s);
+    if (d == 128 && G == 4) return launch_prefill<128, 4>(Q, K, V, idx, O, lse, B, Hq, Hkv, Tq, q_pos0, T_kv_max, topk, sm_scale, s);
+    if (d == 64 && G == 8) return launch_prefill<64, 8>(Q, K, V, idx, O, lse, B, Hq, Hkv, Tq, q_pos0, T_kv_max, topk, sm_scale, s);
+    return launch_prefill<64, 4>(Q, K, V, idx, O, lse, B, Hq, Hkv, Tq, q_pos0, T_kv_max, topk, sm_scale, s);
+}
+
+size_t qsa_decode_workspace(int B, int Hq, int Hkv, int d, int topk)
+{
+    (void)Hq;
+    if (B <= 0 || Hkv <= 0 || !supported_d(d) || topk < 1) return 0;
+    return plan_decode(B, Hkv, d, topk).total;
+}
+
+qsa_status qsa_decode(const void *q, const void *K_cache, const void *V_cache, const int32_t *idx, void *o, int B,
+                      int Hq, int Hkv, int L, int T_kv_max, int d, int topk, float sm_scale, void *workspace,
+                      size_t workspace_bytes, qsa_stream_t stream)
+{
+    if (!q || !K_cache || !V_cache || !idx || !o) return fail(QSA_ERR_INVALID_ARG, "qsa_decode: null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || T_kv_max <= 0 || T_kv_max % 64 || L > T_kv_max || Hq % Hkv)
+        return fail(QSA_ERR_INVALID_ARG, "qsa_decode: bad shape");
+    if ((long)B * Hkv * T_kv_max >= (1L << 31)) return fail(QSA_ERR_UNSUPPORTED, "qsa_decode: cache too large");
+    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "qsa_decode: d=%d", d);
+    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "qsa_decode: topk=%d", topk);
+    const int G = Hq / Hkv;
+    if (G != 4 && G != 8) return fail(QSA_ERR_UNSUPPORTED, "qsa_decode: Hq/Hkv=%d", G);
+    if (!aligned16(q) || !aligned16(K_cache) || !aligned16(V_cache) || !aligned16(idx) || !aligned16(o))
+        return fail(QSA_ERR_INVALID_ARG, "qsa_decode: misaligned pointer");
+    const size_t need = plan_decode(B, Hkv, d, topk).total;
+    if (!workspace || workspace_bytes < need || !aligned16(workspace))
+        return fail(QSA_ERR_WORKSPACE, "qsa_decode: workspace needs %zu bytes", need);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 128 && G == 8) return launch_decode<128, 8>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, workspace, s);
+    if (d == 128 && G == 4) return launch_decode<128, 4>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, workspace, s);
+    if (d == 64 && G == 8) return launch_decode<64, 8>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, workspace, s);
+    return launch_decode<64, 4>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, workspace, s);
+}
+
+qsa_status qsa_get_device_status(qsa_stream_t stream, int *detail)
+{
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return check_launch("cudaStreamSynchronize");
+    int code = 0, det = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&code, qsa::g_status, sizeof(int)) != cudaSuccess ||
+        cudaMemcpyFromSymbol(&det, qsa::g_status_detail, sizeof(int)) != cudaSuccess ||
+        cudaMemcpyToSymbol(qsa::g_status, &zero, sizeof(int)) != cudaSuccess ||
+        cudaMemcpyToSymbol(qsa::g_status_detail, &zero, sizeof(int)) != cudaSuccess)
+        return check_launch("status word");
+    if (detail) *detail = det;
+    return (qsa_status)code;
+}
+
+qsa_status qsa_selftest_wait_timeout(uint64_t timeout_ns, qsa_stream_t stream)
+{
+    if (timeout_ns == 0 || timeout_ns > 1000000000ull)
+        return fail(QSA_ERR_INVALID_ARG, "qsa_selftest_wait_timeout: limit must be in (0, 1 s]");
+    selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(timeout_ns);
+    return launched("selftest_wait_kernel");
+}
+
+const char *qsa_status_string(qsa_status s)
+{
+    switch (s) {
+    case QSA_OK: return "QSA_OK";
+    case QSA_ERR_INVALID_ARG: return "QSA_ERR_INVALID_ARG";
+    case QSA_ERR_UNSUPPORTED: return "QSA_ERR_UNSUPPORTED";
+    case QSA_ERR_CUDA: return "QSA_ERR_CUDA";
+    case QSA_ERR_TIMEOUT: return "QSA_ERR_TIMEOUT";
+    case QSA_ERR_BOUNDS: return "QSA_ERR_BOUNDS";
+    case QSA_ERR_WORKSPACE: return "QSA_ERR_WORKSPACE";
+    }
+    return "QSA_ERR_UNKNOWN";
+}
+
+const char *qsa_last_error(void) { return g_last_error; }
+
+unsigned long long qsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

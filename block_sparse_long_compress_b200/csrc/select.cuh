@@ -1,0 +1,340 @@
+// Steps 2-4 -- pooled query, block scoring and top-k block selection
+// ("indexer scoring" -> "top-k selection", page "Qwen4 in llama.cpp:
+// Dissecting PR #27742", section "QSA Is an Address-Selection Problem, Not
+// a New Attention Equation"; the selection is discontinuous at the cutoff,
+// so the order is made total: score descending, then block index ascending).
+//
+// Kernels:
+//   pool_queries_kernel  one CTA per (row, b): fp32 mean of Q over the row's
+//                        tokens and each group's heads -> Qbar (workspace).
+//   score_select_kernel  one CTA per (candidate chunk, row, b*Hkv): fp32
+//                        scores of the chunk's block summaries into shared
+//                        memory as 64-bit keys, exact radix select of the
+//                        chunk's top-m, compaction in block order.  A row
+//                        with one chunk writes its final indices directly;
+//                        otherwise it writes its chunk's keys to the
+//                        workspace.
+//   merge_select_kernel  one CTA per row with several chunks: the same
+//                        select over the union of the chunks' top-m lists.
+// Key of candidate j with score s: (order-preserving bits of s) << 32 |
+// (0xFFFFFFFF - j); keys are unique, larger = better, and the lower block
+// wins a score tie.  -0.0 is folded into +0.0.
+#pragma once
+#include "device.cuh"
+
+namespace qsa {
+
+constexpr int kSelThreads = 256;
+constexpr int kMaxChosen = 62;   // topk <= 64 minus the two forced blocks
+
+// ------------------------------------------------------------------ pool
+// grid (NR, B); blockDim = Hq*d/8 rounded up to a warp (<= 1024).
+template <int D>
+__global__ void pool_queries_kernel(const __nv_bfloat16 *__restrict__ Q, float *__restrict__ Qbar,
+                                    int Tq, int Hq, int Hkv, int qblk)
+{
+    extern __shared__ float colsum[];   // [Hq * D]
+    const int i = blockIdx.x, b = blockIdx.y, NR = gridDim.x;
+    const int nchunks = Hq * D / 8;
+    const int t = threadIdx.x;
+    const int t0 = i * qblk;
+    const int t1 = min(t0 + qblk, Tq);
+    if (t < nchunks) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(Q + ((long)b * Tq + t0) * Hq * D) + t;
+        const long stride = (long)Hq * D / 8;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; e++) acc[e] = 0.f;
+        int tok = t0;
+        for (; tok + 8 <= t1; tok += 8) {
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; u++) v[u] = __ldg(src + (long)(tok - t0 + u) * stride);
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&v[u]);
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    float2 f = __bfloat1622float2(p[e]);
+                    acc[2 * e] += f.x;
+                    acc[2 * e + 1] += f.y;
+                }
+            }
+        }
+        for (; tok < t1; tok++) {
+            uint4 v = __ldg(src + (long)(tok - t0) * stride);
+            const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                float2 f = __bfloat1622float2(p[e]);
+                acc[2 * e] += f.x;
+                acc[2 * e + 1] += f.y;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; e++) colsum[t * 8 + e] = acc[e];
+    }
+    __syncthreads();
+    const int G = Hq / Hkv;
+    const float inv = 1.0f / (float)((t1 - t0) * G);
+    for (int o = t; o < Hkv * D; o += blockDim.x) {
+        const int g = o / D, c = o % D;
+        float s = 0.f;
+        for (int h = g * G; h < (g + 1) * G; h++) s += colsum[h * D + c];
+        Qbar[(((long)b * Hkv + g) * NR + i) * D + c] = s * inv;
+    }
+}
+
+// ------------------------------------------------------- select helpers
+__device__ __forceinline__ uint64_t make_key(float s, int j)
+{
+    if (s == 0.f) s = 0.f;   // -0.0 -> +0.0
+    const uint32_t b = __float_as_uint(s);
+    const uint32_t k = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return ((uint64_t)k << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
+}
+
+__device__ __forceinline__ int key_block(uint64_t key) { return (int)(0xFFFFFFFFu - (uint32_t)key); }
+
+struct SelectShared {
+    int hist[256];
+    int warp_tot[kSelThreads / 32];
+    int digit, above, bucket;
+};
+
+// Radix select over n unique keys in shared memory: returns (prefix, mask)
+// such that exactly `need` keys satisfy (key & mask) >= prefix.
+// Requires 0 < need < n.  All threads of the CTA must call it.
+__device__ void radix_select(const uint64_t *keys, int n, int need, SelectShared &sh,
+                             uint64_t &prefix_out, uint64_t &mask_out)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint64_t prefix = 0, mask = 0;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+        for (int b = tid; b < 256; b += kSelThreads) sh.hist[b] = 0;
+        __syncthreads();
+        for (int e = tid; e < n; e += kSelThreads) {
+            const uint64_t k = keys[e];
+            if ((k & mask) == prefix) atomicAdd(&sh.hist[(int)((k >> shift) & 0xFF)], 1);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // lane l owns bins 255-8l .. 248-8l (descending)
+            int c[8], tot = 0;
+#pragma unroll
+            for (int q = 0; q < 8; q++) {
+                c[q] = sh.hist[255 - 8 * lane - q];
+                tot += c[q];
+            }
+            int incl = tot;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            const int excl = incl - tot;
+            if (excl < need && need <= incl) {
+                int cum = excl;
+#pragma unroll
+                for (int q = 0; q < 8; q++) {
+                    if (cum + c[q] >= need) {
+                        sh.digit = 255 - 8 * lane - q;
+                        sh.above = cum;
+                        sh.bucket = c[q];
+                        break;
+                    }
+                    cum += c[q];
+                }
+            }
+        }
+        __syncthreads();
+        need -= sh.above;
+        prefix |= (uint64_t)sh.digit << shift;
+        mask |= (uint64_t)0xFF << shift;
+        const bool done = (sh.bucket == need);
+        __syncthreads();   // everyone has read sh.* before the next pass
+        if (done) break;
+    }
+    prefix_out = prefix;
+    mask_out = mask;
+}
+
+// Exclusive CTA-wide prefix sum of one int per thread; also returns the total.
+__device__ __forceinline__ int block_exclusive_scan(int v, SelectShared &sh, int &total)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += u;
+    }
+    if (lane == 31) sh.warp_tot[warp] = incl;
+    __syncthreads();
+    int base = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kSelThreads / 32; w++) {
+        const int x = sh.warp_tot[w];
+        if (w < warp) base += x;
+        tot += x;
+    }
+    __syncthreads();
+    total = tot;
+    return base + incl - v;
+}
+
+// Select the top `need` of n keys (already in ascending block order) and
+// emit them in that order: to `final_row` as block ids between the forced
+// entries (0 first, then the chosen, then D), or to `part` as keys.
+__device__ void select_and_emit(const uint64_t *keys, int n, int need, SelectShared &sh,
+                                int32_t *final_row, int D, int topk, uint64_t *part)
+{
+    uint64_t prefix = 0, mask = 0;
+    bool all = need >= n;
+    if (need > 0 && !all) radix_select(keys, n, need, sh, prefix, mask);
+    const int per = (n + kSelThreads - 1) / kSelThreads;
+    const int e0 = threadIdx.x * per;
+    const int e1 = min(e0 + per, n);
+    int cnt = 0;
+    if (need > 0)
+        for (int e = e0; e < e1; e++) cnt += (all || (keys[e] & mask) >= prefix) ? 1 : 0;
+    int total;
+    int pos = block_exclusive_scan(cnt, sh, total);
+    if (need > 0) {
+        for (int e = e0; e < e1; e++) {
+            const uint64_t k = keys[e];
+            if (all || (k & mask) >= prefix) {
+                if (final_row) final_row[1 + pos] = key_block(k);
+                else part[pos] = k;
+                pos++;
+            }
+        }
+    }
+    if (final_row) {
+        const int chosen = need > 0 ? min(need, n) : 0;
+        for (int s = threadIdx.x; s < topk; s += kSelThreads) {
+            if (s == 0) final_row[0] = 0;
+            else if (s == chosen + 1 && D > 0) final_row[s] = D;
+            else if (s > chosen + (D > 0 ? 1 : 0)) final_row[s] = -1;
+        }
+    }
+}
+
+struct RowGeom {
+    int D, ncand, m, nchunks;
+};
+
+__device__ __forceinline__ RowGeom row_geom(int i, int Tq, int q_pos0, int qblk, int topk, int CH)
+{
+    RowGeom g;
+    const int t_last = min((i + 1) * qblk, Tq) - 1;
+    g.D = (q_pos0 + t_last) / 64;
+    g.ncand = max(g.D - 1, 0);
+    const int nforced = g.D > 0 ? 2 : 1;
+    g.m = min(topk - nforced, g.ncand);
+    g.nchunks = max(1, (g.ncand + CH - 1) / CH);
+    return g;
+}
+
+// --------------------------------------------------------- score+select
+// grid (maxchunks, NR, B*Hkv); dynamic smem CH * 8 bytes.
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) score_select_kernel(
+    const float *__restrict__ Qbar, const float *__restrict__ Kc, int32_t *__restrict__ idx,
+    uint64_t *__restrict__ part, int nblk_max, int Tq, int q_pos0, int qblk, int topk,
+    float sm_scale, int CH, int maxchunks)
+{
+    extern __shared__ uint64_t keys[];
+    __shared__ SelectShared sh;
+    const int chunk = blockIdx.x, i = blockIdx.y, bg = blockIdx.z, NR = gridDim.y;
+    const RowGeom g = row_geom(i, Tq, q_pos0, qblk, topk, CH);
+    if (chunk >= g.nchunks) return;
+    const int j0 = 1 + chunk * CH;
+    const int n = max(0, min(CH, g.ncand - chunk * CH));
+    const long row = (long)bg * NR + i;
+
+    // fp32 scores: each warp takes 8 candidates at a time; lane owns
+    // columns [lane*V, lane*V+V); a transposing butterfly leaves candidate
+    // (lane >> 2) of the group in lanes with (lane & 3) == 0.
+    constexpr int V = D / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float q[V];
+#pragma unroll
+    for (int v = 0; v < V; v++) q[v] = Qbar[row * D + lane * V + v];
+    const float *kc_base = Kc + ((long)bg * nblk_max + j0) * D + lane * V;
+    for (int base = warp * 8; base < n; base += 8 * (kSelThreads / 32)) {
+        float s[8];
+#pragma unroll
+        for (int c = 0; c < 8; c++) {
+            s[c] = 0.f;
+            if (base + c < n) {
+                const float *p = kc_base + (long)(base + c) * D;
+                if constexpr (V == 4) {
+                    const float4 k4 = __ldg(reinterpret_cast<const float4 *>(p));
+                    s[c] = q[0] * k4.x + q[1] * k4.y + q[2] * k4.z + q[3] * k4.w;
+                } else {
+                    const float2 k2 = __ldg(reinterpret_cast<const float2 *>(p));
+                    s[c] = q[0] * k2.x + q[1] * k2.y;
+                }
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; c++) {
+            const bool up = lane & 16;
+            const float send = up ? s[c] : s[c + 4];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+            s[c] = (up ? s[c + 4] : s[c]) + recv;
+        }
+#pragma unroll
+        for (int c = 0; c < 2; c++) {
+            const bool up = lane & 8;
+            const float send = up ? s[c] : s[c + 2];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
+            s[c] = (up ? s[c + 2] : s[c]) + recv;
+        }
+        {
+            const bool up = lane & 4;
+            const float send = up ? s[0] : s[1];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
+            s[0] = (up ? s[1] : s[0]) + recv;
+        }
+        s[0] += __shfl_xor_sync(0xffffffffu, s[0], 2);
+        s[0] += __shfl_xor_sync(0xffffffffu, s[0], 1);
+        const int e = base + (lane >> 2);
+        if ((lane & 3) == 0 && e < n) keys[e] = make_key(s[0] * sm_scale, j0 + e);
+    }
+    __syncthreads();
+
+    const int need = min(g.m, n);
+    if (g.nchunks == 1) {
+        select_and_emit(keys, n, need, sh, idx + row * topk, g.D, topk, nullptr);
+    } else {
+        select_and_emit(keys, n, need, sh, nullptr, g.D, topk,
+                        part + (row * maxchunks + chunk) * kMaxChosen);
+    }
+}
+
+// grid (NR, B*Hkv); dynamic smem maxchunks * kMaxChosen * 8 bytes.
+__global__ void __launch_bounds__(kSelThreads) merge_select_kernel(
+    const uint64_t *__restrict__ part, int32_t *__restrict__ idx, int Tq, int q_pos0, int qblk,
+    int topk, int CH, int maxchunks)
+{
+    extern __shared__ uint64_t keys[];
+    __shared__ SelectShared sh;
+    const int i = blockIdx.x, bg = blockIdx.y, NR = gridDim.x;
+    const RowGeom g = row_geom(i, Tq, q_pos0, qblk, topk, CH);
+    if (g.nchunks <= 1) return;
+    const long row = (long)bg * NR + i;
+    // concatenate the chunks' lists (each ascending, chunks ascending)
+    int n = 0;
+    for (int c = 0; c < g.nchunks; c++) {
+        const int nc = min(g.m, min(CH, g.ncand - c * CH));
+        const uint64_t *src = part + (row * maxchunks + c) * kMaxChosen;
+        for (int e = threadIdx.x; e < nc; e += kSelThreads) keys[n + e] = src[e];
+        n += nc;
+    }
+    __syncthreads();
+    select_and_emit(keys, n, g.m, sh, idx + row * topk, g.D, topk, nullptr);
+}
+
+}  // namespace qsa

@@ -1,0 +1,174 @@
+/*
+ * qsa.h -- C ABI of libqsa.so, the B200 (sm_100a) hot path of Qwen Sparse
+ * Attention (QSA).
+ *
+ * The method (pages "Qwen4 architecture: QSA, GR, PLE", section "1. QSA: not
+ * looking at every token equally", and "Qwen4 in llama.cpp: Dissecting PR
+ * #27742", section "QSA Is an Address-Selection Problem, Not a New Attention
+ * Equation"): keys are compressed into per-block summaries, the summaries are
+ * scored against the queries, the top-k most relevant contiguous token blocks
+ * are selected, and exact softmax attention runs over the selected blocks
+ * only.  The selector returns block addresses, not values.
+ *
+ * Parameterization (the pages give none): key blocks of QSA_BLOCK = 64
+ * tokens, mean-pooled summaries; one selection per (query block of 64
+ * tokens -- or one token in decode --, KV group), shared by all query heads of
+ * the group; block 0 (sink) and the causal diagonal block are always kept
+ * and count toward top-k; ties go to the lower block index.
+ *
+ * Layouts (all dense, row-major, no padding):
+ *   Q, O    [B][Tq][Hq][d]        bf16  (query head h is in group h / (Hq/Hkv))
+ *   K, V    [B][Hkv][T_kv_max][d] bf16  (cache; a 64-token block of one head
+ *                                        is one contiguous 64*d run)
+ *   Kc      [B][Hkv][T_kv_max/64][d] fp32 (block summaries)
+ *   idx     [B][Hkv][NR][topk]     int32 (NR = ceil(Tq/qblk); ascending block
+ *                                        ids, -1 padding at the end)
+ *   lse     [B][Tq][Hq]            fp32  (natural-log softmax normaliser)
+ * The Tq query tokens sit at absolute positions q_pos0 .. q_pos0+Tq-1 of the
+ * cache; their own keys/values must already be written there.
+ *
+ * Supported: d in {64, 128}; Hq/Hkv in {4, 8}; 2 <= topk <= 64 (decode and
+ * score/select: topk <= 64; prefill attention: topk <= 64); every pointer
+ * 16-byte aligned; T_kv_max a multiple of 64.  Anything else returns
+ * QSA_ERR_UNSUPPORTED (or QSA_ERR_INVALID_ARG for malformed arguments).
+ *
+ * Ownership and errors: the caller owns every buffer, including the
+ * workspace; the library allocates no device memory.  All calls are
+ * asynchronous on `stream` (0 = legacy default stream).  Argument checks run
+ * on the host before any launch and return an error without launching.
+ * A failed launch returns QSA_ERR_CUDA (text in qsa_last_error()).  Errors
+ * found by a kernel (a bounded wait that timed out, an index outside the
+ * cache) are recorded in a device status word read by
+ * qsa_get_device_status().
+ */
+#ifndef QSA_H
+#define QSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QSA_BLOCK 64
+
+#if defined(__GNUC__)
+#define QSA_API __attribute__((visibility("default")))
+#else
+#define QSA_API
+#endif
+
+/* ABI-compatible with cudaStream_t / CUstream. */
+typedef struct CUstream_st *qsa_stream_t;
+
+typedef enum {
+    QSA_OK = 0,
+    QSA_ERR_INVALID_ARG = 1, /* null pointer, bad shape or position        */
+    QSA_ERR_UNSUPPORTED = 2, /* valid but outside the supported set above  */
+    QSA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed          */
+    QSA_ERR_TIMEOUT = 4,     /* a kernel's bounded wait ran out            */
+    QSA_ERR_BOUNDS = 5,      /* a kernel met a block index outside its range */
+    QSA_ERR_WORKSPACE = 6    /* workspace pointer null or too small        */
+} qsa_status;
+
+/*
+ * Step 1: compress keys.  Writes the fp32 mean of the 64 keys of every
+ * block j in [blk_begin, blk_end) of every (b, KV head):
+ *     Kc[b][h][j][:] = (1/64) * sum_{r<64} K[b][h][64 j + r][:]
+ * ("compress into small blocks" / "compressed-block representation").
+ * The reduction order is fixed, so summaries are bit-reproducible: a
+ * summary written incrementally (one block as it completes) equals the one
+ * written in a whole-cache pass.  Blocks outside the range are untouched.
+ * Requires 0 <= blk_begin <= blk_end <= T_kv_max/64.
+ */
+QSA_API qsa_status qsa_compress_keys(const void *K, float *Kc, int B, int Hkv, int T_kv_max,
+                             int d, int blk_begin, int blk_end, qsa_stream_t stream);
+
+/*
+ * Steps 2-4: pool queries, score the block summaries and select the top-k
+ * blocks ("indexer scoring" -> "top-k selection").
+ *
+ * Selection rows: qblk = 64 (prefill; q_pos0 must be a multiple of 64) or
+ * qblk = 1 (one selection per query token, e.g. decode with Tq = 1).  Row i
+ * covers query tokens [i*qblk, min((i+1)*qblk, Tq)); its diagonal block is
+ * D = (q_pos0 + last token of the row) / 64.  Its pooled query is the fp32
+ * mean of Q over those tokens and the group's heads, and each candidate
+ * block j in [1, D-1] scores s_j = sm_scale * <pooled query, Kc[b][g][j]>
+ * in fp32.  The row keeps {0, D} plus the min(topk-2, D-1) best candidates
+ * by (s descending, j ascending) -- only {0} when D = 0 -- written ascending
+ * into idx[b][g][i][:] and padded with -1.  Summaries of blocks 1 .. D-1
+ * must be present in Kc.  Scores are assumed finite.
+ *
+ * Workspace: qsa_score_select_workspace() bytes, caller-owned, no
+ * initialisation needed, must not be shared by concurrent calls.
+ */
+QSA_API size_t qsa_score_select_workspace(int B, int Hq, int Hkv, int Tq, int q_pos0, int qblk,
+                                  int d, int topk);
+QSA_API qsa_status qsa_score_select(const void *Q, const float *Kc, int32_t *idx, int B, int Hq,
+                            int Hkv, int Tq, int q_pos0, int qblk, int T_kv_max, int d,
+                            int topk, float sm_scale, void *workspace,
+                            size_t workspace_bytes, qsa_stream_t stream);
+
+/*
+ * Step 5 (prefill): exact softmax attention over the selected blocks
+ * ("attention over those cells").  Query token t (position p = q_pos0 + t,
+ * selection row t/64) of head h sees the keys u <= p of the blocks listed in
+ * idx[b][h/(Hq/Hkv)][t/64][:]:
+ *     O[b][t][h][:] = sum_u softmax_u(sm_scale * <q, k_u>) v_u
+ * computed flash-style (online softmax, fp32 accumulation in tensor memory,
+ * bf16 tensor-core MMA).  Requires q_pos0 % 64 == 0 and q_pos0 + Tq <=
+ * T_kv_max; every listed block must satisfy 0 <= j <= D of its row (a
+ * violation sets QSA_ERR_BOUNDS in the device status and the row's blocks
+ * past the violation are skipped).  lse may be NULL.  No workspace.
+ */
+QSA_API qsa_status qsa_sparse_attn_prefill(const void *Q, const void *K, const void *V,
+                                   const int32_t *idx, void *O, float *lse, int B, int Hq,
+                                   int Hkv, int Tq, int q_pos0, int T_kv_max, int d,
+                                   int topk, float sm_scale, qsa_stream_t stream);
+
+/*
+ * Step 5 (decode): one query token per sequence at position L-1 of its
+ * cache (cache length L includes the token itself), attending to the
+ * blocks listed in idx[b][g][0][:] (as produced by qsa_score_select with
+ * Tq = 1, qblk = 1, q_pos0 = L-1).  q and o are [B][Hq][d] bf16.  Split-K
+ * over the selected blocks; partial results are merged on the device by the
+ * last CTA of each (b, g).
+ * Workspace: qsa_decode_workspace() bytes, caller-owned, no initialisation
+ * needed, must not be shared by concurrent calls.
+ */
+QSA_API size_t qsa_decode_workspace(int B, int Hq, int Hkv, int d, int topk);
+QSA_API qsa_status qsa_decode(const void *q, const void *K_cache, const void *V_cache,
+                      const int32_t *idx, void *o, int B, int Hq, int Hkv, int L,
+                      int T_kv_max, int d, int topk, float sm_scale, void *workspace,
+                      size_t workspace_bytes, qsa_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word
+ * (QSA_OK if no kernel recorded an error since the last call).  If detail
+ * is not NULL it receives a kernel-specific code (0 if none).
+ */
+QSA_API qsa_status qsa_get_device_status(qsa_stream_t stream, int *detail);
+
+/* Test hook for the bounded waits: launches one CTA that waits on an
+ * mbarrier nothing will ever complete, with the given limit in
+ * nanoseconds, and records QSA_ERR_TIMEOUT in the device status word.
+ * The kernel returns normally; the context stays usable. */
+QSA_API qsa_status qsa_selftest_wait_timeout(uint64_t timeout_ns, qsa_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+QSA_API const char *qsa_status_string(qsa_status s);
+
+/* Number of kernels this library has launched in this process (all
+ * threads, all devices); for accounting in benchmarks. */
+QSA_API unsigned long long qsa_launch_count(void);
+
+/* Text of the last QSA_ERR_* returned on this host thread (static per
+ * thread; empty string if none). */
+QSA_API const char *qsa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_H */

@@ -1,0 +1,93 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds and
+loads, exports every entry point include/qsa.h declares, and rejects bad
+arguments before launching anything."""
+import ctypes
+import re
+import subprocess
+
+import pytest
+
+import block_sparse_long_compress_b200 as qsa
+
+
+def test_exports_every_declared_symbol():
+    declared = qsa.declared_symbols()
+    assert len(declared) >= 10
+    out = subprocess.run(["nm", "-D", "--defined-only", qsa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (qsa_\w+)", out))
+    assert set(declared) <= exported, set(declared) - exported
+    for name in declared:
+        assert hasattr(qsa.lib(), name)
+
+
+def test_status_strings_and_last_error():
+    lib = qsa.lib()
+    for code, name in qsa.STATUS.items():
+        assert lib.qsa_status_string(code).decode() == name
+    assert lib.qsa_status_string(99).decode() == "QSA_ERR_UNKNOWN"
+
+
+def test_workspace_sizes_are_host_only():
+    # chunked selection (one 1M-token row per group) needs partial-key space
+    big = qsa.score_select_workspace(1, 16, 2, 4096, 1048576, 64, 128, 64)
+    small = qsa.score_select_workspace(1, 16, 2, 4096, 0, 64, 128, 64)
+    assert big > small > 0
+    assert qsa.score_select_workspace(1, 16, 2, 4096, 0, 7, 128, 64) == 0   # bad qblk
+    assert qsa.decode_workspace(32, 16, 2, 128, 64) > 0
+    assert qsa.decode_workspace(32, 16, 2, 96, 64) == 0                     # bad d
+
+
+def test_argument_checks_return_before_launch():
+    lib = qsa.lib()
+    P = ctypes.c_void_p
+    fake = P(0x1000)       # never dereferenced: checks fail first
+    odd = P(0x1008)
+    # null pointer
+    assert lib.qsa_compress_keys(None, fake, 1, 2, 128, 128, 0, 2, None) == 1
+    assert b"null" in lib.qsa_last_error()
+    # block range outside the cache
+    assert lib.qsa_compress_keys(fake, fake, 1, 2, 128, 128, 0, 3, None) == 1
+    # unsupported head dim
+    assert lib.qsa_compress_keys(fake, fake, 1, 2, 128, 96, 0, 2, None) == 2
+    # misaligned
+    assert lib.qsa_compress_keys(odd, fake, 1, 2, 128, 128, 0, 2, None) == 1
+    # score/select: q_pos0 not block aligned in prefill mode, topk too large, no workspace
+    args = lambda **k: dict(dict(Q=fake, Kc=fake, idx=fake, B=1, Hq=16, Hkv=2, Tq=128, q_pos0=0,
+                                 qblk=64, T=1024, d=128, topk=16, ws=fake, wsb=1 << 30), **k)
+
+    def ss(a):
+        return lib.qsa_score_select(a["Q"], a["Kc"], a["idx"], a["B"], a["Hq"], a["Hkv"], a["Tq"],
+                                    a["q_pos0"], a["qblk"], a["T"], a["d"], a["topk"], 0.088,
+                                    a["ws"], a["wsb"], None)
+    assert ss(args(q_pos0=32)) == 1
+    assert ss(args(topk=65)) == 2
+    assert ss(args(topk=1)) == 2
+    assert ss(args(qblk=16)) == 2
+    assert ss(args(Tq=2000)) == 1          # queries past the cache
+    assert ss(args(ws=None)) == 6
+    assert ss(args(wsb=16)) == 6
+    # prefill: unsupported group size, bad position
+    pf = lambda Hq=16, q_pos0=0, d=128: lib.qsa_sparse_attn_prefill(
+        fake, fake, fake, fake, fake, None, 1, Hq, 2, 128, q_pos0, 1024, d, 16, 0.088, None)
+    assert pf(Hq=12) == 2
+    assert pf(q_pos0=64 * 3 + 1) == 1
+    assert pf(d=256) == 2
+    # decode: L beyond the cache, small workspace
+    dc = lambda L=1000, wsb=1 << 30: lib.qsa_decode(fake, fake, fake, fake, fake, 4, 16, 2, L,
+                                                    1024, 128, 8, 0.088, fake, wsb, None)
+    assert dc(L=2000) == 1
+    assert dc(wsb=8) == 6
+    # self-test limit out of range
+    assert lib.qsa_selftest_wait_timeout(0, None) == 1
+
+
+def test_product_path_has_no_oracle_dependency():
+    """The package must not import or reach the oracle."""
+    import os
+    pkg = os.path.dirname(qsa.__file__)
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(root, f)).read()
+                assert "oracle" not in text.lower(), f
