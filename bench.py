@@ -115,6 +115,22 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def job_throughput(ms_local, units_local, device):
+    """Whole-job throughput over all ranks: sum of the ranks' units divided
+    by the slowest rank's step time.  Returns (units/s, max ms)."""
+    t = torch.tensor([ms_local, float(units_local)], dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        ws = torch.distributed.get_world_size()
+        mx = t[:1].clone()
+        torch.distributed.all_reduce(mx, op=torch.distributed.ReduceOp.MAX)
+        tot = t[1:].clone()
+        torch.distributed.all_reduce(tot, op=torch.distributed.ReduceOp.SUM)
+        ms_max, units = float(mx.item()), float(tot.item())
+    else:
+        ms_max, units = ms_local, float(units_local)
+    return units / (ms_max * 1e-3), ms_max
+
+
 def prefill_flops(w):
     """Algorithmic FLOPs of the sparse attention: 4*d*Hq per unmasked
     (query, key) pair inside the selected blocks (masked half of the
@@ -195,12 +211,7 @@ def run_qsa(args, ws, rank, local):
     t_att = np.array([e[2].elapsed_time(e[3]) for e in evs])
     t_step = np.array([e[0].elapsed_time(e[3]) for e in evs])
     ms = float(t_step.sum() / args.steps)
-    ms_all = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if ws > 1:
-        torch.distributed.all_reduce(ms_all, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(ms_all.item())
-    tokens = wp.B * wp.Tq
-    value = tokens * ws / (ms_max * 1e-3)
+    value, ms_max = job_throughput(ms, wp.B * wp.Tq, dev)
 
     flops = prefill_flops(wp)
     att_s = float(t_att.mean()) * 1e-3
@@ -240,6 +251,8 @@ def run_qsa(args, ws, rank, local):
 
 def bench_decode(args, qsa, dev, peaks, ws, rank, flush):
     wd = synthetic.CONFIGS[args.decode_workload]
+    if args.decode_batch:
+        wd = synthetic.Workload(**{**wd.__dict__, "B": args.decode_batch})
     if ws > 1:
         wd = synthetic.Workload(**{**wd.__dict__, "seed": wd.seed + 1000 * rank})
     x = synthetic.generate(wd, dev)
@@ -321,14 +334,10 @@ def bench_e2e(args, qsa, dev, wp, ws):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if ws > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms = float(t.item())
+    value, ms = job_throughput(e0.elapsed_time(e1) / args.steps, wp.B * wp.Tq, dev)
     h2d = sum(a.numel() * a.element_size() for a in (hQ, hK, hV))
     d2h = hO.numel() * hO.element_size()
-    return {"value": wp.B * wp.Tq * ws / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+    return {"value": value, "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
@@ -406,6 +415,10 @@ def main():
     ap.add_argument("--workload", default=PREFILL, choices=sorted(synthetic.CONFIGS))
     ap.add_argument("--decode-workload", default=DECODE, choices=sorted(synthetic.CONFIGS))
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--only-decode", action="store_true",
+                    help="skip the prefill measurement (profiling the decode kernels)")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="override the decode batch (smaller profiling captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
@@ -428,6 +441,15 @@ def main():
             print(json.dumps(res), flush=True)
         return
 
+    if args.only_decode:
+        import block_sparse_long_compress_b200 as qsa
+        dev = torch.device("cuda", local)
+        torch.cuda.set_device(dev)
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        res = bench_decode(args, qsa, dev, load_peaks(), ws, rank, flush)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return
     res = run_qsa(args, ws, rank, local)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         wp = synthetic.CONFIGS[args.workload]
