@@ -47,6 +47,7 @@ def _load():
         "qsa_compress_keys": (I, [P, P, I, I, I, I, I, I, P]),
         "qsa_score_select_workspace": (S, [I, I, I, I, I, I, I, I]),
         "qsa_score_select": (I, [P, P, P, I, I, I, I, I, I, I, I, I, F, P, S, P]),
+        "qsa_score_select_noalloc": (I, [P, P, P, I, I, I, I, I, I, I, I, I, F, P]),
         "qsa_sparse_attn_prefill": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P]),
         "qsa_decode_workspace": (S, [I, I, I, I, I]),
         "qsa_decode": (I, [P, P, P, P, P, I, I, I, I, I, I, I, F, P, S, P]),

@@ -219,6 +219,38 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns)
 
 }  // namespace
 
+// ------------------------------------------- allocation-free selection
+// Scratch of qsa_score_select_noalloc: a file-scope device array that every
+// GPU loading the library holds until the process exits.  Host code only
+// sees a host-side stand-in for it, so the device address is looked up once
+// per device (with that device current) and cached.
+static __device__ __align__(256) uint8_t g_select_scratch[QSA_SELECT_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 128;
+
+qsa_status select_scratch_address(void **out)
+{
+    static std::mutex mu;
+    static void *addr[kMaxDevices] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return check_launch("cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(QSA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_select_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(QSA_ERR_CUDA, "cudaGetSymbolAddress(select scratch): %s", cudaGetErrorString(e));
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return QSA_OK;
+}
+
+}  // namespace
+
 // ===================================================================== C ABI
 extern "C" {
 
@@ -315,6 +347,23 @@ qsa_status qsa_score_select(const void *Q, const float *Kc, int32_t *idx, int B,
         if ((st = launched("merge_select_kernel")) != QSA_OK) return st;
     }
     return QSA_OK;
+}
+
+qsa_status qsa_score_select_noalloc(const void *Q, const float *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
+                                    int q_pos0, int qblk, int T_kv_max, int d, int topk, float sm_scale,
+                                    qsa_stream_t stream)
+{
+    const size_t need = qsa_score_select_workspace(B, Hq, Hkv, Tq, q_pos0, qblk, d, topk);
+    if (need > QSA_SELECT_SCRATCH_BYTES)
+        return fail(QSA_ERR_WORKSPACE,
+                    "qsa_score_select_noalloc: this shape needs %zu bytes of scratch, the static buffer holds %zu; "
+                    "use qsa_score_select with a caller workspace",
+                    need, (size_t)QSA_SELECT_SCRATCH_BYTES);
+    void *scratch = nullptr;
+    qsa_status st = select_scratch_address(&scratch);
+    if (st != QSA_OK) return st;
+    return qsa_score_select(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, qblk, T_kv_max, d, topk, sm_scale, scratch,
+                            QSA_SELECT_SCRATCH_BYTES, stream);
 }
 
 qsa_status qsa_sparse_attn_prefill(const void *Q, const void *K, const void *V, const int32_t *idx, void *O,

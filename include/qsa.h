@@ -111,6 +111,31 @@ QSA_API qsa_status qsa_score_select(const void *Q, const float *Kc, int32_t *idx
                             size_t workspace_bytes, qsa_stream_t stream);
 
 /*
+ * Allocation-free variant of qsa_score_select.  The pages have no
+ * counterpart: it exists for callers that cannot allocate device memory
+ * themselves -- e.g. a plug-in or custom operator inside a host engine whose
+ * memory planner owns the whole device and forbids side allocations, or a
+ * runtime that has no handle on an allocator at the call site.  Same inputs,
+ * outputs and results as qsa_score_select, but the workspace is a
+ * static device array of QSA_SELECT_SCRATCH_BYTES inside the library, which
+ * every GPU that loads the library holds until the process exits.  Shapes
+ * whose workspace (qsa_score_select_workspace) exceeds that size return
+ * QSA_ERR_WORKSPACE without launching.  The function calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ * The first call on each device looks up the buffer's device address (with
+ * that device current) and caches it; make that first call before any
+ * stream capture.  Every call shares the one buffer and it keeps the last
+ * call's contents (nothing in it needs to start at zero), so calls that
+ * overlap on the GPU -- on different streams, or from different host
+ * threads on the same device -- race with each other: serialise them.
+ */
+#define QSA_SELECT_SCRATCH_BYTES ((size_t)4 << 20)
+QSA_API qsa_status qsa_score_select_noalloc(const void *Q, const float *Kc, int32_t *idx, int B,
+                                            int Hq, int Hkv, int Tq, int q_pos0, int qblk,
+                                            int T_kv_max, int d, int topk, float sm_scale,
+                                            qsa_stream_t stream);
+
+/*
  * Step 5 (prefill): exact softmax attention over the selected blocks
  * ("attention over those cells").  Query token t (position p = q_pos0 + t,
  * selection row t/64) of head h sees the keys u <= p of the blocks listed in
