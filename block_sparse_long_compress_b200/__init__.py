@@ -53,6 +53,7 @@ def _load():
         "qsa_decode": (I, [P, P, P, P, P, I, I, I, I, I, I, I, F, P, S, P]),
         "qsa_get_device_status": (I, [P, ctypes.POINTER(I)]),
         "qsa_selftest_wait_timeout": (I, [ctypes.c_uint64, P]),
+        "qsa_selftest_exp2": (I, [P, P, I, P]),
         "qsa_status_string": (ctypes.c_char_p, [I]),
         "qsa_last_error": (ctypes.c_char_p, []),
         "qsa_launch_count": (ctypes.c_ulonglong, []),
@@ -172,13 +173,13 @@ def decode(q, K, V, idx, o, L, sm_scale=None, workspace=None, stream=None):
     if sm_scale is None:
         sm_scale = d ** -0.5
     need = decode_workspace(B, Hq, Hkv, d, topk)
-    if workspace is None:
+    if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     _check(_lib.qsa_decode(
         _ptr(q, torch.bfloat16, "q"), _ptr(K, torch.bfloat16, "K"), _ptr(V, torch.bfloat16, "V"),
         _ptr(idx, torch.int32, "idx"), _ptr(o, torch.bfloat16, "o"), B, Hq, Hkv, L, T, d, topk,
-        float(sm_scale), _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
-        _stream(stream)), "qsa_decode")
+        float(sm_scale), _ptr(workspace, torch.uint8, "workspace"),
+        0 if workspace is None else workspace.numel(), _stream(stream)), "qsa_decode")
     return o
 
 
@@ -251,8 +252,8 @@ class QSADecode:
         self.Kc = torch.zeros((B, Hkv, T_kv_max // BLOCK, d), dtype=torch.float32, device=dev)
         self.idx = torch.empty((B, Hkv, 1, topk), dtype=torch.int32, device=dev)
         self.o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
-        self.ws_dec = torch.empty(decode_workspace(B, Hq, Hkv, d, topk), dtype=torch.uint8,
-                                  device=dev)
+        n = decode_workspace(B, Hq, Hkv, d, topk)
+        self.ws_dec = torch.empty(n, dtype=torch.uint8, device=dev) if n > 0 else None
         self._sel_ws = {}
 
     def compress(self, K, blk_begin, blk_end, stream=None):

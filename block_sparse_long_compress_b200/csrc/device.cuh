@@ -293,4 +293,70 @@ __device__ __forceinline__ float fast_exp2(float x)
     return y;
 }
 
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^x for a pair of fp32 values with x <= 8, on the FMA pipe instead of the
+// MUFU unit.  Cody-Waite style argument reduction: x = n + f with
+// n = round(x) (obtained by adding 1.5 * 2^23, which leaves n in the low
+// mantissa bits) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose
+// coefficients were fitted for this library (Chebyshev-node weighted least
+// squares towards minimax relative error; max relative error 7.5e-5 on
+// [-1/2, 1/2], far below the 2^-9 of the bf16 rounding that follows); 2^n
+// is applied by adding n to the exponent field.  x is clamped at -126 so
+// the exponent never underflows (2^-126 is negligible next to the row's
+// largest term, which is >= 1).
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2)
+{
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    const uint64_t x = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+    const uint64_t round_c = f2_pack(12582912.f, 12582912.f);
+    const uint64_t t = f2_add(x, round_c);
+    const uint64_t f = f2_sub(x, f2_sub(t, round_c));
+    uint64_t p = f2_fma(f2_pack(5.517164618e-02f, 5.517164618e-02f), f,
+                        f2_pack(2.426111251e-01f, 2.426111251e-01f));
+    p = f2_fma(p, f, f2_pack(6.932609677e-01f, 6.932609677e-01f));
+    p = f2_fma(p, f, f2_pack(9.999280572e-01f, 9.999280572e-01f));
+    float t0, t1, p0, p1;
+    f2_unpack(t, t0, t1);
+    f2_unpack(p, p0, p1);
+    return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                   __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
 }  // namespace qsa

@@ -209,13 +209,25 @@ __global__ void __launch_bounds__(192, 1) sparse_attn_prefill_kernel(
             tmem_ld32(lane_addr + C::S_COL + 64 * buf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
             tmem_wait_ld();
             float s[64];
-            const long limit = p - 64L * sh.blocks[n];   // keys c <= limit are visible
-            float mx = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 64; c++) {
-                s[c] = (c <= limit) ? __uint_as_float(sr[c]) * sm_scale_log2 : -INFINITY;
-                mx = fmaxf(mx, s[c]);
+            for (int c = 0; c < 64; c++) s[c] = __uint_as_float(sr[c]);
+            if (sh.blocks[n] == Dg) {
+                // only the diagonal block has keys after some rows' positions
+                const long limit = p - 64L * Dg;
+#pragma unroll
+                for (int c = 0; c < 64; c++)
+                    if (c > limit) s[c] = -INFINITY;
             }
+            float q0 = s[0], q1 = s[16], q2 = s[32], q3 = s[48];
+#pragma unroll
+            for (int c = 1; c < 15; c += 2) {
+                q0 = max3f(q0, s[c], s[c + 1]);
+                q1 = max3f(q1, s[16 + c], s[17 + c]);
+                q2 = max3f(q2, s[32 + c], s[33 + c]);
+                q3 = max3f(q3, s[48 + c], s[49 + c]);
+            }
+            const float mx = max3f(max3f(q0, q1, s[15]), max3f(q2, q3, s[31]), fmaxf(s[47], s[63])) *
+                             sm_scale_log2;
             if (n == 0) {
                 m_run = mx;
             } else if (__any_sync(0xffffffffu, mx > m_run + 8.0f)) {
@@ -237,15 +249,30 @@ __global__ void __launch_bounds__(192, 1) sparse_attn_prefill_kernel(
                 l *= alpha;
                 m_run = m_new;
             }
+            // P = 2^(s*c - m): 3 of every 8 pairs on the FMA pipe, the rest on MUFU
             uint32_t pk[32];
-            float lsum = 0.f;
+            const uint64_t sc2 = f2_pack(sm_scale_log2, sm_scale_log2);
+            const uint64_t nm2 = f2_pack(-m_run, -m_run);
+            uint64_t lacc = f2_pack(0.f, 0.f);
 #pragma unroll
             for (int c = 0; c < 32; c++) {
-                const float p0 = fast_exp2(s[2 * c] - m_run);
-                const float p1 = fast_exp2(s[2 * c + 1] - m_run);
-                lsum += p0 + p1;
+                const uint64_t x2 = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), sc2, nm2);
+                uint64_t p2;
+                if ((c & 7) == 1 || (c & 7) == 4 || (c & 7) == 6) {
+                    p2 = exp2_poly_x2(x2);
+                } else {
+                    float x0, x1;
+                    f2_unpack(x2, x0, x1);
+                    p2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
+                }
+                lacc = f2_add(lacc, p2);
+                float p0, p1;
+                f2_unpack(p2, p0, p1);
                 pk[c] = pack_bf16x2(p0, p1);
             }
+            float la, lb;
+            f2_unpack(lacc, la, lb);
+            const float lsum = la + lb;
             l += lsum;
             tmem_st32(lane_addr + C::S_COL + 64 * buf, pk);
             tmem_wait_st();

@@ -49,6 +49,8 @@ qsa_status launched(const char *what)
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+constexpr int kMaxDevicesSm = 128;
+
 // ---------------------------------------------------------- tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -130,23 +132,35 @@ SelectPlan plan_select(int B, int Hkv, int Tq, int q_pos0, int qblk, int d)
 }
 
 // ------------------------------------------------------- decode geometry
-constexpr int kDecodeWarps = 2;
+int sm_count()
+{
+    static int cache[kMaxDevicesSm] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= kMaxDevicesSm) return 148;
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
 
+// Splits of a (sequence, group) row: about one CTA per SM over all rows,
+// at most 8 (one portable cluster), at least one slot per CTA.
 struct DecodePlan {
-    int nsplit;
-    size_t m_off, l_off, o_off, t_off, total;
+    int P, spc;
 };
 
-DecodePlan plan_decode(int B, int Hkv, int d, int topk)
+DecodePlan plan_decode(int rows, int topk, int nsm)
 {
+    int P = (nsm + rows / 2) / rows;
+    P = P < 1 ? 1 : P;
+    P = P > 8 ? 8 : P;
+    P = P > topk ? topk : P;
     DecodePlan p;
-    p.nsplit = (topk + kDecodeWarps - 1) / kDecodeWarps;
-    const size_t rows = (size_t)B * Hkv * p.nsplit * 8;
-    p.m_off = 0;
-    p.l_off = align256(rows * 4);
-    p.o_off = p.l_off + align256(rows * 4);
-    p.t_off = p.o_off + align256(rows * d * 4);
-    p.total = p.t_off + align256((size_t)B * Hkv * 4);
+    p.spc = (topk + P - 1) / P;
+    p.P = (topk + p.spc - 1) / p.spc;
     return p;
 }
 
@@ -183,25 +197,47 @@ qsa_status launch_prefill(const void *Q, const void *K, const void *V, const int
 template <int D, int G>
 qsa_status launch_decode(const void *q, const void *K, const void *V, const int32_t *idx, void *o,
                          int B, int Hq, int Hkv, int L, int T_kv_max, int topk, float sm_scale,
-                         void *ws, cudaStream_t s)
+                         cudaStream_t s)
 {
     using C = qsa::DecodeCfg<D>;
     CUtensorMap mk, mv;
     qsa_status st;
     if ((st = make_map_2d(&mk, K, (uint64_t)B * Hkv * T_kv_max, D)) != QSA_OK) return st;
     if ((st = make_map_2d(&mv, V, (uint64_t)B * Hkv * T_kv_max, D)) != QSA_OK) return st;
-    const DecodePlan p = plan_decode(B, Hkv, D, topk);
-    uint8_t *w = static_cast<uint8_t *>(ws);
-    qsa::DecodePartial part{reinterpret_cast<float *>(w + p.m_off), reinterpret_cast<float *>(w + p.l_off),
-                            reinterpret_cast<float *>(w + p.o_off), reinterpret_cast<int *>(w + p.t_off)};
-    if (cudaMemsetAsync(part.ticket, 0, (size_t)B * Hkv * 4, s) != cudaSuccess) return check_launch("memset");
-    auto kern = qsa::decode_kernel<D, G, kDecodeWarps>;
-    const int smem = kDecodeWarps * C::WARP_BYTES + 1024;
-    if ((st = set_smem(kern, smem)) != QSA_OK) return st;
-    dim3 grid(p.nsplit, B * Hkv);
-    kern<<<grid, kDecodeWarps * 32, smem, s>>>(mk, mv, (const __nv_bfloat16 *)q, idx, (__nv_bfloat16 *)o, part,
-                                              Hq, Hkv, L, T_kv_max, topk, sm_scale * 1.4426950408889634f);
+    const DecodePlan p = plan_decode(B * Hkv, topk, sm_count());
+    auto kern = qsa::decode_kernel<D, G>;
+    if ((st = set_smem(kern, C::SMEM_BYTES)) != QSA_OK) return st;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.P, B * Hkv, 1);
+    cfg.blockDim = dim3(C::NW * 32, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.P;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mk, mv, (const __nv_bfloat16 *)q, idx, (__nv_bfloat16 *)o, Hq,
+                                       Hkv, L, T_kv_max, topk, p.spc, sm_scale * 1.4426950408889634f);
+    if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "decode_kernel launch: %s", cudaGetErrorString(e));
     return launched("decode_kernel");
+}
+
+__global__ void selftest_exp2_kernel(const float *__restrict__ x, float *__restrict__ y, int n)
+{
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i + 1 < n) {
+        float a, b;
+        qsa::f2_unpack(qsa::exp2_poly_x2(qsa::f2_pack(x[i], x[i + 1])), a, b);
+        y[i] = a;
+        y[i + 1] = b;
+    } else if (i < n) {
+        float a, b;
+        qsa::f2_unpack(qsa::exp2_poly_x2(qsa::f2_pack(x[i], 0.f)), a, b);
+        y[i] = a;
+    }
 }
 
 __global__ void selftest_wait_kernel(uint64_t limit_ns)
@@ -393,9 +429,12 @@ qsa_status qsa_sparse_attn_prefill(const void *Q, const void *K, const void *V, 
 
 size_t qsa_decode_workspace(int B, int Hq, int Hkv, int d, int topk)
 {
+    (void)B;
     (void)Hq;
-    if (B <= 0 || Hkv <= 0 || !supported_d(d) || topk < 1) return 0;
-    return plan_decode(B, Hkv, d, topk).total;
+    (void)Hkv;
+    (void)d;
+    (void)topk;
+    return 0;   // the split-K merge runs through distributed shared memory
 }
 
 qsa_status qsa_decode(const void *q, const void *K_cache, const void *V_cache, const int32_t *idx, void *o, int B,
@@ -412,14 +451,14 @@ qsa_status qsa_decode(const void *q, const void *K_cache, const void *V_cache, c
     if (G != 4 && G != 8) return fail(QSA_ERR_UNSUPPORTED, "qsa_decode: Hq/Hkv=%d", G);
     if (!aligned16(q) || !aligned16(K_cache) || !aligned16(V_cache) || !aligned16(idx) || !aligned16(o))
         return fail(QSA_ERR_INVALID_ARG, "qsa_decode: misaligned pointer");
-    const size_t need = plan_decode(B, Hkv, d, topk).total;
-    if (!workspace || workspace_bytes < need || !aligned16(workspace))
-        return fail(QSA_ERR_WORKSPACE, "qsa_decode: workspace needs %zu bytes", need);
+    (void)workspace;
+    (void)workspace_bytes;
+    if (B * Hkv > 65535) return fail(QSA_ERR_UNSUPPORTED, "qsa_decode: more than 65535 (sequence, group) rows");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (d == 128 && G == 8) return launch_decode<128, 8>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, workspace, s);
-    if (d == 128 && G == 4) return launch_decode<128, 4>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, workspace, s);
-    if (d == 64 && G == 8) return launch_decode<64, 8>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, workspace, s);
-    return launch_decode<64, 4>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, workspace, s);
+    if (d == 128 && G == 8) return launch_decode<128, 8>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, s);
+    if (d == 128 && G == 4) return launch_decode<128, 4>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, s);
+    if (d == 64 && G == 8) return launch_decode<64, 8>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, s);
+    return launch_decode<64, 4>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, s);
 }
 
 qsa_status qsa_get_device_status(qsa_stream_t stream, int *detail)
@@ -442,6 +481,15 @@ qsa_status qsa_selftest_wait_timeout(uint64_t timeout_ns, qsa_stream_t stream)
         return fail(QSA_ERR_INVALID_ARG, "qsa_selftest_wait_timeout: limit must be in (0, 1 s]");
     selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(timeout_ns);
     return launched("selftest_wait_kernel");
+}
+
+qsa_status qsa_selftest_exp2(const float *x, float *y, int n, qsa_stream_t stream)
+{
+    if (!x || !y || n < 0) return fail(QSA_ERR_INVALID_ARG, "qsa_selftest_exp2: bad arguments");
+    if (n == 0) return QSA_OK;
+    const int pairs = (n + 1) / 2;
+    selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+    return launched("selftest_exp2_kernel");
 }
 
 const char *qsa_status_string(qsa_status s)

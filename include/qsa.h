@@ -157,10 +157,10 @@ QSA_API qsa_status qsa_sparse_attn_prefill(const void *Q, const void *K, const v
  * cache (cache length L includes the token itself), attending to the
  * blocks listed in idx[b][g][0][:] (as produced by qsa_score_select with
  * Tq = 1, qblk = 1, q_pos0 = L-1).  q and o are [B][Hq][d] bf16.  Split-K
- * over the selected blocks; partial results are merged on the device by the
- * last CTA of each (b, g).
- * Workspace: qsa_decode_workspace() bytes, caller-owned, no initialisation
- * needed, must not be shared by concurrent calls.
+ * over the selected blocks: up to 8 CTAs per (b, g) form a thread-block
+ * cluster and merge their partial softmax states through distributed
+ * shared memory.  Needs no workspace: qsa_decode_workspace() returns 0 and
+ * `workspace` may be NULL.  B*Hkv <= 65535.
  */
 QSA_API size_t qsa_decode_workspace(int B, int Hq, int Hkv, int d, int topk);
 QSA_API qsa_status qsa_decode(const void *q, const void *K_cache, const void *V_cache,
@@ -180,6 +180,12 @@ QSA_API qsa_status qsa_get_device_status(qsa_stream_t stream, int *detail);
  * nanoseconds, and records QSA_ERR_TIMEOUT in the device status word.
  * The kernel returns normally; the context stays usable. */
 QSA_API qsa_status qsa_selftest_wait_timeout(uint64_t timeout_ns, qsa_stream_t stream);
+
+/* Test hook for the FMA-pipe exponential used by the prefill softmax:
+ * y[i] = 2^x[i] for n device floats with x <= 8 (Cody-Waite reduction plus a
+ * degree-3 polynomial; inputs below -126 are clamped to -126).  Lets a test
+ * compare it with the CUDA exp2 on the same device. */
+QSA_API qsa_status qsa_selftest_exp2(const float *x, float *y, int n, qsa_stream_t stream);
 
 /* Human-readable name of a status code (static storage). */
 QSA_API const char *qsa_status_string(qsa_status s);

@@ -34,8 +34,8 @@ def test_workspace_sizes_are_host_only():
     small = qsa.score_select_workspace(1, 16, 2, 4096, 0, 64, 128, 64)
     assert big > small > 0
     assert qsa.score_select_workspace(1, 16, 2, 4096, 0, 7, 128, 64) == 0   # bad qblk
-    assert qsa.decode_workspace(32, 16, 2, 128, 64) > 0
-    assert qsa.decode_workspace(32, 16, 2, 96, 64) == 0                     # bad d
+    # decode merges its split-K partials in distributed shared memory: no workspace
+    assert qsa.decode_workspace(32, 16, 2, 128, 64) == 0
 
 
 def test_argument_checks_return_before_launch():
@@ -77,7 +77,8 @@ def test_argument_checks_return_before_launch():
     dc = lambda L=1000, wsb=1 << 30: lib.qsa_decode(fake, fake, fake, fake, fake, 4, 16, 2, L,
                                                     1024, 128, 8, 0.088, fake, wsb, None)
     assert dc(L=2000) == 1
-    assert dc(wsb=8) == 6
+    assert lib.qsa_decode(fake, fake, fake, fake, fake, 40000, 16, 2, 64, 64, 128, 8, 0.088,
+                          None, 0, None) == 2          # too many (sequence, group) rows
     # self-test limit out of range
     assert lib.qsa_selftest_wait_timeout(0, None) == 1
 

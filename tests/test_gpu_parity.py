@@ -99,6 +99,30 @@ def test_bounded_wait_reports_timeout(qsa):
     torch.ones(4, device=DEV).sum().item()
 
 
+def test_fma_pipe_exp2_against_cuda_exp2(qsa):
+    """The polynomial 2^x the prefill softmax runs on the FMA pipe, against
+    CUDA's exp2 on the same device: relative error <= 1e-4 on [-125, 8]
+    (the bf16 rounding of P that follows is 2^-9); tiny at and below -126,
+    where the result is subnormal."""
+    import ctypes
+    g = torch.Generator(device=DEV).manual_seed(5)
+    x = torch.cat([torch.rand(1 << 20, generator=g, device=DEV) * 133.0 - 125.0,
+                   torch.linspace(-1.0, 1.0, 4097, device=DEV),
+                   torch.tensor([0.0, 8.0, -0.5, 0.5, -125.0], device=DEV)])
+    y = torch.empty_like(x)
+    rc = qsa.lib().qsa_selftest_exp2(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()),
+                                     x.numel(), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref).abs() / ref).max().item()
+    assert rel <= 1e-4, rel
+    low = torch.tensor([-126.0, -127.0, -500.0, float("-inf")], device=DEV)
+    yl = torch.empty_like(low)
+    qsa.lib().qsa_selftest_exp2(ctypes.c_void_p(low.data_ptr()), ctypes.c_void_p(yl.data_ptr()), 4,
+                                ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert (yl >= 0).all() and (yl <= 2.0 ** -125).all()
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_compress_parity_and_reproducibility(qsa, d):
     w = synthetic.custom(B=2, Tq=64, T_kv=1280, Hq=8, Hkv=2, d=d, seed=21)
