@@ -4,25 +4,40 @@
 // section "QSA Is an Address-Selection Problem, Not a New Attention
 // Equation": ordinary attention over the visible cells).
 //
-// Work unit (one CTA): 128 MMA rows = TOK query tokens x G query heads of
-// one KV group (row r = token (r / G), head (r % G)), all sharing the same
-// selected key blocks.  Per selected block n:
-//     S = Q K_n^T          tcgen05.mma kind::f16, A = Q (smem, K-major),
-//                          B = K block (smem, K-major), D = S (TMEM, fp32)
-//     P = exp2(S*c - m)    softmax warps: tcgen05.ld S, online max/sum,
-//                          write P as bf16 back over S in TMEM
-//     O += P V_n           tcgen05.mma, A = P (TMEM), B = V block (smem,
-//                          MN-major), D = O (TMEM, fp32)
-// K/V blocks arrive by TMA (128-byte swizzle, 64 x 64 element boxes) into a
-// two-stage ring.  S is double-buffered in TMEM so that the softmax of block
-// n overlaps the QK^T of block n+1.  The running max is only moved (and O
-// rescaled in TMEM) when a block's max exceeds it by more than 2^8, so
-// rescales are rare.
+// Work unit (one CTA, one per SM): two 128-row MMA tiles of one KV group
+// and query block; row r of a tile = token (r / G), query head (r % G) --
+// 256 rows sharing the same selected key blocks, so every gathered K/V
+// block is loaded once for all 256 rows.  Selected blocks are consumed in
+// pairs (128 keys; an odd last pair repeats its first block and masks the
+// copy) through separate 2-deep K and V rings: a K stage is released once
+// both tiles' S are done, well before its V stage.  Per pair n and tile t:
+//     S_t = Q_t K_n^T       tcgen05.mma kind::f16, M=128 N=128 K=16 steps,
+//                           A = Q_t, B = the pair's keys (both K-major in
+//                           shared memory), D = S_t in TMEM (fp32)
+//     P_t = 2^(S_t c - m)   softmax warpgroup t, one thread per row holding
+//                           all 128 scores in registers; bf16 P_t is written
+//                           over the first 64 columns of S_t
+//     O_t += P_t V_n        tcgen05.mma, A = P_t from TMEM, B = the pair's
+//                           values (MN-major in shared memory), D = O_t
+// Each tile has its own MMA-issuing thread, so while one waits for its
+// softmax the other keeps the tensor pipe fed (an mbarrier query stalls the
+// issuing thread for a few hundred cycles, longer than the MMA queue
+// covers).  The two issuers hand the pipe back and forth through "S issued"
+// barriers so that its work strictly alternates between the tiles:
+//     S0(0) | S1(0) | PV0(0) S0(1) | PV1(0) S1(1) | PV0(1) S0(2) | ...
+// and each tile's softmax runs while the pipe works on the other tile (left
+// free, two identical chains drift into lockstep and their softmaxes then
+// compete for the same issue slots while the pipe idles).  Within a tile, S_t(n+1) is issued after PV_t(n) by the same
+// thread; the tensor pipe runs a thread's MMAs in order, so P_t(n) is read
+// before S_t(n+1) overwrites it.  The running max only moves (and O_t is
+// rescaled in TMEM) when a pair's max exceeds it by more than 2^8.
 //
-// Warp roles (192 threads): warps 0-3 softmax + epilogue (thread = row =
-// TMEM lane), warp 4 TMA producer, warp 5 TMEM allocator + MMA issuer.
-// TMEM columns: O [0, D), S/P buffer b at [128 + 64 b, 192 + 64 b).
-// Every mbarrier wait is bounded (QSA_ERR_TIMEOUT + early exit).
+// Warps (352 threads): 0-7 softmax/epilogue (tile = warp/4, TMEM lane
+// quarter = warp%4, thread = row), 8 TMA producer, 9 TMEM allocator + MMA
+// issuer of tile 0, 10 MMA issuer of tile 1.  Each softmax warp signals P
+// with a single arrive.
+// TMEM (512 columns): O_0 [0,128) O_1 [128,256) S_0 [256,384) S_1 [384,512);
+// P_t in S_t columns [0,64).  Every mbarrier wait is bounded.
 #pragma once
 #include "device.cuh"
 
@@ -30,28 +45,29 @@ namespace qsa {
 
 template <int D, int G>
 struct PrefillCfg {
-    static constexpr int M = 128;
-    static constexpr int TOK = M / G;
-    static constexpr int TILES = 64 / TOK;          // CTAs per 64-token query block
-    static constexpr int NH = D / 64;               // 128-byte column halves
-    static constexpr int Q_BYTES = M * D * 2;
-    static constexpr int HALF_BYTES = 64 * 128;     // one 64x64 bf16 TMA box
-    static constexpr int KV_BYTES = 64 * D * 2;     // one K (or V) block
-    static constexpr int NS = 2;                    // K/V stages
-    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
-    static constexpr int SMEM_DATA = Q_BYTES + NS * STAGE_BYTES;
-    static constexpr int THREADS = 192;
-    static constexpr int TMEM_COLS = 256;
-    static constexpr int S_COL = 128;
-    // keep at most two CTAs per SM so their TMEM (2 x 256 columns) fits
-    static constexpr int SMEM_REQUEST = (SMEM_DATA + 1024 > 80 * 1024) ? SMEM_DATA + 1024 : 80 * 1024;
+    static constexpr int M = 128;                  // rows per tile
+    static constexpr int TOK = M / G;              // tokens per tile
+    static constexpr int TILES = 64 / (2 * TOK);   // CTAs per 64-token query block
+    static constexpr int NH = D / 64;              // 128-byte column halves
+    static constexpr int HALF_ROWS_BYTES = 128 * 128;   // 128 rows x 128 B (one half of a tile)
+    static constexpr int QT_BYTES = NH * HALF_ROWS_BYTES;   // one Q tile
+    static constexpr int PAIR_BYTES = NH * HALF_ROWS_BYTES; // K (or V) of a block pair
+    static constexpr int NS = 2;                   // K stages and V stages (pairs)
+    static constexpr int SMEM_DATA = 2 * QT_BYTES + 2 * NS * PAIR_BYTES;
+    // the CTA owns all 512 TMEM columns: ask for enough shared memory that
+    // a second CTA never lands on the same SM
+    static constexpr int SMEM_REQUEST = (SMEM_DATA + 1024 > 120 * 1024) ? SMEM_DATA + 1024 : 120 * 1024;
+    static constexpr int THREADS = 11 * 32;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int O_COL = 0, S_COL = 256;
 };
 
 struct PrefillShared {
     uint64_t q_full;
-    uint64_t kv_full[2];
-    uint64_t kv_empty[2];
+    uint64_t k_full[2], k_empty[2];
+    uint64_t v_full[2], v_empty[2];
     uint64_t s_full[2];
+    uint64_t s_issued[2];
     uint64_t p_full[2];
     uint64_t pv_done[2];
     uint32_t tmem_base;
@@ -61,7 +77,7 @@ struct PrefillShared {
 };
 
 template <int D, int G>
-__global__ void __launch_bounds__(192, 1) sparse_attn_prefill_kernel(
+__global__ void __launch_bounds__(11 * 32, 1) sparse_attn_prefill_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ idx,
     __nv_bfloat16 *__restrict__ O, float *__restrict__ lse, int Tq, int Hq, int Hkv,
@@ -72,13 +88,14 @@ __global__ void __launch_bounds__(192, 1) sparse_attn_prefill_kernel(
     __shared__ PrefillShared sh;
 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *q_smem = smem;
-    uint8_t *kv_smem = smem + C::Q_BYTES;
+    uint8_t *q_smem = smem;                          // [tile][half][128 rows][128 B]
+    uint8_t *k_smem = smem + 2 * C::QT_BYTES;        // [stage][half][128 rows][128 B]
+    uint8_t *v_smem = k_smem + C::NS * C::PAIR_BYTES;
 
     const int NR = (Tq + 63) / 64;
     const int i = blockIdx.x / C::TILES, sub = blockIdx.x % C::TILES;
     const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv;
-    const int token0 = i * 64 + sub * C::TOK;
+    const int token0 = i * 64 + sub * 2 * C::TOK;
     if (token0 >= Tq) return;   // ragged tail: whole CTA idle (uniform exit)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row_last = min(i * 64 + 63, Tq - 1);
@@ -101,20 +118,25 @@ __global__ void __launch_bounds__(192, 1) sparse_attn_prefill_kernel(
         sh.nblk = n;
         sh.abort = 0;
         mbar_init(&sh.q_full, 1);
-        for (int s = 0; s < 2; s++) {
-            mbar_init(&sh.kv_full[s], 1);
-            mbar_init(&sh.kv_empty[s], 1);
-            mbar_init(&sh.s_full[s], 1);
-            mbar_init(&sh.p_full[s], 128);
-            mbar_init(&sh.pv_done[s], 1);
+        for (int s = 0; s < C::NS; s++) {
+            mbar_init(&sh.k_full[s], 1);
+            mbar_init(&sh.k_empty[s], 2);    // one arrive per tile
+            mbar_init(&sh.v_full[s], 1);
+            mbar_init(&sh.v_empty[s], 2);
+        }
+        for (int t = 0; t < 2; t++) {
+            mbar_init(&sh.s_full[t], 1);
+            mbar_init(&sh.s_issued[t], 1);
+            mbar_init(&sh.p_full[t], 4);     // one arrive per softmax warp
+            mbar_init(&sh.pv_done[t], 1);
         }
         fence_barrier_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(&sh.tmem_base, C::TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == 8 && lane == 0) {
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
@@ -124,162 +146,221 @@ __global__ void __launch_bounds__(192, 1) sparse_attn_prefill_kernel(
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
     const int nblk = sh.nblk;
+    const int npair = (nblk + 1) / 2;
     volatile int *abort = &sh.abort;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------ TMA producer
         if (lane == 0 && nblk > 0) {
-            mbar_arrive_expect_tx(&sh.q_full, C::Q_BYTES);
-            for (int h = 0; h < C::NH; h++)
-                tma_load_3d(q_smem + h * (C::M * 128), &tmQ, &sh.q_full, h * 64, g * G,
-                            b * Tq + token0);
-            const long kv_row0 = (long)bg * T_kv_max;
-            for (int n = 0; n < nblk; n++) {
+            mbar_arrive_expect_tx(&sh.q_full, 2 * C::QT_BYTES);
+            for (int t = 0; t < 2; t++)
+                for (int h = 0; h < C::NH; h++)
+                    tma_load_3d(q_smem + t * C::QT_BYTES + h * C::HALF_ROWS_BYTES, &tmQ, &sh.q_full, h * 64,
+                                g * G, b * Tq + token0 + t * C::TOK);
+            const int kv_row0 = bg * T_kv_max;   // host checks B*Hkv*T_kv_max < 2^31
+            for (int n = 0; n < npair; n++) {
                 const int st = n % C::NS;
-                if (n >= C::NS && !mbar_wait(&sh.kv_empty[st], ((n / C::NS) - 1) & 1, abort, 10))
-                    break;
-                uint8_t *ks = kv_smem + st * C::STAGE_BYTES;
-                uint8_t *vs = ks + C::KV_BYTES;
-                const int y = (int)(kv_row0 + 64L * sh.blocks[n]);
-                mbar_arrive_expect_tx(&sh.kv_full[st], C::STAGE_BYTES);
+                const int ya = kv_row0 + 64 * sh.blocks[2 * n];
+                // an odd last pair repeats its first block (its copy is masked)
+                const int yb = kv_row0 + 64 * sh.blocks[2 * n + 1 < nblk ? 2 * n + 1 : 2 * n];
+                if (n >= C::NS && !mbar_wait(&sh.k_empty[st], ((n / C::NS) - 1) & 1, abort, 10)) break;
+                uint8_t *ks = k_smem + st * C::PAIR_BYTES;
+                mbar_arrive_expect_tx(&sh.k_full[st], C::PAIR_BYTES);
                 for (int h = 0; h < C::NH; h++) {
-                    tma_load_2d(ks + h * C::HALF_BYTES, &tmK, &sh.kv_full[st], h * 64, y);
-                    tma_load_2d(vs + h * C::HALF_BYTES, &tmV, &sh.kv_full[st], h * 64, y);
+                    tma_load_2d(ks + h * C::HALF_ROWS_BYTES, &tmK, &sh.k_full[st], h * 64, ya);
+                    tma_load_2d(ks + h * C::HALF_ROWS_BYTES + 64 * 128, &tmK, &sh.k_full[st], h * 64, yb);
+                }
+                if (n >= C::NS && !mbar_wait(&sh.v_empty[st], ((n / C::NS) - 1) & 1, abort, 11)) break;
+                uint8_t *vs = v_smem + st * C::PAIR_BYTES;
+                mbar_arrive_expect_tx(&sh.v_full[st], C::PAIR_BYTES);
+                for (int h = 0; h < C::NH; h++) {
+                    tma_load_2d(vs + h * C::HALF_ROWS_BYTES, &tmV, &sh.v_full[st], h * 64, ya);
+                    tma_load_2d(vs + h * C::HALF_ROWS_BYTES + 64 * 128, &tmV, &sh.v_full[st], h * 64, yb);
                 }
             }
         }
-    } else if (warp == 5) {
-        // ------------------------------------------------- MMA issuer
+    } else if (warp == 9 || warp == 10) {
+        // ----------------------------------------- MMA issuer of tile t
+        const int t = warp - 9;
         if (lane == 0 && nblk > 0) {
-            constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64, 0, 0);
+            constexpr uint32_t idesc_s = umma_idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idesc_o = umma_idesc_bf16(128, D, 0, 1);
-            bool ok = mbar_wait(&sh.q_full, 0, abort, 20);
-            const uint32_t q_addr = smem_u32(q_smem);
-            const uint32_t kv_addr = smem_u32(kv_smem);
-            auto issue_s = [&](int n) -> bool {
-                const int st = n % C::NS, buf = n & 1;
-                if (!mbar_wait(&sh.kv_full[st], (n / C::NS) & 1, abort, 21)) return false;
-                tc_fence_after();
-                const uint32_t ks = kv_addr + st * C::STAGE_BYTES;
+            // descriptor bases, built once: per MMA only a 64-bit add of the
+            // byte offset >> 4 into the start-address field remains (shared
+            // memory addresses stay below 2^18, so the field never carries)
+            const uint64_t qd = umma_smem_desc(smem_u32(q_smem + t * C::QT_BYTES), 16, 1024);
+            const uint64_t kd = umma_smem_desc(smem_u32(k_smem), 16, 1024);
+            const uint64_t vd = umma_smem_desc(smem_u32(v_smem), C::HALF_ROWS_BYTES, 1024);
+            const uint32_t s_tmem = tmem + C::S_COL + 128 * t;
+            const uint32_t o_tmem = tmem + C::O_COL + 128 * t;
+            // S_t(n) = Q_t K(n)^T over the pair's 128 keys
+            auto issue_s = [&](int n) {
+                const uint64_t kds = kd + (uint64_t)(((n % C::NS) * C::PAIR_BYTES) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; kk++) {
-                    const uint32_t off = (kk & 3) * 32;   // 16 bf16 = 32 B inside a 128 B swizzle row
-                    const uint64_t ad = umma_smem_desc(q_addr + (kk >> 2) * (C::M * 128) + off, 16, 1024);
-                    const uint64_t bd = umma_smem_desc(ks + (kk >> 2) * C::HALF_BYTES + off, 16, 1024);
-                    umma_ss(tmem + C::S_COL + 64 * buf, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint64_t off = (uint64_t)((((kk >> 2) * C::HALF_ROWS_BYTES) + (kk & 3) * 32) >> 4);
+                    umma_ss(s_tmem, qd + off, kds + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&sh.s_full[buf]);
-                return true;
+                umma_commit(&sh.s_full[t]);
+                mbar_arrive(&sh.s_issued[t]);
             };
-            if (ok) ok = issue_s(0);
-            for (int n = 0; ok && n < nblk; n++) {
-                const int st = n % C::NS, buf = n & 1;
-                if (n + 1 < nblk) {
-                    // S buffer (n+1)&1 holds P(n-1) until PV(n-1) is done
-                    if (n >= 1 && !mbar_wait(&sh.pv_done[(n + 1) & 1], ((n - 1) >> 1) & 1, abort, 22)) break;
-                    if (!issue_s(n + 1)) break;
-                }
-                if (!mbar_wait(&sh.p_full[buf], (n >> 1) & 1, abort, 23)) break;
+            bool ok = mbar_wait(&sh.q_full, 0, abort, 20) && mbar_wait(&sh.k_full[0], 0, abort, 21);
+            // tile 1's first S goes to the pipe right after tile 0's
+            if (ok && t == 1) ok = mbar_wait(&sh.s_issued[0], 0, abort, 25);
+            if (ok) {
                 tc_fence_after();
-                const uint32_t vs = kv_addr + st * C::STAGE_BYTES + C::KV_BYTES;
+                issue_s(0);
+            }
+            for (int n = 0; ok && n < npair; n++) {
+                const int st = n % C::NS;
+                const bool more = n + 1 < npair;
+                // checks that are normally satisfied long ago, done while this
+                // tile's S MMAs are still queued on the pipe
+                if (!mbar_wait(&sh.v_full[st], (n / C::NS) & 1, abort, 26)) break;
+                if (more && !mbar_wait(&sh.k_full[(n + 1) % C::NS], ((n + 1) / C::NS) & 1, abort, 21)) break;
+                // alternate the pipe: PV0(n) after S1(n) was issued, PV1(n) after S0(n+1)
+                if (t == 0 && !mbar_wait(&sh.s_issued[1], n & 1, abort, 27)) break;
+                if (t == 1 && more && !mbar_wait(&sh.s_issued[0], (n + 1) & 1, abort, 28)) break;
+                // the real dependency: this tile's P of pair n
+                if (!mbar_wait(&sh.p_full[t], n & 1, abort, 22)) break;
+                tc_fence_after();
+                // O_t += P_t V: P in S_t columns 0-63, 16 keys (8 columns) per k-step
+                const uint64_t vds = vd + (uint64_t)((st * C::PAIR_BYTES) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < 4; kk++) {
-                    const uint64_t bd = umma_smem_desc(vs + kk * 2048, C::HALF_BYTES, 1024);
-                    umma_ts(tmem, tmem + C::S_COL + 64 * buf + kk * 8, bd, idesc_o,
+                for (int kk = 0; kk < 8; kk++)
+                    umma_ts(o_tmem, s_tmem + kk * 8, vds + (uint64_t)((kk * 2048) >> 4), idesc_o,
                             (n > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(&sh.kv_empty[st]);
-                umma_commit(&sh.pv_done[buf]);
+                umma_commit(&sh.pv_done[t]);
+                // S_t(n+1) right behind PV_t(n): in order on the pipe, so P_t(n) is
+                // read before S_t(n+1) overwrites it
+                if (more) issue_s(n + 1);
             }
         }
     } else {
-        // ------------------------------------------ softmax + epilogue
-        const int r = threadIdx.x;                       // row = TMEM lane
-        const int tok = token0 + r / G;
+        // -------------------------------- softmax + epilogue (warps 0-7)
+        const int t = warp >> 2;
+        const int r = ((warp & 3) << 5) | lane;              // row = TMEM lane
+        const int tok = token0 + t * C::TOK + r / G;
         const long p = (long)q_pos0 + tok;
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t s_addr = lane_addr + C::S_COL + 128 * t;
+        const uint32_t o_addr = lane_addr + C::O_COL + 128 * t;
+        const uint64_t sc2 = f2_pack(sm_scale_log2, sm_scale_log2);
         float m_run = -INFINITY, l = 0.f;
         bool ok = nblk > 0;
-        for (int n = 0; ok && n < nblk; n++) {
-            const int buf = n & 1;
-            if (!mbar_wait(&sh.s_full[buf], (n >> 1) & 1, abort, 30)) { ok = false; break; }
+        for (int n = 0; ok && n < npair; n++) {
+            if (!mbar_wait(&sh.s_full[t], n & 1, abort, 30)) { ok = false; break; }
             tc_fence_after();
-            uint32_t sr[64];
-            tmem_ld32(lane_addr + C::S_COL + 64 * buf, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            tmem_ld32(lane_addr + C::S_COL + 64 * buf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            // the issuer's commit covers every earlier MMA of this tile: S_t(n)
+            // done frees K stage n, and PV_t(n-1) (issued before it) frees V
+            // stage n-1 -- the stage releases ride on this wait, at no cost to
+            // the issuing thread
+            if ((warp & 3) == 0 && lane == 0) {
+                mbar_arrive(&sh.k_empty[n % C::NS]);
+                if (n > 0) mbar_arrive(&sh.v_empty[(n - 1) % C::NS]);
+            }
+            // keys c <= lim[hb] of the pair's half hb are visible: only the
+            // diagonal block and the copy that pads an odd last pair are masked
+            int lim[2];
+#pragma unroll
+            for (int hb = 0; hb < 2; hb++) {
+                const int bi = 2 * n + hb;
+                const int blk = bi < nblk ? sh.blocks[bi] : -1;
+                lim[hb] = blk < 0 ? -1 : (blk == Dg ? (int)(p - 64L * Dg) : 63);
+            }
+            uint32_t sr[128];
+#pragma unroll
+            for (int c0 = 0; c0 < 128; c0 += 32)
+                tmem_ld32(s_addr + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr[c0]));
             tmem_wait_ld();
-            float s[64];
 #pragma unroll
-            for (int c = 0; c < 64; c++) s[c] = __uint_as_float(sr[c]);
-            if (sh.blocks[n] == Dg) {
-                // only the diagonal block has keys after some rows' positions
-                const long limit = p - 64L * Dg;
+            for (int hb = 0; hb < 2; hb++) {
+                if (lim[hb] < 63) {
 #pragma unroll
-                for (int c = 0; c < 64; c++)
-                    if (c > limit) s[c] = -INFINITY;
+                    for (int c = 0; c < 64; c++)
+                        if (c > lim[hb]) sr[64 * hb + c] = 0xff800000u;   // -inf
+                }
             }
-            float q0 = s[0], q1 = s[16], q2 = s[32], q3 = s[48];
+            float q0 = __uint_as_float(sr[0]), q1 = __uint_as_float(sr[1]);
+            float q2 = __uint_as_float(sr[2]), q3 = __uint_as_float(sr[3]);
 #pragma unroll
-            for (int c = 1; c < 15; c += 2) {
-                q0 = max3f(q0, s[c], s[c + 1]);
-                q1 = max3f(q1, s[16 + c], s[17 + c]);
-                q2 = max3f(q2, s[32 + c], s[33 + c]);
-                q3 = max3f(q3, s[48 + c], s[49 + c]);
+            for (int c = 4; c < 128; c += 8) {
+                q0 = max3f(q0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                q1 = max3f(q1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+                q2 = max3f(q2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+                q3 = max3f(q3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
             }
-            const float mx = max3f(max3f(q0, q1, s[15]), max3f(q2, q3, s[31]), fmaxf(s[47], s[63])) *
-                             sm_scale_log2;
+            const float mx = fmaxf(max3f(q0, q1, q2), q3) * sm_scale_log2;
             if (n == 0) {
                 m_run = mx;
             } else if (__any_sync(0xffffffffu, mx > m_run + 8.0f)) {
                 const float m_new = fmaxf(m_run, mx);
                 const float alpha = fast_exp2(m_run - m_new);
-                // O is stable once PV(n-1) has completed
-                if (!mbar_wait(&sh.pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort, 31)) { ok = false; break; }
+                // O_t is stable once PV_t(n-1) has completed
+                if (!mbar_wait(&sh.pv_done[t], (n - 1) & 1, abort, 31)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int c0 = 0; c0 < D; c0 += 32) {
                     uint32_t o[32];
-                    tmem_ld32(lane_addr + c0, o);
+                    tmem_ld32(o_addr + c0, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 32; c++) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                    tmem_st32(lane_addr + c0, o);
+                    tmem_st32(o_addr + c0, o);
                 }
                 tmem_wait_st();
                 l *= alpha;
                 m_run = m_new;
             }
-            // P = 2^(s*c - m): 3 of every 8 pairs on the FMA pipe, the rest on MUFU
-            uint32_t pk[32];
-            const uint64_t sc2 = f2_pack(sm_scale_log2, sm_scale_log2);
+            // P = 2^(s*c - m), 1 of every 4 pairs on the FMA pipe, the rest on
+            // MUFU; S is re-read from TMEM in 32-column chunks, one chunk ahead
             const uint64_t nm2 = f2_pack(-m_run, -m_run);
             uint64_t lacc = f2_pack(0.f, 0.f);
+            uint32_t cur[32], nxt[32];
+            tmem_ld32(s_addr, cur);
 #pragma unroll
-            for (int c = 0; c < 32; c++) {
-                const uint64_t x2 = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), sc2, nm2);
-                uint64_t p2;
-                if ((c & 7) == 1 || (c & 7) == 4 || (c & 7) == 6) {
-                    p2 = exp2_poly_x2(x2);
-                } else {
-                    float x0, x1;
-                    f2_unpack(x2, x0, x1);
-                    p2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+                tmem_wait_ld();
+                if (c0 + 32 < 128) tmem_ld32(s_addr + c0 + 32, nxt);
+                const int lm = lim[c0 >> 6];
+                if (lm < 63) {
+#pragma unroll
+                    for (int c = 0; c < 32; c++)
+                        if ((c0 & 63) + c > lm) cur[c] = 0xff800000u;   // -inf
                 }
-                lacc = f2_add(lacc, p2);
-                float p0, p1;
-                f2_unpack(p2, p0, p1);
-                pk[c] = pack_bf16x2(p0, p1);
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; c++) {
+                    const uint64_t x2 = f2_fma(
+                        f2_pack(__uint_as_float(cur[2 * c]), __uint_as_float(cur[2 * c + 1])), sc2, nm2);
+                    float p0, p1;
+                    if ((c & 3) == 3) {
+                        f2_unpack(exp2_poly_x2(x2), p0, p1);
+                    } else {
+                        float x0, x1;
+                        f2_unpack(x2, x0, x1);
+                        p0 = fast_exp2(x0);
+                        p1 = fast_exp2(x1);
+                    }
+                    lacc = f2_add(lacc, f2_pack(p0, p1));
+                    pk[c] = pack_bf16x2(p0, p1);
+                }
+                // P over S columns [c0/2, c0/2 + 16), all already read
+                tmem_st16(s_addr + c0 / 2, pk);
+                if (c0 + 32 < 128) {
+#pragma unroll
+                    for (int c = 0; c < 32; c++) cur[c] = nxt[c];
+                }
             }
             float la, lb;
             f2_unpack(lacc, la, lb);
-            const float lsum = la + lb;
-            l += lsum;
-            tmem_st32(lane_addr + C::S_COL + 64 * buf, pk);
+            l += la + lb;
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&sh.p_full[buf]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.p_full[t]);
         }
-        if (ok && !mbar_wait(&sh.pv_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, abort, 32)) ok = false;
+        if (ok && !mbar_wait(&sh.pv_done[t], (npair - 1) & 1, abort, 32)) ok = false;
         tc_fence_after();
         const bool store = tok < Tq;
         const int h = g * G + r % G;
@@ -288,7 +369,7 @@ __global__ void __launch_bounds__(192, 1) sparse_attn_prefill_kernel(
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t o[32];
-            tmem_ld32(lane_addr + c0, o);
+            tmem_ld32(o_addr + c0, o);
             tmem_wait_ld();
             uint32_t pk[16];
 #pragma unroll
@@ -308,7 +389,7 @@ __global__ void __launch_bounds__(192, 1) sparse_attn_prefill_kernel(
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
