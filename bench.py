@@ -10,8 +10,12 @@ persistent state and are built before timing).
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier
 and a device synchronise on both sides; each step is bracketed by CUDA
-events on the launching stream and an L2 flush (a 256 MiB write) runs
-between steps outside the events.  Multi-GPU: one process per GPU, each
+events on the launching stream and an L2 flush runs between steps outside
+the events (a 256 MiB write, then a 256 MiB read, so every step starts
+with a cold L2 that holds none of the flush's dirty lines).  The decode
+step (selection + attention) is captured once as a CUDA graph and
+replayed, as a serving loop would run it, so host launch gaps stay out of
+its device time.  Multi-GPU: one process per GPU, each
 rank runs its own sequence (weak scaling, no data-path collective); the
 time is the max over ranks.
 
@@ -42,6 +46,22 @@ UNIT = "tokens/s"
 
 
 # ------------------------------------------------------------ utilities
+
+class L2Flush:
+    """L2 eviction between timed steps: a 256 MiB write, then a 256 MiB read
+    of another buffer, so a step starts with a cold L2 that holds none of the
+    flush's dirty lines (whose write-back would otherwise land on the step)."""
+    DESCRIPTION = ("flushed between steps (256 MiB write, then 256 MiB read: cold, no dirty "
+                   "lines); inputs also exceed L2")
+
+    def __init__(self, dev):
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(64 << 20, dtype=torch.int32, device=dev)
+
+    def __call__(self, k):
+        self.w.fill_(k & 0xFF)
+        torch.sum(self.r)
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -170,7 +190,7 @@ def run_qsa(args, ws, rank, local):
     run = qsa.QSAPrefill(wp.B, wp.Tq, wp.Hq, wp.Hkv, wp.d, wp.T_kv, wp.topk, wp.q_pos0, device=dev)
     run.precompress_cache(K)
     stream = torch.cuda.current_stream()
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     def step(ev=None):
         if ev is None:
@@ -197,7 +217,7 @@ def run_qsa(args, ws, rank, local):
     n0 = qsa.launch_count()
     with ClockSampler(local) as clk:
         for k in range(args.steps):
-            flush.fill_(k & 0xFF)
+            flush(k)
             step(evs[k])
         torch.cuda.synchronize()
     n_launch = qsa.launch_count() - n0
@@ -223,7 +243,7 @@ def run_qsa(args, ws, rank, local):
         "config": {"workload": wp.name, "batch": wp.B, "seq_len": wp.Tq, "q_heads": wp.Hq,
                    "kv_heads": wp.Hkv, "head_dim": wp.d, "block": 64, "topk": wp.topk,
                    "parallelism": f"dp{ws} (independent sequences)",
-                   "l2": "flushed between steps (256 MiB write); inputs also exceed L2"},
+                   "l2": L2Flush.DESCRIPTION},
         "breakdown_ms": {"compress": float(t_comp.mean()), "score_select": float(t_sel.mean()),
                          "attention": float(t_att.mean())},
         "roofline": {"bound": "tensor", "kernel": "sparse_attn_prefill_kernel",
@@ -261,44 +281,53 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush):
     L = wd.q_pos0 + 1
     dec = qsa.QSADecode(wd.B, wd.Hq, wd.Hkv, wd.d, wd.T_kv, wd.topk, device=dev)
     dec.compress(K, 0, L // 64)           # persistent summaries (untimed)
-    stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
         dec(q, K, V, L)
     torch.cuda.synchronize()
+    n0 = qsa.launch_count()
+    graphs = {"step": dec.graph(q, K, V, L, parts=("select", "attention"))}
+    launches_step = qsa.launch_count() - n0   # kernels captured in the step's graph
+    graphs["select"] = dec.graph(q, K, V, L, parts=("select",))
+    graphs["attention"] = dec.graph(q, K, V, L, parts=("attention",))
+    stream = torch.cuda.current_stream()
     steps = max(args.steps, 20)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
-    sel_ws = dec._sel_ws[L]
-    if ws > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    for k in range(steps):
-        flush.fill_(k & 0xFF)
-        evs[k][0].record(stream)
-        qsa.score_select(q.view(wd.B, 1, wd.Hq, wd.d), dec.Kc, dec.idx, wd.topk, L - 1, 1,
-                         dec.sm_scale, sel_ws)
-        evs[k][1].record(stream)
-        qsa.decode(q, K, V, dec.idx, dec.o, L, dec.sm_scale, dec.ws_dec)
-        evs[k][2].record(stream)
-    torch.cuda.synchronize()
+
+    def timed(g):
+        for _ in range(args.warmup):
+            g.replay()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        if ws > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        for k in range(steps):
+            flush(k)
+            evs[k][0].record(stream)
+            g.replay()
+            evs[k][1].record(stream)
+        torch.cuda.synchronize()
+        return np.array([e[0].elapsed_time(e[1]) for e in evs]) * 1e3   # us
+
+    t = {part: timed(g) for part, g in graphs.items()}
     st, det = qsa.device_status()
     if st != "QSA_OK":
         raise RuntimeError(f"decode device status {st} ({det})")
-    t_sel = np.array([e[0].elapsed_time(e[1]) for e in evs])
-    t_att = np.array([e[1].elapsed_time(e[2]) for e in evs])
-    t_step = t_sel + t_att
-    us_step = float(t_step.mean()) * 1e3
+    us_step = float(t["step"].mean())
+    us_att = float(t["attention"].mean())
+    us_sel = float(t["select"].mean())
     by = decode_bytes(wd)
-    att_gbs = by / (float(t_att.mean()) * 1e-3) / 1e9
+    att_gbs = by / (us_att * 1e-6) / 1e9
     sel_bytes = wd.B * wd.Hkv * ((L - 1) // 64) * wd.d * 4   # fp32 summaries read by scoring
     return {"workload": wd.name, "batch": wd.B, "context": L, "topk": wd.topk,
             "us_per_step": us_step, "us_per_token": us_step / wd.B,
-            "breakdown_us": {"score_select": float(t_sel.mean()) * 1e3,
-                             "attention": float(t_att.mean()) * 1e3},
+            "timing": "CUDA graph of the step replayed; events around each replay",
+            "breakdown_us": {"score_select": us_sel, "attention": us_att},
             "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": att_gbs,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": att_gbs / peaks["hbm_gbs"], "bytes_per_launch": by,
                          "traffic": None},
-            "select_gbs": sel_bytes / (float(t_sel.mean()) * 1e-3) / 1e9}
+            "select_gbs": sel_bytes / (us_sel * 1e-6) / 1e9,
+            "select_hbm_frac": sel_bytes / (us_sel * 1e-6) / 1e9 / peaks["hbm_gbs"],
+            "gpu_launches_per_step": int(launches_step)}
 
 
 def bench_e2e(args, qsa, dev, wp, ws):
@@ -445,7 +474,7 @@ def main():
         import block_sparse_long_compress_b200 as qsa
         dev = torch.device("cuda", local)
         torch.cuda.set_device(dev)
-        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        flush = L2Flush(dev)
         res = bench_decode(args, qsa, dev, load_peaks(), ws, rank, flush)
         if rank == 0:
             print(json.dumps(res), flush=True)

@@ -269,3 +269,24 @@ class QSADecode:
                      self._sel_ws[key], stream)
         decode(q, K, V, self.idx, self.o, L, self.sm_scale, self.ws_dec, stream)
         return self.o
+
+    def graph(self, q, K, V, L, parts=("select", "attention")):
+        """Capture the step (or some of its parts) for these buffers and this
+        cache length as a CUDA graph; ``replay()`` then reruns it on the
+        current stream with no host launch work.  Call the step eagerly once
+        first (it sizes the selection workspace)."""
+        q4 = q.view(self.B, 1, self.Hq, self.d)
+        if L not in self._sel_ws:
+            n = score_select_workspace(self.B, self.Hq, self.Hkv, 1, L - 1, 1, self.d, self.topk)
+            self._sel_ws[L] = torch.empty(max(1, n), dtype=torch.uint8, device=q.device)
+        side = torch.cuda.Stream(device=q.device)
+        side.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            if "select" in parts:
+                score_select(q4, self.Kc, self.idx, self.topk, L - 1, 1, self.sm_scale,
+                             self._sel_ws[L], side)
+            if "attention" in parts:
+                decode(q, K, V, self.idx, self.o, L, self.sm_scale, self.ws_dec, side)
+        torch.cuda.current_stream().wait_stream(side)
+        return g

@@ -4,20 +4,25 @@
 // Optimized After Correctness": indexed K/V gather over the selected cells).
 //
 // HBM-bound: every selected 64-token block is read once (K + V, 2*64*d
-// bf16 = 32 KiB at d = 128).  The k selected slots of a (sequence, group)
-// row are split over P CTAs (P <= 8) that form one thread-block cluster.
-// Each CTA runs NW consumer warps; warp w owns one shared-memory stage and
-// walks the CTA's slots w, w+NW, ...:
-//     wait K(i) -> S = q K^T -> TMA K(i+1) into the freed K region ->
-//     softmax (online, per head) -> wait V(i) -> O += P V -> TMA V(i+1)
-// so the next block's loads overlap the current block's math.  S = q K^T
-// and O = P V are bf16 mma.sync m16n8k16 tiles with fp32 accumulation: the
-// G query heads of the group fill rows 0..G-1 of the 16-row A tile, K and V
-// fragments come from the TMA tiles (128-byte swizzle) by ldmatrix /
-// ldmatrix.trans, and P is reused from the S accumulators as the A
-// fragment.  The warps' (max, sum, O) are merged in shared memory; the
-// cluster's CTAs are merged by the leader CTA through distributed shared
-// memory, which writes o.  No global workspace, no atomics.
+// bf16 = 32 KiB at d = 128) and the arithmetic per byte is tiny, so the
+// kernel is built to keep enough bytes in flight on every SM.
+//
+// The k selected slots of a (sequence, group) row are split into P equal
+// ranges, one per CTA; the row's P CTAs form one thread-block cluster
+// (P <= 8) and two CTAs share an SM.  Per CTA:
+//   producer warp   keeps a ring of NS stages full with TMA loads (one
+//                   stage = one block's K and V, 128-byte swizzle),
+//                   refilling a stage as soon as the consumers release it;
+//   4 consumer warps  every warp takes 16 of each block's 64 keys:
+//                   S^T = K q^T with the keys on the MMA M side (m16n8k16,
+//                   the G heads of the group on N), online softmax per head
+//                   over the warp's keys, P^T turned into the B operand by
+//                   movmatrix, O^T += V^T P^T (d on M, V^T by
+//                   ldmatrix.trans).  No padding rows: 16 MMAs per warp and
+//                   block.
+// The P x 4 warp partials (max, sum, O) of the row are merged in one pass
+// through distributed shared memory, each CTA finishing 1/P of the row's
+// outputs.  No global workspace, no global atomics.
 #pragma once
 #include <cooperative_groups.h>
 
@@ -27,13 +32,21 @@ namespace qsa {
 
 template <int D>
 struct DecodeCfg {
-    static constexpr int NH = D / 64;
-    static constexpr int HALF_BYTES = 64 * 128;
-    static constexpr int KV_BYTES = 64 * D * 2;
-    static constexpr int NW = 6;                       // consumer warps per CTA
-    static constexpr int PART_FLOATS = 16 + 8 * D;     // m[8], l[8], O[8][D]
-    static constexpr int SMEM_BYTES = NW * 2 * KV_BYTES + NW * PART_FLOATS * 4 + 1024;
+    static constexpr int NH = D / 64;                  // 64-column TMA boxes per row
+    static constexpr int HALF_BYTES = 64 * 128;        // one 64-row x 128-byte box
+    static constexpr int KV_BYTES = 64 * D * 2;        // one block's K (or V)
+    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+    static constexpr int CTAS_PER_SM = 2;
+    static constexpr int RING_BYTES = 96 * 1024;       // NS stages; two CTAs per SM
+    static constexpr int NS = RING_BYTES / STAGE_BYTES;
+    static constexpr int NC = 4;                       // consumer warps
+    static constexpr int THREADS = (NC + 1) * 32;
+    static constexpr int PART_FLOATS = 16 + 8 * D;     // m[8], l[8], O[8][D] of one warp
+    static constexpr int SMEM_BYTES = RING_BYTES + 1024;
+    static constexpr int MAX_SLOTS = 64;
     static constexpr int MAX_CLUSTER = 8;
+    static_assert(NS >= 2, "ring too small");
+    static_assert(NC * PART_FLOATS * 4 <= RING_BYTES, "merge scratch must fit in the ring");
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
@@ -50,6 +63,14 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t 
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                  : "r"(addr));
+}
+
+// Transpose of an 8x8 b16 matrix held in the mma fragment layout.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t a)
+{
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -70,233 +91,258 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int c16)
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(DecodeCfg<D>::NW * 32, 1) decode_kernel(
+__global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_SM) decode_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ idx,
     __nv_bfloat16 *__restrict__ o, int Hq, int Hkv, int L, int T_kv_max, int topk, int spc,
     float sm_scale_log2)
 {
     using C = DecodeCfg<D>;
-    constexpr int NW = C::NW;
+    constexpr int NS = C::NS;
+    constexpr int NC = C::NC;
     constexpr int PF = C::PART_FLOATS;
+    constexpr int MAX_SRC = C::MAX_CLUSTER * NC;
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    __shared__ uint64_t bar_k[NW], bar_v[NW];
-    __shared__ int abort_flag;
-    __shared__ float cta_part[PF];   // this CTA's merged (m, l, O), read by the cluster leader
+    __shared__ uint64_t full[NS], empty[NS];
+    __shared__ int blocks[C::MAX_SLOTS];   // the CTA's valid block ids in slot order
+    __shared__ int nb_sh, issued_sh, abort_flag;
+    __shared__ float wgt[MAX_SRC][8];      // per-source, per-head merge weights
+    __shared__ float lsrc[MAX_SRC][8];
+    __shared__ float inv_l[8];
 
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *part = reinterpret_cast<float *>(smem + NW * 2 * C::KV_BYTES);   // [NW][PF]
+    uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *part = reinterpret_cast<float *>(ring);   // after the loop: [NC][PF] warp partials
 
-    const int split = blockIdx.x;
     const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv;
+    const int P = (int)cluster.num_blocks();
+    const int rank = (int)cluster.block_rank();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int slot1 = min(split * spc + spc, topk);
     const int last_blk = (L - 1) / 64;
-    const int32_t *row_idx = idx + (long)bg * topk;
     const int kv_row0 = bg * T_kv_max;       // host checks B*Hkv*T_kv_max < 2^31
 
-    uint8_t *ks = smem + warp * 2 * C::KV_BYTES;
-    uint8_t *vs = ks + C::KV_BYTES;
-    if (threadIdx.x == 0) abort_flag = 0;
-    if (lane == 0) {
-        mbar_init(&bar_k[warp], 1);
-        mbar_init(&bar_v[warp], 1);
+    // the CTA's valid block ids, compacted in slot order
+    const int slot0 = rank * spc;
+    const int slot1 = min(slot0 + spc, topk);
+    if (warp == 0) {
+        int n = 0;
+        for (int base = slot0; base < slot1; base += 32) {
+            const int s = base + lane;
+            int j = s < slot1 ? __ldg(idx + (long)bg * topk + s) : -1;
+            if (j > last_blk) {
+                report(QSA_ERR_BOUNDS, 3);
+                j = -1;
+            }
+            const unsigned m = __ballot_sync(0xffffffffu, j >= 0);
+            if (j >= 0) blocks[n + __popc(m & ((1u << lane) - 1u))] = j;
+            n += __popc(m);
+        }
+        if (lane == 0) nb_sh = n;
+    }
+    if (threadIdx.x == 32) {
+        abort_flag = 0;
+        issued_sh = 0;
+#pragma unroll
+        for (int s = 0; s < NS; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], NC);
+        }
         fence_barrier_init();
     }
     __syncthreads();
+    const int nb = nb_sh;
 
-    // block id of slot s of this CTA's range (-1 past the selection)
-    auto block_of = [&](int s) -> int {
-        if (s >= slot1) return -1;
-        int j = __ldg(row_idx + s);
-        if (j > last_blk) {
-            if (lane == 0) report(QSA_ERR_BOUNDS, 3);
-            j = -1;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    float oacc[D / 16][4];
+#pragma unroll
+    for (int mt = 0; mt < D / 16; mt++) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
+
+    if (warp == NC) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            int i = 0;
+            for (; i < nb; i++) {
+                const int st = i % NS;
+                if (i >= NS) {
+                    if (!mbar_wait(&empty[st], ((i / NS) - 1) & 1, &abort_flag, 42)) break;
+                    fence_proxy_async_smem();
+                }
+                const int row = kv_row0 + 64 * blocks[i];
+                mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
+                uint8_t *ks = ring + st * C::STAGE_BYTES;
+                uint8_t *vs = ks + C::KV_BYTES;
+#pragma unroll
+                for (int h = 0; h < C::NH; h++) tma_load_2d(ks + h * C::HALF_BYTES, &tmK, &full[st], h * 64, row);
+#pragma unroll
+                for (int h = 0; h < C::NH; h++) tma_load_2d(vs + h * C::HALF_BYTES, &tmV, &full[st], h * 64, row);
+            }
+            issued_sh = i;
         }
-        return j;
-    };
-    auto load_k = [&](int j) {
-        mbar_arrive_expect_tx(&bar_k[warp], C::KV_BYTES);
+    } else {
+        // ---------------------------------------------------- consumers
+        // B operand of S^T = K q^T: column n = head lane/4 of the group
+        // (zero for n >= G), rows k = d.
+        const int hn = lane >> 2, qc = (lane & 3) * 2;
+        uint32_t qb[D / 16][2];
+        {
+            const __nv_bfloat16 *qrow = q + ((long)b * Hq + g * G + (hn < G ? hn : 0)) * D;
 #pragma unroll
-        for (int h = 0; h < C::NH; h++)
-            tma_load_2d(ks + h * C::HALF_BYTES, &tmK, &bar_k[warp], h * 64, kv_row0 + 64 * j);
-    };
-    auto load_v = [&](int j) {
-        mbar_arrive_expect_tx(&bar_v[warp], C::KV_BYTES);
-#pragma unroll
-        for (int h = 0; h < C::NH; h++)
-            tma_load_2d(vs + h * C::HALF_BYTES, &tmV, &bar_v[warp], h * 64, kv_row0 + 64 * j);
-    };
-
-    int s = split * spc + warp;
-    int j = block_of(s);
-    if (lane == 0 && j >= 0) {
-        load_k(j);
-        load_v(j);
-    }
-
-    // query fragment: row = lane/4 = head within the group (rows >= G and
-    // 8..15 are zero), columns 16ks + 2(lane%4) + {0,1} and +8.
-    const int hr = lane >> 2, qc = (lane & 3) * 2;
-    uint32_t qa[D / 16][2];
-    {
-        const __nv_bfloat16 *qrow = q + ((long)b * Hq + g * G + (hr < G ? hr : 0)) * D;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; kk++) {
-            const uint32_t lo = *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + qc);
-            const uint32_t hi = *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 8 + qc);
-            qa[kk][0] = hr < G ? lo : 0u;
-            qa[kk][1] = hr < G ? hi : 0u;
-        }
-    }
-
-    float m_run = -INFINITY, l_run = 0.f;
-    float oacc[D / 8][4];
-#pragma unroll
-    for (int nt = 0; nt < D / 8; nt++) oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
-
-    const uint32_t kaddr = smem_u32(ks), vaddr = smem_u32(vs);
-    const int mi = lane >> 3, rr = lane & 7;
-    uint32_t phase = 0;
-    while (j >= 0) {
-        const int s_next = s + NW;
-        const int j_next = block_of(s_next);
-        if (!mbar_wait(&bar_k[warp], phase, &abort_flag, 40)) break;
-        // ---- S = q K^T (ldmatrix.x4: matrix mi = (k-step kk + (mi>>1), half mi&1))
-        float sacc[8][4];
-#pragma unroll
-        for (int nt = 0; nt < 8; nt++) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-#pragma unroll
-        for (int nt = 0; nt < 8; nt++) {
-#pragma unroll
-            for (int kk = 0; kk < D / 16; kk += 2) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4(kaddr + sw128_offset(8 * nt + rr, 2 * (kk + (mi >> 1)) + (mi & 1)), b0, b1, b2, b3);
-                mma_bf16_16816(sacc[nt], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
-                mma_bf16_16816(sacc[nt], qa[kk + 1][0], 0u, qa[kk + 1][1], 0u, b2, b3);
+            for (int kk = 0; kk < D / 16; kk++) {
+                const uint32_t lo = *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + qc);
+                const uint32_t hi = *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 8 + qc);
+                qb[kk][0] = hn < G ? lo : 0u;
+                qb[kk][1] = hn < G ? hi : 0u;
             }
         }
-        // K region consumed: prefetch the next block's keys
-        __syncwarp();
-        if (lane == 0 && j_next >= 0) {
-            fence_proxy_async_smem();
-            load_k(j_next);
-        }
-        // ---- online softmax (per head = per lane quad)
-        const int lim = (L - 1) - 64 * j;    // keys c <= lim are visible
-        float mx = -INFINITY;
+        const int k0 = 16 * warp;                                  // the warp's keys in each block
+        const int krow_a = k0 + (lane & 7) + 8 * ((lane >> 3) & 1);  // K rows for ldmatrix (A of S^T)
+        const int kchunk_a = lane >> 4;
+        const int vrow_a = k0 + (lane & 7) + 8 * (lane >> 4);        // V rows for ldmatrix.trans (A of O^T)
+        const int vchunk_a = (lane >> 3) & 1;
+        const int key_lo = k0 + (lane >> 2);                         // keys of this thread's S^T entries
+        for (int i = 0; i < nb; i++) {
+            const int st = i % NS;
+            if (!mbar_wait(&full[st], (i / NS) & 1, &abort_flag, 40)) break;
+            const int j = blocks[i];
+            const uint32_t kaddr = smem_u32(ring + st * C::STAGE_BYTES);
+            const uint32_t vaddr = kaddr + C::KV_BYTES;
+            // ---- S^T (16 keys x 8 heads) = K q^T
+            float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int nt = 0; nt < 8; nt++) {
-#pragma unroll
-            for (int e = 0; e < 2; e++) {
-                const int key = 8 * nt + qc + e;
-                sacc[nt][e] = key <= lim ? sacc[nt][e] * sm_scale_log2 : -INFINITY;
-                mx = fmaxf(mx, sacc[nt][e]);
+            for (int kk = 0; kk < D / 16; kk++) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(kaddr + sw128_offset(krow_a, 2 * kk + kchunk_a), a0, a1, a2, a3);
+                mma_bf16_16816(s, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
             }
-        }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float m_new = fmaxf(m_run, mx);
-        const float alpha = fast_exp2(m_run - m_new);   // 0 on the first block
-        m_run = m_new;
-        l_run *= alpha;
+            // ---- online softmax per head over the warp's keys
+            const int lim = (L - 1) - 64 * j;   // keys c <= lim are visible
+            const bool v0 = key_lo <= lim, v1 = key_lo + 8 <= lim;
+            s[0] = v0 ? s[0] * sm_scale_log2 : -INFINITY;
+            s[1] = v0 ? s[1] * sm_scale_log2 : -INFINITY;
+            s[2] = v1 ? s[2] * sm_scale_log2 : -INFINITY;
+            s[3] = v1 ? s[3] * sm_scale_log2 : -INFINITY;
+            float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
 #pragma unroll
-        for (int nt = 0; nt < D / 8; nt++) {
-            oacc[nt][0] *= alpha;
-            oacc[nt][1] *= alpha;
-        }
-        uint32_t pa[8];
-#pragma unroll
-        for (int nt = 0; nt < 8; nt++) {
-            const float p0 = fast_exp2(sacc[nt][0] - m_run), p1 = fast_exp2(sacc[nt][1] - m_run);
-            l_run += p0 + p1;
-            pa[nt] = pack_bf16x2(p0, p1);
-        }
-        // ---- O += P V (ldmatrix.trans: matrix mi = (keys half mi&1, column tile nt + (mi>>1)))
-        if (!mbar_wait(&bar_v[warp], phase, &abort_flag, 41)) break;
-#pragma unroll
-        for (int k2 = 0; k2 < 4; k2++) {
-#pragma unroll
-            for (int nt = 0; nt < D / 8; nt += 2) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_t(vaddr + sw128_offset(16 * k2 + 8 * (mi & 1) + rr, nt + (mi >> 1)), b0, b1, b2, b3);
-                mma_bf16_16816(oacc[nt], pa[2 * k2], 0u, pa[2 * k2 + 1], 0u, b0, b1);
-                mma_bf16_16816(oacc[nt + 1], pa[2 * k2], 0u, pa[2 * k2 + 1], 0u, b2, b3);
+            for (int off = 4; off < 32; off <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
             }
-        }
-        __syncwarp();
-        if (lane == 0 && j_next >= 0) {
-            fence_proxy_async_smem();
-            load_v(j_next);
-        }
-        phase ^= 1u;
-        s = s_next;
-        j = j_next;
-    }
-    // row sums of the warp: reduce the quad's partial sums
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-
-    // ---- merge the warps of this CTA in shared memory
-    float *wp = part + warp * PF;
-    if ((lane & 3) == 0) {
-        wp[hr] = m_run;
-        wp[8 + hr] = l_run;
-    }
+            const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+            // a head whose keys are all masked so far keeps a finite reference
+            const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
+            const float al0 = fast_exp2(m_run[0] - mu0), al1 = fast_exp2(m_run[1] - mu1);
+            m_run[0] = mn0;
+            m_run[1] = mn1;
+            const float p0 = fast_exp2(s[0] - mu0), p1 = fast_exp2(s[1] - mu1);
+            const float p2 = fast_exp2(s[2] - mu0), p3 = fast_exp2(s[3] - mu1);
+            l_run[0] = l_run[0] * al0 + (p0 + p2);
+            l_run[1] = l_run[1] * al1 + (p1 + p3);
 #pragma unroll
-    for (int nt = 0; nt < D / 8; nt++) {
-        wp[16 + hr * D + 8 * nt + qc] = oacc[nt][0];
-        wp[16 + hr * D + 8 * nt + qc + 1] = oacc[nt][1];
+            for (int mt = 0; mt < D / 16; mt++) {
+                oacc[mt][0] *= al0;
+                oacc[mt][1] *= al1;
+                oacc[mt][2] *= al0;
+                oacc[mt][3] *= al1;
+            }
+            // P^T as the B operand (k = key, n = head): transpose the two
+            // 8x8 halves of the S^T accumulator fragment
+            const uint32_t pb0 = movmatrix_t(pack_bf16x2(p0, p1));
+            const uint32_t pb1 = movmatrix_t(pack_bf16x2(p2, p3));
+            // ---- O^T (d x heads) += V^T P^T over the warp's 16 keys
+#pragma unroll
+            for (int mt = 0; mt < D / 16; mt++) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(vaddr + sw128_offset(vrow_a, 2 * mt + vchunk_a), a0, a1, a2, a3);
+                mma_bf16_16816(oacc[mt], a0, a1, a2, a3, pb0, pb1);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+        // row sums over the warp's keys: lanes with equal lane%4 hold the same heads
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
+            l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
+        }
     }
     __syncthreads();
-    // CTA partial (shifted by the CTA max, unnormalised)
-    for (int e = threadIdx.x; e < G * D; e += NW * 32) {
-        const int h = e / D, c = e % D;
-        float mc = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < NW; w++) mc = fmaxf(mc, part[w * PF + h]);
-        float oc = 0.f, lc = 0.f;
-        if (mc != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < NW; w++) {
-                const float f = fast_exp2(part[w * PF + h] - mc);
-                oc += f * part[w * PF + 16 + h * D + c];
-                lc += f * part[w * PF + 8 + h];
-            }
+    if (abort_flag && threadIdx.x == NC * 32) {
+        // a wait gave up: let the copies still in flight land before the
+        // ring is reused (bounded, no abort short-cut)
+        const int issued = issued_sh;
+        for (int i = max(0, issued - NS); i < issued; i++)
+            mbar_wait(&full[i % NS], (i / NS) & 1, nullptr, 43, 100000000ull);
+    }
+    __syncthreads();
+
+    // ---- warp partials (m, l, O) into the idle ring
+    if (warp < NC) {
+        float *wp = part + warp * PF;
+        const int hn = lane >> 2, qc = (lane & 3) * 2;
+        if (lane < 4) {
+            wp[qc] = m_run[0];
+            wp[qc + 1] = m_run[1];
+            wp[8 + qc] = l_run[0];
+            wp[8 + qc + 1] = l_run[1];
         }
-        cta_part[16 + h * D + c] = oc;
-        if (c == 0) {
-            cta_part[h] = mc;
-            cta_part[8 + h] = lc;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; mt++) {
+            wp[16 + qc * D + 16 * mt + hn] = oacc[mt][0];
+            wp[16 + (qc + 1) * D + 16 * mt + hn] = oacc[mt][1];
+            wp[16 + qc * D + 16 * mt + 8 + hn] = oacc[mt][2];
+            wp[16 + (qc + 1) * D + 16 * mt + 8 + hn] = oacc[mt][3];
         }
     }
-    // ---- merge the cluster's CTAs (one per split) through distributed shared memory
+    // ---- one merge over the row's P x NC partials (distributed shared memory)
     cluster.sync();
-    if (cluster.block_rank() == 0) {
-        const int P = (int)cluster.num_blocks();
-        for (int e = threadIdx.x; e < G * D; e += NW * 32) {
-            const int h = e / D, c = e % D;
-            float mc = -INFINITY;
-            for (int r = 0; r < P; r++) {
-                const float *rp = cluster.map_shared_rank(cta_part, r);
-                mc = fmaxf(mc, rp[h]);
+    const int nsrc = P * NC;
+    for (int e = threadIdx.x; e < nsrc * G; e += C::THREADS) {
+        const int src = e / G, h = e % G;
+        const float *pp = cluster.map_shared_rank(part, src / NC) + (src % NC) * PF;
+        wgt[src][h] = pp[h];          // m, turned into a weight below
+        lsrc[src][h] = pp[8 + h];
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+        const int h = threadIdx.x;
+        float mc = -INFINITY;
+        for (int src = 0; src < nsrc; src++) mc = fmaxf(mc, wgt[src][h]);
+        float lc = 0.f;
+        for (int src = 0; src < nsrc; src++) {
+            const float f = mc == -INFINITY ? 0.f : fast_exp2(wgt[src][h] - mc);
+            wgt[src][h] = f;
+            lc += f * lsrc[src][h];
+        }
+        inv_l[h] = lc > 0.f ? 1.f / lc : 0.f;
+    }
+    __syncthreads();
+    {
+        const int n4 = G * D / 4;
+        const int per = (n4 + P - 1) / P;
+        const int e_end = min(n4, (rank + 1) * per);
+        for (int e4 = rank * per + threadIdx.x; e4 < e_end; e4 += C::THREADS) {
+            const int h = (e4 * 4) / D, c = (e4 * 4) % D;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+            for (int src = 0; src < nsrc; src++) {
+                const float f = wgt[src][h];
+                const float4 x = *reinterpret_cast<const float4 *>(
+                    cluster.map_shared_rank(part, src / NC) + (src % NC) * PF + 16 + h * D + c);
+                acc.x += f * x.x;
+                acc.y += f * x.y;
+                acc.z += f * x.z;
+                acc.w += f * x.w;
             }
-            float oc = 0.f, lc = 0.f;
-            if (mc != -INFINITY) {
-                for (int r = 0; r < P; r++) {
-                    const float *rp = cluster.map_shared_rank(cta_part, r);
-                    const float f = fast_exp2(rp[h] - mc);
-                    oc += f * rp[16 + h * D + c];
-                    lc += f * rp[8 + h];
-                }
-            }
-            o[((long)b * Hq + g * G + h) * D + c] = __float2bfloat16_rn(lc > 0.f ? oc / lc : 0.f);
+            const float il = inv_l[h];
+            uint2 out;
+            out.x = pack_bf16x2(acc.x * il, acc.y * il);
+            out.y = pack_bf16x2(acc.z * il, acc.w * il);
+            *reinterpret_cast<uint2 *>(o + ((long)b * Hq + g * G + h) * D + c) = out;
         }
     }
-    cluster.sync();   // the other CTAs' shared memory must outlive the leader's reads
+    cluster.sync();   // the other CTAs' shared memory must outlive the reads into it
 }
 
 }  // namespace qsa

@@ -146,15 +146,16 @@ int sm_count()
     return cache[dev];
 }
 
-// Splits of a (sequence, group) row: about one CTA per SM over all rows,
-// at most 8 (one portable cluster), at least one slot per CTA.
+// CTAs per (sequence, group) row: about CTAS_PER_SM * SMs CTAs over all
+// rows without a second wave; at most 8 (one portable cluster) and at
+// least one selected slot per CTA.
 struct DecodePlan {
     int P, spc;
 };
 
-DecodePlan plan_decode(int rows, int topk, int nsm)
+DecodePlan plan_decode(int rows, int topk, int nsm, int ctas_per_sm)
 {
-    int P = (nsm + rows / 2) / rows;
+    int P = (ctas_per_sm * nsm) / rows;
     P = P < 1 ? 1 : P;
     P = P > 8 ? 8 : P;
     P = P > topk ? topk : P;
@@ -204,12 +205,12 @@ qsa_status launch_decode(const void *q, const void *K, const void *V, const int3
     qsa_status st;
     if ((st = make_map_2d(&mk, K, (uint64_t)B * Hkv * T_kv_max, D)) != QSA_OK) return st;
     if ((st = make_map_2d(&mv, V, (uint64_t)B * Hkv * T_kv_max, D)) != QSA_OK) return st;
-    const DecodePlan p = plan_decode(B * Hkv, topk, sm_count());
+    const DecodePlan p = plan_decode(B * Hkv, topk, sm_count(), C::CTAS_PER_SM);
     auto kern = qsa::decode_kernel<D, G>;
     if ((st = set_smem(kern, C::SMEM_BYTES)) != QSA_OK) return st;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.P, B * Hkv, 1);
-    cfg.blockDim = dim3(C::NW * 32, 1, 1);
+    cfg.blockDim = dim3(C::THREADS, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
