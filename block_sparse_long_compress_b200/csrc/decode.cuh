@@ -123,6 +123,10 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_
     const int last_blk = (L - 1) / 64;
     const int kv_row0 = bg * T_kv_max;       // host checks B*Hkv*T_kv_max < 2^31
 
+    // no global memory before the previous kernel on the stream (normally
+    // the selection that writes idx) has completed
+    grid_dependency_wait();
+    grid_launch_dependents();
     // the CTA's valid block ids, compacted in slot order
     const int slot0 = rank * spc;
     const int slot1 = min(slot0 + spc, topk);

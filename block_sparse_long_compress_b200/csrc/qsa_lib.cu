@@ -131,6 +131,38 @@ SelectPlan plan_select(int B, int Hkv, int Tq, int q_pos0, int qblk, int d)
     return p;
 }
 
+// Per-token rows (qblk = 1) take the one-launch path when every row's
+// candidates fit in 8 chunks of at most 8192: the chunks of a row form a
+// cluster of NCH CTAs (enough CTAs to cover the SMs about 4 times).
+struct TokenPlan {
+    bool use;
+    int NCH, CH;
+};
+
+int sm_count();
+
+TokenPlan plan_token(int B, int Hkv, int Tq, int q_pos0, int qblk)
+{
+    TokenPlan p = {false, 1, 32};
+    if (qblk != 1 || Tq > 65535 || (long)B * Hkv > 65535) return p;
+    const int Dmax = (q_pos0 + Tq - 1) / 64;
+    const int ncand = Dmax > 1 ? Dmax - 1 : 0;
+    if (ncand > 8 * 8192) return p;
+    const long rows = (long)B * Hkv * Tq;
+    long nch = (4L * sm_count() + rows - 1) / rows;
+    nch = nch > 8 ? 8 : nch;
+    const long by_size = (ncand + 31) / 32;          // at least 32 candidates per chunk
+    nch = nch > by_size ? by_size : nch;
+    const long need = (ncand + 8191) / 8192;         // at most 8192 per chunk
+    nch = nch < need ? need : nch;
+    nch = nch < 1 ? 1 : nch;
+    p.use = true;
+    p.NCH = (int)nch;
+    const int per = (ncand + p.NCH - 1) / p.NCH;
+    p.CH = per < 32 ? 32 : (per + 31) / 32 * 32;
+    return p;
+}
+
 // ------------------------------------------------------- decode geometry
 int sm_count()
 {
@@ -213,17 +245,56 @@ qsa_status launch_decode(const void *q, const void *K, const void *V, const int3
     cfg.blockDim = dim3(C::THREADS, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = p.P;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see grid_dependency_wait()
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mk, mv, (const __nv_bfloat16 *)q, idx, (__nv_bfloat16 *)o, Hq,
                                        Hkv, L, T_kv_max, topk, p.spc, sm_scale * 1.4426950408889634f);
     if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "decode_kernel launch: %s", cudaGetErrorString(e));
     return launched("decode_kernel");
+}
+
+template <int D>
+qsa_status launch_select_token_d(const void *Q, const float *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
+                                 int q_pos0, int nblk_max, int topk, float sm_scale, const TokenPlan &tp,
+                                 cudaStream_t s)
+{
+    auto kern = qsa::select_token_kernel<D>;
+    const int smem = (tp.CH + tp.NCH * qsa::kMaxChosen) * 8;
+    qsa_status st;
+    if ((st = set_smem(kern, smem)) != QSA_OK) return st;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(tp.NCH, Tq, B * Hkv);
+    cfg.blockDim = dim3(qsa::kSelThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = tp.NCH;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see grid_dependency_wait()
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, (const __nv_bfloat16 *)Q, Kc, idx, nblk_max, Tq, Hq, Hkv,
+                                       q_pos0, topk, sm_scale, tp.CH);
+    if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "select_token_kernel launch: %s", cudaGetErrorString(e));
+    return launched("select_token_kernel");
+}
+
+qsa_status launch_select_token(const void *Q, const float *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
+                               int q_pos0, int nblk_max, int d, int topk, float sm_scale, const TokenPlan &tp,
+                               cudaStream_t s)
+{
+    if (d == 128) return launch_select_token_d<128>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, nblk_max, topk, sm_scale, tp, s);
+    return launch_select_token_d<64>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, nblk_max, topk, sm_scale, tp, s);
 }
 
 __global__ void selftest_exp2_kernel(const float *__restrict__ x, float *__restrict__ y, int n)
@@ -322,6 +393,7 @@ size_t qsa_score_select_workspace(int B, int Hq, int Hkv, int Tq, int q_pos0, in
     (void)Hq;
     (void)topk;
     if (B <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || (qblk != 1 && qblk != 64) || !supported_d(d)) return 0;
+    if (plan_token(B, Hkv, Tq, q_pos0, qblk).use) return 0;
     const SelectPlan p = plan_select(B, Hkv, Tq, q_pos0, qblk, d);
     return p.qbar_bytes + p.part_bytes;
 }
@@ -343,13 +415,16 @@ qsa_status qsa_score_select(const void *Q, const float *Kc, int32_t *idx, int B,
     if ((long)Hq * d / 8 > 1024) return fail(QSA_ERR_UNSUPPORTED, "qsa_score_select: Hq*d too large");
     if (!aligned16(Q) || !aligned16(Kc) || !aligned16(idx))
         return fail(QSA_ERR_INVALID_ARG, "qsa_score_select: misaligned pointer");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const TokenPlan tp = plan_token(B, Hkv, Tq, q_pos0, qblk);
+    if (tp.use) return launch_select_token(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, T_kv_max / 64, d, topk, sm_scale,
+                                           tp, s);
     const SelectPlan p = plan_select(B, Hkv, Tq, q_pos0, qblk, d);
     if (p.maxchunks * qsa::kMaxChosen * 8 > 200 * 1024)
         return fail(QSA_ERR_UNSUPPORTED, "qsa_score_select: context too long");
     if (!workspace || workspace_bytes < p.qbar_bytes + p.part_bytes || !aligned16(workspace))
         return fail(QSA_ERR_WORKSPACE, "qsa_score_select: workspace needs %zu bytes",
                     p.qbar_bytes + p.part_bytes);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     float *Qbar = static_cast<float *>(workspace);
     uint64_t *part = reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(workspace) + p.qbar_bytes);
     const int nblk_max = T_kv_max / 64;

@@ -16,10 +16,19 @@
 //                        workspace.
 //   merge_select_kernel  one CTA per row with several chunks: the same
 //                        select over the union of the chunks' top-m lists.
+//   select_token_kernel  per-token rows (qblk = 1, e.g. decode) in one
+//                        launch: the chunks of a row form a thread-block
+//                        cluster; every CTA pools its token's query over the
+//                        group's heads, scores its chunk and selects the
+//                        chunk's top-m into shared memory; the leader merges
+//                        the chunks' lists through distributed shared memory
+//                        and writes the row.  No workspace.
 // Key of candidate j with score s: (order-preserving bits of s) << 32 |
 // (0xFFFFFFFF - j); keys are unique, larger = better, and the lower block
 // wins a score tie.  -0.0 is folded into +0.0.
 #pragma once
+#include <cooperative_groups.h>
+
 #include "device.cuh"
 
 namespace qsa {
@@ -236,32 +245,21 @@ __device__ __forceinline__ RowGeom row_geom(int i, int Tq, int q_pos0, int qblk,
     return g;
 }
 
-// --------------------------------------------------------- score+select
-// grid (maxchunks, NR, B*Hkv); dynamic smem CH * 8 bytes.
+// fp32 scores of n candidates (block summaries kc[0..n) of d = D floats,
+// block ids j0..j0+n-1) against the pooled query qb, as 64-bit keys.  Each
+// warp takes 8 candidates at a time; lane owns columns [lane*V, lane*V+V);
+// a transposing butterfly leaves candidate (lane >> 2) of the group in
+// lanes with (lane & 3) == 0.
 template <int D>
-__global__ void __launch_bounds__(kSelThreads) score_select_kernel(
-    const float *__restrict__ Qbar, const float *__restrict__ Kc, int32_t *__restrict__ idx,
-    uint64_t *__restrict__ part, int nblk_max, int Tq, int q_pos0, int qblk, int topk,
-    float sm_scale, int CH, int maxchunks)
+__device__ __forceinline__ void score_chunk(const float *qb, const float *__restrict__ kc, int n, int j0,
+                                            float sm_scale, uint64_t *keys)
 {
-    extern __shared__ uint64_t keys[];
-    __shared__ SelectShared sh;
-    const int chunk = blockIdx.x, i = blockIdx.y, bg = blockIdx.z, NR = gridDim.y;
-    const RowGeom g = row_geom(i, Tq, q_pos0, qblk, topk, CH);
-    if (chunk >= g.nchunks) return;
-    const int j0 = 1 + chunk * CH;
-    const int n = max(0, min(CH, g.ncand - chunk * CH));
-    const long row = (long)bg * NR + i;
-
-    // fp32 scores: each warp takes 8 candidates at a time; lane owns
-    // columns [lane*V, lane*V+V); a transposing butterfly leaves candidate
-    // (lane >> 2) of the group in lanes with (lane & 3) == 0.
     constexpr int V = D / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float q[V];
 #pragma unroll
-    for (int v = 0; v < V; v++) q[v] = Qbar[row * D + lane * V + v];
-    const float *kc_base = Kc + ((long)bg * nblk_max + j0) * D + lane * V;
+    for (int v = 0; v < V; v++) q[v] = qb[lane * V + v];
+    const float *kc_base = kc + lane * V;
     for (int base = warp * 8; base < n; base += 8 * (kSelThreads / 32)) {
         float s[8];
 #pragma unroll
@@ -303,6 +301,26 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
         const int e = base + (lane >> 2);
         if ((lane & 3) == 0 && e < n) keys[e] = make_key(s[0] * sm_scale, j0 + e);
     }
+}
+
+// --------------------------------------------------------- score+select
+// grid (maxchunks, NR, B*Hkv); dynamic smem CH * 8 bytes.
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) score_select_kernel(
+    const float *__restrict__ Qbar, const float *__restrict__ Kc, int32_t *__restrict__ idx,
+    uint64_t *__restrict__ part, int nblk_max, int Tq, int q_pos0, int qblk, int topk,
+    float sm_scale, int CH, int maxchunks)
+{
+    extern __shared__ uint64_t keys[];
+    __shared__ SelectShared sh;
+    const int chunk = blockIdx.x, i = blockIdx.y, bg = blockIdx.z, NR = gridDim.y;
+    const RowGeom g = row_geom(i, Tq, q_pos0, qblk, topk, CH);
+    if (chunk >= g.nchunks) return;
+    const int j0 = 1 + chunk * CH;
+    const int n = max(0, min(CH, g.ncand - chunk * CH));
+    const long row = (long)bg * NR + i;
+
+    score_chunk<D>(Qbar + row * D, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
     __syncthreads();
 
     const int need = min(g.m, n);
@@ -335,6 +353,67 @@ __global__ void __launch_bounds__(kSelThreads) merge_select_kernel(
     }
     __syncthreads();
     select_and_emit(keys, n, g.m, sh, idx + row * topk, g.D, topk, nullptr);
+}
+
+// ------------------------------------------------ per-token, one launch
+// grid (NCH, Tq, B*Hkv) with cluster (NCH, 1, 1); dynamic shared memory
+// (CH + NCH * kMaxChosen) * 8 bytes.  Row i = token i (qblk = 1).
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) select_token_kernel(
+    const __nv_bfloat16 *__restrict__ Q, const float *__restrict__ Kc, int32_t *__restrict__ idx,
+    int nblk_max, int Tq, int Hq, int Hkv, int q_pos0, int topk, float sm_scale, int CH)
+{
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    extern __shared__ uint64_t keys[];            // [CH] chunk keys, then [NCH * kMaxChosen] merged
+    __shared__ SelectShared sh;
+    __shared__ __align__(16) float qbar[D];
+    __shared__ uint64_t chosen[kMaxChosen];       // this chunk's top-m, ascending block order
+    const int NCH = (int)cluster.num_blocks();
+    const int chunk = (int)cluster.block_rank();
+    const int i = blockIdx.y, bg = blockIdx.z, NR = gridDim.y;
+    const int b = bg / Hkv, grp = bg % Hkv, G = Hq / Hkv;
+    const RowGeom g = row_geom(i, Tq, q_pos0, 1, topk, CH);
+    const long row = (long)bg * NR + i;
+    grid_dependency_wait();     // Q and Kc come from earlier work on the stream
+    grid_launch_dependents();   // the attention that reads idx may be scheduled
+
+    // pooled query: mean of the token's query over the group's heads
+    {
+        const __nv_bfloat16 *qt = Q + (((long)b * Tq + i) * Hq + (long)grp * G) * D;
+        const float inv = 1.0f / (float)G;
+        for (int c = threadIdx.x; c < D; c += kSelThreads) {
+            float s = 0.f;
+            for (int h = 0; h < G; h++) s += __bfloat162float(qt[(long)h * D + c]);
+            qbar[c] = s * inv;
+        }
+    }
+    __syncthreads();
+    const int j0 = 1 + chunk * CH;
+    const int n = max(0, min(CH, g.ncand - chunk * CH));
+    score_chunk<D>(qbar, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
+    __syncthreads();
+    const int need = min(g.m, n);
+    if (g.nchunks == 1) {
+        if (chunk == 0) select_and_emit(keys, n, need, sh, idx + row * topk, g.D, topk, nullptr);
+    } else {
+        select_and_emit(keys, n, need, sh, nullptr, g.D, topk, chosen);
+    }
+    cluster.sync();
+    if (g.nchunks > 1 && chunk == 0) {
+        // the chunks' lists are ascending and the chunks are in block order
+        uint64_t *merged = keys + CH;
+        int nt = 0;
+        for (int r = 0; r < g.nchunks; r++) {
+            const int nr = min(g.m, max(0, min(CH, g.ncand - r * CH)));
+            const uint64_t *src = cluster.map_shared_rank(chosen, r);
+            for (int e = threadIdx.x; e < nr; e += kSelThreads) merged[nt + e] = src[e];
+            nt += nr;
+        }
+        __syncthreads();
+        select_and_emit(merged, nt, g.m, sh, idx + row * topk, g.D, topk, nullptr);
+    }
+    cluster.sync();   // the chunks' lists must outlive the leader's reads
 }
 
 }  // namespace qsa

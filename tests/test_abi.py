@@ -34,6 +34,10 @@ def test_workspace_sizes_are_host_only():
     small = qsa.score_select_workspace(1, 16, 2, 4096, 0, 64, 128, 64)
     assert big > small > 0
     assert qsa.score_select_workspace(1, 16, 2, 4096, 0, 7, 128, 64) == 0   # bad qblk
+    # per-token selection (decode) is one launch whose chunks merge in distributed
+    # shared memory: no workspace up to 8 x 8192 candidates, the chunked path beyond
+    assert qsa.score_select_workspace(32, 16, 2, 1, 262143, 1, 128, 64) == 0
+    assert qsa.score_select_workspace(1, 16, 2, 1, 64 * 70000, 1, 128, 64) > 0
     # decode merges its split-K partials in distributed shared memory: no workspace
     assert qsa.decode_workspace(32, 16, 2, 128, 64) == 0
 

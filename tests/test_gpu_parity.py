@@ -155,6 +155,9 @@ SELECT_CASES = [
                                Hkv=2, d=128, topk=16)),
     ("decode_many_chunks", dict(B=1, Tq=1, T_kv=64 * 5000, q_pos0=64 * 5000 - 30, qblk=1,
                                 Hq=8, Hkv=2, d=64, topk=64)),
+    # per-token rows inside a prefill chunk (qblk = 1, Tq > 1): ragged diagonals
+    ("token_rows_prefill", dict(B=2, Tq=96, T_kv=640, q_pos0=544, qblk=1, Hq=8, Hkv=2, d=64,
+                                topk=6)),
 ]
 
 
@@ -173,6 +176,30 @@ def test_score_select_parity(qsa, name, kw):
     frac, jac = check_selection(idx.cpu().numpy().reshape(-1, w.topk), sel, sel["scores"],
                                 rows_diag(w), w.topk)
     print(f"{name}: rows gap-checked {frac:.3f}, mean Jaccard {jac:.4f}")
+
+
+def test_score_select_token_rows_past_the_cluster_limit(qsa):
+    """Per-token rows with more than 8 x 8192 candidates leave the one-launch
+    cluster path for the chunked path with a workspace; both must select the
+    same blocks as the oracle.  Random summaries stand in for compressed keys
+    (only the scoring and selection are under test)."""
+    nb = 66000
+    w = synthetic.custom(B=1, Tq=1, T_kv=64 * nb, q_pos0=64 * nb - 1, qblk=1, Hq=8, Hkv=2,
+                         d=64, topk=24, seed=33)
+    assert qsa.score_select_workspace(w.B, w.Hq, w.Hkv, 1, w.q_pos0, 1, w.d, w.topk) > 0
+    assert qsa.score_select_workspace(w.B, w.Hq, w.Hkv, 1, 64 * 5000, 1, w.d, w.topk) == 0
+    gen = torch.Generator().manual_seed(w.seed)
+    Q = torch.randn((w.B, 1, w.Hq, w.d), generator=gen).to(torch.bfloat16)
+    Kc = torch.randn((w.B, w.Hkv, nb, w.d), generator=gen) * 0.2
+    idx = torch.full((w.B, w.Hkv, 1, w.topk), -7, dtype=torch.int32, device=DEV)
+    qsa.score_select(Q.to(DEV), Kc.to(DEV), idx, w.topk, w.q_pos0, 1, w.sm_scale)
+    _status_ok(qsa)
+    Qbar = oracle.pool_queries(Q, w.Hkv, 1)
+    sel = oracle.select(Qbar, Kc.double(), 1, w.q_pos0, 1, w.topk, w.sm_scale,
+                        rows=np.arange(w.B * w.Hkv), want_scores=True)
+    frac, jac = check_selection(idx.cpu().numpy().reshape(-1, w.topk), sel, sel["scores"],
+                                rows_diag(w), w.topk)
+    print(f"66000 candidates: rows gap-checked {frac:.3f}, mean Jaccard {jac:.4f}")
 
 
 PREFILL_CASES = [
