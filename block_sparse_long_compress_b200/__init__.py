@@ -273,12 +273,11 @@ class QSADecode:
     def graph(self, q, K, V, L, parts=("select", "attention")):
         """Capture the step (or some of its parts) for these buffers and this
         cache length as a CUDA graph; ``replay()`` then reruns it on the
-        current stream with no host launch work.  Call the step eagerly once
-        first (it sizes the selection workspace)."""
+        current stream with no host launch work.  The step runs once eagerly
+        first (kernel loading, attributes and the selection workspace stay
+        out of the capture)."""
         q4 = q.view(self.B, 1, self.Hq, self.d)
-        if L not in self._sel_ws:
-            n = score_select_workspace(self.B, self.Hq, self.Hkv, 1, L - 1, 1, self.d, self.topk)
-            self._sel_ws[L] = torch.empty(max(1, n), dtype=torch.uint8, device=q.device)
+        self(q, K, V, L)
         side = torch.cuda.Stream(device=q.device)
         side.wait_stream(torch.cuda.current_stream())
         g = torch.cuda.CUDAGraph()

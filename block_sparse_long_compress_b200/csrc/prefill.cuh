@@ -281,10 +281,12 @@ __global__ void __launch_bounds__(11 * 32, 1) sparse_attn_prefill_kernel(
                         if (c > lim[hb]) sr[64 * hb + c] = 0xff800000u;   // -inf
                 }
             }
-            float q0 = __uint_as_float(sr[0]), q1 = __uint_as_float(sr[1]);
-            float q2 = __uint_as_float(sr[2]), q3 = __uint_as_float(sr[3]);
+            float q0 = fmaxf(__uint_as_float(sr[0]), __uint_as_float(sr[1]));
+            float q1 = fmaxf(__uint_as_float(sr[2]), __uint_as_float(sr[3]));
+            float q2 = fmaxf(__uint_as_float(sr[4]), __uint_as_float(sr[5]));
+            float q3 = fmaxf(__uint_as_float(sr[6]), __uint_as_float(sr[7]));
 #pragma unroll
-            for (int c = 4; c < 128; c += 8) {
+            for (int c = 8; c < 128; c += 8) {
                 q0 = max3f(q0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
                 q1 = max3f(q1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
                 q2 = max3f(q2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));

@@ -20,7 +20,7 @@ import torch
 
 import oracle
 import synthetic
-from tests.helpers import jaccard
+from tests.helpers import check_out, check_selection, jaccard, rows_diag
 
 pytestmark = pytest.mark.gpu
 
@@ -37,47 +37,6 @@ def qsa():
 def _status_ok(qsa):
     st, det = qsa.device_status()
     assert st == "QSA_OK", (st, det)
-
-
-# ----------------------------------------------------------------- checks
-def check_selection(idx_gpu, sel_ref, scores_ref, rows_D, topk, gap_tol=1e-3, valid_tol=1e-5):
-    """idx_gpu, sel_ref['idx']: [nrows, topk]; scores_ref: [nrows, NB]."""
-    idx_ref, gap = sel_ref["idx"], sel_ref["gap"]
-    n = len(idx_gpu)
-    exact = gap > gap_tol
-    assert np.array_equal(idx_gpu[exact], idx_ref[exact]), "indices differ on a clear-gap row"
-    jac = []
-    for r in range(n):
-        row = [int(j) for j in idx_gpu[r] if j >= 0]
-        D = rows_D[r]
-        assert row == sorted(set(row)) and row[0] == 0 and (D == 0 or row[-1] == D)
-        assert all(j == -1 for j in idx_gpu[r][len(row):])
-        assert len(row) == int(np.sum(idx_ref[r] >= 0))
-        chosen = [j for j in row if 0 < j < D]
-        cand = np.arange(1, D)
-        unchosen = np.setdiff1d(cand, chosen)
-        if chosen and len(unchosen):
-            s = scores_ref[r]
-            assert s[chosen].min() >= s[unchosen].max() - valid_tol, f"row {r}: not a valid top-m"
-        jac.append(jaccard(idx_gpu[r], idx_ref[r]))
-    return float(exact.mean()), float(np.mean(jac))
-
-
-def check_out(O_gpu, O_ref, max_tol=1e-2, mean_tol=1e-3):
-    err = np.abs(np.asarray(O_gpu, dtype=np.float64) - O_ref)
-    assert np.isfinite(err).all()
-    assert err.max() <= max_tol and err.mean() <= mean_tol, (err.max(), err.mean())
-    return err.max(), err.mean()
-
-
-def rows_diag(w):
-    NR = w.n_rows
-    D = []
-    for b in range(w.B):
-        for g in range(w.Hkv):
-            for i in range(NR):
-                D.append((w.q_pos0 + min((i + 1) * w.qblk, w.Tq) - 1) // 64)
-    return D
 
 
 def gpu_kc(qsa, K):
@@ -200,6 +159,23 @@ def test_score_select_token_rows_past_the_cluster_limit(qsa):
     frac, jac = check_selection(idx.cpu().numpy().reshape(-1, w.topk), sel, sel["scores"],
                                 rows_diag(w), w.topk)
     print(f"66000 candidates: rows gap-checked {frac:.3f}, mean Jaccard {jac:.4f}")
+
+
+@pytest.mark.parametrize("Hq,d", [(16, 128), (8, 128), (16, 64), (8, 64)])
+def test_prefill_single_key_row_returns_its_value(qsa, Hq, d):
+    """Token 0 of a fresh sequence sees only key 0: softmax weight 1, so
+    its output is V[0] of its group bit for bit, whatever the score's sign
+    (a row max taken over anything but the visible keys breaks this)."""
+    torch.manual_seed(Hq + d)
+    B, T, Hkv = 1, 256, 2
+    G = Hq // Hkv
+    Q = torch.randn(B, T, Hq, d, device=DEV).to(torch.bfloat16)
+    K = (torch.randn(B, Hkv, T, d, device=DEV) * 2).to(torch.bfloat16)
+    V = (torch.randn(B, Hkv, T, d, device=DEV) * 3).to(torch.bfloat16)
+    run = qsa.QSAPrefill(B, T, Hq, Hkv, d, T, 2, 0, device=DEV)
+    O = run(Q, K, V)
+    _status_ok(qsa)
+    assert torch.equal(O[0, 0], V[0, :, 0].repeat_interleave(G, 0))
 
 
 PREFILL_CASES = [
