@@ -262,6 +262,10 @@ def run_qsa(args, ws, rank, local):
         del Q, K, V, run, x
         torch.cuda.empty_cache()
         result["decode"] = bench_decode(args, qsa, dev, peaks, ws, rank, flush)
+        for name in filter(None, args.decode_more.split(",")):
+            torch.cuda.empty_cache()
+            result.setdefault("decode_more", {})[name] = bench_decode(args, qsa, dev, peaks, ws,
+                                                                      rank, flush, name)
 
     # ---- e2e through the public API with host buffers
     if not args.no_e2e:
@@ -269,8 +273,8 @@ def run_qsa(args, ws, rank, local):
     return result
 
 
-def bench_decode(args, qsa, dev, peaks, ws, rank, flush):
-    wd = synthetic.CONFIGS[args.decode_workload]
+def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None):
+    wd = synthetic.CONFIGS[workload or args.decode_workload]
     if args.decode_batch:
         wd = synthetic.Workload(**{**wd.__dict__, "B": args.decode_batch})
     if ws > 1:
@@ -284,30 +288,54 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush):
     for _ in range(args.warmup):
         dec(q, K, V, L)
     torch.cuda.synchronize()
-    n0 = qsa.launch_count()
-    graphs = {"step": dec.graph(q, K, V, L, parts=("select", "attention"))}
-    launches_step = qsa.launch_count() - n0   # kernels captured in the step's graph
-    graphs["select"] = dec.graph(q, K, V, L, parts=("select",))
-    graphs["attention"] = dec.graph(q, K, V, L, parts=("attention",))
     stream = torch.cuda.current_stream()
     steps = max(args.steps, 20)
+    sel_ws = dec._sel_ws[L]
+    q4 = q.view(wd.B, 1, wd.Hq, wd.d)
 
-    def timed(g):
+    def run_parts(parts, s):
+        if "select" in parts:
+            qsa.score_select(q4, dec.Kc, dec.idx, wd.topk, L - 1, 1, dec.sm_scale, sel_ws, s)
+        if "attention" in parts:
+            qsa.decode(q, K, V, dec.idx, dec.o, L, dec.sm_scale, dec.ws_dec, s)
+
+    def capture(parts):
+        """flush -> event -> the step's kernels -> event, as one CUDA graph:
+        the events sit inside the graph, so the launch of the graph itself
+        stays outside the measured interval."""
+        e0 = torch.cuda.Event(enable_timing=True, external=True)
+        e1 = torch.cuda.Event(enable_timing=True, external=True)
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        n0 = qsa.launch_count()
+        with torch.cuda.graph(g, stream=side):
+            flush(0)
+            e0.record(side)
+            run_parts(parts, side)
+            e1.record(side)
+        stream.wait_stream(side)
+        return g, e0, e1, qsa.launch_count() - n0
+
+    def timed(parts):
+        g, e0, e1, launches = capture(parts)
         for _ in range(args.warmup):
             g.replay()
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        torch.cuda.synchronize()
         if ws > 1:
             torch.distributed.barrier()
-        torch.cuda.synchronize()
-        for k in range(steps):
-            flush(k)
-            evs[k][0].record(stream)
+        out = []
+        for _ in range(steps):
             g.replay()
-            evs[k][1].record(stream)
-        torch.cuda.synchronize()
-        return np.array([e[0].elapsed_time(e[1]) for e in evs]) * 1e3   # us
+            torch.cuda.synchronize()
+            out.append(e0.elapsed_time(e1) * 1e3)   # us
+        return np.array(out), launches
 
-    t = {part: timed(g) for part, g in graphs.items()}
+    t = {}
+    t["step"], launches_step = timed(("select", "attention"))
+    t["select"], _ = timed(("select",))
+    t["attention"], _ = timed(("attention",))
+
     st, det = qsa.device_status()
     if st != "QSA_OK":
         raise RuntimeError(f"decode device status {st} ({det})")
@@ -319,7 +347,7 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush):
     sel_bytes = wd.B * wd.Hkv * ((L - 1) // 64) * wd.d * 4   # fp32 summaries read by scoring
     return {"workload": wd.name, "batch": wd.B, "context": L, "topk": wd.topk,
             "us_per_step": us_step, "us_per_token": us_step / wd.B,
-            "timing": "CUDA graph of the step replayed; events around each replay",
+            "timing": "CUDA graph (L2 flush, event, step kernels, event) replayed per step",
             "breakdown_us": {"score_select": us_sel, "attention": us_att},
             "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": att_gbs,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -443,6 +471,8 @@ def main():
     ap.add_argument("--impl", default="qsa", choices=["qsa", "reference"])
     ap.add_argument("--workload", default=PREFILL, choices=sorted(synthetic.CONFIGS))
     ap.add_argument("--decode-workload", default=DECODE, choices=sorted(synthetic.CONFIGS))
+    ap.add_argument("--decode-more", default="decode_262k",
+                    help="comma list of further decode workloads reported under decode_more")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--only-decode", action="store_true",
                     help="skip the prefill measurement (profiling the decode kernels)")
@@ -476,6 +506,10 @@ def main():
         torch.cuda.set_device(dev)
         flush = L2Flush(dev)
         res = bench_decode(args, qsa, dev, load_peaks(), ws, rank, flush)
+        for name in filter(None, args.decode_more.split(",")):
+            torch.cuda.empty_cache()
+            res.setdefault("decode_more", {})[name] = bench_decode(args, qsa, dev, load_peaks(), ws,
+                                                                   rank, flush, name)
         if rank == 0:
             print(json.dumps(res), flush=True)
         return
