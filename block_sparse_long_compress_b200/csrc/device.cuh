@@ -54,6 +54,19 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ------------------------------------------------- split cluster barrier
+// Every thread of every CTA in the cluster arrives once, then waits once,
+// before the next barrier of the cluster.
+__device__ __forceinline__ void cluster_arrive_release()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait_acquire()
+{
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // ---------------------------------------------- programmatic dependent launch
 // A kernel launched with programmatic stream serialization may start while
 // the previous kernel on the stream is still running.  It must not touch

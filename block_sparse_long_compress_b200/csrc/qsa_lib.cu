@@ -266,7 +266,7 @@ qsa_status launch_select_token_d(const void *Q, const float *Kc, int32_t *idx, i
                                  cudaStream_t s)
 {
     auto kern = qsa::select_token_kernel<D>;
-    const int smem = (tp.CH + tp.NCH * qsa::kMaxChosen) * 8;
+    const int smem = tp.CH * 8;
     qsa_status st;
     if ((st = set_smem(kern, smem)) != QSA_OK) return st;
     cudaLaunchConfig_t cfg = {};

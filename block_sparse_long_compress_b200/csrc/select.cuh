@@ -19,10 +19,10 @@
 //   select_token_kernel  per-token rows (qblk = 1, e.g. decode) in one
 //                        launch: the chunks of a row form a thread-block
 //                        cluster; every CTA pools its token's query over the
-//                        group's heads, scores its chunk and selects the
-//                        chunk's top-m into shared memory; the leader merges
-//                        the chunks' lists through distributed shared memory
-//                        and writes the row.  No workspace.
+//                        group's heads and scores its chunk; one radix select
+//                        runs across the cluster (digit counts summed through
+//                        distributed shared memory) and every CTA writes its
+//                        chosen blocks.  No workspace.
 // Key of candidate j with score s: (order-preserving bits of s) << 32 |
 // (0xFFFFFFFF - j); keys are unique, larger = better, and the lower block
 // wins a score tie.  -0.0 is folded into +0.0.
@@ -111,51 +111,69 @@ struct SelectShared {
     int digit, above, bucket;
 };
 
+// Adds 1 to hist[digit] for every lane with active set; lanes of a warp
+// that share a digit are combined into one atomic (keys of a row often
+// share their top digits, which would serialise plain atomics).
+__device__ __forceinline__ void hist_add(int *hist, bool active, int digit)
+{
+    const unsigned act = __ballot_sync(0xffffffffu, active);
+    if (!active) return;
+    const unsigned same = __match_any_sync(act, digit);
+    if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&hist[digit], __popc(same));
+}
+
+// Warp 0: the digit whose bucket holds the need-th largest key of
+// sh.hist (counts by digit), the count above it and the bucket's size.
+__device__ __forceinline__ void find_digit(SelectShared &sh, int need)
+{
+    const int lane = threadIdx.x & 31;
+    // lane l owns bins 255-8l .. 248-8l (descending)
+    int c[8], tot = 0;
+#pragma unroll
+    for (int q = 0; q < 8; q++) {
+        c[q] = sh.hist[255 - 8 * lane - q];
+        tot += c[q];
+    }
+    int incl = tot;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    const int excl = incl - tot;
+    if (excl < need && need <= incl) {
+        int cum = excl;
+#pragma unroll
+        for (int q = 0; q < 8; q++) {
+            if (cum + c[q] >= need) {
+                sh.digit = 255 - 8 * lane - q;
+                sh.above = cum;
+                sh.bucket = c[q];
+                break;
+            }
+            cum += c[q];
+        }
+    }
+}
+
 // Radix select over n unique keys in shared memory: returns (prefix, mask)
 // such that exactly `need` keys satisfy (key & mask) >= prefix.
 // Requires 0 < need < n.  All threads of the CTA must call it.
 __device__ void radix_select(const uint64_t *keys, int n, int need, SelectShared &sh,
                              uint64_t &prefix_out, uint64_t &mask_out)
 {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5;
     uint64_t prefix = 0, mask = 0;
     for (int shift = 56; shift >= 0; shift -= 8) {
         for (int b = tid; b < 256; b += kSelThreads) sh.hist[b] = 0;
         __syncthreads();
-        for (int e = tid; e < n; e += kSelThreads) {
-            const uint64_t k = keys[e];
-            if ((k & mask) == prefix) atomicAdd(&sh.hist[(int)((k >> shift) & 0xFF)], 1);
+        for (int base = 0; base < n; base += kSelThreads) {
+            const int e = base + tid;
+            const uint64_t k = e < n ? keys[e] : 0;
+            hist_add(sh.hist, e < n && (k & mask) == prefix, (int)((k >> shift) & 0xFF));
         }
         __syncthreads();
-        if (warp == 0) {
-            // lane l owns bins 255-8l .. 248-8l (descending)
-            int c[8], tot = 0;
-#pragma unroll
-            for (int q = 0; q < 8; q++) {
-                c[q] = sh.hist[255 - 8 * lane - q];
-                tot += c[q];
-            }
-            int incl = tot;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += v;
-            }
-            const int excl = incl - tot;
-            if (excl < need && need <= incl) {
-                int cum = excl;
-#pragma unroll
-                for (int q = 0; q < 8; q++) {
-                    if (cum + c[q] >= need) {
-                        sh.digit = 255 - 8 * lane - q;
-                        sh.above = cum;
-                        sh.bucket = c[q];
-                        break;
-                    }
-                    cum += c[q];
-                }
-            }
-        }
+        if (warp == 0) find_digit(sh, need);
         __syncthreads();
         need -= sh.above;
         prefix |= (uint64_t)sh.digit << shift;
@@ -357,7 +375,15 @@ __global__ void __launch_bounds__(kSelThreads) merge_select_kernel(
 
 // ------------------------------------------------ per-token, one launch
 // grid (NCH, Tq, B*Hkv) with cluster (NCH, 1, 1); dynamic shared memory
-// (CH + NCH * kMaxChosen) * 8 bytes.  Row i = token i (qblk = 1).
+// CH * 8 bytes.  Row i = token i (qblk = 1).  The row's top-m is one exact
+// radix select over all chunks of the cluster: every pass, each CTA counts
+// its own keys by digit, the counts are summed through distributed shared
+// memory and every CTA takes the same digit; then each CTA writes its
+// chosen blocks at its cluster prefix offset, which keeps the row in block
+// order.  Each CTA adds its own digit counts into the leader's row_hist
+// (distributed-shared-memory atomics, fire and forget); the totals are
+// triple-buffered so every pass needs one cluster barrier: the total a
+// pass fills was last read two passes ago and is zeroed one pass ahead.
 template <int D>
 __global__ void __launch_bounds__(kSelThreads) select_token_kernel(
     const __nv_bfloat16 *__restrict__ Q, const float *__restrict__ Kc, int32_t *__restrict__ idx,
@@ -365,24 +391,32 @@ __global__ void __launch_bounds__(kSelThreads) select_token_kernel(
 {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
-    extern __shared__ uint64_t keys[];            // [CH] chunk keys, then [NCH * kMaxChosen] merged
+    extern __shared__ uint64_t keys[];            // [CH] this chunk's keys
     __shared__ SelectShared sh;
+    __shared__ int chist[256];                    // this chunk's digit counts
+    __shared__ int row_hist[3][256];              // the row's digit counts (leader CTA)
+    __shared__ int nchosen;                       // this chunk's chosen count, read by the cluster
     __shared__ __align__(16) float qbar[D];
-    __shared__ uint64_t chosen[kMaxChosen];       // this chunk's top-m, ascending block order
     const int NCH = (int)cluster.num_blocks();
     const int chunk = (int)cluster.block_rank();
+    const int tid = threadIdx.x, warp = tid >> 5;
     const int i = blockIdx.y, bg = blockIdx.z, NR = gridDim.y;
     const int b = bg / Hkv, grp = bg % Hkv, G = Hq / Hkv;
     const RowGeom g = row_geom(i, Tq, q_pos0, 1, topk, CH);
     const long row = (long)bg * NR + i;
     grid_dependency_wait();     // Q and Kc come from earlier work on the stream
     grid_launch_dependents();   // the attention that reads idx may be scheduled
+    if (chunk == 0)
+        for (int d = tid; d < 256; d += kSelThreads) row_hist[0][d] = 0;
+    // publishes the zeroed total; waited for after the scoring, so the
+    // barrier costs nothing
+    cluster_arrive_release();
 
     // pooled query: mean of the token's query over the group's heads
     {
         const __nv_bfloat16 *qt = Q + (((long)b * Tq + i) * Hq + (long)grp * G) * D;
         const float inv = 1.0f / (float)G;
-        for (int c = threadIdx.x; c < D; c += kSelThreads) {
+        for (int c = tid; c < D; c += kSelThreads) {
             float s = 0.f;
             for (int h = 0; h < G; h++) s += __bfloat162float(qt[(long)h * D + c]);
             qbar[c] = s * inv;
@@ -393,27 +427,69 @@ __global__ void __launch_bounds__(kSelThreads) select_token_kernel(
     const int n = max(0, min(CH, g.ncand - chunk * CH));
     score_chunk<D>(qbar, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
     __syncthreads();
-    const int need = min(g.m, n);
-    if (g.nchunks == 1) {
-        if (chunk == 0) select_and_emit(keys, n, need, sh, idx + row * topk, g.D, topk, nullptr);
-    } else {
-        select_and_emit(keys, n, need, sh, nullptr, g.D, topk, chosen);
-    }
-    cluster.sync();
-    if (g.nchunks > 1 && chunk == 0) {
-        // the chunks' lists are ascending and the chunks are in block order
-        uint64_t *merged = keys + CH;
-        int nt = 0;
-        for (int r = 0; r < g.nchunks; r++) {
-            const int nr = min(g.m, max(0, min(CH, g.ncand - r * CH)));
-            const uint64_t *src = cluster.map_shared_rank(chosen, r);
-            for (int e = threadIdx.x; e < nr; e += kSelThreads) merged[nt + e] = src[e];
-            nt += nr;
+
+    // ---- exact top-m of the row over the cluster's chunks
+    const bool all = g.m >= g.ncand;   // every candidate chosen (or none exist)
+    const bool any = g.m > 0;          // topk = 2 with a diagonal leaves no room
+    uint64_t prefix = 0, mask = 0;
+    cluster_wait_acquire();
+    if (!all && any) {
+        int need = g.m, pass = 0;
+        for (int shift = 56; shift >= 0; shift -= 8, pass++) {
+            const int cur = pass % 3;
+            int *lead = cluster.map_shared_rank(&row_hist[cur][0], 0);
+            for (int d = tid; d < 256; d += kSelThreads) chist[d] = 0;
+            if (chunk == 0)
+                for (int d = tid; d < 256; d += kSelThreads) row_hist[(pass + 1) % 3][d] = 0;
+            __syncthreads();
+            for (int base = 0; base < n; base += kSelThreads) {
+                const int e = base + tid;
+                const uint64_t k = e < n ? keys[e] : 0;
+                hist_add(chist, e < n && (k & mask) == prefix, (int)((k >> shift) & 0xFF));
+            }
+            __syncthreads();
+            for (int d = tid; d < 256; d += kSelThreads)
+                if (chist[d]) atomicAdd(lead + d, chist[d]);
+            cluster.sync();
+            for (int d = tid; d < 256; d += kSelThreads) sh.hist[d] = lead[d];
+            __syncthreads();
+            if (warp == 0) find_digit(sh, need);
+            __syncthreads();
+            need -= sh.above;
+            prefix |= (uint64_t)sh.digit << shift;
+            mask |= (uint64_t)0xFF << shift;
+            const bool done = (sh.bucket == need);   // the same in every CTA
+            __syncthreads();   // sh read everywhere before the next pass writes it
+            if (done) break;
         }
-        __syncthreads();
-        select_and_emit(merged, nt, g.m, sh, idx + row * topk, g.D, topk, nullptr);
     }
-    cluster.sync();   // the chunks' lists must outlive the leader's reads
+    // ---- this chunk's chosen blocks, in block order, at the cluster offset
+    const int per = (n + kSelThreads - 1) / kSelThreads;
+    const int e0 = min(tid * per, n), e1 = min(e0 + per, n);
+    int cnt = 0;
+    for (int e = e0; e < e1; e++) cnt += (all || (any && (keys[e] & mask) >= prefix)) ? 1 : 0;
+    int total;
+    int pos = block_exclusive_scan(cnt, sh, total);
+    if (tid == 0) nchosen = total;
+    cluster.sync();
+    int off = 0;
+#pragma unroll
+    for (int r = 0; r < 8; r++)
+        if (r < chunk) off += *cluster.map_shared_rank(&nchosen, r);
+    int32_t *out = idx + row * topk;
+    for (int e = e0; e < e1; e++) {
+        const uint64_t k = keys[e];
+        if (all || (any && (k & mask) >= prefix)) out[1 + off + pos++] = key_block(k);
+    }
+    if (chunk == 0) {
+        // forced entries: the sink first, the diagonal after the chosen, -1 padding
+        for (int s = tid; s < topk; s += kSelThreads) {
+            if (s == 0) out[0] = 0;
+            else if (s == g.m + 1 && g.D > 0) out[s] = g.D;
+            else if (s > g.m + (g.D > 0 ? 1 : 0)) out[s] = -1;
+        }
+    }
+    cluster.sync();   // the chunks' counts must outlive the other CTAs' reads
 }
 
 }  // namespace qsa

@@ -117,6 +117,11 @@ SELECT_CASES = [
     # per-token rows inside a prefill chunk (qblk = 1, Tq > 1): ragged diagonals
     ("token_rows_prefill", dict(B=2, Tq=96, T_kv=640, q_pos0=544, qblk=1, Hq=8, Hkv=2, d=64,
                                 topk=6)),
+    # top-2 leaves only the forced blocks; top-3 chooses one over several chunks
+    ("decode_top2", dict(B=3, Tq=1, T_kv=64 * 900, q_pos0=64 * 900 - 7, qblk=1, Hq=16, Hkv=2,
+                         d=128, topk=2)),
+    ("decode_top3", dict(B=3, Tq=1, T_kv=64 * 900, q_pos0=64 * 900 - 7, qblk=1, Hq=16, Hkv=2,
+                         d=128, topk=3)),
 ]
 
 
