@@ -6,6 +6,7 @@ runtime's driver entry-point query, so the library needs no libcuda at
 link time and loads on a machine without a GPU.
 """
 import os
+import re
 import subprocess
 import sys
 
@@ -31,6 +32,29 @@ def _sources():
     return out
 
 
+# The prefill kernel moves registers between its warpgroups (setmaxnreg):
+# its split is sized for this many registers per thread at launch (the
+# launch bounds' ceiling for 384 threads).  A kernel launched with fewer
+# would wait forever in setmaxnreg.inc, so the build refuses it.
+PREFILL_LAUNCH_REGS = 168
+
+
+def _check_registers(ptxas_log: str) -> None:
+    entry = None
+    for line in ptxas_log.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            entry = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and entry and "sparse_attn_prefill_kernel" in entry:
+            if int(m.group(1)) != PREFILL_LAUNCH_REGS:
+                raise RuntimeError(
+                    f"{entry} launches with {m.group(1)} registers per thread; its setmaxnreg "
+                    f"split assumes {PREFILL_LAUNCH_REGS}")
+            entry = None
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     """Build libqsa.so if missing or older than any source; return its path."""
     if not force and os.path.exists(LIB):
@@ -41,10 +65,17 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not os.path.exists(nvcc) and os.path.exists("/usr/local/cuda/bin/nvcc"):
         nvcc = "/usr/local/cuda/bin/nvcc"
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, "-o", tmp, MAIN]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
+    cmd = [nvcc, "-Xptxas=-v", *NVCC_FLAGS, "-o", tmp, MAIN]
+    r = subprocess.run(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)
+    if verbose or r.returncode != 0:
+        sys.stdout.write(r.stdout)
+    if r.returncode != 0:
+        raise subprocess.CalledProcessError(r.returncode, cmd)
+    try:
+        _check_registers(r.stdout)
+    except RuntimeError:
+        os.remove(tmp)
+        raise
     os.replace(tmp, LIB)
     return LIB
 

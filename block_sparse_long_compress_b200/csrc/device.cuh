@@ -54,6 +54,22 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ------------------------------------------------- register redistribution
+// Every warp of a warpgroup executes the same one; an increase waits until
+// the warpgroups that decrease have released enough of the CTA's launch
+// registers, so the kernel's split must fit its launch allocation.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------- split cluster barrier
 // Every thread of every CTA in the cluster arrives once, then waits once,
 // before the next barrier of the cluster.

@@ -32,10 +32,12 @@
 // before S_t(n+1) overwrites it.  The running max only moves (and O_t is
 // rescaled in TMEM) when a pair's max exceeds it by more than 2^8.
 //
-// Warps (352 threads): 0-7 softmax/epilogue (tile = warp/4, TMEM lane
-// quarter = warp%4, thread = row), 8 TMA producer, 9 TMEM allocator + MMA
-// issuer of tile 0, 10 MMA issuer of tile 1.  Each softmax warp signals P
-// with a single arrive.
+// Warps (384 threads, three warpgroups): 0-7 softmax/epilogue (tile =
+// warp/4, TMEM lane quarter = warp%4, thread = row; a row's 128 scores stay
+// in registers from the max to the exponentials), 8 TMA producer, 9 TMEM
+// allocator + MMA issuer of tile 0, 10 MMA issuer of tile 1, 11 idle.  The
+// last warpgroup gives registers to the softmax warpgroups (setmaxnreg).
+// Each softmax warp signals P with a single arrive.
 // TMEM (512 columns): O_0 [0,128) O_1 [128,256) S_0 [256,384) S_1 [384,512);
 // P_t in S_t columns [0,64).  Every mbarrier wait is bounded.
 #pragma once
@@ -57,7 +59,16 @@ struct PrefillCfg {
     // the CTA owns all 512 TMEM columns: ask for enough shared memory that
     // a second CTA never lands on the same SM
     static constexpr int SMEM_REQUEST = (SMEM_DATA + 1024 > 120 * 1024) ? SMEM_DATA + 1024 : 120 * 1024;
-    static constexpr int THREADS = 11 * 32;
+    static constexpr int THREADS = 12 * 32;
+    // registers: launched at REG_LAUNCH per thread (the launch bounds'
+    // ceiling for 384 threads, checked by the build); the producer/issuer
+    // warpgroup drops to REG_LOW and the two softmax warpgroups, which hold
+    // a row's 128 scores, rise to REG_HIGH: 256 * REG_HIGH + 128 * REG_LOW
+    // must not exceed 384 * REG_LAUNCH
+    static constexpr int REG_LAUNCH = 168;
+    static constexpr int REG_LOW = 48;
+    static constexpr int REG_HIGH = 224;
+    static_assert(256 * REG_HIGH + 128 * REG_LOW <= 384 * REG_LAUNCH, "register split exceeds the launch pool");
     static constexpr int TMEM_COLS = 512;
     static constexpr int O_COL = 0, S_COL = 256;
 };
@@ -77,7 +88,7 @@ struct PrefillShared {
 };
 
 template <int D, int G>
-__global__ void __launch_bounds__(11 * 32, 1) sparse_attn_prefill_kernel(
+__global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ idx,
     __nv_bfloat16 *__restrict__ O, float *__restrict__ lse, int Tq, int Hq, int Hkv,
@@ -149,6 +160,9 @@ __global__ void __launch_bounds__(11 * 32, 1) sparse_attn_prefill_kernel(
     const int npair = (nblk + 1) / 2;
     volatile int *abort = &sh.abort;
 
+    if (warp >= 8) {
+    // warpgroup 2 (one setmaxnreg for its four warps): producer, issuers
+    setmaxnreg_dec<C::REG_LOW>();
     if (warp == 8) {
         // ------------------------------------------------ TMA producer
         if (lane == 0 && nblk > 0) {
@@ -236,8 +250,10 @@ __global__ void __launch_bounds__(11 * 32, 1) sparse_attn_prefill_kernel(
                 if (more) issue_s(n + 1);
             }
         }
+    }
     } else {
         // -------------------------------- softmax + epilogue (warps 0-7)
+        setmaxnreg_inc<C::REG_HIGH>();
         const int t = warp >> 2;
         const int r = ((warp & 3) << 5) | lane;              // row = TMEM lane
         const int tok = token0 + t * C::TOK + r / G;
@@ -318,23 +334,13 @@ __global__ void __launch_bounds__(11 * 32, 1) sparse_attn_prefill_kernel(
             // MUFU; S is re-read from TMEM in 32-column chunks, one chunk ahead
             const uint64_t nm2 = f2_pack(-m_run, -m_run);
             uint64_t lacc = f2_pack(0.f, 0.f);
-            uint32_t cur[32], nxt[32];
-            tmem_ld32(s_addr, cur);
 #pragma unroll
             for (int c0 = 0; c0 < 128; c0 += 32) {
-                tmem_wait_ld();
-                if (c0 + 32 < 128) tmem_ld32(s_addr + c0 + 32, nxt);
-                const int lm = lim[c0 >> 6];
-                if (lm < 63) {
-#pragma unroll
-                    for (int c = 0; c < 32; c++)
-                        if ((c0 & 63) + c > lm) cur[c] = 0xff800000u;   // -inf
-                }
                 uint32_t pk[16];
 #pragma unroll
                 for (int c = 0; c < 16; c++) {
                     const uint64_t x2 = f2_fma(
-                        f2_pack(__uint_as_float(cur[2 * c]), __uint_as_float(cur[2 * c + 1])), sc2, nm2);
+                        f2_pack(__uint_as_float(sr[c0 + 2 * c]), __uint_as_float(sr[c0 + 2 * c + 1])), sc2, nm2);
                     float p0, p1;
                     if ((c & 3) == 3) {
                         f2_unpack(exp2_poly_x2(x2), p0, p1);
@@ -347,12 +353,8 @@ __global__ void __launch_bounds__(11 * 32, 1) sparse_attn_prefill_kernel(
                     lacc = f2_add(lacc, f2_pack(p0, p1));
                     pk[c] = pack_bf16x2(p0, p1);
                 }
-                // P over S columns [c0/2, c0/2 + 16), all already read
+                // P over S columns [c0/2, c0/2 + 16): S is held in registers
                 tmem_st16(s_addr + c0 / 2, pk);
-                if (c0 + 32 < 128) {
-#pragma unroll
-                    for (int c = 0; c < 32; c++) cur[c] = nxt[c];
-                }
             }
             float la, lb;
             f2_unpack(lacc, la, lb);

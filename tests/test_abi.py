@@ -96,3 +96,22 @@ def test_product_path_has_no_oracle_dependency():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(root, f)).read()
                 assert "oracle" not in text.lower(), f
+
+
+def test_build_refuses_a_prefill_kernel_below_its_register_split():
+    """The prefill kernel's setmaxnreg split assumes its launch register
+    count; the build checks the compiler's report and refuses anything else."""
+    import importlib.util
+    import os
+    spec = importlib.util.spec_from_file_location(
+        "qsa_build", os.path.join(os.path.dirname(__file__), "..", "block_sparse_long_compress_b200",
+                                  "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
+    ok = ("ptxas info    : Compiling entry function '_ZN3qsa26sparse_attn_prefill_kernelILi128ELi8EE'\n"
+          f"ptxas info    : Used {build.PREFILL_LAUNCH_REGS} registers, used 1 barriers\n"
+          "ptxas info    : Compiling entry function '_ZN3qsa13decode_kernelILi128ELi8EE'\n"
+          "ptxas info    : Used 107 registers\n")
+    build._check_registers(ok)
+    with pytest.raises(RuntimeError):
+        build._check_registers(ok.replace(f"Used {build.PREFILL_LAUNCH_REGS}", "Used 160"))
