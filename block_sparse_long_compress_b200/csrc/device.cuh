@@ -437,8 +437,11 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2)
     float t0, t1, p0, p1;
     f2_unpack(t, t0, t1);
     f2_unpack(p, p0, p1);
-    return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
-                   __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+    // p * 2^n: n's low bits sit in t's mantissa; one multiply-add per value
+    // moves them into the exponent field (the wrap-around of the product
+    // is the intended modular arithmetic)
+    return f2_pack(__uint_as_float(__float_as_uint(t0) * 8388608u + __float_as_uint(p0)),
+                   __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(p1)));
 }
 
 }  // namespace qsa

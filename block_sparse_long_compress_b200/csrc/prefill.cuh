@@ -297,18 +297,20 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
                         if (c > lim[hb]) sr[64 * hb + c] = 0xff800000u;   // -inf
                 }
             }
-            float q0 = fmaxf(__uint_as_float(sr[0]), __uint_as_float(sr[1]));
-            float q1 = fmaxf(__uint_as_float(sr[2]), __uint_as_float(sr[3]));
-            float q2 = fmaxf(__uint_as_float(sr[4]), __uint_as_float(sr[5]));
-            float q3 = fmaxf(__uint_as_float(sr[6]), __uint_as_float(sr[7]));
+            // 16 independent chains of 3-input maxima (the instruction's
+            // latency, not its count, sets the time), then a short tree
+            float qm[16];
 #pragma unroll
-            for (int c = 8; c < 128; c += 8) {
-                q0 = max3f(q0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-                q1 = max3f(q1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
-                q2 = max3f(q2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
-                q3 = max3f(q3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+            for (int k = 0; k < 16; k++) qm[k] = fmaxf(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1]));
+#pragma unroll
+            for (int c = 32; c < 128; c += 32) {
+#pragma unroll
+                for (int k = 0; k < 16; k++)
+                    qm[k] = max3f(qm[k], __uint_as_float(sr[c + 2 * k]), __uint_as_float(sr[c + 2 * k + 1]));
             }
-            const float mx = fmaxf(max3f(q0, q1, q2), q3) * sm_scale_log2;
+#pragma unroll
+            for (int k = 0; k < 5; k++) qm[k] = max3f(qm[3 * k], qm[3 * k + 1], qm[3 * k + 2]);
+            const float mx = fmaxf(max3f(qm[0], qm[1], qm[2]), max3f(qm[3], qm[4], qm[15])) * sm_scale_log2;
             if (n == 0) {
                 m_run = mx;
             } else if (__any_sync(0xffffffffu, mx > m_run + 8.0f)) {
@@ -333,7 +335,7 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
             // P = 2^(s*c - m), 1 of every 4 pairs on the FMA pipe, the rest on
             // MUFU; S is re-read from TMEM in 32-column chunks, one chunk ahead
             const uint64_t nm2 = f2_pack(-m_run, -m_run);
-            uint64_t lacc = f2_pack(0.f, 0.f);
+            uint64_t lacc[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
             for (int c0 = 0; c0 < 128; c0 += 32) {
                 uint32_t pk[16];
@@ -350,14 +352,14 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
                         p0 = fast_exp2(x0);
                         p1 = fast_exp2(x1);
                     }
-                    lacc = f2_add(lacc, f2_pack(p0, p1));
+                    lacc[c & 3] = f2_add(lacc[c & 3], f2_pack(p0, p1));
                     pk[c] = pack_bf16x2(p0, p1);
                 }
                 // P over S columns [c0/2, c0/2 + 16): S is held in registers
                 tmem_st16(s_addr + c0 / 2, pk);
             }
             float la, lb;
-            f2_unpack(lacc, la, lb);
+            f2_unpack(f2_add(f2_add(lacc[0], lacc[1]), f2_add(lacc[2], lacc[3])), la, lb);
             l += la + lb;
             tmem_wait_st();
             tc_fence_before();
