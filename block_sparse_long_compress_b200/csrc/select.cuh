@@ -19,10 +19,9 @@
 //   select_token_kernel  per-token rows (qblk = 1, e.g. decode) in one
 //                        launch: the chunks of a row form a thread-block
 //                        cluster; every CTA pools its token's query over the
-//                        group's heads and scores its chunk; one radix select
-//                        runs across the cluster (digit counts summed through
-//                        distributed shared memory) and every CTA writes its
-//                        chosen blocks.  No workspace.
+//                        group's heads, scores its chunk and pushes the
+//                        chunk's top-m into the leader's shared memory; the
+//                        leader selects the row.  No workspace.
 // Key of candidate j with score s: (order-preserving bits of s) << 32 |
 // (0xFFFFFFFF - j); keys are unique, larger = better, and the lower block
 // wins a score tie.  -0.0 is folded into +0.0.
@@ -375,15 +374,13 @@ __global__ void __launch_bounds__(kSelThreads) merge_select_kernel(
 
 // ------------------------------------------------ per-token, one launch
 // grid (NCH, Tq, B*Hkv) with cluster (NCH, 1, 1); dynamic shared memory
-// CH * 8 bytes.  Row i = token i (qblk = 1).  The row's top-m is one exact
-// radix select over all chunks of the cluster: every pass, each CTA counts
-// its own keys by digit, the counts are summed through distributed shared
-// memory and every CTA takes the same digit; then each CTA writes its
-// chosen blocks at its cluster prefix offset, which keeps the row in block
-// order.  Each CTA adds its own digit counts into the leader's row_hist
-// (distributed-shared-memory atomics, fire and forget); the totals are
-// triple-buffered so every pass needs one cluster barrier: the total a
-// pass fills was last read two passes ago and is zeroed one pass ahead.
+// CH * 8 bytes.  Row i = token i (qblk = 1).  Every CTA pools its token's
+// query over the group's heads, scores its chunk of summaries and selects
+// the chunk's top-m; it stores that list straight into the leader's shared
+// memory (distributed-shared-memory stores, padded with key 0, which is
+// below every score's key).  After one cluster barrier the other CTAs are
+// done and the leader selects the row's top-m from the lists, which are in
+// block order.
 template <int D>
 __global__ void __launch_bounds__(kSelThreads) select_token_kernel(
     const __nv_bfloat16 *__restrict__ Q, const float *__restrict__ Kc, int32_t *__restrict__ idx,
@@ -391,26 +388,19 @@ __global__ void __launch_bounds__(kSelThreads) select_token_kernel(
 {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
-    extern __shared__ uint64_t keys[];            // [CH] this chunk's keys
+    extern __shared__ uint64_t keys[];                 // [CH] this chunk's keys
     __shared__ SelectShared sh;
-    __shared__ int chist[256];                    // this chunk's digit counts
-    __shared__ int row_hist[3][256];              // the row's digit counts (leader CTA)
-    __shared__ int nchosen;                       // this chunk's chosen count, read by the cluster
+    __shared__ uint64_t lists[8 * kMaxChosen];         // leader: the chunks' top-m lists
     __shared__ __align__(16) float qbar[D];
     const int NCH = (int)cluster.num_blocks();
     const int chunk = (int)cluster.block_rank();
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x;
     const int i = blockIdx.y, bg = blockIdx.z, NR = gridDim.y;
     const int b = bg / Hkv, grp = bg % Hkv, G = Hq / Hkv;
     const RowGeom g = row_geom(i, Tq, q_pos0, 1, topk, CH);
     const long row = (long)bg * NR + i;
     grid_dependency_wait();     // Q and Kc come from earlier work on the stream
     grid_launch_dependents();   // the attention that reads idx may be scheduled
-    if (chunk == 0)
-        for (int d = tid; d < 256; d += kSelThreads) row_hist[0][d] = 0;
-    // publishes the zeroed total; waited for after the scoring, so the
-    // barrier costs nothing
-    cluster_arrive_release();
 
     // pooled query: mean of the token's query over the group's heads
     {
@@ -427,69 +417,18 @@ __global__ void __launch_bounds__(kSelThreads) select_token_kernel(
     const int n = max(0, min(CH, g.ncand - chunk * CH));
     score_chunk<D>(qbar, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
     __syncthreads();
-
-    // ---- exact top-m of the row over the cluster's chunks
-    const bool all = g.m >= g.ncand;   // every candidate chosen (or none exist)
-    const bool any = g.m > 0;          // topk = 2 with a diagonal leaves no room
-    uint64_t prefix = 0, mask = 0;
-    cluster_wait_acquire();
-    if (!all && any) {
-        int need = g.m, pass = 0;
-        for (int shift = 56; shift >= 0; shift -= 8, pass++) {
-            const int cur = pass % 3;
-            int *lead = cluster.map_shared_rank(&row_hist[cur][0], 0);
-            for (int d = tid; d < 256; d += kSelThreads) chist[d] = 0;
-            if (chunk == 0)
-                for (int d = tid; d < 256; d += kSelThreads) row_hist[(pass + 1) % 3][d] = 0;
-            __syncthreads();
-            for (int base = 0; base < n; base += kSelThreads) {
-                const int e = base + tid;
-                const uint64_t k = e < n ? keys[e] : 0;
-                hist_add(chist, e < n && (k & mask) == prefix, (int)((k >> shift) & 0xFF));
-            }
-            __syncthreads();
-            for (int d = tid; d < 256; d += kSelThreads)
-                if (chist[d]) atomicAdd(lead + d, chist[d]);
-            cluster.sync();
-            for (int d = tid; d < 256; d += kSelThreads) sh.hist[d] = lead[d];
-            __syncthreads();
-            if (warp == 0) find_digit(sh, need);
-            __syncthreads();
-            need -= sh.above;
-            prefix |= (uint64_t)sh.digit << shift;
-            mask |= (uint64_t)0xFF << shift;
-            const bool done = (sh.bucket == need);   // the same in every CTA
-            __syncthreads();   // sh read everywhere before the next pass writes it
-            if (done) break;
-        }
+    const int need = min(g.m, n);
+    if (g.nchunks == 1) {
+        // chunk 0 holds every candidate of the row (the other CTAs only
+        // scored nothing): select directly, no cluster exchange
+        if (chunk == 0) select_and_emit(keys, n, need, sh, idx + row * topk, g.D, topk, nullptr);
+        return;
     }
-    // ---- this chunk's chosen blocks, in block order, at the cluster offset
-    const int per = (n + kSelThreads - 1) / kSelThreads;
-    const int e0 = min(tid * per, n), e1 = min(e0 + per, n);
-    int cnt = 0;
-    for (int e = e0; e < e1; e++) cnt += (all || (any && (keys[e] & mask) >= prefix)) ? 1 : 0;
-    int total;
-    int pos = block_exclusive_scan(cnt, sh, total);
-    if (tid == 0) nchosen = total;
-    cluster.sync();
-    int off = 0;
-#pragma unroll
-    for (int r = 0; r < 8; r++)
-        if (r < chunk) off += *cluster.map_shared_rank(&nchosen, r);
-    int32_t *out = idx + row * topk;
-    for (int e = e0; e < e1; e++) {
-        const uint64_t k = keys[e];
-        if (all || (any && (k & mask) >= prefix)) out[1 + off + pos++] = key_block(k);
-    }
-    if (chunk == 0) {
-        // forced entries: the sink first, the diagonal after the chosen, -1 padding
-        for (int s = tid; s < topk; s += kSelThreads) {
-            if (s == 0) out[0] = 0;
-            else if (s == g.m + 1 && g.D > 0) out[s] = g.D;
-            else if (s > g.m + (g.D > 0 ? 1 : 0)) out[s] = -1;
-        }
-    }
-    cluster.sync();   // the chunks' counts must outlive the other CTAs' reads
+    uint64_t *dst = cluster.map_shared_rank(lists, 0) + chunk * kMaxChosen;
+    select_and_emit(keys, n, need, sh, nullptr, g.D, topk, dst);
+    for (int e = need + tid; e < kMaxChosen; e += kSelThreads) dst[e] = 0;
+    cluster.sync();   // every list is in the leader
+    if (chunk == 0) select_and_emit(lists, NCH * kMaxChosen, g.m, sh, idx + row * topk, g.D, topk, nullptr);
 }
 
 }  // namespace qsa
