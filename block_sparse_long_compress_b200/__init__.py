@@ -239,6 +239,59 @@ class QSAPrefill:
         return self.O
 
 
+class PrefillHostPipeline:
+    """Prefill steps fed from pinned host memory with neighbouring steps'
+    transfers overlapped: step k's Q, K, V upload (copy-in stream), step
+    k-1's compute (compute stream) and step k-2's O download (copy-out
+    stream) run at once over two device buffer sets.  Every step of the
+    path still runs in the library's kernels; this class only orders
+    copies and launches on streams with events."""
+
+    def __init__(self, B, Tq, Hq, Hkv, d, T_kv_max, topk, q_pos0=0, device="cuda"):
+        dev = torch.device(device)
+        self.device = dev
+        self.runs = [QSAPrefill(B, Tq, Hq, Hkv, d, T_kv_max, topk, q_pos0, device=dev) for _ in range(2)]
+        bf = torch.bfloat16
+        self.bufs = [dict(Q=torch.empty((B, Tq, Hq, d), dtype=bf, device=dev),
+                          K=torch.empty((B, Hkv, T_kv_max, d), dtype=bf, device=dev),
+                          V=torch.empty((B, Hkv, T_kv_max, d), dtype=bf, device=dev)) for _ in range(2)]
+        self.s_in = torch.cuda.Stream(device=dev)
+        self.s_cmp = torch.cuda.Stream(device=dev)
+        self.s_out = torch.cuda.Stream(device=dev)
+        self.ev = [dict(up=torch.cuda.Event(), done=torch.cuda.Event(), down=torch.cuda.Event()) for _ in range(2)]
+        self.used = [False, False]
+        self.k = 0
+
+    def submit(self, hQ, hK, hV, hO):
+        """Queue one step: hQ, hK, hV (pinned, the step's inputs) in, O out
+        to hO (pinned).  Returns at once; synchronize() waits."""
+        i = self.k & 1
+        buf, run, ev = self.bufs[i], self.runs[i], self.ev[i]
+        if self.used[i]:
+            self.s_in.wait_event(ev["done"])       # step k-2's compute has read this buffer set
+        with torch.cuda.stream(self.s_in):
+            buf["Q"].copy_(hQ, non_blocking=True)
+            buf["K"].copy_(hK, non_blocking=True)
+            buf["V"].copy_(hV, non_blocking=True)
+            ev["up"].record(self.s_in)
+        self.s_cmp.wait_event(ev["up"])
+        if self.used[i]:
+            self.s_cmp.wait_event(ev["down"])      # step k-2's O has been read out
+        if run.blk_begin > 0:
+            run.precompress_cache(buf["K"], self.s_cmp)
+        run(buf["Q"], buf["K"], buf["V"], self.s_cmp)
+        ev["done"].record(self.s_cmp)
+        self.s_out.wait_event(ev["done"])
+        with torch.cuda.stream(self.s_out):
+            hO.copy_(run.O, non_blocking=True)
+            ev["down"].record(self.s_out)
+        self.used[i] = True
+        self.k += 1
+
+    def synchronize(self):
+        self.s_out.synchronize()
+
+
 class QSADecode:
     """The whole decode path for a batch of single-token queries: select
     (per token) then split-K attention.  Summaries of complete blocks are

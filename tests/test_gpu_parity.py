@@ -269,3 +269,30 @@ def test_bad_block_index_sets_bounds_status(qsa):
     st, det = qsa.device_status()
     assert st == "QSA_ERR_BOUNDS"
     assert qsa.device_status()[0] == "QSA_OK"
+
+
+def test_prefill_host_pipeline_matches_direct_calls(qsa):
+    """The host pipeline (uploads, compute and downloads of neighbouring
+    steps on three streams, two device buffer sets) returns for every step
+    exactly what a direct call on device tensors returns."""
+    w = synthetic.custom(B=1, Tq=320, T_kv=1344, q_pos0=1024, Hq=16, Hkv=2, d=128, topk=8, seed=71)
+    inputs = []
+    for s in range(3):
+        x = synthetic.generate(synthetic.Workload(**{**w.__dict__, "seed": 71 + s}))
+        inputs.append({k: x[k].pin_memory() for k in ("Q", "K", "V")})
+    ref = []
+    for x in inputs:
+        run = qsa.QSAPrefill(w.B, w.Tq, w.Hq, w.Hkv, w.d, w.T_kv, w.topk, w.q_pos0, device=DEV)
+        K = x["K"].to(DEV)
+        run.precompress_cache(K)
+        ref.append(run(x["Q"].to(DEV), K, x["V"].to(DEV)).cpu())
+    pipe = qsa.PrefillHostPipeline(w.B, w.Tq, w.Hq, w.Hkv, w.d, w.T_kv, w.topk, w.q_pos0, device=DEV)
+    order = [0, 1, 2, 0, 1, 2]
+    outs = [torch.empty_like(ref[s]).pin_memory() for s in order]
+    for k, s in enumerate(order):
+        x = inputs[s]
+        pipe.submit(x["Q"], x["K"], x["V"], outs[k])
+    pipe.synchronize()
+    _status_ok(qsa)
+    for k, s in enumerate(order):
+        assert torch.equal(outs[k], ref[s]), f"step {k}"
