@@ -299,10 +299,10 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None):
         if "attention" in parts:
             qsa.decode(q, K, V, dec.idx, dec.o, L, dec.sm_scale, dec.ws_dec, s)
 
-    def capture(parts):
-        """flush -> event -> the step's kernels -> event, as one CUDA graph:
-        the events sit inside the graph, so the launch of the graph itself
-        stays outside the measured interval."""
+    def capture(parts, events=True):
+        """flush [-> event] -> the step's kernels [-> event], as one CUDA
+        graph; with events, they sit inside the graph so the graph's own
+        launch stays outside the measured interval."""
         e0 = torch.cuda.Event(enable_timing=True, external=True)
         e1 = torch.cuda.Event(enable_timing=True, external=True)
         side = torch.cuda.Stream(device=dev)
@@ -311,13 +311,15 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None):
         n0 = qsa.launch_count()
         with torch.cuda.graph(g, stream=side):
             flush(0)
-            e0.record(side)
+            if events:
+                e0.record(side)
             run_parts(parts, side)
-            e1.record(side)
+            if events:
+                e1.record(side)
         stream.wait_stream(side)
         return g, e0, e1, qsa.launch_count() - n0
 
-    def timed(parts):
+    def timed_events(parts):
         g, e0, e1, launches = capture(parts)
         for _ in range(args.warmup):
             g.replay()
@@ -331,24 +333,51 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None):
             out.append(e0.elapsed_time(e1) * 1e3)   # us
         return np.array(out), launches
 
-    t = {}
-    t["step"], launches_step = timed(("select", "attention"))
-    t["select"], _ = timed(("select",))
-    t["attention"], _ = timed(("attention",))
+    def timed_differential(parts):
+        """R back-to-back replays of (flush, kernels) minus R replays of
+        (flush) alone, both between events on the stream: the kernels' cost
+        per step as a stream of steps sees it."""
+        g, _, _, _ = capture(parts, events=False)
+        gf, _, _, _ = capture((), events=False)
+        res = {}
+        for name, gg in (("with", g), ("flush", gf)):
+            for _ in range(args.warmup):
+                gg.replay()
+            torch.cuda.synchronize()
+            if ws > 1:
+                torch.distributed.barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(steps):
+                gg.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            res[name] = e0.elapsed_time(e1) * 1e3 / steps
+        return res["with"] - res["flush"]
 
+    t = {}
+    t["step"], launches_step = timed_events(("select", "attention"))
+    t["select"], _ = timed_events(("select",))
+    t["attention"], _ = timed_events(("attention",))
+    d = {part: timed_differential(parts) for part, parts in
+         (("step", ("select", "attention")), ("select", ("select",)), ("attention", ("attention",)))}
     st, det = qsa.device_status()
     if st != "QSA_OK":
         raise RuntimeError(f"decode device status {st} ({det})")
-    us_step = float(t["step"].mean())
-    us_att = float(t["attention"].mean())
-    us_sel = float(t["select"].mean())
+    # the differential times (see timed_differential) are the reported ones;
+    # the in-graph event times are kept beside them
+    us_step, us_att, us_sel = d["step"], d["attention"], d["select"]
     by = decode_bytes(wd)
     att_gbs = by / (us_att * 1e-6) / 1e9
     sel_bytes = wd.B * wd.Hkv * ((L - 1) // 64) * wd.d * 4   # fp32 summaries read by scoring
     return {"workload": wd.name, "batch": wd.B, "context": L, "topk": wd.topk,
             "us_per_step": us_step, "us_per_token": us_step / wd.B,
-            "timing": "CUDA graph (L2 flush, event, step kernels, event) replayed per step",
+            "timing": ("per step: R back-to-back replays of a CUDA graph (L2 flush, step kernels) "
+                       "minus R replays of (L2 flush) alone, events around each set"),
             "breakdown_us": {"score_select": us_sel, "attention": us_att},
+            "in_graph_events_us": {"step": float(t["step"].mean()),
+                                   "score_select": float(t["select"].mean()),
+                                   "attention": float(t["attention"].mean())},
             "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": att_gbs,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": att_gbs / peaks["hbm_gbs"], "bytes_per_launch": by,
