@@ -105,9 +105,9 @@ __device__ __forceinline__ uint64_t make_key(float s, int j)
 __device__ __forceinline__ int key_block(uint64_t key) { return (int)(0xFFFFFFFFu - (uint32_t)key); }
 
 struct SelectShared {
-    int hist[256];
+    int hist[2][256];           // digit counts, double-buffered across radix passes
     int warp_tot[kSelThreads / 32];
-    int digit, above, bucket;
+    int digit[2], above[2], bucket[2];
 };
 
 // Adds 1 to hist[digit] for every lane with active set; lanes of a warp
@@ -122,15 +122,16 @@ __device__ __forceinline__ void hist_add(int *hist, bool active, int digit)
 }
 
 // Warp 0: the digit whose bucket holds the need-th largest key of
-// sh.hist (counts by digit), the count above it and the bucket's size.
-__device__ __forceinline__ void find_digit(SelectShared &sh, int need)
+// sh.hist[b] (counts by digit), the count above it and the bucket's size,
+// into sh.digit[b], sh.above[b], sh.bucket[b].
+__device__ __forceinline__ void find_digit(SelectShared &sh, int b, int need)
 {
     const int lane = threadIdx.x & 31;
     // lane l owns bins 255-8l .. 248-8l (descending)
     int c[8], tot = 0;
 #pragma unroll
     for (int q = 0; q < 8; q++) {
-        c[q] = sh.hist[255 - 8 * lane - q];
+        c[q] = sh.hist[b][255 - 8 * lane - q];
         tot += c[q];
     }
     int incl = tot;
@@ -145,9 +146,9 @@ __device__ __forceinline__ void find_digit(SelectShared &sh, int need)
 #pragma unroll
         for (int q = 0; q < 8; q++) {
             if (cum + c[q] >= need) {
-                sh.digit = 255 - 8 * lane - q;
-                sh.above = cum;
-                sh.bucket = c[q];
+                sh.digit[b] = 255 - 8 * lane - q;
+                sh.above[b] = cum;
+                sh.bucket[b] = c[q];
                 break;
             }
             cum += c[q];
@@ -161,25 +162,27 @@ __device__ __forceinline__ void find_digit(SelectShared &sh, int need)
 __device__ void radix_select(const uint64_t *keys, int n, int need, SelectShared &sh,
                              uint64_t &prefix_out, uint64_t &mask_out)
 {
+    // two barriers per pass: the counts and the result of a pass live in
+    // one half of the double buffers while the other half, read by warp 0
+    // one pass earlier, is zeroed for the next pass
     const int tid = threadIdx.x, warp = tid >> 5;
     uint64_t prefix = 0, mask = 0;
-    for (int shift = 56; shift >= 0; shift -= 8) {
-        for (int b = tid; b < 256; b += kSelThreads) sh.hist[b] = 0;
-        __syncthreads();
+    for (int d = tid; d < 256; d += kSelThreads) sh.hist[0][d] = 0;
+    __syncthreads();
+    for (int shift = 56, cur = 0; shift >= 0; shift -= 8, cur ^= 1) {
+        for (int d = tid; d < 256; d += kSelThreads) sh.hist[cur ^ 1][d] = 0;
         for (int base = 0; base < n; base += kSelThreads) {
             const int e = base + tid;
             const uint64_t k = e < n ? keys[e] : 0;
-            hist_add(sh.hist, e < n && (k & mask) == prefix, (int)((k >> shift) & 0xFF));
+            hist_add(sh.hist[cur], e < n && (k & mask) == prefix, (int)((k >> shift) & 0xFF));
         }
         __syncthreads();
-        if (warp == 0) find_digit(sh, need);
+        if (warp == 0) find_digit(sh, cur, need);
         __syncthreads();
-        need -= sh.above;
-        prefix |= (uint64_t)sh.digit << shift;
+        need -= sh.above[cur];
+        prefix |= (uint64_t)sh.digit[cur] << shift;
         mask |= (uint64_t)0xFF << shift;
-        const bool done = (sh.bucket == need);
-        __syncthreads();   // everyone has read sh.* before the next pass
-        if (done) break;
+        if (sh.bucket[cur] == need) break;   // the same decision in every thread
     }
     prefix_out = prefix;
     mask_out = mask;
