@@ -350,6 +350,9 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         : "memory");
 }
 
+// Nonzero in one lane (the same one every time) of a converged warp: an
+// MMA warp runs its waits and descriptor arithmetic together, warp-uniform,
+// and lets the elected lane issue the single-thread tcgen05 ops.
 __device__ __forceinline__ uint32_t elect_one()
 {
     uint32_t pred = 0;
