@@ -4,11 +4,16 @@
 // section "QSA Is an Address-Selection Problem, Not a New Attention
 // Equation": ordinary attention over the visible cells).
 //
-// Work unit (one CTA, one per SM): two 128-row MMA tiles of one KV group
-// and query block; row r of a tile = token (r / G), query head (r % G) --
-// 256 rows sharing the same selected key blocks, so every gathered K/V
-// block is loaded once for all 256 rows.  One selected 64-key block per
-// step, through separate 4-deep K and V rings; per block n and tile t:
+// Persistent kernel: one CTA per SM walks the work units u = blockIdx.x,
+// blockIdx.x + gridDim.x, ...  A unit is two 128-row MMA tiles of one KV
+// group and query block; row r of a tile = token (r / G), query head
+// (r % G) -- 256 rows sharing the same selected key blocks, so every
+// gathered K/V block is loaded once for all 256 rows.  The CTA treats the
+// blocks of all its units as one stream (ring stages, S buffers and barrier
+// phases count blocks across units), so the next unit's block list, Q tiles,
+// first K/V blocks and first S MMAs are on their way while the current
+// unit's last blocks and epilogue run.  One selected 64-key block per step,
+// through separate 4-deep K and V rings; per block n and tile t:
 //     S_t(n) = Q_t K_n^T    tcgen05.mma kind::f16, M=128 N=64 K=16 steps,
 //                           A = Q_t, B = the block's keys (both K-major in
 //                           shared memory), D = S buffer n%2 of tile t in
@@ -21,20 +26,26 @@
 // S is double-buffered in TMEM: the issuer of tile t puts S_t(n+2) on the
 // pipe right behind PV_t(n) (the pipe runs a thread's MMAs in order, so
 // PV_t(n) reads P_t(n) before S_t(n+2) overwrites it), and when the
-// softmax finishes block n, S_t(n+1) is normally complete already.  Both
-// tiles' softmaxes therefore run all the time, side by side on the SM's
-// issue slots, while the tensor pipe works through the MMAs both tiles
-// keep queued.  The running max only moves (and O_t is rescaled in TMEM)
-// when a block's max exceeds it by more than 2^8.
+// softmax finishes block n, S_t(n+1) is normally complete already.  Tile 1
+// trails tile 0 by half a block (each waits for the other's block max), so
+// one tile's TMEM loads and max run during the other's exponentials while
+// the tensor pipe works through the MMAs both tiles keep queued.  The
+// running max only moves (and O_t is rescaled in TMEM) when a block's max
+// exceeds it by more than 2^8.  At a unit boundary the issuer puts both
+// last PVs on the pipe before the next unit's first S (which waits for the
+// next Q tiles), and the next unit's first PV -- which overwrites O_t --
+// waits for P of its block, which the softmax warps signal only after
+// their epilogue has read O_t.
 //
 // Warps (384 threads, three warpgroups): 0-7 softmax/epilogue (tile =
-// warp/4, TMEM lane quarter = warp%4, thread = row), 8 TMA producer of Q
-// and K, 9 TMEM allocator + MMA issuer of tile 0, 10 MMA issuer of tile 1,
-// 11 TMA producer of V.  The last warpgroup gives registers to the softmax
-// warpgroups (setmaxnreg).  Each softmax warp signals P with a single
-// arrive, and the softmax warps release the K and V stages: an MMA commit
-// covers every earlier MMA of its thread, so S_t(n) done frees K_n for
-// tile t and, S_t(n) being issued behind PV_t(n-2), V_{n-2} too.
+// warp/4, TMEM lane quarter = warp%4, thread = row), 8 block-list reader
+// and TMA producer of Q and K, 9 TMEM allocator + MMA issuer of tile 0,
+// 10 MMA issuer of tile 1, 11 TMA producer of V.  The last warpgroup gives
+// registers to the softmax warpgroups (setmaxnreg).  Each softmax warp
+// signals P with a single arrive, and the softmax warps release the K and
+// V stages: an MMA commit covers every earlier MMA of its thread, so S_t(n)
+// done frees K_n for tile t and, S_t(n) being issued behind PV_t(n-2),
+// V_{n-2} too.  The issuers' commit after a unit's last S frees the Q tiles.
 // TMEM (512 columns): O_0 [0,128) O_1 [128,256); S buffer b of tile t at
 // [256 + 128t + 64b, +64), P in its first 32 columns.  Every mbarrier wait
 // is bounded.
@@ -47,14 +58,17 @@ template <int D, int G>
 struct PrefillCfg {
     static constexpr int M = 128;                  // rows per tile
     static constexpr int TOK = M / G;              // tokens per tile
-    static constexpr int TILES = 64 / (2 * TOK);   // CTAs per 64-token query block
+    static constexpr int TILES = 64 / (2 * TOK);   // units per 64-token query block
     static constexpr int NH = D / 64;              // 128-byte column halves
     static constexpr int Q_HALF = 128 * 128;       // 128 rows x 128 B
     static constexpr int QT_BYTES = NH * Q_HALF;   // one Q tile
     static constexpr int B_HALF = 64 * 128;        // 64 rows x 128 B
     static constexpr int BLK_BYTES = NH * B_HALF;  // K (or V) of one block
     static constexpr int NS = 4;                   // K stages and V stages (blocks)
-    static constexpr int SMEM_DATA = 2 * QT_BYTES + 2 * NS * BLK_BYTES;
+    // epilogue staging: per softmax warp, 32 rows x 128 B (one 64-column
+    // half of O at a time) for a transpose into coalesced stores
+    static constexpr int STAGE_BYTES = 32 * 128;
+    static constexpr int SMEM_DATA = 2 * QT_BYTES + 2 * NS * BLK_BYTES + 8 * STAGE_BYTES;
     // the CTA owns all 512 TMEM columns: ask for enough shared memory that
     // a second CTA never lands on the same SM
     static constexpr int SMEM_REQUEST = (SMEM_DATA + 1024 > 120 * 1024) ? SMEM_DATA + 1024 : 120 * 1024;
@@ -65,32 +79,53 @@ struct PrefillCfg {
     // REG_HIGH: 256 * REG_HIGH + 128 * REG_LOW must not exceed
     // 384 * REG_LAUNCH
     static constexpr int REG_LAUNCH = 168;
-    static constexpr int REG_LOW = 48;
+    static constexpr int REG_LOW = 56;
     static constexpr int REG_HIGH = 224;
     static_assert(256 * REG_HIGH + 128 * REG_LOW <= 384 * REG_LAUNCH, "register split exceeds the launch pool");
     static constexpr int TMEM_COLS = 512;
     static constexpr int O_COL = 0, S_COL = 256;
+    // arrivals that free a block-list slot: V producer, two issuers, eight
+    // softmax warps
+    static constexpr int LIST_USERS = 11;
 };
 
 struct PrefillShared {
-    uint64_t q_full;
+    uint64_t q_full, q_empty;
     uint64_t k_full[4], k_empty[4];
     uint64_t v_full[4], v_empty[4];
     uint64_t s_full[2][2];      // [tile][S buffer]
     uint64_t p_full[2][2];      // [tile][S buffer]
     uint64_t pv_done[2];        // [tile]
     uint64_t stag[2];           // [tile]: its softmax has its block max
+    uint64_t list_full[2], list_empty[2];   // [list slot]
     uint32_t tmem_base;
-    int nblk;
     int abort;
-    int blocks[64];
+    int nblk[2];                // [list slot] blocks of the unit (>= 1)
+    int none[2];                // [list slot] the row lists no valid block
+    int blocks[2][64];
 };
+
+// Work unit u -> query block i, first token, batch x KV group bg.  False for
+// the idle units past a ragged last query block.
+struct PrefillUnit {
+    int i, bg, token0;
+};
+
+template <int TILES, int TOK>
+__device__ __forceinline__ bool prefill_unit(int u, int NX, int Tq, PrefillUnit &w)
+{
+    const int x = u % NX;
+    w.bg = u / NX;
+    w.i = x / TILES;
+    w.token0 = w.i * 64 + (x % TILES) * 2 * TOK;
+    return w.token0 < Tq;
+}
 
 template <int D, int G>
 __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ idx,
-    __nv_bfloat16 *__restrict__ O, float *__restrict__ lse, int Tq, int Hq, int Hkv,
+    __nv_bfloat16 *__restrict__ O, float *__restrict__ lse, int Tq, int Hq, int Hkv, int BH,
     int q_pos0, int T_kv_max, int topk, float sm_scale_log2)
 {
     using C = PrefillCfg<D, G>;
@@ -101,33 +136,17 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
     uint8_t *q_smem = smem;                          // [tile][half][128 rows][128 B]
     uint8_t *k_smem = smem + 2 * C::QT_BYTES;        // [stage][half][64 rows][128 B]
     uint8_t *v_smem = k_smem + C::NS * C::BLK_BYTES;
+    uint8_t *o_stage = v_smem + C::NS * C::BLK_BYTES;   // [softmax warp][32 rows][8 x 16 B]
 
     const int NR = (Tq + 63) / 64;
-    const int i = blockIdx.x / C::TILES, sub = blockIdx.x % C::TILES;
-    const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv;
-    const int token0 = i * 64 + sub * 2 * C::TOK;
-    if (token0 >= Tq) return;   // ragged tail: whole CTA idle (uniform exit)
+    const int NX = NR * C::TILES;
+    const int U = NX * BH;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row_last = min(i * 64 + 63, Tq - 1);
-    const int Dg = (q_pos0 + row_last) / 64;
 
     if (threadIdx.x == 0) {
-        // selected blocks of this row; stop at the first -1 or bad index
-        const int32_t *sel = idx + ((long)bg * NR + i) * topk;
-        int n = 0;
-        for (int s = 0; s < topk; s++) {
-            const int j = sel[s];
-            if (j < 0) break;
-            if (j > Dg || (n > 0 && j <= sh.blocks[n - 1])) {
-                report(QSA_ERR_BOUNDS, 1);
-                break;
-            }
-            sh.blocks[n++] = j;
-        }
-        if (n == 0) report(QSA_ERR_BOUNDS, 2);
-        sh.nblk = n;
         sh.abort = 0;
         mbar_init(&sh.q_full, 1);
+        mbar_init(&sh.q_empty, 2);           // one commit per issuer
         for (int s = 0; s < C::NS; s++) {
             mbar_init(&sh.k_full[s], 1);
             mbar_init(&sh.k_empty[s], 2);    // one arrive per tile
@@ -141,6 +160,8 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
             }
             mbar_init(&sh.pv_done[t], 1);
             mbar_init(&sh.stag[t], 4);
+            mbar_init(&sh.list_full[t], 1);
+            mbar_init(&sh.list_empty[t], C::LIST_USERS);
         }
         fence_barrier_init();
     }
@@ -157,35 +178,113 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
-    const int nblk = sh.nblk;
     volatile int *abort = &sh.abort;
+    // a wait's outcome, made warp-uniform (a warp never splits on a timeout)
+    auto wait_all = [&](uint64_t *bar, uint32_t parity, int where) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, where));
+    };
 
     if (warp >= 8) {
     // warpgroup 2 (one setmaxnreg for its four warps): producers, issuers
     setmaxnreg_dec<C::REG_LOW>();
-    if (warp == 8 || warp == 11) {
-        // ---------------------------- TMA producers: Q and K (8), V (11)
-        const bool is_k = warp == 8;
-        if (lane == 0 && nblk > 0) {
-            if (is_k) {
-                mbar_arrive_expect_tx(&sh.q_full, 2 * C::QT_BYTES);
-                for (int t = 0; t < 2; t++)
-                    for (int h = 0; h < C::NH; h++)
-                        tma_load_3d(q_smem + t * C::QT_BYTES + h * C::Q_HALF, &tmQ, &sh.q_full, h * 64,
-                                    g * G, b * Tq + token0 + t * C::TOK);
+    if (warp == 8) {
+        // ------------------- block lists (whole warp), Q and K (lane 0)
+        int k = 0, gk = 0;   // units and K blocks so far
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < U; u += gridDim.x) {
+            PrefillUnit w;
+            if (!prefill_unit<C::TILES, C::TOK>(u, NX, Tq, w)) continue;
+            const int slot = k & 1;
+            const int b = w.bg / Hkv, g = w.bg % Hkv;
+            const int Dg = (q_pos0 + min(w.i * 64 + 63, Tq - 1)) / 64;
+            if (k >= 2 && !wait_all(&sh.list_empty[slot], ((k >> 1) - 1) & 1, 12)) break;
+            // the row's list, one entry per lane: it ends at the first -1;
+            // an index past the diagonal or not above its predecessor is an
+            // error and ends it too
+            const int32_t *sel = idx + ((long)w.bg * NR + w.i) * topk;
+            int n = 0, prev = -1;
+            bool bad = false;
+            for (int r0 = 0; r0 < topk; r0 += 32) {
+                const int s = r0 + lane;
+                const int j = s < topk ? sel[s] : -1;
+                int jp = __shfl_up_sync(0xffffffffu, j, 1);
+                if (lane == 0) jp = prev;
+                const bool stop_bad = j >= 0 && (j > Dg || (s > 0 && j <= jp));
+                const unsigned stops = __ballot_sync(0xffffffffu, j < 0 || stop_bad);
+                const int f = stops ? __ffs(stops) - 1 : 32;
+                if (lane < f) sh.blocks[slot][s] = j;
+                n = r0 + f;
+                if (stops) {
+                    bad = __shfl_sync(0xffffffffu, stop_bad, f);
+                    break;
+                }
+                prev = __shfl_sync(0xffffffffu, j, 31);
             }
-            const CUtensorMap *map = is_k ? &tmK : &tmV;
-            uint64_t *full = is_k ? sh.k_full : sh.v_full;
-            uint64_t *empty = is_k ? sh.k_empty : sh.v_empty;
-            uint8_t *ring = is_k ? k_smem : v_smem;
-            const int kv_row0 = bg * T_kv_max;   // host checks B*Hkv*T_kv_max < 2^31
-            for (int n = 0; n < nblk; n++) {
-                const int st = n % C::NS;
-                if (n >= C::NS && !mbar_wait(&empty[st], ((n / C::NS) - 1) & 1, abort, is_k ? 10 : 11)) break;
-                mbar_arrive_expect_tx(&full[st], C::BLK_BYTES);
-                const int row = kv_row0 + 64 * sh.blocks[n];
-                for (int h = 0; h < C::NH; h++)
-                    tma_load_2d(ring + st * C::BLK_BYTES + h * C::B_HALF, map, &full[st], h * 64, row);
+            if (lane == 0) {
+                if (bad) report(QSA_ERR_BOUNDS, 1);
+                if (n == 0) {
+                    // no valid block: block 0 goes through the pipeline (in
+                    // bounds) and the epilogue writes zeros
+                    report(QSA_ERR_BOUNDS, 2);
+                    sh.blocks[slot][0] = 0;
+                }
+                sh.nblk[slot] = max(n, 1);
+                sh.none[slot] = n == 0;
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sh.list_full[slot]);
+                // Q tiles of the unit, once the previous unit's S are done
+                if (k >= 1 && !mbar_wait(&sh.q_empty, (k - 1) & 1, abort, 13)) ok = false;
+                if (ok) {
+                    mbar_arrive_expect_tx(&sh.q_full, 2 * C::QT_BYTES);
+                    for (int t = 0; t < 2; t++)
+                        for (int h = 0; h < C::NH; h++)
+                            tma_load_3d(q_smem + t * C::QT_BYTES + h * C::Q_HALF, &tmQ, &sh.q_full, h * 64,
+                                        g * G, b * Tq + w.token0 + t * C::TOK);
+                }
+                const int kv_row0 = w.bg * T_kv_max;   // host checks B*Hkv*T_kv_max < 2^31
+                for (int nn = 0; ok && nn < max(n, 1); nn++) {
+                    const int gb = gk + nn, st = gb % C::NS;
+                    if (gb >= C::NS && !mbar_wait(&sh.k_empty[st], ((gb / C::NS) - 1) & 1, abort, 10)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sh.k_full[st], C::BLK_BYTES);
+                    const int row = kv_row0 + 64 * sh.blocks[slot][nn];
+                    for (int h = 0; h < C::NH; h++)
+                        tma_load_2d(k_smem + st * C::BLK_BYTES + h * C::B_HALF, &tmK, &sh.k_full[st], h * 64, row);
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            gk += max(n, 1);
+            k++;
+        }
+    } else if (warp == 11) {
+        // --------------------------------------------- V producer (lane 0)
+        if (lane == 0) {
+            int k = 0, gv = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < U; u += gridDim.x) {
+                PrefillUnit w;
+                if (!prefill_unit<C::TILES, C::TOK>(u, NX, Tq, w)) continue;
+                const int slot = k & 1;
+                if (!mbar_wait(&sh.list_full[slot], (k >> 1) & 1, abort, 14)) break;
+                const int nb = sh.nblk[slot];
+                const int kv_row0 = w.bg * T_kv_max;
+                for (int nn = 0; nn < nb; nn++, gv++) {
+                    const int st = gv % C::NS;
+                    if (gv >= C::NS && !mbar_wait(&sh.v_empty[st], ((gv / C::NS) - 1) & 1, abort, 11)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sh.v_full[st], C::BLK_BYTES);
+                    const int row = kv_row0 + 64 * sh.blocks[slot][nn];
+                    for (int h = 0; h < C::NH; h++)
+                        tma_load_2d(v_smem + st * C::BLK_BYTES + h * C::B_HALF, &tmV, &sh.v_full[st], h * 64, row);
+                }
+                mbar_arrive(&sh.list_empty[slot]);
+                k++;
             }
         }
     } else {
@@ -193,53 +292,66 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
         // the whole warp runs the loop (waits and descriptors stay
         // warp-uniform); one elected lane issues the MMAs and commits
         const int t = __shfl_sync(0xffffffffu, warp - 9, 0);
-        // a wait's outcome, made warp-uniform
-        auto wait_all = [&](uint64_t *bar, uint32_t parity, int where) -> bool {
-            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, where));
-        };
-        if (nblk > 0) {
-            constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64, 0, 0);
-            constexpr uint32_t idesc_o = umma_idesc_bf16(128, D, 0, 1);
-            // descriptor bases, built once: per MMA only a 64-bit add of the
-            // byte offset >> 4 into the start-address field remains (shared
-            // memory addresses stay below 2^18, so the field never carries)
-            const uint64_t qd = umma_smem_desc(smem_u32(q_smem + t * C::QT_BYTES), 16, 1024);
-            const uint64_t kd = umma_smem_desc(smem_u32(k_smem), 16, 1024);
-            const uint64_t vd = umma_smem_desc(smem_u32(v_smem), C::B_HALF, 1024);
-            const uint32_t s_tmem0 = tmem + C::S_COL + 128 * t;
-            const uint32_t o_tmem = tmem + C::O_COL + 128 * t;
-            // S_t(n) = Q_t K_n^T into S buffer n%2
-            auto issue_s = [&](int n) -> bool {
-                const int st = n % C::NS;
-                if (!wait_all(&sh.k_full[st], (n / C::NS) & 1, 21)) return false;
-                tc_fence_after();
-                const uint64_t kds = kd + (uint64_t)((st * C::BLK_BYTES) >> 4);
-                const uint32_t s_tmem = s_tmem0 + 64 * (n & 1);
-                if (elect_one()) {
+        constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64, 0, 0);
+        constexpr uint32_t idesc_o = umma_idesc_bf16(128, D, 0, 1);
+        // descriptor bases, built once: per MMA only a 64-bit add of the
+        // byte offset >> 4 into the start-address field remains (shared
+        // memory addresses stay below 2^18, so the field never carries)
+        const uint64_t qd = umma_smem_desc(smem_u32(q_smem + t * C::QT_BYTES), 16, 1024);
+        const uint64_t kd = umma_smem_desc(smem_u32(k_smem), 16, 1024);
+        const uint64_t vd = umma_smem_desc(smem_u32(v_smem), C::B_HALF, 1024);
+        const uint32_t s_tmem0 = tmem + C::S_COL + 128 * t;
+        const uint32_t o_tmem = tmem + C::O_COL + 128 * t;
+        // S_t(gb) = Q_t K_gb^T into S buffer gb%2 (gb counts blocks across
+        // units); after a unit's last S, a commit frees the Q tiles
+        auto issue_s = [&](int gb, bool last_of_unit) -> bool {
+            const int st = gb % C::NS;
+            if (!wait_all(&sh.k_full[st], (gb / C::NS) & 1, 21)) return false;
+            tc_fence_after();
+            const uint64_t kds = kd + (uint64_t)((st * C::BLK_BYTES) >> 4);
+            const uint32_t s_tmem = s_tmem0 + 64 * (gb & 1);
+            if (elect_one()) {
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; kk++) {
-                        const uint64_t qoff = (uint64_t)((((kk >> 2) * C::Q_HALF) + (kk & 3) * 32) >> 4);
-                        const uint64_t koff = (uint64_t)((((kk >> 2) * C::B_HALF) + (kk & 3) * 32) >> 4);
-                        umma_ss(s_tmem, qd + qoff, kds + koff, idesc_s, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&sh.s_full[t][n & 1]);
+                for (int kk = 0; kk < D / 16; kk++) {
+                    const uint64_t qoff = (uint64_t)((((kk >> 2) * C::Q_HALF) + (kk & 3) * 32) >> 4);
+                    const uint64_t koff = (uint64_t)((((kk >> 2) * C::B_HALF) + (kk & 3) * 32) >> 4);
+                    umma_ss(s_tmem, qd + qoff, kds + koff, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                __syncwarp();
-                return true;
-            };
-            bool ok = wait_all(&sh.q_full, 0, 20);
-            if (ok) ok = issue_s(0);
-            if (ok && nblk > 1) ok = issue_s(1);
-            for (int n = 0; ok && n < nblk; n++) {
-                const int st = n % C::NS;
-                if (!wait_all(&sh.v_full[st], (n / C::NS) & 1, 26)) break;
-                // the real dependency: this tile's P of block n
-                if (!wait_all(&sh.p_full[t][n & 1], (n >> 1) & 1, 22)) break;
+                umma_commit(&sh.s_full[t][gb & 1]);
+                if (last_of_unit) umma_commit(&sh.q_empty);
+            }
+            __syncwarp();
+            return true;
+        };
+        auto next_unit = [&](int u) -> int {
+            PrefillUnit w;
+            while (u < U && !prefill_unit<C::TILES, C::TOK>(u, NX, Tq, w)) u += gridDim.x;
+            return u;
+        };
+        // a unit's length from its list slot, then free the slot
+        auto unit_len = [&](int k, int &nb) -> bool {
+            if (!wait_all(&sh.list_full[k & 1], (k >> 1) & 1, 23)) return false;
+            nb = sh.nblk[k & 1];
+            __syncwarp();
+            if (elect_one()) mbar_arrive(&sh.list_empty[k & 1]);
+            return true;
+        };
+        int u = next_unit(blockIdx.x);
+        int k = 0, g0 = 0, nb = 0;   // unit, its first block, its length
+        bool ok = u < U && unit_len(0, nb) && wait_all(&sh.q_full, 0, 20);
+        if (ok) ok = issue_s(0, nb == 1);
+        if (ok && nb > 1) ok = issue_s(1, nb == 2);
+        while (ok) {
+            for (int n = 0; ok && n < nb; n++) {
+                const int gb = g0 + n, st = gb % C::NS;
+                if (!wait_all(&sh.v_full[st], (gb / C::NS) & 1, 26)) { ok = false; break; }
+                // the real dependency: this tile's P of the block
+                if (!wait_all(&sh.p_full[t][gb & 1], (gb >> 1) & 1, 22)) { ok = false; break; }
                 tc_fence_after();
-                // O_t += P_t V: P in the S buffer's columns 0-31, 16 keys
-                // (8 columns) per k-step
+                // O_t (+)= P_t V: P in the S buffer's columns 0-31, 16 keys
+                // (8 columns) per k-step; the unit's first block overwrites
                 const uint64_t vds = vd + (uint64_t)((st * C::BLK_BYTES) >> 4);
-                const uint32_t p_tmem = s_tmem0 + 64 * (n & 1);
+                const uint32_t p_tmem = s_tmem0 + 64 * (gb & 1);
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < 4; kk++)
@@ -248,9 +360,18 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
                     umma_commit(&sh.pv_done[t]);
                 }
                 __syncwarp();
-                // S_t(n+2) into the same buffer, right behind PV_t(n)
-                if (n + 2 < nblk && !issue_s(n + 2)) break;
+                // S_t(gb+2) into the same buffer, right behind PV_t(gb)
+                if (n + 2 < nb && !issue_s(gb + 2, n + 3 == nb)) ok = false;
             }
+            if (!ok) break;
+            // the next unit: its length, its Q tiles, its first two S
+            u = next_unit(u + gridDim.x);
+            if (u >= U) break;
+            k++;
+            g0 += nb;
+            if (!unit_len(k, nb) || !wait_all(&sh.q_full, k & 1, 20)) break;
+            if (!issue_s(g0, nb == 1)) break;
+            if (nb > 1 && !issue_s(g0 + 1, nb == 2)) break;
         }
     }
     } else {
@@ -258,137 +379,174 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
         setmaxnreg_inc<C::REG_HIGH>();
         const int t = warp >> 2;
         const int r = ((warp & 3) << 5) | lane;              // row = TMEM lane
-        const int tok = token0 + t * C::TOK + r / G;
-        const long p = (long)q_pos0 + tok;
         const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const uint32_t s_addr0 = lane_addr + C::S_COL + 128 * t;
         const uint32_t o_addr = lane_addr + C::O_COL + 128 * t;
         const uint64_t sc2 = f2_pack(sm_scale_log2, sm_scale_log2);
-        float m_run = -INFINITY, l = 0.f;
-        bool ok = nblk > 0;
-        for (int n = 0; ok && n < nblk; n++) {
-            // stagger: tile 1 starts block n once tile 0 has the max of n,
-            // tile 0 starts block n once tile 1 has the max of n-1, so one
-            // tile's loads and max run during the other's exponentials
-            if (t == 1 || n > 0) {
-                if (!mbar_wait(&sh.stag[t ^ 1], (n - (t ^ 1)) & 1, abort, 33)) { ok = false; break; }
-            }
-            if (!mbar_wait(&sh.s_full[t][n & 1], (n >> 1) & 1, abort, 30)) { ok = false; break; }
-            tc_fence_after();
-            // the issuer's commit covers every earlier MMA of this tile: S_t(n)
-            // done frees K stage n and, PV_t(n-2) having been issued before
-            // it, V stage n-2 -- the stage releases ride on this wait
-            if ((warp & 3) == 0 && lane == 0) {
-                mbar_arrive(&sh.k_empty[n % C::NS]);
-                if (n >= 2) mbar_arrive(&sh.v_empty[(n - 2) % C::NS]);
-            }
-            const uint32_t s_addr = s_addr0 + 64 * (n & 1);
-            // keys c <= lim of the block are visible: only the diagonal
-            // block is masked
-            const int blk = sh.blocks[n];
-            const int lim = blk == Dg ? (int)(p - 64L * Dg) : 63;
-            uint32_t sr[64];
-            tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-            tmem_wait_ld();
-            if (lim < 63) {
-#pragma unroll
-                for (int c = 0; c < 64; c++)
-                    if (c > lim) sr[c] = 0xff800000u;   // -inf
-            }
-            // 16 independent chains of 3-input maxima (the instruction's
-            // latency, not its count, sets the time), then a short tree
-            float qm[16];
-#pragma unroll
-            for (int k = 0; k < 16; k++)
-                qm[k] = max3f(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1]),
-                              __uint_as_float(sr[32 + 2 * k]));
-#pragma unroll
-            for (int k = 0; k < 16; k++) qm[k] = fmaxf(qm[k], __uint_as_float(sr[33 + 2 * k]));
-#pragma unroll
-            for (int k = 0; k < 5; k++) qm[k] = max3f(qm[3 * k], qm[3 * k + 1], qm[3 * k + 2]);
-            const float mx = fmaxf(max3f(qm[0], qm[1], qm[2]), max3f(qm[3], qm[4], qm[15])) * sm_scale_log2;
-            if (lane == 0) mbar_arrive(&sh.stag[t]);
-            if (n == 0) {
-                m_run = mx;
-            } else if (__any_sync(0xffffffffu, mx > m_run + 8.0f)) {
-                const float m_new = fmaxf(m_run, mx);
-                const float alpha = fast_exp2(m_run - m_new);
-                // O_t is stable once PV_t(n-1) has completed
-                if (!mbar_wait(&sh.pv_done[t], (n - 1) & 1, abort, 31)) { ok = false; break; }
+        int k = 0, g0 = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < U; u += gridDim.x) {
+            PrefillUnit w;
+            if (!prefill_unit<C::TILES, C::TOK>(u, NX, Tq, w)) continue;
+            const int slot = k & 1;
+            if (!wait_all(&sh.list_full[slot], (k >> 1) & 1, 34)) { ok = false; break; }
+            const int nb = sh.nblk[slot];
+            const bool none = sh.none[slot] != 0;
+            const int b = w.bg / Hkv, g = w.bg % Hkv;
+            const int Dg = (q_pos0 + min(w.i * 64 + 63, Tq - 1)) / 64;
+            const int tok = w.token0 + t * C::TOK + r / G;
+            const long p = (long)q_pos0 + tok;
+            float m_run = -INFINITY, l = 0.f;
+            for (int n = 0; n < nb; n++) {
+                const int gb = g0 + n;
+                // stagger: tile 1 starts block gb once tile 0 has its max,
+                // tile 0 starts it once tile 1 has the max of gb-1
+                if (t == 1 || gb > 0) {
+                    if (!wait_all(&sh.stag[t ^ 1], (gb - (t ^ 1)) & 1, 33)) { ok = false; break; }
+                }
+                if (!wait_all(&sh.s_full[t][gb & 1], (gb >> 1) & 1, 30)) { ok = false; break; }
                 tc_fence_after();
-#pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t o[32];
-                    tmem_ld32(o_addr + c0, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int c = 0; c < 32; c++) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                    tmem_st32(o_addr + c0, o);
+                // the issuer's commit covers every earlier MMA of this tile:
+                // S_t(gb) done frees K stage gb and, PV_t(gb-2) having been
+                // issued before it, V stage gb-2
+                if ((warp & 3) == 0 && lane == 0) {
+                    mbar_arrive(&sh.k_empty[gb % C::NS]);
+                    if (gb >= 2) mbar_arrive(&sh.v_empty[(gb - 2) % C::NS]);
                 }
-                tmem_wait_st();
-                l *= alpha;
-                m_run = m_new;
-            }
-            // P = 2^(s*c - m), 1 of every 4 pairs on the FMA pipe, the rest on
-            // MUFU; packed bf16 P goes over the buffer's first 32 columns
-            const uint64_t nm2 = f2_pack(-m_run, -m_run);
-            uint64_t lacc[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+                const uint32_t s_addr = s_addr0 + 64 * (gb & 1);
+                // keys c <= lim of the block are visible: only the diagonal
+                // block is masked
+                const int blk = sh.blocks[slot][n];
+                const int lim = blk == Dg ? (int)(p - 64L * Dg) : 63;
+                uint32_t sr[64];
+                tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                tmem_wait_ld();
+                if (lim < 63) {
 #pragma unroll
-            for (int c0 = 0; c0 < 64; c0 += 32) {
-                uint32_t pk[16];
+                    for (int c = 0; c < 64; c++)
+                        if (c > lim) sr[c] = 0xff800000u;   // -inf
+                }
+                // 16 independent chains of 3-input maxima (the instruction's
+                // latency, not its count, sets the time), then a short tree
+                float qm[16];
 #pragma unroll
-                for (int c = 0; c < 16; c++) {
-                    const uint64_t x2 = f2_fma(
-                        f2_pack(__uint_as_float(sr[c0 + 2 * c]), __uint_as_float(sr[c0 + 2 * c + 1])), sc2, nm2);
-                    float p0, p1;
-                    if ((c & 3) == 3) {
-                        f2_unpack(exp2_poly_x2(x2), p0, p1);
-                    } else {
-                        float x0, x1;
-                        f2_unpack(x2, x0, x1);
-                        p0 = fast_exp2(x0);
-                        p1 = fast_exp2(x1);
+                for (int c = 0; c < 16; c++)
+                    qm[c] = max3f(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]),
+                                  __uint_as_float(sr[32 + 2 * c]));
+#pragma unroll
+                for (int c = 0; c < 16; c++) qm[c] = fmaxf(qm[c], __uint_as_float(sr[33 + 2 * c]));
+#pragma unroll
+                for (int c = 0; c < 5; c++) qm[c] = max3f(qm[3 * c], qm[3 * c + 1], qm[3 * c + 2]);
+                const float mx = fmaxf(max3f(qm[0], qm[1], qm[2]), max3f(qm[3], qm[4], qm[15])) * sm_scale_log2;
+                if (lane == 0) mbar_arrive(&sh.stag[t]);
+                if (n == 0) {
+                    m_run = mx;
+                } else if (__any_sync(0xffffffffu, mx > m_run + 8.0f)) {
+                    const float m_new = fmaxf(m_run, mx);
+                    const float alpha = fast_exp2(m_run - m_new);
+                    // O_t is stable once PV_t(gb-1) has completed
+                    if (!wait_all(&sh.pv_done[t], (gb - 1) & 1, 31)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        uint32_t o[32];
+                        tmem_ld32(o_addr + c0, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; c++) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                        tmem_st32(o_addr + c0, o);
                     }
-                    lacc[c & 3] = f2_add(lacc[c & 3], f2_pack(p0, p1));
-                    pk[c] = pack_bf16x2(p0, p1);
+                    tmem_wait_st();
+                    l *= alpha;
+                    m_run = m_new;
                 }
-                // P over S columns [c0/2, c0/2 + 16): S is held in registers
-                tmem_st16(s_addr + c0 / 2, pk);
+                // P = 2^(s*c - m), 1 of every 4 pairs on the FMA pipe, the
+                // rest on MUFU; packed bf16 P goes over the buffer's first
+                // 32 columns
+                const uint64_t nm2 = f2_pack(-m_run, -m_run);
+                uint64_t lacc[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+#pragma unroll
+                for (int c0 = 0; c0 < 64; c0 += 32) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int c = 0; c < 16; c++) {
+                        const uint64_t x2 = f2_fma(
+                            f2_pack(__uint_as_float(sr[c0 + 2 * c]), __uint_as_float(sr[c0 + 2 * c + 1])), sc2,
+                            nm2);
+                        float p0, p1;
+                        if ((c & 3) == 3) {
+                            f2_unpack(exp2_poly_x2(x2), p0, p1);
+                        } else {
+                            float x0, x1;
+                            f2_unpack(x2, x0, x1);
+                            p0 = fast_exp2(x0);
+                            p1 = fast_exp2(x1);
+                        }
+                        lacc[c & 3] = f2_add(lacc[c & 3], f2_pack(p0, p1));
+                        pk[c] = pack_bf16x2(p0, p1);
+                    }
+                    // P over S columns [c0/2, c0/2 + 16): S is held in registers
+                    tmem_st16(s_addr + c0 / 2, pk);
+                }
+                float la, lb;
+                f2_unpack(f2_add(f2_add(lacc[0], lacc[1]), f2_add(lacc[2], lacc[3])), la, lb);
+                l += la + lb;
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh.p_full[t][gb & 1]);
             }
-            float la, lb;
-            f2_unpack(f2_add(f2_add(lacc[0], lacc[1]), f2_add(lacc[2], lacc[3])), la, lb);
-            l += la + lb;
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.p_full[t][n & 1]);
-        }
-        if (ok && !mbar_wait(&sh.pv_done[t], (nblk - 1) & 1, abort, 32)) ok = false;
-        tc_fence_after();
-        const bool store = tok < Tq;
-        const int h = g * G + r % G;
-        __nv_bfloat16 *orow = O + (((long)b * Tq + tok) * Hq + h) * D;
-        const float inv_l = (ok && l > 0.f) ? 1.0f / l : 0.f;
+            if (!ok) break;
+            if (lane == 0) mbar_arrive(&sh.list_empty[slot]);
+            // epilogue: O_t / l once the unit's last PV is done.  The next
+            // unit's first PV overwrites O_t only after P of its block,
+            // which this warp signals after these loads.
+            if (!wait_all(&sh.pv_done[t], (g0 + nb - 1) & 1, 32)) { ok = false; break; }
+            tc_fence_after();
+            const float inv_l = (!none && l > 0.f) ? 1.0f / l : 0.f;
+            // O_t / l as bf16, one 64-column half at a time: each thread
+            // puts its row into the warp's staging rows (16-byte chunk c of
+            // row rr at chunk c ^ (rr % 8), so that both the row-wise writes
+            // and the column-wise reads below are free of bank conflicts),
+            // then every store instruction writes four whole 128-byte rows
+            uint4 *stage = reinterpret_cast<uint4 *>(o_stage + warp * C::STAGE_BYTES);
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(o_addr + c0, o);
-            tmem_wait_ld();
-            uint32_t pk[16];
+            for (int hh = 0; hh < C::NH; hh++) {
+                uint32_t o[64];
+                tmem_ld32(o_addr + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+                tmem_ld32(o_addr + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+                tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 16; c++)
-                pk[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
-            if (store) {
-                uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+                for (int c = 0; c < 8; c++) {
+                    uint32_t pk[4];
 #pragma unroll
-                for (int v = 0; v < 4; v++)
-                    dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    for (int e = 0; e < 4; e++)
+                        pk[e] = pack_bf16x2(__uint_as_float(o[8 * c + 2 * e]) * inv_l,
+                                            __uint_as_float(o[8 * c + 2 * e + 1]) * inv_l);
+                    stage[lane * 8 + (c ^ (lane & 7))] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int q = 0; q < 8; q++) {
+                    const int rr = 4 * q + (lane >> 3), c = lane & 7;
+                    const uint4 v = stage[rr * 8 + (c ^ (rr & 7))];
+                    const int row = ((warp & 3) << 5) + rr;     // tile row
+                    const int tk = w.token0 + t * C::TOK + row / G;
+                    if (tk < Tq)
+                        reinterpret_cast<uint4 *>(O + (((long)b * Tq + tk) * Hq + g * G + row % G) * D + hh * 64)[c] = v;
+                }
+                __syncwarp();
             }
+            const bool store = tok < Tq;
+            const int h = g * G + r % G;
+            if (store && lse)
+                lse[((long)b * Tq + tok) * Hq + h] =
+                    (!none && l > 0.f) ? (m_run + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+            g0 += nb;
+            k++;
         }
-        if (store && lse)
-            lse[((long)b * Tq + tok) * Hq + h] =
-                (ok && l > 0.f) ? (m_run + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (!ok) *abort = 1;   // a wait gave up: let the other roles' waits end at once
     }
 
     tc_fence_before();

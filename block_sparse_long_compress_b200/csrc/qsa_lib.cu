@@ -219,10 +219,11 @@ qsa_status launch_prefill(const void *Q, const void *K, const void *V, const int
     if ((st = make_map_2d(&mv, V, (uint64_t)B * Hkv * T_kv_max, D)) != QSA_OK) return st;
     auto kern = qsa::sparse_attn_prefill_kernel<D, G>;
     if ((st = set_smem(kern, C::SMEM_REQUEST)) != QSA_OK) return st;
-    const int NR = (Tq + 63) / 64;
-    dim3 grid(NR * C::TILES, B * Hkv);
+    // persistent: one CTA per SM (never more than there are work units)
+    const long units = (long)((Tq + 63) / 64) * C::TILES * B * Hkv;
+    const int grid = (int)std::min<long>(units, sm_count());
     kern<<<grid, C::THREADS, C::SMEM_REQUEST, s>>>(mq, mk, mv, idx, (__nv_bfloat16 *)O, lse, Tq, Hq, Hkv,
-                                                   q_pos0, T_kv_max, topk,
+                                                   B * Hkv, q_pos0, T_kv_max, topk,
                                                    sm_scale * 1.4426950408889634f);
     return launched("sparse_attn_prefill_kernel");
 }
