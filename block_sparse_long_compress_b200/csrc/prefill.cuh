@@ -304,9 +304,9 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
         const uint32_t o_tmem = tmem + C::O_COL + 128 * t;
         // S_t(gb) = Q_t K_gb^T into S buffer gb%2 (gb counts blocks across
         // units); after a unit's last S, a commit frees the Q tiles
-        auto issue_s = [&](int gb, bool last_of_unit) -> bool {
+        auto issue_s = [&](int gb, bool last_of_unit, bool wait_k) -> bool {
             const int st = gb % C::NS;
-            if (!wait_all(&sh.k_full[st], (gb / C::NS) & 1, 21)) return false;
+            if (wait_k && !wait_all(&sh.k_full[st], (gb / C::NS) & 1, 21)) return false;
             tc_fence_after();
             const uint64_t kds = kd + (uint64_t)((st * C::BLK_BYTES) >> 4);
             const uint32_t s_tmem = s_tmem0 + 64 * (gb & 1);
@@ -339,12 +339,23 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
         int u = next_unit(blockIdx.x);
         int k = 0, g0 = 0, nb = 0;   // unit, its first block, its length
         bool ok = u < U && unit_len(0, nb) && wait_all(&sh.q_full, 0, 20);
-        if (ok) ok = issue_s(0, nb == 1);
-        if (ok && nb > 1) ok = issue_s(1, nb == 2);
+        if (ok) ok = issue_s(0, nb == 1, true);
+        if (ok && nb > 1) ok = issue_s(1, nb == 2, true);
+        // An mbarrier wait by this thread holds up its MMA issue while the
+        // (short) queue of issued MMAs drains, so the checks that a block's V
+        // and the K two blocks ahead have landed are made one block early,
+        // while the softmax is still working on P; once P arrives, the PV and
+        // the next S go out back to back.
+        auto prefetch_checks = [&](int g0u, int nbu, int n) -> bool {
+            if (n < nbu && !wait_all(&sh.v_full[(g0u + n) % C::NS], ((g0u + n) / C::NS) & 1, 26)) return false;
+            if (n + 2 < nbu && !wait_all(&sh.k_full[(g0u + n + 2) % C::NS], ((g0u + n + 2) / C::NS) & 1, 21))
+                return false;
+            return true;
+        };
         while (ok) {
+            ok = prefetch_checks(g0, nb, 0);
             for (int n = 0; ok && n < nb; n++) {
                 const int gb = g0 + n, st = gb % C::NS;
-                if (!wait_all(&sh.v_full[st], (gb / C::NS) & 1, 26)) { ok = false; break; }
                 // the real dependency: this tile's P of the block
                 if (!wait_all(&sh.p_full[t][gb & 1], (gb >> 1) & 1, 22)) { ok = false; break; }
                 tc_fence_after();
@@ -361,7 +372,8 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
                 }
                 __syncwarp();
                 // S_t(gb+2) into the same buffer, right behind PV_t(gb)
-                if (n + 2 < nb && !issue_s(gb + 2, n + 3 == nb)) ok = false;
+                if (n + 2 < nb && !issue_s(gb + 2, n + 3 == nb, false)) ok = false;
+                if (ok) ok = prefetch_checks(g0, nb, n + 1);
             }
             if (!ok) break;
             // the next unit: its length, its Q tiles, its first two S
@@ -370,8 +382,8 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
             k++;
             g0 += nb;
             if (!unit_len(k, nb) || !wait_all(&sh.q_full, k & 1, 20)) break;
-            if (!issue_s(g0, nb == 1)) break;
-            if (nb > 1 && !issue_s(g0 + 1, nb == 2)) break;
+            if (!issue_s(g0, nb == 1, true)) break;
+            if (nb > 1 && !issue_s(g0 + 1, nb == 2, true)) break;
         }
     }
     } else {
