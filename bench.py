@@ -298,10 +298,16 @@ def run_qsa(args, ws, rank, local):
         del Q, K, V, run, x
         torch.cuda.empty_cache()
         result["decode"] = bench_decode(args, qsa, dev, peaks, ws, rank, flush)
+        if args.bf16_summaries:
+            result["decode"]["bf16_summaries"] = bench_decode(args, qsa, dev, peaks, ws, rank, flush,
+                                                              summary="bf16")
         for name in filter(None, args.decode_more.split(",")):
             torch.cuda.empty_cache()
             result.setdefault("decode_more", {})[name] = bench_decode(args, qsa, dev, peaks, ws,
                                                                       rank, flush, name)
+            if args.bf16_summaries:
+                result["decode_more"][name]["bf16_summaries"] = bench_decode(
+                    args, qsa, dev, peaks, ws, rank, flush, name, summary="bf16")
 
     # ---- e2e through the public API with host buffers
     if not args.no_e2e:
@@ -309,7 +315,7 @@ def run_qsa(args, ws, rank, local):
     return result
 
 
-def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None):
+def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary="fp32"):
     wd = synthetic.CONFIGS[workload or args.decode_workload]
     if args.decode_batch:
         wd = synthetic.Workload(**{**wd.__dict__, "B": args.decode_batch})
@@ -319,7 +325,8 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None):
     q = x["Q"].view(wd.B, wd.Hq, wd.d)
     K, V = x["K"], x["V"]
     L = wd.q_pos0 + 1
-    dec = qsa.QSADecode(wd.B, wd.Hq, wd.Hkv, wd.d, wd.T_kv, wd.topk, device=dev)
+    sdt = torch.bfloat16 if summary == "bf16" else torch.float32
+    dec = qsa.QSADecode(wd.B, wd.Hq, wd.Hkv, wd.d, wd.T_kv, wd.topk, device=dev, summary_dtype=sdt)
     dec.compress(K, 0, L // 64)           # persistent summaries (untimed)
     for _ in range(args.warmup):
         dec(q, K, V, L)
@@ -405,8 +412,9 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None):
     us_step, us_att, us_sel = d["step"], d["attention"], d["select"]
     by = decode_bytes(wd)
     att_gbs = by / (us_att * 1e-6) / 1e9
-    sel_bytes = wd.B * wd.Hkv * ((L - 1) // 64) * wd.d * 4   # fp32 summaries read by scoring
-    return {"workload": wd.name, "batch": wd.B, "context": L, "topk": wd.topk,
+    # summaries read by scoring (fp32, or bf16 for the bf16-summary option)
+    sel_bytes = wd.B * wd.Hkv * ((L - 1) // 64) * wd.d * (2 if summary == "bf16" else 4)
+    return {"workload": wd.name, "batch": wd.B, "context": L, "topk": wd.topk, "summaries": summary,
             "us_per_step": us_step, "us_per_token": us_step / wd.B,
             "timing": ("per step: R back-to-back replays of a CUDA graph (L2 flush, step kernels) "
                        "minus R replays of (L2 flush) alone, events around each set"),
@@ -535,6 +543,8 @@ def main():
     ap.add_argument("--decode-more", default="decode_262k",
                     help="comma list of further decode workloads reported under decode_more")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-bf16-summaries", dest="bf16_summaries", action="store_false",
+                    help="skip the decode run with the bf16-summary option (reported beside the fp32 one)")
     ap.add_argument("--only-decode", action="store_true",
                     help="skip the prefill measurement (profiling the decode kernels)")
     ap.add_argument("--decode-batch", type=int, default=None,
@@ -567,10 +577,15 @@ def main():
         torch.cuda.set_device(dev)
         flush = L2Flush(dev)
         res = bench_decode(args, qsa, dev, load_peaks(), ws, rank, flush)
+        if args.bf16_summaries:
+            res["bf16_summaries"] = bench_decode(args, qsa, dev, load_peaks(), ws, rank, flush, summary="bf16")
         for name in filter(None, args.decode_more.split(",")):
             torch.cuda.empty_cache()
             res.setdefault("decode_more", {})[name] = bench_decode(args, qsa, dev, load_peaks(), ws,
                                                                    rank, flush, name)
+            if args.bf16_summaries:
+                res["decode_more"][name]["bf16_summaries"] = bench_decode(
+                    args, qsa, dev, load_peaks(), ws, rank, flush, name, summary="bf16")
         if rank == 0:
             print(json.dumps(res), flush=True)
         return

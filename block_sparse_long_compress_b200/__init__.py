@@ -45,8 +45,10 @@ def _load():
     P, I, S, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
     sig = {
         "qsa_compress_keys": (I, [P, P, I, I, I, I, I, I, P]),
+        "qsa_compress_keys_bf16": (I, [P, P, I, I, I, I, I, I, P]),
         "qsa_score_select_workspace": (S, [I, I, I, I, I, I, I, I]),
         "qsa_score_select": (I, [P, P, P, I, I, I, I, I, I, I, I, I, F, P, S, P]),
+        "qsa_score_select_bf16": (I, [P, P, P, I, I, I, I, I, I, I, I, I, F, P, S, P]),
         "qsa_score_select_noalloc": (I, [P, P, P, I, I, I, I, I, I, I, I, I, F, P]),
         "qsa_sparse_attn_prefill": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P]),
         "qsa_decode_workspace": (S, [I, I, I, I, I]),
@@ -103,17 +105,26 @@ def _ptr(t, dtype, name):
 
 
 # ------------------------------------------------------------------ steps
+def _summary_fn(Kc, fp32_fn, bf16_fn):
+    """The entry point for the summaries' dtype: fp32 (default) or bf16."""
+    if isinstance(Kc, torch.Tensor) and Kc.dtype == torch.bfloat16:
+        return bf16_fn, torch.bfloat16
+    return fp32_fn, torch.float32
+
+
 def compress_keys(K, Kc, blk_begin=0, blk_end=None, stream=None):
     """Kc[b,h,j,:] = mean of K[b,h,64j:64j+64,:] for j in [blk_begin, blk_end).
-    K: bf16 [B, Hkv, T_kv_max, d]; Kc: fp32 [B, Hkv, T_kv_max//64, d]."""
+    K: bf16 [B, Hkv, T_kv_max, d]; Kc: fp32 [B, Hkv, T_kv_max//64, d], or bf16
+    for the bf16-summary option (the fp32 mean rounded to nearest even)."""
     B, Hkv, T, d = K.shape
     if blk_end is None:
         blk_end = T // BLOCK
     if tuple(Kc.shape) != (B, Hkv, T // BLOCK, d):
         raise ValueError("Kc shape must be [B, Hkv, T_kv_max//64, d]")
-    _check(_lib.qsa_compress_keys(_ptr(K, torch.bfloat16, "K"), _ptr(Kc, torch.float32, "Kc"),
-                                  B, Hkv, T, d, blk_begin, blk_end, _stream(stream)),
-           "qsa_compress_keys")
+    fn, kdt = _summary_fn(Kc, _lib.qsa_compress_keys, _lib.qsa_compress_keys_bf16)
+    _check(fn(_ptr(K, torch.bfloat16, "K"), _ptr(Kc, kdt, "Kc"),
+              B, Hkv, T, d, blk_begin, blk_end, _stream(stream)),
+           fn.__name__)
     return Kc
 
 
@@ -124,7 +135,7 @@ def score_select_workspace(B, Hq, Hkv, Tq, q_pos0, qblk, d, topk):
 def score_select(Q, Kc, idx, topk, q_pos0, qblk=BLOCK, sm_scale=None, workspace=None,
                  stream=None):
     """Top-k block selection per (query block or token, KV group).
-    Q: bf16 [B, Tq, Hq, d]; Kc: fp32 [B, Hkv, T_kv_max//64, d];
+    Q: bf16 [B, Tq, Hq, d]; Kc: fp32 (or bf16) [B, Hkv, T_kv_max//64, d];
     idx: int32 [B, Hkv, ceil(Tq/qblk), topk] (written)."""
     B, Tq, Hq, d = Q.shape
     _, Hkv, nblk, _ = Kc.shape
@@ -133,12 +144,13 @@ def score_select(Q, Kc, idx, topk, q_pos0, qblk=BLOCK, sm_scale=None, workspace=
     need = score_select_workspace(B, Hq, Hkv, Tq, q_pos0, qblk, d, topk)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
-    _check(_lib.qsa_score_select(_ptr(Q, torch.bfloat16, "Q"), _ptr(Kc, torch.float32, "Kc"),
-                                 _ptr(idx, torch.int32, "idx"), B, Hq, Hkv, Tq, q_pos0, qblk,
-                                 nblk * BLOCK, d, topk, float(sm_scale),
-                                 _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
-                                 _stream(stream)),
-           "qsa_score_select")
+    fn, kdt = _summary_fn(Kc, _lib.qsa_score_select, _lib.qsa_score_select_bf16)
+    _check(fn(_ptr(Q, torch.bfloat16, "Q"), _ptr(Kc, kdt, "Kc"),
+              _ptr(idx, torch.int32, "idx"), B, Hq, Hkv, Tq, q_pos0, qblk,
+              nblk * BLOCK, d, topk, float(sm_scale),
+              _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+              _stream(stream)),
+           fn.__name__)
     return idx
 
 
@@ -207,13 +219,13 @@ class QSAPrefill:
     (allocated once with torch)."""
 
     def __init__(self, B, Tq, Hq, Hkv, d, T_kv_max, topk, q_pos0=0, device="cuda",
-                 with_lse=False):
+                 with_lse=False, summary_dtype=torch.float32):
         self.B, self.Tq, self.Hq, self.Hkv, self.d = B, Tq, Hq, Hkv, d
         self.T_kv_max, self.topk, self.q_pos0 = T_kv_max, topk, q_pos0
         self.sm_scale = d ** -0.5
         NR = -(-Tq // BLOCK)
         dev = torch.device(device)
-        self.Kc = torch.zeros((B, Hkv, T_kv_max // BLOCK, d), dtype=torch.float32, device=dev)
+        self.Kc = torch.zeros((B, Hkv, T_kv_max // BLOCK, d), dtype=summary_dtype, device=dev)
         self.idx = torch.empty((B, Hkv, NR, topk), dtype=torch.int32, device=dev)
         self.O = torch.empty((B, Tq, Hq, d), dtype=torch.bfloat16, device=dev)
         self.lse = (torch.empty((B, Tq, Hq), dtype=torch.float32, device=dev)
@@ -297,12 +309,13 @@ class QSADecode:
     (per token) then split-K attention.  Summaries of complete blocks are
     persistent state; compress_block() adds one as it completes."""
 
-    def __init__(self, B, Hq, Hkv, d, T_kv_max, topk, device="cuda"):
+    def __init__(self, B, Hq, Hkv, d, T_kv_max, topk, device="cuda", summary_dtype=torch.float32):
         self.B, self.Hq, self.Hkv, self.d = B, Hq, Hkv, d
         self.T_kv_max, self.topk = T_kv_max, topk
         self.sm_scale = d ** -0.5
         dev = torch.device(device)
-        self.Kc = torch.zeros((B, Hkv, T_kv_max // BLOCK, d), dtype=torch.float32, device=dev)
+        # summaries: fp32, or bf16 (half the bytes the per-token selection reads)
+        self.Kc = torch.zeros((B, Hkv, T_kv_max // BLOCK, d), dtype=summary_dtype, device=dev)
         self.idx = torch.empty((B, Hkv, 1, topk), dtype=torch.int32, device=dev)
         self.o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
         n = decode_workspace(B, Hq, Hkv, d, topk)

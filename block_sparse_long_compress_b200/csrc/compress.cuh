@@ -9,15 +9,20 @@
 // t % (d/8) and the rows r = t / (d/8) + k*R (R = 128 / (d/8) row lanes),
 // issuing all its loads before the first add.  The reduction order is fixed
 // (each thread adds its rows in increasing r, then row lanes are added in
-// increasing lane order), so results are bit-reproducible.
+// increasing lane order), so results are bit-reproducible.  The summary is
+// stored as fp32, or (the bf16-summary option) as that fp32 mean rounded to
+// the nearest bf16, ties to even -- half the bytes for the scoring to read.
 #pragma once
 #include "device.cuh"
 
 namespace qsa {
 
-template <int D>
+__device__ __forceinline__ void store_summary(float *p, float v) { *p = v; }
+__device__ __forceinline__ void store_summary(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+template <int D, typename KcT>
 __global__ void __launch_bounds__(128) compress_keys_kernel(const __nv_bfloat16 *__restrict__ K,
-                                                            float *__restrict__ Kc, int T_kv_max,
+                                                            KcT *__restrict__ Kc, int T_kv_max,
                                                             int nblk_max, int blk_begin,
                                                             int nblk)
 {
@@ -56,7 +61,7 @@ __global__ void __launch_bounds__(128) compress_keys_kernel(const __nv_bfloat16 
         float s = 0.f;
 #pragma unroll
         for (int l = 0; l < LANES; l++) s += part[l][t];
-        Kc[(bh * nblk_max + j) * D + t] = s * (1.0f / 64.0f);
+        store_summary(Kc + (bh * nblk_max + j) * D + t, s * (1.0f / 64.0f));
     }
 }
 

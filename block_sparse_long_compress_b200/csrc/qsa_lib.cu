@@ -261,12 +261,12 @@ qsa_status launch_decode(const void *q, const void *K, const void *V, const int3
     return launched("decode_kernel");
 }
 
-template <int D>
-qsa_status launch_select_token_d(const void *Q, const float *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
+template <int D, typename KcT>
+qsa_status launch_select_token_d(const void *Q, const KcT *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
                                  int q_pos0, int nblk_max, int topk, float sm_scale, const TokenPlan &tp,
                                  cudaStream_t s)
 {
-    auto kern = qsa::select_token_kernel<D>;
+    auto kern = qsa::select_token_kernel<D, KcT>;
     const int smem = tp.CH * 8;
     qsa_status st;
     if ((st = set_smem(kern, smem)) != QSA_OK) return st;
@@ -290,12 +290,14 @@ qsa_status launch_select_token_d(const void *Q, const float *Kc, int32_t *idx, i
     return launched("select_token_kernel");
 }
 
-qsa_status launch_select_token(const void *Q, const float *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
+template <typename KcT>
+qsa_status launch_select_token(const void *Q, const KcT *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
                                int q_pos0, int nblk_max, int d, int topk, float sm_scale, const TokenPlan &tp,
                                cudaStream_t s)
 {
-    if (d == 128) return launch_select_token_d<128>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, nblk_max, topk, sm_scale, tp, s);
-    return launch_select_token_d<64>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, nblk_max, topk, sm_scale, tp, s);
+    if (d == 128)
+        return launch_select_token_d<128, KcT>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, nblk_max, topk, sm_scale, tp, s);
+    return launch_select_token_d<64, KcT>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, nblk_max, topk, sm_scale, tp, s);
 }
 
 __global__ void selftest_exp2_kernel(const float *__restrict__ x, float *__restrict__ y, int n)
@@ -360,33 +362,117 @@ qsa_status select_scratch_address(void **out)
 
 }  // namespace
 
+namespace {
+
+template <typename KcT>
+qsa_status compress_keys_impl(const char *name, const void *K, KcT *Kc, int B, int Hkv, int T_kv_max, int d,
+                              int blk_begin, int blk_end, qsa_stream_t stream)
+{
+    if (!K || !Kc) return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (B <= 0 || Hkv <= 0 || T_kv_max <= 0 || T_kv_max % 64)
+        return fail(QSA_ERR_INVALID_ARG, "%s: bad shape", name);
+    const int nblk_max = T_kv_max / 64;
+    if (blk_begin < 0 || blk_end < blk_begin || blk_end > nblk_max)
+        return fail(QSA_ERR_INVALID_ARG, "%s: block range [%d,%d) outside [0,%d]", name, blk_begin,
+                    blk_end, nblk_max);
+    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "%s: d=%d", name, d);
+    if (!aligned16(K) || !aligned16(Kc)) return fail(QSA_ERR_INVALID_ARG, "%s: misaligned", name);
+    const int nblk = blk_end - blk_begin;
+    if (nblk == 0) return QSA_OK;
+    const long grid = (long)B * Hkv * nblk;
+    if (grid >= (1L << 31)) return fail(QSA_ERR_UNSUPPORTED, "%s: too many blocks", name);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 128)
+        qsa::compress_keys_kernel<128, KcT><<<(unsigned)grid, 128, 0, s>>>((const __nv_bfloat16 *)K, Kc, T_kv_max,
+                                                                      nblk_max, blk_begin, nblk);
+    else
+        qsa::compress_keys_kernel<64, KcT><<<(unsigned)grid, 128, 0, s>>>((const __nv_bfloat16 *)K, Kc, T_kv_max,
+                                                                     nblk_max, blk_begin, nblk);
+    return launched("compress_keys_kernel");
+}
+
+
+template <typename KcT>
+qsa_status score_select_impl(const char *name, const void *Q, const KcT *Kc, int32_t *idx, int B, int Hq, int Hkv,
+                             int Tq, int q_pos0, int qblk, int T_kv_max, int d, int topk, float sm_scale,
+                             void *workspace, size_t workspace_bytes, qsa_stream_t stream)
+{
+    if (!Q || !Kc || !idx) return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || T_kv_max <= 0 || T_kv_max % 64 ||
+        Hq % Hkv)
+        return fail(QSA_ERR_INVALID_ARG, "%s: bad shape", name);
+    if (qblk != 1 && qblk != 64) return fail(QSA_ERR_UNSUPPORTED, "%s: qblk=%d", name, qblk);
+    if (qblk == 64 && q_pos0 % 64)
+        return fail(QSA_ERR_INVALID_ARG, "%s: q_pos0 must be a multiple of 64 when qblk=64", name);
+    if ((long)q_pos0 + Tq > T_kv_max) return fail(QSA_ERR_INVALID_ARG, "%s: queries past the cache", name);
+    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "%s: d=%d", name, d);
+    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "%s: topk=%d", name, topk);
+    if ((long)Hq * d / 8 > 1024) return fail(QSA_ERR_UNSUPPORTED, "%s: Hq*d too large", name);
+    if (!aligned16(Q) || !aligned16(Kc) || !aligned16(idx))
+        return fail(QSA_ERR_INVALID_ARG, "%s: misaligned pointer", name);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const TokenPlan tp = plan_token(B, Hkv, Tq, q_pos0, qblk);
+    if (tp.use) return launch_select_token(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, T_kv_max / 64, d, topk, sm_scale,
+                                           tp, s);
+    const SelectPlan p = plan_select(B, Hkv, Tq, q_pos0, qblk, d);
+    if (p.maxchunks * qsa::kMaxChosen * 8 > 200 * 1024)
+        return fail(QSA_ERR_UNSUPPORTED, "%s: context too long", name);
+    if (!workspace || workspace_bytes < p.qbar_bytes + p.part_bytes || !aligned16(workspace))
+        return fail(QSA_ERR_WORKSPACE, "%s: workspace needs %zu bytes", name,
+                    p.qbar_bytes + p.part_bytes);
+    float *Qbar = static_cast<float *>(workspace);
+    uint64_t *part = reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(workspace) + p.qbar_bytes);
+    const int nblk_max = T_kv_max / 64;
+    const int pool_threads = ((Hq * d / 8) + 31) / 32 * 32;
+    const int pool_smem = Hq * d * 4;
+    dim3 pgrid(p.NR, B), sgrid(p.maxchunks, p.NR, B * Hkv), mgrid(p.NR, B * Hkv);
+    const int ssmem = p.CH * 8;
+    qsa_status st;
+    if (d == 128) {
+        if ((st = set_smem(qsa::pool_queries_kernel<128>, pool_smem)) != QSA_OK) return st;
+        qsa::pool_queries_kernel<128><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq,
+                                                                             Hq, Hkv, qblk);
+        if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
+        if ((st = set_smem(qsa::score_select_kernel<128, KcT>, ssmem)) != QSA_OK) return st;
+        qsa::score_select_kernel<128, KcT><<<sgrid, qsa::kSelThreads, ssmem, s>>>(
+            Qbar, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk, sm_scale, p.CH, p.maxchunks);
+    } else {
+        if ((st = set_smem(qsa::pool_queries_kernel<64>, pool_smem)) != QSA_OK) return st;
+        qsa::pool_queries_kernel<64><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq,
+                                                                            Hq, Hkv, qblk);
+        if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
+        if ((st = set_smem(qsa::score_select_kernel<64, KcT>, ssmem)) != QSA_OK) return st;
+        qsa::score_select_kernel<64, KcT><<<sgrid, qsa::kSelThreads, ssmem, s>>>(
+            Qbar, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk, sm_scale, p.CH, p.maxchunks);
+    }
+    if ((st = launched("score_select_kernel")) != QSA_OK) return st;
+    if (p.maxchunks > 1) {
+        const int msmem = p.maxchunks * qsa::kMaxChosen * 8;
+        if ((st = set_smem(qsa::merge_select_kernel, msmem)) != QSA_OK) return st;
+        qsa::merge_select_kernel<<<mgrid, qsa::kSelThreads, msmem, s>>>(part, idx, Tq, q_pos0, qblk, topk, p.CH,
+                                                                       p.maxchunks);
+        if ((st = launched("merge_select_kernel")) != QSA_OK) return st;
+    }
+    return QSA_OK;
+}
+
+
+}  // namespace
+
 // ===================================================================== C ABI
 extern "C" {
 
 qsa_status qsa_compress_keys(const void *K, float *Kc, int B, int Hkv, int T_kv_max, int d, int blk_begin,
                              int blk_end, qsa_stream_t stream)
 {
-    if (!K || !Kc) return fail(QSA_ERR_INVALID_ARG, "qsa_compress_keys: null pointer");
-    if (B <= 0 || Hkv <= 0 || T_kv_max <= 0 || T_kv_max % 64)
-        return fail(QSA_ERR_INVALID_ARG, "qsa_compress_keys: bad shape");
-    const int nblk_max = T_kv_max / 64;
-    if (blk_begin < 0 || blk_end < blk_begin || blk_end > nblk_max)
-        return fail(QSA_ERR_INVALID_ARG, "qsa_compress_keys: block range [%d,%d) outside [0,%d]", blk_begin,
-                    blk_end, nblk_max);
-    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "qsa_compress_keys: d=%d", d);
-    if (!aligned16(K) || !aligned16(Kc)) return fail(QSA_ERR_INVALID_ARG, "qsa_compress_keys: misaligned");
-    const int nblk = blk_end - blk_begin;
-    if (nblk == 0) return QSA_OK;
-    const long grid = (long)B * Hkv * nblk;
-    if (grid >= (1L << 31)) return fail(QSA_ERR_UNSUPPORTED, "qsa_compress_keys: too many blocks");
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (d == 128)
-        qsa::compress_keys_kernel<128><<<(unsigned)grid, 128, 0, s>>>((const __nv_bfloat16 *)K, Kc, T_kv_max,
-                                                                      nblk_max, blk_begin, nblk);
-    else
-        qsa::compress_keys_kernel<64><<<(unsigned)grid, 128, 0, s>>>((const __nv_bfloat16 *)K, Kc, T_kv_max,
-                                                                     nblk_max, blk_begin, nblk);
-    return launched("compress_keys_kernel");
+    return compress_keys_impl("qsa_compress_keys", K, Kc, B, Hkv, T_kv_max, d, blk_begin, blk_end, stream);
+}
+
+qsa_status qsa_compress_keys_bf16(const void *K, void *Kc, int B, int Hkv, int T_kv_max, int d, int blk_begin,
+                                  int blk_end, qsa_stream_t stream)
+{
+    return compress_keys_impl("qsa_compress_keys_bf16", K, static_cast<__nv_bfloat16 *>(Kc), B, Hkv, T_kv_max, d,
+                              blk_begin, blk_end, stream);
 }
 
 size_t qsa_score_select_workspace(int B, int Hq, int Hkv, int Tq, int q_pos0, int qblk, int d, int topk)
@@ -403,63 +489,16 @@ qsa_status qsa_score_select(const void *Q, const float *Kc, int32_t *idx, int B,
                             int q_pos0, int qblk, int T_kv_max, int d, int topk, float sm_scale,
                             void *workspace, size_t workspace_bytes, qsa_stream_t stream)
 {
-    if (!Q || !Kc || !idx) return fail(QSA_ERR_INVALID_ARG, "qsa_score_select: null pointer");
-    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || T_kv_max <= 0 || T_kv_max % 64 ||
-        Hq % Hkv)
-        return fail(QSA_ERR_INVALID_ARG, "qsa_score_select: bad shape");
-    if (qblk != 1 && qblk != 64) return fail(QSA_ERR_UNSUPPORTED, "qsa_score_select: qblk=%d", qblk);
-    if (qblk == 64 && q_pos0 % 64)
-        return fail(QSA_ERR_INVALID_ARG, "qsa_score_select: q_pos0 must be a multiple of 64 when qblk=64");
-    if ((long)q_pos0 + Tq > T_kv_max) return fail(QSA_ERR_INVALID_ARG, "qsa_score_select: queries past the cache");
-    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "qsa_score_select: d=%d", d);
-    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "qsa_score_select: topk=%d", topk);
-    if ((long)Hq * d / 8 > 1024) return fail(QSA_ERR_UNSUPPORTED, "qsa_score_select: Hq*d too large");
-    if (!aligned16(Q) || !aligned16(Kc) || !aligned16(idx))
-        return fail(QSA_ERR_INVALID_ARG, "qsa_score_select: misaligned pointer");
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const TokenPlan tp = plan_token(B, Hkv, Tq, q_pos0, qblk);
-    if (tp.use) return launch_select_token(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, T_kv_max / 64, d, topk, sm_scale,
-                                           tp, s);
-    const SelectPlan p = plan_select(B, Hkv, Tq, q_pos0, qblk, d);
-    if (p.maxchunks * qsa::kMaxChosen * 8 > 200 * 1024)
-        return fail(QSA_ERR_UNSUPPORTED, "qsa_score_select: context too long");
-    if (!workspace || workspace_bytes < p.qbar_bytes + p.part_bytes || !aligned16(workspace))
-        return fail(QSA_ERR_WORKSPACE, "qsa_score_select: workspace needs %zu bytes",
-                    p.qbar_bytes + p.part_bytes);
-    float *Qbar = static_cast<float *>(workspace);
-    uint64_t *part = reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(workspace) + p.qbar_bytes);
-    const int nblk_max = T_kv_max / 64;
-    const int pool_threads = ((Hq * d / 8) + 31) / 32 * 32;
-    const int pool_smem = Hq * d * 4;
-    dim3 pgrid(p.NR, B), sgrid(p.maxchunks, p.NR, B * Hkv), mgrid(p.NR, B * Hkv);
-    const int ssmem = p.CH * 8;
-    qsa_status st;
-    if (d == 128) {
-        if ((st = set_smem(qsa::pool_queries_kernel<128>, pool_smem)) != QSA_OK) return st;
-        qsa::pool_queries_kernel<128><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq,
-                                                                             Hq, Hkv, qblk);
-        if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
-        if ((st = set_smem(qsa::score_select_kernel<128>, ssmem)) != QSA_OK) return st;
-        qsa::score_select_kernel<128><<<sgrid, qsa::kSelThreads, ssmem, s>>>(
-            Qbar, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk, sm_scale, p.CH, p.maxchunks);
-    } else {
-        if ((st = set_smem(qsa::pool_queries_kernel<64>, pool_smem)) != QSA_OK) return st;
-        qsa::pool_queries_kernel<64><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq,
-                                                                            Hq, Hkv, qblk);
-        if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
-        if ((st = set_smem(qsa::score_select_kernel<64>, ssmem)) != QSA_OK) return st;
-        qsa::score_select_kernel<64><<<sgrid, qsa::kSelThreads, ssmem, s>>>(
-            Qbar, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk, sm_scale, p.CH, p.maxchunks);
-    }
-    if ((st = launched("score_select_kernel")) != QSA_OK) return st;
-    if (p.maxchunks > 1) {
-        const int msmem = p.maxchunks * qsa::kMaxChosen * 8;
-        if ((st = set_smem(qsa::merge_select_kernel, msmem)) != QSA_OK) return st;
-        qsa::merge_select_kernel<<<mgrid, qsa::kSelThreads, msmem, s>>>(part, idx, Tq, q_pos0, qblk, topk, p.CH,
-                                                                       p.maxchunks);
-        if ((st = launched("merge_select_kernel")) != QSA_OK) return st;
-    }
-    return QSA_OK;
+    return score_select_impl("qsa_score_select", Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, qblk, T_kv_max, d, topk,
+                             sm_scale, workspace, workspace_bytes, stream);
+}
+
+qsa_status qsa_score_select_bf16(const void *Q, const void *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
+                                 int q_pos0, int qblk, int T_kv_max, int d, int topk, float sm_scale,
+                                 void *workspace, size_t workspace_bytes, qsa_stream_t stream)
+{
+    return score_select_impl("qsa_score_select_bf16", Q, static_cast<const __nv_bfloat16 *>(Kc), idx, B, Hq, Hkv,
+                             Tq, q_pos0, qblk, T_kv_max, d, topk, sm_scale, workspace, workspace_bytes, stream);
 }
 
 qsa_status qsa_score_select_noalloc(const void *Q, const float *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,

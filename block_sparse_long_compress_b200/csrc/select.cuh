@@ -265,13 +265,40 @@ __device__ __forceinline__ RowGeom row_geom(int i, int Tq, int q_pos0, int qblk,
     return g;
 }
 
-// fp32 scores of n candidates (block summaries kc[0..n) of d = D floats,
-// block ids j0..j0+n-1) against the pooled query qb, as 64-bit keys.  Each
-// warp takes 8 candidates at a time; lane owns columns [lane*V, lane*V+V);
-// a transposing butterfly leaves candidate (lane >> 2) of the group in
-// lanes with (lane & 3) == 0.
-template <int D>
-__device__ __forceinline__ void score_chunk(const float *qb, const float *__restrict__ kc, int n, int j0,
+// V consecutive summary components as fp32: fp32 summaries as they are,
+// bf16 summaries widened exactly (the scoring arithmetic is fp32 either way).
+template <int V>
+__device__ __forceinline__ void load_summary(const float *p, float (&k)[V])
+{
+    if constexpr (V == 4) {
+        const float4 k4 = __ldg(reinterpret_cast<const float4 *>(p));
+        k[0] = k4.x, k[1] = k4.y, k[2] = k4.z, k[3] = k4.w;
+    } else {
+        const float2 k2 = __ldg(reinterpret_cast<const float2 *>(p));
+        k[0] = k2.x, k[1] = k2.y;
+    }
+}
+
+template <int V>
+__device__ __forceinline__ void load_summary(const __nv_bfloat16 *p, float (&k)[V])
+{
+    if constexpr (V == 4) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+        k[0] = __uint_as_float(u.x << 16), k[1] = __uint_as_float(u.x & 0xFFFF0000u);
+        k[2] = __uint_as_float(u.y << 16), k[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    } else {
+        const uint32_t u = __ldg(reinterpret_cast<const unsigned int *>(p));
+        k[0] = __uint_as_float(u << 16), k[1] = __uint_as_float(u & 0xFFFF0000u);
+    }
+}
+
+// fp32 scores of n candidates (block summaries kc[0..n) of d = D fp32 or
+// bf16 components, block ids j0..j0+n-1) against the pooled query qb, as
+// 64-bit keys.  Each warp takes 8 candidates at a time; lane owns columns
+// [lane*V, lane*V+V); a transposing butterfly leaves candidate (lane >> 2)
+// of the group in lanes with (lane & 3) == 0.
+template <int D, typename KcT>
+__device__ __forceinline__ void score_chunk(const float *qb, const KcT *__restrict__ kc, int n, int j0,
                                             float sm_scale, uint64_t *keys)
 {
     constexpr int V = D / 32;
@@ -279,21 +306,17 @@ __device__ __forceinline__ void score_chunk(const float *qb, const float *__rest
     float q[V];
 #pragma unroll
     for (int v = 0; v < V; v++) q[v] = qb[lane * V + v];
-    const float *kc_base = kc + lane * V;
+    const KcT *kc_base = kc + lane * V;
     for (int base = warp * 8; base < n; base += 8 * (kSelThreads / 32)) {
         float s[8];
 #pragma unroll
         for (int c = 0; c < 8; c++) {
             s[c] = 0.f;
             if (base + c < n) {
-                const float *p = kc_base + (long)(base + c) * D;
-                if constexpr (V == 4) {
-                    const float4 k4 = __ldg(reinterpret_cast<const float4 *>(p));
-                    s[c] = q[0] * k4.x + q[1] * k4.y + q[2] * k4.z + q[3] * k4.w;
-                } else {
-                    const float2 k2 = __ldg(reinterpret_cast<const float2 *>(p));
-                    s[c] = q[0] * k2.x + q[1] * k2.y;
-                }
+                float k[V];
+                load_summary<V>(kc_base + (long)(base + c) * D, k);
+                if constexpr (V == 4) s[c] = q[0] * k[0] + q[1] * k[1] + q[2] * k[2] + q[3] * k[3];
+                else s[c] = q[0] * k[0] + q[1] * k[1];
             }
         }
 #pragma unroll
@@ -325,9 +348,9 @@ __device__ __forceinline__ void score_chunk(const float *qb, const float *__rest
 
 // --------------------------------------------------------- score+select
 // grid (maxchunks, NR, B*Hkv); dynamic smem CH * 8 bytes.
-template <int D>
+template <int D, typename KcT>
 __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
-    const float *__restrict__ Qbar, const float *__restrict__ Kc, int32_t *__restrict__ idx,
+    const float *__restrict__ Qbar, const KcT *__restrict__ Kc, int32_t *__restrict__ idx,
     uint64_t *__restrict__ part, int nblk_max, int Tq, int q_pos0, int qblk, int topk,
     float sm_scale, int CH, int maxchunks)
 {
@@ -340,7 +363,7 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
     const int n = max(0, min(CH, g.ncand - chunk * CH));
     const long row = (long)bg * NR + i;
 
-    score_chunk<D>(Qbar + row * D, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
+    score_chunk<D, KcT>(Qbar + row * D, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
     __syncthreads();
 
     const int need = min(g.m, n);
@@ -384,9 +407,9 @@ __global__ void __launch_bounds__(kSelThreads) merge_select_kernel(
 // below every score's key).  After one cluster barrier the other CTAs are
 // done and the leader selects the row's top-m from the lists, which are in
 // block order.
-template <int D>
+template <int D, typename KcT>
 __global__ void __launch_bounds__(kSelThreads) select_token_kernel(
-    const __nv_bfloat16 *__restrict__ Q, const float *__restrict__ Kc, int32_t *__restrict__ idx,
+    const __nv_bfloat16 *__restrict__ Q, const KcT *__restrict__ Kc, int32_t *__restrict__ idx,
     int nblk_max, int Tq, int Hq, int Hkv, int q_pos0, int topk, float sm_scale, int CH)
 {
     namespace cg = cooperative_groups;
@@ -418,7 +441,7 @@ __global__ void __launch_bounds__(kSelThreads) select_token_kernel(
     __syncthreads();
     const int j0 = 1 + chunk * CH;
     const int n = max(0, min(CH, g.ncand - chunk * CH));
-    score_chunk<D>(qbar, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
+    score_chunk<D, KcT>(qbar, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
     __syncthreads();
     const int need = min(g.m, n);
     if (g.nchunks == 1) {

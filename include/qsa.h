@@ -86,6 +86,16 @@ QSA_API qsa_status qsa_compress_keys(const void *K, float *Kc, int B, int Hkv, i
                              int d, int blk_begin, int blk_end, qsa_stream_t stream);
 
 /*
+ * Step 1 with bf16 summaries (an option; the default summaries are fp32):
+ * the same fp32 mean, stored rounded to the nearest bf16 (ties to even), so
+ * that scoring reads half the bytes -- the selection read of a long decode
+ * cache is as large as the attention's.  Kc is bf16
+ * [B][Hkv][T_kv_max/64][d]; everything else as qsa_compress_keys.
+ */
+QSA_API qsa_status qsa_compress_keys_bf16(const void *K, void *Kc, int B, int Hkv, int T_kv_max,
+                                          int d, int blk_begin, int blk_end, qsa_stream_t stream);
+
+/*
  * Steps 2-4: pool queries, score the block summaries and select the top-k
  * blocks ("indexer scoring" -> "top-k selection").
  *
@@ -109,6 +119,17 @@ QSA_API qsa_status qsa_score_select(const void *Q, const float *Kc, int32_t *idx
                             int Hkv, int Tq, int q_pos0, int qblk, int T_kv_max, int d,
                             int topk, float sm_scale, void *workspace,
                             size_t workspace_bytes, qsa_stream_t stream);
+
+/*
+ * qsa_score_select over bf16 summaries (as written by qsa_compress_keys_bf16):
+ * Kc is bf16 [B][Hkv][T_kv_max/64][d]; each component is widened to fp32
+ * exactly and the scores are computed in fp32 as above.  Same workspace
+ * (qsa_score_select_workspace), rows, ordering, outputs and errors.
+ */
+QSA_API qsa_status qsa_score_select_bf16(const void *Q, const void *Kc, int32_t *idx, int B, int Hq,
+                                         int Hkv, int Tq, int q_pos0, int qblk, int T_kv_max, int d,
+                                         int topk, float sm_scale, void *workspace,
+                                         size_t workspace_bytes, qsa_stream_t stream);
 
 /*
  * Allocation-free variant of qsa_score_select.  The pages have no

@@ -38,6 +38,8 @@ def _load():
         lib.qsa_oracle_threads.restype = I
         lib.qsa_oracle_compress_keys.argtypes = [P, I, I, I, I, I, I, I, P]
         lib.qsa_oracle_compress_keys.restype = None
+        lib.qsa_oracle_round_bf16.argtypes = [P, ctypes.c_int64, P]
+        lib.qsa_oracle_round_bf16.restype = None
         lib.qsa_oracle_pool_queries.argtypes = [P, I, I, I, I, I, I, P]
         lib.qsa_oracle_pool_queries.restype = None
         lib.qsa_oracle_select.argtypes = [P, P, I, I, I, I, I, I, I, I, I, I, Dd,
@@ -70,11 +72,21 @@ def threads() -> int:
     return int(_load().qsa_oracle_threads())
 
 
-def compress_keys(K, blk_begin=0, blk_end=None, blk=BLOCK):
+def round_bf16(x):
+    """Each value rounded to the nearest bf16, ties to even (returned as
+    fp64).  Pinned by exact cases and by torch's fp32 -> bf16 conversion."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    y = np.empty_like(x)
+    _load().qsa_oracle_round_bf16(_ptr(x), x.size, _ptr(y))
+    return y
+
+
+def compress_keys(K, blk_begin=0, blk_end=None, blk=BLOCK, summary="fp32"):
     """Mean-pooled key summaries, fp64.
 
     K: bf16 [B, H, T, d].  Returns Kc [B, H, T//blk, d]; only blocks in
-    [blk_begin, blk_end) are written (others are zero).
+    [blk_begin, blk_end) are written (others are zero).  summary="bf16" is
+    the bf16-summary option: the exact mean rounded to the nearest bf16.
     """
     K = _bits(K)
     B, H, T, d = K.shape
@@ -84,6 +96,10 @@ def compress_keys(K, blk_begin=0, blk_end=None, blk=BLOCK):
     assert 0 <= blk_begin <= blk_end <= NB
     Kc = np.zeros((B, H, NB, d), dtype=np.float64)
     _load().qsa_oracle_compress_keys(_ptr(K), B, H, T, d, blk, blk_begin, blk_end, _ptr(Kc))
+    if summary == "bf16":
+        Kc = round_bf16(Kc)
+    elif summary != "fp32":
+        raise ValueError(f"summary must be 'fp32' or 'bf16', got {summary!r}")
     return Kc
 
 

@@ -83,6 +83,33 @@ void qsa_oracle_compress_keys(const uint16_t *K, int B, int H, int T, int d,
 }
 
 /*
+ * bf16-summary option of step 1: each summary rounded to the nearest bf16
+ * value, ties to even.  bf16 keeps 8 significant bits (an implicit 1 and 7
+ * stored) and fp32's exponent range, so the values representable near x
+ * are the multiples of 2^(max(e, -126) - 7), e = floor(log2 |x|) (the
+ * max() gives the evenly spaced subnormals below 2^-126).  x / q is exact (q
+ * is a power of two), and rint() in the default rounding mode rounds it to
+ * the nearest integer with ties to even; an integer just past 2^8 * 2^e
+ * lands on the next binade's grid, which is also the right bf16 value.
+ * |x| >= 2^128 (never met by means of bf16 keys) is not handled.
+ */
+void qsa_oracle_round_bf16(const double *x, int64_t n, double *y)
+{
+    for (int64_t i = 0; i < n; i++) {
+        if (x[i] == 0.0 || !isfinite(x[i])) {
+            y[i] = x[i];
+            continue;
+        }
+        int E;
+        frexp(x[i], &E);              /* |x| in [2^(E-1), 2^E) */
+        int e = E - 1;
+        if (e < -126) e = -126;
+        const double q = ldexp(1.0, e - 7);
+        y[i] = rint(x[i] / q) * q;
+    }
+}
+
+/*
  * Step 2 -- pooled query of a selection row.  One selection row is one
  * query block (qblk consecutive query tokens; 1 in decode) of one KV group;
  * the selection is shared by all query heads of the group.  The row's query

@@ -104,6 +104,37 @@ def test_compress_parity_and_reproducibility(qsa, d):
     assert torch.equal(Kc3[:, :, 5:9], Kc[:, :, 5:9]) and (Kc3[:, :, :5] == 7).all()
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_compress_bf16_summaries(qsa, d):
+    """bf16-summary option: the GPU's fp32 mean rounded to the nearest bf16.
+    Bit-identical to torch's rounding of the GPU's own fp32 summaries (same
+    reduction order), and against the oracle (the exact mean rounded) equal
+    wherever the exact mean is not within the fp32 summation bound of a
+    rounding boundary; elsewhere a valid rounding of a value within the
+    bound."""
+    w = synthetic.custom(B=2, Tq=64, T_kv=1280, Hq=8, Hkv=2, d=d, seed=22)
+    x = synthetic.generate(w)
+    K = x["K"].to(DEV)
+    Kc32 = gpu_kc(qsa, K)
+    Kb = torch.zeros(Kc32.shape, dtype=torch.bfloat16, device=DEV)
+    qsa.compress_keys(K, Kb)
+    _status_ok(qsa)
+    assert torch.equal(Kb, Kc32.to(torch.bfloat16))
+    exact = oracle.compress_keys(x["K"])
+    ref = oracle.compress_keys(x["K"], summary="bf16")
+    got = Kb.cpu().double().numpy()
+    bound = 64 * 2.0 ** -24 * np.abs(x["K"].double().numpy()).reshape(2, 2, 20, 64, d).mean(axis=3)
+    spacing = np.exp2(np.floor(np.log2(np.maximum(np.abs(exact), 2.0 ** -126))) - 7)
+    differ = got != ref
+    assert (np.abs(got - exact) <= spacing / 2 + bound)[differ].all()
+    assert differ.mean() < 1e-3, differ.mean()
+    # incremental == whole pass, bit for bit
+    Kb2 = torch.full_like(Kb, float("nan"))
+    for j in range(20):
+        qsa.compress_keys(K, Kb2, j, j + 1)
+    assert torch.equal(Kb, Kb2)
+
+
 SELECT_CASES = [
     # name, custom kwargs
     ("tiny_1k", None),
@@ -140,6 +171,32 @@ def test_score_select_parity(qsa, name, kw):
     frac, jac = check_selection(idx.cpu().numpy().reshape(-1, w.topk), sel, sel["scores"],
                                 rows_diag(w), w.topk)
     print(f"{name}: rows gap-checked {frac:.3f}, mean Jaccard {jac:.4f}")
+
+
+BF16_SELECT_CASES = ["tiny_1k", "prefill_offset_d128", "decode_multichunk", "decode_many_chunks",
+                     "token_rows_prefill"]
+
+
+@pytest.mark.parametrize("name", BF16_SELECT_CASES)
+def test_score_select_bf16_summaries(qsa, name):
+    """Selection over bf16 summaries, against the oracle scoring its own
+    bf16-rounded summaries (the same gap rule and top-m validity)."""
+    kw = dict(SELECT_CASES)[name]
+    w = synthetic.CONFIGS["tiny_prefill_1k"] if kw is None else synthetic.custom(seed=32, **kw)
+    x = synthetic.generate(w)
+    Q, K = x["Q"].to(DEV), x["K"].to(DEV)
+    Kb = torch.zeros((w.B, w.Hkv, w.T_kv // 64, w.d), dtype=torch.bfloat16, device=DEV)
+    qsa.compress_keys(K, Kb)
+    idx = torch.full((w.B, w.Hkv, w.n_rows, w.topk), -7, dtype=torch.int32, device=DEV)
+    qsa.score_select(Q, Kb, idx, w.topk, w.q_pos0, w.qblk, w.sm_scale)
+    _status_ok(qsa)
+    Kc_ref = oracle.compress_keys(x["K"], summary="bf16")
+    Qbar = oracle.pool_queries(x["Q"], w.Hkv, w.qblk)
+    sel = oracle.select(Qbar, Kc_ref, w.Tq, w.q_pos0, w.qblk, w.topk, w.sm_scale,
+                        rows=np.arange(w.B * w.Hkv * w.n_rows), want_scores=True)
+    frac, jac = check_selection(idx.cpu().numpy().reshape(-1, w.topk), sel, sel["scores"],
+                                rows_diag(w), w.topk)
+    print(f"{name} (bf16 summaries): rows gap-checked {frac:.3f}, mean Jaccard {jac:.4f}")
 
 
 def test_score_select_token_rows_past_the_cluster_limit(qsa):

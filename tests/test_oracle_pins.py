@@ -75,6 +75,54 @@ def test_compress_page_candidate_count():
     assert Kc.shape[2] == f["blocks"]
 
 
+def test_round_bf16_exact_cases():
+    """The bf16-summary option rounds to the nearest bf16, ties to even:
+    values worked out by hand on the 8-significant-bit grid."""
+    u = 2.0 ** -7                      # spacing of bf16 in [1, 2)
+    cases = [
+        (1.0, 1.0),
+        (1.0 + u / 2, 1.0),            # tie: the even neighbour is 1
+        (1.0 + 3 * u / 2, 1.0 + 2 * u),  # tie: the even neighbour is 1 + 2u
+        (1.0 + u / 2 + 2.0 ** -30, 1.0 + u),   # just above the tie: up
+        (-(1.0 + 3 * u / 2), -(1.0 + 2 * u)),  # symmetric in sign
+        (2.0 - u / 4, 2.0),            # rounds up into the next binade
+        (255.5, 256.0),                # 255.5 is a tie at spacing 1: even is 256
+        (0.1, 0.10009765625),          # 0.1 = 1.6 * 2^-4 -> 205/128 * 2^-4
+        (2.0 ** -130, 2.0 ** -130),    # subnormal, on the grid of 2^-133
+        (1.5 * 2.0 ** -133, 2.0 ** -132),  # subnormal tie: even multiple
+        (0.0, 0.0),
+    ]
+    x = np.array([c[0] for c in cases])
+    assert np.array_equal(oracle.round_bf16(x), np.array([c[1] for c in cases]))
+
+
+def test_round_bf16_matches_torch_fp32_conversion():
+    """On fp32 inputs, rounding to bf16 is what torch's fp32 -> bf16
+    conversion does (round to nearest even): an independent library check."""
+    g = torch.Generator().manual_seed(5)
+    x32 = torch.randn(20000, generator=g) * torch.exp2(torch.randint(-20, 20, (20000,), generator=g).float())
+    # include exact ties: values in [1, 2) of either sign whose 16 dropped
+    # bits are 0x8000 (halfway between two bf16 neighbours)
+    mant = torch.randint(0, 128, (2000,), generator=g, dtype=torch.int32) << 16
+    sign = torch.randint(0, 2, (2000,), generator=g, dtype=torch.int32) << 31
+    ties = sign | 0x3F800000 | mant | 0x8000
+    x32 = torch.cat([x32, ties.view(torch.float32)])
+    assert torch.isfinite(x32).all()
+    ref = x32.to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(oracle.round_bf16(x32.to(torch.float64).numpy()), ref)
+
+
+def test_compress_bf16_option_is_the_rounded_mean():
+    g = torch.Generator().manual_seed(6)
+    K = bf16(torch.randn((1, 2, 256, 16), generator=g))
+    Kc = oracle.compress_keys(K)
+    Kb = oracle.compress_keys(K, summary="bf16")
+    assert np.array_equal(Kb, oracle.round_bf16(Kc))
+    # every value is on the bf16 grid and within half a bf16 spacing
+    assert np.array_equal(Kb, f64(bf16(torch.from_numpy(Kb).float())))
+    assert np.all(np.abs(Kb - Kc) <= np.abs(Kc) * 2.0 ** -8 + 1e-300)
+
+
 # --------------------------------------------------------------------- pool
 def test_pool_closed_form_with_tail():
     B, Tq, Hq, Hkv, d = 1, 100, 8, 2, 4      # rows: 64 tokens, then a 36-token tail
