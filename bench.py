@@ -301,6 +301,9 @@ def run_qsa(args, ws, rank, local):
         if args.bf16_summaries:
             result["decode"]["bf16_summaries"] = bench_decode(args, qsa, dev, peaks, ws, rank, flush,
                                                               summary="bf16")
+        if args.paged:
+            torch.cuda.empty_cache()
+            result["decode"]["ragged_paged"] = bench_decode_paged(args, qsa, dev, peaks, ws, rank, flush)
         for name in filter(None, args.decode_more.split(",")):
             torch.cuda.empty_cache()
             result.setdefault("decode_more", {})[name] = bench_decode(args, qsa, dev, peaks, ws,
@@ -315,32 +318,13 @@ def run_qsa(args, ws, rank, local):
     return result
 
 
-def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary="fp32"):
-    wd = synthetic.CONFIGS[workload or args.decode_workload]
-    if args.decode_batch:
-        wd = synthetic.Workload(**{**wd.__dict__, "B": args.decode_batch})
-    if ws > 1:
-        wd = synthetic.Workload(**{**wd.__dict__, "seed": wd.seed + 1000 * rank})
-    x = synthetic.generate(wd, dev)
-    q = x["Q"].view(wd.B, wd.Hq, wd.d)
-    K, V = x["K"], x["V"]
-    L = wd.q_pos0 + 1
-    sdt = torch.bfloat16 if summary == "bf16" else torch.float32
-    dec = qsa.QSADecode(wd.B, wd.Hq, wd.Hkv, wd.d, wd.T_kv, wd.topk, device=dev, summary_dtype=sdt)
-    dec.compress(K, 0, L // 64)           # persistent summaries (untimed)
-    for _ in range(args.warmup):
-        dec(q, K, V, L)
-    torch.cuda.synchronize()
+def decode_timings(args, qsa, dev, ws, flush, run_parts):
+    """Times a decode step whose kernels run_parts(parts, stream) launches
+    (parts from "select", "attention"): in-graph events and the differential
+    per-step cost, for the whole step and each part.  Returns (events us,
+    differential us, launches per step)."""
     stream = torch.cuda.current_stream()
     steps = max(args.steps, 20)
-    sel_ws = dec._sel_ws[L]
-    q4 = q.view(wd.B, 1, wd.Hq, wd.d)
-
-    def run_parts(parts, s):
-        if "select" in parts:
-            qsa.score_select(q4, dec.Kc, dec.idx, wd.topk, L - 1, 1, dec.sm_scale, sel_ws, s)
-        if "attention" in parts:
-            qsa.decode(q, K, V, dec.idx, dec.o, L, dec.sm_scale, dec.ws_dec, s)
 
     def capture(parts, events=True):
         """flush [-> event] -> the step's kernels [-> event], as one CUDA
@@ -407,28 +391,99 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary=
     st, det = qsa.device_status()
     if st != "QSA_OK":
         raise RuntimeError(f"decode device status {st} ({det})")
-    # the differential times (see timed_differential) are the reported ones;
-    # the in-graph event times are kept beside them
+    return t, d, launches_step
+
+
+def decode_result(wname, B, context, topk, t, d, launches, by, sel_bytes, peaks, extra=None):
+    """The decode part of the JSON line (differential times reported, the
+    in-graph event times kept beside them)."""
     us_step, us_att, us_sel = d["step"], d["attention"], d["select"]
-    by = decode_bytes(wd)
     att_gbs = by / (us_att * 1e-6) / 1e9
+    r = {"workload": wname, "batch": B, "context": context, "topk": topk}
+    r.update(extra or {})
+    r.update({
+        "us_per_step": us_step, "us_per_token": us_step / B,
+        "timing": ("per step: R back-to-back replays of a CUDA graph (L2 flush, step kernels) "
+                   "minus R replays of (L2 flush) alone, events around each set"),
+        "breakdown_us": {"score_select": us_sel, "attention": us_att},
+        "in_graph_events_us": {"step": float(t["step"].mean()),
+                               "score_select": float(t["select"].mean()),
+                               "attention": float(t["attention"].mean())},
+        "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": att_gbs,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": att_gbs / peaks["hbm_gbs"], "bytes_per_launch": by,
+                     "traffic": None},
+        "select_gbs": sel_bytes / (us_sel * 1e-6) / 1e9,
+        "select_hbm_frac": sel_bytes / (us_sel * 1e-6) / 1e9 / peaks["hbm_gbs"],
+        "gpu_launches_per_step": int(launches)})
+    return r
+
+
+def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary="fp32"):
+    wd = synthetic.CONFIGS[workload or args.decode_workload]
+    if args.decode_batch:
+        wd = synthetic.Workload(**{**wd.__dict__, "B": args.decode_batch})
+    if ws > 1:
+        wd = synthetic.Workload(**{**wd.__dict__, "seed": wd.seed + 1000 * rank})
+    x = synthetic.generate(wd, dev)
+    q = x["Q"].view(wd.B, wd.Hq, wd.d)
+    K, V = x["K"], x["V"]
+    L = wd.q_pos0 + 1
+    sdt = torch.bfloat16 if summary == "bf16" else torch.float32
+    dec = qsa.QSADecode(wd.B, wd.Hq, wd.Hkv, wd.d, wd.T_kv, wd.topk, device=dev, summary_dtype=sdt)
+    dec.compress(K, 0, L // 64)           # persistent summaries (untimed)
+    for _ in range(args.warmup):
+        dec(q, K, V, L)
+    torch.cuda.synchronize()
+    sel_ws = dec._sel_ws[L]
+    q4 = q.view(wd.B, 1, wd.Hq, wd.d)
+
+    def run_parts(parts, s):
+        if "select" in parts:
+            qsa.score_select(q4, dec.Kc, dec.idx, wd.topk, L - 1, 1, dec.sm_scale, sel_ws, s)
+        if "attention" in parts:
+            qsa.decode(q, K, V, dec.idx, dec.o, L, dec.sm_scale, dec.ws_dec, s)
+
+    t, d, launches = decode_timings(args, qsa, dev, ws, flush, run_parts)
     # summaries read by scoring (fp32, or bf16 for the bf16-summary option)
     sel_bytes = wd.B * wd.Hkv * ((L - 1) // 64) * wd.d * (2 if summary == "bf16" else 4)
-    return {"workload": wd.name, "batch": wd.B, "context": L, "topk": wd.topk, "summaries": summary,
-            "us_per_step": us_step, "us_per_token": us_step / wd.B,
-            "timing": ("per step: R back-to-back replays of a CUDA graph (L2 flush, step kernels) "
-                       "minus R replays of (L2 flush) alone, events around each set"),
-            "breakdown_us": {"score_select": us_sel, "attention": us_att},
-            "in_graph_events_us": {"step": float(t["step"].mean()),
-                                   "score_select": float(t["select"].mean()),
-                                   "attention": float(t["attention"].mean())},
-            "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": att_gbs,
-                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": att_gbs / peaks["hbm_gbs"], "bytes_per_launch": by,
-                         "traffic": None},
-            "select_gbs": sel_bytes / (us_sel * 1e-6) / 1e9,
-            "select_hbm_frac": sel_bytes / (us_sel * 1e-6) / 1e9 / peaks["hbm_gbs"],
-            "gpu_launches_per_step": int(launches_step)}
+    return decode_result(wd.name, wd.B, L, wd.topk, t, d, launches, decode_bytes(wd), sel_bytes, peaks,
+                         {"summaries": summary})
+
+
+def bench_decode_paged(args, qsa, dev, peaks, ws, rank, flush):
+    """Ragged batch over a paged cache: 32 sequences of 64K-256K tokens
+    (uniform), blocks in randomly placed pages, top-64 per token."""
+    topk, Hq, Hkv, d = 64, 16, 2, 128
+    x = synthetic.paged_decode(B=32, min_len=65536, max_len=262144, Hq=Hq, Hkv=Hkv, d=d,
+                               seed=1007 + 1000 * rank, device=dev)
+    B = x["q"].shape[0]
+    dec = qsa.QSADecodePaged(B, Hq, Hkv, d, x["max_blocks"], topk, device=dev)
+    dec.compress(x["K_pages"], x["block_table"], x["seq_lens"])   # persistent summaries (untimed)
+    args_ = (x["q"], x["K_pages"], x["V_pages"], x["block_table"], x["seq_lens"])
+    for _ in range(args.warmup):
+        dec(*args_, x["max_len"])
+    torch.cuda.synchronize()
+    q4 = x["q"].view(B, 1, Hq, d)
+
+    def run_parts(parts, s):
+        if "select" in parts:
+            qsa.score_select_ragged(q4, dec.Kc, x["seq_lens"], dec.idx, topk, x["max_len"], dec.sm_scale, s)
+        if "attention" in parts:
+            qsa.decode_paged(*args_, dec.idx, dec.o, dec.sm_scale, s)
+
+    t, d_, launches = decode_timings(args, qsa, dev, ws, flush, run_parts)
+    lens = x["seq_lens"].cpu().numpy().astype(np.int64)
+    # selected K + V bytes as decode_bytes counts them: full selected blocks
+    # plus the visible keys of each sequence's diagonal block
+    Dg = (lens - 1) // 64
+    nsel = np.minimum(topk, Dg + 1)
+    keys = 64 * (nsel - 1) + (lens - 64 * Dg)
+    by = int(keys.sum()) * 2 * 2 * d * Hkv
+    sel_bytes = int(((lens - 1) // 64).sum()) * Hkv * d * 4
+    return decode_result("decode_ragged_paged", B, f"{int(lens.min())}-{int(lens.max())}", topk, t, d_,
+                         launches, by, sel_bytes, peaks,
+                         {"layout": "paged: [pages][Hkv][64][d], random block table; lengths uniform 64K-256K"})
 
 
 def bench_e2e(args, qsa, dev, wp, ws):
@@ -543,6 +598,8 @@ def main():
     ap.add_argument("--decode-more", default="decode_262k",
                     help="comma list of further decode workloads reported under decode_more")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-paged", dest="paged", action="store_false",
+                    help="skip the ragged-batch, paged-cache decode run (reported beside the contiguous one)")
     ap.add_argument("--no-bf16-summaries", dest="bf16_summaries", action="store_false",
                     help="skip the decode run with the bf16-summary option (reported beside the fp32 one)")
     ap.add_argument("--only-decode", action="store_true",
@@ -579,6 +636,9 @@ def main():
         res = bench_decode(args, qsa, dev, load_peaks(), ws, rank, flush)
         if args.bf16_summaries:
             res["bf16_summaries"] = bench_decode(args, qsa, dev, load_peaks(), ws, rank, flush, summary="bf16")
+        if args.paged:
+            torch.cuda.empty_cache()
+            res["ragged_paged"] = bench_decode_paged(args, qsa, dev, load_peaks(), ws, rank, flush)
         for name in filter(None, args.decode_more.split(",")):
             torch.cuda.empty_cache()
             res.setdefault("decode_more", {})[name] = bench_decode(args, qsa, dev, load_peaks(), ws,

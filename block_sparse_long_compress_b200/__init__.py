@@ -53,6 +53,9 @@ def _load():
         "qsa_sparse_attn_prefill": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P]),
         "qsa_decode_workspace": (S, [I, I, I, I, I]),
         "qsa_decode": (I, [P, P, P, P, P, I, I, I, I, I, I, I, F, P, S, P]),
+        "qsa_compress_keys_paged": (I, [P, P, P, P, I, I, I, I, I, I, I, P]),
+        "qsa_score_select_ragged": (I, [P, P, P, P, I, I, I, I, I, I, I, F, P]),
+        "qsa_decode_paged": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "qsa_get_device_status": (I, [P, ctypes.POINTER(I)]),
         "qsa_selftest_wait_timeout": (I, [ctypes.c_uint64, P]),
         "qsa_selftest_exp2": (I, [P, P, I, P]),
@@ -193,6 +196,88 @@ def decode(q, K, V, idx, o, L, sm_scale=None, workspace=None, stream=None):
         float(sm_scale), _ptr(workspace, torch.uint8, "workspace"),
         0 if workspace is None else workspace.numel(), _stream(stream)), "qsa_decode")
     return o
+
+
+# ------------------------------------------------ ragged, paged caches
+def compress_keys_paged(K_pages, block_table, seq_lens, Kc, blk_begin=0, blk_end=None, stream=None):
+    """Summaries of the complete blocks among logical blocks [blk_begin,
+    blk_end) of every sequence of a paged cache.  K_pages: bf16 [num_pages,
+    Hkv, 64, d]; block_table: int32 [B, max_blocks]; seq_lens: int32 [B];
+    Kc: fp32 [B, Hkv, max_blocks, d] (logical order)."""
+    num_pages, Hkv, blk, d = K_pages.shape
+    B, max_blocks = block_table.shape
+    if blk != BLOCK or tuple(Kc.shape) != (B, Hkv, max_blocks, d):
+        raise ValueError("K_pages must be [num_pages, Hkv, 64, d] and Kc [B, Hkv, max_blocks, d]")
+    if blk_end is None:
+        blk_end = max_blocks
+    _check(_lib.qsa_compress_keys_paged(_ptr(K_pages, torch.bfloat16, "K_pages"),
+                                        _ptr(block_table, torch.int32, "block_table"),
+                                        _ptr(seq_lens, torch.int32, "seq_lens"),
+                                        _ptr(Kc, torch.float32, "Kc"), B, Hkv, max_blocks, num_pages,
+                                        d, blk_begin, blk_end, _stream(stream)),
+           "qsa_compress_keys_paged")
+    return Kc
+
+
+def score_select_ragged(Q, Kc, seq_lens, idx, topk, max_len, sm_scale=None, stream=None):
+    """Per-token selection for one token per sequence, each at position
+    seq_lens[b] - 1.  Q: bf16 [B, 1, Hq, d]; Kc: fp32 [B, Hkv, max_blocks, d];
+    idx: int32 [B, Hkv, 1, topk] (written); max_len >= every length."""
+    B, _, Hq, d = Q.shape
+    _, Hkv, max_blocks, _ = Kc.shape
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    _check(_lib.qsa_score_select_ragged(_ptr(Q, torch.bfloat16, "Q"), _ptr(Kc, torch.float32, "Kc"),
+                                        _ptr(seq_lens, torch.int32, "seq_lens"),
+                                        _ptr(idx, torch.int32, "idx"), B, Hq, Hkv, max_blocks,
+                                        int(max_len), d, topk, float(sm_scale), _stream(stream)),
+           "qsa_score_select_ragged")
+    return idx
+
+
+def decode_paged(q, K_pages, V_pages, block_table, seq_lens, idx, o, sm_scale=None, stream=None):
+    """Decode attention over the selected blocks of paged caches, each
+    sequence at its own length.  q, o: bf16 [B, Hq, d]."""
+    B, Hq, d = q.shape
+    num_pages, Hkv, _, _ = K_pages.shape
+    max_blocks = block_table.shape[1]
+    topk = idx.shape[-1]
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    _check(_lib.qsa_decode_paged(_ptr(q, torch.bfloat16, "q"), _ptr(K_pages, torch.bfloat16, "K_pages"),
+                                 _ptr(V_pages, torch.bfloat16, "V_pages"),
+                                 _ptr(block_table, torch.int32, "block_table"),
+                                 _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(idx, torch.int32, "idx"),
+                                 _ptr(o, torch.bfloat16, "o"), B, Hq, Hkv, max_blocks, num_pages, d,
+                                 topk, float(sm_scale), _stream(stream)),
+           "qsa_decode_paged")
+    return o
+
+
+class QSADecodePaged:
+    """The decode path for a ragged batch over paged caches: per-token
+    selection at each sequence's own position, then split-K attention
+    through the block table.  Summaries (logical order) are persistent
+    state; compress() adds the blocks that have completed."""
+
+    def __init__(self, B, Hq, Hkv, d, max_blocks, topk, device="cuda"):
+        self.B, self.Hq, self.Hkv, self.d = B, Hq, Hkv, d
+        self.max_blocks, self.topk = max_blocks, topk
+        self.sm_scale = d ** -0.5
+        dev = torch.device(device)
+        self.Kc = torch.zeros((B, Hkv, max_blocks, d), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((B, Hkv, 1, topk), dtype=torch.int32, device=dev)
+        self.o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
+
+    def compress(self, K_pages, block_table, seq_lens, blk_begin=0, blk_end=None, stream=None):
+        compress_keys_paged(K_pages, block_table, seq_lens, self.Kc, blk_begin, blk_end, stream)
+
+    def __call__(self, q, K_pages, V_pages, block_table, seq_lens, max_len, stream=None):
+        score_select_ragged(q.view(self.B, 1, self.Hq, self.d), self.Kc, seq_lens, self.idx, self.topk,
+                            max_len, self.sm_scale, stream)
+        decode_paged(q, K_pages, V_pages, block_table, seq_lens, self.idx, self.o, self.sm_scale,
+                     stream)
+        return self.o
 
 
 def device_status(stream=None):

@@ -12,6 +12,10 @@
 // increasing lane order), so results are bit-reproducible.  The summary is
 // stored as fp32, or (the bf16-summary option) as that fp32 mean rounded to
 // the nearest bf16, ties to even -- half the bytes for the scoring to read.
+// Paged caches (serving): logical block j of sequence b is read from page
+// block_table[b][j] of [num_pages][Hkv][64][d], and with seq_lens given only
+// complete blocks (64 (j+1) <= seq_lens[b]) are written; summaries stay in
+// logical order [B][Hkv][max_blocks][d].
 #pragma once
 #include "device.cuh"
 
@@ -24,7 +28,10 @@ template <int D, typename KcT>
 __global__ void __launch_bounds__(128) compress_keys_kernel(const __nv_bfloat16 *__restrict__ K,
                                                             KcT *__restrict__ Kc, int T_kv_max,
                                                             int nblk_max, int blk_begin,
-                                                            int nblk)
+                                                            int nblk,
+                                                            const int32_t *__restrict__ block_table,
+                                                            const int32_t *__restrict__ seq_lens,
+                                                            int Hkv, int num_pages)
 {
     constexpr int CHUNKS = D / 8;            // 16-byte chunks per key row
     constexpr int LANES = 128 / CHUNKS;      // row lanes
@@ -36,7 +43,18 @@ __global__ void __launch_bounds__(128) compress_keys_kernel(const __nv_bfloat16 
     const int t = threadIdx.x;
     const int c = t % CHUNKS, lane = t / CHUNKS;
 
-    const uint4 *src = reinterpret_cast<const uint4 *>(K + ((bh * T_kv_max) + (long)j * 64) * D);
+    long row0 = bh * T_kv_max + (long)j * 64;
+    if (block_table) {
+        const long b = bh / Hkv, h = bh % Hkv;
+        if (seq_lens && 64L * (j + 1) > (long)__ldg(seq_lens + b)) return;   // incomplete: not yet
+        const int page = __ldg(block_table + b * nblk_max + j);
+        if (page < 0 || page >= num_pages) {
+            if (threadIdx.x == 0) report(QSA_ERR_BOUNDS, 9);
+            return;
+        }
+        row0 = ((long)page * Hkv + h) * 64;
+    }
+    const uint4 *src = reinterpret_cast<const uint4 *>(K + row0 * D);
     uint4 v[ROWS];
 #pragma unroll
     for (int k = 0; k < ROWS; k++) v[k] = __ldg(src + (long)(lane + k * LANES) * CHUNKS + c);

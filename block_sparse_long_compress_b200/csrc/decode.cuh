@@ -23,6 +23,13 @@
 // The P x 4 warp partials (max, sum, O) of the row are merged in one pass
 // through distributed shared memory, each CTA finishing 1/P of the row's
 // outputs.  No global workspace, no global atomics.
+//
+// Caches are either contiguous ([B][Hkv][T_kv_max][d]; one length L for all
+// sequences) or paged for serving: every sequence has its own length
+// seq_lens[b], and its logical block j lives in page block_table[b][j] of
+// [num_pages][Hkv][64][d] -- the cache-cell addresses the selector's indices
+// are turned into.  Indices, lengths and pages are checked before any load
+// (QSA_ERR_BOUNDS; the offending block is skipped).
 #pragma once
 #include <cooperative_groups.h>
 
@@ -95,7 +102,8 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ idx,
     __nv_bfloat16 *__restrict__ o, int Hq, int Hkv, int L, int T_kv_max, int topk, int spc,
-    float sm_scale_log2)
+    float sm_scale_log2, const int32_t *__restrict__ seq_lens, const int32_t *__restrict__ block_table,
+    int max_blocks, int num_pages)
 {
     using C = DecodeCfg<D>;
     constexpr int NS = C::NS;
@@ -108,6 +116,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t full[NS], empty[NS];
     __shared__ int blocks[C::MAX_SLOTS];   // the CTA's valid block ids in slot order
+    __shared__ int rows[C::MAX_SLOTS];     // and the first cache row of each (TMA coordinate)
     __shared__ int nb_sh, issued_sh, abort_flag;
     __shared__ float wgt[MAX_SRC][8];      // per-source, per-head merge weights
     __shared__ float lsrc[MAX_SRC][8];
@@ -120,13 +129,23 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_
     const int P = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int last_blk = (L - 1) / 64;
     const int kv_row0 = bg * T_kv_max;       // host checks B*Hkv*T_kv_max < 2^31
 
     // no global memory before the previous kernel on the stream (normally
     // the selection that writes idx) has completed
     grid_dependency_wait();
     grid_launch_dependents();
+    // this sequence's cache length (the current token is its last position)
+    int Lb = L;
+    if (seq_lens) {
+        Lb = __ldg(seq_lens + b);
+        const long cap = block_table ? 64L * max_blocks : (long)T_kv_max;
+        if (Lb < 1 || Lb > cap) {
+            if (threadIdx.x == 0) report(QSA_ERR_BOUNDS, 6);
+            Lb = 0;   // no block is valid: the row's output is zero
+        }
+    }
+    const int last_blk = Lb > 0 ? (Lb - 1) / 64 : -1;
     // the CTA's valid block ids, compacted in slot order
     const int slot0 = rank * spc;
     const int slot1 = min(slot0 + spc, topk);
@@ -139,8 +158,25 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_
                 report(QSA_ERR_BOUNDS, 3);
                 j = -1;
             }
+            int row = 0;
+            if (j >= 0) {
+                if (block_table) {
+                    const int page = __ldg(block_table + (long)b * max_blocks + j);
+                    if (page < 0 || page >= num_pages) {
+                        report(QSA_ERR_BOUNDS, 7);
+                        j = -1;
+                    } else {
+                        row = (page * Hkv + g) * 64;   // host checks num_pages*Hkv*64 < 2^31
+                    }
+                } else {
+                    row = kv_row0 + 64 * j;
+                }
+            }
             const unsigned m = __ballot_sync(0xffffffffu, j >= 0);
-            if (j >= 0) blocks[n + __popc(m & ((1u << lane) - 1u))] = j;
+            if (j >= 0) {
+                blocks[n + __popc(m & ((1u << lane) - 1u))] = j;
+                rows[n + __popc(m & ((1u << lane) - 1u))] = row;
+            }
             n += __popc(m);
         }
         if (lane == 0) nb_sh = n;
@@ -173,7 +209,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_
                     if (!mbar_wait(&empty[st], ((i / NS) - 1) & 1, &abort_flag, 42)) break;
                     fence_proxy_async_smem();
                 }
-                const int row = kv_row0 + 64 * blocks[i];
+                const int row = rows[i];
                 mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
                 uint8_t *ks = ring + st * C::STAGE_BYTES;
                 uint8_t *vs = ks + C::KV_BYTES;
@@ -221,7 +257,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_
                 mma_bf16_16816(s, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
             }
             // ---- online softmax per head over the warp's keys
-            const int lim = (L - 1) - 64 * j;   // keys c <= lim are visible
+            const int lim = (Lb - 1) - 64 * j;   // keys c <= lim are visible
             const bool v0 = key_lo <= lim, v1 = key_lo + 8 <= lim;
             s[0] = v0 ? s[0] * sm_scale_log2 : -INFINITY;
             s[1] = v0 ? s[1] * sm_scale_log2 : -INFINITY;

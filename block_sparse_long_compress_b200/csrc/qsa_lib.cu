@@ -206,6 +206,14 @@ qsa_status set_smem(K kernel, int bytes)
 }
 
 // ------------------------------------------------------------ launchers
+// Ragged / paged caches: per-sequence lengths and the block table (device
+// arrays; null for the contiguous, one-length layout).
+struct Paging {
+    const int32_t *seq_lens = nullptr;
+    const int32_t *block_table = nullptr;
+    int max_blocks = 0, num_pages = 0;
+};
+
 template <int D, int G>
 qsa_status launch_prefill(const void *Q, const void *K, const void *V, const int32_t *idx, void *O,
                           float *lse, int B, int Hq, int Hkv, int Tq, int q_pos0, int T_kv_max,
@@ -231,13 +239,15 @@ qsa_status launch_prefill(const void *Q, const void *K, const void *V, const int
 template <int D, int G>
 qsa_status launch_decode(const void *q, const void *K, const void *V, const int32_t *idx, void *o,
                          int B, int Hq, int Hkv, int L, int T_kv_max, int topk, float sm_scale,
-                         cudaStream_t s)
+                         cudaStream_t s, const Paging &pg = Paging())
 {
     using C = qsa::DecodeCfg<D>;
     CUtensorMap mk, mv;
     qsa_status st;
-    if ((st = make_map_2d(&mk, K, (uint64_t)B * Hkv * T_kv_max, D)) != QSA_OK) return st;
-    if ((st = make_map_2d(&mv, V, (uint64_t)B * Hkv * T_kv_max, D)) != QSA_OK) return st;
+    // cache rows: [B][Hkv][T_kv_max], or [num_pages][Hkv][64] when paged
+    const uint64_t nrows = pg.block_table ? (uint64_t)pg.num_pages * Hkv * 64 : (uint64_t)B * Hkv * T_kv_max;
+    if ((st = make_map_2d(&mk, K, nrows, D)) != QSA_OK) return st;
+    if ((st = make_map_2d(&mv, V, nrows, D)) != QSA_OK) return st;
     const DecodePlan p = plan_decode(B * Hkv, topk, sm_count(), C::CTAS_PER_SM);
     auto kern = qsa::decode_kernel<D, G>;
     if ((st = set_smem(kern, C::SMEM_BYTES)) != QSA_OK) return st;
@@ -256,7 +266,8 @@ qsa_status launch_decode(const void *q, const void *K, const void *V, const int3
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mk, mv, (const __nv_bfloat16 *)q, idx, (__nv_bfloat16 *)o, Hq,
-                                       Hkv, L, T_kv_max, topk, p.spc, sm_scale * 1.4426950408889634f);
+                                       Hkv, L, T_kv_max, topk, p.spc, sm_scale * 1.4426950408889634f,
+                                       pg.seq_lens, pg.block_table, pg.max_blocks, pg.num_pages);
     if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "decode_kernel launch: %s", cudaGetErrorString(e));
     return launched("decode_kernel");
 }
@@ -264,7 +275,7 @@ qsa_status launch_decode(const void *q, const void *K, const void *V, const int3
 template <int D, typename KcT>
 qsa_status launch_select_token_d(const void *Q, const KcT *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
                                  int q_pos0, int nblk_max, int topk, float sm_scale, const TokenPlan &tp,
-                                 cudaStream_t s)
+                                 cudaStream_t s, const int32_t *seq_lens)
 {
     auto kern = qsa::select_token_kernel<D, KcT>;
     const int smem = tp.CH * 8;
@@ -285,7 +296,7 @@ qsa_status launch_select_token_d(const void *Q, const KcT *Kc, int32_t *idx, int
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, (const __nv_bfloat16 *)Q, Kc, idx, nblk_max, Tq, Hq, Hkv,
-                                       q_pos0, topk, sm_scale, tp.CH);
+                                       q_pos0, topk, sm_scale, tp.CH, seq_lens);
     if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "select_token_kernel launch: %s", cudaGetErrorString(e));
     return launched("select_token_kernel");
 }
@@ -293,11 +304,13 @@ qsa_status launch_select_token_d(const void *Q, const KcT *Kc, int32_t *idx, int
 template <typename KcT>
 qsa_status launch_select_token(const void *Q, const KcT *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
                                int q_pos0, int nblk_max, int d, int topk, float sm_scale, const TokenPlan &tp,
-                               cudaStream_t s)
+                               cudaStream_t s, const int32_t *seq_lens = nullptr)
 {
     if (d == 128)
-        return launch_select_token_d<128, KcT>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, nblk_max, topk, sm_scale, tp, s);
-    return launch_select_token_d<64, KcT>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, nblk_max, topk, sm_scale, tp, s);
+        return launch_select_token_d<128, KcT>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, nblk_max, topk, sm_scale, tp, s,
+                                               seq_lens);
+    return launch_select_token_d<64, KcT>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, nblk_max, topk, sm_scale, tp, s,
+                                          seq_lens);
 }
 
 __global__ void selftest_exp2_kernel(const float *__restrict__ x, float *__restrict__ y, int n)
@@ -366,7 +379,7 @@ namespace {
 
 template <typename KcT>
 qsa_status compress_keys_impl(const char *name, const void *K, KcT *Kc, int B, int Hkv, int T_kv_max, int d,
-                              int blk_begin, int blk_end, qsa_stream_t stream)
+                              int blk_begin, int blk_end, qsa_stream_t stream, const Paging &pg = Paging())
 {
     if (!K || !Kc) return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
     if (B <= 0 || Hkv <= 0 || T_kv_max <= 0 || T_kv_max % 64)
@@ -384,10 +397,12 @@ qsa_status compress_keys_impl(const char *name, const void *K, KcT *Kc, int B, i
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (d == 128)
         qsa::compress_keys_kernel<128, KcT><<<(unsigned)grid, 128, 0, s>>>((const __nv_bfloat16 *)K, Kc, T_kv_max,
-                                                                      nblk_max, blk_begin, nblk);
+                                                                      nblk_max, blk_begin, nblk, pg.block_table,
+                                                                      pg.seq_lens, Hkv, pg.num_pages);
     else
         qsa::compress_keys_kernel<64, KcT><<<(unsigned)grid, 128, 0, s>>>((const __nv_bfloat16 *)K, Kc, T_kv_max,
-                                                                     nblk_max, blk_begin, nblk);
+                                                                     nblk_max, blk_begin, nblk, pg.block_table,
+                                                                     pg.seq_lens, Hkv, pg.num_pages);
     return launched("compress_keys_kernel");
 }
 
@@ -475,6 +490,23 @@ qsa_status qsa_compress_keys_bf16(const void *K, void *Kc, int B, int Hkv, int T
                               blk_begin, blk_end, stream);
 }
 
+qsa_status qsa_compress_keys_paged(const void *K_pages, const int32_t *block_table, const int32_t *seq_lens,
+                                   float *Kc, int B, int Hkv, int max_blocks, int num_pages, int d, int blk_begin,
+                                   int blk_end, qsa_stream_t stream)
+{
+    if (!block_table || !seq_lens) return fail(QSA_ERR_INVALID_ARG, "qsa_compress_keys_paged: null pointer");
+    if (max_blocks <= 0 || num_pages <= 0 || Hkv <= 0 || (long)num_pages * Hkv * 64 >= (1L << 31) ||
+        (long)max_blocks * 64 >= (1L << 31))
+        return fail(QSA_ERR_UNSUPPORTED, "qsa_compress_keys_paged: bad page geometry");
+    Paging pg;
+    pg.seq_lens = seq_lens;
+    pg.block_table = block_table;
+    pg.max_blocks = max_blocks;
+    pg.num_pages = num_pages;
+    return compress_keys_impl("qsa_compress_keys_paged", K_pages, Kc, B, Hkv, 64 * max_blocks, d, blk_begin, blk_end,
+                              stream, pg);
+}
+
 size_t qsa_score_select_workspace(int B, int Hq, int Hkv, int Tq, int q_pos0, int qblk, int d, int topk)
 {
     (void)Hq;
@@ -499,6 +531,26 @@ qsa_status qsa_score_select_bf16(const void *Q, const void *Kc, int32_t *idx, in
 {
     return score_select_impl("qsa_score_select_bf16", Q, static_cast<const __nv_bfloat16 *>(Kc), idx, B, Hq, Hkv,
                              Tq, q_pos0, qblk, T_kv_max, d, topk, sm_scale, workspace, workspace_bytes, stream);
+}
+
+qsa_status qsa_score_select_ragged(const void *Q, const float *Kc, const int32_t *seq_lens, int32_t *idx, int B,
+                                   int Hq, int Hkv, int max_blocks, int max_len, int d, int topk, float sm_scale,
+                                   qsa_stream_t stream)
+{
+    const char *name = "qsa_score_select_ragged";
+    if (!Q || !Kc || !seq_lens || !idx) return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || max_blocks <= 0 || max_len < 1 ||
+        (long)max_len > 64L * max_blocks)
+        return fail(QSA_ERR_INVALID_ARG, "%s: bad shape", name);
+    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "%s: d=%d", name, d);
+    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "%s: topk=%d", name, topk);
+    if ((long)Hq * d / 8 > 1024) return fail(QSA_ERR_UNSUPPORTED, "%s: Hq*d too large", name);
+    if (!aligned16(Q) || !aligned16(Kc) || !aligned16(idx) || (reinterpret_cast<uintptr_t>(seq_lens) & 3))
+        return fail(QSA_ERR_INVALID_ARG, "%s: misaligned pointer", name);
+    const TokenPlan tp = plan_token(B, Hkv, 1, max_len - 1, 1);
+    if (!tp.use) return fail(QSA_ERR_UNSUPPORTED, "%s: more candidates than one cluster of chunks holds", name);
+    return launch_select_token(Q, Kc, idx, B, Hq, Hkv, 1, max_len - 1, max_blocks, d, topk, sm_scale, tp,
+                               reinterpret_cast<cudaStream_t>(stream), seq_lens);
 }
 
 qsa_status qsa_score_select_noalloc(const void *Q, const float *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
@@ -575,6 +627,38 @@ qsa_status qsa_decode(const void *q, const void *K_cache, const void *V_cache, c
     if (d == 128 && G == 4) return launch_decode<128, 4>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, s);
     if (d == 64 && G == 8) return launch_decode<64, 8>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, s);
     return launch_decode<64, 4>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, s);
+}
+
+qsa_status qsa_decode_paged(const void *q, const void *K_pages, const void *V_pages, const int32_t *block_table,
+                            const int32_t *seq_lens, const int32_t *idx, void *o, int B, int Hq, int Hkv,
+                            int max_blocks, int num_pages, int d, int topk, float sm_scale, qsa_stream_t stream)
+{
+    const char *name = "qsa_decode_paged";
+    if (!q || !K_pages || !V_pages || !block_table || !seq_lens || !idx || !o)
+        return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || max_blocks <= 0 || num_pages <= 0)
+        return fail(QSA_ERR_INVALID_ARG, "%s: bad shape", name);
+    if ((long)num_pages * Hkv * 64 >= (1L << 31) || (long)max_blocks * 64 >= (1L << 31))
+        return fail(QSA_ERR_UNSUPPORTED, "%s: cache too large", name);
+    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "%s: d=%d", name, d);
+    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "%s: topk=%d", name, topk);
+    const int G = Hq / Hkv;
+    if (G != 4 && G != 8) return fail(QSA_ERR_UNSUPPORTED, "%s: Hq/Hkv=%d", name, G);
+    if (!aligned16(q) || !aligned16(K_pages) || !aligned16(V_pages) || !aligned16(idx) || !aligned16(o) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3) || (reinterpret_cast<uintptr_t>(seq_lens) & 3))
+        return fail(QSA_ERR_INVALID_ARG, "%s: misaligned pointer", name);
+    if (B * Hkv > 65535) return fail(QSA_ERR_UNSUPPORTED, "%s: more than 65535 (sequence, group) rows", name);
+    Paging pg;
+    pg.seq_lens = seq_lens;
+    pg.block_table = block_table;
+    pg.max_blocks = max_blocks;
+    pg.num_pages = num_pages;
+    const int T = 64 * max_blocks;   // the kernel takes each sequence's length from seq_lens
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 128 && G == 8) return launch_decode<128, 8>(q, K_pages, V_pages, idx, o, B, Hq, Hkv, T, T, topk, sm_scale, s, pg);
+    if (d == 128 && G == 4) return launch_decode<128, 4>(q, K_pages, V_pages, idx, o, B, Hq, Hkv, T, T, topk, sm_scale, s, pg);
+    if (d == 64 && G == 8) return launch_decode<64, 8>(q, K_pages, V_pages, idx, o, B, Hq, Hkv, T, T, topk, sm_scale, s, pg);
+    return launch_decode<64, 4>(q, K_pages, V_pages, idx, o, B, Hq, Hkv, T, T, topk, sm_scale, s, pg);
 }
 
 qsa_status qsa_get_device_status(qsa_stream_t stream, int *detail)

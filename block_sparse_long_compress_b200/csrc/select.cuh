@@ -407,10 +407,15 @@ __global__ void __launch_bounds__(kSelThreads) merge_select_kernel(
 // below every score's key).  After one cluster barrier the other CTAs are
 // done and the leader selects the row's top-m from the lists, which are in
 // block order.
+// Ragged batches: with seq_lens given (one decode token per sequence,
+// Tq = 1), sequence b's token sits at position seq_lens[b] - 1 (checked
+// against the summaries' capacity; an invalid length reports
+// QSA_ERR_BOUNDS and the row keeps block 0 only).
 template <int D, typename KcT>
 __global__ void __launch_bounds__(kSelThreads) select_token_kernel(
     const __nv_bfloat16 *__restrict__ Q, const KcT *__restrict__ Kc, int32_t *__restrict__ idx,
-    int nblk_max, int Tq, int Hq, int Hkv, int q_pos0, int topk, float sm_scale, int CH)
+    int nblk_max, int Tq, int Hq, int Hkv, int q_pos0, int topk, float sm_scale, int CH,
+    const int32_t *__restrict__ seq_lens)
 {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
@@ -423,10 +428,18 @@ __global__ void __launch_bounds__(kSelThreads) select_token_kernel(
     const int tid = threadIdx.x;
     const int i = blockIdx.y, bg = blockIdx.z, NR = gridDim.y;
     const int b = bg / Hkv, grp = bg % Hkv, G = Hq / Hkv;
-    const RowGeom g = row_geom(i, Tq, q_pos0, 1, topk, CH);
     const long row = (long)bg * NR + i;
     grid_dependency_wait();     // Q and Kc come from earlier work on the stream
     grid_launch_dependents();   // the attention that reads idx may be scheduled
+    int qp = q_pos0;
+    if (seq_lens) {
+        qp = __ldg(seq_lens + b) - 1;
+        if (qp < 0 || qp >= 64 * nblk_max) {
+            if (tid == 0 && chunk == 0) report(QSA_ERR_BOUNDS, 8);
+            qp = 0;
+        }
+    }
+    const RowGeom g = row_geom(i, Tq, qp, 1, topk, CH);
 
     // pooled query: mean of the token's query over the group's heads
     {

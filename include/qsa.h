@@ -190,6 +190,46 @@ QSA_API qsa_status qsa_decode(const void *q, const void *K_cache, const void *V_
                       size_t workspace_bytes, qsa_stream_t stream);
 
 /*
+ * Ragged batches over paged caches (serving).  The pages' contract is
+ * "selector -> visible cache-cell IDs -> attention over those cells"; here
+ * a cell is a 64-token page:
+ *   K_pages, V_pages  bf16 [num_pages][Hkv][64][d] (page p holds one block of
+ *                     one sequence for all KV heads);
+ *   block_table       int32 [B][max_blocks] device array: logical block j of
+ *                     sequence b lives in page block_table[b][j];
+ *   seq_lens          int32 [B] device array: sequence b's cache length,
+ *                     1 <= seq_lens[b] <= 64 * max_blocks, its current token
+ *                     at position seq_lens[b] - 1;
+ *   Kc                fp32 [B][Hkv][max_blocks][d], summaries in logical order.
+ * The kernels read lengths, pages and indices on the device and check them
+ * before any access: an invalid one sets QSA_ERR_BOUNDS in the device status
+ * word and its block is skipped (a sequence with an invalid length outputs
+ * zeros).  Host-side checks return errors before any launch as elsewhere.
+ *
+ * qsa_compress_keys_paged: summaries of the complete blocks
+ * (64 (j+1) <= seq_lens[b]) among logical blocks [blk_begin, blk_end) of
+ * every sequence; other entries of Kc are untouched.
+ * qsa_score_select_ragged: the per-token selection of qsa_score_select
+ * (qblk = 1) for one token per sequence, Q [B][1][Hq][d], each at its own
+ * position; idx [B][Hkv][1][topk].  max_len >= every seq_lens[b] sizes the
+ * launch.  No workspace (UNSUPPORTED past 8 x 8192 candidates).
+ * qsa_decode_paged: qsa_decode with each sequence's own length and pages.
+ */
+QSA_API qsa_status qsa_compress_keys_paged(const void *K_pages, const int32_t *block_table,
+                                           const int32_t *seq_lens, float *Kc, int B, int Hkv,
+                                           int max_blocks, int num_pages, int d, int blk_begin,
+                                           int blk_end, qsa_stream_t stream);
+QSA_API qsa_status qsa_score_select_ragged(const void *Q, const float *Kc, const int32_t *seq_lens,
+                                           int32_t *idx, int B, int Hq, int Hkv, int max_blocks,
+                                           int max_len, int d, int topk, float sm_scale,
+                                           qsa_stream_t stream);
+QSA_API qsa_status qsa_decode_paged(const void *q, const void *K_pages, const void *V_pages,
+                                    const int32_t *block_table, const int32_t *seq_lens,
+                                    const int32_t *idx, void *o, int B, int Hq, int Hkv,
+                                    int max_blocks, int num_pages, int d, int topk, float sm_scale,
+                                    qsa_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word
  * (QSA_OK if no kernel recorded an error since the last call).  If detail
  * is not NULL it receives a kernel-specific code (0 if none).

@@ -208,3 +208,32 @@ def generate(w: Workload, device="cpu"):
             V[b].copy_(vb.to(torch.bfloat16))
             del vb
     return {"Q": Qb, "K": K, "V": V, "planted": planted}
+
+
+def paged_decode(B=32, min_len=65536, max_len=262144, Hq=16, Hkv=2, d=128, seed=1007,
+                 device="cpu"):
+    """A ragged decode batch over a paged cache (serving): B single-token
+    queries, sequence lengths drawn uniformly in [min_len, max_len], each
+    sequence's 64-token blocks in pages [num_pages, Hkv, 64, d] placed by a
+    random permutation (the block table), Q, K, V drawn N(0, 1) and rounded
+    to bf16 once.  Returns q [B, Hq, d], K_pages, V_pages, block_table
+    [B, max_blocks] int32, seq_lens [B] int32 and max_blocks."""
+    dev = torch.device(device)
+    cpu = torch.Generator(device="cpu")
+    cpu.manual_seed(seed)
+    lens = torch.randint(min_len, max_len + 1, (B,), generator=cpu, dtype=torch.int64)
+    max_blocks = (max_len + BLOCK - 1) // BLOCK
+    num_pages = B * max_blocks
+    table = torch.randperm(num_pages, generator=cpu).view(B, max_blocks).to(torch.int32)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed + 1)
+    q = torch.randn((B, Hq, d), generator=gen, device=dev).to(torch.bfloat16)
+    K_pages = torch.empty((num_pages, Hkv, BLOCK, d), device=dev, dtype=torch.bfloat16)
+    V_pages = torch.empty_like(K_pages)
+    step = 8192   # pages drawn per chunk (bounds the fp32 staging memory)
+    for p0 in range(0, num_pages, step):
+        n = min(step, num_pages - p0)
+        K_pages[p0:p0 + n] = torch.randn((n, Hkv, BLOCK, d), generator=gen, device=dev).to(torch.bfloat16)
+        V_pages[p0:p0 + n] = torch.randn((n, Hkv, BLOCK, d), generator=gen, device=dev).to(torch.bfloat16)
+    return dict(q=q, K_pages=K_pages, V_pages=V_pages, block_table=table.to(dev),
+                seq_lens=lens.to(torch.int32).to(dev), max_blocks=max_blocks, max_len=int(lens.max()))
