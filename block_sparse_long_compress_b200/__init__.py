@@ -56,6 +56,8 @@ def _load():
         "qsa_compress_keys_paged": (I, [P, P, P, P, I, I, I, I, I, I, I, P]),
         "qsa_score_select_ragged": (I, [P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "qsa_decode_paged": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
+        "qsa_score_select_ragged_prefill": (I, [P, P, P, P, I, I, I, I, I, I, I, I, F, P, S, P]),
+        "qsa_sparse_attn_prefill_paged": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P]),
         "qsa_get_device_status": (I, [P, ctypes.POINTER(I)]),
         "qsa_selftest_wait_timeout": (I, [ctypes.c_uint64, P]),
         "qsa_selftest_exp2": (I, [P, P, I, P]),
@@ -252,6 +254,46 @@ def decode_paged(q, K_pages, V_pages, block_table, seq_lens, idx, o, sm_scale=No
                                  topk, float(sm_scale), _stream(stream)),
            "qsa_decode_paged")
     return o
+
+
+def score_select_ragged_prefill(Q, Kc, q_pos, idx, topk, max_pos, sm_scale=None, workspace=None,
+                                stream=None):
+    """Selection for a chunked prefill of a ragged batch: Q bf16 [B, Tq, Hq, d],
+    sequence b's chunk at positions q_pos[b] .. q_pos[b] + Tq - 1 (int32 [B],
+    multiples of 64); Kc fp32 [B, Hkv, max_blocks, d]; idx int32
+    [B, Hkv, ceil(Tq/64), topk] (written); max_pos >= every q_pos[b]."""
+    B, Tq, Hq, d = Q.shape
+    _, Hkv, max_blocks, _ = Kc.shape
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    need = score_select_workspace(B, Hq, Hkv, Tq, max_pos, BLOCK, d, topk)
+    if workspace is None:
+        workspace = torch.empty(max(1, need), dtype=torch.uint8, device=Q.device)
+    _check(_lib.qsa_score_select_ragged_prefill(
+        _ptr(Q, torch.bfloat16, "Q"), _ptr(Kc, torch.float32, "Kc"), _ptr(q_pos, torch.int32, "q_pos"),
+        _ptr(idx, torch.int32, "idx"), B, Hq, Hkv, Tq, max_blocks, int(max_pos), d, topk, float(sm_scale),
+        _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
+        "qsa_score_select_ragged_prefill")
+    return idx
+
+
+def sparse_attn_prefill_paged(Q, K_pages, V_pages, block_table, q_pos, idx, O, sm_scale=None, lse=None,
+                              stream=None):
+    """Prefill attention of a ragged batch over paged caches (each sequence's
+    chunk at its own position q_pos[b]).  Q, O bf16 [B, Tq, Hq, d]."""
+    B, Tq, Hq, d = Q.shape
+    num_pages, Hkv, _, _ = K_pages.shape
+    max_blocks = block_table.shape[1]
+    topk = idx.shape[-1]
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    _check(_lib.qsa_sparse_attn_prefill_paged(
+        _ptr(Q, torch.bfloat16, "Q"), _ptr(K_pages, torch.bfloat16, "K_pages"),
+        _ptr(V_pages, torch.bfloat16, "V_pages"), _ptr(block_table, torch.int32, "block_table"),
+        _ptr(q_pos, torch.int32, "q_pos"), _ptr(idx, torch.int32, "idx"), _ptr(O, torch.bfloat16, "O"),
+        _ptr(lse, torch.float32, "lse"), B, Hq, Hkv, Tq, max_blocks, num_pages, d, topk, float(sm_scale),
+        _stream(stream)), "qsa_sparse_attn_prefill_paged")
+    return O
 
 
 class QSADecodePaged:

@@ -49,6 +49,12 @@
 // TMEM (512 columns): O_0 [0,128) O_1 [128,256); S buffer b of tile t at
 // [256 + 128t + 64b, +64), P in its first 32 columns.  Every mbarrier wait
 // is bounded.
+//
+// Ragged batches over paged caches (serving, chunked prefill of several
+// requests): sequence b's chunk starts at q_pos[b] (device data) and its
+// logical block j lives in page block_table[b][j] of [num_pages][Hkv][64][d].
+// The list reader checks the position and every page before any load
+// (QSA_ERR_BOUNDS) and hands the producers each block's first cache row.
 #pragma once
 #include "device.cuh"
 
@@ -102,7 +108,9 @@ struct PrefillShared {
     int abort;
     int nblk[2];                // [list slot] blocks of the unit (>= 1)
     int none[2];                // [list slot] the row lists no valid block
-    int blocks[2][64];
+    int qp[2];                  // [list slot] the sequence's first query position
+    int diag[2];                // [list slot] the last listed block is the diagonal block
+    int rows[2][64];            // [list slot] first cache row of each block (TMA coordinate)
 };
 
 // Work unit u -> query block i, first token, batch x KV group bg.  False for
@@ -126,7 +134,8 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ idx,
     __nv_bfloat16 *__restrict__ O, float *__restrict__ lse, int Tq, int Hq, int Hkv, int BH,
-    int q_pos0, int T_kv_max, int topk, float sm_scale_log2)
+    int q_pos0, int T_kv_max, int topk, float sm_scale_log2, const int32_t *__restrict__ q_pos,
+    const int32_t *__restrict__ block_table, int max_blocks, int num_pages)
 {
     using C = PrefillCfg<D, G>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -196,23 +205,45 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
             if (!prefill_unit<C::TILES, C::TOK>(u, NX, Tq, w)) continue;
             const int slot = k & 1;
             const int b = w.bg / Hkv, g = w.bg % Hkv;
-            const int Dg = (q_pos0 + min(w.i * 64 + 63, Tq - 1)) / 64;
+            int qpos = q_pos0;
+            if (q_pos) {
+                qpos = __ldg(q_pos + b);
+                const long cap = block_table ? 64L * max_blocks : (long)T_kv_max;
+                if (qpos < 0 || (qpos & 63) || (long)qpos + Tq > cap) {
+                    if (lane == 0) report(QSA_ERR_BOUNDS, 11);
+                    qpos = 0;
+                }
+            }
+            const int Dg = (qpos + min(w.i * 64 + 63, Tq - 1)) / 64;
+            const long kv_row0 = (long)w.bg * T_kv_max;   // contiguous: host checks B*Hkv*T_kv_max < 2^31
             if (k >= 2 && !wait_all(&sh.list_empty[slot], ((k >> 1) - 1) & 1, 12)) break;
             // the row's list, one entry per lane: it ends at the first -1;
             // an index past the diagonal or not above its predecessor is an
             // error and ends it too
             const int32_t *sel = idx + ((long)w.bg * NR + w.i) * topk;
-            int n = 0, prev = -1;
+            int n = 0, prev = -1, lastj = -1;
             bool bad = false;
             for (int r0 = 0; r0 < topk; r0 += 32) {
                 const int s = r0 + lane;
                 const int j = s < topk ? sel[s] : -1;
                 int jp = __shfl_up_sync(0xffffffffu, j, 1);
                 if (lane == 0) jp = prev;
-                const bool stop_bad = j >= 0 && (j > Dg || (s > 0 && j <= jp));
+                bool stop_bad = j >= 0 && (j > Dg || (s > 0 && j <= jp));
+                int row = 0;
+                if (j >= 0 && !stop_bad) {
+                    if (block_table) {
+                        const int page = __ldg(block_table + (long)b * max_blocks + j);
+                        if (page < 0 || page >= num_pages) stop_bad = true;
+                        else row = (page * Hkv + g) * 64;   // host checks num_pages*Hkv*64 < 2^31
+                    } else {
+                        row = (int)(kv_row0 + 64L * j);
+                    }
+                }
                 const unsigned stops = __ballot_sync(0xffffffffu, j < 0 || stop_bad);
                 const int f = stops ? __ffs(stops) - 1 : 32;
-                if (lane < f) sh.blocks[slot][s] = j;
+                if (lane < f) sh.rows[slot][s] = row;
+                const int jl = __shfl_sync(0xffffffffu, j, f > 0 ? f - 1 : 0);
+                if (f > 0) lastj = jl;
                 n = r0 + f;
                 if (stops) {
                     bad = __shfl_sync(0xffffffffu, stop_bad, f);
@@ -226,10 +257,20 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
                     // no valid block: block 0 goes through the pipeline (in
                     // bounds) and the epilogue writes zeros
                     report(QSA_ERR_BOUNDS, 2);
-                    sh.blocks[slot][0] = 0;
+                    lastj = 0;
+                    int row0 = (int)kv_row0;
+                    if (block_table) {
+                        const int page = __ldg(block_table + (long)b * max_blocks);
+                        row0 = (page >= 0 && page < num_pages) ? (page * Hkv + g) * 64 : 0;
+                    }
+                    sh.rows[slot][0] = row0;
                 }
                 sh.nblk[slot] = max(n, 1);
                 sh.none[slot] = n == 0;
+                sh.qp[slot] = qpos;
+                // a valid list is ascending and ends at or before the
+                // diagonal, so only its last block can be the diagonal
+                sh.diag[slot] = lastj == Dg;
             }
             __syncwarp();
             if (lane == 0) {
@@ -243,7 +284,6 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
                             tma_load_3d(q_smem + t * C::QT_BYTES + h * C::Q_HALF, &tmQ, &sh.q_full, h * 64,
                                         g * G, b * Tq + w.token0 + t * C::TOK);
                 }
-                const int kv_row0 = w.bg * T_kv_max;   // host checks B*Hkv*T_kv_max < 2^31
                 for (int nn = 0; ok && nn < max(n, 1); nn++) {
                     const int gb = gk + nn, st = gb % C::NS;
                     if (gb >= C::NS && !mbar_wait(&sh.k_empty[st], ((gb / C::NS) - 1) & 1, abort, 10)) {
@@ -251,7 +291,7 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
                         break;
                     }
                     mbar_arrive_expect_tx(&sh.k_full[st], C::BLK_BYTES);
-                    const int row = kv_row0 + 64 * sh.blocks[slot][nn];
+                    const int row = sh.rows[slot][nn];
                     for (int h = 0; h < C::NH; h++)
                         tma_load_2d(k_smem + st * C::BLK_BYTES + h * C::B_HALF, &tmK, &sh.k_full[st], h * 64, row);
                 }
@@ -271,7 +311,6 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
                 const int slot = k & 1;
                 if (!mbar_wait(&sh.list_full[slot], (k >> 1) & 1, abort, 14)) break;
                 const int nb = sh.nblk[slot];
-                const int kv_row0 = w.bg * T_kv_max;
                 for (int nn = 0; nn < nb; nn++, gv++) {
                     const int st = gv % C::NS;
                     if (gv >= C::NS && !mbar_wait(&sh.v_empty[st], ((gv / C::NS) - 1) & 1, abort, 11)) {
@@ -279,7 +318,7 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
                         break;
                     }
                     mbar_arrive_expect_tx(&sh.v_full[st], C::BLK_BYTES);
-                    const int row = kv_row0 + 64 * sh.blocks[slot][nn];
+                    const int row = sh.rows[slot][nn];
                     for (int h = 0; h < C::NH; h++)
                         tma_load_2d(v_smem + st * C::BLK_BYTES + h * C::B_HALF, &tmV, &sh.v_full[st], h * 64, row);
                 }
@@ -404,10 +443,12 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
             if (!wait_all(&sh.list_full[slot], (k >> 1) & 1, 34)) { ok = false; break; }
             const int nb = sh.nblk[slot];
             const bool none = sh.none[slot] != 0;
+            const bool diag = sh.diag[slot] != 0;
             const int b = w.bg / Hkv, g = w.bg % Hkv;
-            const int Dg = (q_pos0 + min(w.i * 64 + 63, Tq - 1)) / 64;
+            const int qpos = sh.qp[slot];
+            const int Dg = (qpos + min(w.i * 64 + 63, Tq - 1)) / 64;
             const int tok = w.token0 + t * C::TOK + r / G;
-            const long p = (long)q_pos0 + tok;
+            const long p = (long)qpos + tok;
             float m_run = -INFINITY, l = 0.f;
             for (int n = 0; n < nb; n++) {
                 const int gb = g0 + n;
@@ -427,9 +468,8 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
                 }
                 const uint32_t s_addr = s_addr0 + 64 * (gb & 1);
                 // keys c <= lim of the block are visible: only the diagonal
-                // block is masked
-                const int blk = sh.blocks[slot][n];
-                const int lim = blk == Dg ? (int)(p - 64L * Dg) : 63;
+                // block (the list's last, when listed) is masked
+                const int lim = (n == nb - 1 && diag) ? (int)(p - 64L * Dg) : 63;
                 uint32_t sr[64];
                 tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
                 tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));

@@ -206,10 +206,12 @@ qsa_status set_smem(K kernel, int bytes)
 }
 
 // ------------------------------------------------------------ launchers
-// Ragged / paged caches: per-sequence lengths and the block table (device
-// arrays; null for the contiguous, one-length layout).
+// Ragged / paged caches: per-sequence lengths (decode, compress) or first
+// query positions (prefill) and the block table (device arrays; null for the
+// contiguous, one-length layout).
 struct Paging {
     const int32_t *seq_lens = nullptr;
+    const int32_t *q_pos = nullptr;
     const int32_t *block_table = nullptr;
     int max_blocks = 0, num_pages = 0;
 };
@@ -217,14 +219,16 @@ struct Paging {
 template <int D, int G>
 qsa_status launch_prefill(const void *Q, const void *K, const void *V, const int32_t *idx, void *O,
                           float *lse, int B, int Hq, int Hkv, int Tq, int q_pos0, int T_kv_max,
-                          int topk, float sm_scale, cudaStream_t s)
+                          int topk, float sm_scale, cudaStream_t s, const Paging &pg = Paging())
 {
     using C = qsa::PrefillCfg<D, G>;
     CUtensorMap mq, mk, mv;
     qsa_status st;
     if ((st = make_map_q(&mq, Q, (uint64_t)B * Tq, Hq, D, G, C::TOK)) != QSA_OK) return st;
-    if ((st = make_map_2d(&mk, K, (uint64_t)B * Hkv * T_kv_max, D)) != QSA_OK) return st;
-    if ((st = make_map_2d(&mv, V, (uint64_t)B * Hkv * T_kv_max, D)) != QSA_OK) return st;
+    // cache rows: [B][Hkv][T_kv_max], or [num_pages][Hkv][64] when paged
+    const uint64_t nrows = pg.block_table ? (uint64_t)pg.num_pages * Hkv * 64 : (uint64_t)B * Hkv * T_kv_max;
+    if ((st = make_map_2d(&mk, K, nrows, D)) != QSA_OK) return st;
+    if ((st = make_map_2d(&mv, V, nrows, D)) != QSA_OK) return st;
     auto kern = qsa::sparse_attn_prefill_kernel<D, G>;
     if ((st = set_smem(kern, C::SMEM_REQUEST)) != QSA_OK) return st;
     // persistent: one CTA per SM (never more than there are work units)
@@ -232,7 +236,8 @@ qsa_status launch_prefill(const void *Q, const void *K, const void *V, const int
     const int grid = (int)std::min<long>(units, sm_count());
     kern<<<grid, C::THREADS, C::SMEM_REQUEST, s>>>(mq, mk, mv, idx, (__nv_bfloat16 *)O, lse, Tq, Hq, Hkv,
                                                    B * Hkv, q_pos0, T_kv_max, topk,
-                                                   sm_scale * 1.4426950408889634f);
+                                                   sm_scale * 1.4426950408889634f, pg.q_pos, pg.block_table,
+                                                   pg.max_blocks, pg.num_pages);
     return launched("sparse_attn_prefill_kernel");
 }
 
@@ -410,7 +415,8 @@ qsa_status compress_keys_impl(const char *name, const void *K, KcT *Kc, int B, i
 template <typename KcT>
 qsa_status score_select_impl(const char *name, const void *Q, const KcT *Kc, int32_t *idx, int B, int Hq, int Hkv,
                              int Tq, int q_pos0, int qblk, int T_kv_max, int d, int topk, float sm_scale,
-                             void *workspace, size_t workspace_bytes, qsa_stream_t stream)
+                             void *workspace, size_t workspace_bytes, qsa_stream_t stream,
+                             const int32_t *q_pos = nullptr)
 {
     if (!Q || !Kc || !idx) return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || T_kv_max <= 0 || T_kv_max % 64 ||
@@ -450,7 +456,7 @@ qsa_status score_select_impl(const char *name, const void *Q, const KcT *Kc, int
         if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
         if ((st = set_smem(qsa::score_select_kernel<128, KcT>, ssmem)) != QSA_OK) return st;
         qsa::score_select_kernel<128, KcT><<<sgrid, qsa::kSelThreads, ssmem, s>>>(
-            Qbar, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk, sm_scale, p.CH, p.maxchunks);
+            Qbar, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk, sm_scale, p.CH, p.maxchunks, Hkv, q_pos);
     } else {
         if ((st = set_smem(qsa::pool_queries_kernel<64>, pool_smem)) != QSA_OK) return st;
         qsa::pool_queries_kernel<64><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq,
@@ -458,14 +464,14 @@ qsa_status score_select_impl(const char *name, const void *Q, const KcT *Kc, int
         if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
         if ((st = set_smem(qsa::score_select_kernel<64, KcT>, ssmem)) != QSA_OK) return st;
         qsa::score_select_kernel<64, KcT><<<sgrid, qsa::kSelThreads, ssmem, s>>>(
-            Qbar, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk, sm_scale, p.CH, p.maxchunks);
+            Qbar, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk, sm_scale, p.CH, p.maxchunks, Hkv, q_pos);
     }
     if ((st = launched("score_select_kernel")) != QSA_OK) return st;
     if (p.maxchunks > 1) {
         const int msmem = p.maxchunks * qsa::kMaxChosen * 8;
         if ((st = set_smem(qsa::merge_select_kernel, msmem)) != QSA_OK) return st;
         qsa::merge_select_kernel<<<mgrid, qsa::kSelThreads, msmem, s>>>(part, idx, Tq, q_pos0, qblk, topk, p.CH,
-                                                                       p.maxchunks);
+                                                                       p.maxchunks, Hkv, nblk_max, q_pos);
         if ((st = launched("merge_select_kernel")) != QSA_OK) return st;
     }
     return QSA_OK;
@@ -553,6 +559,19 @@ qsa_status qsa_score_select_ragged(const void *Q, const float *Kc, const int32_t
                                reinterpret_cast<cudaStream_t>(stream), seq_lens);
 }
 
+qsa_status qsa_score_select_ragged_prefill(const void *Q, const float *Kc, const int32_t *q_pos, int32_t *idx,
+                                           int B, int Hq, int Hkv, int Tq, int max_blocks, int max_pos, int d,
+                                           int topk, float sm_scale, void *workspace, size_t workspace_bytes,
+                                           qsa_stream_t stream)
+{
+    if (!q_pos) return fail(QSA_ERR_INVALID_ARG, "qsa_score_select_ragged_prefill: null pointer");
+    if (max_pos < 0 || max_pos % 64 || max_blocks <= 0 || (long)max_blocks * 64 >= (1L << 31))
+        return fail(QSA_ERR_INVALID_ARG, "qsa_score_select_ragged_prefill: bad max_pos / max_blocks");
+    // planned for the furthest position; each row takes its own from q_pos
+    return score_select_impl("qsa_score_select_ragged_prefill", Q, Kc, idx, B, Hq, Hkv, Tq, max_pos, 64,
+                             64 * max_blocks, d, topk, sm_scale, workspace, workspace_bytes, stream, q_pos);
+}
+
 qsa_status qsa_score_select_noalloc(const void *Q, const float *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
                                     int q_pos0, int qblk, int T_kv_max, int d, int topk, float sm_scale,
                                     qsa_stream_t stream)
@@ -627,6 +646,41 @@ qsa_status qsa_decode(const void *q, const void *K_cache, const void *V_cache, c
     if (d == 128 && G == 4) return launch_decode<128, 4>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, s);
     if (d == 64 && G == 8) return launch_decode<64, 8>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, s);
     return launch_decode<64, 4>(q, K_cache, V_cache, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, s);
+}
+
+qsa_status qsa_sparse_attn_prefill_paged(const void *Q, const void *K_pages, const void *V_pages,
+                                         const int32_t *block_table, const int32_t *q_pos, const int32_t *idx,
+                                         void *O, float *lse, int B, int Hq, int Hkv, int Tq, int max_blocks,
+                                         int num_pages, int d, int topk, float sm_scale, qsa_stream_t stream)
+{
+    const char *name = "qsa_sparse_attn_prefill_paged";
+    if (!Q || !K_pages || !V_pages || !block_table || !q_pos || !idx || !O)
+        return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || Hq % Hkv || max_blocks <= 0 || num_pages <= 0 ||
+        (long)Tq > 64L * max_blocks)
+        return fail(QSA_ERR_INVALID_ARG, "%s: bad shape", name);
+    if ((long)num_pages * Hkv * 64 >= (1L << 31) || (long)max_blocks * 64 >= (1L << 31) ||
+        (long)B * Tq >= (1L << 31))
+        return fail(QSA_ERR_UNSUPPORTED, "%s: too large", name);
+    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "%s: d=%d", name, d);
+    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "%s: topk=%d", name, topk);
+    const int G = Hq / Hkv;
+    if (G != 4 && G != 8) return fail(QSA_ERR_UNSUPPORTED, "%s: Hq/Hkv=%d", name, G);
+    if (!aligned16(Q) || !aligned16(K_pages) || !aligned16(V_pages) || !aligned16(idx) || !aligned16(O) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) || (reinterpret_cast<uintptr_t>(block_table) & 3) ||
+        (reinterpret_cast<uintptr_t>(q_pos) & 3))
+        return fail(QSA_ERR_INVALID_ARG, "%s: misaligned pointer", name);
+    Paging pg;
+    pg.q_pos = q_pos;
+    pg.block_table = block_table;
+    pg.max_blocks = max_blocks;
+    pg.num_pages = num_pages;
+    const int T = 64 * max_blocks;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 128 && G == 8) return launch_prefill<128, 8>(Q, K_pages, V_pages, idx, O, lse, B, Hq, Hkv, Tq, 0, T, topk, sm_scale, s, pg);
+    if (d == 128 && G == 4) return launch_prefill<128, 4>(Q, K_pages, V_pages, idx, O, lse, B, Hq, Hkv, Tq, 0, T, topk, sm_scale, s, pg);
+    if (d == 64 && G == 8) return launch_prefill<64, 8>(Q, K_pages, V_pages, idx, O, lse, B, Hq, Hkv, Tq, 0, T, topk, sm_scale, s, pg);
+    return launch_prefill<64, 4>(Q, K_pages, V_pages, idx, O, lse, B, Hq, Hkv, Tq, 0, T, topk, sm_scale, s, pg);
 }
 
 qsa_status qsa_decode_paged(const void *q, const void *K_pages, const void *V_pages, const int32_t *block_table,

@@ -249,6 +249,21 @@ __device__ void select_and_emit(const uint64_t *keys, int n, int need, SelectSha
     }
 }
 
+// First query position of sequence b: q_pos0, or q_pos[b] for a ragged
+// batch (device data, checked: a multiple of 64 with the chunk of Tq tokens
+// inside the summaries' capacity; otherwise QSA_ERR_BOUNDS and position 0).
+__device__ __forceinline__ int seq_q_pos(const int32_t *q_pos, int b, int q_pos0, int Tq, int nblk_max,
+                                         bool reporter)
+{
+    if (!q_pos) return q_pos0;
+    const int qp = __ldg(q_pos + b);
+    if (qp < 0 || (qp & 63) || (long)qp + Tq > 64L * nblk_max) {
+        if (reporter) report(QSA_ERR_BOUNDS, 10);
+        return 0;
+    }
+    return qp;
+}
+
 struct RowGeom {
     int D, ncand, m, nchunks;
 };
@@ -352,12 +367,14 @@ template <int D, typename KcT>
 __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
     const float *__restrict__ Qbar, const KcT *__restrict__ Kc, int32_t *__restrict__ idx,
     uint64_t *__restrict__ part, int nblk_max, int Tq, int q_pos0, int qblk, int topk,
-    float sm_scale, int CH, int maxchunks)
+    float sm_scale, int CH, int maxchunks, int Hkv, const int32_t *__restrict__ q_pos)
 {
     extern __shared__ uint64_t keys[];
     __shared__ SelectShared sh;
     const int chunk = blockIdx.x, i = blockIdx.y, bg = blockIdx.z, NR = gridDim.y;
-    const RowGeom g = row_geom(i, Tq, q_pos0, qblk, topk, CH);
+    const int qp = seq_q_pos(q_pos, bg / Hkv, q_pos0, Tq, nblk_max,
+                             threadIdx.x == 0 && chunk == 0 && i == 0 && bg % Hkv == 0);
+    const RowGeom g = row_geom(i, Tq, qp, qblk, topk, CH);
     if (chunk >= g.nchunks) return;
     const int j0 = 1 + chunk * CH;
     const int n = max(0, min(CH, g.ncand - chunk * CH));
@@ -378,12 +395,13 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
 // grid (NR, B*Hkv); dynamic smem maxchunks * kMaxChosen * 8 bytes.
 __global__ void __launch_bounds__(kSelThreads) merge_select_kernel(
     const uint64_t *__restrict__ part, int32_t *__restrict__ idx, int Tq, int q_pos0, int qblk,
-    int topk, int CH, int maxchunks)
+    int topk, int CH, int maxchunks, int Hkv, int nblk_max, const int32_t *__restrict__ q_pos)
 {
     extern __shared__ uint64_t keys[];
     __shared__ SelectShared sh;
     const int i = blockIdx.x, bg = blockIdx.y, NR = gridDim.x;
-    const RowGeom g = row_geom(i, Tq, q_pos0, qblk, topk, CH);
+    const int qp = seq_q_pos(q_pos, bg / Hkv, q_pos0, Tq, nblk_max, false);
+    const RowGeom g = row_geom(i, Tq, qp, qblk, topk, CH);
     if (g.nchunks <= 1) return;
     const long row = (long)bg * NR + i;
     // concatenate the chunks' lists (each ascending, chunks ascending)

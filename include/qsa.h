@@ -214,6 +214,19 @@ QSA_API qsa_status qsa_decode(const void *q, const void *K_cache, const void *V_
  * position; idx [B][Hkv][1][topk].  max_len >= every seq_lens[b] sizes the
  * launch.  No workspace (UNSUPPORTED past 8 x 8192 candidates).
  * qsa_decode_paged: qsa_decode with each sequence's own length and pages.
+ *
+ * Chunked prefill of a ragged batch (B requests, Tq new tokens each):
+ * sequence b's chunk occupies positions q_pos[b] .. q_pos[b] + Tq - 1
+ * (int32 [B] device array; each a multiple of 64 with
+ * q_pos[b] + Tq <= 64 * max_blocks), its K/V (cache and chunk) already in
+ * its pages and its summaries in Kc (complete blocks; see
+ * qsa_compress_keys_paged with seq_lens = q_pos + Tq).
+ * qsa_score_select_ragged_prefill: qsa_score_select with qblk = 64 and each
+ * sequence at its own position; max_pos (a multiple of 64, >= every
+ * q_pos[b]) sizes the launch and the workspace
+ * (qsa_score_select_workspace(B, Hq, Hkv, Tq, max_pos, 64, d, topk)).
+ * qsa_sparse_attn_prefill_paged: qsa_sparse_attn_prefill over the pages,
+ * each sequence at its own position.
  */
 QSA_API qsa_status qsa_compress_keys_paged(const void *K_pages, const int32_t *block_table,
                                            const int32_t *seq_lens, float *Kc, int B, int Hkv,
@@ -223,6 +236,17 @@ QSA_API qsa_status qsa_score_select_ragged(const void *Q, const float *Kc, const
                                            int32_t *idx, int B, int Hq, int Hkv, int max_blocks,
                                            int max_len, int d, int topk, float sm_scale,
                                            qsa_stream_t stream);
+QSA_API qsa_status qsa_score_select_ragged_prefill(const void *Q, const float *Kc, const int32_t *q_pos,
+                                                   int32_t *idx, int B, int Hq, int Hkv, int Tq,
+                                                   int max_blocks, int max_pos, int d, int topk,
+                                                   float sm_scale, void *workspace,
+                                                   size_t workspace_bytes, qsa_stream_t stream);
+QSA_API qsa_status qsa_sparse_attn_prefill_paged(const void *Q, const void *K_pages,
+                                                 const void *V_pages, const int32_t *block_table,
+                                                 const int32_t *q_pos, const int32_t *idx, void *O,
+                                                 float *lse, int B, int Hq, int Hkv, int Tq,
+                                                 int max_blocks, int num_pages, int d, int topk,
+                                                 float sm_scale, qsa_stream_t stream);
 QSA_API qsa_status qsa_decode_paged(const void *q, const void *K_pages, const void *V_pages,
                                     const int32_t *block_table, const int32_t *seq_lens,
                                     const int32_t *idx, void *o, int B, int Hq, int Hkv,
