@@ -297,6 +297,9 @@ def run_qsa(args, ws, rank, local):
     if not args.no_decode:
         del Q, K, V, run, x
         torch.cuda.empty_cache()
+        if args.paged:
+            result["prefill_ragged_paged"] = bench_prefill_paged(args, qsa, dev, peaks, ws, rank, flush)
+            torch.cuda.empty_cache()
         result["decode"] = bench_decode(args, qsa, dev, peaks, ws, rank, flush)
         if args.bf16_summaries:
             result["decode"]["bf16_summaries"] = bench_decode(args, qsa, dev, peaks, ws, rank, flush,
@@ -449,6 +452,63 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary=
     sel_bytes = wd.B * wd.Hkv * ((L - 1) // 64) * wd.d * (2 if summary == "bf16" else 4)
     return decode_result(wd.name, wd.B, L, wd.topk, t, d, launches, decode_bytes(wd), sel_bytes, peaks,
                          {"summaries": summary})
+
+
+def bench_prefill_paged(args, qsa, dev, peaks, ws, rank, flush):
+    """Chunked prefill of a ragged batch over paged caches: 8 requests of
+    4096 new tokens at positions uniform in [64K, 512K], top-64 per query
+    block; selection and attention timed per step (L2 flushed)."""
+    topk, Tq, Hq, Hkv, d = 64, 4096, 16, 2, 128
+    x = synthetic.paged_prefill(B=8, Tq=Tq, Hq=Hq, Hkv=Hkv, d=d, seed=1008 + 1000 * rank, device=dev)
+    B, max_blocks = x["Q"].shape[0], x["max_blocks"]
+    seq_lens = x["q_pos"] + Tq
+    Kc = torch.zeros((B, Hkv, max_blocks, d), dtype=torch.float32, device=dev)
+    qsa.compress_keys_paged(x["K_pages"], x["block_table"], seq_lens, Kc)   # cache + chunk (untimed)
+    NR = Tq // 64
+    idx = torch.empty((B, Hkv, NR, topk), dtype=torch.int32, device=dev)
+    O = torch.empty_like(x["Q"])
+    ws_sel = torch.empty(max(1, qsa.score_select_workspace(B, Hq, Hkv, Tq, x["max_pos"], 64, d, topk)),
+                         dtype=torch.uint8, device=dev)
+    sm = d ** -0.5
+
+    def select():
+        qsa.score_select_ragged_prefill(x["Q"], Kc, x["q_pos"], idx, topk, x["max_pos"], sm, ws_sel)
+
+    def attend():
+        qsa.sparse_attn_prefill_paged(x["Q"], x["K_pages"], x["V_pages"], x["block_table"], x["q_pos"], idx, O,
+                                      sm)
+
+    for _ in range(args.warmup):
+        select()
+        attend()
+    torch.cuda.synchronize()
+    t_sel, t_att = [], []
+    for _ in range(max(args.steps, 5)):
+        flush(0)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        select()
+        e[1].record()
+        attend()
+        e[2].record()
+        torch.cuda.synchronize()
+        t_sel.append(e[0].elapsed_time(e[1]))
+        t_att.append(e[1].elapsed_time(e[2]))
+    st, det = qsa.device_status()
+    if st != "QSA_OK":
+        raise RuntimeError(f"paged prefill device status {st} ({det})")
+    pos = x["q_pos"].cpu().tolist()
+    flops = sum(prefill_flops(synthetic.custom(B=1, Tq=Tq, T_kv=qp + Tq, q_pos0=qp, qblk=64, Hq=Hq, Hkv=Hkv,
+                                               d=d, topk=topk)) for qp in pos)
+    att = float(np.mean(t_att))
+    achieved = flops / (att * 1e-3) / 1e12
+    return {"workload": "chunked_ragged_paged", "batch": B, "chunk": Tq, "positions": f"{min(pos)}-{max(pos)}",
+            "topk": topk, "layout": "paged: [pages][Hkv][64][d], random block table",
+            "ms": {"score_select": float(np.mean(t_sel)), "attention": att},
+            "tokens_per_s": B * Tq / ((float(np.mean(t_sel)) + att) * 1e-3),
+            "roofline": {"bound": "tensor", "kernel": "sparse_attn_prefill_kernel", "achieved": achieved,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "flops_per_launch": flops, "traffic": None}}
 
 
 def bench_decode_paged(args, qsa, dev, peaks, ws, rank, flush):

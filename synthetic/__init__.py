@@ -237,3 +237,33 @@ def paged_decode(B=32, min_len=65536, max_len=262144, Hq=16, Hkv=2, d=128, seed=
         V_pages[p0:p0 + n] = torch.randn((n, Hkv, BLOCK, d), generator=gen, device=dev).to(torch.bfloat16)
     return dict(q=q, K_pages=K_pages, V_pages=V_pages, block_table=table.to(dev),
                 seq_lens=lens.to(torch.int32).to(dev), max_blocks=max_blocks, max_len=int(lens.max()))
+
+
+def paged_prefill(B=8, Tq=4096, min_pos=65536, max_pos=524288, Hq=16, Hkv=2, d=128, seed=1008,
+                  device="cpu"):
+    """Chunked prefill of a ragged batch over a paged cache: B requests, each
+    with Tq new tokens starting at a position drawn uniformly among the
+    multiples of 64 in [min_pos, max_pos]; every sequence's blocks (cache and
+    chunk) in pages [num_pages, Hkv, 64, d] placed by a random permutation;
+    Q, K, V drawn N(0, 1) and rounded to bf16 once.  Returns Q [B, Tq, Hq, d],
+    K_pages, V_pages, block_table [B, max_blocks] int32, q_pos [B] int32 and
+    max_blocks."""
+    dev = torch.device(device)
+    cpu = torch.Generator(device="cpu")
+    cpu.manual_seed(seed)
+    q_pos = BLOCK * torch.randint(min_pos // BLOCK, max_pos // BLOCK + 1, (B,), generator=cpu)
+    max_blocks = (max_pos + Tq + BLOCK - 1) // BLOCK
+    num_pages = B * max_blocks
+    table = torch.randperm(num_pages, generator=cpu).view(B, max_blocks).to(torch.int32)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed + 1)
+    Q = torch.randn((B, Tq, Hq, d), generator=gen, device=dev).to(torch.bfloat16)
+    K_pages = torch.empty((num_pages, Hkv, BLOCK, d), device=dev, dtype=torch.bfloat16)
+    V_pages = torch.empty_like(K_pages)
+    step = 8192
+    for p0 in range(0, num_pages, step):
+        n = min(step, num_pages - p0)
+        K_pages[p0:p0 + n] = torch.randn((n, Hkv, BLOCK, d), generator=gen, device=dev).to(torch.bfloat16)
+        V_pages[p0:p0 + n] = torch.randn((n, Hkv, BLOCK, d), generator=gen, device=dev).to(torch.bfloat16)
+    return dict(Q=Q, K_pages=K_pages, V_pages=V_pages, block_table=table.to(dev),
+                q_pos=q_pos.to(torch.int32).to(dev), max_blocks=max_blocks, max_pos=int(q_pos.max()))
