@@ -40,6 +40,12 @@ def _load():
         lib.qsa_oracle_compress_keys.restype = None
         lib.qsa_oracle_round_bf16.argtypes = [P, ctypes.c_int64, P]
         lib.qsa_oracle_round_bf16.restype = None
+        lib.qsa_oracle_fwht_f32.argtypes = [P, ctypes.c_int64, I]
+        lib.qsa_oracle_fwht_f32.restype = None
+        lib.qsa_oracle_e4m3.argtypes = [P, ctypes.c_int64, P]
+        lib.qsa_oracle_e4m3.restype = None
+        lib.qsa_oracle_quantize_rows_fp8.argtypes = [P, ctypes.c_int64, I, P, P]
+        lib.qsa_oracle_quantize_rows_fp8.restype = None
         lib.qsa_oracle_pool_queries.argtypes = [P, I, I, I, I, I, I, P]
         lib.qsa_oracle_pool_queries.restype = None
         lib.qsa_oracle_select.argtypes = [P, P, I, I, I, I, I, I, I, I, I, I, Dd,
@@ -197,3 +203,97 @@ def qsa_forward(Q, K, V, Hkv, topk, q_pos0=0, qblk=BLOCK, sm_scale=None, blk=BLO
     sel = select(Qbar, Kc, Tq, q_pos0, qblk, topk, sm_scale, blk=blk)
     O = attend(Q, K, V, sel["idx"], q_pos0, qblk, sm_scale, tokens=tokens, blk=blk)
     return sel, O
+
+
+# ------------------------------------------------------- quantized KV option
+# Page "Qwen4 in llama.cpp: Dissecting PR #27742", section "Quantized KV
+# Exposed a Backend Storage Invariant": K/V stored in a Hadamard-rotated
+# basis, attention in the rotated basis, the output returned to the original
+# basis (H^2 = I for the normalised transform).  Codes are fp8 e4m3 with one
+# fp32 scale per (token, head); the code decisions are fp32 (as the kernels
+# take them), the attention fp64.
+
+def fwht_f32(x):
+    """Unnormalised Walsh-Hadamard transform of the last axis (n = 64 or
+    128), fp32, in the kernels' butterfly order.  Returns float32."""
+    x = np.ascontiguousarray(x, dtype=np.float32).copy()
+    n = x.shape[-1]
+    _load().qsa_oracle_fwht_f32(_ptr(x), x.size // n, n)
+    return x
+
+
+def e4m3(x):
+    """fp32 values -> fp8 e4m3 codes (uint8): nearest, ties to even,
+    saturating to +-448."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    c = np.empty(x.shape, dtype=np.uint8)
+    _load().qsa_oracle_e4m3(_ptr(x), x.size, _ptr(c))
+    return c
+
+
+def e4m3_value(codes):
+    """fp8 e4m3 codes -> their values (fp64), from the format's definition:
+    exponent field 0 gives m * 2^-9, otherwise 2^(e - 7) * (1 + m / 8)."""
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e, m = (c >> 3) & 0xF, c & 0x7
+    mag = np.where(e == 0, m * 2.0 ** -9, np.ldexp(1.0 + m / 8.0, (e - 7).astype(np.int64)))
+    return sign * mag
+
+
+def quantize_kv_fp8(X):
+    """Rotated fp8 cache: X bf16 [..., n] -> (codes uint8 [..., n], scales
+    fp32 [...]) with u = WHT(x) in fp32, s = max|u| / 448, code = e4m3(u / s)."""
+    Xb = _bits(X)
+    n = Xb.shape[-1]
+    rows = Xb.size // n
+    codes = np.empty(Xb.shape, dtype=np.uint8)
+    scales = np.empty(Xb.shape[:-1], dtype=np.float32)
+    _load().qsa_oracle_quantize_rows_fp8(_ptr(Xb), rows, n, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def hadamard(n):
+    """Sylvester Hadamard matrix (entries +-1), fp64."""
+    H = np.ones((1, 1))
+    while H.shape[0] < n:
+        H = np.block([[H, H], [H, -H]])
+    return H
+
+
+def decode_fp8(q, codes_K, scales_K, codes_V, scales_V, idx, L, sm_scale, blk=BLOCK):
+    """Decode attention over a rotated fp8 cache, fp64.  q bf16 [B, Hq, n];
+    codes uint8 [B, Hkv, T, n]; scales fp32 [B, Hkv, T]; idx int32
+    [B, Hkv, 1, topk] (-1 padding); L = cache length (token at L - 1).
+    Scores u_q . u_k / n (= q . k), output H o' / n back in the original
+    basis.  Returns o [B, Hq, n]."""
+    qb = _bits(q)
+    qf = _bf16_f64(qb)
+    B, Hq, n = qf.shape
+    Hkv = codes_K.shape[1]
+    G = Hq // Hkv
+    H = hadamard(n)
+    uq = qf @ H                              # rows: H is symmetric
+    Kr = e4m3_value(codes_K) * np.asarray(scales_K, dtype=np.float64)[..., None]
+    Vr = e4m3_value(codes_V) * np.asarray(scales_V, dtype=np.float64)[..., None]
+    o = np.zeros((B, Hq, n))
+    for b in range(B):
+        for g in range(Hkv):
+            keys = []
+            for j in np.asarray(idx[b, g]).reshape(-1):
+                if j < 0:
+                    continue
+                keys.extend(range(int(j) * blk, min(int(j) * blk + blk, L)))
+            keys = np.array(keys, dtype=np.int64)
+            for h in range(g * G, (g + 1) * G):
+                z = (Kr[b, g, keys] @ uq[b, h]) / n * sm_scale
+                w = np.exp(z - z.max())
+                w /= w.sum()
+                o[b, h] = H @ (w @ Vr[b, g, keys]) / n
+    return o
+
+
+def _bf16_f64(bits):
+    """uint16 bf16 bit patterns -> fp64 values (exact widening)."""
+    u = np.asarray(bits, dtype=np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)

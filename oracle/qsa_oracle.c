@@ -110,6 +110,85 @@ void qsa_oracle_round_bf16(const double *x, int64_t n, double *y)
 }
 
 /*
+ * Quantized-KV option (page "Qwen4 in llama.cpp: Dissecting PR #27742",
+ * section "Quantized KV Exposed a Backend Storage Invariant": K/V stored in
+ * a Hadamard-rotated basis to spread channel outliers before quantization,
+ * attention in the rotated basis, the output returned to the original basis
+ * by the same transform, H^2 = I).  The kernels take every decision that
+ * produces a code in fp32, so these steps are written in fp32 with the same
+ * operations in the same order; the attention itself is fp64 (oracle.py).
+ *
+ * Unnormalised n-point Walsh-Hadamard transform (Sylvester order) of rows of
+ * n fp32 values, in place: for len = 1, 2, 4, ..., n/2, every pair
+ * (j, j + len) with j mod 2 len < len becomes (x_j + x_{j+len},
+ * x_j - x_{j+len}).  Applying it twice multiplies by n.
+ */
+void qsa_oracle_fwht_f32(float *x, int64_t rows, int n)
+{
+    for (int64_t r = 0; r < rows; r++) {
+        float *v = x + r * n;
+        for (int len = 1; len < n; len <<= 1)
+            for (int i = 0; i < n; i += 2 * len)
+                for (int j = i; j < i + len; j++) {
+                    const float a = v[j], b = v[j + len];
+                    v[j] = a + b;
+                    v[j + len] = a - b;
+                }
+    }
+}
+
+/*
+ * fp32 -> fp8 e4m3 code (1 sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits; no infinities; largest finite 448 = 1.75 * 2^8; subnormals are the
+ * multiples of 2^-9 below 2^-6): the nearest representable value, ties to
+ * even, saturating to +-448.  Near v the representable values are the
+ * multiples of 2^(max(e, -6) - 3), e = floor(log2 |v|); a / q is exact.
+ */
+static uint8_t e4m3_rn_sat(float v)
+{
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs((double)v);
+    if (a == 0.0) return sign;
+    int E;
+    frexp(a, &E);
+    int e = E - 1;
+    if (e < -6) e = -6;
+    double r = rint(a / ldexp(1.0, e - 3)) * ldexp(1.0, e - 3);
+    if (r > 448.0) r = 448.0;
+    if (r < ldexp(1.0, -6)) return sign | (uint8_t)(r / ldexp(1.0, -9));   /* subnormal (or zero) */
+    frexp(r, &E);
+    e = E - 1;
+    const int mant = (int)((r / ldexp(1.0, e) - 1.0) * 8.0);
+    return sign | (uint8_t)((e + 7) << 3) | (uint8_t)mant;
+}
+
+void qsa_oracle_e4m3(const float *x, int64_t n, uint8_t *codes)
+{
+    for (int64_t i = 0; i < n; i++) codes[i] = e4m3_rn_sat(x[i]);
+}
+
+/*
+ * Quantized, rotated cache rows: for each row of n bf16 values x,
+ * u = WHT(x) in fp32 (qsa_oracle_fwht_f32), a = max |u|, s = a / 448 (0 when
+ * a = 0), codes = e4m3(u / s) (0 when s = 0).  u ~= s * code; the
+ * normalised rotation is u / sqrt(n).
+ */
+void qsa_oracle_quantize_rows_fp8(const uint16_t *X, int64_t rows, int n, uint8_t *codes, float *scales)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        float u[256];
+        for (int c = 0; c < n; c++) u[c] = (float)bf16_to_f64(X[r * n + c]);
+        qsa_oracle_fwht_f32(u, 1, n);
+        float a = 0.0f;
+        for (int c = 0; c < n; c++) a = fmaxf(a, fabsf(u[c]));
+        const float sc = a > 0.0f ? a / 448.0f : 0.0f;
+        scales[r] = sc;
+        for (int c = 0; c < n; c++) codes[r * n + c] = sc > 0.0f ? e4m3_rn_sat(u[c] / sc) : 0;
+    }
+}
+
+/*
  * Step 2 -- pooled query of a selection row.  One selection row is one
  * query block (qblk consecutive query tokens; 1 in decode) of one KV group;
  * the selection is shared by all query heads of the group.  The row's query

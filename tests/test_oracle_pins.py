@@ -373,3 +373,93 @@ def test_jaccard_definition():
     assert jaccard([0, 1, 2, 5], [0, 2, 5, 7]) == pytest.approx(3 / 5)
     assert jaccard([0, 3], [0, 3]) == 1.0
     assert jaccard([0, -1, 4], [0, 4, -1]) == 1.0
+
+
+# ------------------------------------------------------- quantized KV option
+def test_fwht_is_the_sylvester_hadamard_product():
+    """The rotation is the unnormalised Walsh-Hadamard transform: on integer
+    inputs (exact in fp32) it equals the product with scipy's Sylvester
+    Hadamard matrix, and applying it twice multiplies by n (H^2 = n I)."""
+    import scipy.linalg
+    g = np.random.RandomState(3)
+    for n in (64, 128):
+        x = g.randint(-50, 50, size=(5, n)).astype(np.float32)
+        H = scipy.linalg.hadamard(n).astype(np.float64)
+        assert np.array_equal(oracle.fwht_f32(x).astype(np.float64), x.astype(np.float64) @ H.T)
+        assert np.array_equal(oracle.fwht_f32(oracle.fwht_f32(x)), n * x)
+
+
+def test_e4m3_hand_values():
+    """fp8 e4m3: 3 mantissa bits, bias 7, largest 448, subnormals m * 2^-9;
+    nearest with ties to even, saturating."""
+    cases = [
+        (1.0, 0x38), (1.0625, 0x38),          # tie between 1 and 1.125: even (1)
+        (1.1875, 0x3A),                        # tie between 1.125 and 1.25: even (1.25)
+        (448.0, 0x7E), (460.0, 0x7E),          # 460 rounds to 448
+        (470.0, 0x7E), (1e9, 0x7E),            # would round to 480 / overflow: saturates
+        (-470.0, 0xFE),
+        (2.0 ** -9, 0x01), (1.5 * 2.0 ** -9, 0x02),   # subnormal tie: even multiple
+        (2.0 ** -10, 0x00),                    # tie between 0 and 2^-9: even (0)
+        (2.0 ** -6, 0x08),                     # smallest normal
+        (-3.3, 0xC5), (0.0, 0x00), (-0.0, 0x80),
+    ]
+    got = oracle.e4m3(np.array([c[0] for c in cases], dtype=np.float32))
+    assert got.tolist() == [c[1] for c in cases]
+
+
+def test_e4m3_matches_torch_within_range():
+    """Inside the range where no saturation happens (|x| < 464), the codes
+    are torch's fp32 -> float8_e4m3fn conversion; every finite code decodes
+    to the value torch gives and encodes back to itself."""
+    g = torch.Generator().manual_seed(9)
+    x = torch.randn(50000, generator=g) * torch.exp2(torch.randint(-12, 9, (50000,), generator=g).float())
+    x = x[x.abs() < 464]
+    ref = x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3(x.numpy()), ref)
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(oracle.e4m3_value(codes), vals)
+    assert np.array_equal(oracle.e4m3(vals.astype(np.float32)), codes)
+
+
+def test_quantize_rows_fp8_scale_and_error():
+    g = torch.Generator().manual_seed(10)
+    X = bf16(torch.randn((40, 128), generator=g))
+    codes, scales = oracle.quantize_kv_fp8(X)
+    u = oracle.fwht_f32(f64(X).astype(np.float32))
+    assert np.array_equal(scales, (np.abs(u).max(axis=1) / np.float32(448)).astype(np.float32))
+    deq = oracle.e4m3_value(codes) * scales[:, None].astype(np.float64)
+    # within half a code step (relative 2^-4 for normals) of the rotated row
+    assert np.all(np.abs(deq - u) <= np.abs(u) * 2.0 ** -4 + scales[:, None] * 2.0 ** -10)
+    # the largest element of each row becomes +-448
+    am = np.abs(u).argmax(axis=1)
+    assert np.all(np.abs(oracle.e4m3_value(codes[np.arange(40), am])) == 448.0)
+
+
+def test_decode_fp8_equals_bf16_attention_on_walsh_rows():
+    """Rows whose rotation has a single nonzero component are signed Walsh
+    functions times c*s/n -- exact in bf16 -- and quantize without loss, so
+    the quantized decode (rotated basis, output rotated back) must equal the
+    pinned bf16 attention on the same K, V."""
+    import scipy.linalg
+    n, B, Hq, Hkv, T, L = 128, 2, 8, 2, 256, 200
+    H = scipy.linalg.hadamard(n).astype(np.float64)
+    g = np.random.RandomState(11)
+    def walsh_rows(shape):
+        # c = +-1.75 * 2^k: the rotated row's one nonzero is 16 c, its scale
+        # 16 c / 448 = 2^k / 16 is a power of two, so the code 448 is exact
+        j0 = g.randint(0, n, size=shape)
+        c = g.choice([0.4375, 0.875, 1.75, 3.5, -0.875, -1.75], size=shape)
+        return (c[..., None] * H[j0]) * 2.0 ** -3      # = c * 2^-3 * row j0 of H (exact in bf16)
+    K = bf16(torch.from_numpy(walsh_rows((B, Hkv, T))).float())
+    V = bf16(torch.from_numpy(walsh_rows((B, Hkv, T))).float())
+    q = bf16(torch.randn((B, Hq, n), generator=torch.Generator().manual_seed(12)))
+    ck, sk = oracle.quantize_kv_fp8(K)
+    cv, sv = oracle.quantize_kv_fp8(V)
+    assert np.allclose(oracle.fwht_f32(f64(K).astype(np.float32)),
+                       oracle.e4m3_value(ck) * sk[..., None].astype(np.float64), rtol=0, atol=0)
+    idx = np.array([[0, 1, 3, -1], [0, 2, 3, -1]] * B, dtype=np.int32).reshape(B, Hkv, 1, 4)
+    sm = n ** -0.5
+    o = oracle.decode_fp8(q, ck, sk, cv, sv, idx, L, sm)
+    ref = oracle.attend(q.view(B, 1, Hq, n), K, V, idx, L - 1, 1, sm).reshape(B, Hq, n)
+    assert np.abs(o - ref).max() < 1e-12
