@@ -304,6 +304,10 @@ def run_qsa(args, ws, rank, local):
         if args.bf16_summaries:
             result["decode"]["bf16_summaries"] = bench_decode(args, qsa, dev, peaks, ws, rank, flush,
                                                               summary="bf16")
+        if args.fp8_kv:
+            torch.cuda.empty_cache()
+            result["decode"]["fp8_kv"] = bench_decode(args, qsa, dev, peaks, ws, rank, flush,
+                                                      summary="bf16", kv="fp8")
         if args.paged:
             torch.cuda.empty_cache()
             result["decode"]["ragged_paged"] = bench_decode_paged(args, qsa, dev, peaks, ws, rank, flush)
@@ -422,7 +426,7 @@ def decode_result(wname, B, context, topk, t, d, launches, by, sel_bytes, peaks,
     return r
 
 
-def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary="fp32"):
+def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary="fp32", kv="bf16"):
     wd = synthetic.CONFIGS[workload or args.decode_workload]
     if args.decode_batch:
         wd = synthetic.Workload(**{**wd.__dict__, "B": args.decode_batch})
@@ -440,18 +444,32 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary=
     torch.cuda.synchronize()
     sel_ws = dec._sel_ws[L]
     q4 = q.view(wd.B, 1, wd.Hq, wd.d)
+    by = decode_bytes(wd)
+    extra = {"summaries": summary}
+    if kv == "fp8":
+        # the cache as rotated e4m3 codes + per-row scales (written untimed,
+        # as the cache write path would); summaries stay those of the keys
+        Kq, Ks = qsa.quantize_kv_fp8(K)
+        Vq, Vs = qsa.quantize_kv_fp8(V)
+        del K, V, x
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        by = by // (2 * wd.d) * (wd.d + 4)      # per selected key and head: d code bytes + a 4-byte scale
+        extra["kv_cache"] = "fp8 e4m3, Walsh-Hadamard rotated, per-row fp32 scale"
 
     def run_parts(parts, s):
         if "select" in parts:
             qsa.score_select(q4, dec.Kc, dec.idx, wd.topk, L - 1, 1, dec.sm_scale, sel_ws, s)
         if "attention" in parts:
-            qsa.decode(q, K, V, dec.idx, dec.o, L, dec.sm_scale, dec.ws_dec, s)
+            if kv == "fp8":
+                qsa.decode_fp8(q, Kq, Ks, Vq, Vs, dec.idx, dec.o, L, dec.sm_scale, s)
+            else:
+                qsa.decode(q, K, V, dec.idx, dec.o, L, dec.sm_scale, dec.ws_dec, s)
 
     t, d, launches = decode_timings(args, qsa, dev, ws, flush, run_parts)
     # summaries read by scoring (fp32, or bf16 for the bf16-summary option)
     sel_bytes = wd.B * wd.Hkv * ((L - 1) // 64) * wd.d * (2 if summary == "bf16" else 4)
-    return decode_result(wd.name, wd.B, L, wd.topk, t, d, launches, decode_bytes(wd), sel_bytes, peaks,
-                         {"summaries": summary})
+    return decode_result(wd.name, wd.B, L, wd.topk, t, d, launches, by, sel_bytes, peaks, extra)
 
 
 def bench_prefill_paged(args, qsa, dev, peaks, ws, rank, flush):
@@ -662,8 +680,12 @@ def main():
                     help="skip the ragged-batch, paged-cache decode run (reported beside the contiguous one)")
     ap.add_argument("--no-bf16-summaries", dest="bf16_summaries", action="store_false",
                     help="skip the decode run with the bf16-summary option (reported beside the fp32 one)")
+    ap.add_argument("--no-fp8-kv", dest="fp8_kv", action="store_false",
+                    help="skip the decode run over the rotated fp8 cache (reported beside the bf16 one)")
     ap.add_argument("--only-decode", action="store_true",
                     help="skip the prefill measurement (profiling the decode kernels)")
+    ap.add_argument("--decode-variants", default="fp32,bf16,fp8,paged",
+                    help="with --only-decode: which decode runs (fp32 / bf16 summaries, fp8 cache, paged)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="override the decode batch (smaller profiling captures)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -693,10 +715,14 @@ def main():
         dev = torch.device("cuda", local)
         torch.cuda.set_device(dev)
         flush = L2Flush(dev)
-        res = bench_decode(args, qsa, dev, load_peaks(), ws, rank, flush)
-        if args.bf16_summaries:
+        variants = set(filter(None, args.decode_variants.split(",")))
+        res = bench_decode(args, qsa, dev, load_peaks(), ws, rank, flush) if "fp32" in variants else {}
+        if args.bf16_summaries and "bf16" in variants:
             res["bf16_summaries"] = bench_decode(args, qsa, dev, load_peaks(), ws, rank, flush, summary="bf16")
-        if args.paged:
+        if args.fp8_kv and "fp8" in variants:
+            torch.cuda.empty_cache()
+            res["fp8_kv"] = bench_decode(args, qsa, dev, load_peaks(), ws, rank, flush, summary="bf16", kv="fp8")
+        if args.paged and "paged" in variants:
             torch.cuda.empty_cache()
             res["ragged_paged"] = bench_decode_paged(args, qsa, dev, load_peaks(), ws, rank, flush)
         for name in filter(None, args.decode_more.split(",")):

@@ -57,6 +57,8 @@ def _load():
         "qsa_score_select_ragged": (I, [P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "qsa_decode_paged": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "qsa_score_select_ragged_prefill": (I, [P, P, P, P, I, I, I, I, I, I, I, I, F, P, S, P]),
+        "qsa_quantize_kv_fp8": (I, [P, P, P, ctypes.c_int64, I, P]),
+        "qsa_decode_fp8": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "qsa_sparse_attn_prefill_paged": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P]),
         "qsa_get_device_status": (I, [P, ctypes.POINTER(I)]),
         "qsa_selftest_wait_timeout": (I, [ctypes.c_uint64, P]),
@@ -294,6 +296,40 @@ def sparse_attn_prefill_paged(Q, K_pages, V_pages, block_table, q_pos, idx, O, s
         _ptr(lse, torch.float32, "lse"), B, Hq, Hkv, Tq, max_blocks, num_pages, d, topk, float(sm_scale),
         _stream(stream)), "qsa_sparse_attn_prefill_paged")
     return O
+
+
+# ------------------------------------------------- rotated fp8 KV (decode)
+def quantize_kv_fp8(X, codes=None, scales=None, stream=None):
+    """Rotated fp8 cache rows: X bf16 [..., 128] -> codes uint8 [..., 128]
+    (e4m3 of the Walsh-Hadamard-rotated row over its scale) and scales fp32
+    [...] (max |rotated row| / 448)."""
+    if X.shape[-1] != 128:
+        raise ValueError("rotated fp8 rows are 128 wide")
+    if codes is None:
+        codes = torch.empty(X.shape, dtype=torch.uint8, device=X.device)
+    if scales is None:
+        scales = torch.empty(X.shape[:-1], dtype=torch.float32, device=X.device)
+    rows = X.numel() // 128
+    _check(_lib.qsa_quantize_kv_fp8(_ptr(X, torch.bfloat16, "X"), _ptr(codes, torch.uint8, "codes"),
+                                    _ptr(scales, torch.float32, "scales"), rows, 128, _stream(stream)),
+           "qsa_quantize_kv_fp8")
+    return codes, scales
+
+
+def decode_fp8(q, K_codes, K_scales, V_codes, V_scales, idx, o, L, sm_scale=None, stream=None):
+    """Decode attention over a rotated fp8 cache (codes uint8 [B, Hkv, T, 128],
+    scales fp32 [B, Hkv, T]); q, o bf16 [B, Hq, 128] in the original basis."""
+    B, Hq, d = q.shape
+    _, Hkv, T, _ = K_codes.shape
+    topk = idx.shape[-1]
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    _check(_lib.qsa_decode_fp8(_ptr(q, torch.bfloat16, "q"), _ptr(K_codes, torch.uint8, "K_codes"),
+                               _ptr(K_scales, torch.float32, "K_scales"), _ptr(V_codes, torch.uint8, "V_codes"),
+                               _ptr(V_scales, torch.float32, "V_scales"), _ptr(idx, torch.int32, "idx"),
+                               _ptr(o, torch.bfloat16, "o"), B, Hq, Hkv, L, T, d, topk, float(sm_scale),
+                               _stream(stream)), "qsa_decode_fp8")
+    return o
 
 
 class QSADecodePaged:

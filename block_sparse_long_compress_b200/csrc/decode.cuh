@@ -37,14 +37,19 @@
 
 namespace qsa {
 
-template <int D>
+// FP8: the rotated fp8 cache option (quant.cuh): a stage holds a block's K
+// and V codes (one 64 x 128-byte box each) and their per-row scales; every
+// consumer thread loads the codes of its MMA fragments straight from the
+// stage and expands them to f16 in registers.
+template <int D, bool FP8 = false>
 struct DecodeCfg {
     static constexpr int NH = D / 64;                  // 64-column TMA boxes per row
     static constexpr int HALF_BYTES = 64 * 128;        // one 64-row x 128-byte box
-    static constexpr int KV_BYTES = 64 * D * 2;        // one block's K (or V)
-    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+    static constexpr int KV_BYTES = FP8 ? 64 * D : 64 * D * 2;   // one block's K (or V)
+    static constexpr int SCALE_BYTES = FP8 ? 64 * 4 : 0;         // its per-row scales
+    static constexpr int STAGE_BYTES = FP8 ? (2 * KV_BYTES + 2 * SCALE_BYTES + 1023) / 1024 * 1024 : 2 * KV_BYTES;
     static constexpr int CTAS_PER_SM = 2;
-    static constexpr int RING_BYTES = 96 * 1024;       // NS stages; two CTAs per SM
+    static constexpr int RING_BYTES = FP8 ? 6 * STAGE_BYTES : 96 * 1024;   // NS stages; two CTAs per SM
     static constexpr int NS = RING_BYTES / STAGE_BYTES;
     static constexpr int NC = 4;                       // consumer warps
     static constexpr int THREADS = (NC + 1) * 32;
@@ -53,8 +58,37 @@ struct DecodeCfg {
     static constexpr int MAX_SLOTS = 64;
     static constexpr int MAX_CLUSTER = 8;
     static_assert(NS >= 2, "ring too small");
-    static_assert(NC * PART_FLOATS * 4 <= RING_BYTES, "merge scratch must fit in the ring");
+    static_assert(NC * PART_FLOATS * 4 + 4 * D <= RING_BYTES, "merge scratch must fit in the ring");
+    static_assert(!FP8 || D == 128, "rotated fp8 rows are 128 wide");
+    // FP8 merge: up to 8 heads x 4 source groups x D floats after the partials
+    static_assert(!FP8 || NC * PART_FLOATS * 4 + 8 * 4 * D * 4 <= RING_BYTES, "fp8 merge scratch");
 };
+
+__device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Two e4m3 codes (low and high byte of a 16-bit half of w) to f16x2.
+__device__ __forceinline__ uint32_t e4m3_lo(uint32_t w) { return cvt_e4m3x2_f16x2((uint16_t)(w & 0xFFFFu)); }
+__device__ __forceinline__ uint32_t e4m3_hi(uint32_t w) { return cvt_e4m3x2_f16x2((uint16_t)(w >> 16)); }
+
+__device__ __forceinline__ uint32_t u4_word(const uint4 &v, int i)
+{
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
                                         uint32_t &r3)
@@ -97,15 +131,15 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int c16)
     return (uint32_t)((c16 >> 3) * (64 * 128) + row * 128 + (((c16 & 7) ^ (row & 7)) << 4));
 }
 
-template <int D, int G>
-__global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_SM) decode_kernel(
+template <int D, int G, bool FP8 = false>
+__global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>::CTAS_PER_SM) decode_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ idx,
     __nv_bfloat16 *__restrict__ o, int Hq, int Hkv, int L, int T_kv_max, int topk, int spc,
     float sm_scale_log2, const int32_t *__restrict__ seq_lens, const int32_t *__restrict__ block_table,
-    int max_blocks, int num_pages)
+    int max_blocks, int num_pages, const float *__restrict__ k_scales, const float *__restrict__ v_scales)
 {
-    using C = DecodeCfg<D>;
+    using C = DecodeCfg<D, FP8>;
     constexpr int NS = C::NS;
     constexpr int NC = C::NC;
     constexpr int PF = C::PART_FLOATS;
@@ -121,6 +155,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_
     __shared__ float wgt[MAX_SRC][8];      // per-source, per-head merge weights
     __shared__ float lsrc[MAX_SRC][8];
     __shared__ float inv_l[8];
+    __shared__ __align__(16) uint32_t uq[FP8 ? 8 * (D / 2) : 1];   // FP8: rotated queries, f16 pairs
 
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *part = reinterpret_cast<float *>(ring);   // after the loop: [NC][PF] warp partials
@@ -210,13 +245,25 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_
                     fence_proxy_async_smem();
                 }
                 const int row = rows[i];
-                mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
                 uint8_t *ks = ring + st * C::STAGE_BYTES;
                 uint8_t *vs = ks + C::KV_BYTES;
+                if constexpr (FP8) {
+                    // codes: one 64-row x 128-byte box each; scales: 64 fp32
+                    // per tensor, one plain bulk copy each
+                    mbar_arrive_expect_tx(&full[st], 2 * C::KV_BYTES + 2 * C::SCALE_BYTES);
+                    tma_load_2d(ks, &tmK, &full[st], 0, row);
+                    tma_load_2d(vs, &tmV, &full[st], 0, row);
+                    bulk_load(vs + C::KV_BYTES, k_scales + row, C::SCALE_BYTES, &full[st]);
+                    bulk_load(vs + C::KV_BYTES + C::SCALE_BYTES, v_scales + row, C::SCALE_BYTES, &full[st]);
+                } else {
+                    mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
 #pragma unroll
-                for (int h = 0; h < C::NH; h++) tma_load_2d(ks + h * C::HALF_BYTES, &tmK, &full[st], h * 64, row);
+                    for (int h = 0; h < C::NH; h++)
+                        tma_load_2d(ks + h * C::HALF_BYTES, &tmK, &full[st], h * 64, row);
 #pragma unroll
-                for (int h = 0; h < C::NH; h++) tma_load_2d(vs + h * C::HALF_BYTES, &tmV, &full[st], h * 64, row);
+                    for (int h = 0; h < C::NH; h++)
+                        tma_load_2d(vs + h * C::HALF_BYTES, &tmV, &full[st], h * 64, row);
+                }
             }
             issued_sh = i;
         }
@@ -226,7 +273,32 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_
         // (zero for n >= G), rows k = d.
         const int hn = lane >> 2, qc = (lane & 3) * 2;
         uint32_t qb[D / 16][2];
-        {
+        if constexpr (FP8) {
+            // the group's queries in the rotated basis (unnormalised
+            // transform, as f16 pairs; consumer warp w takes heads w, w + NC,
+            // ...), shared among the consumer warps only, so that the
+            // producer's first copies are not held back by these loads
+            for (int h = warp; h < G; h += NC) {
+                const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(q + ((long)b * Hq + g * G + h) * D) + lane);
+                float x[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                              __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
+                fwht_warp<4>(x);
+                uq[h * (D / 2) + 2 * lane] = pack_f16x2(x[0], x[1]);
+                uq[h * (D / 2) + 2 * lane + 1] = pack_f16x2(x[2], x[3]);
+            }
+            named_barrier_sync(1, NC * 32);
+            // rotated queries (f16) from the shared copy.  The contraction
+            // over d runs in a permuted order that gives every thread 32
+            // contiguous codes of each of its key rows: in k-step kk, MMA k
+            // indices 2c, 2c + 1 (c = lane % 4) stand for d = 32c + 4kk + {0, 1}
+            // and 2c + 8, 2c + 9 for d = 32c + 4kk + {2, 3}.
+            const uint32_t *uqh = uq + (hn < G ? hn : 0) * (D / 2);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; kk++) {
+                qb[kk][0] = hn < G ? uqh[8 * qc + 2 * kk] : 0u;
+                qb[kk][1] = hn < G ? uqh[8 * qc + 2 * kk + 1] : 0u;
+            }
+        } else {
             const __nv_bfloat16 *qrow = q + ((long)b * Hq + g * G + (hn < G ? hn : 0)) * D;
 #pragma unroll
             for (int kk = 0; kk < D / 16; kk++) {
@@ -242,6 +314,127 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_
         const int vrow_a = k0 + (lane & 7) + 8 * (lane >> 4);        // V rows for ldmatrix.trans (A of O^T)
         const int vchunk_a = (lane >> 3) & 1;
         const int key_lo = k0 + (lane >> 2);                         // keys of this thread's S^T entries
+        if constexpr (FP8) {
+            // Two blocks per iteration (one softmax update for both): the
+            // per-block chain (codes -> S MMAs -> row max -> exponentials ->
+            // PV MMAs) is latency-bound with two consumer warps per
+            // scheduler, and the pair doubles the independent work in it.
+            const int c = lane & 3, r = lane >> 2, sw = key_lo & 7;   // (key_lo + 8) & 7 == sw
+            const float sc = sm_scale_log2 * (1.0f / 128.0f);
+            // the thread's codes, straight from the stage (128-byte swizzle):
+            // K rows key_lo and key_lo + 8, bytes 32c .. 32c+31; V rows
+            // k0 + {2c, 2c+1, 2c+8, 2c+9}, bytes 16r .. 16r+15; and the
+            // per-row scales (scores: (u_q . u_k) / 128 = q . k with
+            // u_k = scale * code; the V scale rides on P)
+            auto load = [&](int st, uint4 (&kr)[4], uint4 (&vr)[4], float (&kq)[2], float (&vp)[2]) {
+                const uint8_t *kst = ring + st * C::STAGE_BYTES;
+                const uint8_t *vst = kst + C::KV_BYTES;
+                const float *ksc = reinterpret_cast<const float *>(vst + C::KV_BYTES);
+                const float *vsc = ksc + 64;
+                kr[0] = *reinterpret_cast<const uint4 *>(kst + key_lo * 128 + (((2 * c) ^ sw) << 4));
+                kr[1] = *reinterpret_cast<const uint4 *>(kst + key_lo * 128 + (((2 * c + 1) ^ sw) << 4));
+                kr[2] = *reinterpret_cast<const uint4 *>(kst + (key_lo + 8) * 128 + (((2 * c) ^ sw) << 4));
+                kr[3] = *reinterpret_cast<const uint4 *>(kst + (key_lo + 8) * 128 + (((2 * c + 1) ^ sw) << 4));
+#pragma unroll
+                for (int t = 0; t < 4; t++) {
+                    const int vk = k0 + 2 * c + (t & 1) + 8 * (t >> 1);
+                    vr[t] = *reinterpret_cast<const uint4 *>(vst + vk * 128 + ((r ^ (vk & 7)) << 4));
+                }
+                kq[0] = ksc[key_lo] * sc;
+                kq[1] = ksc[key_lo + 8] * sc;
+                vp[0] = vsc[key_lo];
+                vp[1] = vsc[key_lo + 8];
+            };
+            // S^T (16 keys x 8 heads) = K q^T, two independent chains
+            auto scores = [&](const uint4 (&kr)[4], float (&s)[4]) {
+                float s2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int kk = 0; kk < D / 16; kk++) {
+                    const uint32_t wl = u4_word(kr[kk >> 2], kk & 3);        // row key_lo
+                    const uint32_t wh = u4_word(kr[2 + (kk >> 2)], kk & 3);  // row key_lo + 8
+                    if (kk & 1)
+                        mma_f16_16816(s2, e4m3_lo(wl), e4m3_lo(wh), e4m3_hi(wl), e4m3_hi(wh), qb[kk][0], qb[kk][1]);
+                    else
+                        mma_f16_16816(s, e4m3_lo(wl), e4m3_lo(wh), e4m3_hi(wl), e4m3_hi(wh), qb[kk][0], qb[kk][1]);
+                }
+#pragma unroll
+                for (int t = 0; t < 4; t++) s[t] += s2[t];
+            };
+            // keys c <= lim of the block are visible; scaled scores or -inf
+            auto mask_scale = [&](float (&s)[4], int lim, const float (&kq)[2]) {
+                const bool v0 = key_lo <= lim, v1 = key_lo + 8 <= lim;
+                s[0] = v0 ? s[0] * kq[0] : -INFINITY;
+                s[1] = v0 ? s[1] * kq[0] : -INFINITY;
+                s[2] = v1 ? s[2] * kq[1] : -INFINITY;
+                s[3] = v1 ? s[3] * kq[1] : -INFINITY;
+            };
+            // O^T += V^T P^T: MMA rows (mt, r) and (mt, r + 8) stand for
+            // d = 16r + 2mt and 16r + 2mt + 1, i.e. bytes 2mt, 2mt + 1 of the
+            // thread's chunk of each key, paired across keys by a byte permute
+            auto pv = [&](const uint4 (&vr)[4], uint32_t pb0, uint32_t pb1) {
+#pragma unroll
+                for (int mt = 0; mt < D / 16; mt++) {
+                    const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+                    const uint32_t pa = prmt(u4_word(vr[0], mt >> 1), u4_word(vr[1], mt >> 1), sel);
+                    const uint32_t pc = prmt(u4_word(vr[2], mt >> 1), u4_word(vr[3], mt >> 1), sel);
+                    mma_f16_16816(oacc[mt], e4m3_lo(pa), e4m3_hi(pa), e4m3_lo(pc), e4m3_hi(pc), pb0, pb1);
+                }
+            };
+            for (int i = 0; i < nb; i += 2) {
+                const bool two = i + 1 < nb;   // warp-uniform
+                const int sa = i % NS, sb = (i + 1) % NS;
+                if (!mbar_wait(&full[sa], (i / NS) & 1, &abort_flag, 40)) break;
+                if (two && !mbar_wait(&full[sb], ((i + 1) / NS) & 1, &abort_flag, 40)) break;
+                uint4 kra[4], vra[4], krb[4], vrb[4];
+                float kqa[2], vpa[2], kqb[2] = {0.f, 0.f}, vpb[2] = {0.f, 0.f};
+                load(sa, kra, vra, kqa, vpa);
+                if (two) load(sb, krb, vrb, kqb, vpb);
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&empty[sa]);
+                    if (two) mbar_arrive(&empty[sb]);
+                }
+                float xa[4] = {0.f, 0.f, 0.f, 0.f}, xb[4] = {0.f, 0.f, 0.f, 0.f};
+                scores(kra, xa);
+                if (two) scores(krb, xb);
+                mask_scale(xa, (Lb - 1) - 64 * blocks[i], kqa);
+                mask_scale(xb, two ? (Lb - 1) - 64 * blocks[i + 1] : -1, kqb);
+                // ---- online softmax per head over the warp's keys of both blocks
+                float mx0 = fmaxf(fmaxf(xa[0], xa[2]), fmaxf(xb[0], xb[2]));
+                float mx1 = fmaxf(fmaxf(xa[1], xa[3]), fmaxf(xb[1], xb[3]));
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                }
+                const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+                // a head whose keys are all masked so far keeps a finite reference
+                const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
+                const float al0 = fast_exp2(m_run[0] - mu0), al1 = fast_exp2(m_run[1] - mu1);
+                m_run[0] = mn0;
+                m_run[1] = mn1;
+                const float pa0 = fast_exp2(xa[0] - mu0), pa1 = fast_exp2(xa[1] - mu1);
+                const float pa2 = fast_exp2(xa[2] - mu0), pa3 = fast_exp2(xa[3] - mu1);
+                const float pb0 = fast_exp2(xb[0] - mu0), pb1 = fast_exp2(xb[1] - mu1);
+                const float pb2 = fast_exp2(xb[2] - mu0), pb3 = fast_exp2(xb[3] - mu1);
+                l_run[0] = l_run[0] * al0 + ((pa0 + pa2) + (pb0 + pb2));
+                l_run[1] = l_run[1] * al1 + ((pa1 + pa3) + (pb1 + pb3));
+#pragma unroll
+                for (int mt = 0; mt < D / 16; mt++) {
+                    oacc[mt][0] *= al0;
+                    oacc[mt][1] *= al1;
+                    oacc[mt][2] *= al0;
+                    oacc[mt][3] *= al1;
+                }
+                // P^T as the B operand (k = key, n = head): transpose the two
+                // 8x8 halves of the S^T accumulator fragment
+                pv(vra, movmatrix_t(pack_f16x2(pa0 * vpa[0], pa1 * vpa[0])),
+                   movmatrix_t(pack_f16x2(pa2 * vpa[1], pa3 * vpa[1])));
+                if (two)
+                    pv(vrb, movmatrix_t(pack_f16x2(pb0 * vpb[0], pb1 * vpb[0])),
+                       movmatrix_t(pack_f16x2(pb2 * vpb[1], pb3 * vpb[1])));
+            }
+        } else {
         for (int i = 0; i < nb; i++) {
             const int st = i % NS;
             if (!mbar_wait(&full[st], (i / NS) & 1, &abort_flag, 40)) break;
@@ -300,6 +493,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
         }
+        }
         // row sums over the warp's keys: lanes with equal lane%4 hold the same heads
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1) {
@@ -329,10 +523,14 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_
         }
 #pragma unroll
         for (int mt = 0; mt < D / 16; mt++) {
-            wp[16 + qc * D + 16 * mt + hn] = oacc[mt][0];
-            wp[16 + (qc + 1) * D + 16 * mt + hn] = oacc[mt][1];
-            wp[16 + qc * D + 16 * mt + 8 + hn] = oacc[mt][2];
-            wp[16 + (qc + 1) * D + 16 * mt + 8 + hn] = oacc[mt][3];
+            // MMA row (mt, i) of O^T is d = 16mt + i, or in the fp8 order
+            // d = 16i + 2mt (i < 8) and 16(i - 8) + 2mt + 1
+            const int d0 = FP8 ? 16 * hn + 2 * mt : 16 * mt + hn;
+            const int d1 = FP8 ? 16 * hn + 2 * mt + 1 : 16 * mt + 8 + hn;
+            wp[16 + qc * D + d0] = oacc[mt][0];
+            wp[16 + (qc + 1) * D + d0] = oacc[mt][1];
+            wp[16 + qc * D + d1] = oacc[mt][2];
+            wp[16 + (qc + 1) * D + d1] = oacc[mt][3];
         }
     }
     // ---- one merge over the row's P x NC partials (distributed shared memory)
@@ -358,7 +556,54 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS, DecodeCfg<D>::CTAS_PER_
         inv_l[h] = lc > 0.f ? 1.f / lc : 0.f;
     }
     __syncthreads();
-    {
+    if constexpr (FP8) {
+        // whole heads per CTA (h = rank, rank + P, ...): the heads' rotated
+        // outputs o' are summed over the sources in 4 groups (float4 loads
+        // through distributed shared memory, all of the CTA's heads in one
+        // pass) into scratch after the partials; then one warp per head adds
+        // the groups and rotates back, o = WHT(o') / 128 (the transform
+        // squared is 128 I)
+        float4 *scr = reinterpret_cast<float4 *>(part + NC * PF);   // [head][group][D/4], not read remotely
+        const int nh = (G - rank + P - 1) / P;
+        if (threadIdx.x < 4 * (D / 4)) {
+            const int c4 = threadIdx.x % (D / 4), sg = threadIdx.x / (D / 4);
+            for (int hl = 0; hl < nh; hl++) {
+                const int h = rank + hl * P;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+                for (int src = sg; src < nsrc; src += 4) {
+                    const float f = wgt[src][h];
+                    const float4 x = *reinterpret_cast<const float4 *>(
+                        cluster.map_shared_rank(part, src / NC) + (src % NC) * PF + 16 + h * D + 4 * c4);
+                    acc.x += f * x.x;
+                    acc.y += f * x.y;
+                    acc.z += f * x.z;
+                    acc.w += f * x.w;
+                }
+                scr[(hl * 4 + sg) * (D / 4) + c4] = acc;
+            }
+        }
+        __syncthreads();
+        for (int hl = warp; hl < nh; hl += NC + 1) {
+            const int h = rank + hl * P;
+            float4 a = scr[(hl * 4) * (D / 4) + lane];
+#pragma unroll
+            for (int sg = 1; sg < 4; sg++) {
+                const float4 t = scr[(hl * 4 + sg) * (D / 4) + lane];
+                a.x += t.x;
+                a.y += t.y;
+                a.z += t.z;
+                a.w += t.w;
+            }
+            const float f = inv_l[h] * (1.0f / 128.0f);
+            float x[4] = {a.x, a.y, a.z, a.w};
+            fwht_warp<4>(x);
+            uint2 out;
+            out.x = pack_bf16x2(x[0] * f, x[1] * f);
+            out.y = pack_bf16x2(x[2] * f, x[3] * f);
+            *reinterpret_cast<uint2 *>(o + ((long)b * Hq + g * G + h) * D + 4 * lane) = out;
+        }
+    } else {
         const int n4 = G * D / 4;
         const int per = (n4 + P - 1) / P;
         const int e_end = min(n4, (rank + 1) * per);

@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -196,6 +197,22 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// Untiled bulk copy global -> this CTA's shared memory, completing on an
+// mbarrier (both addresses 16-byte aligned, bytes a multiple of 16).
+// Barrier `id` (1..15) among `count` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_barrier_sync(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -369,6 +386,60 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);   // .x = lo (low half)
     return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
+{
+    __half2 v = __floats2half2_rn(lo, hi);   // .x = lo (low half)
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// ---------------------------------------------- rotated fp8 KV (decode option)
+// Unnormalised Walsh-Hadamard transform of a warp's 32*V values, element
+// e = V*lane + k in x[k], in place: for len = 1, 2, ..., 16V every pair
+// (j, j + len) with j mod 2 len < len becomes (x_j + x_{j+len},
+// x_j - x_{j+len}) -- stage by stage in increasing len, so every output is
+// a fixed sequence of fp32 additions and the codes derived from it are
+// reproducible on any implementation that follows the same order.
+template <int V>
+__device__ __forceinline__ void fwht_warp(float (&x)[V])
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int len = 1; len < V; len <<= 1) {
+#pragma unroll
+        for (int k = 0; k < V; k++) {
+            if (k & len) continue;
+            const float a = x[k], b = x[k + len];
+            x[k] = a + b;
+            x[k + len] = a - b;
+        }
+    }
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {   // len = V * m
+#pragma unroll
+        for (int k = 0; k < V; k++) {
+            const float y = __shfl_xor_sync(0xffffffffu, x[k], m);
+            x[k] = (lane & m) ? y - x[k] : x[k] + y;
+        }
+    }
+}
+
+// Two fp32 values -> fp8 e4m3 codes (lo in the low byte): nearest, ties to
+// even, saturating to +-448.
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Two fp8 e4m3 codes (low byte first) -> f16x2 (exact).
+__device__ __forceinline__ uint32_t cvt_e4m3x2_f16x2(uint16_t v)
+{
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+    return r;
 }
 
 __device__ __forceinline__ float fast_exp2(float x)

@@ -16,6 +16,7 @@
 #include "decode.cuh"
 #include "device.cuh"
 #include "prefill.cuh"
+#include "quant.cuh"
 #include "select.cuh"
 
 namespace {
@@ -84,6 +85,22 @@ qsa_status make_map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t
                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(QSA_ERR_CUDA, "cuTensorMapEncodeTiled(2d) failed: %d", (int)r);
+    return QSA_OK;
+}
+
+// 2-D byte view [rows][cols] (fp8 codes) with 64-row x 128-byte boxes, 128-byte swizzle.
+qsa_status make_map_2d_u8(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(QSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {128, 64};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(QSA_ERR_CUDA, "cuTensorMapEncodeTiled(2d, u8) failed: %d", (int)r);
     return QSA_OK;
 }
 
@@ -241,20 +258,26 @@ qsa_status launch_prefill(const void *Q, const void *K, const void *V, const int
     return launched("sparse_attn_prefill_kernel");
 }
 
-template <int D, int G>
+template <int D, int G, bool FP8 = false>
 qsa_status launch_decode(const void *q, const void *K, const void *V, const int32_t *idx, void *o,
                          int B, int Hq, int Hkv, int L, int T_kv_max, int topk, float sm_scale,
-                         cudaStream_t s, const Paging &pg = Paging())
+                         cudaStream_t s, const Paging &pg = Paging(), const float *k_scales = nullptr,
+                         const float *v_scales = nullptr)
 {
-    using C = qsa::DecodeCfg<D>;
+    using C = qsa::DecodeCfg<D, FP8>;
     CUtensorMap mk, mv;
     qsa_status st;
     // cache rows: [B][Hkv][T_kv_max], or [num_pages][Hkv][64] when paged
     const uint64_t nrows = pg.block_table ? (uint64_t)pg.num_pages * Hkv * 64 : (uint64_t)B * Hkv * T_kv_max;
-    if ((st = make_map_2d(&mk, K, nrows, D)) != QSA_OK) return st;
-    if ((st = make_map_2d(&mv, V, nrows, D)) != QSA_OK) return st;
+    if constexpr (FP8) {
+        if ((st = make_map_2d_u8(&mk, K, nrows, D)) != QSA_OK) return st;
+        if ((st = make_map_2d_u8(&mv, V, nrows, D)) != QSA_OK) return st;
+    } else {
+        if ((st = make_map_2d(&mk, K, nrows, D)) != QSA_OK) return st;
+        if ((st = make_map_2d(&mv, V, nrows, D)) != QSA_OK) return st;
+    }
     const DecodePlan p = plan_decode(B * Hkv, topk, sm_count(), C::CTAS_PER_SM);
-    auto kern = qsa::decode_kernel<D, G>;
+    auto kern = qsa::decode_kernel<D, G, FP8>;
     if ((st = set_smem(kern, C::SMEM_BYTES)) != QSA_OK) return st;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.P, B * Hkv, 1);
@@ -272,7 +295,8 @@ qsa_status launch_decode(const void *q, const void *K, const void *V, const int3
     cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mk, mv, (const __nv_bfloat16 *)q, idx, (__nv_bfloat16 *)o, Hq,
                                        Hkv, L, T_kv_max, topk, p.spc, sm_scale * 1.4426950408889634f,
-                                       pg.seq_lens, pg.block_table, pg.max_blocks, pg.num_pages);
+                                       pg.seq_lens, pg.block_table, pg.max_blocks, pg.num_pages, k_scales,
+                                       v_scales);
     if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "decode_kernel launch: %s", cudaGetErrorString(e));
     return launched("decode_kernel");
 }
@@ -713,6 +737,48 @@ qsa_status qsa_decode_paged(const void *q, const void *K_pages, const void *V_pa
     if (d == 128 && G == 4) return launch_decode<128, 4>(q, K_pages, V_pages, idx, o, B, Hq, Hkv, T, T, topk, sm_scale, s, pg);
     if (d == 64 && G == 8) return launch_decode<64, 8>(q, K_pages, V_pages, idx, o, B, Hq, Hkv, T, T, topk, sm_scale, s, pg);
     return launch_decode<64, 4>(q, K_pages, V_pages, idx, o, B, Hq, Hkv, T, T, topk, sm_scale, s, pg);
+}
+
+qsa_status qsa_quantize_kv_fp8(const void *X, void *codes, float *scales, int64_t rows, int d,
+                               qsa_stream_t stream)
+{
+    if (!X || !codes || !scales) return fail(QSA_ERR_INVALID_ARG, "qsa_quantize_kv_fp8: null pointer");
+    if (rows < 0) return fail(QSA_ERR_INVALID_ARG, "qsa_quantize_kv_fp8: rows=%lld", (long long)rows);
+    if (d != 128) return fail(QSA_ERR_UNSUPPORTED, "qsa_quantize_kv_fp8: d=%d (rotated fp8 rows are 128 wide)", d);
+    if (!aligned16(X) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3))
+        return fail(QSA_ERR_INVALID_ARG, "qsa_quantize_kv_fp8: misaligned pointer");
+    if (rows == 0) return QSA_OK;
+    const long blocks = (rows + 7) / 8;   // 8 rows (warps) per CTA
+    if (blocks >= (1L << 31)) return fail(QSA_ERR_UNSUPPORTED, "qsa_quantize_kv_fp8: too many rows");
+    qsa::quantize_kv_fp8_kernel<128><<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16 *>(X), static_cast<uint8_t *>(codes), scales, (long)rows);
+    return launched("quantize_kv_fp8_kernel");
+}
+
+qsa_status qsa_decode_fp8(const void *q, const void *K_codes, const float *K_scales, const void *V_codes,
+                          const float *V_scales, const int32_t *idx, void *o, int B, int Hq, int Hkv, int L,
+                          int T_kv_max, int d, int topk, float sm_scale, qsa_stream_t stream)
+{
+    const char *name = "qsa_decode_fp8";
+    if (!q || !K_codes || !K_scales || !V_codes || !V_scales || !idx || !o)
+        return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || T_kv_max <= 0 || T_kv_max % 64 || L > T_kv_max || Hq % Hkv)
+        return fail(QSA_ERR_INVALID_ARG, "%s: bad shape", name);
+    if ((long)B * Hkv * T_kv_max >= (1L << 31)) return fail(QSA_ERR_UNSUPPORTED, "%s: cache too large", name);
+    if (d != 128) return fail(QSA_ERR_UNSUPPORTED, "%s: d=%d (rotated fp8 rows are 128 wide)", name, d);
+    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "%s: topk=%d", name, topk);
+    const int G = Hq / Hkv;
+    if (G != 4 && G != 8) return fail(QSA_ERR_UNSUPPORTED, "%s: Hq/Hkv=%d", name, G);
+    if (!aligned16(q) || !aligned16(K_codes) || !aligned16(V_codes) || !aligned16(K_scales) ||
+        !aligned16(V_scales) || !aligned16(idx) || !aligned16(o))
+        return fail(QSA_ERR_INVALID_ARG, "%s: misaligned pointer", name);
+    if (B * Hkv > 65535) return fail(QSA_ERR_UNSUPPORTED, "%s: more than 65535 (sequence, group) rows", name);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (G == 8)
+        return launch_decode<128, 8, true>(q, K_codes, V_codes, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, s,
+                                           Paging(), K_scales, V_scales);
+    return launch_decode<128, 4, true>(q, K_codes, V_codes, idx, o, B, Hq, Hkv, L, T_kv_max, topk, sm_scale, s,
+                                       Paging(), K_scales, V_scales);
 }
 
 qsa_status qsa_get_device_status(qsa_stream_t stream, int *detail)

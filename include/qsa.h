@@ -254,6 +254,43 @@ QSA_API qsa_status qsa_decode_paged(const void *q, const void *K_pages, const vo
                                     qsa_stream_t stream);
 
 /*
+ * Quantized-KV option for decode (page "Qwen4 in llama.cpp: Dissecting PR
+ * #27742", section "Quantized KV Exposed a Backend Storage Invariant"): the
+ * cache holds K and V in a Walsh-Hadamard-rotated basis as fp8 e4m3 codes
+ * with one fp32 scale per (token, head) row; attention runs in that basis
+ * and the output is rotated back.  d = 128.  The selection keeps reading the
+ * summaries of the unrotated keys (qsa_compress_keys on the bf16 K): it
+ * returns cell addresses, which the rotation does not change.
+ *
+ * qsa_quantize_kv_fp8: for each of `rows` rows of 128 bf16 values x (row r
+ * at X + 128 r): u = WHT(x), the unnormalised 128-point Walsh-Hadamard
+ * transform in fp32 (butterfly stages len = 1, 2, ..., 64, each pair
+ * becoming (a + b, a - b)); scales[r] = max|u| / 448; codes (row r at
+ * codes + 128 r) = e4m3(u / scales[r]), nearest with ties to even,
+ * saturating (zeros when the row is zero).  Rows [B][Hkv][T_kv_max] of a
+ * cache are rows = B*Hkv*T_kv_max; a single new token's rows can be written
+ * alone.
+ * qsa_decode_fp8: qsa_decode over such a cache (codes uint8
+ * [B][Hkv][T_kv_max][128], scales fp32 [B][Hkv][T_kv_max]); q and o bf16 in
+ * the original basis.  Scores are (WHT(q) . u) / 128 = q . k up to the
+ * quantization; o = WHT(o') / 128.  idx, L, topk and sm_scale as for
+ * qsa_decode (an index past the token's block sets QSA_ERR_BOUNDS on the
+ * device and is skipped).  All buffers are the caller's device memory.
+ * Errors, before any launch: a null pointer, a bad shape (L > T_kv_max,
+ * T_kv_max not a multiple of 64, Hq not a multiple of Hkv) or a pointer not
+ * 16-byte aligned (X, codes, q, o, idx, both scale arrays of the decode;
+ * the quantizer's scales need 4 bytes) -> QSA_ERR_INVALID_ARG; d != 128,
+ * Hq/Hkv not 4 or 8, topk outside 2..64 or a cache of 2^31 rows or more ->
+ * QSA_ERR_UNSUPPORTED.  rows == 0 is a no-op.
+ */
+QSA_API qsa_status qsa_quantize_kv_fp8(const void *X, void *codes, float *scales, int64_t rows, int d,
+                                       qsa_stream_t stream);
+QSA_API qsa_status qsa_decode_fp8(const void *q, const void *K_codes, const float *K_scales,
+                                  const void *V_codes, const float *V_scales, const int32_t *idx,
+                                  void *o, int B, int Hq, int Hkv, int L, int T_kv_max, int d,
+                                  int topk, float sm_scale, qsa_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word
  * (QSA_OK if no kernel recorded an error since the last call).  If detail
  * is not NULL it receives a kernel-specific code (0 if none).

@@ -83,6 +83,19 @@ def test_argument_checks_return_before_launch():
     assert dc(L=2000) == 1
     assert lib.qsa_decode(fake, fake, fake, fake, fake, 40000, 16, 2, 64, 64, 128, 8, 0.088,
                           None, 0, None) == 2          # too many (sequence, group) rows
+    # rotated fp8 cache: rows are 128 wide, scales 4-byte aligned, no negative count
+    assert lib.qsa_quantize_kv_fp8(fake, fake, fake, 4, 64, None) == 2
+    assert lib.qsa_quantize_kv_fp8(fake, fake, P(0x1002), 4, 128, None) == 1
+    assert lib.qsa_quantize_kv_fp8(fake, fake, fake, -1, 128, None) == 1
+    assert lib.qsa_quantize_kv_fp8(fake, fake, fake, 0, 128, None) == 0      # nothing to do
+    d8 = lambda Hq=16, L=1000, d=128, topk=8, ks=fake: lib.qsa_decode_fp8(
+        fake, fake, ks, fake, fake, fake, fake, 4, Hq, 2, L, 1024, d, topk, 0.088, None)
+    assert d8(d=64) == 2
+    assert d8(Hq=12) == 2
+    assert d8(L=2000) == 1
+    assert d8(topk=65) == 2
+    assert d8(ks=odd) == 1
+    assert d8(ks=None) == 1
     # self-test limit out of range
     assert lib.qsa_selftest_wait_timeout(0, None) == 1
 

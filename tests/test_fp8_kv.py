@@ -1,0 +1,76 @@
+"""Quantized-KV option for decode: the cache in a Walsh-Hadamard-rotated
+basis as fp8 e4m3 codes with a per-row scale, attention in that basis, the
+output rotated back (page "Qwen4 in llama.cpp: Dissecting PR #27742",
+section "Quantized KV Exposed a Backend Storage Invariant").
+
+The codes and scales are integer-like decisions taken in fp32 on both sides,
+so they must match the oracle bit for bit; the attention is compared with
+the oracle's fp64 attention over its own codes (max |err| <= 1e-2, mean
+<= 1e-3).  The difference from attention over the unquantized cache is the
+quantization itself and is only reported.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from tests.helpers import check_out
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def qsa():
+    import block_sparse_long_compress_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+def test_quantize_kv_fp8_matches_oracle_bit_for_bit(qsa):
+    w = synthetic.custom(B=2, Tq=1, T_kv=64 * 40, q_pos0=64 * 40 - 1, qblk=1, Hq=16, Hkv=2, d=128, seed=141)
+    x = synthetic.generate(w)
+    for X in (x["K"], x["V"]):
+        codes, scales = qsa.quantize_kv_fp8(X.to(DEV))
+        st = qsa.device_status()
+        assert st[0] == "QSA_OK", st
+        ref_c, ref_s = oracle.quantize_kv_fp8(X)
+        assert np.array_equal(codes.cpu().numpy(), ref_c)
+        assert np.array_equal(scales.cpu().numpy(), ref_s)
+    # an all-zero row quantizes to zero codes and scale
+    z = torch.zeros((3, 128), dtype=torch.bfloat16, device=DEV)
+    c, s = qsa.quantize_kv_fp8(z)
+    assert (c == 0).all() and (s == 0).all()
+
+
+CASES = [
+    ("g8", dict(B=4, T=64 * 300, L=64 * 300 - 9, Hq=16, Hkv=2, topk=16)),
+    ("g4_short", dict(B=3, T=64 * 60, L=64 * 41 + 5, Hq=8, Hkv=2, topk=8)),
+]
+
+
+@pytest.mark.parametrize("name,kw", CASES, ids=[c[0] for c in CASES])
+def test_decode_fp8_parity(qsa, name, kw):
+    L = kw["L"]
+    w = synthetic.custom(B=kw["B"], Tq=1, T_kv=kw["T"], q_pos0=L - 1, qblk=1, Hq=kw["Hq"], Hkv=kw["Hkv"],
+                         d=128, topk=kw["topk"], seed=151)
+    x = synthetic.generate(w)
+    sel, O_bf16 = oracle.qsa_forward(x["Q"], x["K"][:, :, :L], x["V"][:, :, :L], w.Hkv, w.topk, q_pos0=L - 1,
+                                     qblk=1)
+    idx = torch.from_numpy(sel["idx"]).to(DEV)                # [B, Hkv, 1, topk]
+    q = x["Q"].to(DEV).view(w.B, w.Hq, 128)
+    kc, ks = qsa.quantize_kv_fp8(x["K"].to(DEV))
+    vc, vs = qsa.quantize_kv_fp8(x["V"].to(DEV))
+    o = torch.full_like(q, float("nan"))
+    for _ in range(2):
+        qsa.decode_fp8(q, kc, ks, vc, vs, idx, o, L, w.sm_scale)
+        st = qsa.device_status()
+        assert st[0] == "QSA_OK", st
+    ck, sk = oracle.quantize_kv_fp8(x["K"])
+    cv, sv = oracle.quantize_kv_fp8(x["V"])
+    ref = oracle.decode_fp8(x["Q"].view(w.B, w.Hq, 128), ck, sk, cv, sv, sel["idx"], L, w.sm_scale)
+    mx, mean = check_out(o.float().cpu().numpy(), ref)
+    qerr = np.abs(ref - O_bf16[:, 0]).max()
+    print(f"{name}: o max {mx:.2e} mean {mean:.2e}; quantization vs bf16 cache: max {qerr:.2e}")
