@@ -60,8 +60,8 @@ struct DecodeCfg {
     static_assert(NS >= 2, "ring too small");
     static_assert(NC * PART_FLOATS * 4 + 4 * D <= RING_BYTES, "merge scratch must fit in the ring");
     static_assert(!FP8 || D == 128, "rotated fp8 rows are 128 wide");
-    // FP8 merge: up to 8 heads x 4 source groups x D floats after the partials
-    static_assert(!FP8 || NC * PART_FLOATS * 4 + 8 * 4 * D * 4 <= RING_BYTES, "fp8 merge scratch");
+    // merge inbox after the partials: at most ceil(G/P) * P <= 15 slots of 4 + D floats
+    static_assert((NC * PART_FLOATS + 15 * (4 + D)) * 4 <= RING_BYTES, "merge inbox must fit in the ring");
 };
 
 __device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -143,7 +143,6 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
     constexpr int NS = C::NS;
     constexpr int NC = C::NC;
     constexpr int PF = C::PART_FLOATS;
-    constexpr int MAX_SRC = C::MAX_CLUSTER * NC;
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
 
@@ -152,9 +151,8 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
     __shared__ int blocks[C::MAX_SLOTS];   // the CTA's valid block ids in slot order
     __shared__ int rows[C::MAX_SLOTS];     // and the first cache row of each (TMA coordinate)
     __shared__ int nb_sh, issued_sh, abort_flag;
-    __shared__ float wgt[MAX_SRC][8];      // per-source, per-head merge weights
-    __shared__ float lsrc[MAX_SRC][8];
-    __shared__ float inv_l[8];
+    __shared__ float wloc[NC][8];          // merge weights of the CTA's warps, per head
+    __shared__ float mloc[8], lloc[8];     // the CTA's combined max and sum per head
     __shared__ __align__(16) uint32_t uq[FP8 ? 8 * (D / 2) : 1];   // FP8: rotated queries, f16 pairs
 
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -170,6 +168,31 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
     // the selection that writes idx) has completed
     grid_dependency_wait();
     grid_launch_dependents();
+    // the group's queries, loaded by the consumer warps first thing, ahead
+    // of the cache copies that every CTA starts after the prologue.  B
+    // operand of S^T = K q^T: column n = head lane/4 of the group (zero for
+    // n >= G), rows k = d; FP8: raw rows of heads warp, warp + NC, ...,
+    // rotated below
+    const int hn = lane >> 2, qc = (lane & 3) * 2;
+    uint32_t qb[D / 16][2];
+    uint2 qraw[FP8 ? (G + NC - 1) / NC : 1];
+    if (warp < NC) {
+        if constexpr (FP8) {
+#pragma unroll
+            for (int j = 0; j < (G + NC - 1) / NC; j++)
+                if (warp + j * NC < G)
+                    qraw[j] = __ldg(reinterpret_cast<const uint2 *>(q + ((long)b * Hq + g * G + warp + j * NC) * D) + lane);
+        } else {
+            const __nv_bfloat16 *qrow = q + ((long)b * Hq + g * G + (hn < G ? hn : 0)) * D;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; kk++) {
+                const uint32_t lo = __ldg(reinterpret_cast<const uint32_t *>(qrow + 16 * kk + qc));
+                const uint32_t hi = __ldg(reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 8 + qc));
+                qb[kk][0] = hn < G ? lo : 0u;
+                qb[kk][1] = hn < G ? hi : 0u;
+            }
+        }
+    }
     // this sequence's cache length (the current token is its last position)
     int Lb = L;
     if (seq_lens) {
@@ -269,22 +292,20 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
         }
     } else {
         // ---------------------------------------------------- consumers
-        // B operand of S^T = K q^T: column n = head lane/4 of the group
-        // (zero for n >= G), rows k = d.
-        const int hn = lane >> 2, qc = (lane & 3) * 2;
-        uint32_t qb[D / 16][2];
         if constexpr (FP8) {
             // the group's queries in the rotated basis (unnormalised
-            // transform, as f16 pairs; consumer warp w takes heads w, w + NC,
-            // ...), shared among the consumer warps only, so that the
-            // producer's first copies are not held back by these loads
-            for (int h = warp; h < G; h += NC) {
-                const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(q + ((long)b * Hq + g * G + h) * D) + lane);
-                float x[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
-                              __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
-                fwht_warp<4>(x);
-                uq[h * (D / 2) + 2 * lane] = pack_f16x2(x[0], x[1]);
-                uq[h * (D / 2) + 2 * lane + 1] = pack_f16x2(x[2], x[3]);
+            // transform, as f16 pairs), shared among the consumer warps only
+#pragma unroll
+            for (int j = 0; j < (G + NC - 1) / NC; j++) {
+                const int h = warp + j * NC;
+                if (h < G) {
+                    const uint2 raw = qraw[j];
+                    float x[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                                  __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
+                    fwht_warp<4>(x);
+                    uq[h * (D / 2) + 2 * lane] = pack_f16x2(x[0], x[1]);
+                    uq[h * (D / 2) + 2 * lane + 1] = pack_f16x2(x[2], x[3]);
+                }
             }
             named_barrier_sync(1, NC * 32);
             // rotated queries (f16) from the shared copy.  The contraction
@@ -297,15 +318,6 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
             for (int kk = 0; kk < D / 16; kk++) {
                 qb[kk][0] = hn < G ? uqh[8 * qc + 2 * kk] : 0u;
                 qb[kk][1] = hn < G ? uqh[8 * qc + 2 * kk + 1] : 0u;
-            }
-        } else {
-            const __nv_bfloat16 *qrow = q + ((long)b * Hq + g * G + (hn < G ? hn : 0)) * D;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; kk++) {
-                const uint32_t lo = *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + qc);
-                const uint32_t hi = *reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 8 + qc);
-                qb[kk][0] = hn < G ? lo : 0u;
-                qb[kk][1] = hn < G ? hi : 0u;
             }
         }
         const int k0 = 16 * warp;                                  // the warp's keys in each block
@@ -514,7 +526,6 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
     // ---- warp partials (m, l, O) into the idle ring
     if (warp < NC) {
         float *wp = part + warp * PF;
-        const int hn = lane >> 2, qc = (lane & 3) * 2;
         if (lane < 4) {
             wp[qc] = m_run[0];
             wp[qc + 1] = m_run[1];
@@ -533,101 +544,89 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
             wp[16 + (qc + 1) * D + d1] = oacc[mt][3];
         }
     }
-    // ---- one merge over the row's P x NC partials (distributed shared memory)
-    cluster.sync();
-    const int nsrc = P * NC;
-    for (int e = threadIdx.x; e < nsrc * G; e += C::THREADS) {
-        const int src = e / G, h = e % G;
-        const float *pp = cluster.map_shared_rank(part, src / NC) + (src % NC) * PF;
-        wgt[src][h] = pp[h];          // m, turned into a weight below
-        lsrc[src][h] = pp[8 + h];
-    }
     __syncthreads();
+    // ---- merge.  Head h of the group is finished by CTA h % P of the
+    // cluster.  Each CTA combines its NC warps per head (weights here, before
+    // the cluster barrier, while slower CTAs may still be streaming), then
+    // stores its combined (max, sum, unnormalised O) into slot
+    // [h / P][its rank] of the owner's inbox with plain stores through
+    // distributed shared memory; after a second barrier each owner merges
+    // its inbox locally.  The inbox lies in the owner's ring past its own
+    // partials, so the first barrier (every ring idle) comes before any
+    // store into it.
+    constexpr int SLOT = 4 + D;                          // max, sum, 2 pad, O[D]
+    float *inbox = part + NC * PF;                       // [ceil(G/P)][P][SLOT]
     if (threadIdx.x < G) {
         const int h = threadIdx.x;
         float mc = -INFINITY;
-        for (int src = 0; src < nsrc; src++) mc = fmaxf(mc, wgt[src][h]);
-        float lc = 0.f;
-        for (int src = 0; src < nsrc; src++) {
-            const float f = mc == -INFINITY ? 0.f : fast_exp2(wgt[src][h] - mc);
-            wgt[src][h] = f;
-            lc += f * lsrc[src][h];
-        }
-        inv_l[h] = lc > 0.f ? 1.f / lc : 0.f;
-    }
-    __syncthreads();
-    if constexpr (FP8) {
-        // whole heads per CTA (h = rank, rank + P, ...): the heads' rotated
-        // outputs o' are summed over the sources in 4 groups (float4 loads
-        // through distributed shared memory, all of the CTA's heads in one
-        // pass) into scratch after the partials; then one warp per head adds
-        // the groups and rotates back, o = WHT(o') / 128 (the transform
-        // squared is 128 I)
-        float4 *scr = reinterpret_cast<float4 *>(part + NC * PF);   // [head][group][D/4], not read remotely
-        const int nh = (G - rank + P - 1) / P;
-        if (threadIdx.x < 4 * (D / 4)) {
-            const int c4 = threadIdx.x % (D / 4), sg = threadIdx.x / (D / 4);
-            for (int hl = 0; hl < nh; hl++) {
-                const int h = rank + hl * P;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-                for (int src = sg; src < nsrc; src += 4) {
-                    const float f = wgt[src][h];
-                    const float4 x = *reinterpret_cast<const float4 *>(
-                        cluster.map_shared_rank(part, src / NC) + (src % NC) * PF + 16 + h * D + 4 * c4);
-                    acc.x += f * x.x;
-                    acc.y += f * x.y;
-                    acc.z += f * x.z;
-                    acc.w += f * x.w;
-                }
-                scr[(hl * 4 + sg) * (D / 4) + c4] = acc;
-            }
-        }
-        __syncthreads();
-        for (int hl = warp; hl < nh; hl += NC + 1) {
-            const int h = rank + hl * P;
-            float4 a = scr[(hl * 4) * (D / 4) + lane];
 #pragma unroll
-            for (int sg = 1; sg < 4; sg++) {
-                const float4 t = scr[(hl * 4 + sg) * (D / 4) + lane];
-                a.x += t.x;
-                a.y += t.y;
-                a.z += t.z;
-                a.w += t.w;
-            }
-            const float f = inv_l[h] * (1.0f / 128.0f);
-            float x[4] = {a.x, a.y, a.z, a.w};
-            fwht_warp<4>(x);
-            uint2 out;
-            out.x = pack_bf16x2(x[0] * f, x[1] * f);
-            out.y = pack_bf16x2(x[2] * f, x[3] * f);
-            *reinterpret_cast<uint2 *>(o + ((long)b * Hq + g * G + h) * D + 4 * lane) = out;
+        for (int w = 0; w < NC; w++) mc = fmaxf(mc, part[w * PF + h]);
+        float lc = 0.f;
+#pragma unroll
+        for (int w = 0; w < NC; w++) {
+            const float f = mc == -INFINITY ? 0.f : fast_exp2(part[w * PF + h] - mc);
+            wloc[w][h] = f;
+            lc += f * part[w * PF + 8 + h];
         }
-    } else {
-        const int n4 = G * D / 4;
-        const int per = (n4 + P - 1) / P;
-        const int e_end = min(n4, (rank + 1) * per);
-        for (int e4 = rank * per + threadIdx.x; e4 < e_end; e4 += C::THREADS) {
-            const int h = (e4 * 4) / D, c = (e4 * 4) % D;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-            for (int src = 0; src < nsrc; src++) {
-                const float f = wgt[src][h];
-                const float4 x = *reinterpret_cast<const float4 *>(
-                    cluster.map_shared_rank(part, src / NC) + (src % NC) * PF + 16 + h * D + c);
-                acc.x += f * x.x;
-                acc.y += f * x.y;
-                acc.z += f * x.z;
-                acc.w += f * x.w;
-            }
-            const float il = inv_l[h];
+        mloc[h] = mc;
+        lloc[h] = lc;
+    }
+    cluster.sync();   // every CTA's ring is idle; the local weights are visible
+    for (int e4 = threadIdx.x; e4 < G * D / 4; e4 += C::THREADS) {
+        const int h = (e4 * 4) / D, c = (e4 * 4) % D;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < NC; w++) {
+            const float f = wloc[w][h];
+            const float4 x = *reinterpret_cast<const float4 *>(part + w * PF + 16 + h * D + c);
+            acc.x += f * x.x;
+            acc.y += f * x.y;
+            acc.z += f * x.z;
+            acc.w += f * x.w;
+        }
+        float *slot = cluster.map_shared_rank(inbox, h % P) + ((h / P) * P + rank) * SLOT;
+        *reinterpret_cast<float4 *>(slot + 4 + c) = acc;
+    }
+    if (threadIdx.x < G) {
+        const int h = threadIdx.x;
+        float *slot = cluster.map_shared_rank(inbox, h % P) + ((h / P) * P + rank) * SLOT;
+        slot[0] = mloc[h];
+        slot[1] = lloc[h];
+    }
+    cluster.sync();   // the inboxes are complete; no shared memory is read remotely after this
+    // one warp per owned head: lane owns D/32 consecutive columns
+    constexpr int CPL = D / 32;
+    for (int j = warp; j * P + rank < G; j += NC + 1) {
+        const int h = j * P + rank;
+        const float *sl = inbox + j * P * SLOT;
+        float mc = -INFINITY;
+        for (int src = 0; src < P; src++) mc = fmaxf(mc, sl[src * SLOT]);
+        float lc = 0.f, x[CPL];
+#pragma unroll
+        for (int t = 0; t < CPL; t++) x[t] = 0.f;
+        for (int src = 0; src < P; src++) {
+            const float f = mc == -INFINITY ? 0.f : fast_exp2(sl[src * SLOT] - mc);
+            lc += f * sl[src * SLOT + 1];
+#pragma unroll
+            for (int t = 0; t < CPL; t++) x[t] += f * sl[src * SLOT + 4 + CPL * lane + t];
+        }
+        float il = lc > 0.f ? 1.f / lc : 0.f;
+        if constexpr (FP8) {
+            // back to the original basis: o = WHT(o') / 128 (the transform
+            // squared is 128 I)
+            fwht_warp<CPL>(x);
+            il *= 1.0f / 128.0f;
+        }
+        __nv_bfloat16 *orow = o + ((long)b * Hq + g * G + h) * D + CPL * lane;
+        if constexpr (CPL == 4) {
             uint2 out;
-            out.x = pack_bf16x2(acc.x * il, acc.y * il);
-            out.y = pack_bf16x2(acc.z * il, acc.w * il);
-            *reinterpret_cast<uint2 *>(o + ((long)b * Hq + g * G + h) * D + c) = out;
+            out.x = pack_bf16x2(x[0] * il, x[1] * il);
+            out.y = pack_bf16x2(x[2] * il, x[3] * il);
+            *reinterpret_cast<uint2 *>(orow) = out;
+        } else {
+            *reinterpret_cast<uint32_t *>(orow) = pack_bf16x2(x[0] * il, x[1] * il);
         }
     }
-    cluster.sync();   // the other CTAs' shared memory must outlive the reads into it
 }
 
 }  // namespace qsa
