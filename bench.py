@@ -311,6 +311,10 @@ def run_qsa(args, ws, rank, local):
         if args.paged:
             torch.cuda.empty_cache()
             result["decode"]["ragged_paged"] = bench_decode_paged(args, qsa, dev, peaks, ws, rank, flush)
+            if args.fp8_kv:
+                torch.cuda.empty_cache()
+                result["decode"]["ragged_paged"]["fp8_kv"] = bench_decode_paged(args, qsa, dev, peaks, ws, rank,
+                                                                                flush, kv="fp8")
         for name in filter(None, args.decode_more.split(",")):
             torch.cuda.empty_cache()
             result.setdefault("decode_more", {})[name] = bench_decode(args, qsa, dev, peaks, ws,
@@ -529,9 +533,10 @@ def bench_prefill_paged(args, qsa, dev, peaks, ws, rank, flush):
                          "flops_per_launch": flops, "traffic": None}}
 
 
-def bench_decode_paged(args, qsa, dev, peaks, ws, rank, flush):
+def bench_decode_paged(args, qsa, dev, peaks, ws, rank, flush, kv="bf16"):
     """Ragged batch over a paged cache: 32 sequences of 64K-256K tokens
-    (uniform), blocks in randomly placed pages, top-64 per token."""
+    (uniform), blocks in randomly placed pages, top-64 per token; kv="fp8":
+    the pages hold the rotated fp8 cache (written untimed)."""
     topk, Hq, Hkv, d = 64, 16, 2, 128
     x = synthetic.paged_decode(B=32, min_len=65536, max_len=262144, Hq=Hq, Hkv=Hkv, d=d,
                                seed=1007 + 1000 * rank, device=dev)
@@ -543,12 +548,23 @@ def bench_decode_paged(args, qsa, dev, peaks, ws, rank, flush):
         dec(*args_, x["max_len"])
     torch.cuda.synchronize()
     q4 = x["q"].view(B, 1, Hq, d)
+    if kv == "fp8":
+        kc, ks = qsa.quantize_kv_fp8(x["K_pages"])
+        vc, vs = qsa.quantize_kv_fp8(x["V_pages"])
+        del args_
+        x["K_pages"] = x["V_pages"] = None
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
 
     def run_parts(parts, s):
         if "select" in parts:
             qsa.score_select_ragged(q4, dec.Kc, x["seq_lens"], dec.idx, topk, x["max_len"], dec.sm_scale, s)
         if "attention" in parts:
-            qsa.decode_paged(*args_, dec.idx, dec.o, dec.sm_scale, s)
+            if kv == "fp8":
+                qsa.decode_fp8_paged(x["q"], kc, ks, vc, vs, x["block_table"], x["seq_lens"], dec.idx, dec.o,
+                                     dec.sm_scale, s)
+            else:
+                qsa.decode_paged(*args_, dec.idx, dec.o, dec.sm_scale, s)
 
     t, d_, launches = decode_timings(args, qsa, dev, ws, flush, run_parts)
     lens = x["seq_lens"].cpu().numpy().astype(np.int64)
@@ -557,11 +573,15 @@ def bench_decode_paged(args, qsa, dev, peaks, ws, rank, flush):
     Dg = (lens - 1) // 64
     nsel = np.minimum(topk, Dg + 1)
     keys = 64 * (nsel - 1) + (lens - 64 * Dg)
-    by = int(keys.sum()) * 2 * 2 * d * Hkv
+    # per selected key and head: K and V rows of d bf16 values, or of d
+    # fp8 codes plus a 4-byte scale
+    by = int(keys.sum()) * 2 * Hkv * ((d + 4) if kv == "fp8" else 2 * d)
     sel_bytes = int(((lens - 1) // 64).sum()) * Hkv * d * 4
+    extra = {"layout": "paged: [pages][Hkv][64][d], random block table; lengths uniform 64K-256K"}
+    if kv == "fp8":
+        extra["kv_cache"] = "fp8 e4m3, Walsh-Hadamard rotated, per-row fp32 scale"
     return decode_result("decode_ragged_paged", B, f"{int(lens.min())}-{int(lens.max())}", topk, t, d_,
-                         launches, by, sel_bytes, peaks,
-                         {"layout": "paged: [pages][Hkv][64][d], random block table; lengths uniform 64K-256K"})
+                         launches, by, sel_bytes, peaks, extra)
 
 
 def bench_e2e(args, qsa, dev, wp, ws):
@@ -725,6 +745,10 @@ def main():
         if args.paged and "paged" in variants:
             torch.cuda.empty_cache()
             res["ragged_paged"] = bench_decode_paged(args, qsa, dev, load_peaks(), ws, rank, flush)
+            if args.fp8_kv and "fp8" in variants:
+                torch.cuda.empty_cache()
+                res["ragged_paged"]["fp8_kv"] = bench_decode_paged(args, qsa, dev, load_peaks(), ws, rank, flush,
+                                                                   kv="fp8")
         for name in filter(None, args.decode_more.split(",")):
             torch.cuda.empty_cache()
             res.setdefault("decode_more", {})[name] = bench_decode(args, qsa, dev, load_peaks(), ws,

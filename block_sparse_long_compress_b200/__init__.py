@@ -59,6 +59,7 @@ def _load():
         "qsa_score_select_ragged_prefill": (I, [P, P, P, P, I, I, I, I, I, I, I, I, F, P, S, P]),
         "qsa_quantize_kv_fp8": (I, [P, P, P, ctypes.c_int64, I, P]),
         "qsa_decode_fp8": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
+        "qsa_decode_fp8_paged": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "qsa_sparse_attn_prefill_paged": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P]),
         "qsa_get_device_status": (I, [P, ctypes.POINTER(I)]),
         "qsa_selftest_wait_timeout": (I, [ctypes.c_uint64, P]),
@@ -329,6 +330,27 @@ def decode_fp8(q, K_codes, K_scales, V_codes, V_scales, idx, o, L, sm_scale=None
                                _ptr(V_scales, torch.float32, "V_scales"), _ptr(idx, torch.int32, "idx"),
                                _ptr(o, torch.bfloat16, "o"), B, Hq, Hkv, L, T, d, topk, float(sm_scale),
                                _stream(stream)), "qsa_decode_fp8")
+    return o
+
+
+def decode_fp8_paged(q, K_codes, K_scales, V_codes, V_scales, block_table, seq_lens, idx, o, sm_scale=None,
+                     stream=None):
+    """Decode attention over paged rotated fp8 caches: codes uint8
+    [num_pages, Hkv, 64, 128], scales fp32 [num_pages, Hkv, 64]; the rest as
+    decode_paged."""
+    B, Hq, d = q.shape
+    num_pages, Hkv, _, _ = K_codes.shape
+    max_blocks = block_table.shape[1]
+    topk = idx.shape[-1]
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    _check(_lib.qsa_decode_fp8_paged(_ptr(q, torch.bfloat16, "q"), _ptr(K_codes, torch.uint8, "K_codes"),
+                                     _ptr(K_scales, torch.float32, "K_scales"),
+                                     _ptr(V_codes, torch.uint8, "V_codes"), _ptr(V_scales, torch.float32, "V_scales"),
+                                     _ptr(block_table, torch.int32, "block_table"),
+                                     _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(idx, torch.int32, "idx"),
+                                     _ptr(o, torch.bfloat16, "o"), B, Hq, Hkv, max_blocks, num_pages, d, topk,
+                                     float(sm_scale), _stream(stream)), "qsa_decode_fp8_paged")
     return o
 
 

@@ -781,6 +781,41 @@ qsa_status qsa_decode_fp8(const void *q, const void *K_codes, const float *K_sca
                                        Paging(), K_scales, V_scales);
 }
 
+qsa_status qsa_decode_fp8_paged(const void *q, const void *K_codes, const float *K_scales, const void *V_codes,
+                                const float *V_scales, const int32_t *block_table, const int32_t *seq_lens,
+                                const int32_t *idx, void *o, int B, int Hq, int Hkv, int max_blocks, int num_pages,
+                                int d, int topk, float sm_scale, qsa_stream_t stream)
+{
+    const char *name = "qsa_decode_fp8_paged";
+    if (!q || !K_codes || !K_scales || !V_codes || !V_scales || !block_table || !seq_lens || !idx || !o)
+        return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || max_blocks <= 0 || num_pages <= 0)
+        return fail(QSA_ERR_INVALID_ARG, "%s: bad shape", name);
+    if ((long)num_pages * Hkv * 64 >= (1L << 31) || (long)max_blocks * 64 >= (1L << 31))
+        return fail(QSA_ERR_UNSUPPORTED, "%s: cache too large", name);
+    if (d != 128) return fail(QSA_ERR_UNSUPPORTED, "%s: d=%d (rotated fp8 rows are 128 wide)", name, d);
+    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "%s: topk=%d", name, topk);
+    const int G = Hq / Hkv;
+    if (G != 4 && G != 8) return fail(QSA_ERR_UNSUPPORTED, "%s: Hq/Hkv=%d", name, G);
+    if (!aligned16(q) || !aligned16(K_codes) || !aligned16(V_codes) || !aligned16(K_scales) ||
+        !aligned16(V_scales) || !aligned16(idx) || !aligned16(o) || (reinterpret_cast<uintptr_t>(block_table) & 3) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3))
+        return fail(QSA_ERR_INVALID_ARG, "%s: misaligned pointer", name);
+    if (B * Hkv > 65535) return fail(QSA_ERR_UNSUPPORTED, "%s: more than 65535 (sequence, group) rows", name);
+    Paging pg;
+    pg.seq_lens = seq_lens;
+    pg.block_table = block_table;
+    pg.max_blocks = max_blocks;
+    pg.num_pages = num_pages;
+    const int T = 64 * max_blocks;   // the kernel takes each sequence's length from seq_lens
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (G == 8)
+        return launch_decode<128, 8, true>(q, K_codes, V_codes, idx, o, B, Hq, Hkv, T, T, topk, sm_scale, s, pg,
+                                           K_scales, V_scales);
+    return launch_decode<128, 4, true>(q, K_codes, V_codes, idx, o, B, Hq, Hkv, T, T, topk, sm_scale, s, pg,
+                                       K_scales, V_scales);
+}
+
 qsa_status qsa_get_device_status(qsa_stream_t stream, int *detail)
 {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

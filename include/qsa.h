@@ -291,6 +291,21 @@ QSA_API qsa_status qsa_decode_fp8(const void *q, const void *K_codes, const floa
                                   int topk, float sm_scale, qsa_stream_t stream);
 
 /*
+ * qsa_decode_fp8_paged: qsa_decode_paged over a rotated fp8 cache in pages
+ * -- codes uint8 [num_pages][Hkv][64][128] and scales fp32
+ * [num_pages][Hkv][64] (a page's rows quantized by qsa_quantize_kv_fp8 like
+ * any other rows), block_table, seq_lens and idx as for qsa_decode_paged.
+ * Device-side checks and errors as for qsa_decode_paged; the argument
+ * checks as for qsa_decode_fp8.
+ */
+QSA_API qsa_status qsa_decode_fp8_paged(const void *q, const void *K_codes, const float *K_scales,
+                                        const void *V_codes, const float *V_scales,
+                                        const int32_t *block_table, const int32_t *seq_lens,
+                                        const int32_t *idx, void *o, int B, int Hq, int Hkv,
+                                        int max_blocks, int num_pages, int d, int topk, float sm_scale,
+                                        qsa_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word
  * (QSA_OK if no kernel recorded an error since the last call).  If detail
  * is not NULL it receives a kernel-specific code (0 if none).

@@ -74,3 +74,42 @@ def test_decode_fp8_parity(qsa, name, kw):
     mx, mean = check_out(o.float().cpu().numpy(), ref)
     qerr = np.abs(ref - O_bf16[:, 0]).max()
     print(f"{name}: o max {mx:.2e} mean {mean:.2e}; quantization vs bf16 cache: max {qerr:.2e}")
+
+
+def test_decode_fp8_paged_parity(qsa):
+    """A ragged batch over paged rotated fp8 caches: the pages' rows are
+    quantized like any rows, each sequence is checked against the oracle's
+    fp8 decode on its own logical cache; a page outside the pool is caught
+    on the device."""
+    from tests.test_paged import build_paged
+    lens = [64 * 150 - 5, 64 * 300, 64 * 77 + 31, 1000, 64 * 41 + 1]
+    Hq, Hkv, d, topk = 16, 2, 128, 16
+    p = build_paged(lens, Hq, Hkv, d, seed=171)
+    B, max_blocks = p["B"], p["max_blocks"]
+    sm = d ** -0.5
+    table = torch.from_numpy(p["table"]).to(DEV)
+    seq_lens = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    q = p["q"].to(DEV)
+    kc, ks = qsa.quantize_kv_fp8(p["K_pages"].to(DEV))
+    vc, vs = qsa.quantize_kv_fp8(p["V_pages"].to(DEV))
+    # selection on the unrotated keys' summaries, as the cache write path keeps them
+    Kc = torch.zeros((B, Hkv, max_blocks, d), dtype=torch.float32, device=DEV)
+    qsa.compress_keys_paged(p["K_pages"].to(DEV), table, seq_lens, Kc)
+    idx = torch.full((B, Hkv, 1, topk), -7, dtype=torch.int32, device=DEV)
+    qsa.score_select_ragged(q.view(B, 1, Hq, d), Kc, seq_lens, idx, topk, max(lens), sm)
+    o = torch.full_like(q, float("nan"))
+    qsa.decode_fp8_paged(q, kc, ks, vc, vs, table, seq_lens, idx, o, sm)
+    st = qsa.device_status()
+    assert st[0] == "QSA_OK", st
+    idx_h, o_h = idx.cpu().numpy(), o.float().cpu().numpy()
+    for b, (x, L) in enumerate(zip(p["seqs"], lens)):
+        ck, sk = oracle.quantize_kv_fp8(x["K"])
+        cv, sv = oracle.quantize_kv_fp8(x["V"])
+        ref = oracle.decode_fp8(x["Q"].view(1, Hq, d), ck, sk, cv, sv, idx_h[b:b + 1], L, sm)
+        mx, mean = check_out(o_h[b], ref[0])
+        print(f"paged fp8 seq {b} (L={L}): o max {mx:.2e} mean {mean:.2e}")
+    bad = table.clone()
+    bad[0, int(idx_h[0, 0, 0, 1])] = p["num_pages"] + 3      # a selected block's page is outside the pool
+    qsa.decode_fp8_paged(q, kc, ks, vc, vs, bad, seq_lens, idx, o, sm)
+    assert qsa.device_status()[0] == "QSA_ERR_BOUNDS"
+    assert qsa.device_status()[0] == "QSA_OK"
