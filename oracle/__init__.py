@@ -54,6 +54,10 @@ def _load():
         lib.qsa_oracle_attend.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, I,
                                           Dd, P, I, P, P]
         lib.qsa_oracle_attend.restype = I
+        lib.qsa_oracle_block_scores.argtypes = [P, P, I, I, I, I, I, I, I, I, I, Dd, I, P, I, P]
+        lib.qsa_oracle_block_scores.restype = I
+        lib.qsa_oracle_select_scores.argtypes = [P, I, I, I, I, I, I, I, I, I, P, I, P, P, P]
+        lib.qsa_oracle_select_scores.restype = I
         _lib = lib
     return _lib
 
@@ -150,6 +154,50 @@ def select(Qbar, Kc, Tq, q_pos0, qblk, topk, sm_scale, rows=None, blk=BLOCK,
     if want_scores:
         out["scores"] = scores
     return out
+
+
+AGGREGATORS = {"mean": 0, "max": 1, "softmax_sum": 2}
+
+
+def block_scores(Q, Kc, Tq, q_pos0, qblk, sm_scale, aggregator, rows=None, blk=BLOCK):
+    """Per-row block scores under an aggregator of the per-(head, token)
+    logits ("mean", "max" over tokens of the head mean, or "softmax_sum" of
+    each (head, token)'s softmax over the blocks before the diagonal).
+    Q: bf16 [B, Tq, Hq, d]; Kc: [B, Hkv, NB, d].  Returns [nrows, NB] fp64
+    (or [B, Hkv, NR, NB] when rows is None), s_j for j < D and NaN elsewhere."""
+    Q = _bits(Q)
+    Kc = np.ascontiguousarray(Kc, dtype=np.float64)
+    B, Tq_, Hq, d = Q.shape
+    assert Tq_ == Tq
+    _, Hkv, NB, _ = Kc.shape
+    NR = -(-Tq // qblk)
+    rows_arr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    nrows = B * Hkv * NR if rows is None else len(rows_arr)
+    out = np.empty((nrows, NB), dtype=np.float64)
+    rc = _load().qsa_oracle_block_scores(_ptr(Q), _ptr(Kc), B, Tq, Hq, Hkv, NB, d, q_pos0, qblk, blk,
+                                         float(sm_scale), AGGREGATORS[aggregator], _ptr(rows_arr), nrows,
+                                         _ptr(out))
+    assert rc == 0
+    return out.reshape(B, Hkv, NR, NB) if rows is None else out
+
+
+def select_scores(scores, B, Hkv, Tq, q_pos0, qblk, topk, rows=None, blk=BLOCK):
+    """The selection rule on a score table ([nrows, NB], candidates j in
+    1..D-1 of each row).  Returns a dict like select()."""
+    NR = -(-Tq // qblk)
+    scores = np.ascontiguousarray(scores, dtype=np.float64)
+    NB = scores.shape[-1]
+    scores = scores.reshape(-1, NB)
+    rows_arr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    nrows = scores.shape[0]
+    idx = np.empty((nrows, topk), dtype=np.int32)
+    gap = np.empty(nrows, dtype=np.float64)
+    m = np.empty(nrows, dtype=np.int32)
+    rc = _load().qsa_oracle_select_scores(_ptr(scores), B, Hkv, NR, NB, Tq, q_pos0, qblk, blk, topk,
+                                          _ptr(rows_arr), nrows, _ptr(idx), _ptr(gap), _ptr(m))
+    if rc != 0:
+        raise ValueError("oracle select: topk must be >= 2")
+    return {"idx": idx, "gap": gap, "m": m}
 
 
 def attend(Q, K, V, idx, q_pos0, qblk, sm_scale, tokens=None, blk=BLOCK, want_lse=False):

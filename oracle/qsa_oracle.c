@@ -22,7 +22,10 @@
  * mean-pooled keys per block, scores = <mean pooled query, key summary>
  * scaled by sm_scale, selection shared by one query block and all query
  * heads of a KV group, block 0 (sink) and the causal diagonal block always
- * kept, ties broken by the lower block index.
+ * kept, ties broken by the lower block index.  Two further ways of
+ * combining the query block's tokens and the group's heads (max over
+ * tokens; sum of per-(head, token) softmaxes) are scored by
+ * qsa_oracle_block_scores for the selection variants.
  *
  * Every floating-point quantity is fp64.  bf16 inputs are widened exactly.
  * OpenMP only splits independent rows/tokens; no step is reordered.
@@ -271,6 +274,30 @@ static int diagonal_block(int i, int Tq, int q_pos0, int qblk, int blk)
  * Qbar    : [B][Hkv][NR][d]; Kc : [B][Hkv][NB][d]
  * Returns 0, or -1 if topk < 2.
  */
+/* The selection rule of step 4 for one row: cand[0..ncand) are the scored
+ * candidates {1, ..., D-1}; writes the row's indices, gap and m. */
+static void select_row(scored_block *cand, int ncand, int D, int topk, int32_t *out, double *gap,
+                       int32_t *m_out)
+{
+    qsort(cand, (size_t)ncand, sizeof(scored_block), by_score_then_index);
+    const int nforced = D > 0 ? 2 : 1;
+    int m = topk - nforced;
+    if (m > ncand) m = ncand;
+    *gap = (m == 0 || m == ncand) ? INFINITY : cand[m - 1].s - cand[m].s;
+    *m_out = m;
+    /* ascending output: 0, chosen blocks in increasing index, D */
+    int n = 0;
+    out[n++] = 0;
+    for (int j = 1; j < D; j++) {
+        int chosen = 0;
+        for (int c = 0; c < m; c++)
+            if (cand[c].j == j) { chosen = 1; break; }
+        if (chosen) out[n++] = j;
+    }
+    if (D > 0) out[n++] = D;
+    while (n < topk) out[n++] = -1;
+}
+
 int qsa_oracle_select(const double *Qbar, const double *Kc, int B, int Hkv, int NR,
                       int NB, int d, int Tq, int q_pos0, int qblk, int blk, int topk,
                       double sm_scale, const int32_t *rows, int nrows, int32_t *idx,
@@ -300,25 +327,118 @@ int qsa_oracle_select(const double *Qbar, const double *Kc, int B, int Hkv, int 
             for (int j = 0; j < NB; j++) srow[j] = NAN;
             for (int n = 0; n < ncand; n++) srow[cand[n].j] = cand[n].s;
         }
-        qsort(cand, (size_t)ncand, sizeof(scored_block), by_score_then_index);
-        const int nforced = D > 0 ? 2 : 1;
-        int m = topk - nforced;
-        if (m > ncand) m = ncand;
-        gap[r] = (m == 0 || m == ncand) ? INFINITY : cand[m - 1].s - cand[m].s;
-        m_out[r] = m;
+        select_row(cand, ncand, D, topk, idx + (int64_t)r * topk, &gap[r], &m_out[r]);
+        free(cand);
+    }
+    return 0;
+}
 
-        /* ascending output: 0, chosen blocks in increasing index, D */
-        int32_t *out = idx + (int64_t)r * topk;
-        int n = 0;
-        out[n++] = 0;
-        for (int j = 1; j < D; j++) {
-            int chosen = 0;
-            for (int c = 0; c < m; c++)
-                if (cand[c].j == j) { chosen = 1; break; }
-            if (chosen) out[n++] = j;
+/*
+ * Step 3 with the row's tokens and heads combined in other ways than the
+ * pooled query.  The pages have the selector score compressed keys against
+ * the queries (page "Qwen4 in llama.cpp: Dissecting PR #27742", section "QSA
+ * Is an Address-Selection Problem, Not a New Attention Equation") and leave
+ * open how the query block's tokens and the group's heads are combined.
+ * For row (b, g, i) with diagonal block D, tokens t of the row's query
+ * block (the valid ones) and heads h of group g:
+ *   z[h][t][j] = sm_scale * <Q[b][t][h], Kc[b][g][j]>   for j in {0, ..., D-1}
+ *   aggregator 0 (mean):        s_j = mean over (h, t) of z[h][t][j]
+ *   aggregator 1 (max):         s_j = max over t of (mean over h of z[h][t][j])
+ *   aggregator 2 (softmax-sum): s_j = sum over (h, t) of softmax over
+ *                               j' in {0, ..., D-1} of z[h][t][j'], at j
+ * (the normalisation set of the softmax-sum is every complete block before
+ * the diagonal, the sink included).
+ * Q : [B][Tq][Hq][d] bf16 bits; Kc : [B][Hkv][NB][d]
+ * rows : flat row ids ((b*Hkv + g)*NR + i) or NULL for all
+ * scores : [nrows][NB] -- s_j for j < D, NaN elsewhere
+ * Returns 0, or -1 for an unknown aggregator.
+ */
+int qsa_oracle_block_scores(const uint16_t *Q, const double *Kc, int B, int Tq, int Hq, int Hkv, int NB,
+                            int d, int q_pos0, int qblk, int blk, double sm_scale, int aggregator,
+                            const int32_t *rows, int nrows, double *scores)
+{
+    if (aggregator < 0 || aggregator > 2) return -1;
+    const int G = Hq / Hkv;
+    const int NR = (Tq + qblk - 1) / qblk;
+    if (!rows) nrows = B * Hkv * NR;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < nrows; r++) {
+        const int row = rows ? rows[r] : r;
+        const int i = row % NR, bg = row / NR, b = bg / Hkv, g = bg % Hkv;
+        const int D = diagonal_block(i, Tq, q_pos0, qblk, blk);
+        const int t0 = i * qblk, t1 = (t0 + qblk < Tq) ? t0 + qblk : Tq;
+        double *srow = scores + (int64_t)r * NB;
+        for (int j = 0; j < NB; j++) srow[j] = NAN;
+        if (D < 1) continue;
+        /* z[(t - t0) * G + (h - g*G)][j] */
+        const int nq = (t1 - t0) * G;
+        double *z = (double *)malloc(sizeof(double) * (size_t)nq * D);
+        double *qv = (double *)malloc(sizeof(double) * (size_t)d);
+        for (int t = t0; t < t1; t++)
+            for (int hh = 0; hh < G; hh++) {
+                const uint16_t *qrow = Q + (((int64_t)b * Tq + t) * Hq + g * G + hh) * d;
+                for (int c = 0; c < d; c++) qv[c] = bf16_to_f64(qrow[c]);
+                double *zr = z + (int64_t)((t - t0) * G + hh) * D;
+                for (int j = 0; j < D; j++) {
+                    const double *kc = Kc + ((int64_t)bg * NB + j) * d;
+                    double dot = 0.0;
+                    for (int c = 0; c < d; c++) dot += qv[c] * kc[c];
+                    zr[j] = sm_scale * dot;
+                }
+            }
+        for (int j = 0; j < D; j++) {
+            double s = 0.0;
+            if (aggregator == 0) {
+                for (int n = 0; n < nq; n++) s += z[(int64_t)n * D + j];
+                s /= (double)nq;
+            } else if (aggregator == 1) {
+                s = -INFINITY;
+                for (int t = 0; t < t1 - t0; t++) {
+                    double m = 0.0;
+                    for (int hh = 0; hh < G; hh++) m += z[(int64_t)(t * G + hh) * D + j];
+                    m /= (double)G;
+                    if (m > s) s = m;
+                }
+            }
+            srow[j] = s;
         }
-        if (D > 0) out[n++] = D;
-        while (n < topk) out[n++] = -1;
+        if (aggregator == 2) {
+            for (int j = 0; j < D; j++) srow[j] = 0.0;
+            for (int n = 0; n < nq; n++) {
+                const double *zr = z + (int64_t)n * D;
+                double mx = -INFINITY, sum = 0.0;
+                for (int j = 0; j < D; j++) if (zr[j] > mx) mx = zr[j];
+                for (int j = 0; j < D; j++) sum += exp(zr[j] - mx);
+                for (int j = 0; j < D; j++) srow[j] += exp(zr[j] - mx) / sum;
+            }
+        }
+        free(qv);
+        free(z);
+    }
+    return 0;
+}
+
+/*
+ * Step 4 on a given score table: the selection rule of qsa_oracle_select
+ * with s_j = scores[r][j] for the candidates j in {1, ..., D-1}.
+ */
+int qsa_oracle_select_scores(const double *scores, int B, int Hkv, int NR, int NB, int Tq, int q_pos0,
+                             int qblk, int blk, int topk, const int32_t *rows, int nrows, int32_t *idx,
+                             double *gap, int32_t *m_out)
+{
+    if (topk < 2) return -1;
+    if (!rows) nrows = B * Hkv * NR;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < nrows; r++) {
+        const int row = rows ? rows[r] : r;
+        const int D = diagonal_block(row % NR, Tq, q_pos0, qblk, blk);
+        const int ncand = D > 1 ? D - 1 : 0;
+        scored_block *cand = (scored_block *)malloc(sizeof(scored_block) * (ncand > 0 ? ncand : 1));
+        for (int j = 1; j < D; j++) {
+            cand[j - 1].s = scores[(int64_t)r * NB + j];
+            cand[j - 1].j = j;
+        }
+        select_row(cand, ncand, D, topk, idx + (int64_t)r * topk, &gap[r], &m_out[r]);
         free(cand);
     }
     return 0;

@@ -463,3 +463,94 @@ def test_decode_fp8_equals_bf16_attention_on_walsh_rows():
     o = oracle.decode_fp8(q, ck, sk, cv, sv, idx, L, sm)
     ref = oracle.attend(q.view(B, 1, Hq, n), K, V, idx, L - 1, 1, sm).reshape(B, Hq, n)
     assert np.abs(o - ref).max() < 1e-12
+
+
+# ------------------------------------------------------ score aggregators
+def _agg_case(seed, B=1, Tq=130, Hq=8, Hkv=2, d=64, q_pos0=64 * 6, qblk=64, nblk=10):
+    g = torch.Generator().manual_seed(seed)
+    Q = bf16(torch.randn((B, Tq, Hq, d), generator=g))
+    K = bf16(torch.randn((B, Hkv, 64 * (nblk + 3), d), generator=g))
+    Kc = oracle.compress_keys(K, 0, nblk + 2)
+    return Q, K, Kc
+
+
+def test_mean_aggregator_equals_pooled_query_scores():
+    """Averaging the per-(head, token) logits equals scoring the pooled
+    query (linearity); the two are computed independently."""
+    Q, _, Kc = _agg_case(21)
+    sm = 0.125
+    for qblk, q_pos0 in ((64, 64 * 6), (1, 64 * 9 + 17)):
+        Tq = Q.shape[1]
+        s = oracle.block_scores(Q, Kc, Tq, q_pos0, qblk, sm, "mean")
+        Qbar = oracle.pool_queries(Q, 2, qblk)
+        ref = oracle.select(Qbar, Kc, Tq, q_pos0, qblk, 4, sm, want_scores=True)
+        NB = Kc.shape[2]
+        ref_s = ref["scores"].reshape(s.shape[:3] + (NB,))
+        cand = ~np.isnan(ref_s)                          # candidates 1 .. D-1
+        assert np.allclose(s[cand], ref_s[cand], rtol=0, atol=1e-12)
+        # and the selection rule on the table reproduces the pooled selection
+        sel = oracle.select_scores(s, 1, 2, Tq, q_pos0, qblk, 4)
+        assert np.array_equal(sel["idx"].reshape(ref["idx"].shape), ref["idx"])
+
+
+def test_max_aggregator_special_cases():
+    """Max over tokens of the head mean: one token per row -> the mean;
+    identical tokens in a block -> the mean; never below the mean; invariant
+    under reordering the block's tokens and the group's heads."""
+    Q, _, Kc = _agg_case(22)
+    sm = 0.125
+    Tq = Q.shape[1]
+    one = oracle.block_scores(Q, Kc, Tq, 64 * 9, 1, sm, "max")
+    assert np.array_equal(np.isnan(one), np.isnan(oracle.block_scores(Q, Kc, Tq, 64 * 9, 1, sm, "mean")))
+    assert np.allclose(one, oracle.block_scores(Q, Kc, Tq, 64 * 9, 1, sm, "mean"), rtol=0, atol=1e-12,
+                       equal_nan=True)
+    same = Q.clone()
+    same[:, :64] = Q[:, :1]
+    mx = oracle.block_scores(same, Kc, Tq, 64 * 6, 64, sm, "max")[:, :, 0]
+    mn = oracle.block_scores(same, Kc, Tq, 64 * 6, 64, sm, "mean")[:, :, 0]
+    assert np.allclose(mx, mn, rtol=0, atol=1e-12, equal_nan=True)
+    mx = oracle.block_scores(Q, Kc, Tq, 64 * 6, 64, sm, "max")
+    mn = oracle.block_scores(Q, Kc, Tq, 64 * 6, 64, sm, "mean")
+    ok = ~np.isnan(mx)
+    assert np.all(mx[ok] >= mn[ok] - 1e-12) and np.mean(mx[ok] > mn[ok] + 1e-6) > 0.9
+    perm = Q[:, torch.randperm(64, generator=torch.Generator().manual_seed(5))]
+    perm = torch.cat([perm, Q[:, 64:]], 1)
+    heads = torch.cat([Q[:, :, [3, 1, 0, 2]], Q[:, :, [7, 5, 6, 4]]], 2)
+    for X in (perm, heads):
+        assert np.allclose(oracle.block_scores(X, Kc, Tq, 64 * 6, 64, sm, "max")[:, :, 0], mx[:, :, 0],
+                           rtol=0, atol=1e-12, equal_nan=True)
+
+
+def test_softmax_sum_aggregator_pins():
+    """Per-(head, token) softmax over the blocks before the diagonal, summed:
+    the scores of a row add up to (heads x tokens); a vector added to every
+    key leaves them unchanged (each softmax sees one constant shift); at zero
+    temperature every block gets the same share, at a very low one each
+    (head, token) votes for its best block; one head and token is the
+    textbook softmax (scipy)."""
+    import scipy.special
+    Q, _, Kc = _agg_case(23)
+    sm = 0.125
+    Tq = Q.shape[1]
+    s = oracle.block_scores(Q, Kc, Tq, 64 * 6, 64, sm, "softmax_sum")
+    for i, ntok in ((0, 64), (1, 64), (2, 2)):
+        D = (64 * 6 + min((i + 1) * 64, Tq) - 1) // 64
+        row = s[0, 0, i]
+        assert np.all(~np.isnan(row[:D])) and np.all(np.isnan(row[D:]))
+        assert abs(row[:D].sum() - 4 * ntok) < 1e-9
+    # every summary shifted by the same vector (in fp64: a shift of the bf16
+    # keys would round)
+    c = torch.randn(64, generator=torch.Generator().manual_seed(6)).double().numpy() * 3
+    assert np.allclose(oracle.block_scores(Q, Kc + c, Tq, 64 * 6, 64, sm, "softmax_sum"), s, rtol=0,
+                       atol=1e-10, equal_nan=True)
+    flat = oracle.block_scores(Q, Kc, Tq, 64 * 6, 64, 0.0, "softmax_sum")
+    D0 = 6 + 0   # row 0: diagonal block 6, blocks 0..5
+    assert np.allclose(flat[0, 0, 0, :D0], 4 * 64 / D0, rtol=0, atol=1e-12)
+    cold = oracle.block_scores(Q, Kc, Tq, 64 * 6, 64, 1e9, "softmax_sum")[0, 0, 0, :D0]
+    z = np.einsum("thc,jc->thj", Q[0, :64, :4].double().numpy(), Kc[0, 0, :D0])
+    votes = np.bincount(z.reshape(-1, D0).argmax(axis=1), minlength=D0)
+    assert np.allclose(cold, votes, rtol=0, atol=1e-6)
+    one = Q[:, :1, :2]                                           # one token, Hq = Hkv = 2 (G = 1)
+    s1 = oracle.block_scores(one, Kc, 1, 64 * 7 + 3, 1, sm, "softmax_sum")[0, 1, 0, :7]
+    zz = sm * (Kc[0, 1, :7] @ one[0, 0, 1].double().numpy())
+    assert np.allclose(s1, scipy.special.softmax(zz), rtol=0, atol=1e-14)
