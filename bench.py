@@ -308,6 +308,10 @@ def run_qsa(args, ws, rank, local):
             torch.cuda.empty_cache()
             result["decode"]["fp8_kv"] = bench_decode(args, qsa, dev, peaks, ws, rank, flush,
                                                       summary="bf16", kv="fp8")
+        if args.softmax_sum:
+            torch.cuda.empty_cache()
+            result["decode"]["softmax_sum_selection"] = bench_decode(args, qsa, dev, peaks, ws, rank, flush,
+                                                                     agg="softmax_sum")
         if args.paged:
             torch.cuda.empty_cache()
             result["decode"]["ragged_paged"] = bench_decode_paged(args, qsa, dev, peaks, ws, rank, flush)
@@ -430,7 +434,7 @@ def decode_result(wname, B, context, topk, t, d, launches, by, sel_bytes, peaks,
     return r
 
 
-def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary="fp32", kv="bf16"):
+def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary="fp32", kv="bf16", agg="mean"):
     wd = synthetic.CONFIGS[workload or args.decode_workload]
     if args.decode_batch:
         wd = synthetic.Workload(**{**wd.__dict__, "B": args.decode_batch})
@@ -461,9 +465,15 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary=
         by = by // (2 * wd.d) * (wd.d + 4)      # per selected key and head: d code bytes + a 4-byte scale
         extra["kv_cache"] = "fp8 e4m3, Walsh-Hadamard rotated, per-row fp32 scale"
 
+    if agg != "mean":
+        extra["aggregator"] = agg
+
     def run_parts(parts, s):
         if "select" in parts:
-            qsa.score_select(q4, dec.Kc, dec.idx, wd.topk, L - 1, 1, dec.sm_scale, sel_ws, s)
+            if agg == "mean":
+                qsa.score_select(q4, dec.Kc, dec.idx, wd.topk, L - 1, 1, dec.sm_scale, sel_ws, s)
+            else:
+                qsa.score_select_token_agg(q4, dec.Kc, dec.idx, wd.topk, L - 1, agg, dec.sm_scale, stream=s)
         if "attention" in parts:
             if kv == "fp8":
                 qsa.decode_fp8(q, Kq, Ks, Vq, Vs, dec.idx, dec.o, L, dec.sm_scale, s)
@@ -704,7 +714,9 @@ def main():
                     help="skip the decode run over the rotated fp8 cache (reported beside the bf16 one)")
     ap.add_argument("--only-decode", action="store_true",
                     help="skip the prefill measurement (profiling the decode kernels)")
-    ap.add_argument("--decode-variants", default="fp32,bf16,fp8,paged",
+    ap.add_argument("--no-softmax-sum", dest="softmax_sum", action="store_false",
+                    help="skip the decode run with the softmax-sum selection aggregator")
+    ap.add_argument("--decode-variants", default="fp32,bf16,fp8,paged,softmax_sum",
                     help="with --only-decode: which decode runs (fp32 / bf16 summaries, fp8 cache, paged)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="override the decode batch (smaller profiling captures)")
@@ -742,6 +754,10 @@ def main():
         if args.fp8_kv and "fp8" in variants:
             torch.cuda.empty_cache()
             res["fp8_kv"] = bench_decode(args, qsa, dev, load_peaks(), ws, rank, flush, summary="bf16", kv="fp8")
+        if args.softmax_sum and "softmax_sum" in variants:
+            torch.cuda.empty_cache()
+            res["softmax_sum_selection"] = bench_decode(args, qsa, dev, load_peaks(), ws, rank, flush,
+                                                        agg="softmax_sum")
         if args.paged and "paged" in variants:
             torch.cuda.empty_cache()
             res["ragged_paged"] = bench_decode_paged(args, qsa, dev, load_peaks(), ws, rank, flush)

@@ -57,6 +57,7 @@ def _load():
         "qsa_score_select_ragged": (I, [P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "qsa_decode_paged": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "qsa_score_select_ragged_prefill": (I, [P, P, P, P, I, I, I, I, I, I, I, I, F, P, S, P]),
+        "qsa_score_select_token_agg": (I, [P, P, P, P, I, I, I, I, I, I, I, I, F, I, P]),
         "qsa_quantize_kv_fp8": (I, [P, P, P, ctypes.c_int64, I, P]),
         "qsa_decode_fp8": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "qsa_decode_fp8_paged": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
@@ -257,6 +258,28 @@ def decode_paged(q, K_pages, V_pages, block_table, seq_lens, idx, o, sm_scale=No
                                  topk, float(sm_scale), _stream(stream)),
            "qsa_decode_paged")
     return o
+
+
+AGGREGATORS = {"mean": 0, "max": 1, "softmax_sum": 2}
+
+
+def score_select_token_agg(q, Kc, idx, topk, q_pos0, aggregator="mean", sm_scale=None, seq_lens=None,
+                           stream=None):
+    """Per-token selection with an aggregator of the group's per-head scores
+    ("mean", "max" -- the same for one token --, or "softmax_sum").
+    q: bf16 [B, Tq, Hq, d] at positions q_pos0 .. q_pos0 + Tq - 1, or with
+    seq_lens (int32 [B], Tq = 1) at seq_lens[b] - 1 (q_pos0 = the largest);
+    Kc fp32 [B, Hkv, max_blocks, d]; idx int32 [B, Hkv, Tq, topk] (written)."""
+    B, Tq, Hq, d = q.shape
+    _, Hkv, max_blocks, _ = Kc.shape
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    sl = None if seq_lens is None else _ptr(seq_lens, torch.int32, "seq_lens")
+    _check(_lib.qsa_score_select_token_agg(_ptr(q, torch.bfloat16, "q"), _ptr(Kc, torch.float32, "Kc"), sl,
+                                           _ptr(idx, torch.int32, "idx"), B, Hq, Hkv, Tq, q_pos0, max_blocks, d,
+                                           topk, float(sm_scale), AGGREGATORS[aggregator], _stream(stream)),
+           "qsa_score_select_token_agg")
+    return idx
 
 
 def score_select_ragged_prefill(Q, Kc, q_pos, idx, topk, max_pos, sm_scale=None, workspace=None,

@@ -301,13 +301,17 @@ qsa_status launch_decode(const void *q, const void *K, const void *V, const int3
     return launched("decode_kernel");
 }
 
-template <int D, typename KcT>
+template <int D, typename KcT, bool SOFTMAX = false>
 qsa_status launch_select_token_d(const void *Q, const KcT *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
                                  int q_pos0, int nblk_max, int topk, float sm_scale, const TokenPlan &tp,
                                  cudaStream_t s, const int32_t *seq_lens)
 {
-    auto kern = qsa::select_token_kernel<D, KcT>;
-    const int smem = tp.CH * 8;
+    auto kern = [] {
+        if constexpr (SOFTMAX) return qsa::select_token_softmax_kernel<D, KcT>;
+        else return qsa::select_token_kernel<D, KcT>;
+    }();
+    // keys; the softmax-sum path also keeps its chunk's logits (8 x (CH + 1) floats) when CH is short enough
+    const int smem = tp.CH * 8 + (SOFTMAX && tp.CH <= qsa::kSoftmaxZCap ? 8 * (tp.CH + 1) * 4 : 0);
     qsa_status st;
     if ((st = set_smem(kern, smem)) != QSA_OK) return st;
     cudaLaunchConfig_t cfg = {};
@@ -327,19 +331,19 @@ qsa_status launch_select_token_d(const void *Q, const KcT *Kc, int32_t *idx, int
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, (const __nv_bfloat16 *)Q, Kc, idx, nblk_max, Tq, Hq, Hkv,
                                        q_pos0, topk, sm_scale, tp.CH, seq_lens);
     if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "select_token_kernel launch: %s", cudaGetErrorString(e));
-    return launched("select_token_kernel");
+    return launched(SOFTMAX ? "select_token_softmax_kernel" : "select_token_kernel");
 }
 
-template <typename KcT>
+template <typename KcT, bool SOFTMAX = false>
 qsa_status launch_select_token(const void *Q, const KcT *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
                                int q_pos0, int nblk_max, int d, int topk, float sm_scale, const TokenPlan &tp,
                                cudaStream_t s, const int32_t *seq_lens = nullptr)
 {
     if (d == 128)
-        return launch_select_token_d<128, KcT>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, nblk_max, topk, sm_scale, tp, s,
-                                               seq_lens);
-    return launch_select_token_d<64, KcT>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, nblk_max, topk, sm_scale, tp, s,
-                                          seq_lens);
+        return launch_select_token_d<128, KcT, SOFTMAX>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, nblk_max, topk, sm_scale,
+                                                        tp, s, seq_lens);
+    return launch_select_token_d<64, KcT, SOFTMAX>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, nblk_max, topk, sm_scale, tp,
+                                                   s, seq_lens);
 }
 
 __global__ void selftest_exp2_kernel(const float *__restrict__ x, float *__restrict__ y, int n)
@@ -581,6 +585,33 @@ qsa_status qsa_score_select_ragged(const void *Q, const float *Kc, const int32_t
     if (!tp.use) return fail(QSA_ERR_UNSUPPORTED, "%s: more candidates than one cluster of chunks holds", name);
     return launch_select_token(Q, Kc, idx, B, Hq, Hkv, 1, max_len - 1, max_blocks, d, topk, sm_scale, tp,
                                reinterpret_cast<cudaStream_t>(stream), seq_lens);
+}
+
+qsa_status qsa_score_select_token_agg(const void *Q, const float *Kc, const int32_t *seq_lens, int32_t *idx, int B,
+                                      int Hq, int Hkv, int Tq, int q_pos0, int max_blocks, int d, int topk,
+                                      float sm_scale, int aggregator, qsa_stream_t stream)
+{
+    const char *name = "qsa_score_select_token_agg";
+    if (!Q || !Kc || !idx) return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (aggregator != QSA_AGG_MEAN && aggregator != QSA_AGG_MAX && aggregator != QSA_AGG_SOFTMAX_SUM)
+        return fail(QSA_ERR_INVALID_ARG, "%s: aggregator=%d", name, aggregator);
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Tq <= 0 || q_pos0 < 0 || max_blocks <= 0 ||
+        (long)q_pos0 + Tq > 64L * max_blocks || (seq_lens && Tq != 1))
+        return fail(QSA_ERR_INVALID_ARG, "%s: bad shape", name);
+    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "%s: d=%d", name, d);
+    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "%s: topk=%d", name, topk);
+    if ((long)Hq * d / 8 > 1024 || Hq / Hkv > 8) return fail(QSA_ERR_UNSUPPORTED, "%s: group too large", name);
+    if (!aligned16(Q) || !aligned16(Kc) || !aligned16(idx) || (reinterpret_cast<uintptr_t>(seq_lens) & 3))
+        return fail(QSA_ERR_INVALID_ARG, "%s: misaligned pointer", name);
+    const TokenPlan tp = plan_token(B, Hkv, Tq, q_pos0, 1);
+    if (!tp.use) return fail(QSA_ERR_UNSUPPORTED, "%s: more candidates than one cluster of chunks holds", name);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // one token per row: its maximum over tokens is its mean
+    if (aggregator == QSA_AGG_SOFTMAX_SUM)
+        return launch_select_token<float, true>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, max_blocks, d, topk, sm_scale, tp,
+                                                s, seq_lens);
+    return launch_select_token<float>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, max_blocks, d, topk, sm_scale, tp, s,
+                                      seq_lens);
 }
 
 qsa_status qsa_score_select_ragged_prefill(const void *Q, const float *Kc, const int32_t *q_pos, int32_t *idx,

@@ -307,6 +307,37 @@ __device__ __forceinline__ void load_summary(const __nv_bfloat16 *p, float (&k)[
     }
 }
 
+// Sums over the warp of 8 per-lane partials s[0..8) at once: a transposing
+// butterfly that leaves the total of partial (lane >> 2) in the lanes with
+// (lane & 3) == 0 (returned there).
+__device__ __forceinline__ float reduce8(float (&s)[8])
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int c = 0; c < 4; c++) {
+        const bool up = lane & 16;
+        const float send = up ? s[c] : s[c + 4];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+        s[c] = (up ? s[c + 4] : s[c]) + recv;
+    }
+#pragma unroll
+    for (int c = 0; c < 2; c++) {
+        const bool up = lane & 8;
+        const float send = up ? s[c] : s[c + 2];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
+        s[c] = (up ? s[c + 2] : s[c]) + recv;
+    }
+    {
+        const bool up = lane & 4;
+        const float send = up ? s[0] : s[1];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
+        s[0] = (up ? s[1] : s[0]) + recv;
+    }
+    s[0] += __shfl_xor_sync(0xffffffffu, s[0], 2);
+    s[0] += __shfl_xor_sync(0xffffffffu, s[0], 1);
+    return s[0];
+}
+
 // fp32 scores of n candidates (block summaries kc[0..n) of d = D fp32 or
 // bf16 components, block ids j0..j0+n-1) against the pooled query qb, as
 // 64-bit keys.  Each warp takes 8 candidates at a time; lane owns columns
@@ -334,31 +365,66 @@ __device__ __forceinline__ void score_chunk(const float *qb, const KcT *__restri
                 else s[c] = q[0] * k[0] + q[1] * k[1];
             }
         }
-#pragma unroll
-        for (int c = 0; c < 4; c++) {
-            const bool up = lane & 16;
-            const float send = up ? s[c] : s[c + 4];
-            const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-            s[c] = (up ? s[c + 4] : s[c]) + recv;
-        }
-#pragma unroll
-        for (int c = 0; c < 2; c++) {
-            const bool up = lane & 8;
-            const float send = up ? s[c] : s[c + 2];
-            const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
-            s[c] = (up ? s[c + 2] : s[c]) + recv;
-        }
-        {
-            const bool up = lane & 4;
-            const float send = up ? s[0] : s[1];
-            const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
-            s[0] = (up ? s[1] : s[0]) + recv;
-        }
-        s[0] += __shfl_xor_sync(0xffffffffu, s[0], 2);
-        s[0] += __shfl_xor_sync(0xffffffffu, s[0], 1);
+        const float dot = reduce8(s);
         const int e = base + (lane >> 2);
-        if ((lane & 3) == 0 && e < n) keys[e] = make_key(s[0] * sm_scale, j0 + e);
+        if ((lane & 3) == 0 && e < n) keys[e] = make_key(dot * sm_scale, j0 + e);
     }
+}
+
+// Per-head logits of n blocks (summaries kc[0..n)) for the G <= 8 heads of
+// a group (queries qh[h][0..D), fp32): for every block e, f(e, z) receives
+// z[h] = scale * <qh[h], kc[e]> for h < G, in the lane that holds them
+// ((lane & 3) == 0).  Each warp takes 8 blocks at a time and loads each
+// summary once for all heads.
+template <int D, typename KcT, typename F>
+__device__ __forceinline__ void head_logits(const float (*qh)[D], int G, const KcT *__restrict__ kc, int n,
+                                            float scale, F &&f)
+{
+    constexpr int V = D / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const KcT *kc_base = kc + lane * V;
+    for (int base = warp * 8; base < n; base += 8 * (kSelThreads / 32)) {
+        float k[8][V];
+#pragma unroll
+        for (int c = 0; c < 8; c++) {
+            if (base + c < n) {
+                load_summary<V>(kc_base + (long)(base + c) * D, k[c]);
+            } else {
+#pragma unroll
+                for (int v = 0; v < V; v++) k[c][v] = 0.f;
+            }
+        }
+        float z[8];
+#pragma unroll
+        for (int h = 0; h < 8; h++) {
+            z[h] = 0.f;
+            if (h < G) {
+                float s[8];
+#pragma unroll
+                for (int c = 0; c < 8; c++) {
+                    s[c] = 0.f;
+#pragma unroll
+                    for (int v = 0; v < V; v++) s[c] += qh[h][lane * V + v] * k[c][v];
+                }
+                z[h] = reduce8(s) * scale;
+            }
+        }
+        const int e = base + (lane >> 2);
+        if ((lane & 3) == 0 && e < n) f(e, z);
+    }
+}
+
+// Longest chunk whose softmax-sum logits (8 heads) stay in shared memory.
+constexpr int kSoftmaxZCap = 1024;
+
+// Running (max, sum of 2^(z - max)) pairs, merged; an empty pair is
+// (-inf, 0).
+__device__ __forceinline__ void lse2_merge(float &m, float &s, float m2, float s2)
+{
+    const float mn = fmaxf(m, m2);
+    if (mn == -INFINITY) return;   // both empty
+    s = s * fast_exp2(m - mn) + s2 * fast_exp2(m2 - mn);
+    m = mn;
 }
 
 // --------------------------------------------------------- score+select
@@ -429,8 +495,8 @@ __global__ void __launch_bounds__(kSelThreads) merge_select_kernel(
 // Tq = 1), sequence b's token sits at position seq_lens[b] - 1 (checked
 // against the summaries' capacity; an invalid length reports
 // QSA_ERR_BOUNDS and the row keeps block 0 only).
-template <int D, typename KcT>
-__global__ void __launch_bounds__(kSelThreads) select_token_kernel(
+template <int D, typename KcT, bool SOFTMAX>
+__device__ __forceinline__ void select_token_body(
     const __nv_bfloat16 *__restrict__ Q, const KcT *__restrict__ Kc, int32_t *__restrict__ idx,
     int nblk_max, int Tq, int Hq, int Hkv, int q_pos0, int topk, float sm_scale, int CH,
     const int32_t *__restrict__ seq_lens)
@@ -459,8 +525,8 @@ __global__ void __launch_bounds__(kSelThreads) select_token_kernel(
     }
     const RowGeom g = row_geom(i, Tq, qp, 1, topk, CH);
 
-    // pooled query: mean of the token's query over the group's heads
-    {
+    if constexpr (!SOFTMAX) {
+        // pooled query: mean of the token's query over the group's heads
         const __nv_bfloat16 *qt = Q + (((long)b * Tq + i) * Hq + (long)grp * G) * D;
         const float inv = 1.0f / (float)G;
         for (int c = tid; c < D; c += kSelThreads) {
@@ -468,11 +534,121 @@ __global__ void __launch_bounds__(kSelThreads) select_token_kernel(
             for (int h = 0; h < G; h++) s += __bfloat162float(qt[(long)h * D + c]);
             qbar[c] = s * inv;
         }
+        __syncthreads();
     }
-    __syncthreads();
     const int j0 = 1 + chunk * CH;
     const int n = max(0, min(CH, g.ncand - chunk * CH));
-    score_chunk<D, KcT>(qbar, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
+    if constexpr (SOFTMAX) {
+        // Softmax-sum aggregator: s_j = sum over the group's heads h of
+        // softmax over the blocks {0, ..., D-1} of z_h = sm_scale <q_h, Kc_j>,
+        // at j.  Pass 1: each CTA's (max, sum) per head over its blocks
+        // (chunk 0 also takes block 0, which is in the normalisation set but
+        // not a candidate), merged across the cluster through distributed
+        // shared memory; pass 2: the candidates' scores from the merged
+        // statistics (the summaries are read again, mostly from L2).  Base-2
+        // logits: the softmax is the same.
+        __shared__ float qh[8][D];
+        __shared__ float wst[kSelThreads / 32][8][2];
+        __shared__ float cst[8][2];
+        __shared__ float gst[8][2];
+        const __nv_bfloat16 *qt = Q + (((long)b * Tq + i) * Hq + (long)grp * G) * D;
+        for (int e = tid; e < G * D; e += kSelThreads) qh[e / D][e % D] = __bfloat162float(qt[e]);
+        __syncthreads();
+        const float scale = sm_scale * 1.4426950408889634f;
+        if (g.ncand > 0) {
+            const int js = chunk == 0 ? 0 : j0;
+            const int ns = n + (j0 - js);
+            const int lane = tid & 31, warp = tid >> 5;
+            // logits kept in shared memory after the keys when the chunk is
+            // short enough (kSoftmaxZCap), else recomputed in pass 2
+            const bool zsm = CH <= kSoftmaxZCap;
+            float *zb = reinterpret_cast<float *>(keys + CH);   // [8][CH + 1]
+            const int zs = CH + 1;
+            if (zsm) {
+                head_logits<D, KcT>(qh, G, Kc + ((long)bg * nblk_max + js) * D, ns, scale,
+                                    [&](int e, const float(&z)[8]) {
+#pragma unroll
+                                        for (int h = 0; h < 8; h++)
+                                            if (h < G) zb[h * zs + e] = z[h];
+                                    });
+                __syncthreads();
+                if (warp < G) {   // warp h: head h's (max, sum) over this CTA's blocks
+                    const float *zr = zb + warp * zs;
+                    float m = -INFINITY;
+                    for (int e = lane; e < ns; e += 32) m = fmaxf(m, zr[e]);
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+                    float sum = 0.f;
+                    if (m != -INFINITY)
+                        for (int e = lane; e < ns; e += 32) sum += fast_exp2(zr[e] - m);
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+                    if (lane == 0) cst[warp][0] = m, cst[warp][1] = sum;
+                }
+            } else {
+                float mr[8], sr[8];
+#pragma unroll
+                for (int h = 0; h < 8; h++) mr[h] = -INFINITY, sr[h] = 0.f;
+                head_logits<D, KcT>(qh, G, Kc + ((long)bg * nblk_max + js) * D, ns, scale,
+                                    [&](int, const float(&z)[8]) {
+#pragma unroll
+                                        for (int h = 0; h < 8; h++)
+                                            if (h < G) lse2_merge(mr[h], sr[h], z[h], 1.f);
+                                    });
+#pragma unroll
+                for (int h = 0; h < 8; h++) {
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float m2 = __shfl_xor_sync(0xffffffffu, mr[h], off);
+                        const float s2 = __shfl_xor_sync(0xffffffffu, sr[h], off);
+                        lse2_merge(mr[h], sr[h], m2, s2);
+                    }
+                    if (lane == 0) wst[warp][h][0] = mr[h], wst[warp][h][1] = sr[h];
+                }
+                __syncthreads();
+                if (tid < G) {
+                    float m = -INFINITY, sm = 0.f;
+                    for (int w = 0; w < kSelThreads / 32; w++) lse2_merge(m, sm, wst[w][tid][0], wst[w][tid][1]);
+                    cst[tid][0] = m, cst[tid][1] = sm;
+                }
+            }
+            if (g.nchunks > 1) {
+                cluster.sync();   // every CTA's statistics are in place
+                if (tid < G) {
+                    float m = -INFINITY, sm = 0.f;
+                    for (int c = 0; c < NCH; c++) {
+                        const float *r = &cluster.map_shared_rank(&cst[0][0], c)[2 * tid];
+                        lse2_merge(m, sm, r[0], r[1]);
+                    }
+                    gst[tid][0] = m, gst[tid][1] = 1.f / sm;
+                }
+            } else {
+                __syncthreads();
+                if (tid < G) gst[tid][0] = cst[tid][0], gst[tid][1] = 1.f / cst[tid][1];
+            }
+            __syncthreads();
+            if (zsm) {
+                for (int e = tid; e < n; e += kSelThreads) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int h = 0; h < 8; h++)
+                        if (h < G) acc += fast_exp2(zb[h * zs + e + (j0 - js)] - gst[h][0]) * gst[h][1];
+                    keys[e] = make_key(acc, j0 + e);
+                }
+            } else {
+                head_logits<D, KcT>(qh, G, Kc + ((long)bg * nblk_max + j0) * D, n, scale,
+                                    [&](int e, const float(&z)[8]) {
+                                        float acc = 0.f;
+#pragma unroll
+                                        for (int h = 0; h < 8; h++)
+                                            if (h < G) acc += fast_exp2(z[h] - gst[h][0]) * gst[h][1];
+                                        keys[e] = make_key(acc, j0 + e);
+                                    });
+            }
+        }
+    } else {
+        score_chunk<D, KcT>(qbar, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
+    }
     __syncthreads();
     const int need = min(g.m, n);
     if (g.nchunks == 1) {
@@ -486,6 +662,26 @@ __global__ void __launch_bounds__(kSelThreads) select_token_kernel(
     for (int e = need + tid; e < kMaxChosen; e += kSelThreads) dst[e] = 0;
     cluster.sync();   // every list is in the leader
     if (chunk == 0) select_and_emit(lists, NCH * kMaxChosen, g.m, sh, idx + row * topk, g.D, topk, nullptr);
+}
+
+template <int D, typename KcT>
+__global__ void __launch_bounds__(kSelThreads) select_token_kernel(
+    const __nv_bfloat16 *__restrict__ Q, const KcT *__restrict__ Kc, int32_t *__restrict__ idx,
+    int nblk_max, int Tq, int Hq, int Hkv, int q_pos0, int topk, float sm_scale, int CH,
+    const int32_t *__restrict__ seq_lens)
+{
+    select_token_body<D, KcT, false>(Q, Kc, idx, nblk_max, Tq, Hq, Hkv, q_pos0, topk, sm_scale, CH, seq_lens);
+}
+
+// The softmax-sum aggregator's per-token selection: at most 64 registers,
+// so that 4 CTAs share an SM and a decode batch's clusters run in one wave.
+template <int D, typename KcT>
+__global__ void __launch_bounds__(kSelThreads, 4) select_token_softmax_kernel(
+    const __nv_bfloat16 *__restrict__ Q, const KcT *__restrict__ Kc, int32_t *__restrict__ idx,
+    int nblk_max, int Tq, int Hq, int Hkv, int q_pos0, int topk, float sm_scale, int CH,
+    const int32_t *__restrict__ seq_lens)
+{
+    select_token_body<D, KcT, true>(Q, Kc, idx, nblk_max, Tq, Hq, Hkv, q_pos0, topk, sm_scale, CH, seq_lens);
 }
 
 }  // namespace qsa

@@ -254,6 +254,38 @@ QSA_API qsa_status qsa_decode_paged(const void *q, const void *K_pages, const vo
                                     qsa_stream_t stream);
 
 /*
+ * Per-token selection (decode rows: one query token per row) with another
+ * way of combining the group's heads than the pooled query.  The pages have
+ * the selector score compressed keys against the queries (page "Qwen4 in
+ * llama.cpp: Dissecting PR #27742", section "QSA Is an Address-Selection
+ * Problem, Not a New Attention Equation") and leave the combination open.
+ * With z_h(j) = sm_scale * <q_h, Kc_j> for the group's heads h and the
+ * complete blocks j < D before the token's diagonal block D:
+ *   QSA_AGG_MEAN         s_j = mean over h of z_h(j) (= qsa_score_select)
+ *   QSA_AGG_MAX          s_j = max over the row's tokens of the head mean;
+ *                        with one token per row it equals QSA_AGG_MEAN
+ *   QSA_AGG_SOFTMAX_SUM  s_j = sum over h of exp(z_h(j)) / sum over j' < D
+ *                        of exp(z_h(j')) (block 0 is in the normalisation,
+ *                        not among the candidates)
+ * then the usual rule: block 0 and D forced, the top (topk - forced) of the
+ * candidates 1 .. D-1 by (s descending, index ascending), ascending, -1
+ * padded.  Q bf16 [B][Tq][Hq][d] at positions q_pos0 .. q_pos0 + Tq - 1, or
+ * with seq_lens (int32 [B], Tq = 1) at seq_lens[b] - 1 with q_pos0 the
+ * largest of them (planning); Kc fp32 [B][Hkv][max_blocks][d]; idx int32
+ * [B][Hkv][Tq][topk].  Errors: null pointer, bad shape, unknown aggregator
+ * or misaligned pointer -> QSA_ERR_INVALID_ARG; d not 64/128, Hq/Hkv > 8,
+ * topk outside 2..64 or a row longer than one cluster of chunks holds ->
+ * QSA_ERR_UNSUPPORTED; an invalid seq_lens entry -> QSA_ERR_BOUNDS on the
+ * device.  Prefill rows (64-token query blocks) with the max or softmax-sum
+ * aggregators are not provided.
+ */
+enum { QSA_AGG_MEAN = 0, QSA_AGG_MAX = 1, QSA_AGG_SOFTMAX_SUM = 2 };
+QSA_API qsa_status qsa_score_select_token_agg(const void *Q, const float *Kc, const int32_t *seq_lens,
+                                              int32_t *idx, int B, int Hq, int Hkv, int Tq, int q_pos0,
+                                              int max_blocks, int d, int topk, float sm_scale, int aggregator,
+                                              qsa_stream_t stream);
+
+/*
  * Quantized-KV option for decode (page "Qwen4 in llama.cpp: Dissecting PR
  * #27742", section "Quantized KV Exposed a Backend Storage Invariant"): the
  * cache holds K and V in a Walsh-Hadamard-rotated basis as fp8 e4m3 codes

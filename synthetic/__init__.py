@@ -42,7 +42,7 @@ class Workload:
     q_pos0: int
     qblk: int
     seed: int
-    plant: str = "none"          # "none" | "qhat" | "partner"
+    plant: str = "none"          # "none" | "qhat" | "partner" | "token"
     plant_frac: float = 0.0
     plant_scale: float = 1.0
     description: str = ""
@@ -180,6 +180,24 @@ def generate(w: Workload, device="cpu"):
                     adds_k.append((b, g, j, w.plant_scale * u))
                     adds_q.append((b, g, i, w.plant_scale * u))
                     planted.append((b, g, j, i))
+
+    elif w.plant == "token":
+        # Per-token rows (decode): a fraction of the complete key blocks
+        # before the first token's diagonal (sink excluded) per group get a
+        # unit direction u added to all 64 keys; u is also added to the
+        # group's heads of every query token.
+        assert w.qblk == 1
+        last_cand = w.q_pos0 // BLOCK - 1
+        n_plant = int(w.plant_frac * max(last_cand, 0))
+        for b in range(w.B):
+            for g in range(w.Hkv):
+                js = (torch.randperm(last_cand, generator=pgen)[:n_plant] + 1).tolist() if n_plant else []
+                for j in js:
+                    u = _unit(pgen, w.d)
+                    adds_k.append((b, g, j, w.plant_scale * u))
+                    for i in range(w.n_rows):
+                        adds_q.append((b, g, i, w.plant_scale * u))
+                    planted.append((b, g, j, -1))
 
     for (b, g, i, vec) in adds_q:
         t0, t1 = i * w.qblk, min((i + 1) * w.qblk, w.Tq)

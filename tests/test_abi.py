@@ -96,6 +96,14 @@ def test_argument_checks_return_before_launch():
     assert d8(topk=65) == 2
     assert d8(ks=odd) == 1
     assert d8(ks=None) == 1
+    # per-token selection with an aggregator: unknown aggregator, ragged with
+    # several tokens, a group of more than 8 heads
+    ag = lambda agg=2, Tq=1, sl=None, Hq=16, Hkv=2, pos=1000: lib.qsa_score_select_token_agg(
+        fake, fake, sl, fake, 4, Hq, Hkv, Tq, pos, 64, 128, 16, 0.088, agg, None)
+    assert ag(agg=3) == 1
+    assert ag(Tq=2, sl=fake) == 1
+    assert ag(Hq=32, Hkv=2) == 2
+    assert ag(agg=2, Tq=40, pos=4080) == 1   # queries past the summaries' capacity (64 blocks)
     # self-test limit out of range
     assert lib.qsa_selftest_wait_timeout(0, None) == 1
 

@@ -1,0 +1,127 @@
+"""Per-token selection with other ways of combining the group's heads than
+the pooled query: the softmax-sum aggregator (each head's softmax over the
+complete blocks before the token's diagonal, summed over the heads) and the
+max-over-tokens aggregator (for one token per row, the mean).  The pages
+have the selector score compressed keys against the queries and leave the
+combination open (page "Qwen4 in llama.cpp: Dissecting PR #27742", section
+"QSA Is an Address-Selection Problem, Not a New Attention Equation").
+
+The GPU's indices are compared with the oracle's selection rule applied to
+the oracle's fp64 scores under the same aggregator, from the same fp32
+summaries: exact on rows whose m-th/(m+1)-th score gap exceeds 1e-3, a
+valid top-m (to 1e-5) everywhere.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from tests.helpers import check_selection
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def qsa():
+    import block_sparse_long_compress_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+def _ok(qsa):
+    st = qsa.device_status()
+    assert st[0] == "QSA_OK", st
+
+
+CASES = [
+    # name, B, Tq, q_pos0, Hq, Hkv, d, topk, plant fraction, plant scale
+    ("planted_g8", 4, 1, 64 * 60 + 4, 16, 2, 128, 8, 0.2, 4.0),
+    ("tokens_g4_d64", 2, 3, 64 * 150 + 2, 8, 2, 64, 16, 0.1, 3.0),
+    ("long_multichunk", 2, 1, 64 * 3000 - 1, 16, 2, 128, 32, 0.02, 4.0),
+    # more than 8 x 1024 candidates: chunks too long to keep the softmax-sum
+    # logits in shared memory (they are recomputed)
+    ("very_long_recompute", 1, 1, 64 * 9000 - 1, 16, 2, 128, 16, 0.002, 4.0),
+]
+
+
+@pytest.mark.parametrize("agg", ["softmax_sum", "max"])
+@pytest.mark.parametrize("name,B,Tq,q_pos0,Hq,Hkv,d,topk,frac,scale", CASES, ids=[c[0] for c in CASES])
+def test_token_aggregator_parity(qsa, agg, name, B, Tq, q_pos0, Hq, Hkv, d, topk, frac, scale):
+    nblk = (q_pos0 + Tq + 63) // 64
+    w = synthetic.custom(B=B, Tq=Tq, T_kv=64 * nblk, q_pos0=q_pos0, qblk=1, Hq=Hq, Hkv=Hkv, d=d, topk=topk,
+                         seed=211, plant="token", plant_frac=frac, plant_scale=scale)
+    x = synthetic.generate(w)
+    Kc = torch.from_numpy(oracle.compress_keys(x["K"], 0, nblk).astype(np.float32))   # the summaries both sides use
+    idx = torch.full((B, Hkv, Tq, topk), -7, dtype=torch.int32, device=DEV)
+    qsa.score_select_token_agg(x["Q"].to(DEV), Kc.to(DEV), idx, topk, q_pos0, agg, w.sm_scale)
+    _ok(qsa)
+    s = oracle.block_scores(x["Q"], Kc.double().numpy(), Tq, q_pos0, 1, w.sm_scale, agg)
+    sel = oracle.select_scores(s, B, Hkv, Tq, q_pos0, 1, topk)
+    NB = s.shape[-1]
+    D = [(q_pos0 + i) // 64 for b in range(B) for g in range(Hkv) for i in range(Tq)]
+    frac_checked, jac = check_selection(idx.cpu().numpy().reshape(-1, topk), sel, s.reshape(-1, NB), D, topk)
+    print(f"{agg} {name}: rows gap-checked {frac_checked:.3f}, Jaccard {jac:.4f}")
+    if agg == "softmax_sum" and name == "planted_g8":
+        assert frac_checked > 0.5          # the planted blocks give clear gaps here
+    if agg == "max":
+        # one token per row: the maximum over tokens is the mean, the same kernel
+        ref = torch.full_like(idx, -7)
+        qsa.score_select_token_agg(x["Q"].to(DEV), Kc.to(DEV), ref, topk, q_pos0, "mean", w.sm_scale)
+        assert torch.equal(idx, ref)
+
+
+def test_token_softmax_sum_ragged(qsa):
+    """Per-sequence lengths (one decode token each), softmax-sum aggregator."""
+    lens = [64 * 40 + 7, 64 * 300, 130, 64 * 2 + 1, 64 * 77]
+    Hq, Hkv, d, topk = 16, 2, 128, 16
+    max_blocks = max((L + 63) // 64 for L in lens) + 1
+    Kc_all = torch.zeros((len(lens), Hkv, max_blocks, d), dtype=torch.float32)
+    qs, refs = [], []
+    for b, L in enumerate(lens):
+        w = synthetic.custom(B=1, Tq=1, T_kv=64 * max_blocks, q_pos0=L - 1, qblk=1, Hq=Hq, Hkv=Hkv, d=d,
+                             topk=topk, seed=221 + b, plant="token", plant_frac=0.2, plant_scale=4.0)
+        x = synthetic.generate(w)
+        Kc = oracle.compress_keys(x["K"], 0, L // 64).astype(np.float32)
+        Kc_all[b, :, :L // 64] = torch.from_numpy(Kc[0, :, :L // 64])
+        qs.append(x["Q"])
+        s = oracle.block_scores(x["Q"], Kc_all[b:b + 1].double().numpy(), 1, L - 1, 1, w.sm_scale,
+                                "softmax_sum")
+        refs.append((s, oracle.select_scores(s, 1, Hkv, 1, L - 1, 1, topk), (L - 1) // 64))
+    q = torch.cat(qs, 0).to(DEV)
+    idx = torch.full((len(lens), Hkv, 1, topk), -7, dtype=torch.int32, device=DEV)
+    seq_lens = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    qsa.score_select_token_agg(q, Kc_all.to(DEV), idx, topk, max(lens) - 1, "softmax_sum", d ** -0.5,
+                               seq_lens=seq_lens)
+    _ok(qsa)
+    idx_h = idx.cpu().numpy()
+    for b, (s, sel, D) in enumerate(refs):
+        frac_checked, jac = check_selection(idx_h[b].reshape(-1, topk), sel, s.reshape(Hkv, -1), [D] * Hkv, topk)
+        print(f"ragged softmax-sum seq {b} (L={lens[b]}): gap-checked {frac_checked:.2f}, Jaccard {jac:.4f}")
+
+
+def test_token_softmax_sum_full_size(qsa):
+    """decode_128k (32 sequences at 131072 tokens, top-64), softmax-sum,
+    sampled sequences against the oracle."""
+    w = synthetic.CONFIGS["decode_128k"]
+    x = synthetic.generate(w, DEV)
+    L = w.q_pos0 + 1
+    Kc = torch.zeros((w.B, w.Hkv, w.T_kv // 64, w.d), dtype=torch.float32, device=DEV)
+    qsa.compress_keys(x["K"], Kc, 0, L // 64)
+    idx = torch.full((w.B, w.Hkv, 1, w.topk), -7, dtype=torch.int32, device=DEV)
+    qsa.score_select_token_agg(x["Q"], Kc, idx, w.topk, w.q_pos0, "softmax_sum", w.sm_scale)
+    _ok(qsa)
+    Kc_h = Kc.cpu().double().numpy()
+    Q_h = x["Q"].cpu()
+    idx_h = idx.cpu().numpy()
+    del x
+    torch.cuda.empty_cache()
+    D = (L - 1) // 64
+    for b in (0, 13, w.B - 1):
+        s = oracle.block_scores(Q_h[b:b + 1], Kc_h[b:b + 1], 1, w.q_pos0, 1, w.sm_scale, "softmax_sum")
+        sel = oracle.select_scores(s, 1, w.Hkv, 1, w.q_pos0, 1, w.topk)
+        frac_checked, jac = check_selection(idx_h[b].reshape(-1, w.topk), sel, s.reshape(w.Hkv, -1),
+                                            [D] * w.Hkv, w.topk)
+        print(f"decode_128k softmax-sum seq {b}: gap-checked {frac_checked:.2f}, Jaccard {jac:.4f}")
