@@ -293,6 +293,9 @@ def run_qsa(args, ws, rank, local):
         "clocks": clk.summary(),
     }
 
+    if args.prefill_max:
+        result["prefill_max_selection"] = bench_prefill_max(args, qsa, dev, peaks, wp, Q, K, flush)
+
     # ---- decode at 128K (same process, after the prefill tensors are freed)
     if not args.no_decode:
         del Q, K, V, run, x
@@ -484,6 +487,53 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary=
     # summaries read by scoring (fp32, or bf16 for the bf16-summary option)
     sel_bytes = wd.B * wd.Hkv * ((L - 1) // 64) * wd.d * (2 if summary == "bf16" else 4)
     return decode_result(wd.name, wd.B, L, wd.topk, t, d, launches, by, sel_bytes, peaks, extra)
+
+
+def bench_prefill_max(args, qsa, dev, peaks, wp, Q, K, flush):
+    """Selection of the prefill workload's rows under the max-over-tokens
+    aggregator: per-(head, token) logits of every candidate on the tensor
+    cores (bf16 summaries, written untimed), then the chunked selection.
+    The FLOP rate is over the whole call (scoring + selection)."""
+    nblk = wp.T_kv // 64
+    Kc = torch.empty((wp.B, wp.Hkv, nblk, wp.d), dtype=torch.bfloat16, device=dev)
+    qsa.compress_keys(K, Kc, 0, (wp.q_pos0 + wp.Tq) // 64)
+    NR = -(-wp.Tq // 64)
+    idx = torch.empty((wp.B, wp.Hkv, NR, wp.topk), dtype=torch.int32, device=dev)
+    need = qsa.score_select_prefill_max_workspace(wp.B, wp.Hq, wp.Hkv, wp.Tq, wp.q_pos0, wp.T_kv, wp.d, wp.topk)
+    wsb = torch.empty(need, dtype=torch.uint8, device=dev)
+
+    def call():
+        qsa.score_select_prefill_max(Q, Kc, idx, wp.topk, wp.q_pos0, wp.sm_scale, wsb)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    ts = []
+    for k in range(max(args.steps, 5)):
+        flush(k)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    st, det = qsa.device_status()
+    if st != "QSA_OK":
+        raise RuntimeError(f"prefill max selection device status {st} ({det})")
+    G = wp.Hq // wp.Hkv
+    flops = 0
+    for i in range(NR):
+        t0, t1 = 64 * i, min(64 * (i + 1), wp.Tq)
+        D = (wp.q_pos0 + t1 - 1) // 64
+        flops += 2 * wp.d * (t1 - t0) * G * max(D - 1, 0)
+    flops *= wp.B * wp.Hkv
+    ms = float(np.mean(ts))
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"workload": wp.name, "aggregator": "max over tokens", "summaries": "bf16",
+            "ms": ms, "rows": wp.B * wp.Hkv * NR,
+            "roofline": {"bound": "tensor", "kernel": "block_max_scores_kernel (+ selection, in the time)",
+                         "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"], "flops_per_launch": flops, "traffic": None}}
 
 
 def bench_prefill_paged(args, qsa, dev, peaks, ws, rank, flush):
@@ -714,6 +764,8 @@ def main():
                     help="skip the decode run over the rotated fp8 cache (reported beside the bf16 one)")
     ap.add_argument("--only-decode", action="store_true",
                     help="skip the prefill measurement (profiling the decode kernels)")
+    ap.add_argument("--no-prefill-max", dest="prefill_max", action="store_false",
+                    help="skip the prefill selection with the max-over-tokens aggregator")
     ap.add_argument("--no-softmax-sum", dest="softmax_sum", action="store_false",
                     help="skip the decode run with the softmax-sum selection aggregator")
     ap.add_argument("--decode-variants", default="fp32,bf16,fp8,paged,softmax_sum",

@@ -1,0 +1,213 @@
+// Step 3 for prefill rows under the max-over-tokens aggregator: the score of
+// candidate block j for query block i is the largest, over the block's
+// tokens t, of the group's head mean of sm_scale <q_{h,t}, Kc_j>.  The pages
+// have the selector score compressed keys against the queries (page "Qwen4
+// in llama.cpp: Dissecting PR #27742", section "QSA Is an Address-Selection
+// Problem, Not a New Attention Equation") and leave the combination of the
+// block's tokens and heads open.
+//
+// Unlike the pooled-query score (one dot per block and row), this needs
+// every (head, token) logit: 64 x G rows against every candidate, a dense
+// contraction (0.55 TFLOP over prefill_128k's rows), so it runs on the
+// tensor cores.  The summaries are the bf16 option's (exact bf16 products,
+// fp32 accumulation in TMEM).  The candidates sit on the MMA's M side (128
+// per tile, one TMEM lane each) and the query rows (token, head) on N, so
+// each epilogue thread reduces its own candidate's row: the head sum of
+// every token, then the maximum over the block's valid tokens -- no
+// shuffles.
+//
+// One CTA per (query block, sequence, group), looping over its candidate
+// tiles: warp 0 loads the query block once and streams summary tiles
+// through a 2-stage ring (TMA, 128-byte swizzle), warp 1 issues the MMAs
+// (M = 128, N = 256, K = 128: 8 MMAs per N tile) into one of two TMEM
+// accumulators, warps 2-5 reduce the other.  Scores go to a table
+// [B][Hkv][NR][nblk_max] (candidates 1 .. D-1 of each row); the chunked
+// selection turns the table into indices.
+#pragma once
+
+#include "device.cuh"
+
+namespace qsa {
+
+template <int G>
+struct MaxScoreCfg {
+    static constexpr int D = 128;
+    static constexpr int M = 128;                       // candidates per tile (TMEM lanes)
+    static constexpr int N = 256;                       // query rows (token, head) per MMA
+    static constexpr int TOKN = N / G;                  // tokens per N tile
+    static constexpr int NT = 64 / TOKN;                // N tiles per 64-token query block
+    static constexpr int QHALF_BYTES = N * 128;         // one 64-column half of an N tile (32 KB)
+    static constexpr int QTILE_BYTES = 2 * QHALF_BYTES;
+    static constexpr int Q_BYTES = NT * QTILE_BYTES;    // 128 KB (G = 8) or 64 KB (G = 4)
+    static constexpr int KHALF_BYTES = M * 128;         // 16 KB
+    static constexpr int KSTAGE_BYTES = 2 * KHALF_BYTES;
+    static constexpr int NS = 2;
+    static constexpr int SMEM_BYTES = Q_BYTES + NS * KSTAGE_BYTES + 1024;
+    static constexpr int THREADS = 192;                 // producer, issuer, 4 epilogue warps
+    static constexpr int TMEM_COLS = 2 * N;             // two fp32 accumulators
+    static_assert(N % G == 0 && 64 % TOKN == 0, "tile shape");
+};
+
+template <int G>
+__global__ void __launch_bounds__(MaxScoreCfg<G>::THREADS, 1) block_max_scores_kernel(
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
+    float *__restrict__ scores, int Tq, int q_pos0, int nblk_max, int Hkv, float sm_scale)
+{
+    using C = MaxScoreCfg<G>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ uint64_t q_full, k_full[C::NS], k_empty[C::NS], t_full[2], t_empty[2];
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag, issued_k, issued_mma;
+
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *q_smem = base;
+    uint8_t *k_smem = base + C::Q_BYTES;
+    const int i = blockIdx.x, bg = blockIdx.y, NR = gridDim.x;
+    const int b = bg / Hkv, g = bg % Hkv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t_last = min((i + 1) * 64, Tq) - 1;
+    const int Dg = (q_pos0 + t_last) / 64;              // the row's diagonal block
+    const int ncand = max(Dg - 1, 0);                   // candidates 1 .. Dg-1
+    const int ntiles = (ncand + C::M - 1) / C::M;
+    if (ntiles == 0) return;                            // uniform: no barrier or TMEM yet
+    const int nwork = ntiles * C::NT;                   // (candidate tile, N tile) pairs
+
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        issued_k = 0;
+        issued_mma = 0;
+        mbar_init(&q_full, 1);
+#pragma unroll
+        for (int s = 0; s < C::NS; s++) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+#pragma unroll
+        for (int s = 0; s < 2; s++) {
+            mbar_init(&t_full[s], 1);
+            mbar_init(&t_empty[s], 4);                  // one arrival per epilogue warp
+        }
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+    volatile int *abort = &abort_flag;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            // the query block's rows (token, head) of the group: N tile nt
+            // holds tokens nt*TOKN .. +TOKN, each 64-column half one 3-D box
+            mbar_arrive_expect_tx(&q_full, C::Q_BYTES);
+#pragma unroll
+            for (int nt = 0; nt < C::NT; nt++)
+#pragma unroll
+                for (int h = 0; h < 2; h++)
+                    tma_load_3d(q_smem + nt * C::QTILE_BYTES + h * C::QHALF_BYTES, &tmQ, &q_full, h * 64, g * G,
+                                b * Tq + i * 64 + nt * C::TOKN);
+            int k = 0;
+            for (; k < ntiles; k++) {
+                const int st = k % C::NS;
+                if (k >= C::NS && !mbar_wait(&k_empty[st], ((k / C::NS) - 1) & 1, abort, 70)) break;
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(&k_full[st], C::KSTAGE_BYTES);
+                const int row = bg * nblk_max + 1 + C::M * k;   // host checks B*Hkv*nblk_max < 2^31
+#pragma unroll
+                for (int h = 0; h < 2; h++)
+                    tma_load_2d(k_smem + st * C::KSTAGE_BYTES + h * C::KHALF_BYTES, &tmKc, &k_full[st], h * 64, row);
+            }
+            issued_k = k;
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------- MMA issuer (whole warp)
+        constexpr uint32_t idesc = umma_idesc_bf16(C::M, C::N, 0, 0);
+        const uint64_t qd = umma_smem_desc(smem_u32(q_smem), 16, 1024);
+        const uint64_t kd = umma_smem_desc(smem_u32(k_smem), 16, 1024);
+        auto wait_all = [&](uint64_t *bar, uint32_t parity, int where) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, where));
+        };
+        int w = 0;
+        if (wait_all(&q_full, 0, 71)) {
+            for (; w < nwork; w++) {
+                const int k = w / C::NT, nt = w % C::NT, st = k % C::NS, buf = w & 1;
+                if (nt == 0 && !wait_all(&k_full[st], (k / C::NS) & 1, 72)) break;
+                if (w >= 2 && !wait_all(&t_empty[buf], ((w >> 1) - 1) & 1, 73)) break;
+                tc_fence_after();
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < C::D / 16; kk++) {
+                        const uint64_t aoff = (uint64_t)((st * C::KSTAGE_BYTES + (kk >> 2) * C::KHALF_BYTES + (kk & 3) * 32) >> 4);
+                        const uint64_t boff = (uint64_t)((nt * C::QTILE_BYTES + (kk >> 2) * C::QHALF_BYTES + (kk & 3) * 32) >> 4);
+                        umma_ss(tmem + buf * C::N, kd + aoff, qd + boff, idesc, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&t_full[buf]);
+                    if (nt == C::NT - 1) umma_commit(&k_empty[st]);
+                }
+                __syncwarp();
+            }
+        }
+        if (lane == 0) issued_mma = w;
+    } else {
+        // ------------------------------------------- epilogue (warps 2-5)
+        const int quarter = warp & 3;                  // the TMEM lanes this warp may access
+        const int m = 32 * quarter + lane;             // candidate within the tile
+        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+        float best = -INFINITY;
+        for (int w = 0; w < nwork; w++) {
+            const int k = w / C::NT, nt = w % C::NT, buf = w & 1;
+            // warp-uniform: the TMEM loads below are collective
+            if (!__all_sync(0xffffffffu, mbar_wait(&t_full[buf], (w >> 1) & 1, abort, 74))) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < C::N; c += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_base + buf * C::N + c, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int tt = 0; tt < 32 / G; tt++) {
+                    const int t = i * 64 + nt * C::TOKN + c / G + tt;   // token of these G columns
+                    float sum = 0.f;
+#pragma unroll
+                    for (int h = 0; h < G; h++) sum += __uint_as_float(r[tt * G + h]);
+                    if (t < Tq) best = fmaxf(best, sum);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&t_empty[buf]);
+            if (nt == C::NT - 1) {
+                const int j = 1 + C::M * k + m;
+                if (j < Dg) scores[((long)bg * NR + i) * nblk_max + j] = best * (1.0f / (float)G) * sm_scale;
+                best = -INFINITY;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (abort_flag && threadIdx.x == 0) {
+        // a wait gave up: let the copies and MMAs still in flight finish
+        // before the shared memory and TMEM go away (bounded, no abort
+        // short-cut)
+        mbar_wait(&q_full, 0, nullptr, 75, 100000000ull);
+        for (int k = max(0, issued_k - C::NS); k < issued_k; k++)
+            mbar_wait(&k_full[k % C::NS], (k / C::NS) & 1, nullptr, 76, 100000000ull);
+        if (issued_mma > 0) {
+            const int w = issued_mma - 1;
+            mbar_wait(&t_full[w & 1], (w >> 1) & 1, nullptr, 77, 100000000ull);
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace qsa

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "../../include/qsa.h"
+#include "aggregate.cuh"
 #include "compress.cuh"
 #include "decode.cuh"
 #include "device.cuh"
@@ -73,13 +74,13 @@ EncodeTiledFn encode_fn()
 }
 
 // 2-D bf16 view [rows][cols] (cols contiguous) with 64 x 64 boxes, 128-byte swizzle.
-qsa_status make_map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols)
+qsa_status make_map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows = 64)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return fail(QSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, 64};
+    cuuint32_t box[2] = {64, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -612,6 +613,78 @@ qsa_status qsa_score_select_token_agg(const void *Q, const float *Kc, const int3
                                                 s, seq_lens);
     return launch_select_token<float>(Q, Kc, idx, B, Hq, Hkv, Tq, q_pos0, max_blocks, d, topk, sm_scale, tp, s,
                                       seq_lens);
+}
+
+size_t qsa_score_select_prefill_max_workspace(int B, int Hq, int Hkv, int Tq, int q_pos0, int T_kv_max, int d,
+                                              int topk)
+{
+    (void)Hq;
+    (void)topk;
+    if (B <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || T_kv_max <= 0 || T_kv_max % 64 || d != 128) return 0;
+    const SelectPlan p = plan_select(B, Hkv, Tq, q_pos0, 64, d);
+    return align256((size_t)B * Hkv * p.NR * (T_kv_max / 64) * sizeof(float)) + p.part_bytes;
+}
+
+qsa_status qsa_score_select_prefill_max(const void *Q, const void *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
+                                        int q_pos0, int T_kv_max, int d, int topk, float sm_scale, void *workspace,
+                                        size_t workspace_bytes, qsa_stream_t stream)
+{
+    const char *name = "qsa_score_select_prefill_max";
+    if (!Q || !Kc || !idx) return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || T_kv_max <= 0 || T_kv_max % 64 || Hq % Hkv ||
+        q_pos0 % 64 || (long)q_pos0 + Tq > T_kv_max)
+        return fail(QSA_ERR_INVALID_ARG, "%s: bad shape", name);
+    if (d != 128) return fail(QSA_ERR_UNSUPPORTED, "%s: d=%d", name, d);
+    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "%s: topk=%d", name, topk);
+    const int G = Hq / Hkv;
+    if (G != 4 && G != 8) return fail(QSA_ERR_UNSUPPORTED, "%s: Hq/Hkv=%d", name, G);
+    const int nblk = T_kv_max / 64;
+    if ((long)B * Hkv * nblk >= (1L << 31) || (long)B * Tq >= (1L << 31))
+        return fail(QSA_ERR_UNSUPPORTED, "%s: too large", name);
+    if (!aligned16(Q) || !aligned16(Kc) || !aligned16(idx) || (workspace && !aligned16(workspace)))
+        return fail(QSA_ERR_INVALID_ARG, "%s: misaligned pointer", name);
+    const SelectPlan p = plan_select(B, Hkv, Tq, q_pos0, 64, d);
+    if (p.NR > 65535 || (long)B * Hkv > 65535) return fail(QSA_ERR_UNSUPPORTED, "%s: too many rows", name);
+    if (p.maxchunks * qsa::kMaxChosen * 8 > 200 * 1024) return fail(QSA_ERR_UNSUPPORTED, "%s: context too long", name);
+    const size_t score_bytes = align256((size_t)B * Hkv * p.NR * nblk * sizeof(float));
+    if (!workspace || workspace_bytes < score_bytes + p.part_bytes)
+        return fail(QSA_ERR_WORKSPACE, "%s: workspace needs %zu bytes", name, score_bytes + p.part_bytes);
+    float *scores = static_cast<float *>(workspace);
+    uint64_t *part = reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(workspace) + score_bytes);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    qsa_status st;
+    CUtensorMap mq, mk;
+    if ((st = make_map_2d(&mk, Kc, (uint64_t)B * Hkv * nblk, 128, 128)) != QSA_OK) return st;
+    const dim3 grid(p.NR, B * Hkv);
+    if (G == 8) {
+        using C = qsa::MaxScoreCfg<8>;
+        if ((st = make_map_q(&mq, Q, (uint64_t)B * Tq, Hq, 128, 8, C::TOKN)) != QSA_OK) return st;
+        if ((st = set_smem(qsa::block_max_scores_kernel<8>, C::SMEM_BYTES)) != QSA_OK) return st;
+        qsa::block_max_scores_kernel<8><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, scores, Tq, q_pos0, nblk, Hkv,
+                                                                              sm_scale);
+    } else {
+        using C = qsa::MaxScoreCfg<4>;
+        if ((st = make_map_q(&mq, Q, (uint64_t)B * Tq, Hq, 128, 4, C::TOKN)) != QSA_OK) return st;
+        if ((st = set_smem(qsa::block_max_scores_kernel<4>, C::SMEM_BYTES)) != QSA_OK) return st;
+        qsa::block_max_scores_kernel<4><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, scores, Tq, q_pos0, nblk, Hkv,
+                                                                              sm_scale);
+    }
+    if ((st = launched("block_max_scores_kernel")) != QSA_OK) return st;
+    const dim3 sgrid(p.maxchunks, p.NR, B * Hkv), mgrid(p.NR, B * Hkv);
+    auto skern = qsa::score_select_kernel<128, __nv_bfloat16, true>;
+    if ((st = set_smem(skern, p.CH * 8)) != QSA_OK) return st;
+    skern<<<sgrid, qsa::kSelThreads, p.CH * 8, s>>>(nullptr, static_cast<const __nv_bfloat16 *>(Kc), idx, part, nblk,
+                                                    Tq, q_pos0, 64, topk, sm_scale, p.CH, p.maxchunks, Hkv, nullptr,
+                                                    scores);
+    if ((st = launched("score_select_kernel")) != QSA_OK) return st;
+    if (p.maxchunks > 1) {
+        const int msmem = p.maxchunks * qsa::kMaxChosen * 8;
+        if ((st = set_smem(qsa::merge_select_kernel, msmem)) != QSA_OK) return st;
+        qsa::merge_select_kernel<<<mgrid, qsa::kSelThreads, msmem, s>>>(part, idx, Tq, q_pos0, 64, topk, p.CH,
+                                                                       p.maxchunks, Hkv, nblk, nullptr);
+        if ((st = launched("merge_select_kernel")) != QSA_OK) return st;
+    }
+    return QSA_OK;
 }
 
 qsa_status qsa_score_select_ragged_prefill(const void *Q, const float *Kc, const int32_t *q_pos, int32_t *idx,

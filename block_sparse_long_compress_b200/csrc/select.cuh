@@ -429,11 +429,15 @@ __device__ __forceinline__ void lse2_merge(float &m, float &s, float m2, float s
 
 // --------------------------------------------------------- score+select
 // grid (maxchunks, NR, B*Hkv); dynamic smem CH * 8 bytes.
-template <int D, typename KcT>
+// FROM_SCORES: the candidates' scores come from a table [B*Hkv][NR][nblk_max]
+// written by another scoring kernel (the aggregator variants) instead of
+// the pooled-query dots.
+template <int D, typename KcT, bool FROM_SCORES = false>
 __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
     const float *__restrict__ Qbar, const KcT *__restrict__ Kc, int32_t *__restrict__ idx,
     uint64_t *__restrict__ part, int nblk_max, int Tq, int q_pos0, int qblk, int topk,
-    float sm_scale, int CH, int maxchunks, int Hkv, const int32_t *__restrict__ q_pos)
+    float sm_scale, int CH, int maxchunks, int Hkv, const int32_t *__restrict__ q_pos,
+    const float *__restrict__ scores = nullptr)
 {
     extern __shared__ uint64_t keys[];
     __shared__ SelectShared sh;
@@ -446,7 +450,12 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
     const int n = max(0, min(CH, g.ncand - chunk * CH));
     const long row = (long)bg * NR + i;
 
-    score_chunk<D, KcT>(Qbar + row * D, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
+    if constexpr (FROM_SCORES) {
+        const float *srow = scores + row * nblk_max + j0;
+        for (int e = threadIdx.x; e < n; e += kSelThreads) keys[e] = make_key(__ldg(srow + e), j0 + e);
+    } else {
+        score_chunk<D, KcT>(Qbar + row * D, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
+    }
     __syncthreads();
 
     const int need = min(g.m, n);
