@@ -294,7 +294,9 @@ def run_qsa(args, ws, rank, local):
     }
 
     if args.prefill_max:
-        result["prefill_max_selection"] = bench_prefill_max(args, qsa, dev, peaks, wp, Q, K, flush)
+        result["prefill_max_selection"] = bench_prefill_agg(args, qsa, dev, peaks, wp, Q, K, flush, "max")
+        result["prefill_softmax_sum_selection"] = bench_prefill_agg(args, qsa, dev, peaks, wp, Q, K, flush,
+                                                                    "softmax_sum")
 
     # ---- decode at 128K (same process, after the prefill tensors are freed)
     if not args.no_decode:
@@ -489,21 +491,22 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary=
     return decode_result(wd.name, wd.B, L, wd.topk, t, d, launches, by, sel_bytes, peaks, extra)
 
 
-def bench_prefill_max(args, qsa, dev, peaks, wp, Q, K, flush):
-    """Selection of the prefill workload's rows under the max-over-tokens
-    aggregator: per-(head, token) logits of every candidate on the tensor
-    cores (bf16 summaries, written untimed), then the chunked selection.
-    The FLOP rate is over the whole call (scoring + selection)."""
+def bench_prefill_agg(args, qsa, dev, peaks, wp, Q, K, flush, agg):
+    """Selection of the prefill workload's rows under the max-over-tokens or
+    the softmax-sum aggregator: per-(head, token) logits of every candidate
+    on the tensor cores (bf16 summaries, written untimed), then the chunked
+    selection.  The FLOP rate is over the whole call (scoring, for the
+    softmax-sum both passes, + selection)."""
     nblk = wp.T_kv // 64
     Kc = torch.empty((wp.B, wp.Hkv, nblk, wp.d), dtype=torch.bfloat16, device=dev)
     qsa.compress_keys(K, Kc, 0, (wp.q_pos0 + wp.Tq) // 64)
     NR = -(-wp.Tq // 64)
     idx = torch.empty((wp.B, wp.Hkv, NR, wp.topk), dtype=torch.int32, device=dev)
-    need = qsa.score_select_prefill_max_workspace(wp.B, wp.Hq, wp.Hkv, wp.Tq, wp.q_pos0, wp.T_kv, wp.d, wp.topk)
+    need = qsa.score_select_prefill_agg_workspace(wp.B, wp.Hq, wp.Hkv, wp.Tq, wp.q_pos0, wp.T_kv, wp.d, wp.topk, agg)
     wsb = torch.empty(need, dtype=torch.uint8, device=dev)
 
     def call():
-        qsa.score_select_prefill_max(Q, Kc, idx, wp.topk, wp.q_pos0, wp.sm_scale, wsb)
+        qsa.score_select_prefill_agg(Q, Kc, idx, wp.topk, wp.q_pos0, agg, wp.sm_scale, wsb)
 
     for _ in range(args.warmup):
         call()
@@ -519,17 +522,19 @@ def bench_prefill_max(args, qsa, dev, peaks, wp, Q, K, flush):
         ts.append(e0.elapsed_time(e1))
     st, det = qsa.device_status()
     if st != "QSA_OK":
-        raise RuntimeError(f"prefill max selection device status {st} ({det})")
+        raise RuntimeError(f"prefill {agg} selection device status {st} ({det})")
     G = wp.Hq // wp.Hkv
     flops = 0
     for i in range(NR):
         t0, t1 = 64 * i, min(64 * (i + 1), wp.Tq)
         D = (wp.q_pos0 + t1 - 1) // 64
-        flops += 2 * wp.d * (t1 - t0) * G * max(D - 1, 0)
+        # logits of the candidates (and, for the softmax-sum's statistics
+        # pass, of every block before the diagonal)
+        flops += 2 * wp.d * (t1 - t0) * G * (max(D - 1, 0) + (D if agg == "softmax_sum" and D > 1 else 0))
     flops *= wp.B * wp.Hkv
     ms = float(np.mean(ts))
     achieved = flops / (ms * 1e-3) / 1e12
-    return {"workload": wp.name, "aggregator": "max over tokens", "summaries": "bf16",
+    return {"workload": wp.name, "aggregator": agg, "summaries": "bf16",
             "ms": ms, "rows": wp.B * wp.Hkv * NR,
             "roofline": {"bound": "tensor", "kernel": "block_max_scores_kernel (+ selection, in the time)",
                          "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",

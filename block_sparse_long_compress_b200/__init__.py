@@ -58,8 +58,8 @@ def _load():
         "qsa_decode_paged": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "qsa_score_select_ragged_prefill": (I, [P, P, P, P, I, I, I, I, I, I, I, I, F, P, S, P]),
         "qsa_score_select_token_agg": (I, [P, P, P, P, I, I, I, I, I, I, I, I, F, I, P]),
-        "qsa_score_select_prefill_max_workspace": (S, [I, I, I, I, I, I, I, I]),
-        "qsa_score_select_prefill_max": (I, [P, P, P, I, I, I, I, I, I, I, I, F, P, S, P]),
+        "qsa_score_select_prefill_agg_workspace": (S, [I, I, I, I, I, I, I, I, I]),
+        "qsa_score_select_prefill_agg": (I, [P, P, P, I, I, I, I, I, I, I, I, F, I, P, S, P]),
         "qsa_quantize_kv_fp8": (I, [P, P, P, ctypes.c_int64, I, P]),
         "qsa_decode_fp8": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "qsa_decode_fp8_paged": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
@@ -284,27 +284,30 @@ def score_select_token_agg(q, Kc, idx, topk, q_pos0, aggregator="mean", sm_scale
     return idx
 
 
-def score_select_prefill_max_workspace(B, Hq, Hkv, Tq, q_pos0, T_kv_max, d, topk):
-    return int(_lib.qsa_score_select_prefill_max_workspace(B, Hq, Hkv, Tq, q_pos0, T_kv_max, d, topk))
+def score_select_prefill_agg_workspace(B, Hq, Hkv, Tq, q_pos0, T_kv_max, d, topk, aggregator):
+    return int(_lib.qsa_score_select_prefill_agg_workspace(B, Hq, Hkv, Tq, q_pos0, T_kv_max, d, topk,
+                                                          AGGREGATORS[aggregator]))
 
 
-def score_select_prefill_max(Q, Kc, idx, topk, q_pos0, sm_scale=None, workspace=None, stream=None):
-    """Selection for 64-token query blocks under the max-over-tokens
-    aggregator (per-(head, token) logits on the tensor cores).  Q bf16
-    [B, Tq, Hq, 128]; Kc bf16 summaries [B, Hkv, T_kv_max//64, 128]; idx int32
-    [B, Hkv, ceil(Tq/64), topk] (written)."""
+def score_select_prefill_agg(Q, Kc, idx, topk, q_pos0, aggregator="max", sm_scale=None, workspace=None,
+                             stream=None):
+    """Selection for 64-token query blocks under the max-over-tokens or the
+    softmax-sum aggregator (per-(head, token) logits on the tensor cores).
+    Q bf16 [B, Tq, Hq, 128]; Kc bf16 summaries [B, Hkv, T_kv_max//64, 128];
+    idx int32 [B, Hkv, ceil(Tq/64), topk] (written)."""
     B, Tq, Hq, d = Q.shape
     _, Hkv, nblk, _ = Kc.shape
     if sm_scale is None:
         sm_scale = d ** -0.5
-    need = score_select_prefill_max_workspace(B, Hq, Hkv, Tq, q_pos0, 64 * nblk, d, topk)
+    need = score_select_prefill_agg_workspace(B, Hq, Hkv, Tq, q_pos0, 64 * nblk, d, topk, aggregator)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=Q.device)
-    _check(_lib.qsa_score_select_prefill_max(_ptr(Q, torch.bfloat16, "Q"), _ptr(Kc, torch.bfloat16, "Kc"),
+    _check(_lib.qsa_score_select_prefill_agg(_ptr(Q, torch.bfloat16, "Q"), _ptr(Kc, torch.bfloat16, "Kc"),
                                              _ptr(idx, torch.int32, "idx"), B, Hq, Hkv, Tq, q_pos0, 64 * nblk, d,
-                                             topk, float(sm_scale), _ptr(workspace, torch.uint8, "workspace"),
-                                             workspace.numel(), _stream(stream)),
-           "qsa_score_select_prefill_max")
+                                             topk, float(sm_scale), AGGREGATORS[aggregator],
+                                             _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                                             _stream(stream)),
+           "qsa_score_select_prefill_agg")
     return idx
 
 

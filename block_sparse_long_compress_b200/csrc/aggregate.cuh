@@ -23,6 +23,14 @@
 // accumulators, warps 2-5 reduce the other.  Scores go to a table
 // [B][Hkv][NR][nblk_max] (candidates 1 .. D-1 of each row); the chunked
 // selection turns the table into indices.
+//
+// The softmax-sum aggregator (s_j = sum over the block's (head, token) rows
+// of each row's softmax over the blocks 0 .. D-1, at j) takes two passes:
+// block_softmax_stats_kernel puts the (head, token) rows on M and the blocks
+// on N -- the shape of an attention score tile -- so that every thread keeps
+// its row's running (max, sum) in base 2; then block_max_scores_kernel in
+// its SOFTMAX mode forms, per candidate, the sum of 2^(z - max) / sum over
+// the rows, with the rows' statistics in shared memory.
 #pragma once
 
 #include "device.cuh"
@@ -48,16 +56,20 @@ struct MaxScoreCfg {
     static_assert(N % G == 0 && 64 % TOKN == 0, "tile shape");
 };
 
-template <int G>
+// SOFTMAX: the softmax-sum's second pass -- stats[(bg*NR + i)][64*G][2]
+// holds each (token, head) row's base-2 (max, sum) from the first pass.
+template <int G, bool SOFTMAX = false>
 __global__ void __launch_bounds__(MaxScoreCfg<G>::THREADS, 1) block_max_scores_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
-    float *__restrict__ scores, int Tq, int q_pos0, int nblk_max, int Hkv, float sm_scale)
+    float *__restrict__ scores, int Tq, int q_pos0, int nblk_max, int Hkv, float sm_scale,
+    const float *__restrict__ stats = nullptr)
 {
     using C = MaxScoreCfg<G>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t q_full, k_full[C::NS], k_empty[C::NS], t_full[2], t_empty[2];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag, issued_k, issued_mma;
+    __shared__ float rstat[SOFTMAX ? 64 * G : 1][2];   // SOFTMAX: (max, 1/sum) per (token, head) row
 
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *q_smem = base;
@@ -92,6 +104,13 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::THREADS, 1) block_max_scores_k
     if (warp == 1) {
         tmem_alloc(&tmem_base, C::TMEM_COLS);
         tmem_relinquish();
+    }
+    if constexpr (SOFTMAX) {
+        const float *st = stats + ((long)bg * NR + i) * (64 * G) * 2;
+        for (int r = threadIdx.x; r < 64 * G; r += C::THREADS) {
+            rstat[r][0] = st[2 * r];
+            rstat[r][1] = st[2 * r + 1] > 0.f ? 1.f / st[2 * r + 1] : 0.f;
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -172,10 +191,23 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::THREADS, 1) block_max_scores_k
 #pragma unroll
                 for (int tt = 0; tt < 32 / G; tt++) {
                     const int t = i * 64 + nt * C::TOKN + c / G + tt;   // token of these G columns
-                    float sum = 0.f;
+                    if constexpr (SOFTMAX) {
+                        // best accumulates the rows' shares of this block
+                        const int r0 = (nt * C::TOKN + c / G + tt) * G;  // (token, head) row in the block
+                        const float sc2 = sm_scale * 1.4426950408889634f;
+                        if (t < Tq) {
+                            if (best == -INFINITY) best = 0.f;
 #pragma unroll
-                    for (int h = 0; h < G; h++) sum += __uint_as_float(r[tt * G + h]);
-                    if (t < Tq) best = fmaxf(best, sum);
+                            for (int h = 0; h < G; h++)
+                                best += fast_exp2(__uint_as_float(r[tt * G + h]) * sc2 - rstat[r0 + h][0]) *
+                                        rstat[r0 + h][1];
+                        }
+                    } else {
+                        float sum = 0.f;
+#pragma unroll
+                        for (int h = 0; h < G; h++) sum += __uint_as_float(r[tt * G + h]);
+                        if (t < Tq) best = fmaxf(best, sum);
+                    }
                 }
             }
             tc_fence_before();
@@ -183,7 +215,9 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::THREADS, 1) block_max_scores_k
             if (lane == 0) mbar_arrive(&t_empty[buf]);
             if (nt == C::NT - 1) {
                 const int j = 1 + C::M * k + m;
-                if (j < Dg) scores[((long)bg * NR + i) * nblk_max + j] = best * (1.0f / (float)G) * sm_scale;
+                if (j < Dg)
+                    scores[((long)bg * NR + i) * nblk_max + j] =
+                        SOFTMAX ? best : best * (1.0f / (float)G) * sm_scale;
                 best = -INFINITY;
             }
         }
@@ -201,6 +235,183 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::THREADS, 1) block_max_scores_k
         if (issued_mma > 0) {
             const int w = issued_mma - 1;
             mbar_wait(&t_full[w & 1], (w >> 1) & 1, nullptr, 77, 100000000ull);
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// First pass of the softmax-sum: per (token, head) row of the query block,
+// the base-2 (max, sum of 2^(z - max)) of z = sm_scale log2(e) <q, Kc_j>
+// over the blocks j in 0 .. D-1.  One CTA per (query block, sequence, group,
+// 128-row M tile of 128/G tokens x G heads); the blocks stream through in
+// N tiles of 256 (the same warp roles as block_max_scores_kernel).  Output:
+// stats[(bg*NR + i)][64*G][2], row (token, head) = t_local*G + h.
+template <int G>
+struct SoftmaxStatsCfg {
+    static constexpr int D = 128;
+    static constexpr int M = 128;                       // (token, head) rows per CTA
+    static constexpr int N = 256;                       // blocks per tile
+    static constexpr int TOKM = M / G;                  // tokens per CTA
+    static constexpr int NMT = 64 / TOKM;               // M tiles per query block
+    static constexpr int QHALF_BYTES = M * 128;         // 16 KB
+    static constexpr int Q_BYTES = 2 * QHALF_BYTES;
+    static constexpr int KHALF_BYTES = N * 128;         // 32 KB
+    static constexpr int KSTAGE_BYTES = 2 * KHALF_BYTES;
+    static constexpr int NS = 2;
+    static constexpr int SMEM_BYTES = Q_BYTES + NS * KSTAGE_BYTES + 1024;
+    static constexpr int THREADS = 192;
+    static constexpr int TMEM_COLS = 2 * N;
+};
+
+template <int G>
+__global__ void __launch_bounds__(SoftmaxStatsCfg<G>::THREADS, 1) block_softmax_stats_kernel(
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
+    float *__restrict__ stats, int Tq, int q_pos0, int nblk_max, int Hkv, float sm_scale)
+{
+    using C = SoftmaxStatsCfg<G>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ uint64_t q_full, k_full[C::NS], k_empty[C::NS], t_full[2], t_empty[2];
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag, issued_k, issued_mma;
+
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *q_smem = base;
+    uint8_t *k_smem = base + C::Q_BYTES;
+    const int i = blockIdx.x / C::NMT, mt = blockIdx.x % C::NMT, bg = blockIdx.y, NR = gridDim.x / C::NMT;
+    const int b = bg / Hkv, g = bg % Hkv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t_last = min((i + 1) * 64, Tq) - 1;
+    const int Dg = (q_pos0 + t_last) / 64;              // blocks 0 .. Dg-1 normalise
+    const int ntiles = (Dg + C::N - 1) / C::N;
+    if (Dg < 2) return;                                 // no candidate: nothing reads these rows
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        issued_k = 0;
+        issued_mma = 0;
+        mbar_init(&q_full, 1);
+#pragma unroll
+        for (int s = 0; s < C::NS; s++) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+#pragma unroll
+        for (int s = 0; s < 2; s++) {
+            mbar_init(&t_full[s], 1);
+            mbar_init(&t_empty[s], 4);
+        }
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+    volatile int *abort = &abort_flag;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&q_full, C::Q_BYTES);
+#pragma unroll
+            for (int h = 0; h < 2; h++)
+                tma_load_3d(q_smem + h * C::QHALF_BYTES, &tmQ, &q_full, h * 64, g * G, b * Tq + i * 64 + mt * C::TOKM);
+            int k = 0;
+            for (; k < ntiles; k++) {
+                const int st = k % C::NS;
+                if (k >= C::NS && !mbar_wait(&k_empty[st], ((k / C::NS) - 1) & 1, abort, 80)) break;
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(&k_full[st], C::KSTAGE_BYTES);
+                const int row = bg * nblk_max + C::N * k;   // host checks B*Hkv*nblk_max < 2^31
+#pragma unroll
+                for (int h = 0; h < 2; h++)
+                    tma_load_2d(k_smem + st * C::KSTAGE_BYTES + h * C::KHALF_BYTES, &tmKc, &k_full[st], h * 64, row);
+            }
+            issued_k = k;
+        }
+    } else if (warp == 1) {
+        constexpr uint32_t idesc = umma_idesc_bf16(C::M, C::N, 0, 0);
+        const uint64_t qd = umma_smem_desc(smem_u32(q_smem), 16, 1024);
+        const uint64_t kd = umma_smem_desc(smem_u32(k_smem), 16, 1024);
+        auto wait_all = [&](uint64_t *bar, uint32_t parity, int where) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, where));
+        };
+        int k = 0;
+        if (wait_all(&q_full, 0, 81)) {
+            for (; k < ntiles; k++) {
+                const int st = k % C::NS, buf = k & 1;
+                if (!wait_all(&k_full[st], (k / C::NS) & 1, 82)) break;
+                if (k >= 2 && !wait_all(&t_empty[buf], ((k >> 1) - 1) & 1, 83)) break;
+                tc_fence_after();
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < C::D / 16; kk++) {
+                        const uint64_t aoff = (uint64_t)(((kk >> 2) * C::QHALF_BYTES + (kk & 3) * 32) >> 4);
+                        const uint64_t boff = (uint64_t)((st * C::KSTAGE_BYTES + (kk >> 2) * C::KHALF_BYTES + (kk & 3) * 32) >> 4);
+                        umma_ss(tmem + buf * C::N, qd + aoff, kd + boff, idesc, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&t_full[buf]);
+                    umma_commit(&k_empty[st]);
+                }
+                __syncwarp();
+            }
+        }
+        if (lane == 0) issued_mma = k;
+    } else {
+        const int quarter = warp & 3;
+        const int r = 32 * quarter + lane;             // (token, head) row of the M tile
+        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+        const float sc2 = sm_scale * 1.4426950408889634f;
+        float m_run = -INFINITY, s_run = 0.f;
+        int k = 0;
+        for (; k < ntiles; k++) {
+            const int buf = k & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&t_full[buf], (k >> 1) & 1, abort, 84))) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < C::N; c += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + buf * C::N + c, v);
+                tmem_wait_ld();
+                const int j0 = C::N * k + c;            // block of column 0 of this chunk
+                float mx = -INFINITY;
+#pragma unroll
+                for (int e = 0; e < 32; e++)
+                    if (j0 + e < Dg) mx = fmaxf(mx, __uint_as_float(v[e]) * sc2);
+                if (mx == -INFINITY) continue;
+                const float mn = fmaxf(m_run, mx);
+                float acc = 0.f;
+#pragma unroll
+                for (int e = 0; e < 32; e++)
+                    if (j0 + e < Dg) acc += fast_exp2(__uint_as_float(v[e]) * sc2 - mn);
+                s_run = s_run * fast_exp2(m_run - mn) + acc;
+                m_run = mn;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&t_empty[buf]);
+        }
+        if (k == ntiles) {
+            float *out = stats + (((long)bg * NR + i) * (64 * G) + mt * C::M + r) * 2;
+            out[0] = m_run;
+            out[1] = s_run;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (abort_flag && threadIdx.x == 0) {
+        mbar_wait(&q_full, 0, nullptr, 85, 100000000ull);
+        for (int k = max(0, issued_k - C::NS); k < issued_k; k++)
+            mbar_wait(&k_full[k % C::NS], (k / C::NS) & 1, nullptr, 86, 100000000ull);
+        if (issued_mma > 0) {
+            const int w = issued_mma - 1;
+            mbar_wait(&t_full[w & 1], (w >> 1) & 1, nullptr, 87, 100000000ull);
         }
     }
     __syncthreads();

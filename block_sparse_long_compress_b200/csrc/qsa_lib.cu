@@ -507,6 +507,36 @@ qsa_status score_select_impl(const char *name, const void *Q, const KcT *Kc, int
 }
 
 
+template <int G>
+qsa_status launch_prefill_agg(const void *Q, const void *Kc, float *scores, float *stats, int B, int Hq, int Hkv,
+                              int Tq, int q_pos0, int nblk, int NR, float sm_scale, int aggregator, cudaStream_t s)
+{
+    qsa_status st;
+    CUtensorMap mq, mk;
+    if ((st = make_map_2d(&mk, Kc, (uint64_t)B * Hkv * nblk, 128, 128)) != QSA_OK) return st;
+    if (aggregator == QSA_AGG_SOFTMAX_SUM) {
+        using S = qsa::SoftmaxStatsCfg<G>;
+        CUtensorMap mq1, mk1;
+        if ((st = make_map_q(&mq1, Q, (uint64_t)B * Tq, Hq, 128, G, S::TOKM)) != QSA_OK) return st;
+        if ((st = make_map_2d(&mk1, Kc, (uint64_t)B * Hkv * nblk, 128, 256)) != QSA_OK) return st;
+        if ((st = set_smem(qsa::block_softmax_stats_kernel<G>, S::SMEM_BYTES)) != QSA_OK) return st;
+        qsa::block_softmax_stats_kernel<G><<<dim3(NR * S::NMT, B * Hkv), S::THREADS, S::SMEM_BYTES, s>>>(
+            mq1, mk1, stats, Tq, q_pos0, nblk, Hkv, sm_scale);
+        if ((st = launched("block_softmax_stats_kernel")) != QSA_OK) return st;
+    }
+    using C = qsa::MaxScoreCfg<G>;
+    if ((st = make_map_q(&mq, Q, (uint64_t)B * Tq, Hq, 128, G, C::TOKN)) != QSA_OK) return st;
+    if (aggregator == QSA_AGG_SOFTMAX_SUM) {
+        if ((st = set_smem(qsa::block_max_scores_kernel<G, true>, C::SMEM_BYTES)) != QSA_OK) return st;
+        qsa::block_max_scores_kernel<G, true><<<dim3(NR, B * Hkv), C::THREADS, C::SMEM_BYTES, s>>>(
+            mq, mk, scores, Tq, q_pos0, nblk, Hkv, sm_scale, stats);
+    } else {
+        if ((st = set_smem(qsa::block_max_scores_kernel<G>, C::SMEM_BYTES)) != QSA_OK) return st;
+        qsa::block_max_scores_kernel<G><<<dim3(NR, B * Hkv), C::THREADS, C::SMEM_BYTES, s>>>(
+            mq, mk, scores, Tq, q_pos0, nblk, Hkv, sm_scale);
+    }
+    return launched("block_max_scores_kernel");
+}
 }  // namespace
 
 // ===================================================================== C ABI
@@ -615,22 +645,29 @@ qsa_status qsa_score_select_token_agg(const void *Q, const float *Kc, const int3
                                       seq_lens);
 }
 
-size_t qsa_score_select_prefill_max_workspace(int B, int Hq, int Hkv, int Tq, int q_pos0, int T_kv_max, int d,
-                                              int topk)
+size_t qsa_score_select_prefill_agg_workspace(int B, int Hq, int Hkv, int Tq, int q_pos0, int T_kv_max, int d,
+                                              int topk, int aggregator)
 {
-    (void)Hq;
     (void)topk;
-    if (B <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || T_kv_max <= 0 || T_kv_max % 64 || d != 128) return 0;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || T_kv_max <= 0 || T_kv_max % 64 || d != 128)
+        return 0;
     const SelectPlan p = plan_select(B, Hkv, Tq, q_pos0, 64, d);
-    return align256((size_t)B * Hkv * p.NR * (T_kv_max / 64) * sizeof(float)) + p.part_bytes;
+    const size_t rows = (size_t)B * Hkv * p.NR;
+    size_t bytes = align256(rows * (T_kv_max / 64) * sizeof(float)) + p.part_bytes;
+    if (aggregator == QSA_AGG_SOFTMAX_SUM) bytes += align256(rows * 64 * (Hq / Hkv) * 2 * sizeof(float));
+    return bytes;
 }
 
-qsa_status qsa_score_select_prefill_max(const void *Q, const void *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
-                                        int q_pos0, int T_kv_max, int d, int topk, float sm_scale, void *workspace,
-                                        size_t workspace_bytes, qsa_stream_t stream)
+
+qsa_status qsa_score_select_prefill_agg(const void *Q, const void *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
+                                        int q_pos0, int T_kv_max, int d, int topk, float sm_scale, int aggregator,
+                                        void *workspace, size_t workspace_bytes, qsa_stream_t stream)
 {
-    const char *name = "qsa_score_select_prefill_max";
+    const char *name = "qsa_score_select_prefill_agg";
     if (!Q || !Kc || !idx) return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (aggregator != QSA_AGG_MAX && aggregator != QSA_AGG_SOFTMAX_SUM)
+        return fail(aggregator == QSA_AGG_MEAN ? QSA_ERR_UNSUPPORTED : QSA_ERR_INVALID_ARG,
+                    "%s: aggregator=%d (the mean is qsa_score_select_bf16)", name, aggregator);
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || T_kv_max <= 0 || T_kv_max % 64 || Hq % Hkv ||
         q_pos0 % 64 || (long)q_pos0 + Tq > T_kv_max)
         return fail(QSA_ERR_INVALID_ARG, "%s: bad shape", name);
@@ -644,32 +681,22 @@ qsa_status qsa_score_select_prefill_max(const void *Q, const void *Kc, int32_t *
     if (!aligned16(Q) || !aligned16(Kc) || !aligned16(idx) || (workspace && !aligned16(workspace)))
         return fail(QSA_ERR_INVALID_ARG, "%s: misaligned pointer", name);
     const SelectPlan p = plan_select(B, Hkv, Tq, q_pos0, 64, d);
-    if (p.NR > 65535 || (long)B * Hkv > 65535) return fail(QSA_ERR_UNSUPPORTED, "%s: too many rows", name);
+    if ((long)p.NR * 4 > 65535 || (long)B * Hkv > 65535) return fail(QSA_ERR_UNSUPPORTED, "%s: too many rows", name);
     if (p.maxchunks * qsa::kMaxChosen * 8 > 200 * 1024) return fail(QSA_ERR_UNSUPPORTED, "%s: context too long", name);
-    const size_t score_bytes = align256((size_t)B * Hkv * p.NR * nblk * sizeof(float));
-    if (!workspace || workspace_bytes < score_bytes + p.part_bytes)
-        return fail(QSA_ERR_WORKSPACE, "%s: workspace needs %zu bytes", name, score_bytes + p.part_bytes);
+    const size_t rows = (size_t)B * Hkv * p.NR;
+    const size_t score_bytes = align256(rows * nblk * sizeof(float));
+    const size_t stat_bytes = aggregator == QSA_AGG_SOFTMAX_SUM ? align256(rows * 64 * G * 2 * sizeof(float)) : 0;
+    if (!workspace || workspace_bytes < score_bytes + stat_bytes + p.part_bytes)
+        return fail(QSA_ERR_WORKSPACE, "%s: workspace needs %zu bytes", name, score_bytes + stat_bytes + p.part_bytes);
     float *scores = static_cast<float *>(workspace);
-    uint64_t *part = reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(workspace) + score_bytes);
+    float *stats = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + score_bytes);
+    uint64_t *part = reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(workspace) + score_bytes + stat_bytes);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    qsa_status st;
-    CUtensorMap mq, mk;
-    if ((st = make_map_2d(&mk, Kc, (uint64_t)B * Hkv * nblk, 128, 128)) != QSA_OK) return st;
-    const dim3 grid(p.NR, B * Hkv);
-    if (G == 8) {
-        using C = qsa::MaxScoreCfg<8>;
-        if ((st = make_map_q(&mq, Q, (uint64_t)B * Tq, Hq, 128, 8, C::TOKN)) != QSA_OK) return st;
-        if ((st = set_smem(qsa::block_max_scores_kernel<8>, C::SMEM_BYTES)) != QSA_OK) return st;
-        qsa::block_max_scores_kernel<8><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, scores, Tq, q_pos0, nblk, Hkv,
-                                                                              sm_scale);
-    } else {
-        using C = qsa::MaxScoreCfg<4>;
-        if ((st = make_map_q(&mq, Q, (uint64_t)B * Tq, Hq, 128, 4, C::TOKN)) != QSA_OK) return st;
-        if ((st = set_smem(qsa::block_max_scores_kernel<4>, C::SMEM_BYTES)) != QSA_OK) return st;
-        qsa::block_max_scores_kernel<4><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, scores, Tq, q_pos0, nblk, Hkv,
-                                                                              sm_scale);
-    }
-    if ((st = launched("block_max_scores_kernel")) != QSA_OK) return st;
+    qsa_status st = G == 8 ? launch_prefill_agg<8>(Q, Kc, scores, stats, B, Hq, Hkv, Tq, q_pos0, nblk, p.NR, sm_scale,
+                                                   aggregator, s)
+                           : launch_prefill_agg<4>(Q, Kc, scores, stats, B, Hq, Hkv, Tq, q_pos0, nblk, p.NR, sm_scale,
+                                                   aggregator, s);
+    if (st != QSA_OK) return st;
     const dim3 sgrid(p.maxchunks, p.NR, B * Hkv), mgrid(p.NR, B * Hkv);
     auto skern = qsa::score_select_kernel<128, __nv_bfloat16, true>;
     if ((st = set_smem(skern, p.CH * 8)) != QSA_OK) return st;

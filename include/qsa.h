@@ -287,27 +287,33 @@ QSA_API qsa_status qsa_score_select_token_agg(const void *Q, const float *Kc, co
 
 /*
  * Selection for prefill rows (64-token query blocks) under the max-over-
- * tokens aggregator: s_j = max over the block's valid tokens t of the mean
- * over the group's heads h of sm_scale * <Q[b][t][h], Kc[b][g][j]>, then the
- * usual rule (sink and diagonal forced, top (topk - forced) of the
+ * tokens or the softmax-sum aggregator (QSA_AGG_MAX, QSA_AGG_SOFTMAX_SUM; the
+ * mean is qsa_score_select_bf16).  With z_{h,t}(j) = sm_scale *
+ * <Q[b][t][h], Kc[b][g][j]> over the group's heads h, the block's valid
+ * tokens t and the complete blocks j < D before the row's diagonal block D:
+ *   QSA_AGG_MAX          s_j = max over t of (mean over h of z_{h,t}(j))
+ *   QSA_AGG_SOFTMAX_SUM  s_j = sum over (h, t) of exp(z_{h,t}(j)) / sum over
+ *                        j' < D of exp(z_{h,t}(j'))
+ * then the usual rule (sink and diagonal forced, top (topk - forced) of the
  * candidates 1 .. D-1 by (s descending, index ascending), ascending, -1
  * padded).  The per-(head, token) logits are a dense contraction and run on
  * the tensor cores, so the summaries are the bf16 option's (Kc bf16
  * [B][Hkv][T_kv_max/64][128] from qsa_compress_keys_bf16: exact products,
  * fp32 sums).  Q bf16 [B][Tq][Hq][128] at positions q_pos0 .. q_pos0+Tq-1
  * (q_pos0 a multiple of 64); idx int32 [B][Hkv][ceil(Tq/64)][topk].  The
- * caller's workspace (16-byte aligned, qsa_score_select_prefill_max_workspace
- * bytes) holds the score table and the chunk lists.  Errors: null pointer,
- * bad shape or misaligned pointer -> QSA_ERR_INVALID_ARG; d != 128, Hq/Hkv
- * not 4 or 8, topk outside 2..64 or too large a problem ->
- * QSA_ERR_UNSUPPORTED; a short workspace -> QSA_ERR_WORKSPACE.
+ * caller's workspace (16-byte aligned, qsa_score_select_prefill_agg_workspace
+ * bytes) holds the score table, the softmax statistics and the chunk lists.
+ * Errors: null pointer, unknown aggregator, bad shape or misaligned pointer
+ * -> QSA_ERR_INVALID_ARG; the mean, d != 128, Hq/Hkv not 4 or 8, topk
+ * outside 2..64 or too large a problem -> QSA_ERR_UNSUPPORTED; a short
+ * workspace -> QSA_ERR_WORKSPACE.
  */
-QSA_API size_t qsa_score_select_prefill_max_workspace(int B, int Hq, int Hkv, int Tq, int q_pos0,
-                                                      int T_kv_max, int d, int topk);
-QSA_API qsa_status qsa_score_select_prefill_max(const void *Q, const void *Kc, int32_t *idx, int B, int Hq,
+QSA_API size_t qsa_score_select_prefill_agg_workspace(int B, int Hq, int Hkv, int Tq, int q_pos0,
+                                                      int T_kv_max, int d, int topk, int aggregator);
+QSA_API qsa_status qsa_score_select_prefill_agg(const void *Q, const void *Kc, int32_t *idx, int B, int Hq,
                                                 int Hkv, int Tq, int q_pos0, int T_kv_max, int d, int topk,
-                                                float sm_scale, void *workspace, size_t workspace_bytes,
-                                                qsa_stream_t stream);
+                                                float sm_scale, int aggregator, void *workspace,
+                                                size_t workspace_bytes, qsa_stream_t stream);
 
 /*
  * Quantized-KV option for decode (page "Qwen4 in llama.cpp: Dissecting PR

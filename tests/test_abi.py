@@ -105,13 +105,17 @@ def test_argument_checks_return_before_launch():
     assert ag(Hq=32, Hkv=2) == 2
     assert ag(agg=2, Tq=40, pos=4080) == 1   # queries past the summaries' capacity (64 blocks)
     # prefill rows, max aggregator: d must be 128, q_pos0 block aligned, a workspace
-    pm = lambda d=128, pos=0, ws=fake, wsb=1 << 30, Hq=16: lib.qsa_score_select_prefill_max(
-        fake, fake, fake, 1, Hq, 2, 128, pos, 1024, d, 16, 0.088, ws, wsb, None)
+    pm = lambda d=128, pos=0, ws=fake, wsb=1 << 30, Hq=16, agg=1: lib.qsa_score_select_prefill_agg(
+        fake, fake, fake, 1, Hq, 2, 128, pos, 1024, d, 16, 0.088, agg, ws, wsb, None)
     assert pm(d=64) == 2
     assert pm(pos=32) == 1
     assert pm(Hq=12) == 2
     assert pm(ws=None) == 6
-    assert lib.qsa_score_select_prefill_max_workspace(1, 16, 2, 128, 0, 1024, 128, 16) >= 2 * 2 * 16 * 4
+    assert pm(agg=0) == 2                  # the mean has its own entry
+    assert pm(agg=7) == 1
+    wmax = lib.qsa_score_select_prefill_agg_workspace(1, 16, 2, 128, 0, 1024, 128, 16, 1)
+    wsum = lib.qsa_score_select_prefill_agg_workspace(1, 16, 2, 128, 0, 1024, 128, 16, 2)
+    assert wmax >= 2 * 2 * 16 * 4 and wsum >= wmax + 2 * 2 * 64 * 8 * 2 * 4
     # self-test limit out of range
     assert lib.qsa_selftest_wait_timeout(0, None) == 1
 

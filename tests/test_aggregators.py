@@ -135,11 +135,12 @@ PREFILL_MAX = [
 ]
 
 
+@pytest.mark.parametrize("agg", ["max", "softmax_sum"])
 @pytest.mark.parametrize("name,B,Tq,q_pos0,Hq,Hkv,topk,frac", PREFILL_MAX, ids=[c[0] for c in PREFILL_MAX])
-def test_prefill_max_aggregator_parity(qsa, name, B, Tq, q_pos0, Hq, Hkv, topk, frac):
-    """Prefill rows under the max-over-tokens aggregator (tensor-core
-    logits over bf16 summaries) against the oracle's max aggregator on the
-    same bf16 summaries."""
+def test_prefill_aggregator_parity(qsa, agg, name, B, Tq, q_pos0, Hq, Hkv, topk, frac):
+    """Prefill rows under the max-over-tokens and softmax-sum aggregators
+    (tensor-core logits over bf16 summaries) against the oracle's
+    aggregators on the same bf16 summaries."""
     d = 128
     nblk = (q_pos0 + Tq + 63) // 64
     w = synthetic.custom(B=B, Tq=Tq, T_kv=64 * nblk, q_pos0=q_pos0, qblk=64, Hq=Hq, Hkv=Hkv, d=d, topk=topk,
@@ -149,17 +150,18 @@ def test_prefill_max_aggregator_parity(qsa, name, B, Tq, q_pos0, Hq, Hkv, topk, 
     Kc = torch.from_numpy(Kc_ref).to(torch.bfloat16).to(DEV)                   # exact
     NR = (Tq + 63) // 64
     idx = torch.full((B, Hkv, NR, topk), -7, dtype=torch.int32, device=DEV)
-    qsa.score_select_prefill_max(x["Q"].to(DEV), Kc, idx, topk, q_pos0, w.sm_scale)
+    qsa.score_select_prefill_agg(x["Q"].to(DEV), Kc, idx, topk, q_pos0, agg, w.sm_scale)
     _ok(qsa)
-    s = oracle.block_scores(x["Q"], Kc_ref, Tq, q_pos0, 64, w.sm_scale, "max")
+    s = oracle.block_scores(x["Q"], Kc_ref, Tq, q_pos0, 64, w.sm_scale, agg)
     sel = oracle.select_scores(s, B, Hkv, Tq, q_pos0, 64, topk)
     D = [(q_pos0 + min((i + 1) * 64, Tq) - 1) // 64 for b in range(B) for g in range(Hkv) for i in range(NR)]
     frac_checked, jac = check_selection(idx.cpu().numpy().reshape(-1, topk), sel, s.reshape(-1, s.shape[-1]), D,
                                         topk)
-    print(f"prefill max {name}: rows gap-checked {frac_checked:.3f}, Jaccard {jac:.4f}")
+    print(f"prefill {agg} {name}: rows gap-checked {frac_checked:.3f}, Jaccard {jac:.4f}")
 
 
-def test_prefill_max_aggregator_full_size(qsa):
+@pytest.mark.parametrize("agg", ["max", "softmax_sum"])
+def test_prefill_aggregator_full_size(qsa, agg):
     """prefill_32k (32768 tokens, top-16, bf16 summaries), sampled rows."""
     w = synthetic.CONFIGS["prefill_32k"]
     x = synthetic.generate(w, DEV)
@@ -168,14 +170,14 @@ def test_prefill_max_aggregator_full_size(qsa):
     qsa.compress_keys(x["K"], Kc, 0, (w.q_pos0 + w.Tq) // 64)
     NR = w.Tq // 64
     idx = torch.full((w.B, w.Hkv, NR, w.topk), -7, dtype=torch.int32, device=DEV)
-    qsa.score_select_prefill_max(x["Q"], Kc, idx, w.topk, w.q_pos0, w.sm_scale)
+    qsa.score_select_prefill_agg(x["Q"], Kc, idx, w.topk, w.q_pos0, agg, w.sm_scale)
     _ok(qsa)
     idx_h = idx.cpu().numpy().reshape(-1, w.topk)
     Q_h = x["Q"].cpu()
     Kc_h = Kc.float().cpu().double().numpy()
     rows = np.array([0, 1, 2, 63, 200, 255, 256, 400, 511, NR + 3, NR + 300, 2 * NR - 1], dtype=np.int32)
-    s = oracle.block_scores(Q_h, Kc_h, w.Tq, w.q_pos0, 64, w.sm_scale, "max", rows=rows)
+    s = oracle.block_scores(Q_h, Kc_h, w.Tq, w.q_pos0, 64, w.sm_scale, agg, rows=rows)
     sel = oracle.select_scores(s, w.B, w.Hkv, w.Tq, w.q_pos0, 64, w.topk, rows=rows)
     D = [(w.q_pos0 + min((r % NR + 1) * 64, w.Tq) - 1) // 64 for r in rows]
     frac_checked, jac = check_selection(idx_h[rows], sel, s, D, w.topk)
-    print(f"prefill_32k max: sampled rows gap-checked {frac_checked:.3f}, Jaccard {jac:.4f}")
+    print(f"prefill_32k {agg}: sampled rows gap-checked {frac_checked:.3f}, Jaccard {jac:.4f}")
