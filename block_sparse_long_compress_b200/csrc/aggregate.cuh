@@ -20,7 +20,9 @@
 // tiles: warp 0 loads the query block once and streams summary tiles
 // through a 2-stage ring (TMA, 128-byte swizzle), warp 1 issues the MMAs
 // (M = 128, N = 256, K = 128: 8 MMAs per N tile) into one of two TMEM
-// accumulators, warps 2-5 reduce the other.  Scores go to a table
+// accumulators, warps 2-5 reduce the other (for the softmax-sum warps 2-9:
+// two warps per TMEM lane quarter, each taking half of the columns; the
+// halves meet in shared memory once per candidate tile).  Scores go to a table
 // [B][Hkv][NR][nblk_max] (candidates 1 .. D-1 of each row); the chunked
 // selection turns the table into indices.
 //
@@ -51,7 +53,9 @@ struct MaxScoreCfg {
     static constexpr int KSTAGE_BYTES = 2 * KHALF_BYTES;
     static constexpr int NS = 2;
     static constexpr int SMEM_BYTES = Q_BYTES + NS * KSTAGE_BYTES + 1024;
-    static constexpr int THREADS = 192;                 // producer, issuer, 4 epilogue warps
+    // producer, issuer and 4 epilogue warps (max), or 8 (softmax-sum, whose
+    // per-column exponentials need the second warp per scheduler)
+    __host__ __device__ static constexpr int threads(bool softmax) { return 64 + 32 * (softmax ? 8 : 4); }
     static constexpr int TMEM_COLS = 2 * N;             // two fp32 accumulators
     static_assert(N % G == 0 && 64 % TOKN == 0, "tile shape");
 };
@@ -59,17 +63,21 @@ struct MaxScoreCfg {
 // SOFTMAX: the softmax-sum's second pass -- stats[(bg*NR + i)][64*G][2]
 // holds each (token, head) row's base-2 (max, sum) from the first pass.
 template <int G, bool SOFTMAX = false>
-__global__ void __launch_bounds__(MaxScoreCfg<G>::THREADS, 1) block_max_scores_kernel(
+__global__ void __launch_bounds__(MaxScoreCfg<G>::threads(SOFTMAX), 1) block_max_scores_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
     float *__restrict__ scores, int Tq, int q_pos0, int nblk_max, int Hkv, float sm_scale,
     const float *__restrict__ stats = nullptr)
 {
     using C = MaxScoreCfg<G>;
+    constexpr int THREADS = C::threads(SOFTMAX);
+    constexpr int EPI = (THREADS - 64) / 32;            // epilogue warps
+    constexpr int HALVES = EPI / 4;                     // column ranges per TMEM lane quarter (softmax: 2)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t q_full, k_full[C::NS], k_empty[C::NS], t_full[2], t_empty[2];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag, issued_k, issued_mma;
-    __shared__ float rstat[SOFTMAX ? 64 * G : 1][2];   // SOFTMAX: (max, 1/sum) per (token, head) row
+    __shared__ float rstat[SOFTMAX ? 64 * G : 1];   // SOFTMAX: max + log2(sum) per (token, head) row
+    __shared__ float xch[128];                      // the second column half's partial per candidate
 
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *q_smem = base;
@@ -97,7 +105,7 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::THREADS, 1) block_max_scores_k
 #pragma unroll
         for (int s = 0; s < 2; s++) {
             mbar_init(&t_full[s], 1);
-            mbar_init(&t_empty[s], 4);                  // one arrival per epilogue warp
+            mbar_init(&t_empty[s], EPI);                // one arrival per epilogue warp
         }
         fence_barrier_init();
     }
@@ -106,11 +114,10 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::THREADS, 1) block_max_scores_k
         tmem_relinquish();
     }
     if constexpr (SOFTMAX) {
+        // 2^(z - max) / sum = 2^(z - (max + log2 sum))
         const float *st = stats + ((long)bg * NR + i) * (64 * G) * 2;
-        for (int r = threadIdx.x; r < 64 * G; r += C::THREADS) {
-            rstat[r][0] = st[2 * r];
-            rstat[r][1] = st[2 * r + 1] > 0.f ? 1.f / st[2 * r + 1] : 0.f;
-        }
+        for (int r = threadIdx.x; r < 64 * G; r += THREADS)
+            rstat[r] = st[2 * r + 1] > 0.f ? st[2 * r] + __log2f(st[2 * r + 1]) : INFINITY;
     }
     tc_fence_before();
     __syncthreads();
@@ -173,6 +180,7 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::THREADS, 1) block_max_scores_k
         }
         if (lane == 0) issued_mma = w;
     } else {
+      if constexpr (!SOFTMAX) {
         // ------------------------------------------- epilogue (warps 2-5)
         const int quarter = warp & 3;                  // the TMEM lanes this warp may access
         const int m = 32 * quarter + lane;             // candidate within the tile
@@ -191,23 +199,10 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::THREADS, 1) block_max_scores_k
 #pragma unroll
                 for (int tt = 0; tt < 32 / G; tt++) {
                     const int t = i * 64 + nt * C::TOKN + c / G + tt;   // token of these G columns
-                    if constexpr (SOFTMAX) {
-                        // best accumulates the rows' shares of this block
-                        const int r0 = (nt * C::TOKN + c / G + tt) * G;  // (token, head) row in the block
-                        const float sc2 = sm_scale * 1.4426950408889634f;
-                        if (t < Tq) {
-                            if (best == -INFINITY) best = 0.f;
+                    float sum = 0.f;
 #pragma unroll
-                            for (int h = 0; h < G; h++)
-                                best += fast_exp2(__uint_as_float(r[tt * G + h]) * sc2 - rstat[r0 + h][0]) *
-                                        rstat[r0 + h][1];
-                        }
-                    } else {
-                        float sum = 0.f;
-#pragma unroll
-                        for (int h = 0; h < G; h++) sum += __uint_as_float(r[tt * G + h]);
-                        if (t < Tq) best = fmaxf(best, sum);
-                    }
+                    for (int h = 0; h < G; h++) sum += __uint_as_float(r[tt * G + h]);
+                    if (t < Tq) best = fmaxf(best, sum);
                 }
             }
             tc_fence_before();
@@ -215,12 +210,56 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::THREADS, 1) block_max_scores_k
             if (lane == 0) mbar_arrive(&t_empty[buf]);
             if (nt == C::NT - 1) {
                 const int j = 1 + C::M * k + m;
-                if (j < Dg)
-                    scores[((long)bg * NR + i) * nblk_max + j] =
-                        SOFTMAX ? best : best * (1.0f / (float)G) * sm_scale;
+                if (j < Dg) scores[((long)bg * NR + i) * nblk_max + j] = best * (1.0f / (float)G) * sm_scale;
                 best = -INFINITY;
             }
         }
+      } else {
+        // ------------------------------------------- epilogue (warps 2-9)
+        const int quarter = warp & 3;                  // the TMEM lanes this warp may access
+        const int half = (warp - 2) >> 2;              // the columns it reduces (HALVES ranges)
+        const int m = 32 * quarter + lane;             // candidate within the tile
+        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+        const float sc2 = sm_scale * 1.4426950408889634f;
+        float best = 0.f;
+        for (int w = 0; w < nwork; w++) {
+            const int k = w / C::NT, nt = w % C::NT, buf = w & 1;
+            // warp-uniform: the TMEM loads below are collective.  A failed
+            // wait (an abort, after which every wait returns at once) skips
+            // the work but not the exchanges below: all eight warps must
+            // reach the same named barriers
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&t_full[buf], (w >> 1) & 1, abort, 74));
+            if (ok) tc_fence_after();
+#pragma unroll 1
+            for (int c = half * (C::N / HALVES); ok && c < (half + 1) * (C::N / HALVES); c += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_base + buf * C::N + c, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int tt = 0; tt < 32 / G; tt++) {
+                    const int tl = nt * C::TOKN + c / G + tt;    // token of these G columns, in the block
+                    if (i * 64 + tl < Tq) {
+                        // the rows' shares of this block
+#pragma unroll
+                        for (int h = 0; h < G; h++)
+                            best += fast_exp2(__uint_as_float(r[tt * G + h]) * sc2 - rstat[tl * G + h]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&t_empty[buf]);
+            if (nt == C::NT - 1) {
+                // the two column halves of each candidate meet
+                if (half == 1) xch[m] = best;
+                named_barrier_sync(1, 32 * EPI);
+                const int j = 1 + C::M * k + m;
+                if (half == 0 && j < Dg) scores[((long)bg * NR + i) * nblk_max + j] = best + xch[m];
+                named_barrier_sync(1, 32 * EPI);
+                best = 0.f;
+            }
+        }
+      }
     }
 
     tc_fence_before();
@@ -263,7 +302,7 @@ struct SoftmaxStatsCfg {
     static constexpr int KSTAGE_BYTES = 2 * KHALF_BYTES;
     static constexpr int NS = 2;
     static constexpr int SMEM_BYTES = Q_BYTES + NS * KSTAGE_BYTES + 1024;
-    static constexpr int THREADS = 192;
+    static constexpr int THREADS = 320;                 // producer, issuer, 8 epilogue warps
     static constexpr int TMEM_COLS = 2 * N;
 };
 
@@ -301,7 +340,7 @@ __global__ void __launch_bounds__(SoftmaxStatsCfg<G>::THREADS, 1) block_softmax_
 #pragma unroll
         for (int s = 0; s < 2; s++) {
             mbar_init(&t_full[s], 1);
-            mbar_init(&t_empty[s], 4);
+            mbar_init(&t_empty[s], 8);
         }
         fence_barrier_init();
     }
@@ -364,6 +403,7 @@ __global__ void __launch_bounds__(SoftmaxStatsCfg<G>::THREADS, 1) block_softmax_
         if (lane == 0) issued_mma = k;
     } else {
         const int quarter = warp & 3;
+        const int half = (warp - 2) >> 2;              // the half of each tile's blocks it takes
         const int r = 32 * quarter + lane;             // (token, head) row of the M tile
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
         const float sc2 = sm_scale * 1.4426950408889634f;
@@ -374,21 +414,31 @@ __global__ void __launch_bounds__(SoftmaxStatsCfg<G>::THREADS, 1) block_softmax_
             if (!__all_sync(0xffffffffu, mbar_wait(&t_full[buf], (k >> 1) & 1, abort, 84))) break;
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < C::N; c += 32) {
+            for (int c = half * (C::N / 2); c < (half + 1) * (C::N / 2); c += 32) {
+                const int j0 = C::N * k + c;            // block of column 0 of this chunk (uniform)
+                if (j0 >= Dg) break;
                 uint32_t v[32];
                 tmem_ld32(tmem + lane_base + buf * C::N + c, v);
                 tmem_wait_ld();
-                const int j0 = C::N * k + c;            // block of column 0 of this chunk
+                float x[32];
                 float mx = -INFINITY;
+                if (j0 + 32 <= Dg) {
 #pragma unroll
-                for (int e = 0; e < 32; e++)
-                    if (j0 + e < Dg) mx = fmaxf(mx, __uint_as_float(v[e]) * sc2);
-                if (mx == -INFINITY) continue;
+                    for (int e = 0; e < 32; e++) {
+                        x[e] = __uint_as_float(v[e]) * sc2;
+                        mx = fmaxf(mx, x[e]);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; e++) {
+                        x[e] = j0 + e < Dg ? __uint_as_float(v[e]) * sc2 : -INFINITY;
+                        mx = fmaxf(mx, x[e]);
+                    }
+                }
                 const float mn = fmaxf(m_run, mx);
                 float acc = 0.f;
 #pragma unroll
-                for (int e = 0; e < 32; e++)
-                    if (j0 + e < Dg) acc += fast_exp2(__uint_as_float(v[e]) * sc2 - mn);
+                for (int e = 0; e < 32; e++) acc += fast_exp2(x[e] - mn);
                 s_run = s_run * fast_exp2(m_run - mn) + acc;
                 m_run = mn;
             }
@@ -396,10 +446,18 @@ __global__ void __launch_bounds__(SoftmaxStatsCfg<G>::THREADS, 1) block_softmax_
             __syncwarp();
             if (lane == 0) mbar_arrive(&t_empty[buf]);
         }
-        if (k == ntiles) {
+        // the two halves of each row meet (this exchange reuses no ring
+        // memory: a small array of its own)
+        __shared__ float xm[128], xs[128];
+        if (half == 1) xm[r] = m_run, xs[r] = s_run;
+        named_barrier_sync(1, 256);
+        if (half == 0 && k == ntiles) {
+            float m2 = xm[r], s2 = xs[r];
+            const float mn = fmaxf(m_run, m2);
+            const float sum = mn == -INFINITY ? 0.f : s_run * fast_exp2(m_run - mn) + s2 * fast_exp2(m2 - mn);
             float *out = stats + (((long)bg * NR + i) * (64 * G) + mt * C::M + r) * 2;
-            out[0] = m_run;
-            out[1] = s_run;
+            out[0] = mn;
+            out[1] = sum;
         }
     }
 
