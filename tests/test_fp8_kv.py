@@ -113,3 +113,32 @@ def test_decode_fp8_paged_parity(qsa):
     qsa.decode_fp8_paged(q, kc, ks, vc, vs, bad, seq_lens, idx, o, sm)
     assert qsa.device_status()[0] == "QSA_ERR_BOUNDS"
     assert qsa.device_status()[0] == "QSA_OK"
+
+
+def test_decode_fp8_full_size(qsa):
+    """decode_128k over the rotated fp8 cache, in the benchmark's launch
+    configuration (32 sequences at 131072 tokens, top-64, bf16 summaries of
+    the unrotated keys), sampled sequences against the oracle's fp8 decode
+    with the GPU's indices."""
+    w = synthetic.CONFIGS["decode_128k"]
+    x = synthetic.generate(w, DEV)
+    L = w.q_pos0 + 1
+    q = x["Q"].view(w.B, w.Hq, w.d)
+    dec = qsa.QSADecode(w.B, w.Hq, w.Hkv, w.d, w.T_kv, w.topk, device=DEV, summary_dtype=torch.bfloat16)
+    dec.compress(x["K"], 0, L // 64)
+    qsa.score_select(q.view(w.B, 1, w.Hq, w.d), dec.Kc, dec.idx, w.topk, L - 1, 1, dec.sm_scale)
+    kc, ks = qsa.quantize_kv_fp8(x["K"])
+    vc, vs = qsa.quantize_kv_fp8(x["V"])
+    o = torch.full_like(q, float("nan"))
+    qsa.decode_fp8(q, kc, ks, vc, vs, dec.idx, o, L, w.sm_scale)
+    st = qsa.device_status()
+    assert st[0] == "QSA_OK", st
+    idx_h, o_h = dec.idx.cpu().numpy(), o.float().cpu().numpy()
+    for b in (0, 17, w.B - 1):
+        # the oracle quantizes this sequence's rows itself (codes are a
+        # per-row function of the row)
+        ck, sk = oracle.quantize_kv_fp8(x["K"][b:b + 1].cpu())
+        cv, sv = oracle.quantize_kv_fp8(x["V"][b:b + 1].cpu())
+        ref = oracle.decode_fp8(q[b:b + 1].cpu(), ck, sk, cv, sv, idx_h[b:b + 1], L, w.sm_scale)
+        mx, mean = check_out(o_h[b], ref[0])
+        print(f"decode_128k fp8 seq {b}: o max {mx:.2e} mean {mean:.2e}")
