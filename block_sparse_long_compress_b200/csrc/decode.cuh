@@ -37,8 +37,8 @@
 
 namespace qsa {
 
-// FP8: the rotated fp8 cache option (quant.cuh): a stage holds a block's K
-// and V codes (one 64 x 128-byte box each) and their per-row scales; every
+// FP8: the rotated fp8 cache option (quant.cuh): a stage holds two blocks'
+// K and V codes (one 64 x 128-byte box each) and per-row scales; every
 // consumer thread loads the codes of its MMA fragments straight from the
 // stage and expands them to f16 in registers.
 template <int D, bool FP8 = false>
@@ -47,9 +47,13 @@ struct DecodeCfg {
     static constexpr int HALF_BYTES = 64 * 128;        // one 64-row x 128-byte box
     static constexpr int KV_BYTES = FP8 ? 64 * D : 64 * D * 2;   // one block's K (or V)
     static constexpr int SCALE_BYTES = FP8 ? 64 * 4 : 0;         // its per-row scales
-    static constexpr int STAGE_BYTES = FP8 ? (2 * KV_BYTES + 2 * SCALE_BYTES + 1023) / 1024 * 1024 : 2 * KV_BYTES;
+    // FP8: a stage holds two blocks (codes and scales of each, 1024-aligned),
+    // so that one full/empty round trip moves as many bytes as a bf16 block
+    static constexpr int BLK_BYTES = FP8 ? (2 * KV_BYTES + 2 * SCALE_BYTES + 1023) / 1024 * 1024 : 2 * KV_BYTES;
+    static constexpr int BPS = FP8 ? 2 : 1;            // blocks per stage
+    static constexpr int STAGE_BYTES = BPS * BLK_BYTES;
     static constexpr int CTAS_PER_SM = 2;
-    static constexpr int RING_BYTES = FP8 ? 6 * STAGE_BYTES : 96 * 1024;   // NS stages; two CTAs per SM
+    static constexpr int RING_BYTES = FP8 ? 3 * STAGE_BYTES : 96 * 1024;   // NS stages; two CTAs per SM
     static constexpr int NS = RING_BYTES / STAGE_BYTES;
     static constexpr int NC = 4;                       // consumer warps
     static constexpr int THREADS = (NC + 1) * 32;
@@ -260,25 +264,33 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
     if (warp == NC) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
+            // slot i holds blocks BPS*i .. BPS*i + BPS - 1 (fewer at the end)
+            const int nslots = (nb + C::BPS - 1) / C::BPS;
             int i = 0;
-            for (; i < nb; i++) {
+            for (; i < nslots; i++) {
                 const int st = i % NS;
                 if (i >= NS) {
                     if (!mbar_wait(&empty[st], ((i / NS) - 1) & 1, &abort_flag, 42)) break;
                     fence_proxy_async_smem();
                 }
-                const int row = rows[i];
                 uint8_t *ks = ring + st * C::STAGE_BYTES;
                 uint8_t *vs = ks + C::KV_BYTES;
                 if constexpr (FP8) {
-                    // codes: one 64-row x 128-byte box each; scales: 64 fp32
-                    // per tensor, one plain bulk copy each
-                    mbar_arrive_expect_tx(&full[st], 2 * C::KV_BYTES + 2 * C::SCALE_BYTES);
-                    tma_load_2d(ks, &tmK, &full[st], 0, row);
-                    tma_load_2d(vs, &tmV, &full[st], 0, row);
-                    bulk_load(vs + C::KV_BYTES, k_scales + row, C::SCALE_BYTES, &full[st]);
-                    bulk_load(vs + C::KV_BYTES + C::SCALE_BYTES, v_scales + row, C::SCALE_BYTES, &full[st]);
+                    // per block: codes, one 64-row x 128-byte box each; scales,
+                    // 64 fp32 per tensor, one plain bulk copy each
+                    const int nbk = min(C::BPS, nb - C::BPS * i);
+                    mbar_arrive_expect_tx(&full[st], nbk * (2 * C::KV_BYTES + 2 * C::SCALE_BYTES));
+                    for (int h = 0; h < nbk; h++) {
+                        const int row = rows[C::BPS * i + h];
+                        uint8_t *kb = ks + h * C::BLK_BYTES;
+                        uint8_t *vb = kb + C::KV_BYTES;
+                        tma_load_2d(kb, &tmK, &full[st], 0, row);
+                        tma_load_2d(vb, &tmV, &full[st], 0, row);
+                        bulk_load(vb + C::KV_BYTES, k_scales + row, C::SCALE_BYTES, &full[st]);
+                        bulk_load(vb + C::KV_BYTES + C::SCALE_BYTES, v_scales + row, C::SCALE_BYTES, &full[st]);
+                    }
                 } else {
+                    const int row = rows[i];
                     mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
 #pragma unroll
                     for (int h = 0; h < C::NH; h++)
@@ -338,8 +350,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
             // k0 + {2c, 2c+1, 2c+8, 2c+9}, bytes 16r .. 16r+15; and the
             // per-row scales (scores: (u_q . u_k) / 128 = q . k with
             // u_k = scale * code; the V scale rides on P)
-            auto load = [&](int st, uint4 (&kr)[4], uint4 (&vr)[4], float (&kq)[2], float (&vp)[2]) {
-                const uint8_t *kst = ring + st * C::STAGE_BYTES;
+            auto load = [&](const uint8_t *kst, uint4 (&kr)[4], uint4 (&vr)[4], float (&kq)[2], float (&vp)[2]) {
                 const uint8_t *vst = kst + C::KV_BYTES;
                 const float *ksc = reinterpret_cast<const float *>(vst + C::KV_BYTES);
                 const float *vsc = ksc + 64;
@@ -392,20 +403,18 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
                     mma_f16_16816(oacc[mt], e4m3_lo(pa), e4m3_hi(pa), e4m3_lo(pc), e4m3_hi(pc), pb0, pb1);
                 }
             };
+            static_assert(!FP8 || C::BPS == 2, "a stage holds the pair");
             for (int i = 0; i < nb; i += 2) {
                 const bool two = i + 1 < nb;   // warp-uniform
-                const int sa = i % NS, sb = (i + 1) % NS;
-                if (!mbar_wait(&full[sa], (i / NS) & 1, &abort_flag, 40)) break;
-                if (two && !mbar_wait(&full[sb], ((i + 1) / NS) & 1, &abort_flag, 40)) break;
+                const int slot = i / 2, st = slot % NS;
+                if (!mbar_wait(&full[st], (slot / NS) & 1, &abort_flag, 40)) break;
+                const uint8_t *stage = ring + st * C::STAGE_BYTES;
                 uint4 kra[4], vra[4], krb[4], vrb[4];
                 float kqa[2], vpa[2], kqb[2] = {0.f, 0.f}, vpb[2] = {0.f, 0.f};
-                load(sa, kra, vra, kqa, vpa);
-                if (two) load(sb, krb, vrb, kqb, vpb);
+                load(stage, kra, vra, kqa, vpa);
+                if (two) load(stage + C::BLK_BYTES, krb, vrb, kqb, vpb);
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&empty[sa]);
-                    if (two) mbar_arrive(&empty[sb]);
-                }
+                if (lane == 0) mbar_arrive(&empty[st]);
                 float xa[4] = {0.f, 0.f, 0.f, 0.f}, xb[4] = {0.f, 0.f, 0.f, 0.f};
                 scores(kra, xa);
                 if (two) scores(krb, xb);
