@@ -272,6 +272,8 @@ def score_select_token_agg(q, Kc, idx, topk, q_pos0, aggregator="mean", sm_scale
     q: bf16 [B, Tq, Hq, d] at positions q_pos0 .. q_pos0 + Tq - 1, or with
     seq_lens (int32 [B], Tq = 1) at seq_lens[b] - 1 (q_pos0 = the largest);
     Kc fp32 [B, Hkv, max_blocks, d]; idx int32 [B, Hkv, Tq, topk] (written)."""
+    if aggregator not in AGGREGATORS:
+        raise ValueError(f"aggregator must be one of {sorted(AGGREGATORS)}, got {aggregator!r}")
     B, Tq, Hq, d = q.shape
     _, Hkv, max_blocks, _ = Kc.shape
     if sm_scale is None:
@@ -295,6 +297,9 @@ def score_select_prefill_agg(Q, Kc, idx, topk, q_pos0, aggregator="max", sm_scal
     softmax-sum aggregator (per-(head, token) logits on the tensor cores).
     Q bf16 [B, Tq, Hq, 128]; Kc bf16 summaries [B, Hkv, T_kv_max//64, 128];
     idx int32 [B, Hkv, ceil(Tq/64), topk] (written)."""
+    if aggregator not in ("max", "softmax_sum"):
+        raise ValueError(f"prefill rows take the 'max' or 'softmax_sum' aggregator, got {aggregator!r} "
+                         "(the mean is score_select over bf16 summaries)")
     B, Tq, Hq, d = Q.shape
     _, Hkv, nblk, _ = Kc.shape
     if sm_scale is None:

@@ -20,9 +20,11 @@
 //                   movmatrix, O^T += V^T P^T (d on M, V^T by
 //                   ldmatrix.trans).  No padding rows: 16 MMAs per warp and
 //                   block.
-// The P x 4 warp partials (max, sum, O) of the row are merged in one pass
-// through distributed shared memory, each CTA finishing 1/P of the row's
-// outputs.  No global workspace, no global atomics.
+// The row's partials merge through distributed shared memory: each CTA
+// combines its 4 warps' (max, sum, O) per head, then pushes the result into
+// the inbox of the CTA that finishes that head (head h -> CTA h mod P) with
+// plain remote stores between two cluster barriers; each owner merges its
+// inbox locally.  No global workspace, no global atomics, no remote loads.
 //
 // Caches are either contiguous ([B][Hkv][T_kv_max][d]; one length L for all
 // sequences) or paged for serving: every sequence has its own length

@@ -6,6 +6,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import block_sparse_long_compress_b200 as qsa
 
@@ -148,3 +149,28 @@ def test_build_refuses_a_prefill_kernel_below_its_register_split():
     build._check_registers(ok)
     with pytest.raises(RuntimeError):
         build._check_registers(ok.replace(f"Used {build.PREFILL_LAUNCH_REGS}", "Used 160"))
+
+
+def test_binding_refuses_host_tensors_and_wrong_types():
+    """The Python wrappers check device, dtype and shape before any call into
+    the library (no GPU needed to see them refuse)."""
+    bf = torch.bfloat16
+    with pytest.raises(ValueError):
+        qsa.quantize_kv_fp8(torch.zeros((2, 64), dtype=bf))            # rows must be 128 wide
+    with pytest.raises(TypeError):
+        qsa.quantize_kv_fp8(torch.zeros((2, 128), dtype=bf))           # a host tensor
+    q = torch.zeros((1, 8, 128), dtype=bf)
+    codes = torch.zeros((1, 2, 64, 128), dtype=torch.uint8)
+    scales = torch.zeros((1, 2, 64), dtype=torch.float32)
+    idx = torch.zeros((1, 2, 1, 4), dtype=torch.int32)
+    with pytest.raises(TypeError):
+        qsa.decode_fp8(q, codes, scales, codes, scales, idx, q.clone(), 64)
+    with pytest.raises(ValueError):
+        qsa.score_select_token_agg(torch.zeros((1, 1, 8, 128), dtype=bf), torch.zeros((1, 2, 4, 128)),
+                                   idx, 4, 100, "median")
+    with pytest.raises(ValueError):
+        qsa.score_select_prefill_agg(torch.zeros((1, 64, 8, 128), dtype=bf), torch.zeros((1, 2, 4, 128)),
+                                     torch.zeros((1, 2, 1, 4), dtype=torch.int32), 4, 0, "mean")
+    with pytest.raises(TypeError):
+        qsa.score_select_prefill_agg(torch.zeros((1, 64, 8, 128), dtype=bf), torch.zeros((1, 2, 4, 128)),
+                                     torch.zeros((1, 2, 1, 4), dtype=torch.int32), 4, 0, "max")
