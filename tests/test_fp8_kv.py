@@ -139,6 +139,9 @@ def test_decode_fp8_full_size(qsa):
         # per-row function of the row)
         ck, sk = oracle.quantize_kv_fp8(x["K"][b:b + 1].cpu())
         cv, sv = oracle.quantize_kv_fp8(x["V"][b:b + 1].cpu())
+        # the codes and scales of the whole sequence, bit for bit
+        assert np.array_equal(kc[b:b + 1].cpu().numpy(), ck) and np.array_equal(ks[b:b + 1].cpu().numpy(), sk)
+        assert np.array_equal(vc[b:b + 1].cpu().numpy(), cv) and np.array_equal(vs[b:b + 1].cpu().numpy(), sv)
         ref = oracle.decode_fp8(q[b:b + 1].cpu(), ck, sk, cv, sv, idx_h[b:b + 1], L, w.sm_scale)
         mx, mean = check_out(o_h[b], ref[0])
         print(f"decode_128k fp8 seq {b}: o max {mx:.2e} mean {mean:.2e}")
