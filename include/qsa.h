@@ -32,6 +32,15 @@
  * 16-byte aligned; T_kv_max a multiple of 64.  Anything else returns
  * QSA_ERR_UNSUPPORTED (or QSA_ERR_INVALID_ARG for malformed arguments).
  *
+ * Beyond the hot path the header declares, each with its own layouts:
+ * bf16 summaries (qsa_*_bf16), ragged batches over paged caches
+ * (qsa_*_paged, qsa_score_select_ragged*), the Walsh-Hadamard-rotated fp8
+ * cache for decode (qsa_quantize_kv_fp8, qsa_decode_fp8*), and the selection
+ * variants with other aggregators of the row's tokens and heads
+ * (qsa_score_select_token_agg, qsa_score_select_prefill_agg).  Some of them
+ * narrow the supported set (d = 128 only for the fp8 cache and the
+ * prefill-row aggregators).
+ *
  * Ownership and errors: the caller owns every buffer, including the
  * workspace; the library allocates no device memory.  All calls are
  * asynchronous on `stream` (0 = legacy default stream).  Argument checks run
