@@ -181,3 +181,34 @@ def test_prefill_aggregator_full_size(qsa, agg):
     D = [(w.q_pos0 + min((r % NR + 1) * 64, w.Tq) - 1) // 64 for r in rows]
     frac_checked, jac = check_selection(idx_h[rows], sel, s, D, w.topk)
     print(f"prefill_32k {agg}: sampled rows gap-checked {frac_checked:.3f}, Jaccard {jac:.4f}")
+
+
+@pytest.mark.parametrize("agg", ["max", "softmax_sum"])
+def test_aggregators_degenerate_rows(qsa, agg):
+    """Rows with no candidate (diagonal block 0 or 1) keep only the forced
+    blocks; the rows right after them have one or two candidates."""
+    d, Hq, Hkv, topk = 128, 16, 2, 8
+    # prefill rows from the first block of the sequence (diagonals 0, 1, 2, 3)
+    w = synthetic.custom(B=1, Tq=200, T_kv=256, q_pos0=0, qblk=64, Hq=Hq, Hkv=Hkv, d=d, topk=topk, seed=241)
+    x = synthetic.generate(w)
+    Kc_ref = oracle.compress_keys(x["K"], 0, 4, summary="bf16")
+    idx = torch.full((1, Hkv, 4, topk), -7, dtype=torch.int32, device=DEV)
+    qsa.score_select_prefill_agg(x["Q"].to(DEV), torch.from_numpy(Kc_ref).to(torch.bfloat16).to(DEV), idx, topk, 0,
+                                 agg, w.sm_scale)
+    _ok(qsa)
+    s = oracle.block_scores(x["Q"], Kc_ref, 200, 0, 64, w.sm_scale, agg)
+    ref = oracle.select_scores(s, 1, Hkv, 200, 0, 64, topk)["idx"].reshape(idx.shape)
+    assert np.array_equal(idx.cpu().numpy(), ref)
+    assert idx[0, 0, 0].tolist() == [0] + [-1] * (topk - 1)          # diagonal 0: the sink alone
+    assert idx[0, 0, 1].tolist() == [0, 1] + [-1] * (topk - 2)       # diagonal 1: sink and diagonal
+    # per-token rows at positions in blocks 0, 1 and 2
+    for pos in (3, 70, 130):
+        wt = synthetic.custom(B=2, Tq=1, T_kv=256, q_pos0=pos, qblk=1, Hq=Hq, Hkv=Hkv, d=d, topk=topk, seed=242)
+        xt = synthetic.generate(wt)
+        Kc = oracle.compress_keys(xt["K"], 0, 4).astype(np.float32)
+        it = torch.full((2, Hkv, 1, topk), -7, dtype=torch.int32, device=DEV)
+        qsa.score_select_token_agg(xt["Q"].to(DEV), torch.from_numpy(Kc).to(DEV), it, topk, pos, agg, wt.sm_scale)
+        _ok(qsa)
+        st = oracle.block_scores(xt["Q"], Kc.astype(np.float64), 1, pos, 1, wt.sm_scale, agg)
+        rt = oracle.select_scores(st, 2, Hkv, 1, pos, 1, topk)["idx"].reshape(it.shape)
+        assert np.array_equal(it.cpu().numpy(), rt)

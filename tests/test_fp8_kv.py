@@ -145,3 +145,34 @@ def test_decode_fp8_full_size(qsa):
         ref = oracle.decode_fp8(q[b:b + 1].cpu(), ck, sk, cv, sv, idx_h[b:b + 1], L, w.sm_scale)
         mx, mean = check_out(o_h[b], ref[0])
         print(f"decode_128k fp8 seq {b}: o max {mx:.2e} mean {mean:.2e}")
+
+
+@pytest.mark.parametrize("L", [1, 2, 65, 130])
+def test_decode_fp8_short_caches(qsa, L):
+    """Caches of one token, of a partial first block, and of a few blocks:
+    the diagonal block's causal limit and the sink alone.  With one visible
+    key the output is that key's value row, of magnitude 1 for N(0, 1)
+    values, where the bf16 output's own rounding is already about 1e-3 on
+    average; the values are scaled by 1/4 (exact in bf16) so that the
+    standard tolerance measures the kernel, as it does for averaged rows."""
+    w = synthetic.custom(B=2, Tq=1, T_kv=256, q_pos0=L - 1, qblk=1, Hq=16, Hkv=2, d=128, topk=4, seed=251)
+    x = synthetic.generate(w)
+    x["V"] = x["V"] * 0.25
+    D = (L - 1) // 64
+    idx_np = np.full((2, 2, 1, 4), -1, dtype=np.int32)
+    for b in range(2):
+        for g in range(2):
+            blocks = sorted(set([0, D]))
+            idx_np[b, g, 0, :len(blocks)] = blocks
+    idx = torch.from_numpy(idx_np).to(DEV)
+    q = x["Q"].to(DEV).view(2, 16, 128)
+    kc, ks = qsa.quantize_kv_fp8(x["K"].to(DEV))
+    vc, vs = qsa.quantize_kv_fp8(x["V"].to(DEV))
+    o = torch.full_like(q, float("nan"))
+    qsa.decode_fp8(q, kc, ks, vc, vs, idx, o, L, w.sm_scale)
+    st = qsa.device_status()
+    assert st[0] == "QSA_OK", st
+    ck, sk = oracle.quantize_kv_fp8(x["K"])
+    cv, sv = oracle.quantize_kv_fp8(x["V"])
+    ref = oracle.decode_fp8(x["Q"].view(2, 16, 128), ck, sk, cv, sv, idx_np, L, w.sm_scale)
+    check_out(o.float().cpu().numpy(), ref)
