@@ -76,14 +76,15 @@ def test_decode_fp8_parity(qsa, name, kw):
     print(f"{name}: o max {mx:.2e} mean {mean:.2e}; quantization vs bf16 cache: max {qerr:.2e}")
 
 
-def test_decode_fp8_paged_parity(qsa):
+@pytest.mark.parametrize("Hq", [16, 8], ids=["g8", "g4"])
+def test_decode_fp8_paged_parity(qsa, Hq):
     """A ragged batch over paged rotated fp8 caches: the pages' rows are
     quantized like any rows, each sequence is checked against the oracle's
     fp8 decode on its own logical cache; a page outside the pool is caught
     on the device."""
     from tests.test_paged import build_paged
     lens = [64 * 150 - 5, 64 * 300, 64 * 77 + 31, 1000, 64 * 41 + 1]
-    Hq, Hkv, d, topk = 16, 2, 128, 16
+    Hkv, d, topk = 2, 128, 16
     p = build_paged(lens, Hq, Hkv, d, seed=171)
     B, max_blocks = p["B"], p["max_blocks"]
     sm = d ** -0.5
