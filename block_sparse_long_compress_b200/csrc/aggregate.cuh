@@ -1,6 +1,7 @@
-// Step 3 for prefill rows under the max-over-tokens aggregator: the score of
-// candidate block j for query block i is the largest, over the block's
-// tokens t, of the group's head mean of sm_scale <q_{h,t}, Kc_j>.  The pages
+// Step 3 for prefill rows under the max-over-tokens and softmax-sum
+// aggregators.  Max: the score of candidate block j for query block i is
+// the largest, over the block's tokens t, of the group's head mean of
+// sm_scale <q_{h,t}, Kc_j>.  The pages
 // have the selector score compressed keys against the queries (page "Qwen4
 // in llama.cpp: Dissecting PR #27742", section "QSA Is an Address-Selection
 // Problem, Not a New Attention Equation") and leave the combination of the
@@ -8,7 +9,8 @@
 //
 // Unlike the pooled-query score (one dot per block and row), this needs
 // every (head, token) logit: 64 x G rows against every candidate, a dense
-// contraction (0.55 TFLOP over prefill_128k's rows), so it runs on the
+// contraction (0.55 TFLOP over the rows of a 131072-token prefill with 16
+// query heads), so it runs on the
 // tensor cores.  The summaries are the bf16 option's (exact bf16 products,
 // fp32 accumulation in TMEM).  The candidates sit on the MMA's M side (128
 // per tile, one TMEM lane each) and the query rows (token, head) on N, so
