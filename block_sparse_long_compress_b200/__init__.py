@@ -26,6 +26,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqsa.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "qsa.h")
 
+# Size of the static scratch buffer of qsa_score_select_noalloc
+# (QSA_SELECT_SCRATCH_BYTES in include/qsa.h).
+SELECT_SCRATCH_BYTES = 4 << 20
+
 STATUS = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_UNSUPPORTED", 3: "QSA_ERR_CUDA",
           4: "QSA_ERR_TIMEOUT", 5: "QSA_ERR_BOUNDS", 6: "QSA_ERR_WORKSPACE"}
 

@@ -22,6 +22,13 @@ def test_exports_every_declared_symbol():
         assert hasattr(qsa.lib(), name)
 
 
+def test_noalloc_scratch_size_matches_header():
+    text = open(qsa.HEADER_PATH).read()
+    m = re.search(r"#define QSA_SELECT_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", text)
+    assert m, "QSA_SELECT_SCRATCH_BYTES not found"
+    assert qsa.SELECT_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
 def test_status_strings_and_last_error():
     lib = qsa.lib()
     for code, name in qsa.STATUS.items():

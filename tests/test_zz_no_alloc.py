@@ -9,9 +9,16 @@ this entry point uses it instead of a caller workspace.
 
 The test calls the new entry point through the C ABI and checks that two
 calls in a row reproduce the selection of the workspace-taking entry point
-exactly (block indices are integer results, compared bit for bit), on a
-prefill case and on a decode case whose rows are split into several chunks
-(so the scratch holds both the pooled queries and the per-chunk keys).
+exactly (block indices are integer results, compared bit for bit).  Every
+case needs scratch memory, so every case reads and writes the static buffer:
+  * prefill_tiny: one chunk per row -- the scratch holds the pooled queries;
+  * prefill_chunked: rows of 2999 candidates split into chunks of 512 -- the
+    scratch also holds each chunk's top-m list, merged by a second kernel;
+  * decode_long_rows: per-token rows of 69999 candidates (a 4.48M-token
+    context), too long for the one-launch cluster path, so they take the
+    same pooled-query + chunk-list + merge route.
+The summaries of the two larger cases are drawn directly (the comparison is
+between two entry points on the same inputs, not against the oracle).
 This file is collected last on purpose.
 """
 import ctypes
@@ -23,10 +30,13 @@ import synthetic
 
 pytestmark = pytest.mark.gpu
 
+# (name, workload keywords, compress the drawn keys (True) or draw summaries)
 CASES = [
-    ("prefill_tiny", None),
-    ("decode_multichunk", dict(B=4, Tq=1, T_kv=64 * 700, q_pos0=64 * 700 - 1, qblk=1, Hq=16,
-                               Hkv=2, d=128, topk=16)),
+    ("prefill_tiny", None, True),
+    ("prefill_chunked", dict(B=1, Tq=128, T_kv=64 * 3002, q_pos0=64 * 3000, qblk=64, Hq=16, Hkv=2,
+                             d=128, topk=16), False),
+    ("decode_long_rows", dict(B=1, Tq=1, T_kv=64 * 70001, q_pos0=64 * 70001 - 1, qblk=1, Hq=16,
+                              Hkv=2, d=128, topk=64), False),
 ]
 
 
@@ -38,18 +48,38 @@ def _noalloc(qsa, Q, Kc, idx, w):
               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("name,kw", CASES, ids=[c[0] for c in CASES])
-def test_noalloc_selection_matches_workspace_entry_point(name, kw):
+def _inputs(w, compress):
+    import block_sparse_long_compress_b200 as qsa
+    if compress:
+        x = synthetic.generate(w)
+        Q, K = x["Q"].cuda(), x["K"].cuda()
+        Kc = torch.zeros((w.B, w.Hkv, w.T_kv // 64, w.d), dtype=torch.float32, device="cuda")
+        qsa.compress_keys(K, Kc)
+        return Q, Kc
+    g = torch.Generator(device="cuda")
+    g.manual_seed(w.seed)
+    Q = torch.randn((w.B, w.Tq, w.Hq, w.d), generator=g, device="cuda").to(torch.bfloat16)
+    # summaries of 64 N(0,1) keys have a spread of 1/8 per component
+    Kc = torch.randn((w.B, w.Hkv, w.T_kv // 64, w.d), generator=g, device="cuda") / 8
+    return Q, Kc
+
+
+@pytest.mark.parametrize("name,kw,compress", CASES, ids=[c[0] for c in CASES])
+def test_noalloc_selection_matches_workspace_entry_point(name, kw, compress):
     import block_sparse_long_compress_b200 as qsa
     w = synthetic.CONFIGS["tiny_prefill_1k"] if kw is None else synthetic.custom(seed=71, **kw)
-    x = synthetic.generate(w)
-    Q, K = x["Q"].cuda(), x["K"].cuda()
-    Kc = torch.zeros((w.B, w.Hkv, w.T_kv // 64, w.d), dtype=torch.float32, device="cuda")
-    qsa.compress_keys(K, Kc)
+    Q, Kc = _inputs(w, compress)
+    need = qsa.score_select_workspace(w.B, w.Hq, w.Hkv, w.Tq, w.q_pos0, w.qblk, w.d, w.topk)
+    qbar_bytes = -(-w.B * w.Hkv * w.n_rows * w.d * 4 // 256) * 256
+    assert need > 0, "this case must use the scratch buffer"
+    if name != "prefill_tiny":
+        assert need > qbar_bytes, "this case must also keep per-chunk lists in the scratch"
+    assert need <= qsa.SELECT_SCRATCH_BYTES
     shape = (w.B, w.Hkv, w.n_rows, w.topk)
     ref = torch.full(shape, -7, dtype=torch.int32, device="cuda")
     qsa.score_select(Q, Kc, ref, w.topk, w.q_pos0, w.qblk, w.sm_scale)
     assert qsa.device_status()[0] == "QSA_OK"
+    assert (ref[..., 0] == 0).all() and (ref >= -1).all()
     for call in range(2):
         out = torch.full(shape, -7, dtype=torch.int32, device="cuda")
         rc = _noalloc(qsa, Q, Kc, out, w)
@@ -62,7 +92,7 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     import block_sparse_long_compress_b200 as qsa
     # 8 x 131072 prefill rows would need ~8 MiB of pooled queries: refused on the host
     need = qsa.score_select_workspace(8, 16, 2, 131072, 0, 64, 128, 32)
-    assert need > 4 << 20
+    assert need > qsa.SELECT_SCRATCH_BYTES
     dummy = torch.empty(16, dtype=torch.int32, device="cuda")
     p = ctypes.c_void_p(dummy.data_ptr())
     rc = qsa.lib().qsa_score_select_noalloc(p, p, p, 8, 16, 2, 131072, 0, 64, 131072, 128, 32,
