@@ -157,6 +157,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
     __shared__ int blocks[C::MAX_SLOTS];   // the CTA's valid block ids in slot order
     __shared__ int rows[C::MAX_SLOTS];     // and the first cache row of each (TMA coordinate)
     __shared__ int nb_sh, issued_sh, abort_flag;
+    __shared__ int ring_bad;               // a copy may still land in the ring (see the drain)
     __shared__ float wloc[NC][8];          // merge weights of the CTA's warps, per head
     __shared__ float mloc[8], lloc[8];     // the CTA's combined max and sum per head
     __shared__ __align__(16) uint32_t uq[FP8 ? 8 * (D / 2) : 1];   // FP8: rotated queries, f16 pairs
@@ -248,6 +249,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
     if (threadIdx.x == 32) {
         abort_flag = 0;
         issued_sh = 0;
+        ring_bad = 0;
 #pragma unroll
         for (int s = 0; s < NS; s++) {
             mbar_init(&full[s], 1);
@@ -527,15 +529,19 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
     __syncthreads();
     if (abort_flag && threadIdx.x == NC * 32) {
         // a wait gave up: let the copies still in flight land before the
-        // ring is reused (bounded, no abort short-cut)
+        // ring is reused (bounded, no abort short-cut).  If one still has
+        // not landed, the ring is not reused at all: this CTA contributes
+        // nothing to the merge and writes zeros for the heads it owns (the
+        // timeout is in the status word either way)
         const int issued = issued_sh;
         for (int i = max(0, issued - NS); i < issued; i++)
-            mbar_wait(&full[i % NS], (i / NS) & 1, nullptr, 43, 100000000ull);
+            if (!mbar_wait(&full[i % NS], (i / NS) & 1, nullptr, 43, 100000000ull)) ring_bad = 1;
     }
     __syncthreads();
+    const bool ring_ok = ring_bad == 0;
 
     // ---- warp partials (m, l, O) into the idle ring
-    if (warp < NC) {
+    if (warp < NC && ring_ok) {
         float *wp = part + warp * PF;
         if (lane < 4) {
             wp[qc] = m_run[0];
@@ -570,14 +576,16 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
     if (threadIdx.x < G) {
         const int h = threadIdx.x;
         float mc = -INFINITY;
+        if (ring_ok) {
 #pragma unroll
-        for (int w = 0; w < NC; w++) mc = fmaxf(mc, part[w * PF + h]);
+            for (int w = 0; w < NC; w++) mc = fmaxf(mc, part[w * PF + h]);
+        }
         float lc = 0.f;
 #pragma unroll
         for (int w = 0; w < NC; w++) {
             const float f = mc == -INFINITY ? 0.f : fast_exp2(part[w * PF + h] - mc);
             wloc[w][h] = f;
-            lc += f * part[w * PF + 8 + h];
+            lc += f * (ring_ok ? part[w * PF + 8 + h] : 0.f);
         }
         mloc[h] = mc;
         lloc[h] = lc;
@@ -587,7 +595,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
         const int h = (e4 * 4) / D, c = (e4 * 4) % D;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int w = 0; w < NC; w++) {
+        for (int w = 0; w < NC && ring_ok; w++) {
             const float f = wloc[w][h];
             const float4 x = *reinterpret_cast<const float4 *>(part + w * PF + 16 + h * D + c);
             acc.x += f * x.x;
@@ -615,13 +623,13 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
         float lc = 0.f, x[CPL];
 #pragma unroll
         for (int t = 0; t < CPL; t++) x[t] = 0.f;
-        for (int src = 0; src < P; src++) {
+        for (int src = 0; src < P && ring_ok; src++) {
             const float f = mc == -INFINITY ? 0.f : fast_exp2(sl[src * SLOT] - mc);
             lc += f * sl[src * SLOT + 1];
 #pragma unroll
             for (int t = 0; t < CPL; t++) x[t] += f * sl[src * SLOT + 4 + CPL * lane + t];
         }
-        float il = lc > 0.f ? 1.f / lc : 0.f;
+        float il = lc > 0.f && ring_ok ? 1.f / lc : 0.f;
         if constexpr (FP8) {
             // back to the original basis: o = WHT(o') / 128 (the transform
             // squared is 128 I)

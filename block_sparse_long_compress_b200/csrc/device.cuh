@@ -18,14 +18,10 @@ namespace qsa {
 // qsa_get_device_status().
 __device__ int g_status = 0;
 __device__ int g_status_detail = 0;
-
-__device__ __forceinline__ void report(int code, int detail)
-{
-    if (atomicCAS(&g_status, 0, code) == 0) atomicExch(&g_status_detail, detail);
-}
-
-// Default limit of every bounded wait: 1 s of wall time.
-constexpr uint64_t kWaitLimitNs = 1000000000ull;
+// Global time (ns) of the latest timeout any wait recorded: a wait gives up
+// early only on a timeout recorded after it started, so a timeout left in the
+// status word by an earlier kernel does not cut short the waits of later ones.
+__device__ unsigned long long g_timeout_at = 0;
 
 __device__ __forceinline__ uint64_t globaltimer_ns()
 {
@@ -33,6 +29,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
+
+__device__ __forceinline__ void report(int code, int detail)
+{
+    if (code == QSA_ERR_TIMEOUT) atomicMax(&g_timeout_at, (unsigned long long)globaltimer_ns());
+    if (atomicCAS(&g_status, 0, code) == 0) atomicExch(&g_status_detail, detail);
+}
+
+// Default limit of every bounded wait: 1 s of wall time.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -152,8 +157,9 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity
 // Bounded wait for the phase of `parity` to complete.  Returns false (and
 // records QSA_ERR_TIMEOUT with `where`) when the limit runs out, or early if
 // *abort is set (another wait of this CTA gave up) or, after the first
-// millisecond, if any CTA has already recorded a timeout.  Sets *abort on
-// a timeout so that the other waits of the CTA give up immediately.
+// millisecond, if any CTA has recorded a timeout since this wait began.
+// Sets *abort on a timeout so that the other waits of the CTA give up
+// immediately.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           int where, uint64_t limit_ns = kWaitLimitNs)
 {
@@ -164,7 +170,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         if (abort && *abort) return false;
         if (mbar_try_wait_hint(a, parity, 200000u)) return true;
         const uint64_t dt = globaltimer_ns() - t0;
-        if (dt > 1000000ull && *(volatile int *)&g_status == QSA_ERR_TIMEOUT) {
+        if (dt > 1000000ull && *(volatile unsigned long long *)&g_timeout_at >= t0) {
             if (abort) *abort = 1;
             return false;
         }

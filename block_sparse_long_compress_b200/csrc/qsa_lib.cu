@@ -248,6 +248,19 @@ qsa_status launch_prefill(const void *Q, const void *K, const void *V, const int
     if ((st = make_map_2d(&mk, K, nrows, D)) != QSA_OK) return st;
     if ((st = make_map_2d(&mv, V, nrows, D)) != QSA_OK) return st;
     auto kern = qsa::sparse_attn_prefill_kernel<D, G>;
+    // the kernel's setmaxnreg split waits without a limit unless every
+    // thread starts with C::REG_LAUNCH registers: refuse any other build
+    {
+        static int regs = 0;
+        if (!regs) {
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return check_launch("cudaFuncGetAttributes");
+            regs = fa.numRegs;
+        }
+        if (regs != C::REG_LAUNCH)
+            return fail(QSA_ERR_UNSUPPORTED, "sparse_attn_prefill_kernel built with %d registers per thread, "
+                        "its register split needs %d", regs, C::REG_LAUNCH);
+    }
     if ((st = set_smem(kern, C::SMEM_REQUEST)) != QSA_OK) return st;
     // persistent: one CTA per SM (never more than there are work units)
     const long units = (long)((Tq + 63) / 64) * C::TILES * B * Hkv;

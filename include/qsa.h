@@ -154,7 +154,10 @@ QSA_API qsa_status qsa_score_select_bf16(const void *Q, const void *Kc, int32_t 
  * cudaFree or other allocating routine.
  * The first call on each device looks up the buffer's device address (with
  * that device current) and caches it; make that first call before any
- * stream capture.  Every call shares the one buffer and it keeps the last
+ * stream capture.  The cached address lives as long as the process's
+ * context on that device: after cudaDeviceReset() the library's device
+ * memory is gone and this entry point must not be called again in the
+ * process.  Every call shares the one buffer and it keeps the last
  * call's contents (nothing in it needs to start at zero), so calls that
  * overlap on the GPU -- on different streams, or from different host
  * threads on the same device -- race with each other: serialise them.
@@ -199,9 +202,11 @@ QSA_API qsa_status qsa_decode(const void *q, const void *K_cache, const void *V_
                       size_t workspace_bytes, qsa_stream_t stream);
 
 /*
- * Ragged batches over paged caches (serving).  The pages' contract is
- * "selector -> visible cache-cell IDs -> attention over those cells"; here
- * a cell is a 64-token page:
+ * Ragged batches over paged caches (serving).  The selector hands the
+ * attention the addresses of the cache cells it may see, and attention runs
+ * over those cells only (page "Qwen4 in llama.cpp: Dissecting PR #27742",
+ * section "QSA Is an Address-Selection Problem, Not a New Attention
+ * Equation"); here a cell is a 64-token page:
  *   K_pages, V_pages  bf16 [num_pages][Hkv][64][d] (page p holds one block of
  *                     one sequence for all KV heads);
  *   block_table       int32 [B][max_blocks] device array: logical block j of
@@ -379,7 +384,11 @@ QSA_API qsa_status qsa_decode_fp8_paged(const void *q, const void *K_codes, cons
 /*
  * Synchronises `stream`, then returns and clears the device status word
  * (QSA_OK if no kernel recorded an error since the last call).  If detail
- * is not NULL it receives a kernel-specific code (0 if none).
+ * is not NULL it receives a kernel-specific code (0 if none).  The word
+ * keeps the first error until it is read here; a recorded timeout does not
+ * cut short the bounded waits of kernels launched after it (they give up
+ * early only on a timeout recorded while they wait), but read and clear
+ * the word after any error so that later errors are seen.
  */
 QSA_API qsa_status qsa_get_device_status(qsa_stream_t stream, int *detail);
 
