@@ -322,8 +322,6 @@ def decode_fp8(q, codes_K, scales_K, codes_V, scales_V, idx, L, sm_scale, blk=BL
     G = Hq // Hkv
     H = hadamard(n)
     uq = qf @ H                              # rows: H is symmetric
-    Kr = e4m3_value(codes_K) * np.asarray(scales_K, dtype=np.float64)[..., None]
-    Vr = e4m3_value(codes_V) * np.asarray(scales_V, dtype=np.float64)[..., None]
     o = np.zeros((B, Hq, n))
     for b in range(B):
         for g in range(Hkv):
@@ -333,11 +331,14 @@ def decode_fp8(q, codes_K, scales_K, codes_V, scales_V, idx, L, sm_scale, blk=BL
                     continue
                 keys.extend(range(int(j) * blk, min(int(j) * blk + blk, L)))
             keys = np.array(keys, dtype=np.int64)
+            # dequantized rows of the visible keys: code value times row scale
+            Kr = e4m3_value(codes_K[b, g, keys]) * np.asarray(scales_K[b, g, keys], dtype=np.float64)[:, None]
+            Vr = e4m3_value(codes_V[b, g, keys]) * np.asarray(scales_V[b, g, keys], dtype=np.float64)[:, None]
             for h in range(g * G, (g + 1) * G):
-                z = (Kr[b, g, keys] @ uq[b, h]) / n * sm_scale
+                z = (Kr @ uq[b, h]) / n * sm_scale
                 w = np.exp(z - z.max())
                 w /= w.sum()
-                o[b, h] = H @ (w @ Vr[b, g, keys]) / n
+                o[b, h] = H @ (w @ Vr) / n
     return o
 
 
