@@ -212,21 +212,22 @@ def decode_bytes(w):
 
 
 # ------------------------------------------------------------- our arm
-def run_qsa(args, ws, rank, local):
-    import block_sparse_long_compress_b200 as qsa
-
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    peaks = load_peaks()
-    wp = synthetic.CONFIGS[args.workload]
+def bench_prefill(args, qsa, dev, wname, ws, rank, flush, keep=False, clocks=False):
+    """One prefill workload: W untimed warm-up steps, then exactly K steps
+    (compress of the step's new key blocks -> pool/score/select ->
+    attention), each bracketed by CUDA events on the launching stream, the L2
+    flushed between steps.  Returns a dict with the workload, the per-part
+    times, the launches in the timed region, the clock record (when asked)
+    and, with keep, host copies of the inputs and outputs for the oracle's
+    parity check (taken after the timed region)."""
+    wp = synthetic.CONFIGS[wname]
     if ws > 1:
         wp = synthetic.Workload(**{**wp.__dict__, "seed": wp.seed + 1000 * rank})
     x = synthetic.generate(wp, dev)
     Q, K, V = x["Q"], x["K"], x["V"]
     run = qsa.QSAPrefill(wp.B, wp.Tq, wp.Hq, wp.Hkv, wp.d, wp.T_kv, wp.topk, wp.q_pos0, device=dev)
-    run.precompress_cache(K)
+    run.precompress_cache(K)           # the cache's summaries: persistent state (untimed)
     stream = torch.cuda.current_stream()
-    flush = L2Flush(dev)
 
     def step(ev=None):
         if ev is None:
@@ -244,34 +245,79 @@ def run_qsa(args, ws, rank, local):
     torch.cuda.synchronize()
     st, det = qsa.device_status()
     if st != "QSA_OK":
-        raise RuntimeError(f"device status {st} ({det})")
+        raise RuntimeError(f"{wname}: device status {st} ({det})")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     if ws > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     n0 = qsa.launch_count()
-    with ClockSampler(local) as clk:
-        for k in range(args.steps):
-            flush(k)
-            step(evs[k])
-        torch.cuda.synchronize()
+    clk = ClockSampler(dev.index) if clocks else None
+    if clk:
+        clk.__enter__()
+    for k in range(args.steps):
+        flush(k)
+        step(evs[k])
+    torch.cuda.synchronize()
+    if clk:
+        clk.__exit__(None, None, None)
     n_launch = qsa.launch_count() - n0
     if ws > 1:
         torch.distributed.barrier()
     st, det = qsa.device_status()
     if st != "QSA_OK":
-        raise RuntimeError(f"device status {st} ({det})")
-    t_comp = np.array([e[0].elapsed_time(e[1]) for e in evs])
-    t_sel = np.array([e[1].elapsed_time(e[2]) for e in evs])
-    t_att = np.array([e[2].elapsed_time(e[3]) for e in evs])
-    t_step = np.array([e[0].elapsed_time(e[3]) for e in evs])
-    ms = float(t_step.sum() / args.steps)
-    value, ms_max = job_throughput(ms, wp.B * wp.Tq, dev)
+        raise RuntimeError(f"{wname}: device status {st} ({det})")
+    t = {"compress": np.array([e[0].elapsed_time(e[1]) for e in evs]),
+         "score_select": np.array([e[1].elapsed_time(e[2]) for e in evs]),
+         "attention": np.array([e[2].elapsed_time(e[3]) for e in evs]),
+         "step": np.array([e[0].elapsed_time(e[3]) for e in evs])}
+    out = {"w": wp, "t": t, "launches": int(n_launch), "clocks": clk.summary() if clk else None}
+    if keep:
+        out["kept"] = {"w": wp, "x": {k: x[k].cpu() for k in ("Q", "K", "V")},
+                       "idx": run.idx.cpu().numpy(), "O": run.O.cpu()}
+    del Q, K, V, x, run
+    torch.cuda.empty_cache()
+    return out
 
+
+def prefill_roofline(wp, att_ms, peaks):
     flops = prefill_flops(wp)
-    att_s = float(t_att.mean()) * 1e-3
-    achieved = flops / att_s / 1e12
+    achieved = flops / (att_ms * 1e-3) / 1e12
+    return {"bound": "tensor", "kernel": "sparse_attn_prefill_kernel",
+            "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": achieved / peaks["bf16_tflops"],
+            "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
+                                  if peaks.get("bf16_tflops_sustained") else None),
+            "peak_source": peaks["source"] + " bf16 burst", "flops_per_launch": flops,
+            "traffic": None}
+
+
+def prefill_subline(pr, peaks):
+    """A further prefill workload's part of the line (timed like the headline)."""
+    wp, t = pr["w"], pr["t"]
+    ms = float(t["step"].mean())
+    return {"workload": wp.name, "batch": wp.B, "new_tokens": wp.Tq, "context": wp.q_pos0 + wp.Tq,
+            "topk": wp.topk, "tokens_per_s": wp.B * wp.Tq / (ms * 1e-3), "ms_per_step": ms,
+            "breakdown_ms": {k: float(t[k].mean()) for k in ("compress", "score_select", "attention")},
+            "roofline": prefill_roofline(wp, float(t["attention"].mean()), peaks)}
+
+
+def run_qsa(args, ws, rank, local, kept):
+    """Our arm.  Appends to `kept` the host copies the parity check needs
+    (rank 0 at N=1 only)."""
+    import block_sparse_long_compress_b200 as qsa
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    flush = L2Flush(dev)
+    want_keep = ws == 1 and not args.no_cpu_baseline
+    pr = bench_prefill(args, qsa, dev, args.workload, ws, rank, flush, keep=want_keep, clocks=True)
+    wp, t = pr["w"], pr["t"]
+    if want_keep:
+        kept.append(("prefill", pr["kept"]))
+    ms = float(t["step"].sum() / args.steps)
+    value, ms_max = job_throughput(ms, wp.B * wp.Tq, dev)
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
@@ -280,32 +326,33 @@ def run_qsa(args, ws, rank, local):
                    "kv_heads": wp.Hkv, "head_dim": wp.d, "block": 64, "topk": wp.topk,
                    "parallelism": f"dp{ws} (independent sequences)",
                    "l2": L2Flush.DESCRIPTION},
-        "breakdown_ms": {"compress": float(t_comp.mean()), "score_select": float(t_sel.mean()),
-                         "attention": float(t_att.mean())},
-        "roofline": {"bound": "tensor", "kernel": "sparse_attn_prefill_kernel",
-                     "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved / peaks["bf16_tflops"],
-                     "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
-                                           if peaks.get("bf16_tflops_sustained") else None),
-                     "peak_source": peaks["source"] + " bf16 burst", "flops_per_launch": flops,
-                     "traffic": None},
-        "gpu_launches": int(n_launch),
-        "clocks": clk.summary(),
+        "breakdown_ms": {k: float(t[k].mean()) for k in ("compress", "score_select", "attention")},
+        "roofline": prefill_roofline(wp, float(t["attention"].mean()), peaks),
+        "gpu_launches": pr["launches"],
+        "clocks": pr["clocks"],
     }
 
+    # ---- the other prefill workloads, timed the same way
+    for name in filter(None, args.prefill_more.split(",")):
+        sub = bench_prefill(args, qsa, dev, name, ws, rank, flush, keep=want_keep)
+        if want_keep:
+            kept.append(("prefill", sub["kept"]))
+        result.setdefault("prefill_more", {})[name] = prefill_subline(sub, peaks)
+
     if args.prefill_max:
-        result["prefill_max_selection"] = bench_prefill_agg(args, qsa, dev, peaks, wp, Q, K, flush, "max")
-        result["prefill_softmax_sum_selection"] = bench_prefill_agg(args, qsa, dev, peaks, wp, Q, K, flush,
-                                                                    "softmax_sum")
+        x = synthetic.generate(wp, dev)
+        result["prefill_max_selection"] = bench_prefill_agg(args, qsa, dev, peaks, wp, x["Q"], x["K"], flush, "max")
+        result["prefill_softmax_sum_selection"] = bench_prefill_agg(args, qsa, dev, peaks, wp, x["Q"], x["K"],
+                                                                    flush, "softmax_sum")
+        del x
+        torch.cuda.empty_cache()
 
     # ---- decode at 128K (same process, after the prefill tensors are freed)
     if not args.no_decode:
-        del Q, K, V, run, x
-        torch.cuda.empty_cache()
         if args.paged:
             result["prefill_ragged_paged"] = bench_prefill_paged(args, qsa, dev, peaks, ws, rank, flush)
             torch.cuda.empty_cache()
-        result["decode"] = bench_decode(args, qsa, dev, peaks, ws, rank, flush)
+        result["decode"] = bench_decode(args, qsa, dev, peaks, ws, rank, flush, kept=kept if want_keep else None)
         if args.bf16_summaries:
             result["decode"]["bf16_summaries"] = bench_decode(args, qsa, dev, peaks, ws, rank, flush,
                                                               summary="bf16")
@@ -327,7 +374,8 @@ def run_qsa(args, ws, rank, local):
         for name in filter(None, args.decode_more.split(",")):
             torch.cuda.empty_cache()
             result.setdefault("decode_more", {})[name] = bench_decode(args, qsa, dev, peaks, ws,
-                                                                      rank, flush, name)
+                                                                      rank, flush, name,
+                                                                      kept=kept if want_keep else None)
             if args.bf16_summaries:
                 result["decode_more"][name]["bf16_summaries"] = bench_decode(
                     args, qsa, dev, peaks, ws, rank, flush, name, summary="bf16")
@@ -439,7 +487,8 @@ def decode_result(wname, B, context, topk, t, d, launches, by, sel_bytes, peaks,
     return r
 
 
-def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary="fp32", kv="bf16", agg="mean"):
+def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary="fp32", kv="bf16", agg="mean",
+                 kept=None):
     wd = synthetic.CONFIGS[workload or args.decode_workload]
     if args.decode_batch:
         wd = synthetic.Workload(**{**wd.__dict__, "B": args.decode_batch})
@@ -486,6 +535,13 @@ def bench_decode(args, qsa, dev, peaks, ws, rank, flush, workload=None, summary=
                 qsa.decode(q, K, V, dec.idx, dec.o, L, dec.sm_scale, dec.ws_dec, s)
 
     t, d, launches = decode_timings(args, qsa, dev, ws, flush, run_parts)
+    if kept is not None:
+        # host copies for the oracle's parity check: the last replayed step's
+        # indices and outputs, the queries, and two sequences' caches
+        seqs = sorted({0, wd.B - 1})
+        kept.append(("decode", {"w": wd, "q": x["Q"].cpu(), "idx": dec.idx.cpu().numpy(),
+                                "o": dec.o.float().cpu().numpy(),
+                                "seqs": {b: (K[b:b + 1].cpu(), V[b:b + 1].cpu()) for b in seqs}}))
     # summaries read by scoring (fp32, or bf16 for the bf16-summary option)
     sel_bytes = wd.B * wd.Hkv * ((L - 1) // 64) * wd.d * (2 if summary == "bf16" else 4)
     return decode_result(wd.name, wd.B, L, wd.topk, t, d, launches, by, sel_bytes, peaks, extra)
@@ -727,6 +783,95 @@ def oracle_sample(wp, x_cpu, budget_s):
     return n / t, desc, nthreads
 
 
+def parity_check(kept, rng_seed=5):
+    """The oracle against the GPU's outputs of the timed runs (part of the
+    CPU-baseline leg, after every timed region): for each prefill workload,
+    a sample of selection rows (exact-match and Jaccard overlap, the
+    indices required to match wherever the oracle's gap exceeds 1e-3) and
+    the outputs of a sample of their tokens over the GPU's own selection;
+    for each decode workload, the rows and outputs of two sequences."""
+    import oracle
+
+    def jaccard(a, b):
+        A, B = {int(v) for v in a if v >= 0}, {int(v) for v in b if v >= 0}
+        return len(A & B) / len(A | B) if (A or B) else 1.0
+
+    rng = np.random.RandomState(rng_seed)
+    out = {}
+    for kind, k in kept:
+        w = k["w"]
+        t0 = time.perf_counter()
+        if kind == "prefill":
+            x, idx = k["x"], k["idx"]
+            NR = w.n_rows
+            n_complete = (w.q_pos0 + w.Tq) // 64
+            Kc = oracle.compress_keys(x["K"], 0, n_complete)
+            Qbar = oracle.pool_queries(x["Q"], w.Hkv, w.qblk)
+            nrows = w.B * w.Hkv * NR
+            rows = np.unique(np.concatenate([[0, NR - 1, nrows - 1],
+                                             rng.choice(nrows, size=min(nrows, 61), replace=False)]))
+            sel = oracle.select(Qbar, Kc, w.Tq, w.q_pos0, w.qblk, w.topk, w.sm_scale, rows=rows)
+            gidx = idx.reshape(-1, w.topk)[rows]
+            # tokens: the first and the last 8 of up to 16 of the sampled rows (b = row // (Hkv NR))
+            toks = []
+            for r in rows[:16]:
+                b, i = r // (w.Hkv * NR), r % NR
+                t0_, t1_ = i * 64, min((i + 1) * 64, w.Tq)
+                toks += [b * w.Tq + t for t in list(range(t0_, min(t0_ + 8, t1_))) + list(range(max(t1_ - 8, t0_), t1_))]
+            toks = np.unique(np.array(toks, dtype=np.int64))
+            O_ref = oracle.attend(x["Q"], x["K"], x["V"], idx, w.q_pos0, w.qblk, w.sm_scale, tokens=toks)
+            O_gpu = k["O"].reshape(w.B * w.Tq, w.Hq, w.d)[torch.from_numpy(toks)].float().numpy()
+        else:
+            L = w.q_pos0 + 1
+            sels, gl, O_ref, O_gpu = [], [], [], []
+            for b, (Kb, Vb) in k["seqs"].items():
+                qb = k["q"][b:b + 1]
+                Kc = oracle.compress_keys(Kb, 0, L // 64)
+                sel = oracle.select(oracle.pool_queries(qb, w.Hkv, 1), Kc, 1, w.q_pos0, 1, w.topk, w.sm_scale,
+                                    rows=np.arange(w.Hkv))
+                sels.append(sel)
+                gl.append(k["idx"][b].reshape(-1, w.topk))
+                O_ref.append(oracle.attend(qb, Kb, Vb, k["idx"][b:b + 1], w.q_pos0, 1, w.sm_scale)[0, 0])
+                O_gpu.append(k["o"][b])
+            sel = {"idx": np.concatenate([s_["idx"] for s_ in sels]), "gap": np.concatenate([s_["gap"] for s_ in sels])}
+            gidx = np.concatenate(gl)
+            O_ref, O_gpu = np.stack(O_ref), np.stack(O_gpu)
+            rows, toks = np.arange(len(gidx)), np.arange(len(O_gpu))
+        same = np.all(gidx == sel["idx"], axis=1)
+        clear = sel["gap"] > 1e-3
+        err = np.abs(O_gpu - O_ref)
+        out[w.name] = {"rows": int(len(rows)), "gap_checked": float(clear.mean()),
+                       "exact_where_gap_checked": float(same[clear].mean()) if clear.any() else None,
+                       "identical": float(same.mean()),
+                       "jaccard": float(np.mean([jaccard(a, b) for a, b in zip(gidx, sel["idx"])])),
+                       "outputs": int(err.size), "max_abs_err": float(err.max()),
+                       "mean_abs_err": float(err.mean()), "oracle_s": time.perf_counter() - t0}
+    return out
+
+
+def headline(res):
+    """The line's key numbers in a few hundred characters, as its last key."""
+    r = lambda v: None if v is None else float(f"{v:.4g}")
+    h = {"prefill_128k" if res["config"]["workload"] == "prefill_128k" else res["config"]["workload"]: {
+        "Mtok_s": r(res["value"] / 1e6), "select_ms": r(res["breakdown_ms"]["score_select"]),
+        "attn_ms": r(res["breakdown_ms"]["attention"]), "attn_frac": r(res["roofline"]["frac"])}}
+    for name, sub in res.get("prefill_more", {}).items():
+        h[name] = {"Mtok_s": r(sub["tokens_per_s"] / 1e6), "select_ms": r(sub["breakdown_ms"]["score_select"]),
+                   "attn_ms": r(sub["breakdown_ms"]["attention"]), "attn_frac": r(sub["roofline"]["frac"])}
+    decs = [res["decode"]] if "decode" in res else []
+    decs += list(res.get("decode_more", {}).values())
+    for d in decs:
+        h[d["workload"]] = {"us_per_token": r(d["us_per_token"]), "us_step": r(d["us_per_step"]),
+                            "select_us": r(d["breakdown_us"]["score_select"]),
+                            "attn_us": r(d["breakdown_us"]["attention"]), "attn_frac": r(d["roofline"]["frac"]),
+                            "select_frac": r(d["select_hbm_frac"])}
+    par = res.get("cpu_baseline", {}).get("parity")
+    if par:
+        h["parity"] = {n: {"max": r(p["max_abs_err"]), "mean": r(p["mean_abs_err"]), "identical": r(p["identical"]),
+                           "jaccard": r(p["jaccard"])} for n, p in par.items()}
+    return h
+
+
 def run_reference(args, ws, rank):
     if rank != 0:
         return None
@@ -764,6 +909,8 @@ def main():
     ap.add_argument("--decode-workload", default=DECODE, choices=sorted(synthetic.CONFIGS))
     ap.add_argument("--decode-more", default="decode_262k",
                     help="comma list of further decode workloads reported under decode_more")
+    ap.add_argument("--prefill-more", default="prefill_32k,chunked_1m",
+                    help="comma list of further prefill workloads reported under prefill_more")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-paged", dest="paged", action="store_false",
                     help="skip the ragged-batch, paged-cache decode run (reported beside the contiguous one)")
@@ -836,15 +983,16 @@ def main():
         if rank == 0:
             print(json.dumps(res), flush=True)
         return
-    res = run_qsa(args, ws, rank, local)
+    kept = []
+    res = run_qsa(args, ws, rank, local, kept)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         wp = synthetic.CONFIGS[args.workload]
-        g = synthetic.generate(wp, torch.device("cuda", local))
-        x_cpu = {k: g[k].cpu() for k in ("Q", "K", "V")}
-        del g
+        x_cpu = next(k["x"] for kind, k in kept if kind == "prefill" and k["w"].name == wp.name)
         v, desc, threads = oracle_sample(wp, x_cpu, args.cpu_budget)
         res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
-                               "sample": desc}
+                               "sample": desc, "parity": parity_check(kept)}
+    del kept
+    res["headline"] = headline(res)
     if ws > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
