@@ -101,7 +101,8 @@ struct PrefillShared {
     uint64_t v_full[4], v_empty[4];
     uint64_t s_full[2][2];      // [tile][S buffer]
     uint64_t p_full[2][2];      // [tile][S buffer]
-    uint64_t pv_done[2];        // [tile]
+    uint64_t pv_done[2];        // [tile]: completes once per block (its PV)
+    uint64_t o_full[2];         // [tile]: completes once per unit (its last PV)
     uint64_t stag[2];           // [tile]: its softmax has its block max
     uint64_t list_full[2], list_empty[2];   // [list slot]
     uint32_t tmem_base;
@@ -168,6 +169,7 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
                 mbar_init(&sh.p_full[t][bf], 4);   // one arrive per softmax warp
             }
             mbar_init(&sh.pv_done[t], 1);
+            mbar_init(&sh.o_full[t], 1);
             mbar_init(&sh.stag[t], 4);
             mbar_init(&sh.list_full[t], 1);
             mbar_init(&sh.list_empty[t], C::LIST_USERS);
@@ -408,6 +410,7 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
                         umma_ts(o_tmem, p_tmem + kk * 8, vds + (uint64_t)((kk * 2048) >> 4), idesc_o,
                                 (n > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&sh.pv_done[t]);
+                    if (n == nb - 1) umma_commit(&sh.o_full[t]);
                 }
                 __syncwarp();
                 // S_t(gb+2) into the same buffer, right behind PV_t(gb)
@@ -552,10 +555,13 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
             }
             if (!ok) break;
             if (lane == 0) mbar_arrive(&sh.list_empty[slot]);
-            // epilogue: O_t / l once the unit's last PV is done.  The next
-            // unit's first PV overwrites O_t only after P of its block,
-            // which this warp signals after these loads.
-            if (!wait_all(&sh.pv_done[t], (g0 + nb - 1) & 1, 32)) { ok = false; break; }
+            // epilogue: O_t / l once the unit's last PV is done.  That is
+            // the unit's own barrier (one phase per unit): pv_done counts
+            // blocks, and here only PV(g0 + nb - 3) is known to be done, so
+            // its parity could not tell PV(g0 + nb - 1) from PV(g0 + nb - 3).
+            // The next unit's first PV overwrites O_t only after P of its
+            // block, which this warp signals after these loads.
+            if (!wait_all(&sh.o_full[t], k & 1, 32)) { ok = false; break; }
             tc_fence_after();
             const float inv_l = (!none && l > 0.f) ? 1.0f / l : 0.f;
             // O_t / l as bf16, one 64-column half at a time: each thread
