@@ -129,7 +129,8 @@ bool supported_d(int d) { return d == 64 || d == 128; }
 // ------------------------------------------------------- select geometry
 struct SelectPlan {
     int NR, CH, maxchunks;
-    size_t qbar_bytes, part_bytes;
+    int TS;               // prefill rows: score-table row stride (floats)
+    size_t qbar_bytes, part_bytes, table_bytes;
 };
 
 SelectPlan plan_select(int B, int Hkv, int Tq, int q_pos0, int qblk, int d)
@@ -146,6 +147,10 @@ SelectPlan plan_select(int B, int Hkv, int Tq, int q_pos0, int qblk, int d)
     p.maxchunks = ncand > 0 ? (ncand + CH - 1) / CH : 1;
     p.qbar_bytes = align256((size_t)rows * d * sizeof(float));
     p.part_bytes = p.maxchunks > 1 ? align256((size_t)rows * p.maxchunks * qsa::kMaxChosen * 8) : 0;
+    // prefill rows (qblk = 64) are scored 8 rows at a time into a table
+    // whose rows hold candidates 1 .. Dmax - 1 at their block index
+    p.TS = qblk == 64 ? (Dmax + 3) / 4 * 4 : 0;
+    p.table_bytes = qblk == 64 ? align256((size_t)rows * p.TS * sizeof(float)) : 0;
     return p;
 }
 
@@ -454,6 +459,43 @@ qsa_status compress_keys_impl(const char *name, const void *K, KcT *Kc, int B, i
 }
 
 
+// Pooling, then scoring and selection: prefill rows through the score
+// table (score_table_kernel, then score_select_kernel from the table),
+// long per-token rows by score_select_kernel's own scoring.
+template <int D, typename KcT>
+qsa_status launch_score_select(const void *Q, const KcT *Kc, int32_t *idx, float *Qbar, uint64_t *part, float *table,
+                               const SelectPlan &p, dim3 pgrid, int pool_threads, int pool_smem, dim3 sgrid, int ssmem,
+                               int B, int Hq, int Hkv, int Tq, int q_pos0, int qblk, int nblk_max, int topk,
+                               float sm_scale, const int32_t *q_pos, cudaStream_t s)
+{
+    qsa_status st;
+    if ((st = set_smem(qsa::pool_queries_kernel<D>, pool_smem)) != QSA_OK) return st;
+    qsa::pool_queries_kernel<D><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq, Hq, Hkv,
+                                                                       qblk);
+    if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
+    if (qblk == 64) {
+        const int Dmax = (q_pos0 + Tq - 1) / 64;
+        constexpr int TT = qsa::kTableTile;
+        const dim3 tgrid((unsigned)std::max(1, (Dmax - 1 + TT - 1) / TT), (unsigned)((p.NR + TT - 1) / TT),
+                         (unsigned)(B * Hkv));
+        const int tsmem = 2 * TT * (D + 4) * (int)sizeof(float);
+        if ((st = set_smem(qsa::score_table_kernel<D, KcT>, tsmem)) != QSA_OK) return st;
+        qsa::score_table_kernel<D, KcT><<<tgrid, 256, tsmem, s>>>(Qbar, Kc, table, nblk_max, Tq, q_pos0, p.TS,
+                                                                  sm_scale, Hkv, q_pos);
+        if ((st = launched("score_table_kernel")) != QSA_OK) return st;
+        auto kern = qsa::score_select_kernel<D, KcT, true>;
+        if ((st = set_smem(kern, ssmem)) != QSA_OK) return st;
+        kern<<<sgrid, qsa::kSelThreads, ssmem, s>>>(nullptr, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk,
+                                                    sm_scale, p.CH, p.maxchunks, Hkv, q_pos, table, p.TS);
+    } else {
+        auto kern = qsa::score_select_kernel<D, KcT>;
+        if ((st = set_smem(kern, ssmem)) != QSA_OK) return st;
+        kern<<<sgrid, qsa::kSelThreads, ssmem, s>>>(Qbar, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk, sm_scale,
+                                                    p.CH, p.maxchunks, Hkv, q_pos, nullptr, 0);
+    }
+    return launched("score_select_kernel");
+}
+
 template <typename KcT>
 qsa_status score_select_impl(const char *name, const void *Q, const KcT *Kc, int32_t *idx, int B, int Hq, int Hkv,
                              int Tq, int q_pos0, int qblk, int T_kv_max, int d, int topk, float sm_scale,
@@ -480,35 +522,25 @@ qsa_status score_select_impl(const char *name, const void *Q, const KcT *Kc, int
     const SelectPlan p = plan_select(B, Hkv, Tq, q_pos0, qblk, d);
     if (p.maxchunks * qsa::kMaxChosen * 8 > 200 * 1024)
         return fail(QSA_ERR_UNSUPPORTED, "%s: context too long", name);
-    if (!workspace || workspace_bytes < p.qbar_bytes + p.part_bytes || !aligned16(workspace))
-        return fail(QSA_ERR_WORKSPACE, "%s: workspace needs %zu bytes", name,
-                    p.qbar_bytes + p.part_bytes);
+    const size_t need = p.qbar_bytes + p.part_bytes + p.table_bytes;
+    if (!workspace || workspace_bytes < need || !aligned16(workspace))
+        return fail(QSA_ERR_WORKSPACE, "%s: workspace needs %zu bytes", name, need);
     float *Qbar = static_cast<float *>(workspace);
     uint64_t *part = reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(workspace) + p.qbar_bytes);
+    float *table = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + p.qbar_bytes + p.part_bytes);
     const int nblk_max = T_kv_max / 64;
     const int pool_threads = ((Hq * d / 8) + 31) / 32 * 32;
     const int pool_smem = Hq * d * 4;
     dim3 pgrid(p.NR, B), sgrid(p.maxchunks, p.NR, B * Hkv), mgrid(p.NR, B * Hkv);
     const int ssmem = p.CH * 8;
     qsa_status st;
-    if (d == 128) {
-        if ((st = set_smem(qsa::pool_queries_kernel<128>, pool_smem)) != QSA_OK) return st;
-        qsa::pool_queries_kernel<128><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq,
-                                                                             Hq, Hkv, qblk);
-        if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
-        if ((st = set_smem(qsa::score_select_kernel<128, KcT>, ssmem)) != QSA_OK) return st;
-        qsa::score_select_kernel<128, KcT><<<sgrid, qsa::kSelThreads, ssmem, s>>>(
-            Qbar, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk, sm_scale, p.CH, p.maxchunks, Hkv, q_pos);
-    } else {
-        if ((st = set_smem(qsa::pool_queries_kernel<64>, pool_smem)) != QSA_OK) return st;
-        qsa::pool_queries_kernel<64><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq,
-                                                                            Hq, Hkv, qblk);
-        if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
-        if ((st = set_smem(qsa::score_select_kernel<64, KcT>, ssmem)) != QSA_OK) return st;
-        qsa::score_select_kernel<64, KcT><<<sgrid, qsa::kSelThreads, ssmem, s>>>(
-            Qbar, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk, sm_scale, p.CH, p.maxchunks, Hkv, q_pos);
-    }
-    if ((st = launched("score_select_kernel")) != QSA_OK) return st;
+    if (d == 128) st = launch_score_select<128, KcT>(Q, Kc, idx, Qbar, part, table, p, pgrid, pool_threads,
+                                                      pool_smem, sgrid, ssmem, B, Hq, Hkv, Tq, q_pos0, qblk,
+                                                      nblk_max, topk, sm_scale, q_pos, s);
+    else st = launch_score_select<64, KcT>(Q, Kc, idx, Qbar, part, table, p, pgrid, pool_threads, pool_smem,
+                                           sgrid, ssmem, B, Hq, Hkv, Tq, q_pos0, qblk, nblk_max, topk, sm_scale,
+                                           q_pos, s);
+    if (st != QSA_OK) return st;
     if (p.maxchunks > 1) {
         const int msmem = p.maxchunks * qsa::kMaxChosen * 8;
         if ((st = set_smem(qsa::merge_select_kernel, msmem)) != QSA_OK) return st;
@@ -592,7 +624,7 @@ size_t qsa_score_select_workspace(int B, int Hq, int Hkv, int Tq, int q_pos0, in
     if (B <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || (qblk != 1 && qblk != 64) || !supported_d(d)) return 0;
     if (plan_token(B, Hkv, Tq, q_pos0, qblk).use) return 0;
     const SelectPlan p = plan_select(B, Hkv, Tq, q_pos0, qblk, d);
-    return p.qbar_bytes + p.part_bytes;
+    return p.qbar_bytes + p.part_bytes + p.table_bytes;
 }
 
 qsa_status qsa_score_select(const void *Q, const float *Kc, int32_t *idx, int B, int Hq, int Hkv, int Tq,
@@ -715,7 +747,7 @@ qsa_status qsa_score_select_prefill_agg(const void *Q, const void *Kc, int32_t *
     if ((st = set_smem(skern, p.CH * 8)) != QSA_OK) return st;
     skern<<<sgrid, qsa::kSelThreads, p.CH * 8, s>>>(nullptr, static_cast<const __nv_bfloat16 *>(Kc), idx, part, nblk,
                                                     Tq, q_pos0, 64, topk, sm_scale, p.CH, p.maxchunks, Hkv, nullptr,
-                                                    scores);
+                                                    scores, 0);
     if ((st = launched("score_select_kernel")) != QSA_OK) return st;
     if (p.maxchunks > 1) {
         const int msmem = p.maxchunks * qsa::kMaxChosen * 8;

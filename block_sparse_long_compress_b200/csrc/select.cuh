@@ -249,15 +249,151 @@ __device__ void select_and_emit(const uint64_t *keys, int n, int need, SelectSha
     }
 }
 
+// ------------------------------------------ warp-level top-64 lists
+// Per-token rows select from short chunks (a few hundred candidates per
+// CTA), where the radix passes' barriers dominate.  There each warp sorts 64
+// keys in registers with a bitonic network (element e = 32 r + lane in
+// register r: a for r = 0, b for r = 1; 21 compare-exchange stages, strides
+// below 32 through shuffles), and two sorted lists are cut to the top 64 of
+// their union by one elementwise maximum against the other list reversed,
+// which leaves a bitonic sequence, and a 6-stage bitonic merge.  Keys are
+// unique, so every list is the exact top 64 by key; padding is key 0, below
+// every candidate's key.
+__device__ __forceinline__ uint64_t max64(uint64_t x, uint64_t y) { return x > y ? x : y; }
+__device__ __forceinline__ uint64_t min64(uint64_t x, uint64_t y) { return x < y ? x : y; }
+
+// One stage (block size k, stride j < 32) of a descending bitonic network.
+__device__ __forceinline__ void bitonic_stage(uint64_t &a, uint64_t &b, int k, int j)
+{
+    const int lane = threadIdx.x & 31;
+    const uint64_t pa = __shfl_xor_sync(0xffffffffu, a, j);
+    const uint64_t pb = __shfl_xor_sync(0xffffffffu, b, j);
+    const bool lower = (lane & j) == 0;
+    // the lower element of a pair keeps the maximum in a descending block
+    const bool max_a = lower == ((lane & k) == 0);
+    const bool max_b = lower == (((32 + lane) & k) == 0);
+    a = max_a ? max64(a, pa) : min64(a, pa);
+    b = max_b ? max64(b, pb) : min64(b, pb);
+}
+
+// Sorts the warp's 64 keys descending.
+__device__ __forceinline__ void warp_sort64_desc(uint64_t &a, uint64_t &b)
+{
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) bitonic_stage(a, b, k, j);
+    }
+    // k = 64: the whole list descending
+    const uint64_t hi = max64(a, b), lo = min64(a, b);
+    a = hi;
+    b = lo;
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) bitonic_stage(a, b, 64, j);
+}
+
+// A bitonic sequence of 64 keys -> descending.
+__device__ __forceinline__ void warp_merge64_desc(uint64_t &a, uint64_t &b)
+{
+    const uint64_t hi = max64(a, b), lo = min64(a, b);
+    a = hi;
+    b = lo;
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) bitonic_stage(a, b, 64, j);
+}
+
+// (a, b) := the top 64 of the union of two descending lists (a, b) and
+// (x, y), descending.
+__device__ __forceinline__ void warp_top64_union(uint64_t &a, uint64_t &b, uint64_t x, uint64_t y)
+{
+    const int lane = threadIdx.x & 31;
+    // element e of the other list reversed is its element 63 - e
+    a = max64(a, __shfl_sync(0xffffffffu, y, 31 - lane));
+    b = max64(b, __shfl_sync(0xffffffffu, x, 31 - lane));
+    warp_merge64_desc(a, b);
+}
+
+// Top 64 (descending, padded with 0) of the n keys keys[0..n): each warp
+// folds batches of 64 into a running list (a batch with no key above the
+// list's 64th is skipped), then the warps' lists meet in a tree through
+// `scratch` (8 x 64 keys), one block barrier per level.  The result is in
+// warp 0's registers.  Every thread of the CTA calls it.
+__device__ void cta_top64(const uint64_t *keys, int n, uint64_t *scratch, uint64_t &a_out, uint64_t &b_out)
+{
+    constexpr int NW = kSelThreads / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nbatch = (n + 63) / 64;
+    const int nl = min(nbatch, NW);       // warps that hold a list
+    uint64_t a = 0, b = 0;
+    if (warp < nl) {
+        bool first = true;
+        for (int bt = warp; bt < nbatch; bt += NW) {
+            const int e0 = bt * 64;
+            uint64_t x = e0 + lane < n ? keys[e0 + lane] : 0;
+            uint64_t y = e0 + 32 + lane < n ? keys[e0 + 32 + lane] : 0;
+            if (!first) {
+                const uint64_t thr = __shfl_sync(0xffffffffu, b, 31);
+                if (!__any_sync(0xffffffffu, x > thr || y > thr)) continue;
+            }
+            warp_sort64_desc(x, y);
+            if (first) {
+                a = x;
+                b = y;
+                first = false;
+            } else {
+                warp_top64_union(a, b, x, y);
+            }
+        }
+    }
+    for (int step = 1; step < nl; step <<= 1) {
+        // writers of this level and readers of the previous one use
+        // different slots, so one barrier per level suffices
+        if (warp < nl && (warp & (2 * step - 1)) == step) {
+            scratch[warp * 64 + lane] = a;
+            scratch[warp * 64 + 32 + lane] = b;
+        }
+        __syncthreads();
+        if ((warp & (2 * step - 1)) == 0 && warp + step < nl) {
+            const uint64_t *y = scratch + (warp + step) * 64;
+            a = max64(a, y[63 - lane]);
+            b = max64(b, y[31 - lane]);
+            warp_merge64_desc(a, b);
+        }
+    }
+    a_out = a;
+    b_out = b;
+}
+
+// Warp 0 (holding the row's top-64 keys, descending): writes the row's
+// indices -- 0, the m best candidates in ascending block order, D (if
+// D > 0), then -1 -- by sorting the m block ids ascending in registers.
+__device__ __forceinline__ void warp_emit_row(uint64_t a, uint64_t b, int m, int32_t *row, int D, int topk)
+{
+    const int lane = threadIdx.x & 31;
+    // ascending ids = descending complements; unused slots sort last
+    uint64_t x = lane < m ? (uint64_t)(0xFFFFFFFFu - (uint32_t)key_block(a)) : 0;
+    uint64_t y = 32 + lane < m ? (uint64_t)(0xFFFFFFFFu - (uint32_t)key_block(b)) : 0;
+    warp_sort64_desc(x, y);
+    if (lane < m) row[1 + lane] = (int)(0xFFFFFFFFu - (uint32_t)x);
+    if (32 + lane < m) row[33 + lane] = (int)(0xFFFFFFFFu - (uint32_t)y);
+    for (int s = lane; s < topk; s += 32) {
+        if (s == 0) row[0] = 0;
+        else if (s == m + 1 && D > 0) row[s] = D;
+        else if (s > m + (D > 0 ? 1 : 0)) row[s] = -1;
+    }
+}
+
 // First query position of sequence b: q_pos0, or q_pos[b] for a ragged
-// batch (device data, checked: a multiple of 64 with the chunk of Tq tokens
-// inside the summaries' capacity; otherwise QSA_ERR_BOUNDS and position 0).
+// batch (device data, checked: a multiple of 64, at most q_pos0 -- the
+// launch is planned for that furthest position -- and with the chunk of Tq
+// tokens inside the summaries' capacity; otherwise QSA_ERR_BOUNDS and
+// position 0).
 __device__ __forceinline__ int seq_q_pos(const int32_t *q_pos, int b, int q_pos0, int Tq, int nblk_max,
                                          bool reporter)
 {
     if (!q_pos) return q_pos0;
     const int qp = __ldg(q_pos + b);
-    if (qp < 0 || (qp & 63) || (long)qp + Tq > 64L * nblk_max) {
+    if (qp < 0 || (qp & 63) || qp > q_pos0 || (long)qp + Tq > 64L * nblk_max) {
         if (reporter) report(QSA_ERR_BOUNDS, 10);
         return 0;
     }
@@ -371,6 +507,55 @@ __device__ __forceinline__ void score_chunk(const float *qb, const KcT *__restri
     }
 }
 
+// Per-token rows: this lane's columns [lane*V, lane*V+V) of the pooled query
+// -- the fp32 sum over the token's G head rows (qt: the group's first head),
+// in head order, times 1/G -- in registers, so that no block barrier stands
+// between the query's loads and the first summary loads.
+template <int D>
+__device__ __forceinline__ void pooled_query_lane(const __nv_bfloat16 *__restrict__ qt, int G, float (&q)[D / 32])
+{
+    constexpr int V = D / 32;
+    const int lane = threadIdx.x & 31;
+    float acc[V];
+#pragma unroll
+    for (int v = 0; v < V; v++) acc[v] = 0.f;
+    for (int h = 0; h < G; h++) {
+        float x[V];
+        load_summary<V>(qt + (long)h * D + lane * V, x);   // bf16 widened exactly
+#pragma unroll
+        for (int v = 0; v < V; v++) acc[v] += x[v];
+    }
+    const float inv = 1.0f / (float)G;
+#pragma unroll
+    for (int v = 0; v < V; v++) q[v] = acc[v] * inv;
+}
+
+// score_chunk with the pooled query in registers (pooled_query_lane).
+template <int D, typename KcT>
+__device__ __forceinline__ void score_chunk_q(const float (&q)[D / 32], const KcT *__restrict__ kc, int n, int j0,
+                                              float sm_scale, uint64_t *keys)
+{
+    constexpr int V = D / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const KcT *kc_base = kc + lane * V;
+    for (int base = warp * 8; base < n; base += 8 * (kSelThreads / 32)) {
+        float s[8];
+#pragma unroll
+        for (int c = 0; c < 8; c++) {
+            s[c] = 0.f;
+            if (base + c < n) {
+                float k[V];
+                load_summary<V>(kc_base + (long)(base + c) * D, k);
+                if constexpr (V == 4) s[c] = q[0] * k[0] + q[1] * k[1] + q[2] * k[2] + q[3] * k[3];
+                else s[c] = q[0] * k[0] + q[1] * k[1];
+            }
+        }
+        const float dot = reduce8(s);
+        const int e = base + (lane >> 2);
+        if ((lane & 3) == 0 && e < n) keys[e] = make_key(dot * sm_scale, j0 + e);
+    }
+}
+
 // Per-head logits of n blocks (summaries kc[0..n)) for the G <= 8 heads of
 // a group (queries qh[h][0..D), fp32): for every block e, f(e, z) receives
 // z[h] = scale * <qh[h], kc[e]> for h < G, in the lane that holds them
@@ -437,7 +622,7 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
     const float *__restrict__ Qbar, const KcT *__restrict__ Kc, int32_t *__restrict__ idx,
     uint64_t *__restrict__ part, int nblk_max, int Tq, int q_pos0, int qblk, int topk,
     float sm_scale, int CH, int maxchunks, int Hkv, const int32_t *__restrict__ q_pos,
-    const float *__restrict__ scores = nullptr)
+    const float *__restrict__ scores = nullptr, int score_stride = 0)
 {
     extern __shared__ uint64_t keys[];
     __shared__ SelectShared sh;
@@ -451,7 +636,7 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
     const long row = (long)bg * NR + i;
 
     if constexpr (FROM_SCORES) {
-        const float *srow = scores + row * nblk_max + j0;
+        const float *srow = scores + row * (score_stride ? score_stride : nblk_max) + j0;
         for (int e = threadIdx.x; e < n; e += kSelThreads) keys[e] = make_key(__ldg(srow + e), j0 + e);
     } else {
         score_chunk<D, KcT>(Qbar + row * D, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
@@ -464,6 +649,91 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
     } else {
         select_and_emit(keys, n, need, sh, nullptr, g.D, topk,
                         part + (row * maxchunks + chunk) * kMaxChosen);
+    }
+}
+
+// ---------------------------------------------- prefill rows: score table
+// Consecutive prefill rows of one (b, g) share almost all their candidates
+// (row i's are blocks 1 .. D_i - 1), so the scores of a 64-row x 64-candidate
+// tile are an fp32 matrix product Qbar_tile (64 x D) * Kc_tile^T (D x 64)
+// over shared memory: every summary and pooled query crosses L2 once per
+// tile instead of once per row.  Each thread forms a 4 x 4 block of dots
+// (rows 4 ty .. 4 ty + 3, candidates tx, tx + 16, tx + 32, tx + 48) with
+// fp32 FMAs in increasing d; rows are padded to D + 4 floats so the
+// 16-byte shared loads of the 16 candidate columns a warp reads fall in
+// distinct banks.  The scores go into a table [B*Hkv][NR][stride] that
+// score_select_kernel<.., true> selects from; tiles wholly past their rows'
+// diagonals exit at once.
+// grid (ceil(max candidates / 64), ceil(NR / 64), B*Hkv); 256 threads;
+// dynamic shared memory 2 * 64 * (D + 4) * 4 bytes.
+constexpr int kTableTile = 64;
+
+template <int D, typename KcT>
+__global__ void __launch_bounds__(256) score_table_kernel(
+    const float *__restrict__ Qbar, const KcT *__restrict__ Kc, float *__restrict__ table, int nblk_max, int Tq,
+    int q_pos0, int stride, float sm_scale, int Hkv, const int32_t *__restrict__ q_pos)
+{
+    constexpr int T = kTableTile, LD = D + 4;
+    extern __shared__ __align__(16) float tsm[];
+    float *qs = tsm;            // [T][LD] pooled queries of the tile's rows
+    float *ks = tsm + T * LD;   // [T][LD] summaries of the tile's candidates
+    const int bg = blockIdx.z, NR = (Tq + 63) / 64;
+    const int qp = seq_q_pos(q_pos, bg / Hkv, q_pos0, Tq, nblk_max, false);
+    const int r0 = blockIdx.y * T, nr = min(T, NR - r0);
+    const int j0 = 1 + blockIdx.x * T;
+    // candidates of the tile that some row of it has (j < D of its last row)
+    const int Dlast = (qp + min((r0 + nr) * 64, Tq) - 1) / 64;
+    const int nc = min(T, Dlast - j0);
+    if (nc <= 0) return;
+    const int tid = threadIdx.x;
+    // tiles into shared memory: 16-byte chunks, rows past the tile are zero
+    constexpr int CPR = D / 4;   // 16-byte chunks (of fp32) per row
+    for (int e = tid; e < T * CPR; e += 256) {
+        const int rr = e / CPR, c = e % CPR;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (rr < nr) v = *reinterpret_cast<const float4 *>(Qbar + ((long)bg * NR + r0 + rr) * D + 4 * c);
+        *reinterpret_cast<float4 *>(qs + rr * LD + 4 * c) = v;
+        float k4[4] = {0.f, 0.f, 0.f, 0.f};
+        if (rr < nc) load_summary<4>(Kc + ((long)bg * nblk_max + j0 + rr) * D + 4 * c, k4);
+        *reinterpret_cast<float4 *>(ks + rr * LD + 4 * c) = make_float4(k4[0], k4[1], k4[2], k4[3]);
+    }
+    __syncthreads();
+    const int ty = tid >> 4, tx = tid & 15;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; i++)
+#pragma unroll
+        for (int jj = 0; jj < 4; jj++) acc[i][jj] = 0.f;
+    const float *qrow = qs + (4 * ty) * LD;
+    const float *krow = ks + tx * LD;
+#pragma unroll 4
+    for (int d = 0; d < D; d += 4) {
+        float4 a[4], b[4];
+#pragma unroll
+        for (int i = 0; i < 4; i++) a[i] = *reinterpret_cast<const float4 *>(qrow + i * LD + d);
+#pragma unroll
+        for (int jj = 0; jj < 4; jj++) b[jj] = *reinterpret_cast<const float4 *>(krow + 16 * jj * LD + d);
+#pragma unroll
+        for (int i = 0; i < 4; i++)
+#pragma unroll
+            for (int jj = 0; jj < 4; jj++) {
+                acc[i][jj] = fmaf(a[i].x, b[jj].x, acc[i][jj]);
+                acc[i][jj] = fmaf(a[i].y, b[jj].y, acc[i][jj]);
+                acc[i][jj] = fmaf(a[i].z, b[jj].z, acc[i][jj]);
+                acc[i][jj] = fmaf(a[i].w, b[jj].w, acc[i][jj]);
+            }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const int rr = 4 * ty + i;
+        if (rr >= nr) break;
+        const int Drow = (qp + min((r0 + rr + 1) * 64, Tq) - 1) / 64;
+        float *trow = table + ((long)bg * NR + r0 + rr) * stride + j0;
+#pragma unroll
+        for (int jj = 0; jj < 4; jj++) {
+            const int e = tx + 16 * jj;
+            if (e < nc && j0 + e < Drow) trow[e] = acc[i][jj] * sm_scale;
+        }
     }
 }
 
@@ -513,12 +783,11 @@ __device__ __forceinline__ void select_token_body(
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     extern __shared__ uint64_t keys[];                 // [CH] this chunk's keys
-    __shared__ SelectShared sh;
-    __shared__ uint64_t lists[8 * kMaxChosen];         // leader: the chunks' top-m lists
-    __shared__ __align__(16) float qbar[D];
+    __shared__ uint64_t scratch[8 * 64];               // the warps' top-64 lists meeting in a tree
+    __shared__ uint64_t lists[8 * 64];                 // leader: the chunks' top-64 lists
     const int NCH = (int)cluster.num_blocks();
     const int chunk = (int)cluster.block_rank();
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int i = blockIdx.y, bg = blockIdx.z, NR = gridDim.y;
     const int b = bg / Hkv, grp = bg % Hkv, G = Hq / Hkv;
     const long row = (long)bg * NR + i;
@@ -534,17 +803,6 @@ __device__ __forceinline__ void select_token_body(
     }
     const RowGeom g = row_geom(i, Tq, qp, 1, topk, CH);
 
-    if constexpr (!SOFTMAX) {
-        // pooled query: mean of the token's query over the group's heads
-        const __nv_bfloat16 *qt = Q + (((long)b * Tq + i) * Hq + (long)grp * G) * D;
-        const float inv = 1.0f / (float)G;
-        for (int c = tid; c < D; c += kSelThreads) {
-            float s = 0.f;
-            for (int h = 0; h < G; h++) s += __bfloat162float(qt[(long)h * D + c]);
-            qbar[c] = s * inv;
-        }
-        __syncthreads();
-    }
     const int j0 = 1 + chunk * CH;
     const int n = max(0, min(CH, g.ncand - chunk * CH));
     if constexpr (SOFTMAX) {
@@ -567,7 +825,6 @@ __device__ __forceinline__ void select_token_body(
         if (g.ncand > 0) {
             const int js = chunk == 0 ? 0 : j0;
             const int ns = n + (j0 - js);
-            const int lane = tid & 31, warp = tid >> 5;
             // logits kept in shared memory after the keys when the chunk is
             // short enough (kSoftmaxZCap), else recomputed in pass 2
             const bool zsm = CH <= kSoftmaxZCap;
@@ -656,21 +913,49 @@ __device__ __forceinline__ void select_token_body(
             }
         }
     } else {
-        score_chunk<D, KcT>(qbar, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
+        // pooled query: mean of the token's query over the group's heads
+        float q[D / 32];
+        pooled_query_lane<D>(Q + (((long)b * Tq + i) * Hq + (long)grp * G) * D, G, q);
+        score_chunk_q<D, KcT>(q, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
     }
     __syncthreads();
-    const int need = min(g.m, n);
+    // the chunk's top 64 (the row keeps at most 62 candidates)
+    uint64_t a, bk;
+    cta_top64(keys, n, scratch, a, bk);
     if (g.nchunks == 1) {
         // chunk 0 holds every candidate of the row (the other CTAs only
-        // scored nothing): select directly, no cluster exchange
-        if (chunk == 0) select_and_emit(keys, n, need, sh, idx + row * topk, g.D, topk, nullptr);
+        // scored nothing): emit directly, no cluster exchange
+        if (chunk == 0 && warp == 0) warp_emit_row(a, bk, g.m, idx + row * topk, g.D, topk);
         return;
     }
-    uint64_t *dst = cluster.map_shared_rank(lists, 0) + chunk * kMaxChosen;
-    select_and_emit(keys, n, need, sh, nullptr, g.D, topk, dst);
-    for (int e = need + tid; e < kMaxChosen; e += kSelThreads) dst[e] = 0;
+    if (warp == 0) {
+        // this chunk's list into the leader's shared memory
+        uint64_t *dst = cluster.map_shared_rank(lists, 0) + chunk * 64;
+        dst[lane] = a;
+        dst[32 + lane] = bk;
+    }
     cluster.sync();   // every list is in the leader
-    if (chunk == 0) select_and_emit(lists, NCH * kMaxChosen, g.m, sh, idx + row * topk, g.D, topk, nullptr);
+    if (chunk != 0) return;
+    // the leader: the chunks' lists meet in a tree (warp c starts from list c)
+    a = bk = 0;
+    if (warp < NCH) {
+        a = lists[warp * 64 + lane];
+        bk = lists[warp * 64 + 32 + lane];
+    }
+    for (int step = 1; step < NCH; step <<= 1) {
+        if (warp < NCH && (warp & (2 * step - 1)) == step) {
+            scratch[warp * 64 + lane] = a;
+            scratch[warp * 64 + 32 + lane] = bk;
+        }
+        __syncthreads();
+        if ((warp & (2 * step - 1)) == 0 && warp + step < NCH) {
+            const uint64_t *y = scratch + (warp + step) * 64;
+            a = max64(a, y[63 - lane]);
+            bk = max64(bk, y[31 - lane]);
+            warp_merge64_desc(a, bk);
+        }
+    }
+    if (warp == 0) warp_emit_row(a, bk, g.m, idx + row * topk, g.D, topk);
 }
 
 template <int D, typename KcT>

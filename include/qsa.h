@@ -238,7 +238,9 @@ QSA_API qsa_status qsa_decode(const void *q, const void *K_cache, const void *V_
  * qsa_score_select_ragged_prefill: qsa_score_select with qblk = 64 and each
  * sequence at its own position; max_pos (a multiple of 64, >= every
  * q_pos[b]) sizes the launch and the workspace
- * (qsa_score_select_workspace(B, Hq, Hkv, Tq, max_pos, 64, d, topk)).
+ * (qsa_score_select_workspace(B, Hq, Hkv, Tq, max_pos, 64, d, topk)); a
+ * q_pos[b] above max_pos is an invalid position (QSA_ERR_BOUNDS, the
+ * sequence treated as starting at 0).
  * qsa_sparse_attn_prefill_paged: qsa_sparse_attn_prefill over the pages,
  * each sequence at its own position.
  */

@@ -133,6 +133,30 @@ def test_paged_bounds_are_reported(qsa):
     assert _status(qsa)[0] == "QSA_OK"
 
 
+def test_ragged_prefill_position_past_the_plan_is_reported(qsa):
+    """A chunk position above the max_pos the selection was planned for
+    (device data) is reported as QSA_ERR_BOUNDS -- the row's scores would
+    not fit the score table sized for max_pos -- and that sequence is
+    treated as starting at 0; the other sequences are selected as usual."""
+    B, Tq, Hq, Hkv, d, topk, max_blocks = 2, 128, 8, 2, 64, 6, 64
+    g = torch.Generator(device=DEV)
+    g.manual_seed(5)
+    Q = torch.randn((B, Tq, Hq, d), generator=g, device=DEV).to(torch.bfloat16)
+    Kc = torch.randn((B, Hkv, max_blocks, d), generator=g, device=DEV) / 8
+    idx = torch.full((B, Hkv, 2, topk), -7, dtype=torch.int32, device=DEV)
+    good = torch.tensor([64 * 20, 64 * 30], dtype=torch.int32, device=DEV)
+    qsa.score_select_ragged_prefill(Q, Kc, good, idx, topk, 64 * 30)
+    assert _status(qsa)[0] == "QSA_OK"
+    ref = idx.clone()
+    past = torch.tensor([64 * 20, 64 * 40], dtype=torch.int32, device=DEV)   # 64 * 40 > max_pos
+    idx.fill_(-7)
+    qsa.score_select_ragged_prefill(Q, Kc, past, idx, topk, 64 * 30)
+    assert _status(qsa)[0] == "QSA_ERR_BOUNDS"
+    assert torch.equal(idx[0], ref[0])                     # the valid sequence is untouched by the error
+    assert (idx[1, :, :, 0] == 0).all()                    # the invalid one keeps the sink
+    assert _status(qsa)[0] == "QSA_OK"
+
+
 PREFILL_CASES = [
     # name, chunk start per sequence (multiples of 64), Tq, Hq, Hkv, d, topk
     ("d128_g8", [64 * 40, 64 * 100, 0], 192, 16, 2, 128, 8),
