@@ -68,6 +68,12 @@ def _load():
         "qsa_decode_fp8": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "qsa_decode_fp8_paged": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "qsa_sparse_attn_prefill_paged": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P]),
+        "qsa_select_local_lists": (I, [I, I, I, I]),
+        "qsa_score_select_local_workspace": (S, [I, I, I, I, I, I, I, I]),
+        "qsa_score_select_local": (I, [P, P, P, I, I, I, I, I, I, I, I, I, I, F, P, S, P]),
+        "qsa_merge_select_lists": (I, [P, P, I, I, I, I, I, I, I, P]),
+        "qsa_sparse_attn_prefill_local": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, F, P]),
+        "qsa_merge_partials": (I, [P, P, P, P, I, ctypes.c_int64, I, P]),
         "qsa_get_device_status": (I, [P, ctypes.POINTER(I)]),
         "qsa_selftest_wait_timeout": (I, [ctypes.c_uint64, P]),
         "qsa_selftest_exp2": (I, [P, P, I, P]),
@@ -439,6 +445,141 @@ class QSADecodePaged:
         decode_paged(q, K_pages, V_pages, block_table, seq_lens, self.idx, self.o, self.sm_scale,
                      stream)
         return self.o
+
+
+# ----------------------------------- one sequence over several GPUs
+def shard_ranges(n_blocks, world):
+    """Contiguous block ranges [lo, hi) of a cache of n_blocks blocks split
+    over `world` ranks, as equal as possible, in rank order."""
+    if world <= 0 or n_blocks < world:
+        raise ValueError("need at least one block per rank")
+    base, extra = divmod(n_blocks, world)
+    out, lo = [], 0
+    for r in range(world):
+        hi = lo + base + (1 if r < extra else 0)
+        out.append((lo, hi))
+        lo = hi
+    return out
+
+
+def select_local_lists(Tq, q_pos0, blk_lo, blk_hi):
+    """Lists per selection row a rank holding blocks [blk_lo, blk_hi) emits."""
+    return int(_lib.qsa_select_local_lists(Tq, q_pos0, blk_lo, blk_hi))
+
+
+def score_select_local_workspace(B, Hq, Hkv, Tq, q_pos0, d, blk_lo, blk_hi):
+    return int(_lib.qsa_score_select_local_workspace(B, Hq, Hkv, Tq, q_pos0, d, blk_lo, blk_hi))
+
+
+def score_select_local(Q, Kc_local, lists, q_pos0, blk_lo, blk_hi, topk, sm_scale=None, workspace=None,
+                       stream=None):
+    """A rank's candidate lists for prefill rows (64-token blocks) over its
+    own blocks [blk_lo, blk_hi).  Q bf16 [B, Tq, Hq, d]; Kc_local fp32
+    [B, Hkv, blk_hi - blk_lo, d]; lists int64 (uint64 keys) [B, Hkv, NR,
+    nlists, 62] (written)."""
+    B, Tq, Hq, d = Q.shape
+    Hkv = Kc_local.shape[1]
+    nlists = lists.shape[3]
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    need = score_select_local_workspace(B, Hq, Hkv, Tq, q_pos0, d, blk_lo, blk_hi)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=Q.device)
+    _check(_lib.qsa_score_select_local(_ptr(Q, torch.bfloat16, "Q"), _ptr(Kc_local, torch.float32, "Kc_local"),
+                                       _ptr(lists, torch.int64, "lists"), B, Hq, Hkv, Tq, q_pos0, blk_lo, blk_hi,
+                                       nlists, d, topk, float(sm_scale), _ptr(workspace, torch.uint8, "workspace"),
+                                       workspace.numel(), _stream(stream)), "qsa_score_select_local")
+    return lists
+
+
+def merge_select_lists(lists, idx, Tq, q_pos0, stream=None):
+    """Selection from all ranks' gathered lists ([R, B, Hkv, NR, nlists, 62]
+    int64, rank-major) of a chunk of Tq tokens at q_pos0 into idx int32
+    [B, Hkv, NR, topk]."""
+    R, B, Hkv, NR, nlists, _ = lists.shape
+    if NR != -(-Tq // BLOCK):
+        raise ValueError("lists do not match Tq")
+    topk = idx.shape[-1]
+    _check(_lib.qsa_merge_select_lists(_ptr(lists, torch.int64, "lists"), _ptr(idx, torch.int32, "idx"), B, Hkv,
+                                       Tq, q_pos0, R, nlists, topk, _stream(stream)), "qsa_merge_select_lists")
+    return idx
+
+
+def sparse_attn_prefill_local(Q, K_local, V_local, idx, O, lse, q_pos0, blk_lo, blk_hi, sm_scale=None, stream=None):
+    """Attention over the listed blocks this rank holds ([blk_lo, blk_hi),
+    block j at row 64 (j - blk_lo) of K_local / V_local bf16 [B, Hkv,
+    T_local, d]); O bf16 [B, Tq, Hq, d] and lse fp32 [B, Tq, Hq] over the
+    rank's keys (0 and -inf where it holds none of a row's blocks)."""
+    B, Tq, Hq, d = Q.shape
+    _, Hkv, T_local, _ = K_local.shape
+    topk = idx.shape[-1]
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    _check(_lib.qsa_sparse_attn_prefill_local(
+        _ptr(Q, torch.bfloat16, "Q"), _ptr(K_local, torch.bfloat16, "K_local"),
+        _ptr(V_local, torch.bfloat16, "V_local"), _ptr(idx, torch.int32, "idx"), _ptr(O, torch.bfloat16, "O"),
+        _ptr(lse, torch.float32, "lse"), B, Hq, Hkv, Tq, q_pos0, T_local, blk_lo, blk_hi, d, topk,
+        float(sm_scale), _stream(stream)), "qsa_sparse_attn_prefill_local")
+    return O, lse
+
+
+def merge_partials(O_parts, lse_parts, O, lse=None, stream=None):
+    """O = sum_r exp(lse_r - L) O_r, L = logsumexp_r lse_r.  O_parts bf16
+    [R, ..., d]; lse_parts fp32 [R, ...]; O bf16 [..., d]; lse fp32 [...]."""
+    R = O_parts.shape[0]
+    d = O_parts.shape[-1]
+    rows = lse_parts[0].numel()
+    _check(_lib.qsa_merge_partials(_ptr(O_parts, torch.bfloat16, "O_parts"), _ptr(lse_parts, torch.float32, "lse_parts"),
+                                   _ptr(O, torch.bfloat16, "O"), _ptr(lse, torch.float32, "lse"), R, rows, d,
+                                   _stream(stream)), "qsa_merge_partials")
+    return O
+
+
+def all_gather_rank_major(t, group=None):
+    """[R, *t.shape]: every rank's tensor in rank order (a collective:
+    every rank of the group calls it with a tensor of the same shape)."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    parts = [torch.empty_like(t) for _ in range(world)]
+    dist.all_gather(parts, t.contiguous(), group=group)
+    return torch.stack(parts)
+
+
+class QSAShardedPrefill:
+    """A chunked prefill of one sequence whose cache is split over the ranks
+    of a process group (one GPU each): rank r holds the cache blocks
+    blk_ranges[r] (contiguous, ascending in rank order; the last rank's range
+    ends with the chunk's own blocks) with their summaries, and the whole Q.
+    A step: the rank's candidate lists, an all-gather of the lists (a few
+    KB), the merged selection (identical on every rank), attention over the
+    rank's selected blocks, an all-gather of the partial outputs and their
+    log-sum-exp merge.  Every rank gets the full output."""
+
+    def __init__(self, B, Tq, Hq, Hkv, d, topk, q_pos0, blk_ranges, rank, group=None, device="cuda"):
+        self.B, self.Tq, self.Hq, self.Hkv, self.d = B, Tq, Hq, Hkv, d
+        self.topk, self.q_pos0, self.rank, self.group = topk, q_pos0, rank, group
+        self.sm_scale = d ** -0.5
+        self.blk_lo, self.blk_hi = blk_ranges[rank]
+        self.nlists = max(select_local_lists(Tq, q_pos0, lo, hi) for lo, hi in blk_ranges)
+        NR = -(-Tq // BLOCK)
+        dev = torch.device(device)
+        self.lists = torch.empty((B, Hkv, NR, self.nlists, 62), dtype=torch.int64, device=dev)
+        self.ws = torch.empty(max(16, score_select_local_workspace(B, Hq, Hkv, Tq, q_pos0, d, self.blk_lo,
+                                                                    self.blk_hi)), dtype=torch.uint8, device=dev)
+        self.idx = torch.empty((B, Hkv, NR, topk), dtype=torch.int32, device=dev)
+        self.O_part = torch.empty((B, Tq, Hq, d), dtype=torch.bfloat16, device=dev)
+        self.lse_part = torch.empty((B, Tq, Hq), dtype=torch.float32, device=dev)
+        self.O = torch.empty((B, Tq, Hq, d), dtype=torch.bfloat16, device=dev)
+
+    def __call__(self, Q, K_local, V_local, Kc_local, stream=None):
+        score_select_local(Q, Kc_local, self.lists, self.q_pos0, self.blk_lo, self.blk_hi, self.topk,
+                           self.sm_scale, self.ws, stream)
+        merge_select_lists(all_gather_rank_major(self.lists, self.group), self.idx, self.Tq, self.q_pos0, stream)
+        sparse_attn_prefill_local(Q, K_local, V_local, self.idx, self.O_part, self.lse_part, self.q_pos0,
+                                  self.blk_lo, self.blk_hi, self.sm_scale, stream)
+        merge_partials(all_gather_rank_major(self.O_part, self.group),
+                       all_gather_rank_major(self.lse_part, self.group), self.O, None, stream)
+        return self.O
 
 
 def device_status(stream=None):

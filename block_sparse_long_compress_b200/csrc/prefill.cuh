@@ -136,7 +136,8 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
     const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ idx,
     __nv_bfloat16 *__restrict__ O, float *__restrict__ lse, int Tq, int Hq, int Hkv, int BH,
     int q_pos0, int T_kv_max, int topk, float sm_scale_log2, const int32_t *__restrict__ q_pos,
-    const int32_t *__restrict__ block_table, int max_blocks, int num_pages)
+    const int32_t *__restrict__ block_table, int max_blocks, int num_pages, int blk_lo, int blk_hi,
+    int partial)
 {
     using C = PrefillCfg<D, G>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -221,7 +222,9 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
             if (k >= 2 && !wait_all(&sh.list_empty[slot], ((k >> 1) - 1) & 1, 12)) break;
             // the row's list, one entry per lane: it ends at the first -1;
             // an index past the diagonal or not above its predecessor is an
-            // error and ends it too
+            // error and ends it too.  Listed blocks outside [blk_lo, blk_hi)
+            // belong to another rank's cache and are skipped; an owned
+            // block j is cache block j - blk_lo of this rank.
             const int32_t *sel = idx + ((long)w.bg * NR + w.i) * topk;
             int n = 0, prev = -1, lastj = -1;
             bool bad = false;
@@ -231,22 +234,24 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
                 int jp = __shfl_up_sync(0xffffffffu, j, 1);
                 if (lane == 0) jp = prev;
                 bool stop_bad = j >= 0 && (j > Dg || (s > 0 && j <= jp));
+                const bool owned = j >= blk_lo && j < blk_hi;
                 int row = 0;
-                if (j >= 0 && !stop_bad) {
+                if (j >= 0 && !stop_bad && owned) {
                     if (block_table) {
                         const int page = __ldg(block_table + (long)b * max_blocks + j);
                         if (page < 0 || page >= num_pages) stop_bad = true;
                         else row = (page * Hkv + g) * 64;   // host checks num_pages*Hkv*64 < 2^31
                     } else {
-                        row = (int)(kv_row0 + 64L * j);
+                        row = (int)(kv_row0 + 64L * (j - blk_lo));
                     }
                 }
                 const unsigned stops = __ballot_sync(0xffffffffu, j < 0 || stop_bad);
                 const int f = stops ? __ffs(stops) - 1 : 32;
-                if (lane < f) sh.rows[slot][s] = row;
-                const int jl = __shfl_sync(0xffffffffu, j, f > 0 ? f - 1 : 0);
-                if (f > 0) lastj = jl;
-                n = r0 + f;
+                const bool keep = lane < f && owned;
+                const unsigned kept = __ballot_sync(0xffffffffu, keep);
+                if (keep) sh.rows[slot][n + __popc(kept & ((1u << lane) - 1u))] = row;
+                if (kept) lastj = __shfl_sync(0xffffffffu, j, 31 - __clz(kept));
+                n += __popc(kept);
                 if (stops) {
                     bad = __shfl_sync(0xffffffffu, stop_bad, f);
                     break;
@@ -257,8 +262,9 @@ __global__ void __launch_bounds__(12 * 32, 1) sparse_attn_prefill_kernel(
                 if (bad) report(QSA_ERR_BOUNDS, 1);
                 if (n == 0) {
                     // no valid block: block 0 goes through the pipeline (in
-                    // bounds) and the epilogue writes zeros
-                    report(QSA_ERR_BOUNDS, 2);
+                    // bounds) and the epilogue writes zeros -- an error,
+                    // unless this rank owns none of a row's blocks (partial)
+                    if (!partial) report(QSA_ERR_BOUNDS, 2);
                     lastj = 0;
                     int row0 = (int)kv_row0;
                     if (block_table) {

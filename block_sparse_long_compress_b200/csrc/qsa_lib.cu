@@ -9,6 +9,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <climits>
 #include <mutex>
 
 #include "../../include/qsa.h"
@@ -239,10 +240,18 @@ struct Paging {
     int max_blocks = 0, num_pages = 0;
 };
 
+// A rank's share of a sharded cache: the blocks [lo, hi) it holds (block j
+// at row 64 (j - lo) of its cache); partial: rows with none of their blocks
+// here are not an error (O = 0, lse = -inf).  The default is the whole cache.
+struct Ownership {
+    int lo = 0, hi = INT_MAX, partial = 0;
+};
+
 template <int D, int G>
 qsa_status launch_prefill(const void *Q, const void *K, const void *V, const int32_t *idx, void *O,
                           float *lse, int B, int Hq, int Hkv, int Tq, int q_pos0, int T_kv_max,
-                          int topk, float sm_scale, cudaStream_t s, const Paging &pg = Paging())
+                          int topk, float sm_scale, cudaStream_t s, const Paging &pg = Paging(),
+                          const Ownership &own = Ownership())
 {
     using C = qsa::PrefillCfg<D, G>;
     CUtensorMap mq, mk, mv;
@@ -273,7 +282,7 @@ qsa_status launch_prefill(const void *Q, const void *K, const void *V, const int
     kern<<<grid, C::THREADS, C::SMEM_REQUEST, s>>>(mq, mk, mv, idx, (__nv_bfloat16 *)O, lse, Tq, Hq, Hkv,
                                                    B * Hkv, q_pos0, T_kv_max, topk,
                                                    sm_scale * 1.4426950408889634f, pg.q_pos, pg.block_table,
-                                                   pg.max_blocks, pg.num_pages);
+                                                   pg.max_blocks, pg.num_pages, own.lo, own.hi, own.partial);
     return launched("sparse_attn_prefill_kernel");
 }
 
@@ -481,7 +490,7 @@ qsa_status launch_score_select(const void *Q, const KcT *Kc, int32_t *idx, float
         const int tsmem = 2 * TT * (D + 4) * (int)sizeof(float);
         if ((st = set_smem(qsa::score_table_kernel<D, KcT>, tsmem)) != QSA_OK) return st;
         qsa::score_table_kernel<D, KcT><<<tgrid, 256, tsmem, s>>>(Qbar, Kc, table, nblk_max, Tq, q_pos0, p.TS,
-                                                                  sm_scale, Hkv, q_pos);
+                                                                  sm_scale, Hkv, q_pos, 1, INT_MAX, 0, nblk_max, 0);
         if ((st = launched("score_table_kernel")) != QSA_OK) return st;
         auto kern = qsa::score_select_kernel<D, KcT, true>;
         if ((st = set_smem(kern, ssmem)) != QSA_OK) return st;
@@ -990,6 +999,187 @@ qsa_status qsa_decode_fp8_paged(const void *q, const void *K_codes, const float 
                                            K_scales, V_scales);
     return launch_decode<128, 4, true>(q, K_codes, V_codes, idx, o, B, Hq, Hkv, T, T, topk, sm_scale, s, pg,
                                        K_scales, V_scales);
+}
+
+// ------------------------------------------------------ sharded caches
+namespace {
+// Candidates of the rows of a chunk at q_pos0 .. q_pos0 + Tq - 1 that lie in
+// [blk_lo, blk_hi): their count for the longest row, and their first block.
+void local_candidates(int Tq, int q_pos0, int blk_lo, int blk_hi, int &first, int &count)
+{
+    const int Dmax = (q_pos0 + Tq - 1) / 64;
+    first = blk_lo > 1 ? blk_lo : 1;
+    const int last = (Dmax - 1 < blk_hi - 1) ? Dmax - 1 : blk_hi - 1;
+    count = last >= first ? last - first + 1 : 0;
+}
+constexpr int kLocalCH = 2048;
+}  // namespace
+
+int qsa_select_local_lists(int Tq, int q_pos0, int blk_lo, int blk_hi)
+{
+    if (Tq <= 0 || q_pos0 < 0 || blk_lo < 0 || blk_hi < blk_lo) return 0;
+    int first, count;
+    local_candidates(Tq, q_pos0, blk_lo, blk_hi, first, count);
+    return count > 0 ? (count + kLocalCH - 1) / kLocalCH : 1;
+}
+
+size_t qsa_score_select_local_workspace(int B, int Hq, int Hkv, int Tq, int q_pos0, int d, int blk_lo, int blk_hi)
+{
+    (void)Hq;
+    if (B <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || !supported_d(d) || blk_lo < 0 || blk_hi < blk_lo) return 0;
+    int first, count;
+    local_candidates(Tq, q_pos0, blk_lo, blk_hi, first, count);
+    const size_t rows = (size_t)B * Hkv * ((Tq + 63) / 64);
+    return align256(rows * d * sizeof(float)) + align256(rows * (size_t)((count + 3) / 4 * 4) * sizeof(float));
+}
+
+qsa_status qsa_score_select_local(const void *Q, const float *Kc_local, uint64_t *lists, int B, int Hq, int Hkv,
+                                  int Tq, int q_pos0, int blk_lo, int blk_hi, int nlists, int d, int topk,
+                                  float sm_scale, void *workspace, size_t workspace_bytes, qsa_stream_t stream)
+{
+    const char *name = "qsa_score_select_local";
+    if (!Q || !Kc_local || !lists) return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || q_pos0 % 64 || Hq % Hkv || blk_lo < 0 ||
+        blk_hi <= blk_lo)
+        return fail(QSA_ERR_INVALID_ARG, "%s: bad shape or block range", name);
+    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "%s: d=%d", name, d);
+    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "%s: topk=%d", name, topk);
+    if ((long)Hq * d / 8 > 1024) return fail(QSA_ERR_UNSUPPORTED, "%s: Hq*d too large", name);
+    const int need_lists = qsa_select_local_lists(Tq, q_pos0, blk_lo, blk_hi);
+    if (nlists < need_lists || nlists > 64)
+        return fail(QSA_ERR_INVALID_ARG, "%s: nlists=%d (this range needs %d, at most 64)", name, nlists, need_lists);
+    if (!aligned16(Q) || !aligned16(Kc_local) || !aligned16(lists) || (workspace && !aligned16(workspace)))
+        return fail(QSA_ERR_INVALID_ARG, "%s: misaligned pointer", name);
+    const size_t need = qsa_score_select_local_workspace(B, Hq, Hkv, Tq, q_pos0, d, blk_lo, blk_hi);
+    if (!workspace || workspace_bytes < need)
+        return fail(QSA_ERR_WORKSPACE, "%s: workspace needs %zu bytes", name, need);
+    int first, count;
+    local_candidates(Tq, q_pos0, blk_lo, blk_hi, first, count);
+    const int NR = (Tq + 63) / 64;
+    const size_t rows = (size_t)B * Hkv * NR;
+    float *Qbar = static_cast<float *>(workspace);
+    float *table = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + align256(rows * d * sizeof(float)));
+    const int TS = (count + 3) / 4 * 4;
+    const int nblk_max = (q_pos0 + Tq + 63) / 64;    // positions of the chunk bound every row's diagonal
+    const int kc_n = blk_hi - blk_lo;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 pgrid(NR, B);
+    const int pool_threads = ((Hq * d / 8) + 31) / 32 * 32, pool_smem = Hq * d * 4;
+    constexpr int TT = qsa::kTableTile;
+    const dim3 tgrid((unsigned)std::max(1, (count + TT - 1) / TT), (unsigned)((NR + TT - 1) / TT), (unsigned)(B * Hkv));
+    qsa_status st;
+    if (d == 128) {
+        if ((st = set_smem(qsa::pool_queries_kernel<128>, pool_smem)) != QSA_OK) return st;
+        qsa::pool_queries_kernel<128><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq, Hq,
+                                                                             Hkv, 64);
+        if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
+        if (count > 0) {
+            const int tsmem = 2 * TT * (128 + 4) * (int)sizeof(float);
+            if ((st = set_smem(qsa::score_table_kernel<128, float>, tsmem)) != QSA_OK) return st;
+            qsa::score_table_kernel<128, float><<<tgrid, 256, tsmem, s>>>(Qbar, Kc_local, table, nblk_max, Tq, q_pos0,
+                                                                          TS, sm_scale, Hkv, nullptr, first, blk_hi,
+                                                                          blk_lo, kc_n, first);
+            if ((st = launched("score_table_kernel")) != QSA_OK) return st;
+        }
+    } else {
+        if ((st = set_smem(qsa::pool_queries_kernel<64>, pool_smem)) != QSA_OK) return st;
+        qsa::pool_queries_kernel<64><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq, Hq,
+                                                                            Hkv, 64);
+        if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
+        if (count > 0) {
+            const int tsmem = 2 * TT * (64 + 4) * (int)sizeof(float);
+            if ((st = set_smem(qsa::score_table_kernel<64, float>, tsmem)) != QSA_OK) return st;
+            qsa::score_table_kernel<64, float><<<tgrid, 256, tsmem, s>>>(Qbar, Kc_local, table, nblk_max, Tq, q_pos0,
+                                                                         TS, sm_scale, Hkv, nullptr, first, blk_hi,
+                                                                         blk_lo, kc_n, first);
+            if ((st = launched("score_table_kernel")) != QSA_OK) return st;
+        }
+    }
+    const int ssmem = kLocalCH * 8;
+    if ((st = set_smem(qsa::local_lists_kernel, ssmem)) != QSA_OK) return st;
+    qsa::local_lists_kernel<<<dim3(nlists, NR, B * Hkv), qsa::kSelThreads, ssmem, s>>>(
+        table, lists, nblk_max, Tq, q_pos0, topk, kLocalCH, nlists, Hkv, first, blk_hi, TS);
+    return launched("local_lists_kernel");
+}
+
+qsa_status qsa_merge_select_lists(const uint64_t *lists, int32_t *idx, int B, int Hkv, int Tq, int q_pos0,
+                                  int nranks, int nlists, int topk, qsa_stream_t stream)
+{
+    const char *name = "qsa_merge_select_lists";
+    if (!lists || !idx) return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (B <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || q_pos0 % 64 || nlists <= 0 || nranks <= 0)
+        return fail(QSA_ERR_INVALID_ARG, "%s: bad shape", name);
+    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "%s: topk=%d", name, topk);
+    if ((long)nranks * nlists * qsa::kMaxChosen * 8 > 200 * 1024)
+        return fail(QSA_ERR_UNSUPPORTED, "%s: too many lists", name);
+    if (!aligned16(lists) || !aligned16(idx)) return fail(QSA_ERR_INVALID_ARG, "%s: misaligned pointer", name);
+    const int NR = (Tq + 63) / 64;
+    const int msmem = nranks * nlists * qsa::kMaxChosen * 8;
+    qsa_status st;
+    if ((st = set_smem(qsa::merge_lists_kernel, msmem)) != QSA_OK) return st;
+    qsa::merge_lists_kernel<<<dim3(NR, B * Hkv), qsa::kSelThreads, msmem, reinterpret_cast<cudaStream_t>(stream)>>>(
+        lists, idx, Tq, q_pos0, topk, nlists, nranks);
+    return launched("merge_lists_kernel");
+}
+
+qsa_status qsa_sparse_attn_prefill_local(const void *Q, const void *K_local, const void *V_local, const int32_t *idx,
+                                         void *O, float *lse, int B, int Hq, int Hkv, int Tq, int q_pos0, int T_local,
+                                         int blk_lo, int blk_hi, int d, int topk, float sm_scale, qsa_stream_t stream)
+{
+    const char *name = "qsa_sparse_attn_prefill_local";
+    if (!Q || !K_local || !V_local || !idx || !O || !lse) return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || q_pos0 % 64 || T_local <= 0 || T_local % 64 ||
+        Hq % Hkv || blk_lo < 0 || blk_hi <= blk_lo || (long)(blk_hi - blk_lo) * 64 > T_local)
+        return fail(QSA_ERR_INVALID_ARG, "%s: bad shape or block range", name);
+    if ((long)B * Hkv * T_local >= (1L << 31) || (long)B * Tq >= (1L << 31))
+        return fail(QSA_ERR_UNSUPPORTED, "%s: tensor too large", name);
+    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "%s: d=%d", name, d);
+    if (topk < 2 || topk > 64) return fail(QSA_ERR_UNSUPPORTED, "%s: topk=%d", name, topk);
+    const int G = Hq / Hkv;
+    if (G != 4 && G != 8) return fail(QSA_ERR_UNSUPPORTED, "%s: Hq/Hkv=%d", name, G);
+    if (!aligned16(Q) || !aligned16(K_local) || !aligned16(V_local) || !aligned16(idx) || !aligned16(O) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3))
+        return fail(QSA_ERR_INVALID_ARG, "%s: misaligned pointer", name);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    Ownership own;
+    own.lo = blk_lo;
+    own.hi = blk_hi;
+    own.partial = 1;
+    const Paging pg;
+    if (d == 128 && G == 8)
+        return launch_prefill<128, 8>(Q, K_local, V_local, idx, O, lse, B, Hq, Hkv, Tq, q_pos0, T_local, topk, sm_scale,
+                                      s, pg, own);
+    if (d == 128 && G == 4)
+        return launch_prefill<128, 4>(Q, K_local, V_local, idx, O, lse, B, Hq, Hkv, Tq, q_pos0, T_local, topk, sm_scale,
+                                      s, pg, own);
+    if (d == 64 && G == 8)
+        return launch_prefill<64, 8>(Q, K_local, V_local, idx, O, lse, B, Hq, Hkv, Tq, q_pos0, T_local, topk, sm_scale,
+                                     s, pg, own);
+    return launch_prefill<64, 4>(Q, K_local, V_local, idx, O, lse, B, Hq, Hkv, Tq, q_pos0, T_local, topk, sm_scale, s,
+                                 pg, own);
+}
+
+qsa_status qsa_merge_partials(const void *O_parts, const float *lse_parts, void *O, float *lse, int nparts,
+                              int64_t rows, int d, qsa_stream_t stream)
+{
+    const char *name = "qsa_merge_partials";
+    if (!O_parts || !lse_parts || !O) return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (nparts <= 0 || rows < 0) return fail(QSA_ERR_INVALID_ARG, "%s: bad shape", name);
+    if (!supported_d(d)) return fail(QSA_ERR_UNSUPPORTED, "%s: d=%d", name, d);
+    if ((reinterpret_cast<uintptr_t>(O_parts) & 15) || (reinterpret_cast<uintptr_t>(O) & 15) ||
+        (reinterpret_cast<uintptr_t>(lse_parts) & 3) || (reinterpret_cast<uintptr_t>(lse) & 3))
+        return fail(QSA_ERR_INVALID_ARG, "%s: misaligned pointer", name);
+    if (rows == 0) return QSA_OK;
+    if ((rows + 7) / 8 >= (1L << 31)) return fail(QSA_ERR_UNSUPPORTED, "%s: too many rows", name);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const unsigned grid = (unsigned)((rows + 7) / 8);
+    if (d == 128)
+        qsa::merge_partials_kernel<128><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)O_parts, lse_parts,
+                                                             (__nv_bfloat16 *)O, lse, nparts, rows);
+    else
+        qsa::merge_partials_kernel<64><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)O_parts, lse_parts,
+                                                            (__nv_bfloat16 *)O, lse, nparts, rows);
+    return launched("merge_partials_kernel");
 }
 
 qsa_status qsa_get_device_status(qsa_stream_t stream, int *detail)

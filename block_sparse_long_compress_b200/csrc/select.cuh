@@ -668,10 +668,16 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
 // dynamic shared memory 2 * 64 * (D + 4) * 4 bytes.
 constexpr int kTableTile = 64;
 
+// Sharded caches: the candidates are restricted to blocks [lo, hi) (lo >= 1),
+// Kc holds the summaries of blocks kc_lo .. kc_lo + kc_n - 1 of each (b, g)
+// (the rank's own range), and table column c is block tab_lo + c.  The
+// whole cache: lo = 1, hi = INT_MAX, kc_lo = 0, kc_n = T_kv_max / 64,
+// tab_lo = 0 (column = block index).
 template <int D, typename KcT>
 __global__ void __launch_bounds__(256) score_table_kernel(
     const float *__restrict__ Qbar, const KcT *__restrict__ Kc, float *__restrict__ table, int nblk_max, int Tq,
-    int q_pos0, int stride, float sm_scale, int Hkv, const int32_t *__restrict__ q_pos)
+    int q_pos0, int stride, float sm_scale, int Hkv, const int32_t *__restrict__ q_pos, int lo, int hi, int kc_lo,
+    int kc_n, int tab_lo)
 {
     constexpr int T = kTableTile, LD = D + 4;
     extern __shared__ __align__(16) float tsm[];
@@ -680,10 +686,10 @@ __global__ void __launch_bounds__(256) score_table_kernel(
     const int bg = blockIdx.z, NR = (Tq + 63) / 64;
     const int qp = seq_q_pos(q_pos, bg / Hkv, q_pos0, Tq, nblk_max, false);
     const int r0 = blockIdx.y * T, nr = min(T, NR - r0);
-    const int j0 = 1 + blockIdx.x * T;
+    const int j0 = lo + blockIdx.x * T;
     // candidates of the tile that some row of it has (j < D of its last row)
     const int Dlast = (qp + min((r0 + nr) * 64, Tq) - 1) / 64;
-    const int nc = min(T, Dlast - j0);
+    const int nc = min(T, min(Dlast, hi) - j0);
     if (nc <= 0) return;
     const int tid = threadIdx.x;
     // tiles into shared memory: 16-byte chunks, rows past the tile are zero
@@ -694,7 +700,7 @@ __global__ void __launch_bounds__(256) score_table_kernel(
         if (rr < nr) v = *reinterpret_cast<const float4 *>(Qbar + ((long)bg * NR + r0 + rr) * D + 4 * c);
         *reinterpret_cast<float4 *>(qs + rr * LD + 4 * c) = v;
         float k4[4] = {0.f, 0.f, 0.f, 0.f};
-        if (rr < nc) load_summary<4>(Kc + ((long)bg * nblk_max + j0 + rr) * D + 4 * c, k4);
+        if (rr < nc) load_summary<4>(Kc + ((long)bg * kc_n + (j0 - kc_lo) + rr) * D + 4 * c, k4);
         *reinterpret_cast<float4 *>(ks + rr * LD + 4 * c) = make_float4(k4[0], k4[1], k4[2], k4[3]);
     }
     __syncthreads();
@@ -728,7 +734,7 @@ __global__ void __launch_bounds__(256) score_table_kernel(
         const int rr = 4 * ty + i;
         if (rr >= nr) break;
         const int Drow = (qp + min((r0 + rr + 1) * 64, Tq) - 1) / 64;
-        float *trow = table + ((long)bg * NR + r0 + rr) * stride + j0;
+        float *trow = table + ((long)bg * NR + r0 + rr) * stride + (j0 - tab_lo);
 #pragma unroll
         for (int jj = 0; jj < 4; jj++) {
             const int e = tx + 16 * jj;
@@ -759,6 +765,96 @@ __global__ void __launch_bounds__(kSelThreads) merge_select_kernel(
     }
     __syncthreads();
     select_and_emit(keys, n, g.m, sh, idx + row * topk, g.D, topk, nullptr);
+}
+
+// ---------------------------------------------------- sharded caches
+// A rank that owns the cache blocks [lo, hi) selects, for every prefill row,
+// the top m of its own candidates (blocks j in [lo, hi) with 1 <= j < D) in
+// chunks of CH from the score table (column j - lo), and writes each
+// chunk's keys, in block order, as a list of kMaxChosen keys padded with 0
+// (below every candidate's key): part[row][chunk][kMaxChosen].  The lists
+// of all ranks, gathered, hold the row's top m (a candidate outside a
+// list's top m has m better ones in the same list), and merge_lists_kernel
+// picks it from them.
+// grid (maxchunks, NR, B*Hkv); dynamic smem CH * 8 bytes.
+__global__ void __launch_bounds__(kSelThreads) local_lists_kernel(
+    const float *__restrict__ table, uint64_t *__restrict__ part, int nblk_max, int Tq, int q_pos0, int topk, int CH,
+    int maxchunks, int Hkv, int lo, int hi, int stride)
+{
+    extern __shared__ uint64_t keys[];
+    __shared__ SelectShared sh;
+    const int chunk = blockIdx.x, i = blockIdx.y, bg = blockIdx.z, NR = gridDim.y;
+    const RowGeom g = row_geom(i, Tq, q_pos0, 64, topk, CH);
+    const int first = max(1, lo), last = min(g.D - 1, hi - 1);   // the row's own candidates
+    const int j0 = first + chunk * CH;
+    const int n = max(0, min(CH, last - j0 + 1));
+    const long row = (long)bg * NR + i;
+    uint64_t *dst = part + (row * maxchunks + chunk) * kMaxChosen;
+    const float *srow = table + row * stride + (j0 - lo);
+    for (int e = threadIdx.x; e < n; e += kSelThreads) keys[e] = make_key(__ldg(srow + e), j0 + e);
+    __syncthreads();
+    const int need = min(g.m, n);
+    select_and_emit(keys, n, need, sh, nullptr, g.D, topk, dst);
+    for (int e = max(need, 0) + threadIdx.x; e < kMaxChosen; e += kSelThreads) dst[e] = 0;
+}
+
+// The row's selection from the ranks' lists as an all-gather leaves them
+// (rank-major: lists[r][row][nlists][kMaxChosen], 0 = padding), taken in
+// rank order -- ascending block ranges, each rank's chunks in order -- so
+// the keys stand in ascending block order: the top m by key, then the
+// forced blocks.
+// grid (NR, B*Hkv); dynamic smem nranks * nlists * kMaxChosen * 8 bytes.
+__global__ void __launch_bounds__(kSelThreads) merge_lists_kernel(
+    const uint64_t *__restrict__ lists, int32_t *__restrict__ idx, int Tq, int q_pos0, int topk, int nlists,
+    int nranks)
+{
+    extern __shared__ uint64_t keys[];
+    __shared__ SelectShared sh;
+    const int i = blockIdx.x, bg = blockIdx.y, NR = gridDim.x;
+    const RowGeom g = row_geom(i, Tq, q_pos0, 64, topk, 1 << 30);
+    const long row = (long)bg * NR + i, rows = (long)gridDim.y * NR;
+    const int per = nlists * kMaxChosen, n = nranks * per;
+    for (int e = threadIdx.x; e < n; e += kSelThreads) keys[e] = lists[((long)(e / per) * rows + row) * per + e % per];
+    __syncthreads();
+    select_and_emit(keys, n, g.m, sh, idx + row * topk, g.D, topk, nullptr);
+}
+
+// Partial attention outputs of the ranks (each over its own blocks, with its
+// natural-log normaliser lse_r; lse_r = -inf when it owns none of the row's
+// blocks) merged into the row's output: O = sum_r exp(lse_r - L) O_r with
+// L = log sum_r exp(lse_r), and lse = L.  One warp per (token, head) row,
+// lane owns D/32 consecutive columns; fp32 arithmetic.
+// grid ceil(rows / 8); 256 threads.
+template <int D>
+__global__ void __launch_bounds__(256) merge_partials_kernel(const __nv_bfloat16 *__restrict__ O_parts,
+                                                             const float *__restrict__ lse_parts,
+                                                             __nv_bfloat16 *__restrict__ O, float *__restrict__ lse,
+                                                             int nparts, long rows)
+{
+    constexpr int CPL = D / 32;
+    const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    float m = -INFINITY;
+    for (int r = 0; r < nparts; r++) m = fmaxf(m, __ldg(lse_parts + (long)r * rows + row));
+    float acc[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; c++) acc[c] = 0.f;
+    float wsum = 0.f;
+    if (m != -INFINITY) {
+        for (int r = 0; r < nparts; r++) {
+            const float w = __expf(__ldg(lse_parts + (long)r * rows + row) - m);
+            wsum += w;
+            const __nv_bfloat16 *src = O_parts + ((long)r * rows + row) * D + lane * CPL;
+#pragma unroll
+            for (int c = 0; c < CPL; c++) acc[c] += w * __bfloat162float(src[c]);
+        }
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    __nv_bfloat16 *dst = O + row * D + lane * CPL;
+#pragma unroll
+    for (int c = 0; c < CPL; c++) dst[c] = __float2bfloat16_rn(acc[c] * inv);
+    if (lse && lane == 0) lse[row] = m == -INFINITY ? -INFINITY : m + __logf(wsum);
 }
 
 // ------------------------------------------------ per-token, one launch

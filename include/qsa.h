@@ -384,6 +384,67 @@ QSA_API qsa_status qsa_decode_fp8_paged(const void *q, const void *K_codes, cons
                                         qsa_stream_t stream);
 
 /*
+ * One long sequence whose cache is split across GPUs (contiguous block
+ * ranges, one per rank).  The pages set the regime -- contexts from 262K
+ * tokens up (page "Qwen4 in llama.cpp: Dissecting PR #27742", section "Why
+ * Short-Context Tests Can Lie"; the cache of page "Qwen3.8 Flash Next
+ * VRAM", section "What It Needs") -- and the selection's two-part cost, so
+ * both the scoring and the attention are split by block range and only
+ * small lists cross between GPUs.  A chunk of Tq new query tokens at
+ * positions q_pos0 .. q_pos0 + Tq - 1 (q_pos0 a multiple of 64; prefill
+ * rows of 64 tokens) is processed by every rank r, which holds the blocks
+ * [blk_lo, blk_hi) of the sequence (the rank with the chunk's own blocks
+ * holds them at the end of its range) and the whole Q:
+ *   1. qsa_score_select_local: pooled queries, scores of the rank's own
+ *      candidates (blocks j in [blk_lo, blk_hi) with 1 <= j < D of the row;
+ *      Kc_local fp32 [B][Hkv][blk_hi - blk_lo][d] holds their summaries),
+ *      and per row nlists lists of 62 keys (lists uint64
+ *      [B][Hkv][ceil(Tq/64)][nlists][62]): chunk c's top m candidates as
+ *      (order-preserving score bits << 32 | ~j), in block order, padded with
+ *      0.  nlists >= qsa_select_local_lists(Tq, q_pos0, blk_lo, blk_hi) and
+ *      the same on every rank; the workspace is
+ *      qsa_score_select_local_workspace() bytes.
+ *   2. all ranks' lists gathered in rank order (ranges ascending) as an
+ *      all-gather leaves them: [R][B][Hkv][NR][nlists][62];
+ *   3. qsa_merge_select_lists (nranks = R): the row's top m of the gathered
+ *      keys by
+ *      (score descending, block ascending) plus blocks 0 and D -- exactly
+ *      qsa_score_select's indices of the whole cache, on every rank;
+ *   4. qsa_sparse_attn_prefill_local: attention over the listed blocks the
+ *      rank holds (K_local, V_local bf16 [B][Hkv][T_local][d], block j at row
+ *      64 (j - blk_lo); T_local >= 64 (blk_hi - blk_lo)), other listed
+ *      blocks skipped; O bf16 [B][Tq][Hq][d] normalised over the rank's
+ *      keys and lse fp32 [B][Tq][Hq] (required) their natural-log
+ *      normaliser, O = 0 and lse = -inf for a row none of whose blocks the
+ *      rank holds;
+ *   5. the ranks' (O, lse) gathered as O_parts bf16 [R][rows][d] and
+ *      lse_parts fp32 [R][rows] (rows = B * Tq * Hq), and qsa_merge_partials:
+ *      O = sum_r exp(lse_r - L) O_r, L = log sum_r exp(lse_r) (lse may be
+ *      NULL).
+ * The gathers are the caller's collectives (e.g. NCCL all-gather).
+ * Errors: null pointers, a bad range or shape, nlists below what the range
+ * needs or above 64, misaligned pointers -> QSA_ERR_INVALID_ARG; d, topk
+ * or group size outside the supported set -> QSA_ERR_UNSUPPORTED; a short
+ * workspace -> QSA_ERR_WORKSPACE.  Device-side checks as for
+ * qsa_sparse_attn_prefill.
+ */
+QSA_API int qsa_select_local_lists(int Tq, int q_pos0, int blk_lo, int blk_hi);
+QSA_API size_t qsa_score_select_local_workspace(int B, int Hq, int Hkv, int Tq, int q_pos0, int d, int blk_lo,
+                                                int blk_hi);
+QSA_API qsa_status qsa_score_select_local(const void *Q, const float *Kc_local, uint64_t *lists, int B, int Hq,
+                                          int Hkv, int Tq, int q_pos0, int blk_lo, int blk_hi, int nlists, int d,
+                                          int topk, float sm_scale, void *workspace, size_t workspace_bytes,
+                                          qsa_stream_t stream);
+QSA_API qsa_status qsa_merge_select_lists(const uint64_t *lists, int32_t *idx, int B, int Hkv, int Tq, int q_pos0,
+                                          int nranks, int nlists, int topk, qsa_stream_t stream);
+QSA_API qsa_status qsa_sparse_attn_prefill_local(const void *Q, const void *K_local, const void *V_local,
+                                                 const int32_t *idx, void *O, float *lse, int B, int Hq, int Hkv,
+                                                 int Tq, int q_pos0, int T_local, int blk_lo, int blk_hi, int d,
+                                                 int topk, float sm_scale, qsa_stream_t stream);
+QSA_API qsa_status qsa_merge_partials(const void *O_parts, const float *lse_parts, void *O, float *lse, int nparts,
+                                      int64_t rows, int d, qsa_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word
  * (QSA_OK if no kernel recorded an error since the last call).  If detail
  * is not NULL it receives a kernel-specific code (0 if none).  The word

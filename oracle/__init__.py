@@ -253,6 +253,77 @@ def qsa_forward(Q, K, V, Hkv, topk, q_pos0=0, qblk=BLOCK, sm_scale=None, blk=BLO
     return sel, O
 
 
+# ------------------------------------------- one sequence over several GPUs
+# The cache of one long sequence split by contiguous block ranges, one per
+# rank (the long-context regime of page "Qwen4 in llama.cpp: Dissecting PR
+# #27742", section "Why Short-Context Tests Can Lie"): each rank keeps the
+# top m of its own candidates by the same order (score descending, block
+# ascending), and the union of the ranks' lists holds the row's top m (a
+# candidate outside its rank's list has m better ones there).  Attention
+# over disjoint key sets combines through their log-sum-exp: with
+# L = log sum_r exp(lse_r), O = sum_r exp(lse_r - L) O_r.
+
+def select_shard(Qbar, Kc, Tq, q_pos0, topk, sm_scale, blk_lo, blk_hi, qblk=BLOCK):
+    """A rank's candidate lists: for every row, the top m (the row's m, as
+    select() sets it) of the candidates j in [blk_lo, blk_hi) with
+    1 <= j < D, ordered by (score descending, block ascending).  Returns
+    (scores, blocks), each [nrows, 62] (fp64 padded with -inf, int32 padded
+    with -1), rows flat (b, g, i) like select(rows=...)."""
+    sel = select(Qbar, Kc, Tq, q_pos0, qblk, topk, sm_scale, rows=np.arange(int(np.prod(Qbar.shape[:3]))),
+                 want_scores=True)
+    scores, m = sel["scores"], sel["m"]
+    nrows = len(m)
+    NR = Qbar.shape[2]
+    out_s = np.full((nrows, 62), -np.inf)
+    out_j = np.full((nrows, 62), -1, dtype=np.int32)
+    for r in range(nrows):
+        i = r % NR
+        D = (q_pos0 + min((i + 1) * qblk, Tq) - 1) // BLOCK
+        js = np.arange(max(1, blk_lo), min(D - 1, blk_hi - 1) + 1)
+        if len(js) == 0 or m[r] == 0:
+            continue
+        order = sorted(js.tolist(), key=lambda j: (-scores[r, j], j))[:m[r]]
+        out_s[r, :len(order)] = scores[r, order]
+        out_j[r, :len(order)] = order
+    return out_s, out_j
+
+
+def merge_shard_lists(scores, blocks, Tq, q_pos0, topk, qblk=BLOCK):
+    """The rows' selection from all ranks' lists (scores, blocks: [R, nrows,
+    L]): the top m of their union by (score descending, block ascending),
+    plus blocks 0 and D, ascending, padded with -1 to topk.  Returns idx
+    [nrows, topk] int32."""
+    R, nrows, _ = blocks.shape
+    idx = np.full((nrows, topk), -1, dtype=np.int32)
+    NR = -(-Tq // qblk)
+    for r in range(nrows):
+        i = r % NR
+        D = (q_pos0 + min((i + 1) * qblk, Tq) - 1) // BLOCK
+        forced = [0] if D == 0 else [0, D]
+        m = min(topk - len(forced), max(D - 1, 0))
+        cand = [(float(scores[k, r, e]), int(blocks[k, r, e])) for k in range(R)
+                for e in range(blocks.shape[2]) if blocks[k, r, e] >= 0]
+        chosen = [j for _, j in sorted(cand, key=lambda t: (-t[0], t[1]))[:m]]
+        row = sorted(set(forced) | set(chosen))
+        idx[r, :len(row)] = row
+    return idx
+
+
+def merge_partials(O_parts, lse_parts):
+    """Outputs of attention over disjoint key sets merged by their
+    log-sum-exp, fp64: O_parts [R, ..., d], lse_parts [R, ...] (-inf for an
+    empty set).  Returns (O, lse)."""
+    O_parts = np.asarray(O_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    mx = lse_parts.max(axis=0)
+    safe = np.where(np.isfinite(mx), mx, 0.0)
+    w = np.exp(lse_parts - safe)                       # exp(-inf) = 0
+    tot = w.sum(axis=0)
+    O = (w[..., None] * O_parts).sum(axis=0) / np.where(tot > 0, tot, 1.0)[..., None]
+    lse = np.where(tot > 0, safe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    return O, lse
+
+
 # ------------------------------------------------------- quantized KV option
 # Page "Qwen4 in llama.cpp: Dissecting PR #27742", section "Quantized KV
 # Exposed a Backend Storage Invariant": K/V stored in a Hadamard-rotated
