@@ -130,9 +130,13 @@ bool supported_d(int d) { return d == 64 || d == 128; }
 // ------------------------------------------------------- select geometry
 struct SelectPlan {
     int NR, CH, maxchunks;
+    bool wide;            // prefill rows each selected whole by one 1024-thread CTA
     int TS;               // prefill rows: score-table row stride (floats)
     size_t qbar_bytes, part_bytes, table_bytes;
 };
+
+int sm_count();
+constexpr int kWideMax = 24576;   // candidates of one row whose keys (192 KiB) fit one CTA
 
 SelectPlan plan_select(int B, int Hkv, int Tq, int q_pos0, int qblk, int d)
 {
@@ -144,6 +148,11 @@ SelectPlan plan_select(int B, int Hkv, int Tq, int q_pos0, int qblk, int d)
     int CH = 2048;
     // enough CTAs to cover the SMs a few times over
     while (CH > 512 && rows * ((ncand + CH - 1) / CH) < 4 * 148) CH /= 2;
+    // prefill rows longer than one chunk, few enough for about one wave of
+    // 1024-thread CTAs, are selected whole from the score table by one CTA
+    // each (the keys in shared memory), with no chunk lists and no merge
+    p.wide = qblk == 64 && ncand > CH && ncand <= kWideMax && rows <= 2L * sm_count();
+    if (p.wide) CH = (ncand + 3) / 4 * 4;
     p.CH = CH;
     p.maxchunks = ncand > 0 ? (ncand + CH - 1) / CH : 1;
     p.qbar_bytes = align256((size_t)rows * d * sizeof(float));
@@ -468,19 +477,34 @@ qsa_status compress_keys_impl(const char *name, const void *K, KcT *Kc, int B, i
 }
 
 
+// Pooling launch: the 16-byte column chunks of a token's heads, times up to
+// four token splits for rows of several tokens (at most 1024 threads).
+struct PoolLaunch {
+    int threads, TS, smem;
+};
+
+PoolLaunch plan_pool(int Hq, int d, int qblk, long ctas)
+{
+    const int nc = ((Hq * d / 8) + 31) / 32 * 32;
+    // split tokens only when the rows' CTAs are too few to fill the GPU
+    int TS = (qblk > 1 && ctas < 2L * sm_count()) ? 1024 / nc : 1;
+    TS = TS > 4 ? 4 : (TS < 1 ? 1 : TS);
+    return {nc * TS, TS, TS * Hq * d * (int)sizeof(float)};
+}
+
 // Pooling, then scoring and selection: prefill rows through the score
 // table (score_table_kernel, then score_select_kernel from the table),
 // long per-token rows by score_select_kernel's own scoring.
 template <int D, typename KcT>
 qsa_status launch_score_select(const void *Q, const KcT *Kc, int32_t *idx, float *Qbar, uint64_t *part, float *table,
-                               const SelectPlan &p, dim3 pgrid, int pool_threads, int pool_smem, dim3 sgrid, int ssmem,
+                               const SelectPlan &p, dim3 pgrid, const PoolLaunch &pl, dim3 sgrid, int ssmem,
                                int B, int Hq, int Hkv, int Tq, int q_pos0, int qblk, int nblk_max, int topk,
                                float sm_scale, const int32_t *q_pos, cudaStream_t s)
 {
     qsa_status st;
-    if ((st = set_smem(qsa::pool_queries_kernel<D>, pool_smem)) != QSA_OK) return st;
-    qsa::pool_queries_kernel<D><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq, Hq, Hkv,
-                                                                       qblk);
+    if ((st = set_smem(qsa::pool_queries_kernel<D>, pl.smem)) != QSA_OK) return st;
+    qsa::pool_queries_kernel<D><<<pgrid, pl.threads, pl.smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq, Hq, Hkv, qblk,
+                                                                   pl.TS);
     if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
     if (qblk == 64) {
         const int Dmax = (q_pos0 + Tq - 1) / 64;
@@ -492,10 +516,17 @@ qsa_status launch_score_select(const void *Q, const KcT *Kc, int32_t *idx, float
         qsa::score_table_kernel<D, KcT><<<tgrid, 256, tsmem, s>>>(Qbar, Kc, table, nblk_max, Tq, q_pos0, p.TS,
                                                                   sm_scale, Hkv, q_pos, 1, INT_MAX, 0, nblk_max, 0);
         if ((st = launched("score_table_kernel")) != QSA_OK) return st;
-        auto kern = qsa::score_select_kernel<D, KcT, true>;
-        if ((st = set_smem(kern, ssmem)) != QSA_OK) return st;
-        kern<<<sgrid, qsa::kSelThreads, ssmem, s>>>(nullptr, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk,
-                                                    sm_scale, p.CH, p.maxchunks, Hkv, q_pos, table, p.TS);
+        if (p.wide) {
+            auto kern = qsa::score_select_kernel<D, KcT, true, 1024>;
+            if ((st = set_smem(kern, ssmem)) != QSA_OK) return st;
+            kern<<<sgrid, 1024, ssmem, s>>>(nullptr, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk, sm_scale, p.CH,
+                                            p.maxchunks, Hkv, q_pos, table, p.TS);
+        } else {
+            auto kern = qsa::score_select_kernel<D, KcT, true>;
+            if ((st = set_smem(kern, ssmem)) != QSA_OK) return st;
+            kern<<<sgrid, qsa::kSelThreads, ssmem, s>>>(nullptr, Kc, idx, part, nblk_max, Tq, q_pos0, qblk, topk,
+                                                        sm_scale, p.CH, p.maxchunks, Hkv, q_pos, table, p.TS);
+        }
     } else {
         auto kern = qsa::score_select_kernel<D, KcT>;
         if ((st = set_smem(kern, ssmem)) != QSA_OK) return st;
@@ -538,15 +569,14 @@ qsa_status score_select_impl(const char *name, const void *Q, const KcT *Kc, int
     uint64_t *part = reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(workspace) + p.qbar_bytes);
     float *table = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + p.qbar_bytes + p.part_bytes);
     const int nblk_max = T_kv_max / 64;
-    const int pool_threads = ((Hq * d / 8) + 31) / 32 * 32;
-    const int pool_smem = Hq * d * 4;
+    const PoolLaunch pl = plan_pool(Hq, d, qblk, (long)p.NR * B);
     dim3 pgrid(p.NR, B), sgrid(p.maxchunks, p.NR, B * Hkv), mgrid(p.NR, B * Hkv);
     const int ssmem = p.CH * 8;
     qsa_status st;
-    if (d == 128) st = launch_score_select<128, KcT>(Q, Kc, idx, Qbar, part, table, p, pgrid, pool_threads,
-                                                      pool_smem, sgrid, ssmem, B, Hq, Hkv, Tq, q_pos0, qblk,
+    if (d == 128) st = launch_score_select<128, KcT>(Q, Kc, idx, Qbar, part, table, p, pgrid, pl,
+                                                      sgrid, ssmem, B, Hq, Hkv, Tq, q_pos0, qblk,
                                                       nblk_max, topk, sm_scale, q_pos, s);
-    else st = launch_score_select<64, KcT>(Q, Kc, idx, Qbar, part, table, p, pgrid, pool_threads, pool_smem,
+    else st = launch_score_select<64, KcT>(Q, Kc, idx, Qbar, part, table, p, pgrid, pl,
                                            sgrid, ssmem, B, Hq, Hkv, Tq, q_pos0, qblk, nblk_max, topk, sm_scale,
                                            q_pos, s);
     if (st != QSA_OK) return st;
@@ -752,11 +782,18 @@ qsa_status qsa_score_select_prefill_agg(const void *Q, const void *Kc, int32_t *
                                                    aggregator, s);
     if (st != QSA_OK) return st;
     const dim3 sgrid(p.maxchunks, p.NR, B * Hkv), mgrid(p.NR, B * Hkv);
-    auto skern = qsa::score_select_kernel<128, __nv_bfloat16, true>;
-    if ((st = set_smem(skern, p.CH * 8)) != QSA_OK) return st;
-    skern<<<sgrid, qsa::kSelThreads, p.CH * 8, s>>>(nullptr, static_cast<const __nv_bfloat16 *>(Kc), idx, part, nblk,
-                                                    Tq, q_pos0, 64, topk, sm_scale, p.CH, p.maxchunks, Hkv, nullptr,
-                                                    scores, 0);
+    if (p.wide) {
+        auto skern = qsa::score_select_kernel<128, __nv_bfloat16, true, 1024>;
+        if ((st = set_smem(skern, p.CH * 8)) != QSA_OK) return st;
+        skern<<<sgrid, 1024, p.CH * 8, s>>>(nullptr, static_cast<const __nv_bfloat16 *>(Kc), idx, part, nblk, Tq, q_pos0,
+                                            64, topk, sm_scale, p.CH, p.maxchunks, Hkv, nullptr, scores, 0);
+    } else {
+        auto skern = qsa::score_select_kernel<128, __nv_bfloat16, true>;
+        if ((st = set_smem(skern, p.CH * 8)) != QSA_OK) return st;
+        skern<<<sgrid, qsa::kSelThreads, p.CH * 8, s>>>(nullptr, static_cast<const __nv_bfloat16 *>(Kc), idx, part,
+                                                        nblk, Tq, q_pos0, 64, topk, sm_scale, p.CH, p.maxchunks, Hkv,
+                                                        nullptr, scores, 0);
+    }
     if ((st = launched("score_select_kernel")) != QSA_OK) return st;
     if (p.maxchunks > 1) {
         const int msmem = p.maxchunks * qsa::kMaxChosen * 8;
@@ -1064,14 +1101,14 @@ qsa_status qsa_score_select_local(const void *Q, const float *Kc_local, uint64_t
     const int kc_n = blk_hi - blk_lo;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const dim3 pgrid(NR, B);
-    const int pool_threads = ((Hq * d / 8) + 31) / 32 * 32, pool_smem = Hq * d * 4;
+    const PoolLaunch pl = plan_pool(Hq, d, 64, (long)NR * B);
     constexpr int TT = qsa::kTableTile;
     const dim3 tgrid((unsigned)std::max(1, (count + TT - 1) / TT), (unsigned)((NR + TT - 1) / TT), (unsigned)(B * Hkv));
     qsa_status st;
     if (d == 128) {
-        if ((st = set_smem(qsa::pool_queries_kernel<128>, pool_smem)) != QSA_OK) return st;
-        qsa::pool_queries_kernel<128><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq, Hq,
-                                                                             Hkv, 64);
+        if ((st = set_smem(qsa::pool_queries_kernel<128>, pl.smem)) != QSA_OK) return st;
+        qsa::pool_queries_kernel<128><<<pgrid, pl.threads, pl.smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq, Hq, Hkv,
+                                                                         64, pl.TS);
         if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
         if (count > 0) {
             const int tsmem = 2 * TT * (128 + 4) * (int)sizeof(float);
@@ -1082,9 +1119,9 @@ qsa_status qsa_score_select_local(const void *Q, const float *Kc_local, uint64_t
             if ((st = launched("score_table_kernel")) != QSA_OK) return st;
         }
     } else {
-        if ((st = set_smem(qsa::pool_queries_kernel<64>, pool_smem)) != QSA_OK) return st;
-        qsa::pool_queries_kernel<64><<<pgrid, pool_threads, pool_smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq, Hq,
-                                                                            Hkv, 64);
+        if ((st = set_smem(qsa::pool_queries_kernel<64>, pl.smem)) != QSA_OK) return st;
+        qsa::pool_queries_kernel<64><<<pgrid, pl.threads, pl.smem, s>>>((const __nv_bfloat16 *)Q, Qbar, Tq, Hq, Hkv,
+                                                                        64, pl.TS);
         if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
         if (count > 0) {
             const int tsmem = 2 * TT * (64 + 4) * (int)sizeof(float);

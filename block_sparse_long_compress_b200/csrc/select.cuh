@@ -36,15 +36,23 @@ constexpr int kSelThreads = 256;
 constexpr int kMaxChosen = 62;   // topk <= 64 minus the two forced blocks
 
 // ------------------------------------------------------------------ pool
-// grid (NR, B); blockDim = Hq*d/8 rounded up to a warp (<= 1024).
+// grid (NR, B); blockDim = TS * NC where NC = Hq*D/8 rounded up to a warp
+// (the 16-byte column chunks of a token's heads) and TS = token splits
+// (TS * NC <= 1024).  Thread (s, c) sums chunk c over the tokens t0 + s,
+// t0 + s + TS, ...; the TS partial sums then add in order s = 0, 1, ... and
+// the group's heads fold in order -- a fixed order, so the pooled queries
+// are bit-reproducible.  Splitting the tokens keeps four times the loads in
+// flight for a row of few CTAs (a short chunk is latency-bound).
 template <int D>
-__global__ void pool_queries_kernel(const __nv_bfloat16 *__restrict__ Q, float *__restrict__ Qbar,
-                                    int Tq, int Hq, int Hkv, int qblk)
+__global__ void __launch_bounds__(1024) pool_queries_kernel(const __nv_bfloat16 *__restrict__ Q,
+                                                            float *__restrict__ Qbar, int Tq, int Hq, int Hkv,
+                                                            int qblk, int TS)
 {
-    extern __shared__ float colsum[];   // [Hq * D]
+    extern __shared__ float colsum[];   // [TS][Hq * D]
     const int i = blockIdx.x, b = blockIdx.y, NR = gridDim.x;
     const int nchunks = Hq * D / 8;
-    const int t = threadIdx.x;
+    const int NC = blockDim.x / TS;
+    const int t = threadIdx.x % NC, sp = threadIdx.x / NC;
     const int t0 = i * qblk;
     const int t1 = min(t0 + qblk, Tq);
     if (t < nchunks) {
@@ -53,13 +61,13 @@ __global__ void pool_queries_kernel(const __nv_bfloat16 *__restrict__ Q, float *
         float acc[8];
 #pragma unroll
         for (int e = 0; e < 8; e++) acc[e] = 0.f;
-        int tok = t0;
-        for (; tok + 8 <= t1; tok += 8) {
-            uint4 v[8];
+        int tok = t0 + sp;
+        for (; tok + 3 * TS < t1; tok += 4 * TS) {
+            uint4 v[4];
 #pragma unroll
-            for (int u = 0; u < 8; u++) v[u] = __ldg(src + (long)(tok - t0 + u) * stride);
+            for (int u = 0; u < 4; u++) v[u] = __ldg(src + (long)(tok - t0 + u * TS) * stride);
 #pragma unroll
-            for (int u = 0; u < 8; u++) {
+            for (int u = 0; u < 4; u++) {
                 const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&v[u]);
 #pragma unroll
                 for (int e = 0; e < 4; e++) {
@@ -69,7 +77,7 @@ __global__ void pool_queries_kernel(const __nv_bfloat16 *__restrict__ Q, float *
                 }
             }
         }
-        for (; tok < t1; tok++) {
+        for (; tok < t1; tok += TS) {
             uint4 v = __ldg(src + (long)(tok - t0) * stride);
             const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&v);
 #pragma unroll
@@ -80,16 +88,20 @@ __global__ void pool_queries_kernel(const __nv_bfloat16 *__restrict__ Q, float *
             }
         }
 #pragma unroll
-        for (int e = 0; e < 8; e++) colsum[t * 8 + e] = acc[e];
+        for (int e = 0; e < 8; e++) colsum[(long)sp * Hq * D + t * 8 + e] = acc[e];
     }
     __syncthreads();
     const int G = Hq / Hkv;
     const float inv = 1.0f / (float)((t1 - t0) * G);
-    for (int o = t; o < Hkv * D; o += blockDim.x) {
+    for (int o = threadIdx.x; o < Hkv * D; o += blockDim.x) {
         const int g = o / D, c = o % D;
-        float s = 0.f;
-        for (int h = g * G; h < (g + 1) * G; h++) s += colsum[h * D + c];
-        Qbar[(((long)b * Hkv + g) * NR + i) * D + c] = s * inv;
+        float sum = 0.f;
+        for (int h = g * G; h < (g + 1) * G; h++) {
+            float col = 0.f;
+            for (int q = 0; q < TS; q++) col += colsum[(long)q * Hq * D + h * D + c];
+            sum += col;
+        }
+        Qbar[(((long)b * Hkv + g) * NR + i) * D + c] = sum * inv;
     }
 }
 
@@ -104,27 +116,37 @@ __device__ __forceinline__ uint64_t make_key(float s, int j)
 
 __device__ __forceinline__ int key_block(uint64_t key) { return (int)(0xFFFFFFFFu - (uint32_t)key); }
 
-struct SelectShared {
+template <int NT>
+struct SelectSharedT {
     int hist[2][256];           // digit counts, double-buffered across radix passes
-    int warp_tot[kSelThreads / 32];
+    int warp_tot[NT / 32];
     int digit[2], above[2], bucket[2];
 };
+using SelectShared = SelectSharedT<kSelThreads>;
 
-// Adds 1 to hist[digit] for every lane with active set; lanes of a warp
-// that share a digit are combined into one atomic (keys of a row often
-// share their top digits, which would serialise plain atomics).
+// Adds 1 to hist[digit] for every lane with active set (called by the
+// whole warp).  When every active lane has the same digit -- the first
+// passes, where a row's keys share their top digits -- one lane adds the
+// count; otherwise each active lane adds its own 1 (later digits are spread
+// out, so those atomics rarely collide).
 __device__ __forceinline__ void hist_add(int *hist, bool active, int digit)
 {
     const unsigned act = __ballot_sync(0xffffffffu, active);
-    if (!active) return;
-    const unsigned same = __match_any_sync(act, digit);
-    if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&hist[digit], __popc(same));
+    if (!act) return;
+    const int lead = __ffs(act) - 1;
+    const int d0 = __shfl_sync(0xffffffffu, digit, lead);
+    if (__all_sync(0xffffffffu, !active || digit == d0)) {
+        if ((threadIdx.x & 31) == lead) atomicAdd(&hist[d0], __popc(act));
+        return;
+    }
+    if (active) atomicAdd(&hist[digit], 1);
 }
 
 // Warp 0: the digit whose bucket holds the need-th largest key of
 // sh.hist[b] (counts by digit), the count above it and the bucket's size,
 // into sh.digit[b], sh.above[b], sh.bucket[b].
-__device__ __forceinline__ void find_digit(SelectShared &sh, int b, int need)
+template <int NT>
+__device__ __forceinline__ void find_digit(SelectSharedT<NT> &sh, int b, int need)
 {
     const int lane = threadIdx.x & 31;
     // lane l owns bins 255-8l .. 248-8l (descending)
@@ -159,7 +181,8 @@ __device__ __forceinline__ void find_digit(SelectShared &sh, int b, int need)
 // Radix select over n unique keys in shared memory: returns (prefix, mask)
 // such that exactly `need` keys satisfy (key & mask) >= prefix.
 // Requires 0 < need < n.  All threads of the CTA must call it.
-__device__ void radix_select(const uint64_t *keys, int n, int need, SelectShared &sh,
+template <int NT>
+__device__ void radix_select(const uint64_t *keys, int n, int need, SelectSharedT<NT> &sh,
                              uint64_t &prefix_out, uint64_t &mask_out)
 {
     // two barriers per pass: the counts and the result of a pass live in
@@ -167,11 +190,11 @@ __device__ void radix_select(const uint64_t *keys, int n, int need, SelectShared
     // one pass earlier, is zeroed for the next pass
     const int tid = threadIdx.x, warp = tid >> 5;
     uint64_t prefix = 0, mask = 0;
-    for (int d = tid; d < 256; d += kSelThreads) sh.hist[0][d] = 0;
+    for (int d = tid; d < 256; d += NT) sh.hist[0][d] = 0;
     __syncthreads();
     for (int shift = 56, cur = 0; shift >= 0; shift -= 8, cur ^= 1) {
-        for (int d = tid; d < 256; d += kSelThreads) sh.hist[cur ^ 1][d] = 0;
-        for (int base = 0; base < n; base += kSelThreads) {
+        for (int d = tid; d < 256; d += NT) sh.hist[cur ^ 1][d] = 0;
+        for (int base = 0; base < n; base += NT) {
             const int e = base + tid;
             const uint64_t k = e < n ? keys[e] : 0;
             hist_add(sh.hist[cur], e < n && (k & mask) == prefix, (int)((k >> shift) & 0xFF));
@@ -189,7 +212,8 @@ __device__ void radix_select(const uint64_t *keys, int n, int need, SelectShared
 }
 
 // Exclusive CTA-wide prefix sum of one int per thread; also returns the total.
-__device__ __forceinline__ int block_exclusive_scan(int v, SelectShared &sh, int &total)
+template <int NT>
+__device__ __forceinline__ int block_exclusive_scan(int v, SelectSharedT<NT> &sh, int &total)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int incl = v;
@@ -202,7 +226,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, SelectShared &sh, int
     __syncthreads();
     int base = 0, tot = 0;
 #pragma unroll
-    for (int w = 0; w < kSelThreads / 32; w++) {
+    for (int w = 0; w < NT / 32; w++) {
         const int x = sh.warp_tot[w];
         if (w < warp) base += x;
         tot += x;
@@ -215,13 +239,14 @@ __device__ __forceinline__ int block_exclusive_scan(int v, SelectShared &sh, int
 // Select the top `need` of n keys (already in ascending block order) and
 // emit them in that order: to `final_row` as block ids between the forced
 // entries (0 first, then the chosen, then D), or to `part` as keys.
-__device__ void select_and_emit(const uint64_t *keys, int n, int need, SelectShared &sh,
+template <int NT>
+__device__ void select_and_emit(const uint64_t *keys, int n, int need, SelectSharedT<NT> &sh,
                                 int32_t *final_row, int D, int topk, uint64_t *part)
 {
     uint64_t prefix = 0, mask = 0;
     bool all = need >= n;
     if (need > 0 && !all) radix_select(keys, n, need, sh, prefix, mask);
-    const int per = (n + kSelThreads - 1) / kSelThreads;
+    const int per = (n + NT - 1) / NT;
     const int e0 = threadIdx.x * per;
     const int e1 = min(e0 + per, n);
     int cnt = 0;
@@ -241,7 +266,7 @@ __device__ void select_and_emit(const uint64_t *keys, int n, int need, SelectSha
     }
     if (final_row) {
         const int chosen = need > 0 ? min(need, n) : 0;
-        for (int s = threadIdx.x; s < topk; s += kSelThreads) {
+        for (int s = threadIdx.x; s < topk; s += NT) {
             if (s == 0) final_row[0] = 0;
             else if (s == chosen + 1 && D > 0) final_row[s] = D;
             else if (s > chosen + (D > 0 ? 1 : 0)) final_row[s] = -1;
@@ -617,15 +642,16 @@ __device__ __forceinline__ void lse2_merge(float &m, float &s, float m2, float s
 // FROM_SCORES: the candidates' scores come from a table [B*Hkv][NR][nblk_max]
 // written by another scoring kernel (the aggregator variants) instead of
 // the pooled-query dots.
-template <int D, typename KcT, bool FROM_SCORES = false>
-__global__ void __launch_bounds__(kSelThreads) score_select_kernel(
+template <int D, typename KcT, bool FROM_SCORES = false, int NT = kSelThreads>
+__global__ void __launch_bounds__(NT) score_select_kernel(
     const float *__restrict__ Qbar, const KcT *__restrict__ Kc, int32_t *__restrict__ idx,
     uint64_t *__restrict__ part, int nblk_max, int Tq, int q_pos0, int qblk, int topk,
     float sm_scale, int CH, int maxchunks, int Hkv, const int32_t *__restrict__ q_pos,
     const float *__restrict__ scores = nullptr, int score_stride = 0)
 {
+    static_assert(FROM_SCORES || NT == kSelThreads, "the scoring path is written for kSelThreads threads");
     extern __shared__ uint64_t keys[];
-    __shared__ SelectShared sh;
+    __shared__ SelectSharedT<NT> sh;
     const int chunk = blockIdx.x, i = blockIdx.y, bg = blockIdx.z, NR = gridDim.y;
     const int qp = seq_q_pos(q_pos, bg / Hkv, q_pos0, Tq, nblk_max,
                              threadIdx.x == 0 && chunk == 0 && i == 0 && bg % Hkv == 0);
@@ -637,7 +663,15 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(
 
     if constexpr (FROM_SCORES) {
         const float *srow = scores + row * (score_stride ? score_stride : nblk_max) + j0;
-        for (int e = threadIdx.x; e < n; e += kSelThreads) keys[e] = make_key(__ldg(srow + e), j0 + e);
+        // four loads in flight per thread before their keys are stored
+        for (int e0 = threadIdx.x; e0 < n; e0 += 4 * NT) {
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; u++) v[u] = e0 + u * NT < n ? __ldg(srow + e0 + u * NT) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; u++)
+                if (e0 + u * NT < n) keys[e0 + u * NT] = make_key(v[u], j0 + e0 + u * NT);
+        }
     } else {
         score_chunk<D, KcT>(Qbar + row * D, Kc + ((long)bg * nblk_max + j0) * D, n, j0, sm_scale, keys);
     }

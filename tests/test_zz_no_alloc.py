@@ -11,12 +11,14 @@ The test calls the new entry point through the C ABI and checks that two
 calls in a row reproduce the selection of the workspace-taking entry point
 exactly (block indices are integer results, compared bit for bit).  Every
 case needs scratch memory, so every case reads and writes the static buffer:
-  * prefill_tiny: one chunk per row -- the scratch holds the pooled queries;
-  * prefill_chunked: rows of 2999 candidates split into chunks of 512 -- the
-    scratch also holds each chunk's top-m list, merged by a second kernel;
+  * prefill_tiny: the scratch holds the pooled queries and the rows' score
+    table;
+  * prefill_long_rows: rows of 2999 candidates, each selected whole from
+    the score table (a larger table);
   * decode_long_rows: per-token rows of 69999 candidates (a 4.48M-token
-    context), too long for the one-launch cluster path, so they take the
-    same pooled-query + chunk-list + merge route.
+    context), too long for the one-launch cluster path: the scratch holds
+    the pooled queries and each chunk's top-m list, merged by a second
+    kernel.
 The summaries of the two larger cases are drawn directly (the comparison is
 between two entry points on the same inputs, not against the oracle).
 This file is collected last on purpose.
@@ -33,7 +35,7 @@ pytestmark = pytest.mark.gpu
 # (name, workload keywords, compress the drawn keys (True) or draw summaries)
 CASES = [
     ("prefill_tiny", None, True),
-    ("prefill_chunked", dict(B=1, Tq=128, T_kv=64 * 3002, q_pos0=64 * 3000, qblk=64, Hq=16, Hkv=2,
+    ("prefill_long_rows", dict(B=1, Tq=128, T_kv=64 * 3002, q_pos0=64 * 3000, qblk=64, Hq=16, Hkv=2,
                              d=128, topk=16), False),
     ("decode_long_rows", dict(B=1, Tq=1, T_kv=64 * 70001, q_pos0=64 * 70001 - 1, qblk=1, Hq=16,
                               Hkv=2, d=128, topk=64), False),
@@ -73,7 +75,7 @@ def test_noalloc_selection_matches_workspace_entry_point(name, kw, compress):
     qbar_bytes = -(-w.B * w.Hkv * w.n_rows * w.d * 4 // 256) * 256
     assert need > 0, "this case must use the scratch buffer"
     if name != "prefill_tiny":
-        assert need > qbar_bytes, "this case must also keep per-chunk lists in the scratch"
+        assert need > qbar_bytes, "this case must also keep a score table or chunk lists in the scratch"
     assert need <= qsa.SELECT_SCRATCH_BYTES
     shape = (w.B, w.Hkv, w.n_rows, w.topk)
     ref = torch.full(shape, -7, dtype=torch.int32, device="cuda")
