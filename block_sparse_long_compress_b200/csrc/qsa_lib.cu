@@ -477,6 +477,25 @@ qsa_status compress_keys_impl(const char *name, const void *K, KcT *Kc, int B, i
 }
 
 
+// Score-table launch: one CTA per (64-row tile, 64-candidate tile) of the
+// candidates in [lo, hi) up to the last row's diagonal.
+struct TableLaunch {
+    dim3 grid;
+    int smem;
+};
+
+TableLaunch plan_table(int B, int Hkv, int Tq, int q_pos0, int lo, int hi, int d)
+{
+    constexpr int T = qsa::kTableTile;
+    const int NR = (Tq + 63) / 64;
+    const int Dmax = (q_pos0 + Tq - 1) / 64;
+    const int n = std::min(Dmax, hi) - lo;
+    TableLaunch tl;
+    tl.grid = dim3((unsigned)std::max(1, (n + T - 1) / T), (unsigned)((NR + T - 1) / T), (unsigned)(B * Hkv));
+    tl.smem = 2 * T * (d + 4) * (int)sizeof(float);
+    return tl;
+}
+
 // Pooling launch: the 16-byte column chunks of a token's heads, times up to
 // four token splits for rows of several tokens (at most 1024 threads).
 struct PoolLaunch {
@@ -507,14 +526,10 @@ qsa_status launch_score_select(const void *Q, const KcT *Kc, int32_t *idx, float
                                                                    pl.TS);
     if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
     if (qblk == 64) {
-        const int Dmax = (q_pos0 + Tq - 1) / 64;
-        constexpr int TT = qsa::kTableTile;
-        const dim3 tgrid((unsigned)std::max(1, (Dmax - 1 + TT - 1) / TT), (unsigned)((p.NR + TT - 1) / TT),
-                         (unsigned)(B * Hkv));
-        const int tsmem = 2 * TT * (D + 4) * (int)sizeof(float);
-        if ((st = set_smem(qsa::score_table_kernel<D, KcT>, tsmem)) != QSA_OK) return st;
-        qsa::score_table_kernel<D, KcT><<<tgrid, 256, tsmem, s>>>(Qbar, Kc, table, nblk_max, Tq, q_pos0, p.TS,
-                                                                  sm_scale, Hkv, q_pos, 1, INT_MAX, 0, nblk_max, 0);
+        const TableLaunch tl = plan_table(B, Hkv, Tq, q_pos0, 1, INT_MAX, D);
+        if ((st = set_smem(qsa::score_table_kernel<D, KcT>, tl.smem)) != QSA_OK) return st;
+        qsa::score_table_kernel<D, KcT><<<tl.grid, 256, tl.smem, s>>>(Qbar, Kc, table, nblk_max, Tq, q_pos0, p.TS,
+                                                                      sm_scale, Hkv, q_pos, 1, INT_MAX, 0, nblk_max, 0);
         if ((st = launched("score_table_kernel")) != QSA_OK) return st;
         if (p.wide) {
             auto kern = qsa::score_select_kernel<D, KcT, true, 1024>;
@@ -1102,8 +1117,7 @@ qsa_status qsa_score_select_local(const void *Q, const float *Kc_local, uint64_t
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const dim3 pgrid(NR, B);
     const PoolLaunch pl = plan_pool(Hq, d, 64, (long)NR * B);
-    constexpr int TT = qsa::kTableTile;
-    const dim3 tgrid((unsigned)std::max(1, (count + TT - 1) / TT), (unsigned)((NR + TT - 1) / TT), (unsigned)(B * Hkv));
+    const TableLaunch tl = plan_table(B, Hkv, Tq, q_pos0, first, blk_hi, d);
     qsa_status st;
     if (d == 128) {
         if ((st = set_smem(qsa::pool_queries_kernel<128>, pl.smem)) != QSA_OK) return st;
@@ -1111,11 +1125,10 @@ qsa_status qsa_score_select_local(const void *Q, const float *Kc_local, uint64_t
                                                                          64, pl.TS);
         if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
         if (count > 0) {
-            const int tsmem = 2 * TT * (128 + 4) * (int)sizeof(float);
-            if ((st = set_smem(qsa::score_table_kernel<128, float>, tsmem)) != QSA_OK) return st;
-            qsa::score_table_kernel<128, float><<<tgrid, 256, tsmem, s>>>(Qbar, Kc_local, table, nblk_max, Tq, q_pos0,
-                                                                          TS, sm_scale, Hkv, nullptr, first, blk_hi,
-                                                                          blk_lo, kc_n, first);
+            if ((st = set_smem(qsa::score_table_kernel<128, float>, tl.smem)) != QSA_OK) return st;
+            qsa::score_table_kernel<128, float><<<tl.grid, 256, tl.smem, s>>>(Qbar, Kc_local, table, nblk_max, Tq,
+                                                                              q_pos0, TS, sm_scale, Hkv, nullptr, first,
+                                                                              blk_hi, blk_lo, kc_n, first);
             if ((st = launched("score_table_kernel")) != QSA_OK) return st;
         }
     } else {
@@ -1124,11 +1137,10 @@ qsa_status qsa_score_select_local(const void *Q, const float *Kc_local, uint64_t
                                                                         64, pl.TS);
         if ((st = launched("pool_queries_kernel")) != QSA_OK) return st;
         if (count > 0) {
-            const int tsmem = 2 * TT * (64 + 4) * (int)sizeof(float);
-            if ((st = set_smem(qsa::score_table_kernel<64, float>, tsmem)) != QSA_OK) return st;
-            qsa::score_table_kernel<64, float><<<tgrid, 256, tsmem, s>>>(Qbar, Kc_local, table, nblk_max, Tq, q_pos0,
-                                                                         TS, sm_scale, Hkv, nullptr, first, blk_hi,
-                                                                         blk_lo, kc_n, first);
+            if ((st = set_smem(qsa::score_table_kernel<64, float>, tl.smem)) != QSA_OK) return st;
+            qsa::score_table_kernel<64, float><<<tl.grid, 256, tl.smem, s>>>(Qbar, Kc_local, table, nblk_max, Tq,
+                                                                             q_pos0, TS, sm_scale, Hkv, nullptr, first,
+                                                                             blk_hi, blk_lo, kc_n, first);
             if ((st = launched("score_table_kernel")) != QSA_OK) return st;
         }
     }

@@ -663,13 +663,13 @@ __global__ void __launch_bounds__(NT) score_select_kernel(
 
     if constexpr (FROM_SCORES) {
         const float *srow = scores + row * (score_stride ? score_stride : nblk_max) + j0;
-        // four loads in flight per thread before their keys are stored
-        for (int e0 = threadIdx.x; e0 < n; e0 += 4 * NT) {
-            float v[4];
+        // eight loads in flight per thread before their keys are stored
+        for (int e0 = threadIdx.x; e0 < n; e0 += 8 * NT) {
+            float v[8];
 #pragma unroll
-            for (int u = 0; u < 4; u++) v[u] = e0 + u * NT < n ? __ldg(srow + e0 + u * NT) : 0.f;
+            for (int u = 0; u < 8; u++) v[u] = e0 + u * NT < n ? __ldg(srow + e0 + u * NT) : 0.f;
 #pragma unroll
-            for (int u = 0; u < 4; u++)
+            for (int u = 0; u < 8; u++)
                 if (e0 + u * NT < n) keys[e0 + u * NT] = make_key(v[u], j0 + e0 + u * NT);
         }
     } else {
@@ -691,88 +691,103 @@ __global__ void __launch_bounds__(NT) score_select_kernel(
 // (row i's are blocks 1 .. D_i - 1), so the scores of a 64-row x 64-candidate
 // tile are an fp32 matrix product Qbar_tile (64 x D) * Kc_tile^T (D x 64)
 // over shared memory: every summary and pooled query crosses L2 once per
-// tile instead of once per row.  Each thread forms a 4 x 4 block of dots
-// (rows 4 ty .. 4 ty + 3, candidates tx, tx + 16, tx + 32, tx + 48) with
-// fp32 FMAs in increasing d; rows are padded to D + 4 floats so the
-// 16-byte shared loads of the 16 candidate columns a warp reads fall in
-// distinct banks.  The scores go into a table [B*Hkv][NR][stride] that
-// score_select_kernel<.., true> selects from; tiles wholly past their rows'
-// diagonals exit at once.
-// grid (ceil(max candidates / 64), ceil(NR / 64), B*Hkv); 256 threads;
-// dynamic shared memory 2 * 64 * (D + 4) * 4 bytes.
-constexpr int kTableTile = 64;
-
+// tile instead of once per row.  One CTA per tile; the tiles go to shared
+// memory by cp.async (fp32; bf16 summaries are widened on the way).  Each
+// thread forms a 4 x 4 block of dots (rows 4 ty .. 4 ty + 3, candidates tx,
+// tx + 16, tx + 32, tx + 48) with fp32 FMAs in increasing d; rows are padded
+// to D + 4 floats so the 16-byte shared loads of the 16 candidate columns a
+// warp reads fall in distinct banks.  The scores go into a table
+// [B*Hkv][NR][stride] that score_select_kernel<.., true> selects from;
+// tiles wholly past their rows' diagonals are skipped.
 // Sharded caches: the candidates are restricted to blocks [lo, hi) (lo >= 1),
 // Kc holds the summaries of blocks kc_lo .. kc_lo + kc_n - 1 of each (b, g)
 // (the rank's own range), and table column c is block tab_lo + c.  The
 // whole cache: lo = 1, hi = INT_MAX, kc_lo = 0, kc_n = T_kv_max / 64,
 // tab_lo = 0 (column = block index).
+// grid (ceil(max candidates / 64), ceil(NR / 64), B*Hkv); 256 threads;
+// dynamic shared memory 2 * 64 * (D + 4) * 4 bytes.
+constexpr int kTableTile = 64;
+
 template <int D, typename KcT>
 __global__ void __launch_bounds__(256) score_table_kernel(
     const float *__restrict__ Qbar, const KcT *__restrict__ Kc, float *__restrict__ table, int nblk_max, int Tq,
     int q_pos0, int stride, float sm_scale, int Hkv, const int32_t *__restrict__ q_pos, int lo, int hi, int kc_lo,
     int kc_n, int tab_lo)
 {
-    constexpr int T = kTableTile, LD = D + 4;
+    constexpr int T = kTableTile, LD = D + 4, CPR = D / 4;   // CPR: 16-byte chunks (of fp32) per row
     extern __shared__ __align__(16) float tsm[];
-    float *qs = tsm;            // [T][LD] pooled queries of the tile's rows
-    float *ks = tsm + T * LD;   // [T][LD] summaries of the tile's candidates
+    float *qs = tsm;                  // [T][LD] pooled queries of the tile's rows
+    float *ks = tsm + T * LD;         // [T][LD] summaries of the tile's candidates
     const int bg = blockIdx.z, NR = (Tq + 63) / 64;
     const int qp = seq_q_pos(q_pos, bg / Hkv, q_pos0, Tq, nblk_max, false);
     const int r0 = blockIdx.y * T, nr = min(T, NR - r0);
-    const int j0 = lo + blockIdx.x * T;
-    // candidates of the tile that some row of it has (j < D of its last row)
+    // candidates of the CTA that some row of its tile has (j < D of the last row)
     const int Dlast = (qp + min((r0 + nr) * 64, Tq) - 1) / 64;
-    const int nc = min(T, min(Dlast, hi) - j0);
-    if (nc <= 0) return;
+    const int j0 = lo + blockIdx.x * T;
+    const int jend = min(min(Dlast, hi), j0 + T);
+    if (jend <= j0) return;
     const int tid = threadIdx.x;
-    // tiles into shared memory: 16-byte chunks, rows past the tile are zero
-    constexpr int CPR = D / 4;   // 16-byte chunks (of fp32) per row
+    // summaries of candidates j0 .. j0 + T - 1 (zero past jend)
+    {
+        for (int e = tid; e < T * CPR; e += 256) {
+            const int rr = e / CPR, c = e % CPR;
+            const bool valid = j0 + rr < jend;
+            const KcT *src = Kc + ((long)bg * kc_n + (valid ? j0 + rr - kc_lo : 0)) * D + 4 * c;
+            if constexpr (sizeof(KcT) == 4) {
+                cp_async16(ks + rr * LD + 4 * c, src, valid);
+            } else {
+                float k4[4] = {0.f, 0.f, 0.f, 0.f};
+                if (valid) load_summary<4>(src, k4);
+                *reinterpret_cast<float4 *>(ks + rr * LD + 4 * c) = make_float4(k4[0], k4[1], k4[2], k4[3]);
+            }
+        }
+    }
     for (int e = tid; e < T * CPR; e += 256) {
         const int rr = e / CPR, c = e % CPR;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (rr < nr) v = *reinterpret_cast<const float4 *>(Qbar + ((long)bg * NR + r0 + rr) * D + 4 * c);
-        *reinterpret_cast<float4 *>(qs + rr * LD + 4 * c) = v;
-        float k4[4] = {0.f, 0.f, 0.f, 0.f};
-        if (rr < nc) load_summary<4>(Kc + ((long)bg * kc_n + (j0 - kc_lo) + rr) * D + 4 * c, k4);
-        *reinterpret_cast<float4 *>(ks + rr * LD + 4 * c) = make_float4(k4[0], k4[1], k4[2], k4[3]);
+        const bool valid = rr < nr;
+        cp_async16(qs + rr * LD + 4 * c, Qbar + ((long)bg * NR + r0 + (valid ? rr : 0)) * D + 4 * c, valid);
     }
+    cp_async_commit();
+    cp_async_wait<0>();
     __syncthreads();
     const int ty = tid >> 4, tx = tid & 15;
-    float acc[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; i++)
-#pragma unroll
-        for (int jj = 0; jj < 4; jj++) acc[i][jj] = 0.f;
-    const float *qrow = qs + (4 * ty) * LD;
-    const float *krow = ks + tx * LD;
-#pragma unroll 4
-    for (int d = 0; d < D; d += 4) {
-        float4 a[4], b[4];
-#pragma unroll
-        for (int i = 0; i < 4; i++) a[i] = *reinterpret_cast<const float4 *>(qrow + i * LD + d);
-#pragma unroll
-        for (int jj = 0; jj < 4; jj++) b[jj] = *reinterpret_cast<const float4 *>(krow + 16 * jj * LD + d);
+    {
+        float acc[4][4];
 #pragma unroll
         for (int i = 0; i < 4; i++)
 #pragma unroll
+            for (int jj = 0; jj < 4; jj++) acc[i][jj] = 0.f;
+        const float *qrow = qs + (4 * ty) * LD;
+        const float *krow = ks + tx * LD;
+#pragma unroll 4
+        for (int d = 0; d < D; d += 4) {
+            float4 a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) a[i] = *reinterpret_cast<const float4 *>(qrow + i * LD + d);
+#pragma unroll
+            for (int jj = 0; jj < 4; jj++) b[jj] = *reinterpret_cast<const float4 *>(krow + 16 * jj * LD + d);
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+#pragma unroll
+                for (int jj = 0; jj < 4; jj++) {
+                    acc[i][jj] = fmaf(a[i].x, b[jj].x, acc[i][jj]);
+                    acc[i][jj] = fmaf(a[i].y, b[jj].y, acc[i][jj]);
+                    acc[i][jj] = fmaf(a[i].z, b[jj].z, acc[i][jj]);
+                    acc[i][jj] = fmaf(a[i].w, b[jj].w, acc[i][jj]);
+                }
+        }
+        const int nc = min(T, jend - j0);
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int rr = 4 * ty + i;
+            if (rr >= nr) break;
+            const int Drow = (qp + min((r0 + rr + 1) * 64, Tq) - 1) / 64;
+            float *trow = table + ((long)bg * NR + r0 + rr) * stride + (j0 - tab_lo);
+#pragma unroll
             for (int jj = 0; jj < 4; jj++) {
-                acc[i][jj] = fmaf(a[i].x, b[jj].x, acc[i][jj]);
-                acc[i][jj] = fmaf(a[i].y, b[jj].y, acc[i][jj]);
-                acc[i][jj] = fmaf(a[i].z, b[jj].z, acc[i][jj]);
-                acc[i][jj] = fmaf(a[i].w, b[jj].w, acc[i][jj]);
+                const int e = tx + 16 * jj;
+                if (e < nc && j0 + e < Drow) trow[e] = acc[i][jj] * sm_scale;
             }
-    }
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        const int rr = 4 * ty + i;
-        if (rr >= nr) break;
-        const int Drow = (qp + min((r0 + rr + 1) * 64, Tq) - 1) / 64;
-        float *trow = table + ((long)bg * NR + r0 + rr) * stride + (j0 - tab_lo);
-#pragma unroll
-        for (int jj = 0; jj < 4; jj++) {
-            const int e = tx + 16 * jj;
-            if (e < nc && j0 + e < Drow) trow[e] = acc[i][jj] * sm_scale;
         }
     }
 }

@@ -263,3 +263,53 @@ def test_sharded_class_over_a_one_rank_nccl_group():
         assert err.max() <= 1e-2 and err.mean() <= 1e-3, (err.max(), err.mean())
     finally:
         torch.distributed.destroy_process_group()
+
+
+@pytest.mark.gpu
+def test_sharded_kernels_at_chunked_1m():
+    """chunked_1m (4096 new tokens after a 1,048,576-token cache, top-64)
+    split over 4 ranks, emulated one after another on one GPU: the merged
+    indices equal the whole-cache path's bit for bit on all 128 rows, and the
+    merged outputs of 512 tokens (the chunk's first and last query blocks
+    and 384 drawn at random) are within the tolerance of the oracle."""
+    import block_sparse_long_compress_b200 as qsa
+    w = synthetic.CONFIGS["chunked_1m"]
+    x = synthetic.generate(w, DEV)
+    Q, K, V = x["Q"], x["K"], x["V"]
+    nb = w.T_kv // 64
+    run = qsa.QSAPrefill(w.B, w.Tq, w.Hq, w.Hkv, w.d, w.T_kv, w.topk, w.q_pos0, device=DEV)
+    run.precompress_cache(K)
+    run(Q, K, V)
+    assert qsa.device_status()[0] == "QSA_OK"
+    ranges = qsa.shard_ranges(nb, 4)
+    nlists = max(qsa.select_local_lists(w.Tq, w.q_pos0, lo, hi) for lo, hi in ranges)
+    lists = []
+    for lo, hi in ranges:
+        L = torch.empty((w.B, w.Hkv, w.n_rows, nlists, 62), dtype=torch.int64, device=DEV)
+        qsa.score_select_local(Q, run.Kc[:, :, lo:hi].contiguous(), L, w.q_pos0, lo, hi, w.topk, w.sm_scale)
+        lists.append(L)
+    idx = torch.full_like(run.idx, -7)
+    qsa.merge_select_lists(torch.stack(lists), idx, w.Tq, w.q_pos0)
+    assert qsa.device_status()[0] == "QSA_OK"
+    assert torch.equal(idx, run.idx)
+    Os, ls = [], []
+    for lo, hi in ranges:
+        Kl, Vl = K[:, :, 64 * lo:64 * hi].contiguous(), V[:, :, 64 * lo:64 * hi].contiguous()
+        O_r = torch.empty_like(Q)
+        lse_r = torch.empty((w.B, w.Tq, w.Hq), dtype=torch.float32, device=DEV)
+        qsa.sparse_attn_prefill_local(Q, Kl, Vl, idx, O_r, lse_r, w.q_pos0, lo, hi, w.sm_scale)
+        Os.append(O_r)
+        ls.append(lse_r)
+        del Kl, Vl
+    assert qsa.device_status()[0] == "QSA_OK"
+    O = torch.empty_like(Q)
+    qsa.merge_partials(torch.stack(Os), torch.stack(ls), O)
+    assert qsa.device_status()[0] == "QSA_OK"
+    rng = np.random.RandomState(29)
+    toks = np.unique(np.concatenate([np.arange(64), np.arange(w.Tq - 64, w.Tq),
+                                     rng.choice(np.arange(64, w.Tq - 64), 384, replace=False)]))
+    O_ref = oracle.attend(Q.cpu(), K.cpu(), V.cpu(), idx.cpu().numpy(), w.q_pos0, w.qblk, w.sm_scale, tokens=toks)
+    O_gpu = O.reshape(w.Tq, w.Hq, w.d)[torch.from_numpy(toks).to(DEV)].float().cpu().numpy()
+    err = np.abs(O_gpu - O_ref)
+    print(f"sharded chunked_1m (4 ranks): {err.size} outputs, max|err| {err.max():.3e} mean {err.mean():.3e}")
+    assert err.max() <= 1e-2 and err.mean() <= 1e-3, (err.max(), err.mean())
