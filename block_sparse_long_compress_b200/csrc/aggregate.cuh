@@ -22,9 +22,9 @@
 // tiles: warp 0 loads the query block once and streams summary tiles
 // through a 2-stage ring (TMA, 128-byte swizzle), warp 1 issues the MMAs
 // (M = 128, N = 256, K = 128: 8 MMAs per N tile) into one of two TMEM
-// accumulators, warps 2-5 reduce the other (for the softmax-sum warps 2-9:
-// two warps per TMEM lane quarter, each taking half of the columns; the
-// halves meet in shared memory once per candidate tile).  Scores go to a table
+// accumulators, warps 2-5 reduce the other (for the softmax-sum warps 2-17:
+// four warps per TMEM lane quarter, each taking a quarter of the columns;
+// the quarters meet in shared memory once per candidate tile).  Scores go to a table
 // [B][Hkv][NR][nblk_max] (candidates 1 .. D-1 of each row); the chunked
 // selection turns the table into indices.
 //
@@ -55,9 +55,9 @@ struct MaxScoreCfg {
     static constexpr int KSTAGE_BYTES = 2 * KHALF_BYTES;
     static constexpr int NS = 2;
     static constexpr int SMEM_BYTES = Q_BYTES + NS * KSTAGE_BYTES + 1024;
-    // producer, issuer and 4 epilogue warps (max), or 8 (softmax-sum, whose
-    // per-column exponentials need the second warp per scheduler)
-    __host__ __device__ static constexpr int threads(bool softmax) { return 64 + 32 * (softmax ? 8 : 4); }
+    // producer, issuer and 4 epilogue warps (max), or 16 (softmax-sum: the
+    // exponentials' dependency chains need four warps per scheduler)
+    __host__ __device__ static constexpr int threads(bool softmax) { return 64 + 32 * (softmax ? 16 : 4); }
     static constexpr int TMEM_COLS = 2 * N;             // two fp32 accumulators
     static_assert(N % G == 0 && 64 % TOKN == 0, "tile shape");
 };
@@ -73,13 +73,13 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::threads(SOFTMAX), 1) block_max
     using C = MaxScoreCfg<G>;
     constexpr int THREADS = C::threads(SOFTMAX);
     constexpr int EPI = (THREADS - 64) / 32;            // epilogue warps
-    constexpr int HALVES = EPI / 4;                     // column ranges per TMEM lane quarter (softmax: 2)
+    constexpr int SPLIT = EPI / 4;                      // column ranges per TMEM lane quarter (softmax: 4)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t q_full, k_full[C::NS], k_empty[C::NS], t_full[2], t_empty[2];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag, issued_k, issued_mma;
-    __shared__ float rstat[SOFTMAX ? 64 * G : 1];   // SOFTMAX: max + log2(sum) per (token, head) row
-    __shared__ float xch[128];                      // the second column half's partial per candidate
+    __shared__ __align__(16) float nrstat[SOFTMAX ? 64 * G : 4];   // SOFTMAX: -(max + log2 sum) per (token, head) row
+    __shared__ float xch[SPLIT > 1 ? SPLIT - 1 : 1][128];   // the other column ranges' partials per candidate
 
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *q_smem = base;
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::threads(SOFTMAX), 1) block_max
         // 2^(z - max) / sum = 2^(z - (max + log2 sum))
         const float *st = stats + ((long)bg * NR + i) * (64 * G) * 2;
         for (int r = threadIdx.x; r < 64 * G; r += THREADS)
-            rstat[r] = st[2 * r + 1] > 0.f ? st[2 * r] + __log2f(st[2 * r + 1]) : INFINITY;
+            nrstat[r] = st[2 * r + 1] > 0.f ? -(st[2 * r] + __log2f(st[2 * r + 1])) : -INFINITY;
     }
     tc_fence_before();
     __syncthreads();
@@ -219,46 +219,73 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::threads(SOFTMAX), 1) block_max
       } else {
         // ------------------------------------------- epilogue (warps 2-9)
         const int quarter = warp & 3;                  // the TMEM lanes this warp may access
-        const int half = (warp - 2) >> 2;              // the columns it reduces (HALVES ranges)
+        const int part = (warp - 2) >> 2;              // the columns it reduces (one of SPLIT ranges)
         const int m = 32 * quarter + lane;             // candidate within the tile
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
         const float sc2 = sm_scale * 1.4426950408889634f;
-        float best = 0.f;
+        const uint64_t s2 = f2_pack(sc2, sc2);
+        uint64_t best2 = f2_pack(0.f, 0.f);            // two partial sums (even, odd columns)
         for (int w = 0; w < nwork; w++) {
             const int k = w / C::NT, nt = w % C::NT, buf = w & 1;
             // warp-uniform: the TMEM loads below are collective.  A failed
             // wait (an abort, after which every wait returns at once) skips
-            // the work but not the exchanges below: all eight warps must
+            // the work but not the exchanges below: all epilogue warps must
             // reach the same named barriers
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&t_full[buf], (w >> 1) & 1, abort, 74));
             if (ok) tc_fence_after();
 #pragma unroll 1
-            for (int c = half * (C::N / HALVES); ok && c < (half + 1) * (C::N / HALVES); c += 32) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_base + buf * C::N + c, r);
-                tmem_wait_ld();
+            // the warp's 64 columns: both 32-column loads in flight, one wait
+            static_assert(C::N / SPLIT == 64, "two TMEM loads per epilogue warp");
+            auto chunk = [&](const uint32_t (&r)[32], int c) {
 #pragma unroll
                 for (int tt = 0; tt < 32 / G; tt++) {
                     const int tl = nt * C::TOKN + c / G + tt;    // token of these G columns, in the block
                     if (i * 64 + tl < Tq) {
-                        // the rows' shares of this block
+                        // the rows' shares of this block: 2^(z sc2 - (max + log2 sum)),
+                        // arguments two at a time, row statistics four at a time
 #pragma unroll
-                        for (int h = 0; h < G; h++)
-                            best += fast_exp2(__uint_as_float(r[tt * G + h]) * sc2 - rstat[tl * G + h]);
+                        for (int h = 0; h < G; h += 4) {
+                            const float4 ns = *reinterpret_cast<const float4 *>(&nrstat[tl * G + h]);
+                            const uint64_t a = f2_fma(f2_pack(__uint_as_float(r[tt * G + h]), __uint_as_float(r[tt * G + h + 1])),
+                                                      s2, f2_pack(ns.x, ns.y));
+                            const uint64_t b = f2_fma(f2_pack(__uint_as_float(r[tt * G + h + 2]), __uint_as_float(r[tt * G + h + 3])),
+                                                      s2, f2_pack(ns.z, ns.w));
+                            float a0, a1, b0, b1;
+                            f2_unpack(a, a0, a1);
+                            f2_unpack(b, b0, b1);
+                            best2 = f2_add(best2, f2_pack(fast_exp2(a0), fast_exp2(a1)));
+                            best2 = f2_add(best2, f2_pack(fast_exp2(b0), fast_exp2(b1)));
+                        }
                     }
                 }
+            };
+            if (ok) {
+                const int c = part * 64;
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_base + buf * C::N + c, r0);
+                tmem_ld32(tmem + lane_base + buf * C::N + c + 32, r1);
+                tmem_wait_ld();
+                chunk(r0, c);
+                chunk(r1, c + 32);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&t_empty[buf]);
             if (nt == C::NT - 1) {
-                // the two column halves of each candidate meet
-                if (half == 1) xch[m] = best;
+                // the column ranges of each candidate meet
+                float e0, e1;
+                f2_unpack(best2, e0, e1);
+                float best = e0 + e1;
+                if (part > 0) xch[part - 1][m] = best;
                 named_barrier_sync(1, 32 * EPI);
                 const int j = 1 + C::M * k + m;
-                if (half == 0 && j < Dg) scores[((long)bg * NR + i) * nblk_max + j] = best + xch[m];
+                if (part == 0 && j < Dg) {
+#pragma unroll
+                    for (int q = 0; q < SPLIT - 1; q++) best += xch[q][m];
+                    scores[((long)bg * NR + i) * nblk_max + j] = best;
+                }
                 named_barrier_sync(1, 32 * EPI);
-                best = 0.f;
+                best2 = f2_pack(0.f, 0.f);
             }
         }
       }
@@ -287,62 +314,80 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::threads(SOFTMAX), 1) block_max
 
 // First pass of the softmax-sum: per (token, head) row of the query block,
 // the base-2 (max, sum of 2^(z - max)) of z = sm_scale log2(e) <q, Kc_j>
-// over the blocks j in 0 .. D-1.  One CTA per (query block, sequence, group,
-// 128-row M tile of 128/G tokens x G heads); the blocks stream through in
-// N tiles of 256 (the same warp roles as block_max_scores_kernel).  Output:
+// over the blocks j in 0 .. D-1.  A work unit is (sequence and group, query
+// block, 128-row M tile of 128/G tokens x G heads); the blocks stream
+// through it in N tiles of 256.  Persistent: one CTA per SM walks the units
+// u = blockIdx.x + n * gridDim.x (the query blocks with the most blocks
+// first) as one stream -- the K ring, the two TMEM accumulators and their
+// barriers count tiles across units, and the M tile's queries sit in one of
+// two slots, so the next unit's queries and first tiles load while the
+// current unit's last tiles are reduced.  Warp roles as in
+// block_max_scores_kernel (producer, issuer, 16 epilogue warps, four per
+// TMEM lane quarter, each on a quarter of every tile's columns).  Output:
 // stats[(bg*NR + i)][64*G][2], row (token, head) = t_local*G + h.
 template <int G>
 struct SoftmaxStatsCfg {
     static constexpr int D = 128;
-    static constexpr int M = 128;                       // (token, head) rows per CTA
+    static constexpr int M = 128;                       // (token, head) rows per unit
     static constexpr int N = 256;                       // blocks per tile
-    static constexpr int TOKM = M / G;                  // tokens per CTA
+    static constexpr int TOKM = M / G;                  // tokens per unit
     static constexpr int NMT = 64 / TOKM;               // M tiles per query block
     static constexpr int QHALF_BYTES = M * 128;         // 16 KB
-    static constexpr int Q_BYTES = 2 * QHALF_BYTES;
+    static constexpr int Q_BYTES = 2 * QHALF_BYTES;     // one slot
     static constexpr int KHALF_BYTES = N * 128;         // 32 KB
     static constexpr int KSTAGE_BYTES = 2 * KHALF_BYTES;
     static constexpr int NS = 2;
-    static constexpr int SMEM_BYTES = Q_BYTES + NS * KSTAGE_BYTES + 1024;
-    static constexpr int THREADS = 320;                 // producer, issuer, 8 epilogue warps
+    static constexpr int SMEM_BYTES = 2 * Q_BYTES + NS * KSTAGE_BYTES + 1024;
+    static constexpr int SPLIT = 4;                     // epilogue warps per TMEM lane quarter
+    static constexpr int EPI = 4 * SPLIT;
+    static constexpr int THREADS = 64 + 32 * EPI;       // producer, issuer, epilogue warps
     static constexpr int TMEM_COLS = 2 * N;
 };
 
 template <int G>
 __global__ void __launch_bounds__(SoftmaxStatsCfg<G>::THREADS, 1) block_softmax_stats_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
-    float *__restrict__ stats, int Tq, int q_pos0, int nblk_max, int Hkv, float sm_scale)
+    float *__restrict__ stats, int Tq, int q_pos0, int nblk_max, int Hkv, float sm_scale, int NR, int nunits)
 {
     using C = SoftmaxStatsCfg<G>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    __shared__ uint64_t q_full, k_full[C::NS], k_empty[C::NS], t_full[2], t_empty[2];
+    __shared__ uint64_t q_full[2], q_empty[2], k_full[C::NS], k_empty[C::NS], t_full[2], t_empty[2];
     __shared__ uint32_t tmem_base;
-    __shared__ int abort_flag, issued_k, issued_mma;
+    __shared__ int abort_flag, issued_q, issued_k, issued_mma;
+    __shared__ float xm[2][C::SPLIT - 1][128], xs[2][C::SPLIT - 1][128];   // the column ranges meet here (slot = unit parity)
 
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *q_smem = base;
-    uint8_t *k_smem = base + C::Q_BYTES;
-    const int i = blockIdx.x / C::NMT, mt = blockIdx.x % C::NMT, bg = blockIdx.y, NR = gridDim.x / C::NMT;
-    const int b = bg / Hkv, g = bg % Hkv;
+    uint8_t *q_smem = base;                             // two slots
+    uint8_t *k_smem = base + 2 * C::Q_BYTES;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t_last = min((i + 1) * 64, Tq) - 1;
-    const int Dg = (q_pos0 + t_last) / 64;              // blocks 0 .. Dg-1 normalise
-    const int ntiles = (Dg + C::N - 1) / C::N;
-    if (Dg < 2) return;                                 // no candidate: nothing reads these rows
+    // unit u -> (bg, i, mt) and the row's diagonal block Dg (blocks 0 .. Dg-1
+    // normalise); units with Dg < 2 have no candidate and are skipped by
+    // every role alike
+    auto unit = [&](int u, int &bg, int &i, int &mt) -> int {
+        const int per = NR * C::NMT;
+        bg = u / per;
+        const int rem = u - bg * per;
+        i = NR - 1 - rem / C::NMT;
+        mt = rem % C::NMT;
+        return (q_pos0 + min((i + 1) * 64, Tq) - 1) / 64;
+    };
+
     if (threadIdx.x == 0) {
         abort_flag = 0;
+        issued_q = 0;
         issued_k = 0;
         issued_mma = 0;
-        mbar_init(&q_full, 1);
+#pragma unroll
+        for (int s = 0; s < 2; s++) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
+            mbar_init(&t_full[s], 1);
+            mbar_init(&t_empty[s], C::EPI);
+        }
 #pragma unroll
         for (int s = 0; s < C::NS; s++) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
-        }
-#pragma unroll
-        for (int s = 0; s < 2; s++) {
-            mbar_init(&t_full[s], 1);
-            mbar_init(&t_empty[s], 8);
         }
         fence_barrier_init();
     }
@@ -357,37 +402,64 @@ __global__ void __launch_bounds__(SoftmaxStatsCfg<G>::THREADS, 1) block_softmax_
     volatile int *abort = &abort_flag;
 
     if (warp == 0) {
+        // ------------------------------------------------------ producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(&q_full, C::Q_BYTES);
-#pragma unroll
-            for (int h = 0; h < 2; h++)
-                tma_load_3d(q_smem + h * C::QHALF_BYTES, &tmQ, &q_full, h * 64, g * G, b * Tq + i * 64 + mt * C::TOKM);
-            int k = 0;
-            for (; k < ntiles; k++) {
-                const int st = k % C::NS;
-                if (k >= C::NS && !mbar_wait(&k_empty[st], ((k / C::NS) - 1) & 1, abort, 80)) break;
-                fence_proxy_async_smem();
-                mbar_arrive_expect_tx(&k_full[st], C::KSTAGE_BYTES);
-                const int row = bg * nblk_max + C::N * k;   // host checks B*Hkv*nblk_max < 2^31
+            int kt = 0, un = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+                int bg, i, mt;
+                const int Dg = unit(u, bg, i, mt);
+                if (Dg < 2) continue;
+                const int b = bg / Hkv, g = bg % Hkv, qs = un & 1;
+                if (un >= 2 && !mbar_wait(&q_empty[qs], ((un >> 1) - 1) & 1, abort, 88)) break;
+                mbar_arrive_expect_tx(&q_full[qs], C::Q_BYTES);
 #pragma unroll
                 for (int h = 0; h < 2; h++)
-                    tma_load_2d(k_smem + st * C::KSTAGE_BYTES + h * C::KHALF_BYTES, &tmKc, &k_full[st], h * 64, row);
+                    tma_load_3d(q_smem + qs * C::Q_BYTES + h * C::QHALF_BYTES, &tmQ, &q_full[qs], h * 64, g * G,
+                                b * Tq + i * 64 + mt * C::TOKM);
+                un++;
+                const int ntiles = (Dg + C::N - 1) / C::N;
+                for (int k = 0; k < ntiles; k++, kt++) {
+                    const int st = kt % C::NS;
+                    if (kt >= C::NS && !mbar_wait(&k_empty[st], ((kt / C::NS) - 1) & 1, abort, 80)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive_expect_tx(&k_full[st], C::KSTAGE_BYTES);
+                    const int row = bg * nblk_max + C::N * k;   // host checks B*Hkv*nblk_max < 2^31
+#pragma unroll
+                    for (int h = 0; h < 2; h++)
+                        tma_load_2d(k_smem + st * C::KSTAGE_BYTES + h * C::KHALF_BYTES, &tmKc, &k_full[st], h * 64, row);
+                }
             }
-            issued_k = k;
+            issued_q = un;
+            issued_k = kt;
         }
     } else if (warp == 1) {
+        // ------------------------------------------- MMA issuer (whole warp)
         constexpr uint32_t idesc = umma_idesc_bf16(C::M, C::N, 0, 0);
-        const uint64_t qd = umma_smem_desc(smem_u32(q_smem), 16, 1024);
         const uint64_t kd = umma_smem_desc(smem_u32(k_smem), 16, 1024);
         auto wait_all = [&](uint64_t *bar, uint32_t parity, int where) -> bool {
             return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, where));
         };
-        int k = 0;
-        if (wait_all(&q_full, 0, 81)) {
-            for (; k < ntiles; k++) {
-                const int st = k % C::NS, buf = k & 1;
-                if (!wait_all(&k_full[st], (k / C::NS) & 1, 82)) break;
-                if (k >= 2 && !wait_all(&t_empty[buf], ((k >> 1) - 1) & 1, 83)) break;
+        int kt = 0, un = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+            int bg, i, mt;
+            const int Dg = unit(u, bg, i, mt);
+            if (Dg < 2) continue;
+            const int qs = un & 1;
+            if (!wait_all(&q_full[qs], (un >> 1) & 1, 81)) break;
+            const uint64_t qd = umma_smem_desc(smem_u32(q_smem + qs * C::Q_BYTES), 16, 1024);
+            const int ntiles = (Dg + C::N - 1) / C::N;
+            for (int k = 0; k < ntiles; k++) {
+                const int st = kt % C::NS, buf = kt & 1;
+                if (!wait_all(&k_full[st], (kt / C::NS) & 1, 82) ||
+                    (kt >= 2 && !wait_all(&t_empty[buf], ((kt >> 1) - 1) & 1, 83))) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 if (elect_one()) {
 #pragma unroll
@@ -400,73 +472,116 @@ __global__ void __launch_bounds__(SoftmaxStatsCfg<G>::THREADS, 1) block_softmax_
                     umma_commit(&k_empty[st]);
                 }
                 __syncwarp();
+                kt++;
             }
+            if (!ok) break;
+            // the slot's queries are free once the unit's MMAs are done
+            if (elect_one()) umma_commit(&q_empty[qs]);
+            __syncwarp();
+            un++;
         }
-        if (lane == 0) issued_mma = k;
+        if (lane == 0) issued_mma = kt;
     } else {
+        // ------------------------------------------- epilogue (warps 2-9)
         const int quarter = warp & 3;
-        const int half = (warp - 2) >> 2;              // the half of each tile's blocks it takes
+        const int part = (warp - 2) >> 2;              // the range of each tile's blocks it takes
         const int r = 32 * quarter + lane;             // (token, head) row of the M tile
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
         const float sc2 = sm_scale * 1.4426950408889634f;
-        float m_run = -INFINITY, s_run = 0.f;
-        int k = 0;
-        for (; k < ntiles; k++) {
-            const int buf = k & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&t_full[buf], (k >> 1) & 1, abort, 84))) break;
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = half * (C::N / 2); c < (half + 1) * (C::N / 2); c += 32) {
-                const int j0 = C::N * k + c;            // block of column 0 of this chunk (uniform)
-                if (j0 >= Dg) break;
-                uint32_t v[32];
-                tmem_ld32(tmem + lane_base + buf * C::N + c, v);
-                tmem_wait_ld();
-                float x[32];
-                float mx = -INFINITY;
-                if (j0 + 32 <= Dg) {
+        const uint64_t s2 = f2_pack(sc2, sc2);
+        int kt = 0, un = 0;
+        for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+            int bg, i, mt;
+            const int Dg = unit(u, bg, i, mt);
+            if (Dg < 2) continue;
+            const int ntiles = (Dg + C::N - 1) / C::N;
+            float m_run = -INFINITY, s_run = 0.f;
+            // a failed wait (an abort, after which every wait returns at
+            // once) skips the work but not the exchange below: all
+            // epilogue warps reach the same named barriers
+            bool ok = true;
+            for (int k = 0; k < ntiles; k++, kt++) {
+                const int buf = kt & 1;
+                ok = ok && __all_sync(0xffffffffu, mbar_wait(&t_full[buf], (kt >> 1) & 1, abort, 84));
+                if (!ok) continue;
+                tc_fence_after();
+                // the warp's 64 columns: both 32-column loads in flight, one
+                // wait, one online-softmax step
+                static_assert(C::N / C::SPLIT == 64, "two TMEM loads per epilogue warp");
+                const int c = part * 64;
+                const int j0 = C::N * k + c;            // block of column 0 of this range (uniform)
+                if (j0 < Dg) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32(tmem + lane_base + buf * C::N + c, v0);
+                    tmem_ld32(tmem + lane_base + buf * C::N + c + 32, v1);
+                    tmem_wait_ld();
+                    float x0[32], x1[32];
 #pragma unroll
                     for (int e = 0; e < 32; e++) {
-                        x[e] = __uint_as_float(v[e]) * sc2;
-                        mx = fmaxf(mx, x[e]);
+                        x0[e] = __uint_as_float(v0[e]);
+                        x1[e] = __uint_as_float(v1[e]);
                     }
-                } else {
+                    if (j0 + 64 > Dg) {
 #pragma unroll
-                    for (int e = 0; e < 32; e++) {
-                        x[e] = j0 + e < Dg ? __uint_as_float(v[e]) * sc2 : -INFINITY;
-                        mx = fmaxf(mx, x[e]);
+                        for (int e = 0; e < 32; e++) {
+                            if (j0 + e >= Dg) x0[e] = -INFINITY;   // 2^(-inf) = 0 below
+                            if (j0 + 32 + e >= Dg) x1[e] = -INFINITY;
+                        }
                     }
+                    // sc2 > 0, so the largest scaled logit is the largest raw
+                    // one scaled (rounding preserves the order); column j0 is
+                    // valid, so mn is finite
+                    const float mn = fmaxf(m_run, fmaxf(max32(x0), max32(x1)) * sc2);
+                    const uint64_t nm2 = f2_pack(-mn, -mn);
+                    uint64_t acc2 = f2_pack(0.f, 0.f);
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        float a0, a1, b0, b1;
+                        f2_unpack(f2_fma(f2_pack(x0[e], x0[e + 1]), s2, nm2), a0, a1);
+                        f2_unpack(f2_fma(f2_pack(x1[e], x1[e + 1]), s2, nm2), b0, b1);
+                        acc2 = f2_add(acc2, f2_pack(fast_exp2(a0), fast_exp2(a1)));
+                        acc2 = f2_add(acc2, f2_pack(fast_exp2(b0), fast_exp2(b1)));
+                    }
+                    float c0, c1;
+                    f2_unpack(acc2, c0, c1);
+                    s_run = s_run * fast_exp2(m_run - mn) + (c0 + c1);
+                    m_run = mn;
                 }
-                const float mn = fmaxf(m_run, mx);
-                float acc = 0.f;
-#pragma unroll
-                for (int e = 0; e < 32; e++) acc += fast_exp2(x[e] - mn);
-                s_run = s_run * fast_exp2(m_run - mn) + acc;
-                m_run = mn;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&t_empty[buf]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&t_empty[buf]);
-        }
-        // the two halves of each row meet (this exchange reuses no ring
-        // memory: a small array of its own)
-        __shared__ float xm[128], xs[128];
-        if (half == 1) xm[r] = m_run, xs[r] = s_run;
-        named_barrier_sync(1, 256);
-        if (half == 0 && k == ntiles) {
-            float m2 = xm[r], s2 = xs[r];
-            const float mn = fmaxf(m_run, m2);
-            const float sum = mn == -INFINITY ? 0.f : s_run * fast_exp2(m_run - mn) + s2 * fast_exp2(m2 - mn);
-            float *out = stats + (((long)bg * NR + i) * (64 * G) + mt * C::M + r) * 2;
-            out[0] = mn;
-            out[1] = sum;
+            // the column ranges of each row meet; the slot alternates with
+            // the unit, so the next unit's writes cannot overtake this read
+            const int xslot = un & 1;
+            if (part > 0) xm[xslot][part - 1][r] = m_run, xs[xslot][part - 1][r] = s_run;
+            named_barrier_sync(1, 32 * C::EPI);
+            if (part == 0 && ok) {
+                float mn = m_run;
+#pragma unroll
+                for (int q = 0; q < C::SPLIT - 1; q++) mn = fmaxf(mn, xm[xslot][q][r]);
+                float sum = 0.f;
+                if (mn != -INFINITY) {
+                    sum = s_run * fast_exp2(m_run - mn);
+#pragma unroll
+                    for (int q = 0; q < C::SPLIT - 1; q++) sum += xs[xslot][q][r] * fast_exp2(xm[xslot][q][r] - mn);
+                }
+                float *out = stats + (((long)bg * NR + i) * (64 * G) + mt * C::M + r) * 2;
+                out[0] = mn;
+                out[1] = sum;
+            }
+            un++;
         }
     }
 
     tc_fence_before();
     __syncthreads();
     if (abort_flag && threadIdx.x == 0) {
-        mbar_wait(&q_full, 0, nullptr, 85, 100000000ull);
+        // a wait gave up: let the copies and MMAs still in flight finish
+        // before the shared memory and TMEM go away (bounded, no abort
+        // short-cut)
+        for (int n = max(0, issued_q - 2); n < issued_q; n++)
+            mbar_wait(&q_full[n & 1], (n >> 1) & 1, nullptr, 85, 100000000ull);
         for (int k = max(0, issued_k - C::NS); k < issued_k; k++)
             mbar_wait(&k_full[k % C::NS], (k / C::NS) & 1, nullptr, 86, 100000000ull);
         if (issued_mma > 0) {

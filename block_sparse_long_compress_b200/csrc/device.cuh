@@ -480,6 +480,18 @@ __device__ __forceinline__ float max3f(float a, float b, float c)
     return d;
 }
 
+// Largest of 32 values: a tree of 3-input maxima (depth 4, 16 instructions).
+__device__ __forceinline__ float max32(const float (&x)[32])
+{
+    float t[11];
+#pragma unroll
+    for (int q = 0; q < 10; q++) t[q] = max3f(x[3 * q], x[3 * q + 1], x[3 * q + 2]);
+    t[10] = fmaxf(x[30], x[31]);
+    const float u0 = max3f(t[0], t[1], t[2]), u1 = max3f(t[3], t[4], t[5]);
+    const float u2 = max3f(t[6], t[7], t[8]), u3 = fmaxf(t[9], t[10]);
+    return fmaxf(max3f(u0, u1, u2), u3);
+}
+
 // ---- packed fp32 pairs (sm_100 f32x2 arithmetic)
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi)
 {

@@ -619,8 +619,12 @@ qsa_status launch_prefill_agg(const void *Q, const void *Kc, float *scores, floa
         if ((st = make_map_q(&mq1, Q, (uint64_t)B * Tq, Hq, 128, G, S::TOKM)) != QSA_OK) return st;
         if ((st = make_map_2d(&mk1, Kc, (uint64_t)B * Hkv * nblk, 128, 256)) != QSA_OK) return st;
         if ((st = set_smem(qsa::block_softmax_stats_kernel<G>, S::SMEM_BYTES)) != QSA_OK) return st;
-        qsa::block_softmax_stats_kernel<G><<<dim3(NR * S::NMT, B * Hkv), S::THREADS, S::SMEM_BYTES, s>>>(
-            mq1, mk1, stats, Tq, q_pos0, nblk, Hkv, sm_scale);
+        // persistent: one CTA per SM over the (sequence and group, query block, M tile) units
+        const long nunits = (long)NR * S::NMT * B * Hkv;
+        if (nunits >= (1L << 31)) return fail(QSA_ERR_UNSUPPORTED, "softmax statistics: too many rows");
+        const int grid = (int)std::min<long>(nunits, sm_count());
+        qsa::block_softmax_stats_kernel<G><<<grid, S::THREADS, S::SMEM_BYTES, s>>>(
+            mq1, mk1, stats, Tq, q_pos0, nblk, Hkv, sm_scale, NR, (int)nunits);
         if ((st = launched("block_softmax_stats_kernel")) != QSA_OK) return st;
     }
     using C = qsa::MaxScoreCfg<G>;
@@ -1219,9 +1223,10 @@ qsa_status qsa_merge_partials(const void *O_parts, const float *lse_parts, void 
         (reinterpret_cast<uintptr_t>(lse_parts) & 3) || (reinterpret_cast<uintptr_t>(lse) & 3))
         return fail(QSA_ERR_INVALID_ARG, "%s: misaligned pointer", name);
     if (rows == 0) return QSA_OK;
-    if ((rows + 7) / 8 >= (1L << 31)) return fail(QSA_ERR_UNSUPPORTED, "%s: too many rows", name);
+    const long per_cta = 8L * (256 / d);   // 8 warps, 256 / d rows per warp
+    if ((rows + per_cta - 1) / per_cta >= (1L << 31)) return fail(QSA_ERR_UNSUPPORTED, "%s: too many rows", name);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const unsigned grid = (unsigned)((rows + 7) / 8);
+    const unsigned grid = (unsigned)((rows + per_cta - 1) / per_cta);
     if (d == 128)
         qsa::merge_partials_kernel<128><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)O_parts, lse_parts,
                                                              (__nv_bfloat16 *)O, lse, nparts, rows);

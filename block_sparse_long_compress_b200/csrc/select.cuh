@@ -871,39 +871,68 @@ __global__ void __launch_bounds__(kSelThreads) merge_lists_kernel(
 // Partial attention outputs of the ranks (each over its own blocks, with its
 // natural-log normaliser lse_r; lse_r = -inf when it owns none of the row's
 // blocks) merged into the row's output: O = sum_r exp(lse_r - L) O_r with
-// L = log sum_r exp(lse_r), and lse = L.  One warp per (token, head) row,
-// lane owns D/32 consecutive columns; fp32 arithmetic.
-// grid ceil(rows / 8); 256 threads.
+// L = log sum_r exp(lse_r), and lse = L.  D/8 lanes per (token, head) row,
+// each owning 8 consecutive columns (one 16-byte load per rank; the first
+// 8 ranks' loads all in flight before any arithmetic); the ranks are added
+// in ascending order, in fp32.  grid ceil(rows / (8 * 256 / D)); 256 threads.
 template <int D>
 __global__ void __launch_bounds__(256) merge_partials_kernel(const __nv_bfloat16 *__restrict__ O_parts,
                                                              const float *__restrict__ lse_parts,
                                                              __nv_bfloat16 *__restrict__ O, float *__restrict__ lse,
                                                              int nparts, long rows)
 {
-    constexpr int CPL = D / 32;
-    const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
+    // a lane owns 8 columns (one 16-byte load per rank); D / 8 lanes per row
+    constexpr int LPR = D / 8, RPW = 32 / LPR;
+    const int lane = threadIdx.x & 31, cl = lane % LPR;
+    const long row = ((long)blockIdx.x * 8 + (threadIdx.x >> 5)) * RPW + lane / LPR;
     if (row >= rows) return;
-    float m = -INFINITY;
-    for (int r = 0; r < nparts; r++) m = fmaxf(m, __ldg(lse_parts + (long)r * rows + row));
-    float acc[CPL];
+    const uint4 *src = reinterpret_cast<const uint4 *>(O_parts + row * D) + cl;
+    const long rstride = rows * (D / 8);   // uint4 per rank
+    // the first (up to) 8 ranks' normalisers and columns all in flight at once
+    constexpr int RF = 8;
+    const int nf = min(nparts, RF);
+    float l[RF];
+    uint4 v[RF];
 #pragma unroll
-    for (int c = 0; c < CPL; c++) acc[c] = 0.f;
-    float wsum = 0.f;
-    if (m != -INFINITY) {
-        for (int r = 0; r < nparts; r++) {
-            const float w = __expf(__ldg(lse_parts + (long)r * rows + row) - m);
-            wsum += w;
-            const __nv_bfloat16 *src = O_parts + ((long)r * rows + row) * D + lane * CPL;
-#pragma unroll
-            for (int c = 0; c < CPL; c++) acc[c] += w * __bfloat162float(src[c]);
+    for (int r = 0; r < RF; r++)
+        if (r < nf) {
+            l[r] = __ldg(lse_parts + (long)r * rows + row);
+            v[r] = __ldg(src + r * rstride);
         }
+    float m = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < RF; r++)
+        if (r < nf) m = fmaxf(m, l[r]);
+    for (int r = RF; r < nparts; r++) m = fmaxf(m, __ldg(lse_parts + (long)r * rows + row));
+    float acc[8];
+#pragma unroll
+    for (int c = 0; c < 8; c++) acc[c] = 0.f;
+    float wsum = 0.f;
+    // ranks in ascending order
+    auto add = [&](float lr, const uint4 &vr) {
+        const float w = __expf(lr - m);
+        wsum += w;
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&vr);
+#pragma unroll
+        for (int c = 0; c < 4; c++) {
+            const float2 f = __bfloat1622float2(h[c]);
+            acc[2 * c] += w * f.x;
+            acc[2 * c + 1] += w * f.y;
+        }
+    };
+    if (m != -INFINITY) {
+#pragma unroll
+        for (int r = 0; r < RF; r++)
+            if (r < nf) add(l[r], v[r]);
+        for (int r = RF; r < nparts; r++) add(__ldg(lse_parts + (long)r * rows + row), __ldg(src + r * rstride));
     }
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-    __nv_bfloat16 *dst = O + row * D + lane * CPL;
+    uint4 out;
+    __nv_bfloat162 *oh = reinterpret_cast<__nv_bfloat162 *>(&out);
 #pragma unroll
-    for (int c = 0; c < CPL; c++) dst[c] = __float2bfloat16_rn(acc[c] * inv);
-    if (lse && lane == 0) lse[row] = m == -INFINITY ? -INFINITY : m + __logf(wsum);
+    for (int c = 0; c < 4; c++) oh[c] = __floats2bfloat162_rn(acc[2 * c] * inv, acc[2 * c + 1] * inv);
+    reinterpret_cast<uint4 *>(O + row * D)[cl] = out;
+    if (lse && cl == 0) lse[row] = m == -INFINITY ? -INFINITY : m + __logf(wsum);
 }
 
 // ------------------------------------------------ per-token, one launch
