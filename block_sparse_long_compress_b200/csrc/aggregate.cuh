@@ -22,19 +22,19 @@
 // tiles: warp 0 loads the query block once and streams summary tiles
 // through a 2-stage ring (TMA, 128-byte swizzle), warp 1 issues the MMAs
 // (M = 128, N = 256, K = 128: 8 MMAs per N tile) into one of two TMEM
-// accumulators, warps 2-5 reduce the other (for the softmax-sum warps 2-17:
-// four warps per TMEM lane quarter, each taking a quarter of the columns;
-// the quarters meet in shared memory once per candidate tile).  Scores go to a table
+// accumulators, warps 2-5 reduce the other.  Scores go to a table
 // [B][Hkv][NR][nblk_max] (candidates 1 .. D-1 of each row); the chunked
 // selection turns the table into indices.
 //
 // The softmax-sum aggregator (s_j = sum over the block's (head, token) rows
-// of each row's softmax over the blocks 0 .. D-1, at j) takes two passes:
+// of each row's softmax over the blocks 0 .. D-1, at j) takes two passes,
+// both persistent (one CTA per SM) with 16 epilogue warps (four per TMEM
+// lane quarter, 64 columns each, the ranges meeting in shared memory):
 // block_softmax_stats_kernel puts the (head, token) rows on M and the blocks
 // on N -- the shape of an attention score tile -- so that every thread keeps
-// its row's running (max, sum) in base 2; then block_max_scores_kernel in
-// its SOFTMAX mode forms, per candidate, the sum of 2^(z - max) / sum over
-// the rows, with the rows' statistics in shared memory.
+// its row's running (max, sum) in base 2; then block_softmax_scores_kernel
+// forms, per candidate, the sum of 2^(z - max) / sum over the rows, with the
+// rows' statistics in shared memory.
 #pragma once
 
 #include "device.cuh"
@@ -55,31 +55,22 @@ struct MaxScoreCfg {
     static constexpr int KSTAGE_BYTES = 2 * KHALF_BYTES;
     static constexpr int NS = 2;
     static constexpr int SMEM_BYTES = Q_BYTES + NS * KSTAGE_BYTES + 1024;
-    // producer, issuer and 4 epilogue warps (max), or 16 (softmax-sum: the
-    // exponentials' dependency chains need four warps per scheduler)
-    __host__ __device__ static constexpr int threads(bool softmax) { return 64 + 32 * (softmax ? 16 : 4); }
+    static constexpr int THREADS = 64 + 32 * 4;         // producer, issuer, 4 epilogue warps
     static constexpr int TMEM_COLS = 2 * N;             // two fp32 accumulators
     static_assert(N % G == 0 && 64 % TOKN == 0, "tile shape");
 };
 
-// SOFTMAX: the softmax-sum's second pass -- stats[(bg*NR + i)][64*G][2]
-// holds each (token, head) row's base-2 (max, sum) from the first pass.
-template <int G, bool SOFTMAX = false>
-__global__ void __launch_bounds__(MaxScoreCfg<G>::threads(SOFTMAX), 1) block_max_scores_kernel(
+template <int G>
+__global__ void __launch_bounds__(MaxScoreCfg<G>::THREADS, 1) block_max_scores_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
-    float *__restrict__ scores, int Tq, int q_pos0, int nblk_max, int Hkv, float sm_scale,
-    const float *__restrict__ stats = nullptr)
+    float *__restrict__ scores, int Tq, int q_pos0, int nblk_max, int Hkv, float sm_scale)
 {
     using C = MaxScoreCfg<G>;
-    constexpr int THREADS = C::threads(SOFTMAX);
-    constexpr int EPI = (THREADS - 64) / 32;            // epilogue warps
-    constexpr int SPLIT = EPI / 4;                      // column ranges per TMEM lane quarter (softmax: 4)
+    constexpr int EPI = 4;                              // epilogue warps
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t q_full, k_full[C::NS], k_empty[C::NS], t_full[2], t_empty[2];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag, issued_k, issued_mma;
-    __shared__ __align__(16) float nrstat[SOFTMAX ? 64 * G : 4];   // SOFTMAX: -(max + log2 sum) per (token, head) row
-    __shared__ float xch[SPLIT > 1 ? SPLIT - 1 : 1][128];   // the other column ranges' partials per candidate
 
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *q_smem = base;
@@ -114,12 +105,6 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::threads(SOFTMAX), 1) block_max
     if (warp == 1) {
         tmem_alloc(&tmem_base, C::TMEM_COLS);
         tmem_relinquish();
-    }
-    if constexpr (SOFTMAX) {
-        // 2^(z - max) / sum = 2^(z - (max + log2 sum))
-        const float *st = stats + ((long)bg * NR + i) * (64 * G) * 2;
-        for (int r = threadIdx.x; r < 64 * G; r += THREADS)
-            nrstat[r] = st[2 * r + 1] > 0.f ? -(st[2 * r] + __log2f(st[2 * r + 1])) : -INFINITY;
     }
     tc_fence_before();
     __syncthreads();
@@ -182,7 +167,6 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::threads(SOFTMAX), 1) block_max
         }
         if (lane == 0) issued_mma = w;
     } else {
-      if constexpr (!SOFTMAX) {
         // ------------------------------------------- epilogue (warps 2-5)
         const int quarter = warp & 3;                  // the TMEM lanes this warp may access
         const int m = 32 * quarter + lane;             // candidate within the tile
@@ -216,79 +200,6 @@ __global__ void __launch_bounds__(MaxScoreCfg<G>::threads(SOFTMAX), 1) block_max
                 best = -INFINITY;
             }
         }
-      } else {
-        // ------------------------------------------- epilogue (warps 2-9)
-        const int quarter = warp & 3;                  // the TMEM lanes this warp may access
-        const int part = (warp - 2) >> 2;              // the columns it reduces (one of SPLIT ranges)
-        const int m = 32 * quarter + lane;             // candidate within the tile
-        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-        const float sc2 = sm_scale * 1.4426950408889634f;
-        const uint64_t s2 = f2_pack(sc2, sc2);
-        uint64_t best2 = f2_pack(0.f, 0.f);            // two partial sums (even, odd columns)
-        for (int w = 0; w < nwork; w++) {
-            const int k = w / C::NT, nt = w % C::NT, buf = w & 1;
-            // warp-uniform: the TMEM loads below are collective.  A failed
-            // wait (an abort, after which every wait returns at once) skips
-            // the work but not the exchanges below: all epilogue warps must
-            // reach the same named barriers
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(&t_full[buf], (w >> 1) & 1, abort, 74));
-            if (ok) tc_fence_after();
-#pragma unroll 1
-            // the warp's 64 columns: both 32-column loads in flight, one wait
-            static_assert(C::N / SPLIT == 64, "two TMEM loads per epilogue warp");
-            auto chunk = [&](const uint32_t (&r)[32], int c) {
-#pragma unroll
-                for (int tt = 0; tt < 32 / G; tt++) {
-                    const int tl = nt * C::TOKN + c / G + tt;    // token of these G columns, in the block
-                    if (i * 64 + tl < Tq) {
-                        // the rows' shares of this block: 2^(z sc2 - (max + log2 sum)),
-                        // arguments two at a time, row statistics four at a time
-#pragma unroll
-                        for (int h = 0; h < G; h += 4) {
-                            const float4 ns = *reinterpret_cast<const float4 *>(&nrstat[tl * G + h]);
-                            const uint64_t a = f2_fma(f2_pack(__uint_as_float(r[tt * G + h]), __uint_as_float(r[tt * G + h + 1])),
-                                                      s2, f2_pack(ns.x, ns.y));
-                            const uint64_t b = f2_fma(f2_pack(__uint_as_float(r[tt * G + h + 2]), __uint_as_float(r[tt * G + h + 3])),
-                                                      s2, f2_pack(ns.z, ns.w));
-                            float a0, a1, b0, b1;
-                            f2_unpack(a, a0, a1);
-                            f2_unpack(b, b0, b1);
-                            best2 = f2_add(best2, f2_pack(fast_exp2(a0), fast_exp2(a1)));
-                            best2 = f2_add(best2, f2_pack(fast_exp2(b0), fast_exp2(b1)));
-                        }
-                    }
-                }
-            };
-            if (ok) {
-                const int c = part * 64;
-                uint32_t r0[32], r1[32];
-                tmem_ld32(tmem + lane_base + buf * C::N + c, r0);
-                tmem_ld32(tmem + lane_base + buf * C::N + c + 32, r1);
-                tmem_wait_ld();
-                chunk(r0, c);
-                chunk(r1, c + 32);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&t_empty[buf]);
-            if (nt == C::NT - 1) {
-                // the column ranges of each candidate meet
-                float e0, e1;
-                f2_unpack(best2, e0, e1);
-                float best = e0 + e1;
-                if (part > 0) xch[part - 1][m] = best;
-                named_barrier_sync(1, 32 * EPI);
-                const int j = 1 + C::M * k + m;
-                if (part == 0 && j < Dg) {
-#pragma unroll
-                    for (int q = 0; q < SPLIT - 1; q++) best += xch[q][m];
-                    scores[((long)bg * NR + i) * nblk_max + j] = best;
-                }
-                named_barrier_sync(1, 32 * EPI);
-                best2 = f2_pack(0.f, 0.f);
-            }
-        }
-      }
     }
 
     tc_fence_before();
@@ -587,6 +498,326 @@ __global__ void __launch_bounds__(SoftmaxStatsCfg<G>::THREADS, 1) block_softmax_
         if (issued_mma > 0) {
             const int w = issued_mma - 1;
             mbar_wait(&t_full[w & 1], (w >> 1) & 1, nullptr, 87, 100000000ull);
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// Second pass of the softmax-sum: the score of candidate j is the sum, over
+// the query block's (token, head) rows r, of 2^(z_rj - (max_r + log2
+// sum_r)) with the rows' statistics from the first pass.  Candidates on the
+// MMA's M side (128 per tile, one TMEM lane each) and the query rows on N
+// (256 per MMA: 256/G tokens x G heads), as in block_max_scores_kernel.
+// Persistent: one CTA per SM walks the (sequence and group, query block)
+// units, the query blocks with the most candidates first; a unit runs as
+// NT sub-units, one per 256-row N tile, each streaming the unit's candidate
+// tiles (the tiles are read from L2 once per sub-unit).  The sub-units'
+// query tiles sit in two slots, so the next sub-unit's queries load while
+// the current one is reduced; the K ring, the two TMEM accumulators and
+// their barriers count tiles across sub-units.  Each candidate's sub-unit
+// partial sums meet in the score table: the thread that owns the candidate
+// stores the first and adds the others in order (same thread, so no
+// atomics and a fixed order).  16 epilogue warps (four per TMEM lane
+// quarter, 64 columns each); the next unit's row statistics are fetched
+// while the current unit is reduced.
+template <int G>
+struct SoftmaxScoresCfg {
+    static constexpr int D = 128;
+    static constexpr int M = 128;                       // candidates per tile (TMEM lanes)
+    static constexpr int N = 256;                       // query rows (token, head) per MMA
+    static constexpr int TOKN = N / G;                  // tokens per sub-unit
+    static constexpr int NT = 64 / TOKN;                // sub-units per 64-token query block
+    static constexpr int QHALF_BYTES = N * 128;         // one 64-column half (32 KB)
+    static constexpr int QTILE_BYTES = 2 * QHALF_BYTES; // one slot
+    static constexpr int KHALF_BYTES = M * 128;         // 16 KB
+    static constexpr int KSTAGE_BYTES = 2 * KHALF_BYTES;
+    static constexpr int NS = 2;
+    static constexpr int SMEM_BYTES = 2 * QTILE_BYTES + NS * KSTAGE_BYTES + 1024;
+    static constexpr int SPLIT = 4;                     // epilogue warps per TMEM lane quarter
+    static constexpr int EPI = 4 * SPLIT;
+    static constexpr int THREADS = 64 + 32 * EPI;
+    static constexpr int TMEM_COLS = 2 * N;
+    static constexpr int ROWS = 64 * G;                 // (token, head) rows of a query block
+    static_assert(N / SPLIT == 64, "two TMEM loads per epilogue warp");
+    static_assert(ROWS <= 32 * EPI, "one statistics row per epilogue thread");
+};
+
+template <int G>
+__global__ void __launch_bounds__(SoftmaxScoresCfg<G>::THREADS, 1) block_softmax_scores_kernel(
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
+    float *__restrict__ scores, const float *__restrict__ stats, int Tq, int q_pos0, int nblk_max, int Hkv,
+    float sm_scale, int NR, int nunits)
+{
+    using C = SoftmaxScoresCfg<G>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ uint64_t q_full[2], q_empty[2], k_full[C::NS], k_empty[C::NS], t_full[2], t_empty[2];
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag, issued_q, issued_k, issued_mma;
+    __shared__ __align__(16) float nrstat[2][C::ROWS];  // -(max + log2 sum) per row (slot = unit parity)
+    __shared__ float xch[2][C::SPLIT - 1][128];         // the column ranges' partials (slot = tile parity)
+
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *q_smem = base;                             // two slots
+    uint8_t *k_smem = base + 2 * C::QTILE_BYTES;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // unit u -> (bg, i); returns the number of candidate tiles (0: no
+    // candidate, the unit is skipped by every role alike)
+    auto unit = [&](int u, int &bg, int &i, int &Dg) -> int {
+        bg = u / NR;
+        i = NR - 1 - (u - bg * NR);
+        Dg = (q_pos0 + min((i + 1) * 64, Tq) - 1) / 64;   // the row's diagonal block
+        return (max(Dg - 1, 0) + C::M - 1) / C::M;          // candidates 1 .. Dg-1
+    };
+
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        issued_q = 0;
+        issued_k = 0;
+        issued_mma = 0;
+#pragma unroll
+        for (int s = 0; s < 2; s++) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
+            mbar_init(&t_full[s], 1);
+            mbar_init(&t_empty[s], C::EPI);
+        }
+#pragma unroll
+        for (int s = 0; s < C::NS; s++) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+    volatile int *abort = &abort_flag;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            int kt = 0, sq = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+                int bg, i, Dg;
+                const int ntiles = unit(u, bg, i, Dg);
+                if (ntiles == 0) continue;
+                const int b = bg / Hkv, g = bg % Hkv;
+                for (int nt = 0; ok && nt < C::NT; nt++) {
+                    const int qs = sq & 1;
+                    if (sq >= 2 && !mbar_wait(&q_empty[qs], ((sq >> 1) - 1) & 1, abort, 90)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&q_full[qs], C::QTILE_BYTES);
+#pragma unroll
+                    for (int h = 0; h < 2; h++)
+                        tma_load_3d(q_smem + qs * C::QTILE_BYTES + h * C::QHALF_BYTES, &tmQ, &q_full[qs], h * 64,
+                                    g * G, b * Tq + i * 64 + nt * C::TOKN);
+                    sq++;
+                    for (int k = 0; k < ntiles; k++, kt++) {
+                        const int st = kt % C::NS;
+                        if (kt >= C::NS && !mbar_wait(&k_empty[st], ((kt / C::NS) - 1) & 1, abort, 91)) {
+                            ok = false;
+                            break;
+                        }
+                        fence_proxy_async_smem();
+                        mbar_arrive_expect_tx(&k_full[st], C::KSTAGE_BYTES);
+                        const int row = bg * nblk_max + 1 + C::M * k;   // host checks B*Hkv*nblk_max < 2^31
+#pragma unroll
+                        for (int h = 0; h < 2; h++)
+                            tma_load_2d(k_smem + st * C::KSTAGE_BYTES + h * C::KHALF_BYTES, &tmKc, &k_full[st], h * 64,
+                                        row);
+                    }
+                }
+            }
+            issued_q = sq;
+            issued_k = kt;
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------- MMA issuer (whole warp)
+        constexpr uint32_t idesc = umma_idesc_bf16(C::M, C::N, 0, 0);
+        const uint64_t kd = umma_smem_desc(smem_u32(k_smem), 16, 1024);
+        auto wait_all = [&](uint64_t *bar, uint32_t parity, int where) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, where));
+        };
+        int kt = 0, sq = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+            int bg, i, Dg;
+            const int ntiles = unit(u, bg, i, Dg);
+            if (ntiles == 0) continue;
+            for (int nt = 0; ok && nt < C::NT; nt++) {
+                const int qs = sq & 1;
+                if (!wait_all(&q_full[qs], (sq >> 1) & 1, 92)) {
+                    ok = false;
+                    break;
+                }
+                const uint64_t qd = umma_smem_desc(smem_u32(q_smem + qs * C::QTILE_BYTES), 16, 1024);
+                for (int k = 0; k < ntiles; k++) {
+                    const int st = kt % C::NS, buf = kt & 1;
+                    if (!wait_all(&k_full[st], (kt / C::NS) & 1, 93) ||
+                        (kt >= 2 && !wait_all(&t_empty[buf], ((kt >> 1) - 1) & 1, 94))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (elect_one()) {
+#pragma unroll
+                        for (int kk = 0; kk < C::D / 16; kk++) {
+                            const uint64_t aoff = (uint64_t)((st * C::KSTAGE_BYTES + (kk >> 2) * C::KHALF_BYTES + (kk & 3) * 32) >> 4);
+                            const uint64_t boff = (uint64_t)(((kk >> 2) * C::QHALF_BYTES + (kk & 3) * 32) >> 4);
+                            umma_ss(tmem + buf * C::N, kd + aoff, qd + boff, idesc, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&t_full[buf]);
+                        umma_commit(&k_empty[st]);
+                    }
+                    __syncwarp();
+                    kt++;
+                }
+                if (!ok) break;
+                // the slot's queries are free once the sub-unit's MMAs are done
+                if (elect_one()) umma_commit(&q_empty[qs]);
+                __syncwarp();
+                sq++;
+            }
+        }
+        if (lane == 0) issued_mma = kt;
+    } else {
+        // ------------------------------------------- epilogue (warps 2-17)
+        const int quarter = warp & 3;                  // the TMEM lanes this warp may access
+        const int part = (warp - 2) >> 2;              // its 64 of the tile's 256 columns
+        const int m = 32 * quarter + lane;             // candidate within the tile
+        const int e = threadIdx.x - 64;                // epilogue thread: statistics row e
+        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+        const float sc2 = sm_scale * 1.4426950408889634f;
+        const uint64_t s2 = f2_pack(sc2, sc2);
+        // 2^(z sc2 - max - log2 sum): the row's negated exponent offset
+        auto offset = [](float mx, float sum) { return sum > 0.f ? -(mx + __log2f(sum)) : -INFINITY; };
+        auto next_unit = [&](int u) {
+            int bg, i, Dg;
+            for (u += gridDim.x; u < nunits; u += gridDim.x)
+                if (unit(u, bg, i, Dg) > 0) break;
+            return u;
+        };
+        int u = next_unit(blockIdx.x - (int)gridDim.x);   // the first unit with candidates
+        if (u < nunits && e < C::ROWS) {
+            int bg, i, Dg;
+            unit(u, bg, i, Dg);
+            const float *st = stats + (((long)bg * NR + i) * C::ROWS + e) * 2;
+            nrstat[0][e] = offset(st[0], st[1]);
+        }
+        named_barrier_sync(1, 32 * C::EPI);
+        int kt = 0, un = 0;
+        bool ok = true;
+        for (; u < nunits; un++) {
+            int bg, i, Dg;
+            const int ntiles = unit(u, bg, i, Dg);
+            const int slot = un & 1;
+            // the next unit's statistics, in flight while this unit is reduced
+            const int u2 = next_unit(u);
+            float pm = 0.f, ps = 0.f;
+            if (u2 < nunits && e < C::ROWS) {
+                int bg2, i2, Dg2;
+                unit(u2, bg2, i2, Dg2);
+                const float *st = stats + (((long)bg2 * NR + i2) * C::ROWS + e) * 2;
+                pm = st[0];
+                ps = st[1];
+            }
+            float *srow = scores + ((long)bg * NR + i) * nblk_max;
+            for (int nt = 0; nt < C::NT; nt++) {
+                for (int k = 0; k < ntiles; k++, kt++) {
+                    const int buf = kt & 1;
+                    // a failed wait (an abort, after which every wait returns
+                    // at once) skips the work but not the exchange below: all
+                    // epilogue warps reach the same named barriers
+                    ok = ok && __all_sync(0xffffffffu, mbar_wait(&t_full[buf], (kt >> 1) & 1, abort, 95));
+                    uint64_t best2 = f2_pack(0.f, 0.f);   // two partial sums (even, odd columns)
+                    auto chunk = [&](const uint32_t (&r)[32], int c) {
+#pragma unroll
+                        for (int tt = 0; tt < 32 / G; tt++) {
+                            const int tl = nt * C::TOKN + c / G + tt;   // token of these G columns, in the block
+                            if (i * 64 + tl < Tq) {
+#pragma unroll
+                                for (int h = 0; h < G; h += 4) {
+                                    const float4 ns = *reinterpret_cast<const float4 *>(&nrstat[slot][tl * G + h]);
+                                    const uint64_t a = f2_fma(f2_pack(__uint_as_float(r[tt * G + h]),
+                                                                      __uint_as_float(r[tt * G + h + 1])),
+                                                              s2, f2_pack(ns.x, ns.y));
+                                    const uint64_t bb = f2_fma(f2_pack(__uint_as_float(r[tt * G + h + 2]),
+                                                                       __uint_as_float(r[tt * G + h + 3])),
+                                                               s2, f2_pack(ns.z, ns.w));
+                                    float a0, a1, b0, b1;
+                                    f2_unpack(a, a0, a1);
+                                    f2_unpack(bb, b0, b1);
+                                    best2 = f2_add(best2, f2_pack(fast_exp2(a0), fast_exp2(a1)));
+                                    best2 = f2_add(best2, f2_pack(fast_exp2(b0), fast_exp2(b1)));
+                                }
+                            }
+                        }
+                    };
+                    if (ok) {
+                        tc_fence_after();
+                        const int c = part * 64;
+                        uint32_t r0[32], r1[32];
+                        tmem_ld32(tmem + lane_base + buf * C::N + c, r0);
+                        tmem_ld32(tmem + lane_base + buf * C::N + c + 32, r1);
+                        tmem_wait_ld();
+                        chunk(r0, c);
+                        chunk(r1, c + 32);
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&t_empty[buf]);
+                    }
+                    // the column ranges of each candidate meet (slot = tile
+                    // parity: the writes for tile kt+2 follow the barrier of
+                    // tile kt+1, which the reader passes after this read)
+                    float e0, e1;
+                    f2_unpack(best2, e0, e1);
+                    float best = e0 + e1;
+                    const int xs = kt & 1;
+                    if (part > 0) xch[xs][part - 1][m] = best;
+                    named_barrier_sync(1, 32 * C::EPI);
+                    const int j = 1 + C::M * k + m;
+                    if (part == 0 && ok && j < Dg) {
+#pragma unroll
+                        for (int q = 0; q < C::SPLIT - 1; q++) best += xch[xs][q][m];
+                        // sub-unit 0 stores, the later ones add (same thread)
+                        srow[j] = nt == 0 ? best : srow[j] + best;
+                    }
+                }
+            }
+            // the next unit's statistics into the other slot (its last
+            // readers finished before this unit's first exchange barrier)
+            if (u2 < nunits && e < C::ROWS) nrstat[slot ^ 1][e] = offset(pm, ps);
+            named_barrier_sync(1, 32 * C::EPI);
+            u = u2;
+        }
+        if (!ok) *abort = 1;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (abort_flag && threadIdx.x == 0) {
+        // a wait gave up: let the copies and MMAs still in flight finish
+        // before the shared memory and TMEM go away (bounded, no abort
+        // short-cut)
+        for (int n = max(0, issued_q - 2); n < issued_q; n++)
+            mbar_wait(&q_full[n & 1], (n >> 1) & 1, nullptr, 96, 100000000ull);
+        for (int k = max(0, issued_k - C::NS); k < issued_k; k++)
+            mbar_wait(&k_full[k % C::NS], (k / C::NS) & 1, nullptr, 97, 100000000ull);
+        if (issued_mma > 0) {
+            const int w = issued_mma - 1;
+            mbar_wait(&t_full[w & 1], (w >> 1) & 1, nullptr, 98, 100000000ull);
         }
     }
     __syncthreads();
