@@ -596,7 +596,10 @@ def bench_prefill_agg(args, qsa, dev, peaks, wp, Q, K, flush, agg):
     achieved = flops / (ms * 1e-3) / 1e12
     return {"workload": wp.name, "aggregator": agg, "summaries": "bf16",
             "ms": ms, "rows": wp.B * wp.Hkv * NR, "timing": f"{R} calls back to back between two events",
-            "roofline": {"bound": "tensor", "kernel": "block_max_scores_kernel (+ selection, in the time)",
+            "roofline": {"bound": "tensor",
+                         "kernel": ("block_max_scores_kernel" if agg == "max" else
+                                    "block_softmax_stats_kernel + block_softmax_scores_kernel")
+                         + " (+ selection, in the time)",
                          "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["bf16_tflops"], "flops_per_launch": flops, "traffic": None}}
 
@@ -921,7 +924,7 @@ def main():
     ap.add_argument("--only-decode", action="store_true",
                     help="skip the prefill measurement (profiling the decode kernels)")
     ap.add_argument("--no-prefill-max", dest="prefill_max", action="store_false",
-                    help="skip the prefill selection with the max-over-tokens aggregator")
+                    help="skip the prefill selections with the max-over-tokens and softmax-sum aggregators")
     ap.add_argument("--no-softmax-sum", dest="softmax_sum", action="store_false",
                     help="skip the decode run with the softmax-sum selection aggregator")
     ap.add_argument("--decode-variants", default="fp32,bf16,fp8,paged,softmax_sum",
