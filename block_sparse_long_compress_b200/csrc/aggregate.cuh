@@ -18,13 +18,11 @@
 // every token, then the maximum over the block's valid tokens -- no
 // shuffles.
 //
-// One CTA per (query block, sequence, group), looping over its candidate
-// tiles: warp 0 loads the query block once and streams summary tiles
-// through a 2-stage ring (TMA, 128-byte swizzle), warp 1 issues the MMAs
-// (M = 128, N = 256, K = 128: 8 MMAs per N tile) into one of two TMEM
-// accumulators, warps 2-5 reduce the other.  Scores go to a table
-// [B][Hkv][NR][nblk_max] (candidates 1 .. D-1 of each row); the chunked
-// selection turns the table into indices.
+// Both aggregators' candidate scores come from one persistent kernel body
+// (block_scores_body: candidate tiles streamed through a TMA ring, tcgen05
+// MMAs into two TMEM accumulators, 16 epilogue warps reducing them); scores
+// go to a table [B][Hkv][NR][nblk_max] (candidates 1 .. D-1 of each row),
+// and the chunked selection turns the table into indices.
 //
 // The softmax-sum aggregator (s_j = sum over the block's (head, token) rows
 // of each row's softmax over the blocks 0 .. D-1, at j) takes two passes,
@@ -40,188 +38,6 @@
 #include "device.cuh"
 
 namespace qsa {
-
-template <int G>
-struct MaxScoreCfg {
-    static constexpr int D = 128;
-    static constexpr int M = 128;                       // candidates per tile (TMEM lanes)
-    static constexpr int N = 256;                       // query rows (token, head) per MMA
-    static constexpr int TOKN = N / G;                  // tokens per N tile
-    static constexpr int NT = 64 / TOKN;                // N tiles per 64-token query block
-    static constexpr int QHALF_BYTES = N * 128;         // one 64-column half of an N tile (32 KB)
-    static constexpr int QTILE_BYTES = 2 * QHALF_BYTES;
-    static constexpr int Q_BYTES = NT * QTILE_BYTES;    // 128 KB (G = 8) or 64 KB (G = 4)
-    static constexpr int KHALF_BYTES = M * 128;         // 16 KB
-    static constexpr int KSTAGE_BYTES = 2 * KHALF_BYTES;
-    static constexpr int NS = 2;
-    static constexpr int SMEM_BYTES = Q_BYTES + NS * KSTAGE_BYTES + 1024;
-    static constexpr int THREADS = 64 + 32 * 4;         // producer, issuer, 4 epilogue warps
-    static constexpr int TMEM_COLS = 2 * N;             // two fp32 accumulators
-    static_assert(N % G == 0 && 64 % TOKN == 0, "tile shape");
-};
-
-template <int G>
-__global__ void __launch_bounds__(MaxScoreCfg<G>::THREADS, 1) block_max_scores_kernel(
-    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
-    float *__restrict__ scores, int Tq, int q_pos0, int nblk_max, int Hkv, float sm_scale)
-{
-    using C = MaxScoreCfg<G>;
-    constexpr int EPI = 4;                              // epilogue warps
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    __shared__ uint64_t q_full, k_full[C::NS], k_empty[C::NS], t_full[2], t_empty[2];
-    __shared__ uint32_t tmem_base;
-    __shared__ int abort_flag, issued_k, issued_mma;
-
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *q_smem = base;
-    uint8_t *k_smem = base + C::Q_BYTES;
-    const int i = blockIdx.x, bg = blockIdx.y, NR = gridDim.x;
-    const int b = bg / Hkv, g = bg % Hkv;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t_last = min((i + 1) * 64, Tq) - 1;
-    const int Dg = (q_pos0 + t_last) / 64;              // the row's diagonal block
-    const int ncand = max(Dg - 1, 0);                   // candidates 1 .. Dg-1
-    const int ntiles = (ncand + C::M - 1) / C::M;
-    if (ntiles == 0) return;                            // uniform: no barrier or TMEM yet
-    const int nwork = ntiles * C::NT;                   // (candidate tile, N tile) pairs
-
-    if (threadIdx.x == 0) {
-        abort_flag = 0;
-        issued_k = 0;
-        issued_mma = 0;
-        mbar_init(&q_full, 1);
-#pragma unroll
-        for (int s = 0; s < C::NS; s++) {
-            mbar_init(&k_full[s], 1);
-            mbar_init(&k_empty[s], 1);
-        }
-#pragma unroll
-        for (int s = 0; s < 2; s++) {
-            mbar_init(&t_full[s], 1);
-            mbar_init(&t_empty[s], EPI);                // one arrival per epilogue warp
-        }
-        fence_barrier_init();
-    }
-    if (warp == 1) {
-        tmem_alloc(&tmem_base, C::TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = tmem_base;
-    volatile int *abort = &abort_flag;
-
-    if (warp == 0) {
-        // ------------------------------------------------------ producer
-        if (lane == 0) {
-            // the query block's rows (token, head) of the group: N tile nt
-            // holds tokens nt*TOKN .. +TOKN, each 64-column half one 3-D box
-            mbar_arrive_expect_tx(&q_full, C::Q_BYTES);
-#pragma unroll
-            for (int nt = 0; nt < C::NT; nt++)
-#pragma unroll
-                for (int h = 0; h < 2; h++)
-                    tma_load_3d(q_smem + nt * C::QTILE_BYTES + h * C::QHALF_BYTES, &tmQ, &q_full, h * 64, g * G,
-                                b * Tq + i * 64 + nt * C::TOKN);
-            int k = 0;
-            for (; k < ntiles; k++) {
-                const int st = k % C::NS;
-                if (k >= C::NS && !mbar_wait(&k_empty[st], ((k / C::NS) - 1) & 1, abort, 70)) break;
-                fence_proxy_async_smem();
-                mbar_arrive_expect_tx(&k_full[st], C::KSTAGE_BYTES);
-                const int row = bg * nblk_max + 1 + C::M * k;   // host checks B*Hkv*nblk_max < 2^31
-#pragma unroll
-                for (int h = 0; h < 2; h++)
-                    tma_load_2d(k_smem + st * C::KSTAGE_BYTES + h * C::KHALF_BYTES, &tmKc, &k_full[st], h * 64, row);
-            }
-            issued_k = k;
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------- MMA issuer (whole warp)
-        constexpr uint32_t idesc = umma_idesc_bf16(C::M, C::N, 0, 0);
-        const uint64_t qd = umma_smem_desc(smem_u32(q_smem), 16, 1024);
-        const uint64_t kd = umma_smem_desc(smem_u32(k_smem), 16, 1024);
-        auto wait_all = [&](uint64_t *bar, uint32_t parity, int where) -> bool {
-            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, where));
-        };
-        int w = 0;
-        if (wait_all(&q_full, 0, 71)) {
-            for (; w < nwork; w++) {
-                const int k = w / C::NT, nt = w % C::NT, st = k % C::NS, buf = w & 1;
-                if (nt == 0 && !wait_all(&k_full[st], (k / C::NS) & 1, 72)) break;
-                if (w >= 2 && !wait_all(&t_empty[buf], ((w >> 1) - 1) & 1, 73)) break;
-                tc_fence_after();
-                if (elect_one()) {
-#pragma unroll
-                    for (int kk = 0; kk < C::D / 16; kk++) {
-                        const uint64_t aoff = (uint64_t)((st * C::KSTAGE_BYTES + (kk >> 2) * C::KHALF_BYTES + (kk & 3) * 32) >> 4);
-                        const uint64_t boff = (uint64_t)((nt * C::QTILE_BYTES + (kk >> 2) * C::QHALF_BYTES + (kk & 3) * 32) >> 4);
-                        umma_ss(tmem + buf * C::N, kd + aoff, qd + boff, idesc, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&t_full[buf]);
-                    if (nt == C::NT - 1) umma_commit(&k_empty[st]);
-                }
-                __syncwarp();
-            }
-        }
-        if (lane == 0) issued_mma = w;
-    } else {
-        // ------------------------------------------- epilogue (warps 2-5)
-        const int quarter = warp & 3;                  // the TMEM lanes this warp may access
-        const int m = 32 * quarter + lane;             // candidate within the tile
-        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-        float best = -INFINITY;
-        for (int w = 0; w < nwork; w++) {
-            const int k = w / C::NT, nt = w % C::NT, buf = w & 1;
-            // warp-uniform: the TMEM loads below are collective
-            if (!__all_sync(0xffffffffu, mbar_wait(&t_full[buf], (w >> 1) & 1, abort, 74))) break;
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < C::N; c += 32) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_base + buf * C::N + c, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int tt = 0; tt < 32 / G; tt++) {
-                    const int t = i * 64 + nt * C::TOKN + c / G + tt;   // token of these G columns
-                    float sum = 0.f;
-#pragma unroll
-                    for (int h = 0; h < G; h++) sum += __uint_as_float(r[tt * G + h]);
-                    if (t < Tq) best = fmaxf(best, sum);
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&t_empty[buf]);
-            if (nt == C::NT - 1) {
-                const int j = 1 + C::M * k + m;
-                if (j < Dg) scores[((long)bg * NR + i) * nblk_max + j] = best * (1.0f / (float)G) * sm_scale;
-                best = -INFINITY;
-            }
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (abort_flag && threadIdx.x == 0) {
-        // a wait gave up: let the copies and MMAs still in flight finish
-        // before the shared memory and TMEM go away (bounded, no abort
-        // short-cut)
-        mbar_wait(&q_full, 0, nullptr, 75, 100000000ull);
-        for (int k = max(0, issued_k - C::NS); k < issued_k; k++)
-            mbar_wait(&k_full[k % C::NS], (k / C::NS) & 1, nullptr, 76, 100000000ull);
-        if (issued_mma > 0) {
-            const int w = issued_mma - 1;
-            mbar_wait(&t_full[w & 1], (w >> 1) & 1, nullptr, 77, 100000000ull);
-        }
-    }
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, C::TMEM_COLS);
-    }
-}
 
 // First pass of the softmax-sum: per (token, head) row of the query block,
 // the base-2 (max, sum of 2^(z - max)) of z = sm_scale log2(e) <q, Kc_j>
@@ -507,11 +323,16 @@ __global__ void __launch_bounds__(SoftmaxStatsCfg<G>::THREADS, 1) block_softmax_
     }
 }
 
-// Second pass of the softmax-sum: the score of candidate j is the sum, over
-// the query block's (token, head) rows r, of 2^(z_rj - (max_r + log2
-// sum_r)) with the rows' statistics from the first pass.  Candidates on the
-// MMA's M side (128 per tile, one TMEM lane each) and the query rows on N
-// (256 per MMA: 256/G tokens x G heads), as in block_max_scores_kernel.
+// Candidate scores from the per-(head, token) logits z_rj = <q_r, Kc_j> of
+// the query block's rows r = (token, head):
+//   max mode      s_j = sm_scale * max over the block's valid tokens of the
+//                 mean over the group's heads of z_rj;
+//   SOFTMAX mode  s_j = sum over the rows of 2^(z_rj sm_scale log2(e) -
+//                 (max_r + log2 sum_r)), the rows' statistics from
+//                 block_softmax_stats_kernel (the softmax-sum's second pass).
+// Candidates on the MMA's M side (128 per tile, one TMEM lane each) and the
+// query rows on N (256 per MMA: 256/G tokens x G heads), so each epilogue
+// thread reduces its own candidate's columns.
 // Persistent: one CTA per SM walks the (sequence and group, query block)
 // units, the query blocks with the most candidates first; a unit runs as
 // NT sub-units, one per 256-row N tile, each streaming the unit's candidate
@@ -519,13 +340,14 @@ __global__ void __launch_bounds__(SoftmaxStatsCfg<G>::THREADS, 1) block_softmax_
 // query tiles sit in two slots, so the next sub-unit's queries load while
 // the current one is reduced; the K ring, the two TMEM accumulators and
 // their barriers count tiles across sub-units.  Each candidate's sub-unit
-// partial sums meet in the score table: the thread that owns the candidate
-// stores the first and adds the others in order (same thread, so no
-// atomics and a fixed order).  16 epilogue warps (four per TMEM lane
-// quarter, 64 columns each); the next unit's row statistics are fetched
-// while the current unit is reduced.
+// partials meet in the score table: the thread that owns the candidate
+// stores the first and folds in the others in order (same thread, so no
+// atomics and a fixed order; the max mode's maximum is order-free anyway).
+// 16 epilogue warps (four per TMEM lane quarter, 64 columns each); in the
+// SOFTMAX mode the next unit's row statistics are fetched while the
+// current unit is reduced.
 template <int G>
-struct SoftmaxScoresCfg {
+struct TokenScoresCfg {
     static constexpr int D = 128;
     static constexpr int M = 128;                       // candidates per tile (TMEM lanes)
     static constexpr int N = 256;                       // query rows (token, head) per MMA
@@ -546,18 +368,18 @@ struct SoftmaxScoresCfg {
     static_assert(ROWS <= 32 * EPI, "one statistics row per epilogue thread");
 };
 
-template <int G>
-__global__ void __launch_bounds__(SoftmaxScoresCfg<G>::THREADS, 1) block_softmax_scores_kernel(
-    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
-    float *__restrict__ scores, const float *__restrict__ stats, int Tq, int q_pos0, int nblk_max, int Hkv,
-    float sm_scale, int NR, int nunits)
+template <int G, bool SOFTMAX>
+__device__ __forceinline__ void block_scores_body(const CUtensorMap &tmQ, const CUtensorMap &tmKc,
+                                                  float *__restrict__ scores, const float *__restrict__ stats,
+                                                  int Tq, int q_pos0, int nblk_max, int Hkv, float sm_scale,
+                                                  int NR, int nunits)
 {
-    using C = SoftmaxScoresCfg<G>;
+    using C = TokenScoresCfg<G>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t q_full[2], q_empty[2], k_full[C::NS], k_empty[C::NS], t_full[2], t_empty[2];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag, issued_q, issued_k, issued_mma;
-    __shared__ __align__(16) float nrstat[2][C::ROWS];  // -(max + log2 sum) per row (slot = unit parity)
+    __shared__ __align__(16) float nrstat[SOFTMAX ? 2 : 1][SOFTMAX ? C::ROWS : 4];   // SOFTMAX: -(max + log2 sum) per row (slot = unit parity)
     __shared__ float xch[2][C::SPLIT - 1][128];         // the column ranges' partials (slot = tile parity)
 
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -710,7 +532,7 @@ __global__ void __launch_bounds__(SoftmaxScoresCfg<G>::THREADS, 1) block_softmax
             return u;
         };
         int u = next_unit(blockIdx.x - (int)gridDim.x);   // the first unit with candidates
-        if (u < nunits && e < C::ROWS) {
+        if (SOFTMAX && u < nunits && e < C::ROWS) {
             int bg, i, Dg;
             unit(u, bg, i, Dg);
             const float *st = stats + (((long)bg * NR + i) * C::ROWS + e) * 2;
@@ -726,7 +548,7 @@ __global__ void __launch_bounds__(SoftmaxScoresCfg<G>::THREADS, 1) block_softmax
             // the next unit's statistics, in flight while this unit is reduced
             const int u2 = next_unit(u);
             float pm = 0.f, ps = 0.f;
-            if (u2 < nunits && e < C::ROWS) {
+            if (SOFTMAX && u2 < nunits && e < C::ROWS) {
                 int bg2, i2, Dg2;
                 unit(u2, bg2, i2, Dg2);
                 const float *st = stats + (((long)bg2 * NR + i2) * C::ROWS + e) * 2;
@@ -741,12 +563,18 @@ __global__ void __launch_bounds__(SoftmaxScoresCfg<G>::THREADS, 1) block_softmax
                     // at once) skips the work but not the exchange below: all
                     // epilogue warps reach the same named barriers
                     ok = ok && __all_sync(0xffffffffu, mbar_wait(&t_full[buf], (kt >> 1) & 1, abort, 95));
-                    uint64_t best2 = f2_pack(0.f, 0.f);   // two partial sums (even, odd columns)
+                    uint64_t best2 = f2_pack(0.f, 0.f);   // SOFTMAX: two partial sums (even, odd columns)
+                    float bmax = -INFINITY;                 // max mode: the best token so far
                     auto chunk = [&](const uint32_t (&r)[32], int c) {
 #pragma unroll
                         for (int tt = 0; tt < 32 / G; tt++) {
                             const int tl = nt * C::TOKN + c / G + tt;   // token of these G columns, in the block
-                            if (i * 64 + tl < Tq) {
+                            if constexpr (!SOFTMAX) {
+                                float sum = 0.f;
+#pragma unroll
+                                for (int h = 0; h < G; h++) sum += __uint_as_float(r[tt * G + h]);
+                                if (i * 64 + tl < Tq) bmax = fmaxf(bmax, sum);
+                            } else if (i * 64 + tl < Tq) {
 #pragma unroll
                                 for (int h = 0; h < G; h += 4) {
                                     const float4 ns = *reinterpret_cast<const float4 *>(&nrstat[slot][tl * G + h]);
@@ -781,24 +609,36 @@ __global__ void __launch_bounds__(SoftmaxScoresCfg<G>::THREADS, 1) block_softmax
                     // the column ranges of each candidate meet (slot = tile
                     // parity: the writes for tile kt+2 follow the barrier of
                     // tile kt+1, which the reader passes after this read)
-                    float e0, e1;
-                    f2_unpack(best2, e0, e1);
-                    float best = e0 + e1;
+                    float best = bmax;
+                    if constexpr (SOFTMAX) {
+                        float e0, e1;
+                        f2_unpack(best2, e0, e1);
+                        best = e0 + e1;
+                    }
                     const int xs = kt & 1;
                     if (part > 0) xch[xs][part - 1][m] = best;
                     named_barrier_sync(1, 32 * C::EPI);
                     const int j = 1 + C::M * k + m;
                     if (part == 0 && ok && j < Dg) {
+                        if constexpr (SOFTMAX) {
 #pragma unroll
-                        for (int q = 0; q < C::SPLIT - 1; q++) best += xch[xs][q][m];
-                        // sub-unit 0 stores, the later ones add (same thread)
-                        srow[j] = nt == 0 ? best : srow[j] + best;
+                            for (int q = 0; q < C::SPLIT - 1; q++) best += xch[xs][q][m];
+                            // sub-unit 0 stores, the later ones add (same thread)
+                            srow[j] = nt == 0 ? best : srow[j] + best;
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < C::SPLIT - 1; q++) best = fmaxf(best, xch[xs][q][m]);
+                            // the head mean and the scale are monotone, so each
+                            // sub-unit's scaled maximum folds in exactly
+                            best = best * (1.0f / (float)G) * sm_scale;
+                            srow[j] = nt == 0 ? best : fmaxf(srow[j], best);
+                        }
                     }
                 }
             }
             // the next unit's statistics into the other slot (its last
             // readers finished before this unit's first exchange barrier)
-            if (u2 < nunits && e < C::ROWS) nrstat[slot ^ 1][e] = offset(pm, ps);
+            if (SOFTMAX && u2 < nunits && e < C::ROWS) nrstat[slot ^ 1][e] = offset(pm, ps);
             named_barrier_sync(1, 32 * C::EPI);
             u = u2;
         }
@@ -825,6 +665,22 @@ __global__ void __launch_bounds__(SoftmaxScoresCfg<G>::THREADS, 1) block_softmax
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
+}
+
+template <int G>
+__global__ void __launch_bounds__(TokenScoresCfg<G>::THREADS, 1) block_max_scores_kernel(
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc, float *__restrict__ scores,
+    int Tq, int q_pos0, int nblk_max, int Hkv, float sm_scale, int NR, int nunits)
+{
+    block_scores_body<G, false>(tmQ, tmKc, scores, nullptr, Tq, q_pos0, nblk_max, Hkv, sm_scale, NR, nunits);
+}
+
+template <int G>
+__global__ void __launch_bounds__(TokenScoresCfg<G>::THREADS, 1) block_softmax_scores_kernel(
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc, float *__restrict__ scores,
+    const float *__restrict__ stats, int Tq, int q_pos0, int nblk_max, int Hkv, float sm_scale, int NR, int nunits)
+{
+    block_scores_body<G, true>(tmQ, tmKc, scores, stats, Tq, q_pos0, nblk_max, Hkv, sm_scale, NR, nunits);
 }
 
 }  // namespace qsa

@@ -627,22 +627,20 @@ qsa_status launch_prefill_agg(const void *Q, const void *Kc, float *scores, floa
             mq1, mk1, stats, Tq, q_pos0, nblk, Hkv, sm_scale, NR, (int)nunits);
         if ((st = launched("block_softmax_stats_kernel")) != QSA_OK) return st;
     }
-    using C = qsa::MaxScoreCfg<G>;
+    using C = qsa::TokenScoresCfg<G>;
     if ((st = make_map_q(&mq, Q, (uint64_t)B * Tq, Hq, 128, G, C::TOKN)) != QSA_OK) return st;
+    // persistent: one CTA per SM over the (sequence and group, query block) units
+    const long nunits = (long)NR * B * Hkv;
+    const int grid = (int)std::min<long>(nunits, sm_count());
     if (aggregator == QSA_AGG_SOFTMAX_SUM) {
-        using S = qsa::SoftmaxScoresCfg<G>;
-        static_assert(S::TOKN == C::TOKN, "the query map's box serves both kernels");
-        if ((st = set_smem(qsa::block_softmax_scores_kernel<G>, S::SMEM_BYTES)) != QSA_OK) return st;
-        // persistent: one CTA per SM over the (sequence and group, query block) units
-        const long nunits = (long)NR * B * Hkv;
-        const int grid = (int)std::min<long>(nunits, sm_count());
-        qsa::block_softmax_scores_kernel<G><<<grid, S::THREADS, S::SMEM_BYTES, s>>>(
+        if ((st = set_smem(qsa::block_softmax_scores_kernel<G>, C::SMEM_BYTES)) != QSA_OK) return st;
+        qsa::block_softmax_scores_kernel<G><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(
             mq, mk, scores, stats, Tq, q_pos0, nblk, Hkv, sm_scale, NR, (int)nunits);
         return launched("block_softmax_scores_kernel");
     }
     if ((st = set_smem(qsa::block_max_scores_kernel<G>, C::SMEM_BYTES)) != QSA_OK) return st;
-    qsa::block_max_scores_kernel<G><<<dim3(NR, B * Hkv), C::THREADS, C::SMEM_BYTES, s>>>(
-        mq, mk, scores, Tq, q_pos0, nblk, Hkv, sm_scale);
+    qsa::block_max_scores_kernel<G><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, scores, Tq, q_pos0, nblk, Hkv,
+                                                                           sm_scale, NR, (int)nunits);
     return launched("block_max_scores_kernel");
 }
 }  // namespace
