@@ -77,6 +77,7 @@ def _load():
         "qsa_get_device_status": (I, [P, ctypes.POINTER(I)]),
         "qsa_selftest_wait_timeout": (I, [ctypes.c_uint64, P]),
         "qsa_selftest_exp2": (I, [P, P, I, P]),
+        "qsa_selftest_exp2_weight": (I, [P, P, I, P]),
         "qsa_status_string": (ctypes.c_char_p, [I]),
         "qsa_last_error": (ctypes.c_char_p, []),
         "qsa_launch_count": (ctypes.c_ulonglong, []),

@@ -39,6 +39,12 @@
 
 namespace qsa {
 
+// The softmax-sum passes evaluate one exponential pair in kPolyEvery with
+// the degree-5 polynomial on the FMA pipe (exp2_poly5_x2) and the rest on
+// MUFU, whose issue queue bounds both passes.
+constexpr int kPolyEvery = 4;
+__host__ __device__ constexpr bool poly_pair(int q) { return q % kPolyEvery == kPolyEvery - 1; }
+
 // First pass of the softmax-sum: per (token, head) row of the query block,
 // the base-2 (max, sum of 2^(z - max)) of z = sm_scale log2(e) <q, Kc_j>
 // over the blocks j in 0 .. D-1.  A work unit is (sequence and group, query
@@ -263,11 +269,9 @@ __global__ void __launch_bounds__(SoftmaxStatsCfg<G>::THREADS, 1) block_softmax_
                     uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
-                        float a0, a1, b0, b1;
-                        f2_unpack(f2_fma(f2_pack(x0[e], x0[e + 1]), s2, nm2), a0, a1);
-                        f2_unpack(f2_fma(f2_pack(x1[e], x1[e + 1]), s2, nm2), b0, b1);
-                        acc2 = f2_add(acc2, f2_pack(fast_exp2(a0), fast_exp2(a1)));
-                        acc2 = f2_add(acc2, f2_pack(fast_exp2(b0), fast_exp2(b1)));
+                        // pairs q = e (x0) and e + 1 (x1); one in kPolyEvery on the FMA pipe
+                        acc2 = f2_add(acc2, exp2_pair(poly_pair(e), f2_fma(f2_pack(x0[e], x0[e + 1]), s2, nm2)));
+                        acc2 = f2_add(acc2, exp2_pair(poly_pair(e + 1), f2_fma(f2_pack(x1[e], x1[e + 1]), s2, nm2)));
                     }
                     float c0, c1;
                     f2_unpack(acc2, c0, c1);
@@ -584,11 +588,9 @@ __device__ __forceinline__ void block_scores_body(const CUtensorMap &tmQ, const 
                                     const uint64_t bb = f2_fma(f2_pack(__uint_as_float(r[tt * G + h + 2]),
                                                                        __uint_as_float(r[tt * G + h + 3])),
                                                                s2, f2_pack(ns.z, ns.w));
-                                    float a0, a1, b0, b1;
-                                    f2_unpack(a, a0, a1);
-                                    f2_unpack(bb, b0, b1);
-                                    best2 = f2_add(best2, f2_pack(fast_exp2(a0), fast_exp2(a1)));
-                                    best2 = f2_add(best2, f2_pack(fast_exp2(b0), fast_exp2(b1)));
+                                    // pairs q and q + 1 of the chunk; one in kPolyEvery on the FMA pipe
+                                    best2 = f2_add(best2, exp2_pair(poly_pair((tt * G + h) / 2), a));
+                                    best2 = f2_add(best2, exp2_pair(poly_pair((tt * G + h) / 2 + 1), bb));
                                 }
                             }
                         }

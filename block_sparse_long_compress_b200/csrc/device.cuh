@@ -554,4 +554,43 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2)
                    __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(p1)));
 }
 
+// 2^x for a pair of fp32 values with x <= 0 (a softmax weight), on the FMA
+// pipe, accurate enough to stand in for ex2.approx in sums that decide a
+// selection: the same argument reduction as exp2_poly_x2 (x = n + f, n =
+// round(x), f in [-1/2, 1/2]), then 2^f from a degree-5 polynomial with
+// coefficients fitted for this library (Lawson-weighted least squares on
+// Chebyshev nodes towards minimax relative error: 7.5e-8 in exact
+// arithmetic, 2.1e-7 with fp32 Horner steps, against 2^-22 for ex2.approx);
+// x is clamped at -126 (a weight below 2^-126 is negligible in the sum).
+__device__ __forceinline__ uint64_t exp2_poly5_x2(uint64_t x2)
+{
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    const uint64_t x = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+    const uint64_t round_c = f2_pack(12582912.f, 12582912.f);
+    const uint64_t t = f2_add(x, round_c);
+    const uint64_t f = f2_sub(x, f2_sub(t, round_c));
+    uint64_t p = f2_fma(f2_pack(1.327647152e-03f, 1.327647152e-03f), f,
+                        f2_pack(9.6755413307e-03f, 9.6755413307e-03f));
+    p = f2_fma(p, f, f2_pack(5.550713275e-02f, 5.550713275e-02f));
+    p = f2_fma(p, f, f2_pack(2.4022119724e-01f, 2.4022119724e-01f));
+    p = f2_fma(p, f, f2_pack(6.9314696706e-01f, 6.9314696706e-01f));
+    p = f2_fma(p, f, f2_pack(1.0000000717f, 1.0000000717f));
+    float t0, t1, p0, p1;
+    f2_unpack(t, t0, t1);
+    f2_unpack(p, p0, p1);
+    return f2_pack(__uint_as_float(__float_as_uint(t0) * 8388608u + __float_as_uint(p0)),
+                   __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(p1)));
+}
+
+// 2^x of a pair: on the FMA pipe (exp2_poly5_x2) when poly, else on MUFU
+// (in unrolled loops the choice folds away at compile time).
+__device__ __forceinline__ uint64_t exp2_pair(bool poly, uint64_t x2)
+{
+    if (poly) return exp2_poly5_x2(x2);
+    float a, b;
+    f2_unpack(x2, a, b);
+    return f2_pack(fast_exp2(a), fast_exp2(b));
+}
+
 }  // namespace qsa

@@ -383,17 +383,21 @@ qsa_status launch_select_token(const void *Q, const KcT *Kc, int32_t *idx, int B
                                                    s, seq_lens);
 }
 
+template <bool WEIGHT>
 __global__ void selftest_exp2_kernel(const float *__restrict__ x, float *__restrict__ y, int n)
 {
     const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    auto e2 = [](float a, float b) {
+        return WEIGHT ? qsa::exp2_poly5_x2(qsa::f2_pack(a, b)) : qsa::exp2_poly_x2(qsa::f2_pack(a, b));
+    };
     if (i + 1 < n) {
         float a, b;
-        qsa::f2_unpack(qsa::exp2_poly_x2(qsa::f2_pack(x[i], x[i + 1])), a, b);
+        qsa::f2_unpack(e2(x[i], x[i + 1]), a, b);
         y[i] = a;
         y[i + 1] = b;
     } else if (i < n) {
         float a, b;
-        qsa::f2_unpack(qsa::exp2_poly_x2(qsa::f2_pack(x[i], 0.f)), a, b);
+        qsa::f2_unpack(e2(x[i], 0.f), a, b);
         y[i] = a;
     }
 }
@@ -1266,7 +1270,16 @@ qsa_status qsa_selftest_exp2(const float *x, float *y, int n, qsa_stream_t strea
     if (!x || !y || n < 0) return fail(QSA_ERR_INVALID_ARG, "qsa_selftest_exp2: bad arguments");
     if (n == 0) return QSA_OK;
     const int pairs = (n + 1) / 2;
-    selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+    selftest_exp2_kernel<false><<<(pairs + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+    return launched("selftest_exp2_kernel");
+}
+
+qsa_status qsa_selftest_exp2_weight(const float *x, float *y, int n, qsa_stream_t stream)
+{
+    if (!x || !y || n < 0) return fail(QSA_ERR_INVALID_ARG, "qsa_selftest_exp2_weight: bad arguments");
+    if (n == 0) return QSA_OK;
+    const int pairs = (n + 1) / 2;
+    selftest_exp2_kernel<true><<<(pairs + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
     return launched("selftest_exp2_kernel");
 }
 

@@ -467,6 +467,11 @@ QSA_API qsa_status qsa_selftest_wait_timeout(uint64_t timeout_ns, qsa_stream_t s
  * compare it with the CUDA exp2 on the same device. */
 QSA_API qsa_status qsa_selftest_exp2(const float *x, float *y, int n, qsa_stream_t stream);
 
+/* Test hook for the FMA-pipe exponential used by the softmax-sum selection
+ * passes: y[i] = 2^x[i] for n device floats with x <= 0 (the same reduction
+ * plus a degree-5 polynomial; inputs below -126 are clamped to -126). */
+QSA_API qsa_status qsa_selftest_exp2_weight(const float *x, float *y, int n, qsa_stream_t stream);
+
 /* Human-readable name of a status code (static storage). */
 QSA_API const char *qsa_status_string(qsa_status s);
 

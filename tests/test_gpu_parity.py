@@ -82,6 +82,30 @@ def test_fma_pipe_exp2_against_cuda_exp2(qsa):
     assert (yl >= 0).all() and (yl <= 2.0 ** -125).all()
 
 
+def test_fma_pipe_softmax_weight_exp2_against_cuda_exp2(qsa):
+    """The degree-5 polynomial 2^x the softmax-sum selection passes run on
+    the FMA pipe for a share of their weights, against CUDA's exp2 on the
+    same device: relative error <= 4e-7 on [-125, 0] (ex2.approx itself is
+    within 2^-22 = 2.4e-7 of 2^x); tiny at and below -126."""
+    import ctypes
+    g = torch.Generator(device=DEV).manual_seed(6)
+    x = torch.cat([-torch.rand(1 << 20, generator=g, device=DEV) * 125.0,
+                   torch.linspace(-2.0, 0.0, 8193, device=DEV),
+                   torch.tensor([0.0, -0.5, -1.5, -125.0], device=DEV)])
+    y = torch.empty_like(x)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = qsa.lib().qsa_selftest_exp2_weight(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()),
+                                            x.numel(), stream)
+    assert rc == 0
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref).abs() / ref).max().item()
+    assert rel <= 4e-7, rel
+    low = torch.tensor([-126.0, -127.0, -500.0, float("-inf")], device=DEV)
+    yl = torch.empty_like(low)
+    qsa.lib().qsa_selftest_exp2_weight(ctypes.c_void_p(low.data_ptr()), ctypes.c_void_p(yl.data_ptr()), 4, stream)
+    assert (yl >= 0).all() and (yl <= 2.0 ** -125).all()
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_compress_parity_and_reproducibility(qsa, d):
     w = synthetic.custom(B=2, Tq=64, T_kv=1280, Hq=8, Hkv=2, d=d, seed=21)
