@@ -74,6 +74,11 @@ def _load():
         "qsa_merge_select_lists": (I, [P, P, I, I, I, I, I, I, I, P]),
         "qsa_sparse_attn_prefill_local": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, F, P]),
         "qsa_merge_partials": (I, [P, P, P, P, I, ctypes.c_int64, I, P]),
+        "qsa_prefill_pipeline_create": (I, [ctypes.POINTER(P), I, I, I, I, I, I, I, I, F]),
+        "qsa_prefill_pipeline_submit": (I, [P, P, P, P, P]),
+        "qsa_prefill_pipeline_synchronize": (I, [P]),
+        "qsa_prefill_pipeline_streams": (I, [P, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P)]),
+        "qsa_prefill_pipeline_destroy": (I, [P]),
         "qsa_get_device_status": (I, [P, ctypes.POINTER(I)]),
         "qsa_selftest_wait_timeout": (I, [ctypes.c_uint64, P]),
         "qsa_selftest_exp2": (I, [P, P, I, P]),
@@ -640,56 +645,62 @@ class QSAPrefill:
 
 
 class PrefillHostPipeline:
-    """Prefill steps fed from pinned host memory with neighbouring steps'
-    transfers overlapped: step k's Q, K, V upload (copy-in stream), step
-    k-1's compute (compute stream) and step k-2's O download (copy-out
-    stream) run at once over two device buffer sets.  Every step of the
-    path still runs in the library's kernels; this class only orders
-    copies and launches on streams with events."""
+    """Prefill steps fed from pinned host memory: the library's native
+    pipeline object (qsa_prefill_pipeline_*) owns two device buffer sets and
+    three streams, so that step k's Q, K, V upload, step k-1's compute and
+    step k-2's O download run at once.  This class only marshals arguments;
+    s_in / s_out are the object's copy-in and copy-out streams (for timing
+    events)."""
 
     def __init__(self, B, Tq, Hq, Hkv, d, T_kv_max, topk, q_pos0=0, device="cuda"):
         dev = torch.device(device)
-        self.device = dev
-        self.runs = [QSAPrefill(B, Tq, Hq, Hkv, d, T_kv_max, topk, q_pos0, device=dev) for _ in range(2)]
-        bf = torch.bfloat16
-        self.bufs = [dict(Q=torch.empty((B, Tq, Hq, d), dtype=bf, device=dev),
-                          K=torch.empty((B, Hkv, T_kv_max, d), dtype=bf, device=dev),
-                          V=torch.empty((B, Hkv, T_kv_max, d), dtype=bf, device=dev)) for _ in range(2)]
-        self.s_in = torch.cuda.Stream(device=dev)
-        self.s_cmp = torch.cuda.Stream(device=dev)
-        self.s_out = torch.cuda.Stream(device=dev)
-        self.ev = [dict(up=torch.cuda.Event(), done=torch.cuda.Event(), down=torch.cuda.Event()) for _ in range(2)]
-        self.used = [False, False]
-        self.k = 0
+        if dev.type != "cuda":
+            raise ValueError("the pipeline runs on a CUDA device")
+        self.shape_q = (B, Tq, Hq, d)
+        self.shape_kv = (B, Hkv, T_kv_max, d)
+        self._h = ctypes.c_void_p()
+        with torch.cuda.device(dev):
+            _check(_lib.qsa_prefill_pipeline_create(ctypes.byref(self._h), B, Hq, Hkv, Tq, q_pos0, T_kv_max, d,
+                                                    topk, float(d ** -0.5)), "qsa_prefill_pipeline_create")
+        sin, scmp, sout = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
+        _check(_lib.qsa_prefill_pipeline_streams(self._h, ctypes.byref(sin), ctypes.byref(scmp),
+                                                 ctypes.byref(sout)), "qsa_prefill_pipeline_streams")
+        self.s_in = torch.cuda.ExternalStream(sin.value, device=dev)
+        self.s_cmp = torch.cuda.ExternalStream(scmp.value, device=dev)
+        self.s_out = torch.cuda.ExternalStream(sout.value, device=dev)
+
+    @staticmethod
+    def _host(t, shape, name):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be a bf16 host tensor")
+        if tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous {tuple(shape)}")
+        if not t.is_pinned():
+            raise ValueError(f"{name} must be in pinned (page-locked) memory")
+        return ctypes.c_void_p(t.data_ptr())
 
     def submit(self, hQ, hK, hV, hO):
         """Queue one step: hQ, hK, hV (pinned, the step's inputs) in, O out
         to hO (pinned).  Returns at once; synchronize() waits."""
-        i = self.k & 1
-        buf, run, ev = self.bufs[i], self.runs[i], self.ev[i]
-        if self.used[i]:
-            self.s_in.wait_event(ev["done"])       # step k-2's compute has read this buffer set
-        with torch.cuda.stream(self.s_in):
-            buf["Q"].copy_(hQ, non_blocking=True)
-            buf["K"].copy_(hK, non_blocking=True)
-            buf["V"].copy_(hV, non_blocking=True)
-            ev["up"].record(self.s_in)
-        self.s_cmp.wait_event(ev["up"])
-        if self.used[i]:
-            self.s_cmp.wait_event(ev["down"])      # step k-2's O has been read out
-        if run.blk_begin > 0:
-            run.precompress_cache(buf["K"], self.s_cmp)
-        run(buf["Q"], buf["K"], buf["V"], self.s_cmp)
-        ev["done"].record(self.s_cmp)
-        self.s_out.wait_event(ev["done"])
-        with torch.cuda.stream(self.s_out):
-            hO.copy_(run.O, non_blocking=True)
-            ev["down"].record(self.s_out)
-        self.used[i] = True
-        self.k += 1
+        _check(_lib.qsa_prefill_pipeline_submit(self._h, self._host(hQ, self.shape_q, "hQ"),
+                                                self._host(hK, self.shape_kv, "hK"),
+                                                self._host(hV, self.shape_kv, "hV"),
+                                                self._host(hO, self.shape_q, "hO")),
+               "qsa_prefill_pipeline_submit")
 
     def synchronize(self):
-        self.s_out.synchronize()
+        _check(_lib.qsa_prefill_pipeline_synchronize(self._h), "qsa_prefill_pipeline_synchronize")
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            _lib.qsa_prefill_pipeline_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class QSADecode:

@@ -649,6 +649,42 @@ qsa_status launch_prefill_agg(const void *Q, const void *Kc, float *scores, floa
 }
 }  // namespace
 
+// ------------------------------------------- host-buffer prefill pipeline
+// Two device buffer sets and three streams; step k uses set k % 2.
+struct qsa_prefill_pipeline {
+    struct Set {
+        void *Q = nullptr, *K = nullptr, *V = nullptr, *O = nullptr, *ws = nullptr;
+        float *Kc = nullptr;
+        int32_t *idx = nullptr;
+        cudaEvent_t up = nullptr, done = nullptr, down = nullptr;
+        bool used = false;
+    };
+    int B = 0, Hq = 0, Hkv = 0, Tq = 0, q_pos0 = 0, T_kv_max = 0, d = 0, topk = 0;
+    float sm_scale = 0.f;
+    size_t q_bytes = 0, kv_bytes = 0, kc_bytes = 0, idx_bytes = 0, ws_bytes = 0;
+    Set set[2];
+    cudaStream_t s_in = nullptr, s_cmp = nullptr, s_out = nullptr;
+    long k = 0;
+};
+
+namespace {
+void pipeline_free(qsa_prefill_pipeline *p)
+{
+    if (!p) return;
+    for (auto *s : {p->s_in, p->s_cmp, p->s_out})
+        if (s) cudaStreamSynchronize(s);
+    for (auto &x : p->set) {
+        for (void *m : {x.Q, x.K, x.V, x.O, x.ws, (void *)x.Kc, (void *)x.idx})
+            if (m) cudaFree(m);
+        for (cudaEvent_t e : {x.up, x.done, x.down})
+            if (e) cudaEventDestroy(e);
+    }
+    for (auto *s : {p->s_in, p->s_cmp, p->s_out})
+        if (s) cudaStreamDestroy(s);
+    delete p;
+}
+}  // namespace
+
 // ===================================================================== C ABI
 extern "C" {
 
@@ -1241,6 +1277,121 @@ qsa_status qsa_merge_partials(const void *O_parts, const float *lse_parts, void 
         qsa::merge_partials_kernel<64><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)O_parts, lse_parts,
                                                             (__nv_bfloat16 *)O, lse, nparts, rows);
     return launched("merge_partials_kernel");
+}
+
+qsa_status qsa_prefill_pipeline_create(qsa_prefill_pipeline **out, int B, int Hq, int Hkv, int Tq, int q_pos0,
+                                       int T_kv_max, int d, int topk, float sm_scale)
+{
+    const char *name = "qsa_prefill_pipeline_create";
+    if (!out) return fail(QSA_ERR_INVALID_ARG, "%s: null out", name);
+    *out = nullptr;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || q_pos0 < 0 || T_kv_max <= 0 || Hq % Hkv != 0 ||
+        (T_kv_max & 63) || (q_pos0 & 63) || (long)q_pos0 + Tq > T_kv_max || !(sm_scale > 0.f))
+        return fail(QSA_ERR_INVALID_ARG, "%s: bad shape", name);
+    const int G = Hq / Hkv;
+    if (!supported_d(d) || (G != 4 && G != 8) || topk < 2 || topk > 64)
+        return fail(QSA_ERR_UNSUPPORTED, "%s: d=%d G=%d topk=%d", name, d, G, topk);
+    auto *p = new qsa_prefill_pipeline;
+    p->B = B, p->Hq = Hq, p->Hkv = Hkv, p->Tq = Tq, p->q_pos0 = q_pos0, p->T_kv_max = T_kv_max, p->d = d;
+    p->topk = topk, p->sm_scale = sm_scale;
+    const int NR = (Tq + 63) / 64;
+    p->q_bytes = (size_t)B * Tq * Hq * d * 2;
+    p->kv_bytes = (size_t)B * Hkv * T_kv_max * d * 2;
+    p->kc_bytes = (size_t)B * Hkv * (T_kv_max / 64) * d * 4;
+    p->idx_bytes = (size_t)B * Hkv * NR * topk * 4;
+    p->ws_bytes = qsa_score_select_workspace(B, Hq, Hkv, Tq, q_pos0, 64, d, topk);
+    cudaError_t e = cudaSuccess;
+    auto chk = [&](cudaError_t r) {
+        if (e == cudaSuccess) e = r;
+    };
+    chk(cudaStreamCreateWithFlags(&p->s_in, cudaStreamNonBlocking));
+    chk(cudaStreamCreateWithFlags(&p->s_cmp, cudaStreamNonBlocking));
+    chk(cudaStreamCreateWithFlags(&p->s_out, cudaStreamNonBlocking));
+    for (auto &x : p->set) {
+        chk(cudaMalloc(&x.Q, p->q_bytes));
+        chk(cudaMalloc(&x.O, p->q_bytes));
+        chk(cudaMalloc(&x.K, p->kv_bytes));
+        chk(cudaMalloc(&x.V, p->kv_bytes));
+        chk(cudaMalloc(reinterpret_cast<void **>(&x.Kc), p->kc_bytes));
+        chk(cudaMalloc(reinterpret_cast<void **>(&x.idx), p->idx_bytes));
+        if (p->ws_bytes) chk(cudaMalloc(&x.ws, p->ws_bytes));
+        if (e == cudaSuccess) chk(cudaMemsetAsync(x.Kc, 0, p->kc_bytes, p->s_cmp));
+        chk(cudaEventCreateWithFlags(&x.up, cudaEventDisableTiming));
+        chk(cudaEventCreateWithFlags(&x.done, cudaEventDisableTiming));
+        chk(cudaEventCreateWithFlags(&x.down, cudaEventDisableTiming));
+    }
+    if (e != cudaSuccess) {
+        pipeline_free(p);
+        return fail(QSA_ERR_CUDA, "%s: %s", name, cudaGetErrorString(e));
+    }
+    *out = p;
+    return QSA_OK;
+}
+
+qsa_status qsa_prefill_pipeline_submit(qsa_prefill_pipeline *p, const void *hQ, const void *hK, const void *hV,
+                                       void *hO)
+{
+    const char *name = "qsa_prefill_pipeline_submit";
+    if (!p || !hQ || !hK || !hV || !hO) return fail(QSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    auto &x = p->set[p->k & 1];
+    cudaError_t e = cudaSuccess;
+    auto chk = [&](cudaError_t r) {
+        if (e == cudaSuccess) e = r;
+    };
+    // upload: once step k-2's compute has read this set's inputs
+    if (x.used) chk(cudaStreamWaitEvent(p->s_in, x.done, 0));
+    chk(cudaMemcpyAsync(x.Q, hQ, p->q_bytes, cudaMemcpyHostToDevice, p->s_in));
+    chk(cudaMemcpyAsync(x.K, hK, p->kv_bytes, cudaMemcpyHostToDevice, p->s_in));
+    chk(cudaMemcpyAsync(x.V, hV, p->kv_bytes, cudaMemcpyHostToDevice, p->s_in));
+    chk(cudaEventRecord(x.up, p->s_in));
+    // compute: once the upload is in and step k-2's O has been read out
+    chk(cudaStreamWaitEvent(p->s_cmp, x.up, 0));
+    if (x.used) chk(cudaStreamWaitEvent(p->s_cmp, x.down, 0));
+    if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "%s: %s", name, cudaGetErrorString(e));
+    qsa_stream_t sc = reinterpret_cast<qsa_stream_t>(p->s_cmp);
+    qsa_status st = qsa_compress_keys(x.K, x.Kc, p->B, p->Hkv, p->T_kv_max, p->d, 0, (p->q_pos0 + p->Tq) / 64, sc);
+    if (st == QSA_OK)
+        st = qsa_score_select(x.Q, x.Kc, x.idx, p->B, p->Hq, p->Hkv, p->Tq, p->q_pos0, 64, p->T_kv_max, p->d,
+                              p->topk, p->sm_scale, x.ws, p->ws_bytes, sc);
+    if (st == QSA_OK)
+        st = qsa_sparse_attn_prefill(x.Q, x.K, x.V, x.idx, x.O, nullptr, p->B, p->Hq, p->Hkv, p->Tq, p->q_pos0,
+                                     p->T_kv_max, p->d, p->topk, p->sm_scale, sc);
+    if (st != QSA_OK) return st;
+    chk(cudaEventRecord(x.done, p->s_cmp));
+    // download: once the step's compute is done
+    chk(cudaStreamWaitEvent(p->s_out, x.done, 0));
+    chk(cudaMemcpyAsync(hO, x.O, p->q_bytes, cudaMemcpyDeviceToHost, p->s_out));
+    chk(cudaEventRecord(x.down, p->s_out));
+    if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "%s: %s", name, cudaGetErrorString(e));
+    x.used = true;
+    p->k++;
+    return QSA_OK;
+}
+
+qsa_status qsa_prefill_pipeline_synchronize(qsa_prefill_pipeline *p)
+{
+    if (!p) return fail(QSA_ERR_INVALID_ARG, "qsa_prefill_pipeline_synchronize: null pipeline");
+    for (cudaStream_t s : {p->s_in, p->s_cmp, p->s_out}) {
+        const cudaError_t e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "qsa_prefill_pipeline_synchronize: %s", cudaGetErrorString(e));
+    }
+    return QSA_OK;
+}
+
+qsa_status qsa_prefill_pipeline_streams(qsa_prefill_pipeline *p, qsa_stream_t *copy_in, qsa_stream_t *compute,
+                                        qsa_stream_t *copy_out)
+{
+    if (!p) return fail(QSA_ERR_INVALID_ARG, "qsa_prefill_pipeline_streams: null pipeline");
+    if (copy_in) *copy_in = reinterpret_cast<qsa_stream_t>(p->s_in);
+    if (compute) *compute = reinterpret_cast<qsa_stream_t>(p->s_cmp);
+    if (copy_out) *copy_out = reinterpret_cast<qsa_stream_t>(p->s_out);
+    return QSA_OK;
+}
+
+qsa_status qsa_prefill_pipeline_destroy(qsa_prefill_pipeline *p)
+{
+    pipeline_free(p);
+    return QSA_OK;
 }
 
 qsa_status qsa_get_device_status(qsa_stream_t stream, int *detail)

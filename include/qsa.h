@@ -42,7 +42,9 @@
  * prefill-row aggregators).
  *
  * Ownership and errors: the caller owns every buffer, including the
- * workspace; the library allocates no device memory.  All calls are
+ * workspace; the library allocates no device memory, except inside the
+ * host-buffer prefill pipeline object (qsa_prefill_pipeline_*), which owns
+ * the device buffers it stages steps through.  All calls are
  * asynchronous on `stream` (0 = legacy default stream).  Argument checks run
  * on the host before any launch and return an error without launching.
  * A failed launch returns QSA_ERR_CUDA (text in qsa_last_error()).  Errors
@@ -471,6 +473,41 @@ QSA_API qsa_status qsa_selftest_exp2(const float *x, float *y, int n, qsa_stream
  * passes: y[i] = 2^x[i] for n device floats with x <= 0 (the same reduction
  * plus a degree-5 polynomial; inputs below -126 are clamped to -126). */
 QSA_API qsa_status qsa_selftest_exp2_weight(const float *x, float *y, int n, qsa_stream_t stream);
+
+/*
+ * Host-buffer prefill pipeline: the whole prefill step (steps 1-5 as
+ * qsa_compress_keys over blocks [0, (q_pos0+Tq)/64), qsa_score_select with
+ * qblk = 64 and qsa_sparse_attn_prefill) fed from host memory, the way a
+ * serving loop feeds it.  The object owns two device buffer sets (Q, K, V,
+ * O, summaries, indices, selection workspace) and three non-blocking
+ * streams; each submitted step uploads its Q, K, V on the copy-in stream,
+ * runs on the compute stream and downloads its O on the copy-out stream,
+ * with events ordering them, so that step k's upload, step k-1's compute
+ * and step k-2's download overlap.  Host buffers use the layouts above
+ * (Q [B][Tq][Hq][d], K and V [B][Hkv][T_kv_max][d], O [B][Tq][Hq][d], all
+ * bf16); they must be page-locked (cudaHostAlloc / cudaHostRegister) for
+ * the copies to overlap, and must stay valid and unmodified until the step
+ * has completed (qsa_prefill_pipeline_synchronize).
+ *
+ * create: checks the shape (as the step's entry points would, plus
+ * 0 <= q_pos0, q_pos0 % 64 == 0, q_pos0 + Tq <= T_kv_max) before touching
+ * the device -- QSA_ERR_INVALID_ARG / QSA_ERR_UNSUPPORTED with *out left
+ * NULL -- then allocates on the current device (QSA_ERR_CUDA if that
+ * fails, nothing left allocated).  submit: returns once the step is queued;
+ * errors of the launches it makes are returned as by the entry points.
+ * synchronize: waits for every queued step.  streams: the copy-in, compute
+ * and copy-out streams (owned by the object; e.g. to record timing events
+ * on).  destroy: waits, then frees everything; NULL is accepted.
+ */
+typedef struct qsa_prefill_pipeline qsa_prefill_pipeline;
+QSA_API qsa_status qsa_prefill_pipeline_create(qsa_prefill_pipeline **out, int B, int Hq, int Hkv, int Tq,
+                                               int q_pos0, int T_kv_max, int d, int topk, float sm_scale);
+QSA_API qsa_status qsa_prefill_pipeline_submit(qsa_prefill_pipeline *p, const void *hQ, const void *hK,
+                                               const void *hV, void *hO);
+QSA_API qsa_status qsa_prefill_pipeline_synchronize(qsa_prefill_pipeline *p);
+QSA_API qsa_status qsa_prefill_pipeline_streams(qsa_prefill_pipeline *p, qsa_stream_t *copy_in,
+                                                qsa_stream_t *compute, qsa_stream_t *copy_out);
+QSA_API qsa_status qsa_prefill_pipeline_destroy(qsa_prefill_pipeline *p);
 
 /* Human-readable name of a status code (static storage). */
 QSA_API const char *qsa_status_string(qsa_status s);

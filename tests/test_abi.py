@@ -181,3 +181,31 @@ def test_binding_refuses_host_tensors_and_wrong_types():
     with pytest.raises(TypeError):
         qsa.score_select_prefill_agg(torch.zeros((1, 64, 8, 128), dtype=bf), torch.zeros((1, 2, 4, 128)),
                                      torch.zeros((1, 2, 1, 4), dtype=torch.int32), 4, 0, "max")
+
+
+def test_host_pipeline_checks_the_shape_before_touching_a_device():
+    """qsa_prefill_pipeline_create validates on the host first: bad shapes
+    return INVALID_ARG / UNSUPPORTED and leave *out NULL (this runs without
+    a GPU, so any CUDA call would fail instead)."""
+    lib = qsa.lib()
+    h = ctypes.c_void_p(0)
+    cases = [
+        ((1, 16, 2, 256, 32, 1024, 128, 32, 0.088), 1),    # q_pos0 not a multiple of 64
+        ((1, 16, 2, 256, 896, 1024, 128, 32, 0.088), 1),   # q_pos0 + Tq > T_kv_max
+        ((1, 16, 3, 256, 0, 1024, 128, 32, 0.088), 1),     # Hq % Hkv != 0
+        ((1, 16, 2, 256, 0, 1000, 128, 32, 0.088), 1),     # T_kv_max not a multiple of 64
+        ((1, 16, 2, 256, 0, 1024, 96, 32, 0.088), 2),      # d unsupported
+        ((1, 12, 2, 256, 0, 1024, 128, 32, 0.088), 2),     # G = 6 unsupported
+        ((1, 16, 2, 256, 0, 1024, 128, 65, 0.088), 2),     # topk > 64
+        ((1, 16, 2, 256, 0, 1024, 128, 32, 0.0), 1),       # sm_scale <= 0
+    ]
+    for (B, Hq, Hkv, Tq, q0, T, d, topk, sc), want in cases:
+        rc = lib.qsa_prefill_pipeline_create(ctypes.byref(h), B, Hq, Hkv, Tq, q0, T, d, topk,
+                                             ctypes.c_float(sc))
+        assert rc == want, ((B, Hq, Hkv, Tq, q0, T, d, topk, sc), rc)
+        assert not h.value
+    assert lib.qsa_prefill_pipeline_create(None, 1, 16, 2, 256, 0, 1024, 128, 32, ctypes.c_float(0.088)) == 1
+    assert lib.qsa_prefill_pipeline_submit(None, None, None, None, None) == 1
+    assert lib.qsa_prefill_pipeline_synchronize(None) == 1
+    assert lib.qsa_prefill_pipeline_destroy(None) == 0
+
