@@ -66,8 +66,10 @@ struct DecodeCfg {
     static_assert(NS >= 2, "ring too small");
     static_assert(NC * PART_FLOATS * 4 + 4 * D <= RING_BYTES, "merge scratch must fit in the ring");
     static_assert(!FP8 || D == 128, "rotated fp8 rows are 128 wide");
-    // merge inbox after the partials: at most ceil(G/P) * P <= 15 slots of 4 + D floats
-    static_assert((NC * PART_FLOATS + 15 * (4 + D)) * 4 <= RING_BYTES, "merge inbox must fit in the ring");
+    // the merge inbox follows the ring in dynamic shared memory: ceil(G/P) * P
+    // slots of (max, sum, 2 pad, O[D]) floats, sized by the host for its P
+    static constexpr int SLOT_FLOATS = 4 + D;
+    __host__ __device__ static constexpr int inbox_bytes(int G, int P) { return (G + P - 1) / P * P * SLOT_FLOATS * 4; }
 };
 
 __device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -563,16 +565,14 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
     }
     __syncthreads();
     // ---- merge.  Head h of the group is finished by CTA h % P of the
-    // cluster.  Each CTA combines its NC warps per head (weights here, before
-    // the cluster barrier, while slower CTAs may still be streaming), then
-    // stores its combined (max, sum, unnormalised O) into slot
-    // [h / P][its rank] of the owner's inbox with plain stores through
-    // distributed shared memory; after a second barrier each owner merges
-    // its inbox locally.  The inbox lies in the owner's ring past its own
-    // partials, so the first barrier (every ring idle) comes before any
-    // store into it.
-    constexpr int SLOT = 4 + D;                          // max, sum, 2 pad, O[D]
-    float *inbox = part + NC * PF;                       // [ceil(G/P)][P][SLOT]
+    // cluster.  Each CTA combines its NC warps per head, then stores its
+    // combined (max, sum, unnormalised O) into slot [h / P][its rank] of the
+    // owner's inbox with plain stores through distributed shared memory --
+    // at once, while slower CTAs may still be streaming: the inbox has
+    // shared memory of its own (after the ring), which nothing else uses;
+    // after one cluster barrier each owner merges its inbox locally.
+    constexpr int SLOT = C::SLOT_FLOATS;                 // max, sum, 2 pad, O[D]
+    float *inbox = reinterpret_cast<float *>(ring + C::RING_BYTES);   // [ceil(G/P)][P][SLOT]
     if (threadIdx.x < G) {
         const int h = threadIdx.x;
         float mc = -INFINITY;
@@ -590,7 +590,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, FP8>::THREADS, DecodeCfg<D, FP8>:
         mloc[h] = mc;
         lloc[h] = lc;
     }
-    cluster.sync();   // every CTA's ring is idle; the local weights are visible
+    __syncthreads();   // the local weights are visible
     for (int e4 = threadIdx.x; e4 < G * D / 4; e4 += C::THREADS) {
         const int h = (e4 * 4) / D, c = (e4 * 4) % D;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);

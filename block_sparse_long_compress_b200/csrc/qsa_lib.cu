@@ -218,11 +218,11 @@ struct DecodePlan {
     int P, spc;
 };
 
-DecodePlan plan_decode(int rows, int topk, int nsm, int ctas_per_sm)
+DecodePlan plan_decode(int rows, int topk, int nsm, int ctas_per_sm, int max_p = 8)
 {
     int P = (ctas_per_sm * nsm) / rows;
     P = P < 1 ? 1 : P;
-    P = P > 8 ? 8 : P;
+    P = P > max_p ? max_p : P;
     P = P > topk ? topk : P;
     DecodePlan p;
     p.spc = (topk + P - 1) / P;
@@ -313,13 +313,30 @@ qsa_status launch_decode(const void *q, const void *K, const void *V, const int3
         if ((st = make_map_2d(&mk, K, nrows, D)) != QSA_OK) return st;
         if ((st = make_map_2d(&mv, V, nrows, D)) != QSA_OK) return st;
     }
-    const DecodePlan p = plan_decode(B * Hkv, topk, sm_count(), C::CTAS_PER_SM);
     auto kern = qsa::decode_kernel<D, G, FP8>;
-    if ((st = set_smem(kern, C::SMEM_BYTES)) != QSA_OK) return st;
+    DecodePlan p = plan_decode(B * Hkv, topk, sm_count(), C::CTAS_PER_SM);
+    // the ring, then the merge inbox for this cluster size; a cluster size
+    // whose inbox would leave no room for C::CTAS_PER_SM CTAs per SM gives
+    // way to the next smaller one
+    {
+        cudaFuncAttributes fa;
+        int dev = 0, per_sm = 0, reserved = 0;
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+            return check_launch("decode_kernel attributes");
+        auto fits = [&](int P) {
+            return (long)C::CTAS_PER_SM * ((long)fa.sharedSizeBytes + C::SMEM_BYTES + C::inbox_bytes(G, P) + reserved) <=
+                   per_sm;
+        };
+        while (p.P > 1 && !fits(p.P)) p = plan_decode(B * Hkv, topk, sm_count(), C::CTAS_PER_SM, p.P - 1);
+    }
+    const int smem = C::SMEM_BYTES + C::inbox_bytes(G, p.P);
+    if ((st = set_smem(kern, smem)) != QSA_OK) return st;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.P, B * Hkv, 1);
     cfg.blockDim = dim3(C::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
