@@ -132,6 +132,9 @@ PREFILL_MAX = [
     ("g4_ragged_tail", 1, 200, 64 * 5, 8, 2, 8, 0.3),
     ("g8_three_tiles", 2, 256, 64 * 300, 16, 2, 16, 0.1),
     ("g8_chunked_rows", 1, 128, 64 * 3000, 16, 2, 32, 0.02),
+    # last query block of 32 tokens: its second 32-token half has no valid
+    # token and its query tile reaches into the next sequence's rows
+    ("g8_ragged_b2", 2, 224, 64 * 40, 16, 2, 16, 0.1),
 ]
 
 
