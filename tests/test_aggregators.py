@@ -163,10 +163,20 @@ def test_prefill_aggregator_parity(qsa, agg, name, B, Tq, q_pos0, Hq, Hkv, topk,
     print(f"prefill {agg} {name}: rows gap-checked {frac_checked:.3f}, Jaccard {jac:.4f}")
 
 
+FULL_ROWS = {
+    # per workload: sampled selection rows (row r = (b*Hkv + g)*NR + i) --
+    # the first rows (fewest candidates), middle and last rows of both groups
+    "prefill_32k": lambda NR: [0, 1, 2, 63, 200, 255, 256, 400, 511, NR + 3, NR + 300, 2 * NR - 1],
+    "prefill_128k": lambda NR: [0, 1, 2, 5, 700, 1024, 1500, 2047, NR + 3, NR + 1000, NR + 1800, 2 * NR - 1],
+}
+
+
+@pytest.mark.parametrize("wname", ["prefill_32k", "prefill_128k"])
 @pytest.mark.parametrize("agg", ["max", "softmax_sum"])
-def test_prefill_aggregator_full_size(qsa, agg):
-    """prefill_32k (32768 tokens, top-16, bf16 summaries), sampled rows."""
-    w = synthetic.CONFIGS["prefill_32k"]
+def test_prefill_aggregator_full_size(qsa, agg, wname):
+    """The benchmark's workloads (bf16 summaries; 32768 tokens top-16 and
+    131072 tokens top-32), sampled rows against the oracle."""
+    w = synthetic.CONFIGS[wname]
     x = synthetic.generate(w, DEV)
     nblk = w.T_kv // 64
     Kc = torch.empty((w.B, w.Hkv, nblk, w.d), dtype=torch.bfloat16, device=DEV)
@@ -178,12 +188,13 @@ def test_prefill_aggregator_full_size(qsa, agg):
     idx_h = idx.cpu().numpy().reshape(-1, w.topk)
     Q_h = x["Q"].cpu()
     Kc_h = Kc.float().cpu().double().numpy()
-    rows = np.array([0, 1, 2, 63, 200, 255, 256, 400, 511, NR + 3, NR + 300, 2 * NR - 1], dtype=np.int32)
+    del x
+    rows = np.array(FULL_ROWS[wname](NR), dtype=np.int32)
     s = oracle.block_scores(Q_h, Kc_h, w.Tq, w.q_pos0, 64, w.sm_scale, agg, rows=rows)
     sel = oracle.select_scores(s, w.B, w.Hkv, w.Tq, w.q_pos0, 64, w.topk, rows=rows)
     D = [(w.q_pos0 + min((r % NR + 1) * 64, w.Tq) - 1) // 64 for r in rows]
     frac_checked, jac = check_selection(idx_h[rows], sel, s, D, w.topk)
-    print(f"prefill_32k {agg}: sampled rows gap-checked {frac_checked:.3f}, Jaccard {jac:.4f}")
+    print(f"{wname} {agg}: sampled rows gap-checked {frac_checked:.3f}, Jaccard {jac:.4f}")
 
 
 @pytest.mark.parametrize("agg", ["max", "softmax_sum"])
