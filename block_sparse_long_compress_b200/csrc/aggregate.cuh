@@ -282,11 +282,13 @@ __global__ void __launch_bounds__(SoftmaxStatsCfg<G>::THREADS, 1) block_softmax_
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&t_empty[buf]);
             }
-            // the column ranges of each row meet; the slot alternates with
+            // the column ranges of each row meet: rows of one TMEM lane
+            // quarter involve only that quarter's four warps, so they meet at
+            // the quarter's own barrier (ids 2-5); the slot alternates with
             // the unit, so the next unit's writes cannot overtake this read
             const int xslot = un & 1;
             if (part > 0) xm[xslot][part - 1][r] = m_run, xs[xslot][part - 1][r] = s_run;
-            named_barrier_sync(1, 32 * C::EPI);
+            named_barrier_sync(2 + quarter, 32 * C::SPLIT);
             if (part == 0 && ok) {
                 float mn = m_run;
 #pragma unroll
@@ -608,9 +610,10 @@ __device__ __forceinline__ void block_scores_body(const CUtensorMap &tmQ, const 
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&t_empty[buf]);
                     }
-                    // the column ranges of each candidate meet (slot = tile
-                    // parity: the writes for tile kt+2 follow the barrier of
-                    // tile kt+1, which the reader passes after this read)
+                    // the column ranges of each candidate meet, at the barrier
+                    // of its TMEM lane quarter (slot = tile parity: the writes
+                    // for tile kt+2 follow the quarter's barrier of tile
+                    // kt+1, which the reader passes after this read)
                     float best = bmax;
                     if constexpr (SOFTMAX) {
                         float e0, e1;
@@ -619,7 +622,7 @@ __device__ __forceinline__ void block_scores_body(const CUtensorMap &tmQ, const 
                     }
                     const int xs = kt & 1;
                     if (part > 0) xch[xs][part - 1][m] = best;
-                    named_barrier_sync(1, 32 * C::EPI);
+                    named_barrier_sync(2 + quarter, 32 * C::SPLIT);   // the quarter's four warps
                     const int j = 1 + C::M * k + m;
                     if (part == 0 && ok && j < Dg) {
                         if constexpr (SOFTMAX) {
