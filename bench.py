@@ -280,6 +280,15 @@ def bench_prefill(args, qsa, dev, wname, ws, rank, flush, keep=False, clocks=Fal
     return out
 
 
+# DRAM bytes (read + written) per launch of the prefill attention kernel,
+# from one-pass ncu captures (dram__bytes_read.sum + dram__bytes_write.sum)
+# of this build's kernel on the workload itself; the summary with its
+# command is kept with the other ncu summaries
+# (sparse_attn_prefill_traffic.md).  A workload without a capture reports
+# null.
+ATTN_TRAFFIC = {"prefill_128k": 899.11e6 + 519.84e6, "prefill_32k": 168.17e6 + 98.41e6}
+
+
 def prefill_roofline(wp, att_ms, peaks):
     flops = prefill_flops(wp)
     achieved = flops / (att_ms * 1e-3) / 1e12
@@ -289,7 +298,7 @@ def prefill_roofline(wp, att_ms, peaks):
             "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
                                   if peaks.get("bf16_tflops_sustained") else None),
             "peak_source": peaks["source"] + " bf16 burst", "flops_per_launch": flops,
-            "traffic": None}
+            "traffic": ATTN_TRAFFIC.get(wp.name)}
 
 
 def prefill_subline(pr, peaks):
