@@ -282,10 +282,9 @@ def bench_prefill(args, qsa, dev, wname, ws, rank, flush, keep=False, clocks=Fal
 
 # DRAM bytes (read + written) per launch of the prefill attention kernel,
 # from one-pass ncu captures (dram__bytes_read.sum + dram__bytes_write.sum)
-# of this build's kernel on the workload itself; the summary with its
-# command is kept with the other ncu summaries
-# (sparse_attn_prefill_traffic.md).  A workload without a capture reports
-# null.
+# of this kernel on the workload itself, recorded with the command that
+# took them among the repository's ncu summaries.  A workload without a
+# capture reports null.
 ATTN_TRAFFIC = {"prefill_128k": 899.11e6 + 519.84e6, "prefill_32k": 168.17e6 + 98.41e6}
 
 
