@@ -497,7 +497,10 @@ QSA_API qsa_status qsa_selftest_exp2_weight(const float *x, float *y, int n, qsa
  * errors of the launches it makes are returned as by the entry points.
  * synchronize: waits for every queued step.  streams: the copy-in, compute
  * and copy-out streams (owned by the object; e.g. to record timing events
- * on).  destroy: waits, then frees everything; NULL is accepted.
+ * on).  destroy: waits, then frees everything; NULL is accepted.  After a
+ * submit that returned an error the order of the object's buffer reuse is
+ * no longer guaranteed: synchronize and destroy it.  One object is not to
+ * be used from several host threads at once.
  */
 typedef struct qsa_prefill_pipeline qsa_prefill_pipeline;
 QSA_API qsa_status qsa_prefill_pipeline_create(qsa_prefill_pipeline **out, int B, int Hq, int Hkv, int Tq,
