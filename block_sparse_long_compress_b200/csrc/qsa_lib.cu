@@ -10,6 +10,7 @@
 
 #include <atomic>
 #include <climits>
+#include <new>
 #include <mutex>
 
 #include "../../include/qsa.h"
@@ -1308,7 +1309,8 @@ qsa_status qsa_prefill_pipeline_create(qsa_prefill_pipeline **out, int B, int Hq
     const int G = Hq / Hkv;
     if (!supported_d(d) || (G != 4 && G != 8) || topk < 2 || topk > 64)
         return fail(QSA_ERR_UNSUPPORTED, "%s: d=%d G=%d topk=%d", name, d, G, topk);
-    auto *p = new qsa_prefill_pipeline;
+    auto *p = new (std::nothrow) qsa_prefill_pipeline;   // no exception crosses the C ABI
+    if (!p) return fail(QSA_ERR_CUDA, "%s: host allocation failed", name);
     p->B = B, p->Hq = Hq, p->Hkv = Hkv, p->Tq = Tq, p->q_pos0 = q_pos0, p->T_kv_max = T_kv_max, p->d = d;
     p->topk = topk, p->sm_scale = sm_scale;
     const int NR = (Tq + 63) / 64;
