@@ -287,22 +287,26 @@ __device__ void select_and_emit(const uint64_t *keys, int n, int need, SelectSha
 __device__ __forceinline__ uint64_t max64(uint64_t x, uint64_t y) { return x > y ? x : y; }
 __device__ __forceinline__ uint64_t min64(uint64_t x, uint64_t y) { return x < y ? x : y; }
 
-// One stage (block size k, stride j < 32) of a descending bitonic network.
-__device__ __forceinline__ void bitonic_stage(uint64_t &a, uint64_t &b, int k, int j)
+// One stage (block size k, stride j < 32) of a descending bitonic network
+// (K: 64-bit selection keys, or 32-bit keys where they suffice -- half the
+// shuffles).
+template <typename K>
+__device__ __forceinline__ void bitonic_stage(K &a, K &b, int k, int j)
 {
     const int lane = threadIdx.x & 31;
-    const uint64_t pa = __shfl_xor_sync(0xffffffffu, a, j);
-    const uint64_t pb = __shfl_xor_sync(0xffffffffu, b, j);
+    const K pa = __shfl_xor_sync(0xffffffffu, a, j);
+    const K pb = __shfl_xor_sync(0xffffffffu, b, j);
     const bool lower = (lane & j) == 0;
     // the lower element of a pair keeps the maximum in a descending block
     const bool max_a = lower == ((lane & k) == 0);
     const bool max_b = lower == (((32 + lane) & k) == 0);
-    a = max_a ? max64(a, pa) : min64(a, pa);
-    b = max_b ? max64(b, pb) : min64(b, pb);
+    a = max_a ? (a > pa ? a : pa) : (a < pa ? a : pa);
+    b = max_b ? (b > pb ? b : pb) : (b < pb ? b : pb);
 }
 
 // Sorts the warp's 64 keys descending.
-__device__ __forceinline__ void warp_sort64_desc(uint64_t &a, uint64_t &b)
+template <typename K>
+__device__ __forceinline__ void warp_sort64_desc(K &a, K &b)
 {
 #pragma unroll
     for (int k = 2; k <= 32; k <<= 1) {
@@ -310,7 +314,7 @@ __device__ __forceinline__ void warp_sort64_desc(uint64_t &a, uint64_t &b)
         for (int j = k >> 1; j > 0; j >>= 1) bitonic_stage(a, b, k, j);
     }
     // k = 64: the whole list descending
-    const uint64_t hi = max64(a, b), lo = min64(a, b);
+    const K hi = a > b ? a : b, lo = a < b ? a : b;
     a = hi;
     b = lo;
 #pragma unroll
@@ -395,9 +399,10 @@ __device__ void cta_top64(const uint64_t *keys, int n, uint64_t *scratch, uint64
 __device__ __forceinline__ void warp_emit_row(uint64_t a, uint64_t b, int m, int32_t *row, int D, int topk)
 {
     const int lane = threadIdx.x & 31;
-    // ascending ids = descending complements; unused slots sort last
-    uint64_t x = lane < m ? (uint64_t)(0xFFFFFFFFu - (uint32_t)key_block(a)) : 0;
-    uint64_t y = 32 + lane < m ? (uint64_t)(0xFFFFFFFFu - (uint32_t)key_block(b)) : 0;
+    // ascending ids = descending complements (32-bit keys: a candidate's id
+    // is at least 1, so its complement is above the unused slots' 0)
+    uint32_t x = lane < m ? 0xFFFFFFFFu - (uint32_t)key_block(a) : 0u;
+    uint32_t y = 32 + lane < m ? 0xFFFFFFFFu - (uint32_t)key_block(b) : 0u;
     warp_sort64_desc(x, y);
     if (lane < m) row[1 + lane] = (int)(0xFFFFFFFFu - (uint32_t)x);
     if (32 + lane < m) row[33 + lane] = (int)(0xFFFFFFFFu - (uint32_t)y);
